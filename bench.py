@@ -1,0 +1,323 @@
+"""Benchmark of the hashed N-gram embedding forward on B200: one JSON line.
+
+Workload (default): prefill, V0 = 131072, D = 2048, N = 3, K = 2 (4 sub-tables of width
+512, V_{n,k} ~ 2.16M primes), 8 sequences x 4096 Zipf(1.1) tokens, bf16 tables (8.9 GB).
+A step is one call of the C ABI's ngram_embed_fwd over the whole batch (context + hash,
+gather, projection, E_0 add, scale), inputs resident in HBM; the L2 is flushed (a
+256 MB write) between timed steps, outside the timed events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+N > 1 (launched under torch.distributed.run): each rank runs its own batch of the same
+size (data parallel, no collective on the data path), `value` = all ranks' tokens / the
+slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import configs, gen, workloads  # noqa: E402
+
+METRIC = "N-gram embed tokens/s (prefill & decode) + % of tensor/HBM roofline, 1 B200"
+UNIT = "tokens/s"
+WORKLOADS = {
+    "prefill_d2048": configs.PREFILL_D2048,
+    "prefill_varlen_d4096": configs.PREFILL_D4096_VARLEN,
+    "full_scale_prefill": configs.FULL_SCALE,
+}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------ reference arm: the oracle
+
+def oracle_sample_rate(cfg, budget_s: float = 15.0, max_tokens: int = 4096):
+    """Time the fp64 CPU oracle (exact hash + Eq. 3 combine) on a bounded sample of the
+    workload's tokens; the table rows it reads are regenerated beforehand (not timed)."""
+    import oracle
+    from synth.tables import host_W, host_rows
+    tokens, offsets = workloads.prefill_tokens(cfg)
+    W = host_W(cfg)
+    rng = np.random.default_rng(0)
+
+    def run(n):
+        rows = np.sort(rng.choice(len(tokens), size=n, replace=False))
+        win = oracle.context_windows(cfg.N, tokens, offsets)[rows]
+        t0 = time.perf_counter()
+        idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, win)
+        t_hash = time.perf_counter() - t0
+        e0 = host_rows(cfg, gen.TAG_E0, tokens[rows], cfg.D, cfg.e_std)
+        sub = np.stack([host_rows(cfg, gen.TAG_SUBTABLE0 + s, idx[:, s], cfg.d, cfg.e_std) for s in range(cfg.S)], 1)
+        t1 = time.perf_counter()
+        oracle.combine(cfg.D, cfg.S, e0, sub, W)
+        return t_hash + time.perf_counter() - t1
+
+    n = max(oracle.num_threads(), 8)
+    dt = run(n)
+    n2 = int(min(max_tokens, max(n, n * budget_s / max(dt, 1e-6) * 0.8)))
+    dt2 = run(n2)
+    return {"value": n2 / dt2, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n2} tokens sampled from the workload (exact hash + fp64 Eq. 3), {dt2:.1f} s"}
+
+
+def run_reference(args, cfg):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    steps = []
+    per = None
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample_rate(cfg, budget_s=args.ref_step_seconds, max_tokens=2048)
+        if i >= args.warmup:
+            steps.append(r)
+        per = r
+    value = float(np.mean([s["value"] for s in steps]))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * cfg.num_seqs * cfg.seq_len / value
+        if cfg.seq_len else None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_block(cfg, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": per["cores"], "kind": "oracle",
+                         "sample": per["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_block(cfg, args):
+    T = cfg.num_seqs * cfg.seq_len if cfg.seq_len else cfg.extras.get("total_tokens")
+    return {"workload": cfg.name, "V0": cfg.V0, "D": cfg.D, "N": cfg.N, "K": cfg.K, "V_nk": list(cfg.V_nk),
+            "tokens_per_step": T, "num_seqs": cfg.num_seqs, "token_dist": f"zipf({cfg.zipf_alpha})",
+            "tables_gb": round(cfg.table_bytes() / 1e9, 2), "parallelism": f"dp{args.gpus}",
+            "l2": "flushed between timed steps (256 MB write)"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill_d2048", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    args = ap.parse_args()
+    cfg = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import hashed_gram_embedding_horner_b200 as ne
+    from synth.tables import device_tables
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # each rank: its own batch of the same shape (seeded per rank), tables identical
+    tokens_h, offsets_h = workloads.prefill_tokens(cfg.with_(seed=cfg.seed) if rank == 0 else cfg.with_(seed=rank))
+    T, B = len(tokens_h), len(offsets_h) - 1
+    E0, E, W = device_tables(cfg)
+    tokens = torch.from_numpy(tokens_h).to(dev)
+    offsets = torch.from_numpy(offsets_h).to(dev)
+    plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
+    ws = ne.new_workspace(plan, T)
+    out = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        ne.ngram_embed_fwd(plan, tokens, offsets, E0, E, W, out, ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if ne.ngram_embed_get_status(ws) != 0:
+        raise RuntimeError(f"device status {ne.status_names(ne.ngram_embed_get_status(ws))}")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(np.sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * T / (ms_per_step / 1e3)
+
+    # --- dominant kernel alone: the projection (gather + tcgen05 GEMM + epilogue) from
+    # precomputed indices, CUDA events on the launching stream.
+    idx = torch.empty((T, cfg.S), dtype=torch.int32, device=dev)
+    ne.ngram_hash_indices(plan, tokens, offsets, idx, ws, stream=stream)
+    pe = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    hs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        hs[i][0].record(stream)
+        ne.ngram_hash_indices(plan, tokens, offsets, idx, ws, stream=stream)
+        hs[i][1].record(stream)
+        flush.fill_((i + 1) & 0xFF)
+        pe[i][0].record(stream)
+        ne.ngram_embed_project(plan, tokens, idx, E0, E, W, out, ws, stream=stream)
+        pe[i][1].record(stream)
+    torch.cuda.synchronize()
+    proj_ms = float(np.mean([a.elapsed_time(b) for a, b in pe]))
+    hash_ms = float(np.mean([a.elapsed_time(b) for a, b in hs]))
+    pk = peaks()
+    flops = 2.0 * T * cfg.D * cfg.D
+    achieved = flops / (proj_ms / 1e3) / 1e12
+    algo_bytes = T * (2 * cfg.D * 2 + 4) + cfg.D * cfg.D * 2
+
+    # --- end to end through the C ABI with host buffers: H2D inputs, fwd, D2H output
+    tok_pin = torch.from_numpy(tokens_h).pin_memory()
+    off_pin = torch.from_numpy(offsets_h).pin_memory()
+    out_pin = torch.empty((T, cfg.D), dtype=torch.bfloat16).pin_memory()
+    tok_d = torch.empty_like(tokens)
+    off_d = torch.empty_like(offsets)
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ee[i][0].record(stream)
+        tok_d.copy_(tok_pin, non_blocking=True)
+        off_d.copy_(off_pin, non_blocking=True)
+        ne.ngram_embed_fwd(plan, tok_d, off_d, E0, E, W, out, ws, stream=stream)
+        out_pin.copy_(out, non_blocking=True)
+        ee[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in ee]))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    status = ne.ngram_embed_get_status(ws)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample_rate(cfg)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_block(cfg, argparse.Namespace(gpus=world)),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                         "kernel": "proj_sm100_kernel (gather + tcgen05 projection + epilogue)",
+                         "kernel_ms": proj_ms, "peak_source": pk["source"] + " (burst)",
+                         "layer_frac": (flops / (ms_per_step / 1e3) / 1e12) / pk["bf16_tflops"],
+                         "hash_kernel_ms": hash_ms,
+                         "algorithmic_bytes": algo_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": tokens.numel() * 4 + offsets.numel() * 4,
+                    "d2h_bytes_per_step": out.numel() * 2},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk.summary(),
+            "device_status": status,
+            "impl": "ours",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,247 @@
+"""Python binding of libngram_embed.so (the C ABI in include/ngram_embed.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. Tensors are torch CUDA tensors (PyTorch provides device memory and
+streams); the binding passes their device pointers and sizes, checks the
+return code and raises `NgramError` on failure. Importing this module fails
+loudly if the library has not been built (`python -m
+hashed_gram_embedding_horner_b200.build`); there is no fallback.
+
+Names follow the C ABI. The layer is the hashed N-gram embedding of
+"Scaling Embeddings Outperforms Scaling Experts in Language Models", section 2
+(Eq. 2, Eq. 3), with the decode-side N-gram cache of section 4.2.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libngram_embed.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m hashed_gram_embedding_horner_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P = ctypes.c_void_p
+_I32, _I64, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+NGRAM_BF16, NGRAM_F32 = 0, 1
+STATUS_BITS = {
+    0x1: "BAD_TOKEN", 0x2: "BAD_OFFSETS", 0x4: "BAD_SLOT", 0x8: "BAD_APPEND",
+    0x10: "BAD_ROLLBACK", 0x20: "EVICTED", 0x40: "TIMEOUT",
+}
+VARIANT_AUTO, VARIANT_TC_GATHER4, VARIANT_TC_CPASYNC, VARIANT_SIMT = 0, 1, 2, 3
+
+EXPORTED = [
+    "ngram_embed_plan_create", "ngram_embed_plan_destroy", "ngram_embed_workspace_bytes",
+    "ngram_embed_fwd", "ngram_hash_indices", "ngram_embed_project", "ngram_embed_gather",
+    "ngram_cache_reset", "ngram_cache_append", "ngram_cache_rollback", "ngram_embed_get_status",
+    "ngram_embed_clear_status", "ngram_embed_error_string", "ngram_embed_plan_uses_tensor_cores",
+    "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_selftest_wait_timeout",
+]
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("V0", _I64), ("D", _I32), ("N", _I32), ("K", _I32), ("V_nk", ctypes.POINTER(_I64)),
+                ("dtype", _I32)]
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [("ring", _P), ("len", _P), ("valid_from", _P), ("capacity", _I32), ("max_seqs", _I32)]
+
+
+def _sig(name, args, res=ctypes.c_int):
+    f = getattr(_lib, name)
+    f.argtypes, f.restype = args, res
+
+
+_sig("ngram_embed_plan_create", [ctypes.POINTER(_Config), ctypes.POINTER(_P)])
+_sig("ngram_embed_plan_destroy", [_P])
+_sig("ngram_embed_workspace_bytes", [_P, _I64], _SZ)
+_sig("ngram_embed_fwd", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P])
+_sig("ngram_hash_indices", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _SZ, _P])
+_sig("ngram_embed_project", [_P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P])
+_sig("ngram_embed_gather", [_P, _P, _I64, _P, _P, _P, _SZ, _P])
+_sig("ngram_cache_reset", [_P, _P, _P, _I32, _P, _SZ, _P])
+_sig("ngram_cache_append", [_P, _P, _P, _P, _P, _I32, _P, _SZ, _P])
+_sig("ngram_cache_rollback", [_P, _P, _P, _P, _I32, _P, _SZ, _P])
+_sig("ngram_embed_get_status", [_P, _P, ctypes.POINTER(_I32)])
+_sig("ngram_embed_clear_status", [_P, _P])
+_sig("ngram_embed_error_string", [ctypes.c_int], ctypes.c_char_p)
+_sig("ngram_embed_plan_uses_tensor_cores", [_P])
+_sig("ngram_embed_plan_set_variant", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_tile_n", [_P, ctypes.c_int])
+_sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
+
+
+class NgramError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise NgramError(f"{what}: {_lib.ngram_embed_error_string(rc).decode()} ({rc})")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _i32(t, name):
+    import torch
+    if t is not None and (t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous()):
+        raise NgramError(f"{name} must be a contiguous int32 CUDA tensor")
+    return _ptr(t)
+
+
+class Plan:
+    """Host-side plan for one layer shape (owns the C plan)."""
+
+    def __init__(self, handle, V0, D, N, K, V_nk, dtype):
+        self.handle, self.V0, self.D, self.N, self.K = handle, V0, D, N, K
+        self.V_nk, self.dtype = tuple(V_nk), dtype
+        self.S = (N - 1) * K
+        self.d = D // self.S if self.S else 0
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            _lib.ngram_embed_plan_destroy(h)
+            self.handle = None
+
+
+class Cache:
+    """The N-gram cache arrays (caller-owned torch tensors): ring int32 [max_seqs, C],
+    len int64 [max_seqs], valid_from int64 [max_seqs]."""
+
+    def __init__(self, ring, length, valid_from):
+        self.ring, self.len, self.valid_from = ring, length, valid_from
+        self.struct = _Cache(ring.data_ptr(), length.data_ptr(), valid_from.data_ptr(), ring.shape[1],
+                             ring.shape[0])
+
+    @classmethod
+    def empty(cls, max_seqs: int, capacity: int, device="cuda"):
+        import torch
+        return cls(torch.zeros((max_seqs, capacity), dtype=torch.int32, device=device),
+                   torch.zeros(max_seqs, dtype=torch.int64, device=device),
+                   torch.zeros(max_seqs, dtype=torch.int64, device=device))
+
+
+def ngram_embed_plan_create(V0: int, D: int, N: int, K: int, V_nk, dtype: int = NGRAM_BF16) -> Plan:
+    S = (N - 1) * K
+    arr = (_I64 * max(S, 1))(*[int(v) for v in V_nk])
+    cfg = _Config(V0, D, N, K, ctypes.cast(arr, ctypes.POINTER(_I64)), dtype)
+    h = _P()
+    _check(_lib.ngram_embed_plan_create(ctypes.byref(cfg), ctypes.byref(h)), "ngram_embed_plan_create")
+    return Plan(h, V0, D, N, K, V_nk, dtype)
+
+
+def ngram_embed_plan_set_variant(plan: Plan, variant: int):
+    _check(_lib.ngram_embed_plan_set_variant(plan.handle, variant), "ngram_embed_plan_set_variant")
+
+
+def ngram_embed_plan_set_tile_n(plan: Plan, tile_n: int):
+    _check(_lib.ngram_embed_plan_set_tile_n(plan.handle, tile_n), "ngram_embed_plan_set_tile_n")
+
+
+def ngram_embed_plan_uses_tensor_cores(plan: Plan) -> bool:
+    return bool(_lib.ngram_embed_plan_uses_tensor_cores(plan.handle))
+
+
+def ngram_embed_workspace_bytes(plan: Plan, max_tokens: int) -> int:
+    return int(_lib.ngram_embed_workspace_bytes(plan.handle, max_tokens))
+
+
+def _tables(E_nk):
+    arr = (_P * max(len(E_nk), 1))(*[t.data_ptr() for t in E_nk])
+    return arr
+
+
+def ngram_embed_fwd(plan: Plan, tokens, seq_offsets, E0, E_nk, W_stacked, out, workspace,
+                    cache: Cache | None = None, cache_slots=None, stream=None):
+    tabs = _tables(E_nk)
+    rc = _lib.ngram_embed_fwd(plan.handle, _i32(tokens, "tokens"), _i32(seq_offsets, "seq_offsets"),
+                              seq_offsets.numel() - 1, tokens.numel(), _ptr(E0), tabs, _ptr(W_stacked),
+                              ctypes.byref(cache.struct) if cache else None, _i32(cache_slots, "cache_slots"),
+                              _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream))
+    _check(rc, "ngram_embed_fwd")
+
+
+def ngram_hash_indices(plan: Plan, tokens, seq_offsets, idx_out, workspace, cache: Cache | None = None,
+                       cache_slots=None, stream=None):
+    rc = _lib.ngram_hash_indices(plan.handle, _i32(tokens, "tokens"), _i32(seq_offsets, "seq_offsets"),
+                                 seq_offsets.numel() - 1, tokens.numel(),
+                                 ctypes.byref(cache.struct) if cache else None,
+                                 _i32(cache_slots, "cache_slots"), _i32(idx_out, "idx_out"), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_hash_indices")
+
+
+def ngram_embed_project(plan: Plan, tokens, idx, E0, E_nk, W_stacked, out, workspace, stream=None):
+    tabs = _tables(E_nk)
+    rc = _lib.ngram_embed_project(plan.handle, _i32(tokens, "tokens"), _i32(idx, "idx"), tokens.numel(),
+                                  _ptr(E0), tabs, _ptr(W_stacked), _ptr(out), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_embed_project")
+
+
+def ngram_embed_gather(plan: Plan, idx, E_nk, G_out, workspace, stream=None):
+    tabs = _tables(E_nk)
+    rc = _lib.ngram_embed_gather(plan.handle, _i32(idx, "idx"), idx.shape[0], tabs, _ptr(G_out),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_embed_gather")
+
+
+def ngram_cache_reset(plan: Plan, cache: Cache, workspace, slots=None, n=None, stream=None):
+    n = cache.struct.max_seqs if slots is None and n is None else (slots.numel() if n is None else n)
+    rc = _lib.ngram_cache_reset(plan.handle, ctypes.byref(cache.struct), _i32(slots, "slots"), n,
+                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_cache_reset")
+
+
+def ngram_cache_append(plan: Plan, cache: Cache, tokens, tok_offsets, workspace, slots=None, stream=None):
+    rc = _lib.ngram_cache_append(plan.handle, ctypes.byref(cache.struct), _i32(slots, "slots"),
+                                 _i32(tokens, "tokens"), _i32(tok_offsets, "tok_offsets"), tok_offsets.numel() - 1,
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_cache_append")
+
+
+def ngram_cache_rollback(plan: Plan, cache: Cache, counts, workspace, slots=None, stream=None):
+    rc = _lib.ngram_cache_rollback(plan.handle, ctypes.byref(cache.struct), _i32(slots, "slots"),
+                                   _i32(counts, "counts"), counts.numel(), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_cache_rollback")
+
+
+def ngram_embed_get_status(workspace, stream=None) -> int:
+    v = _I32(0)
+    _check(_lib.ngram_embed_get_status(_ptr(workspace), _stream(stream), ctypes.byref(v)), "ngram_embed_get_status")
+    return int(v.value)
+
+
+def ngram_embed_clear_status(workspace, stream=None):
+    _check(_lib.ngram_embed_clear_status(_ptr(workspace), _stream(stream)), "ngram_embed_clear_status")
+
+
+def ngram_embed_selftest_wait_timeout(workspace, limit_ns: int, stream=None):
+    _check(_lib.ngram_embed_selftest_wait_timeout(_ptr(workspace), limit_ns, _stream(stream)),
+           "ngram_embed_selftest_wait_timeout")
+
+
+def status_names(status: int):
+    return [name for bit, name in STATUS_BITS.items() if status & bit]
+
+
+def new_workspace(plan: Plan, max_tokens: int, device="cuda"):
+    """A zeroed uint8 workspace tensor of ngram_embed_workspace_bytes(plan, max_tokens)."""
+    import torch
+    n = ngram_embed_workspace_bytes(plan, max_tokens)
+    return torch.zeros(n, dtype=torch.uint8, device=device)

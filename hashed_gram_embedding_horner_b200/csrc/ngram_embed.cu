@@ -1,0 +1,520 @@
+// libngram_embed.so — host side of the C ABI declared in include/ngram_embed.h.
+//
+// Plan creation validates a layer shape (section 2 of "Scaling Embeddings Outperforms
+// Scaling Experts in Language Models", Eq. 3) and picks the projection kernel:
+//   - bf16, D % 128 == 0, d % 64 == 0, N >= 2: the fused gather + tcgen05 kernel
+//     (proj_sm100.cuh), 128 x 256 tiles (128 x 128 when D % 256 != 0);
+//   - otherwise the CUDA-core kernel (simt.cuh).
+// Every entry point checks its arguments on the host, launches on the caller's
+// stream, and returns without synchronising.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "common.cuh"
+#include "hash.cuh"
+#include "proj_sm100.cuh"
+#include "simt.cuh"
+
+using namespace ngram;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;  // status word + padding; the index buffer follows
+constexpr int kStages = 4;
+
+enum Variant : int { kAuto = 0, kTcGather4 = 1, kTcCpAsync = 2, kSimt = 3 };
+
+}  // namespace
+
+struct ngram_embed_plan {
+  int64_t V0;
+  int D, N, K, S, d;
+  int dtype;
+  int elt;  // bytes per element
+  int64_t V[kMaxS];
+  uint64_t barrett[kMaxS];
+  int device;
+  int sms;
+  int variant;  // resolved: kTcGather4, kTcCpAsync or kSimt
+  int bn;       // tensor-core tile width (256 or 128)
+  bool tc_ok;   // the shape admits the tensor-core kernel
+  // tensor-map cache (re-encoded when a table or W pointer changes)
+  ProjMaps maps;
+  const void* map_W = nullptr;
+  const void* map_E[kMaxS] = {};
+  bool maps_valid = false;
+  bool smem_attr_set[4] = {};  // per (tile width, A loader) kernel instance, on `device`
+};
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int32_t* status_ptr(void* ws) { return static_cast<int32_t*>(ws); }
+int32_t* idx_ptr(void* ws) { return reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kStatusBytes); }
+
+size_t ws_bytes(const ngram_embed_plan* p, int64_t T) {
+  const size_t idx = static_cast<size_t>(T) * static_cast<size_t>(p->S) * sizeof(int32_t);
+  return kStatusBytes + ((idx + 255) & ~size_t(255));
+}
+
+int check_launch() { return cudaGetLastError() == cudaSuccess ? NGRAM_OK : NGRAM_ERR_CUDA; }
+
+int encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+              uint32_t box_inner, uint32_t box_outer, CUtensorMapL2promotion promo) {
+  auto fn = encode_fn();
+  if (!fn) return NGRAM_ERR_CUDA;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NGRAM_OK : NGRAM_ERR_CUDA;
+}
+
+int refresh_maps(ngram_embed_plan* p, const void* const* E_nk, const void* W) {
+  bool same = p->maps_valid && p->map_W == W;
+  for (int s = 0; same && s < p->S; ++s) same = p->map_E[s] == E_nk[s];
+  if (same) return NGRAM_OK;
+  p->maps_valid = false;
+  int rc = encode_2d(&p->maps.W, W, p->D, p->D, static_cast<uint64_t>(p->D) * 2, kBK, p->bn,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (rc) return rc;
+  for (int s = 0; s < p->S; ++s) {
+    rc = encode_2d(&p->maps.E[s], E_nk[s], p->d, p->V[s], static_cast<uint64_t>(p->d) * 2, kBK, 1,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
+    if (rc) return rc;
+    p->map_E[s] = E_nk[s];
+  }
+  p->map_W = W;
+  p->maps_valid = true;
+  return NGRAM_OK;
+}
+
+template <int BN, int AMODE>
+int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
+  using L = ProjSmem<BN, kStages>;
+  auto kern = proj_sm100_kernel<BN, kStages, AMODE>;
+  const int key = (BN == 256 ? 2 : 0) + AMODE;
+  if (!p->smem_attr_set[key]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess)
+      return NGRAM_ERR_CUDA;
+    p->smem_attr_set[key] = true;
+  }
+  const int tiles = prm.num_m_blocks * prm.num_n_blocks;
+  const int grid = tiles < p->sms ? tiles : p->sms;
+  kern<<<grid, kProjThreads, L::kLaunchBytes, st>>>(p->maps, prm);
+  return check_launch();
+}
+
+int validate_common(const ngram_embed_plan* p, void* ws, size_t ws_size, int64_t T) {
+  if (!p || !ws || T < 0 || T > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return NGRAM_ERR_MISALIGNED;
+  if (ws_size < ws_bytes(p, T)) return NGRAM_ERR_WORKSPACE;
+  return NGRAM_OK;
+}
+
+int set_device(const ngram_embed_plan* p) {
+  if (p->device < 0) return NGRAM_ERR_CUDA;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return NGRAM_ERR_CUDA;
+  if (cur != p->device && cudaSetDevice(p->device) != cudaSuccess) return NGRAM_ERR_CUDA;
+  return NGRAM_OK;
+}
+
+int launch_hash(const ngram_embed_plan* p, const int32_t* tokens, const int32_t* offsets, int32_t num_seqs,
+                int64_t T, const ngram_cache* cache, const int32_t* slots, int32_t* idx_out, void* ws,
+                cudaStream_t st) {
+  HashParams h{};
+  h.tokens = tokens;
+  h.offsets = offsets;
+  h.num_seqs = num_seqs;
+  h.T = T;
+  h.V0 = static_cast<uint32_t>(p->V0);
+  h.N = p->N;
+  h.K = p->K;
+  h.S = p->S;
+  for (int s = 0; s < p->S; ++s) {
+    h.V[s] = static_cast<uint32_t>(p->V[s]);
+    h.barrett[s] = p->barrett[s];
+  }
+  if (cache) {
+    h.ring = cache->ring;
+    h.len = cache->len;
+    h.valid_from = cache->valid_from;
+    h.capacity = cache->capacity;
+    h.max_seqs = cache->max_seqs;
+    h.slots = slots;
+  }
+  h.idx_out = idx_out;
+  h.status = status_ptr(ws);
+  const int64_t work = T > num_seqs + 1 ? T : num_seqs + 1;
+  const int64_t blocks = (work + 255) / 256;
+  hash_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(h);
+  return check_launch();
+}
+
+int validate_cache(const ngram_embed_plan* p, const ngram_cache* c) {
+  if (!c->ring || !c->len || !c->valid_from || c->max_seqs < 0) return NGRAM_ERR_INVALID_ARG;
+  if (c->capacity < 1 || c->capacity < p->N - 1) return NGRAM_ERR_INVALID_ARG;
+  return NGRAM_OK;
+}
+
+template <typename T>
+int launch_simt(const ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int64_t n_tok,
+                const void* E0, const void* const* E_nk, const void* W, void* out, void* ws, cudaStream_t st) {
+  SimtParams<T> s{};
+  s.tokens = tokens;
+  s.idx = idx;
+  s.E0 = static_cast<const T*>(E0);
+  for (int i = 0; i < p->S; ++i) {
+    s.E[i] = static_cast<const T*>(E_nk[i]);
+    s.Vs[i] = static_cast<uint32_t>(p->V[i]);
+  }
+  s.W = static_cast<const T*>(W);
+  s.out = static_cast<T*>(out);
+  s.T_tokens = n_tok;
+  s.V0 = static_cast<uint32_t>(p->V0);
+  s.D = p->D;
+  s.S = p->S;
+  s.d = p->d;
+  int tpb = static_cast<int>((48 * 1024) / (static_cast<size_t>(p->D) * sizeof(float)));
+  if (tpb > 8) tpb = 8;
+  if (tpb < 1) tpb = 1;
+  s.tokens_per_block = tpb;
+  s.scale = 1.0f / static_cast<float>(p->S + 1);
+  s.status = status_ptr(ws);
+  const size_t smem = static_cast<size_t>(tpb) * p->D * sizeof(float);
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(proj_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return NGRAM_ERR_CUDA;
+  }
+  const int64_t blocks = (n_tok + tpb - 1) / tpb;
+  proj_simt_kernel<T><<<static_cast<unsigned>(blocks), 256, smem, st>>>(s);
+  return check_launch();
+}
+
+int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int64_t T, const void* E0,
+            const void* const* E_nk, const void* W, void* out, void* ws, cudaStream_t st) {
+  if (p->variant == kSimt) {
+    return p->dtype == NGRAM_F32
+               ? launch_simt<float>(p, tokens, idx, T, E0, E_nk, W, out, ws, st)
+               : launch_simt<uint16_t>(p, tokens, idx, T, E0, E_nk, W, out, ws, st);
+  }
+  int rc = refresh_maps(p, E_nk, W);
+  if (rc) return rc;
+  ProjParams prm{};
+  prm.tokens = tokens;
+  prm.idx = idx;
+  prm.E0 = static_cast<const uint16_t*>(E0);
+  for (int s = 0; s < p->S; ++s) {
+    prm.E[s] = static_cast<const uint16_t*>(E_nk[s]);
+    prm.Vs[s] = static_cast<uint32_t>(p->V[s]);
+  }
+  prm.out = static_cast<uint16_t*>(out);
+  prm.T = T;
+  prm.V0 = static_cast<uint32_t>(p->V0);
+  prm.D = p->D;
+  prm.S = p->S;
+  prm.d = p->d;
+  prm.num_m_blocks = static_cast<int>((T + kBM - 1) / kBM);
+  prm.num_n_blocks = p->D / p->bn;
+  prm.num_k_blocks = p->D / kBK;
+  prm.scale = 1.0f / static_cast<float>(p->S + 1);
+  prm.status = status_ptr(ws);
+  if (p->bn == 256)
+    return p->variant == kTcGather4 ? launch_tc<256, kGather4>(p, prm, st) : launch_tc<256, kCpAsync>(p, prm, st);
+  return p->variant == kTcGather4 ? launch_tc<128, kGather4>(p, prm, st) : launch_tc<128, kCpAsync>(p, prm, st);
+}
+
+int check_tables(const ngram_embed_plan* p, const void* E0, const void* const* E_nk, const void* W) {
+  if (!E0 || (p->S > 0 && (!E_nk || !W))) return NGRAM_ERR_INVALID_ARG;
+  if (!aligned16(E0)) return NGRAM_ERR_MISALIGNED;
+  for (int s = 0; s < p->S; ++s) {
+    if (!E_nk[s]) return NGRAM_ERR_INVALID_ARG;
+    if (!aligned16(E_nk[s])) return NGRAM_ERR_MISALIGNED;
+  }
+  if (p->S > 0 && !aligned16(W)) return NGRAM_ERR_MISALIGNED;
+  return NGRAM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ngram_embed_error_string(int code) {
+  switch (code) {
+    case NGRAM_OK: return "ok";
+    case NGRAM_ERR_INVALID_ARG: return "invalid argument";
+    case NGRAM_ERR_UNSUPPORTED: return "unsupported configuration";
+    case NGRAM_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case NGRAM_ERR_WORKSPACE: return "workspace too small";
+    case NGRAM_ERR_CUDA: return "CUDA call or launch failed";
+    default: return "unknown error";
+  }
+}
+
+int ngram_embed_plan_create(const ngram_embed_config* cfg, ngram_embed_plan** out) {
+  if (!cfg || !out) return NGRAM_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (cfg->V0 < 1 || cfg->V0 >= (int64_t(1) << 31) || cfg->D < 1 || cfg->N < 1 || cfg->K < 1)
+    return NGRAM_ERR_INVALID_ARG;
+  if (cfg->dtype != NGRAM_BF16 && cfg->dtype != NGRAM_F32) return NGRAM_ERR_INVALID_ARG;
+  if (cfg->N > kMaxN) return NGRAM_ERR_UNSUPPORTED;
+  const int64_t S = static_cast<int64_t>(cfg->N - 1) * cfg->K;
+  if (S > kMaxS) return NGRAM_ERR_UNSUPPORTED;
+  if (S > 0 && (cfg->D % S != 0)) return NGRAM_ERR_INVALID_ARG;
+  if (S > 0 && !cfg->V_nk) return NGRAM_ERR_INVALID_ARG;
+  const int elt = cfg->dtype == NGRAM_BF16 ? 2 : 4;
+  const int d = S ? static_cast<int>(cfg->D / S) : 0;
+  if ((static_cast<int64_t>(cfg->D) * elt) % 16 != 0) return NGRAM_ERR_UNSUPPORTED;
+  if (S > 0 && (static_cast<int64_t>(d) * elt) % 16 != 0) return NGRAM_ERR_UNSUPPORTED;
+  for (int s = 0; s < S; ++s)
+    if (cfg->V_nk[s] < 1 || cfg->V_nk[s] >= (int64_t(1) << 31)) return NGRAM_ERR_INVALID_ARG;
+
+  auto* p = new (std::nothrow) ngram_embed_plan();
+  if (!p) return NGRAM_ERR_INVALID_ARG;
+  p->V0 = cfg->V0;
+  p->D = cfg->D;
+  p->N = cfg->N;
+  p->K = cfg->K;
+  p->S = static_cast<int>(S);
+  p->d = d;
+  p->dtype = cfg->dtype;
+  p->elt = elt;
+  for (int s = 0; s < S; ++s) {
+    p->V[s] = cfg->V_nk[s];
+    p->barrett[s] = ~uint64_t(0) / static_cast<uint64_t>(cfg->V_nk[s]);
+  }
+  // Without a usable device the plan still validates arguments; launches then fail
+  // with NGRAM_ERR_CUDA.
+  if (cudaGetDevice(&p->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&p->sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess) {
+    cudaGetLastError();
+    p->device = -1;
+    p->sms = 0;
+  }
+  p->tc_ok = cfg->dtype == NGRAM_BF16 && S > 0 && cfg->D % 128 == 0 && d % kBK == 0;
+  p->bn = cfg->D % 256 == 0 ? 256 : 128;
+  p->variant = p->tc_ok ? kTcGather4 : kSimt;
+  *out = p;
+  return NGRAM_OK;
+}
+
+int ngram_embed_plan_destroy(ngram_embed_plan* plan) {
+  delete plan;
+  return NGRAM_OK;
+}
+
+int ngram_embed_plan_uses_tensor_cores(const ngram_embed_plan* plan) {
+  return plan && plan->variant != kSimt ? 1 : 0;
+}
+
+// Select the projection kernel: 0 = automatic, 1 = tensor cores with TMA row gathers,
+// 2 = tensor cores with cp.async row gathers, 3 = CUDA cores.
+int ngram_embed_plan_set_variant(ngram_embed_plan* plan, int variant) {
+  if (!plan || variant < kAuto || variant > kSimt) return NGRAM_ERR_INVALID_ARG;
+  if ((variant == kTcGather4 || variant == kTcCpAsync) && !plan->tc_ok) return NGRAM_ERR_UNSUPPORTED;
+  plan->variant = variant == kAuto ? (plan->tc_ok ? kTcGather4 : kSimt) : variant;
+  return NGRAM_OK;
+}
+
+// Tensor-core tile width: 256 or 128 output columns per tile (D must divide).
+int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int bn) {
+  if (!plan || (bn != 128 && bn != 256) || plan->D % bn != 0) return NGRAM_ERR_INVALID_ARG;
+  plan->bn = bn;
+  plan->maps_valid = false;
+  return NGRAM_OK;
+}
+
+size_t ngram_embed_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens) {
+  if (!plan || max_tokens < 0) return 0;
+  return ws_bytes(plan, max_tokens);
+}
+
+int ngram_hash_indices(const ngram_embed_plan* plan, const int32_t* tokens, const int32_t* seq_offsets,
+                       int32_t num_seqs, int64_t num_tokens, const ngram_cache* cache,
+                       const int32_t* cache_slots, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  int rc = validate_common(plan, workspace, workspace_bytes, 0);
+  if (rc) return rc;
+  if (num_tokens < 0 || num_tokens > INT32_MAX || num_seqs < 0) return NGRAM_ERR_INVALID_ARG;
+  if (num_tokens == 0) return NGRAM_OK;
+  if (!tokens || !seq_offsets || num_seqs == 0 || (plan->S > 0 && !idx_out)) return NGRAM_ERR_INVALID_ARG;
+  if (cache && (rc = validate_cache(plan, cache))) return rc;
+  if (plan->S == 0) return NGRAM_OK;
+  if ((rc = set_device(plan))) return rc;
+  return launch_hash(plan, tokens, seq_offsets, num_seqs, num_tokens, cache, cache_slots, idx_out, workspace,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int ngram_embed_project(const ngram_embed_plan* plan_c, const int32_t* tokens, const int32_t* idx,
+                        int64_t num_tokens, const void* E0, const void* const* E_nk, const void* W_stacked,
+                        void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  auto* plan = const_cast<ngram_embed_plan*>(plan_c);
+  int rc = validate_common(plan, workspace, workspace_bytes, 0);
+  if (rc) return rc;
+  if (num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
+  if (num_tokens == 0) return NGRAM_OK;
+  if (!tokens || !out || (plan->S > 0 && !idx)) return NGRAM_ERR_INVALID_ARG;
+  if (!aligned16(out)) return NGRAM_ERR_MISALIGNED;
+  if ((rc = check_tables(plan, E0, E_nk, W_stacked))) return rc;
+  if ((rc = set_device(plan))) return rc;
+  return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace,
+                 static_cast<cudaStream_t>(stream));
+}
+
+int ngram_embed_fwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const int32_t* seq_offsets,
+                    int32_t num_seqs, int64_t num_tokens, const void* E0, const void* const* E_nk,
+                    const void* W_stacked, const ngram_cache* cache, const int32_t* cache_slots, void* out,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  auto* plan = const_cast<ngram_embed_plan*>(plan_c);
+  int rc = validate_common(plan, workspace, workspace_bytes, num_tokens);
+  if (rc) return rc;
+  if (num_seqs < 0) return NGRAM_ERR_INVALID_ARG;
+  if (num_tokens == 0) return NGRAM_OK;
+  if (!tokens || !seq_offsets || num_seqs == 0 || !out) return NGRAM_ERR_INVALID_ARG;
+  if (!aligned16(out)) return NGRAM_ERR_MISALIGNED;
+  if ((rc = check_tables(plan, E0, E_nk, W_stacked))) return rc;
+  if (cache && (rc = validate_cache(plan, cache))) return rc;
+  if ((rc = set_device(plan))) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* idx = idx_ptr(workspace);
+  if (plan->S > 0) {
+    rc = launch_hash(plan, tokens, seq_offsets, num_seqs, num_tokens, cache, cache_slots, idx, workspace, st);
+    if (rc) return rc;
+  }
+  return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace, st);
+}
+
+int ngram_embed_gather(const ngram_embed_plan* plan, const int32_t* idx, int64_t num_tokens,
+                       const void* const* E_nk, void* G_out, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  int rc = validate_common(plan, workspace, workspace_bytes, 0);
+  if (rc) return rc;
+  if (num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
+  if (num_tokens == 0 || plan->S == 0) return NGRAM_OK;
+  if (!idx || !E_nk || !G_out) return NGRAM_ERR_INVALID_ARG;
+  if (!aligned16(G_out)) return NGRAM_ERR_MISALIGNED;
+  GatherParams g{};
+  for (int s = 0; s < plan->S; ++s) {
+    if (!E_nk[s]) return NGRAM_ERR_INVALID_ARG;
+    if (!aligned16(E_nk[s])) return NGRAM_ERR_MISALIGNED;
+    g.E[s] = static_cast<const uint8_t*>(E_nk[s]);
+    g.Vs[s] = static_cast<uint32_t>(plan->V[s]);
+  }
+  if ((rc = set_device(plan))) return rc;
+  g.idx = idx;
+  g.G = static_cast<uint8_t*>(G_out);
+  g.T = num_tokens;
+  g.S = plan->S;
+  g.row_bytes = plan->d * plan->elt;
+  g.status = status_ptr(workspace);
+  const int64_t rows = num_tokens * plan->S;
+  int64_t blocks = (rows + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(plan->sms) * 16;
+  if (blocks > cap) blocks = cap;
+  gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(g);
+  return check_launch();
+}
+
+static int cache_launch(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots,
+                        const int32_t* tokens, const int32_t* tok_offsets, const int32_t* counts, int32_t n,
+                        void* workspace, size_t workspace_bytes, void* stream, int which) {
+  int rc = validate_common(plan, workspace, workspace_bytes, 0);
+  if (rc) return rc;
+  if (!cache || n < 0) return NGRAM_ERR_INVALID_ARG;
+  if ((rc = validate_cache(plan, cache))) return rc;
+  if (n == 0) return NGRAM_OK;
+  if (which == 1 && (!tokens || !tok_offsets)) return NGRAM_ERR_INVALID_ARG;
+  if (which == 2 && !counts) return NGRAM_ERR_INVALID_ARG;
+  if ((rc = set_device(plan))) return rc;
+  CacheParams c{};
+  c.ring = cache->ring;
+  c.len = cache->len;
+  c.valid_from = cache->valid_from;
+  c.capacity = cache->capacity;
+  c.max_seqs = cache->max_seqs;
+  c.N = plan->N;
+  c.V0 = static_cast<uint32_t>(plan->V0);
+  c.slots = slots;
+  c.tokens = tokens;
+  c.tok_offsets = tok_offsets;
+  c.counts = counts;
+  c.n = n;
+  c.status = status_ptr(workspace);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (which == 0)
+    cache_reset_kernel<<<(n + 255) / 256, 256, 0, st>>>(c);
+  else if (which == 1)
+    cache_append_kernel<<<(n + 7) / 8, 256, 0, st>>>(c);
+  else
+    cache_rollback_kernel<<<(n + 255) / 256, 256, 0, st>>>(c);
+  return check_launch();
+}
+
+int ngram_cache_reset(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots, int32_t n,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  return cache_launch(plan, cache, slots, nullptr, nullptr, nullptr, n, workspace, workspace_bytes, stream, 0);
+}
+
+int ngram_cache_append(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots,
+                       const int32_t* tokens, const int32_t* tok_offsets, int32_t n, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return cache_launch(plan, cache, slots, tokens, tok_offsets, nullptr, n, workspace, workspace_bytes, stream, 1);
+}
+
+int ngram_cache_rollback(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots,
+                         const int32_t* counts, int32_t n, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  return cache_launch(plan, cache, slots, nullptr, nullptr, counts, n, workspace, workspace_bytes, stream, 2);
+}
+
+int ngram_embed_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream) {
+  if (!workspace || limit_ns <= 0 || limit_ns > 2000000000LL) return NGRAM_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NGRAM_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status_ptr(workspace),
+                                                                         static_cast<uint64_t>(limit_ns));
+  return check_launch();
+}
+
+int ngram_embed_get_status(const void* workspace, void* stream, int32_t* status_out) {
+  if (!workspace || !status_out) return NGRAM_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(status_out, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return NGRAM_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? NGRAM_OK : NGRAM_ERR_CUDA;
+}
+
+int ngram_embed_clear_status(void* workspace, void* stream) {
+  if (!workspace) return NGRAM_ERR_INVALID_ARG;
+  return cudaMemsetAsync(workspace, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? NGRAM_OK
+             : NGRAM_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,230 @@
+// CUDA-core kernels: the projection for fp32 tables and for shapes the tensor-core
+// kernel does not take (N = 1, D % 128 != 0, d % 64 != 0), the stand-alone sub-row
+// gather, and the N-gram cache ring updates.
+#pragma once
+
+#include "common.cuh"
+
+namespace ngram {
+
+// ------------------------------------------------------------------ element access
+
+template <typename T> struct Elt;
+template <> struct Elt<float> {
+  static __device__ __forceinline__ float load(const float* p, int64_t i) { return __ldg(p + i); }
+  static __device__ __forceinline__ void store(float* p, int64_t i, float v) { p[i] = v; }
+};
+template <> struct Elt<uint16_t> {  // bf16 bit patterns
+  static __device__ __forceinline__ float load(const uint16_t* p, int64_t i) {
+    return bf16_bits_to_float(__ldg(p + i));
+  }
+  static __device__ __forceinline__ void store(uint16_t* p, int64_t i, float v) {
+    p[i] = static_cast<uint16_t>(pack_bf16x2(v, 0.f) & 0xFFFFu);
+  }
+};
+
+// ------------------------------------------------------------------ SIMT projection
+
+template <typename T>
+struct SimtParams {
+  const int32_t* tokens;
+  const int32_t* idx;
+  const T* E0;
+  const T* E[kMaxS];
+  uint32_t Vs[kMaxS];
+  const T* W;
+  T* out;
+  int64_t T_tokens;
+  uint32_t V0;
+  int D, S, d;
+  int tokens_per_block;
+  float scale;
+  int* status;
+};
+
+// Block = 8 warps over `tokens_per_block` tokens. The tokens' gathered rows G (fp32)
+// sit in shared memory; each warp takes output columns o and reduces
+// sum_k W[o][k] * G[t][k] across its lanes (coalesced reads of W's row o).
+template <typename T>
+__global__ void __launch_bounds__(256) proj_simt_kernel(const __grid_constant__ SimtParams<T> p) {
+  extern __shared__ float g[];  // [tokens_per_block][D]
+  const int TPB = p.tokens_per_block;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * TPB;
+  const int64_t left = p.T_tokens - t0;
+  const int nt = static_cast<int>(left < TPB ? left : TPB);
+  if (nt <= 0) return;
+
+  for (int e = threadIdx.x; e < nt * p.D; e += blockDim.x) {
+    const int t = e / p.D, k = e - t * p.D;
+    float v = 0.f;
+    if (p.S > 0) {
+      const int s = k / p.d, c = k - s * p.d;
+      int32_t r = p.idx[(t0 + t) * p.S + s];
+      if (static_cast<uint32_t>(r) >= p.Vs[s]) {
+        set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+        r = 0;
+      }
+      v = Elt<T>::load(p.E[s], static_cast<int64_t>(r) * p.d + c);
+    }
+    g[t * p.D + k] = v;
+  }
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kMaxTPB = 8;
+  int32_t tok[kMaxTPB];
+#pragma unroll
+  for (int t = 0; t < kMaxTPB; ++t) {
+    int32_t x = t < nt ? p.tokens[t0 + t] : 0;
+    if (x < 0 || static_cast<uint32_t>(x) >= p.V0) x = 0;  // flagged by the hash stage
+    tok[t] = x;
+  }
+  for (int o = warp; o < p.D; o += 8) {
+    float acc[kMaxTPB];
+#pragma unroll
+    for (int t = 0; t < kMaxTPB; ++t) acc[t] = 0.f;
+    if (p.S > 0) {
+      for (int k = lane; k < p.D; k += 32) {
+        const float w = Elt<T>::load(p.W, static_cast<int64_t>(o) * p.D + k);
+#pragma unroll
+        for (int t = 0; t < kMaxTPB; ++t)
+          if (t < nt) acc[t] = fmaf(w, g[t * p.D + k], acc[t]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kMaxTPB; ++t) {
+      float a = acc[t];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+      if (lane == 0 && t < nt) {
+        const float e0 = Elt<T>::load(p.E0, static_cast<int64_t>(tok[t]) * p.D + o);
+        Elt<T>::store(p.out, (t0 + t) * p.D + o, (a + e0) * p.scale);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ gather (stand-alone)
+
+struct GatherParams {
+  const int32_t* idx;
+  const uint8_t* E[kMaxS];
+  uint32_t Vs[kMaxS];
+  uint8_t* G;
+  int64_t T;
+  int S;
+  int row_bytes;  // d * element size, a multiple of 16
+  int* status;
+};
+
+// One warp per (token, sub-table) row: 16-byte vector copies of E_s[idx] into
+// G[i][s*d .. (s+1)*d). Grid-stride over rows.
+__global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ GatherParams p) {
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int vec = p.row_bytes >> 4;
+  for (int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       w < p.T * p.S; w += warps) {
+    const int64_t i = w / p.S;
+    const int s = static_cast<int>(w - i * p.S);
+    int32_t r = p.idx[w];
+    if (static_cast<uint32_t>(r) >= p.Vs[s]) {
+      if (lane == 0) set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+      r = 0;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(p.E[s] + static_cast<int64_t>(r) * p.row_bytes);
+    uint4* dst = reinterpret_cast<uint4*>(p.G + (i * p.S + s) * static_cast<int64_t>(p.row_bytes));
+    for (int v = lane; v < vec; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+// ------------------------------------------------------------------ N-gram cache ring
+
+struct CacheParams {
+  int32_t* ring;
+  int64_t* len;
+  int64_t* valid_from;
+  int32_t capacity, max_seqs;
+  int N;
+  uint32_t V0;
+  const int32_t* slots;       // nullptr: entry i -> slot i
+  const int32_t* tokens;      // append
+  const int32_t* tok_offsets; // append
+  const int32_t* counts;      // rollback
+  int32_t n;
+  int* status;
+};
+
+__device__ __forceinline__ int32_t entry_slot(const CacheParams& p, int32_t i) {
+  const int32_t s = p.slots ? p.slots[i] : i;
+  if (s < 0 || s >= p.max_seqs) {
+    set_status(p.status, NGRAM_STATUS_BAD_SLOT);
+    return -1;
+  }
+  return s;
+}
+
+__global__ void cache_reset_kernel(const __grid_constant__ CacheParams p) {
+  const int32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.n) return;
+  const int32_t s = entry_slot(p, i);
+  if (s < 0) return;
+  p.len[s] = 0;
+  p.valid_from[s] = 0;
+}
+
+// One warp per entry: write the ids at positions len .. len+m-1 (slot pos % C), then
+// len += m and valid_from = max(valid_from, len - C). Rejected entries change nothing.
+__global__ void cache_append_kernel(const __grid_constant__ CacheParams p) {
+  const int32_t i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (i >= p.n) return;
+  int32_t s = -1;
+  if (lane == 0) s = entry_slot(p, i);
+  s = __shfl_sync(0xffffffffu, s, 0);
+  if (s < 0) return;
+  const int32_t b = p.tok_offsets[i], e = p.tok_offsets[i + 1];
+  const int32_t m = e - b;
+  if (b < 0 || m < 0 || m > p.capacity) {
+    if (lane == 0) set_status(p.status, (b < 0 || m < 0) ? NGRAM_STATUS_BAD_OFFSETS : NGRAM_STATUS_BAD_APPEND);
+    return;
+  }
+  bool bad = false;
+  for (int k = lane; k < m; k += 32) {
+    const int32_t t = p.tokens[b + k];
+    bad |= (t < 0 || static_cast<uint32_t>(t) >= p.V0);
+  }
+  if (__any_sync(0xffffffffu, bad)) {
+    if (lane == 0) set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+    return;
+  }
+  const int64_t L = p.len[s];
+  int32_t* ring = p.ring + static_cast<int64_t>(s) * p.capacity;
+  for (int k = lane; k < m; k += 32) ring[(L + k) % p.capacity] = p.tokens[b + k];
+  __syncwarp();
+  if (lane == 0) {
+    const int64_t nl = L + m;
+    p.len[s] = nl;
+    const int64_t vf = nl - p.capacity;
+    if (vf > p.valid_from[s]) p.valid_from[s] = vf;
+  }
+}
+
+// One thread per entry: drop the newest counts[i] ids if the ring still holds the
+// newest N-1 positions that remain; otherwise flag and leave the slot unchanged.
+__global__ void cache_rollback_kernel(const __grid_constant__ CacheParams p) {
+  const int32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.n) return;
+  const int32_t s = entry_slot(p, i);
+  if (s < 0) return;
+  const int64_t r = p.counts[i];
+  const int64_t L = p.len[s];
+  const int64_t need = L - r - (p.N - 1);
+  if (r < 0 || r > L || (need > 0 ? need : 0) < p.valid_from[s]) {
+    set_status(p.status, NGRAM_STATUS_BAD_ROLLBACK);
+    return;
+  }
+  p.len[s] = L - r;
+}
+
+}  // namespace ngram

@@ -1,0 +1,206 @@
+/*
+ * ngram_embed.h — C ABI of libngram_embed.so: the forward hot path of the hashed
+ * N-gram embedding layer ("Over-Encoding") on one NVIDIA B200 (sm_100a).
+ *
+ * The operation is defined in "Scaling Embeddings Outperforms Scaling Experts in
+ * Language Models" (LongCat team), section 2 "N-gram Embedding":
+ *   Eq. 2  H_{n,k}(t_{i-n+1..i}) = (sum_{j=0}^{n-1} t_{i-j} * V0^j) mod V_{n,k}
+ *   Eq. 3  e_i = ( E_0(t_i) + sum_{n=2..N} sum_{k=1..K} W_{n,k} E_{n,k}(H_{n,k}(...)) )
+ *                / ((N-1)K + 1)
+ * with E_0 in R^{V0 x D}, E_{n,k} in R^{V_{n,k} x d}, W_{n,k} in R^{D x d}, d = D/((N-1)K);
+ * and in section 4.2 "N-gram Cache": n-gram context ids kept per sequence on the
+ * device, updated as speculative tokens are accepted or rejected.
+ *
+ * Conventions (the paper is silent on them):
+ *   - S = (N-1)K sub-tables in the order s = (n-2)K + (k-1), n = 2..N, k = 1..K.
+ *   - W_stacked is [D x D] row-major with W_stacked[o][s*d + c] = W_{n,k}[o][c], so the
+ *     projection is G * W_stacked^T, G[i] = concat_s E_s[idx[i][s]].
+ *   - A position before the start of a sequence reads the pad id 0 (prefill), or the
+ *     sequence's committed history in the N-gram cache (decode).
+ *   - Eq. 2 is evaluated exactly (Horner's rule, every step reduced mod V_{n,k} in
+ *     64-bit integers; no wrap-around).
+ *
+ * Memory and ownership: every device buffer (tables, W, tokens, offsets, outputs, cache
+ * arrays, workspace) is allocated and owned by the caller. The library owns only the
+ * host-side plan. No call allocates device memory or synchronises, except
+ * ngram_embed_get_status (which synchronises its stream). Calls are asynchronous and
+ * ordered by `stream` (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ * A plan may be used from one host thread at a time.
+ *
+ * Layouts: all tables are dense row-major. bf16 tables hold raw bf16 bit patterns.
+ * Device pointers to tables, W, outputs and the workspace must be 16-byte aligned;
+ * for the tensor-core path (bf16, D % 128 == 0, d % 64 == 0) table rows are d*2 bytes,
+ * a multiple of 16, and the base pointers 16-byte aligned.
+ *
+ * Errors: functions return NGRAM_OK (0) or a negative NGRAM_ERR_* code for bad
+ * arguments found on the host; nothing is launched then. Errors that only the device
+ * can see (a token id outside [0, V0), decreasing offsets, a bad cache slot, an invalid
+ * rollback, an evicted context position, a bounded wait that ran out) set bits of a
+ * sticky status word in the workspace (NGRAM_STATUS_*); the kernels then substitute a
+ * safe value (row 0, the pad id, or leave the cache slot unchanged) and never trap.
+ * Read the word with ngram_embed_get_status; clear it with ngram_embed_clear_status.
+ */
+#ifndef NGRAM_EMBED_H
+#define NGRAM_EMBED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes (host-side checks) ---- */
+#define NGRAM_OK 0
+#define NGRAM_ERR_INVALID_ARG -1   /* NULL pointer, negative size, bad config value */
+#define NGRAM_ERR_UNSUPPORTED -2   /* config outside the supported limits */
+#define NGRAM_ERR_MISALIGNED -3    /* a pointer is not 16-byte aligned */
+#define NGRAM_ERR_WORKSPACE -4     /* workspace smaller than ngram_embed_workspace_bytes */
+#define NGRAM_ERR_CUDA -5          /* a CUDA runtime/driver call or a launch failed */
+
+/* ---- sticky device status bits (in the workspace) ---- */
+#define NGRAM_STATUS_BAD_TOKEN 0x1       /* token id outside [0, V0); row 0 / pad used */
+#define NGRAM_STATUS_BAD_OFFSETS 0x2     /* seq/tok offsets not non-decreasing from 0 to T */
+#define NGRAM_STATUS_BAD_SLOT 0x4        /* cache slot outside [0, max_seqs) */
+#define NGRAM_STATUS_BAD_APPEND 0x8      /* append of more than `capacity` ids */
+#define NGRAM_STATUS_BAD_ROLLBACK 0x10   /* rollback < 0, > committed, or past the ring */
+#define NGRAM_STATUS_EVICTED 0x20        /* context position no longer held by the ring */
+#define NGRAM_STATUS_TIMEOUT 0x40        /* a bounded device wait ran out (kernel returned) */
+
+/* ---- element types ---- */
+#define NGRAM_BF16 0
+#define NGRAM_F32 1
+
+/* ---- limits ---- */
+#define NGRAM_MAX_N 8          /* largest n-gram order */
+#define NGRAM_MAX_SUBTABLES 32 /* largest S = (N-1)K */
+
+typedef struct ngram_embed_plan ngram_embed_plan; /* opaque, host-side */
+
+/* Shape of one N-gram embedding layer (section 2, Eq. 3). */
+typedef struct {
+  int64_t V0;          /* base vocabulary size, 1 <= V0 < 2^31 */
+  int32_t D;           /* hidden size; D % S == 0 */
+  int32_t N;           /* largest n-gram order, 1 <= N <= NGRAM_MAX_N (N = 1: e_i = E_0(t_i)) */
+  int32_t K;           /* sub-tables per order, K >= 1, S = (N-1)K <= NGRAM_MAX_SUBTABLES */
+  const int64_t* V_nk; /* host array of S sub-table sizes in order s, 1 <= V_nk < 2^31 */
+  int32_t dtype;       /* NGRAM_BF16 or NGRAM_F32 (tables, W and output) */
+} ngram_embed_config;
+
+/* The decode-side N-gram cache (section 4.2): per slot, a ring of the newest ids.
+ * All arrays are caller-owned device memory.
+ *   ring[slot * capacity + (pos % capacity)] = committed id at position pos,
+ *   len[slot]        = number of committed ids (positions 0 .. len-1),
+ *   valid_from[slot] = oldest position the ring still holds.
+ * capacity must be >= N-1 (a decode step of P ids per sequence needs >= N-1+P to roll
+ * back a whole step). ngram_cache_reset zeroes len and valid_from. */
+typedef struct {
+  int32_t* ring;
+  int64_t* len;
+  int64_t* valid_from;
+  int32_t capacity;
+  int32_t max_seqs;
+} ngram_cache;
+
+/* Validate a config and build a plan on the current CUDA device.
+ * Returns NGRAM_ERR_INVALID_ARG / NGRAM_ERR_UNSUPPORTED on a bad config. */
+int ngram_embed_plan_create(const ngram_embed_config* cfg, ngram_embed_plan** out);
+int ngram_embed_plan_destroy(ngram_embed_plan* plan);
+
+/* Device workspace bytes needed for calls of up to max_tokens tokens (status word plus
+ * the [max_tokens x S] int32 index buffer). Must be zeroed once before first use
+ * (ngram_embed_clear_status does that for the status word; the rest needs no init). */
+size_t ngram_embed_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens);
+
+/* The whole layer (section 2, Eq. 2 + Eq. 3) for num_tokens tokens in num_seqs sequences.
+ *   tokens       [num_tokens] int32 device ids in [0, V0)
+ *   seq_offsets  [num_seqs + 1] int32 device CSR offsets, 0 = off[0] <= ... <= off[B] = T
+ *   E0           [V0 x D] device table; E_nk: HOST array of S device pointers, table s
+ *                is [V_nk[s] x d]; W_stacked [D x D] device
+ *   cache        NULL: positions before a sequence start read pad 0 (prefill).
+ *                non-NULL: they read the committed history of cache slot
+ *                cache_slots[b] (or b if cache_slots is NULL), as the ring holds it
+ *                when the kernel runs.
+ *   out          [num_tokens x D] device, dtype of the plan
+ *   workspace    device, >= ngram_embed_workspace_bytes(plan, num_tokens) bytes
+ * num_tokens may be 0 (nothing is launched). */
+int ngram_embed_fwd(const ngram_embed_plan* plan, const int32_t* tokens,
+                    const int32_t* seq_offsets, int32_t num_seqs, int64_t num_tokens,
+                    const void* E0, const void* const* E_nk, const void* W_stacked,
+                    const ngram_cache* cache, const int32_t* cache_slots, void* out,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Eq. 2 alone (context assembly + hash): idx_out[i * S + s] = H_{n,k}(...) as int32,
+ * bit-exact. Arguments as for ngram_embed_fwd; idx_out is [num_tokens x S] device. */
+int ngram_hash_indices(const ngram_embed_plan* plan, const int32_t* tokens,
+                       const int32_t* seq_offsets, int32_t num_seqs, int64_t num_tokens,
+                       const ngram_cache* cache, const int32_t* cache_slots, int32_t* idx_out,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Eq. 3 given indices from ngram_hash_indices: sub-row lookup, projection, E_0 add and
+ * the 1/((N-1)K+1) scale. idx is [num_tokens x S] int32 device. */
+int ngram_embed_project(const ngram_embed_plan* plan, const int32_t* tokens,
+                        const int32_t* idx, int64_t num_tokens, const void* E0,
+                        const void* const* E_nk, const void* W_stacked, void* out,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* The sub-row lookup of Eq. 3 alone: G_out[i][s*d + c] = E_s[idx[i][s]][c], [T x D]
+ * device, plan dtype (the concatenated gathered rows the projection multiplies). */
+int ngram_embed_gather(const ngram_embed_plan* plan, const int32_t* idx, int64_t num_tokens,
+                       const void* const* E_nk, void* G_out, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* ---- N-gram cache (section 4.2) ----
+ * slots: [n] int32 device cache slots, distinct within one call (NULL: slot i for entry i).
+ * Invalid entries set a status bit and leave their slot unchanged. */
+
+/* Forget the history of the listed slots (len = valid_from = 0). */
+int ngram_cache_reset(const ngram_embed_plan* plan, const ngram_cache* cache,
+                      const int32_t* slots, int32_t n, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* Commit ids: entry i appends tokens[tok_offsets[i] .. tok_offsets[i+1]) (device CSR,
+ * at most `capacity` ids) to slot slots[i]. */
+int ngram_cache_append(const ngram_embed_plan* plan, const ngram_cache* cache,
+                       const int32_t* slots, const int32_t* tokens, const int32_t* tok_offsets,
+                       int32_t n, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Un-commit ids: entry i drops the newest counts[i] ids (device int32) of slot slots[i].
+ * Rejected (status bit, slot unchanged) if counts[i] < 0, counts[i] > len, or the newest
+ * N-1 remaining positions are no longer all held by the ring. */
+int ngram_cache_rollback(const ngram_embed_plan* plan, const ngram_cache* cache,
+                         const int32_t* slots, const int32_t* counts, int32_t n,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream` and copy the sticky status word to *status_out. */
+int ngram_embed_get_status(const void* workspace, void* stream, int32_t* status_out);
+/* Zero the status word (asynchronous on `stream`). */
+int ngram_embed_clear_status(void* workspace, void* stream);
+
+/* Self-test of the device-side bounded wait used by every pipeline barrier of the
+ * tensor-core kernel: launches one warp that waits on a barrier nothing completes.
+ * The wait must give up after limit_ns (<= 2 s), set NGRAM_STATUS_TIMEOUT in the
+ * workspace status word and return; the context stays usable. */
+int ngram_embed_selftest_wait_timeout(void* workspace, int64_t limit_ns, void* stream);
+
+/* Static description of a return code. */
+const char* ngram_embed_error_string(int code);
+
+/* Which projection kernel a plan uses: 1 = tcgen05 tensor-core kernel, 0 = CUDA-core kernel. */
+int ngram_embed_plan_uses_tensor_cores(const ngram_embed_plan* plan);
+
+/* Choose the projection kernel of a plan (for testing one implementation against another):
+ *   0 = automatic (tensor cores when the shape allows: bf16, D % 128 == 0, d % 64 == 0, N >= 2),
+ *   1 = tensor cores, A rows gathered by TMA (tile::gather4),
+ *   2 = tensor cores, A rows gathered by 16-byte cp.async,
+ *   3 = CUDA cores.
+ * Returns NGRAM_ERR_UNSUPPORTED if the shape does not admit the chosen kernel. */
+int ngram_embed_plan_set_variant(ngram_embed_plan* plan, int variant);
+
+/* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */
+int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NGRAM_EMBED_H */

@@ -1,0 +1,118 @@
+"""The C ABI library: loads, exports every declared symbol, validates on the host.
+
+These run without a GPU: no kernel is launched (every call below is rejected by a
+host-side check before any launch, or needs no device).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ngram_embed.h")
+
+
+@pytest.fixture(scope="module")
+def ne():
+    from hashed_gram_embedding_horner_b200 import build
+    build.build()
+    import hashed_gram_embedding_horner_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(ngram_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(ne):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(ne._lib, n), n
+    assert sorted(ne.EXPORTED) == names
+
+
+def test_no_cpu_fallback_symbols(ne):
+    """The library is CUDA-only: it neither links nor names the oracle."""
+    so = open(ne.LIB_PATH, "rb").read()
+    assert b"oracle_" not in so
+
+
+def _cfg(ne, V0=131072, D=2048, N=3, K=2, V=(2162717, 2162737, 2162747, 2162803), dtype=0):
+    arr = (ctypes.c_int64 * max(len(V), 1))(*V)
+    return ne._Config(V0, D, N, K, ctypes.cast(arr, ctypes.POINTER(ctypes.c_int64)), dtype), arr
+
+
+def _create(ne, **kw):
+    cfg, keep = _cfg(ne, **kw)
+    h = ctypes.c_void_p()
+    rc = ne._lib.ngram_embed_plan_create(ctypes.byref(cfg), ctypes.byref(h))
+    return rc, h
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(V0=0), -1), (dict(V0=2 ** 31), -1), (dict(D=0), -1), (dict(N=0), -1), (dict(K=0), -1),
+    (dict(N=9, K=1, V=(5,) * 8), -2),                 # N above the limit
+    (dict(N=5, K=9, V=(5,) * 36), -2),                # S above the limit
+    (dict(D=2046), -1),                               # D % S != 0
+    (dict(V=(0, 1, 2, 3)), -1), (dict(V=(2 ** 31, 1, 2, 3)), -1),
+    (dict(dtype=7), -1),
+    (dict(D=20, N=2, K=4, V=(7, 7, 7, 7)), -2),       # d * elt not a multiple of 16 bytes
+])
+def test_plan_rejects_bad_configs(ne, kw, code):
+    rc, h = _create(ne, **kw)
+    assert rc == code and not h.value
+
+
+def test_plan_without_device_validates_then_fails_launch(ne):
+    import torch
+    rc, h = _create(ne)
+    if torch.cuda.is_available():
+        assert rc == 0
+        ne._lib.ngram_embed_plan_destroy(h)
+        return
+    # No GPU here: the plan is created for argument checks; anything that would launch
+    # reports NGRAM_ERR_CUDA, while bad arguments are still reported first.
+    assert rc == 0 and h.value
+    lib = ne._lib
+    ws_need = lib.ngram_embed_workspace_bytes(h, 1000)
+    assert ws_need == 256 + ((1000 * 4 * 4 + 255) // 256) * 256
+    fake = ctypes.c_void_p(0x10000)           # never dereferenced
+    odd = ctypes.c_void_p(0x10004)
+    tabs = (ctypes.c_void_p * 4)(0x20000, 0x30000, 0x40000, 0x50000)
+    P = ctypes.c_void_p
+    fwd = lambda ws, wsb, out=fake, T=1000: lib.ngram_embed_fwd(h, fake, fake, 1, T, fake, tabs, fake, None, None,
+                                                                 out, ws, wsb, None)
+    assert fwd(fake, 10) == -4                 # workspace too small
+    assert fwd(odd, ws_need) == -3             # misaligned workspace
+    assert fwd(fake, ws_need, out=odd) == -3   # misaligned output
+    assert fwd(None, ws_need) == -1
+    assert fwd(fake, ws_need, T=0) == 0        # nothing to do, nothing launched
+    assert fwd(fake, ws_need) == -5            # would launch: no device
+    assert lib.ngram_embed_plan_set_variant(h, 9) == -1
+    assert lib.ngram_embed_plan_set_tile_n(h, 64) == -1
+    assert lib.ngram_embed_plan_uses_tensor_cores(h) == 1
+    bad_cache = ne._Cache(0, 0, 0, 4, 8)
+    assert lib.ngram_cache_rollback(h, ctypes.byref(bad_cache), None, fake, 3, fake, ws_need, None) == -1
+    small_cap = ne._Cache(0x1000, 0x2000, 0x3000, 1, 8)  # capacity < N - 1
+    assert lib.ngram_cache_append(h, ctypes.byref(small_cap), None, fake, fake, 3, fake, ws_need, None) == -1
+    lib.ngram_embed_plan_destroy(h)
+
+
+def test_fp32_and_small_shapes_use_cuda_cores(ne):
+    rc, h = _create(ne, V0=1000, D=64, N=3, K=2, V=(4099, 5003, 6007, 7001), dtype=1)
+    assert rc == 0
+    assert ne._lib.ngram_embed_plan_uses_tensor_cores(h) == 0
+    assert ne._lib.ngram_embed_plan_set_variant(h, 1) == -2
+    ne._lib.ngram_embed_plan_destroy(h)
+    rc, h = _create(ne, D=384, N=2, K=3, V=(11, 13, 17))  # D % 128 == 0, d = 128
+    assert rc == 0 and ne._lib.ngram_embed_plan_uses_tensor_cores(h) == 1
+    ne._lib.ngram_embed_plan_destroy(h)
+
+
+def test_error_strings(ne):
+    for c in (0, -1, -2, -3, -4, -5, -99):
+        assert ne._lib.ngram_embed_error_string(c)

@@ -1,0 +1,159 @@
+"""GPU N-gram cache (section 4.2 "N-gram Cache" of "Scaling Embeddings Outperforms
+Scaling Experts in Language Models"): ring updates vs the oracle's history model, and
+decode-step hashes read through the ring vs the oracle over the committed history.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import configs, workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ne():
+    import hashed_gram_embedding_horner_b200 as m
+    return m
+
+
+def dev_i32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+
+def csr(lists):
+    off = np.concatenate([[0], np.cumsum([len(x) for x in lists])]).astype(np.int32)
+    flat = np.concatenate([np.asarray(x, np.int32) for x in lists]) if off[-1] else np.zeros(0, np.int32)
+    return flat, off
+
+
+def check_ring(ne, cache, ref: oracle.RingOracle):
+    ln = cache.len.cpu().numpy()
+    vf = cache.valid_from.cpu().numpy()
+    ring = cache.ring.cpu().numpy()
+    C = ring.shape[1]
+    assert ln.tolist() == ref.lengths()
+    assert vf.tolist() == ref.valid_from
+    for b, h in enumerate(ref.hist):
+        for pos in range(max(ref.valid_from[b], 0), len(h)):
+            assert ring[b, pos % C] == h[pos], (b, pos)
+
+
+def test_append_rollback_match_history_model(ne):
+    rng = np.random.default_rng(3)
+    N, C, B, V0 = 5, 16, 6, 131072
+    plan = ne.ngram_embed_plan_create(V0, 4096, N, 2, configs.FULL_SCALE.V_nk, ne.NGRAM_BF16)
+    ws = ne.new_workspace(plan, 64)
+    cache = ne.Cache.empty(B, C)
+    ne.ngram_cache_reset(plan, cache, ws)
+    ref = oracle.RingOracle(B, C, N)
+    for step in range(40):
+        slots = rng.permutation(B)[: rng.integers(1, B + 1)].astype(np.int32)
+        if rng.random() < 0.6:
+            ids = [rng.integers(0, V0, rng.integers(0, C + 3)).tolist() for _ in slots]
+            flat, off = csr(ids)
+            ne.ngram_cache_append(plan, cache, dev_i32(flat) if len(flat) else dev_i32([0])[:0], dev_i32(off), ws,
+                                  slots=dev_i32(slots))
+            want_bad = False
+            for s, x in zip(slots, ids):
+                want_bad |= not ref.append(int(s), x)
+        else:
+            counts = rng.integers(-1, 8, len(slots)).astype(np.int32)
+            ne.ngram_cache_rollback(plan, cache, dev_i32(counts), ws, slots=dev_i32(slots))
+            want_bad = False
+            for s, r in zip(slots, counts):
+                want_bad |= not ref.rollback(int(s), int(r))
+        status = ne.ngram_embed_get_status(ws)
+        names = ne.status_names(status)
+        assert bool(names) == want_bad, (step, names)
+        ne.ngram_embed_clear_status(ws)
+        check_ring(ne, cache, ref)
+
+
+def test_commit_paths_agree_on_device(ne):
+    """append(5) + rollback(4 - a) leaves the same committed history as append(1 + a)."""
+    N, C, B = 3, 8, 5
+    plan = ne.ngram_embed_plan_create(1000, 64, N, 2, [4099, 5003, 6007, 7001], ne.NGRAM_BF16)
+    ws = ne.new_workspace(plan, 64)
+    c1, c2 = ne.Cache.empty(B, C), ne.Cache.empty(B, C)
+    for c in (c1, c2):
+        ne.ngram_cache_reset(plan, c, ws)
+    step = np.arange(B * 5, dtype=np.int32) % 1000
+    off5 = (np.arange(B + 1) * 5).astype(np.int32)
+    for rnd in range(4):
+        a = np.array([(b + rnd) % 5 for b in range(B)], np.int32)
+        ne.ngram_cache_append(plan, c1, dev_i32(step + rnd), dev_i32(off5), ws)
+        ne.ngram_cache_rollback(plan, c1, dev_i32(4 - a), ws)
+        acc = [list(step[b * 5: b * 5 + 1 + a[b]] + rnd) for b in range(B)]
+        flat, off = csr(acc)
+        ne.ngram_cache_append(plan, c2, dev_i32(flat), dev_i32(off), ws)
+    assert ne.ngram_embed_get_status(ws) == 0
+    assert torch.equal(c1.len, c2.len)
+    ln = c1.len.cpu().numpy()
+    r1, r2 = c1.ring.cpu().numpy(), c2.ring.cpu().numpy()
+    for b in range(B):
+        for pos in range(int(ln[b]) - (N - 1), int(ln[b])):
+            assert r1[b, pos % C] == r2[b, pos % C]
+
+
+def test_decode_hashes_through_ring(ne):
+    """Spec-decode workload: per step, hashes of the 5 in-step ids read the ring's
+    committed history; equal (bit-exact) to the oracle over the full history."""
+    cfg = configs.SPEC_DECODE
+    ds = workloads.DecodeStream(cfg, num_seqs=64)
+    B, P, C = ds.B, ds.P, cfg.ring_capacity
+    plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
+    ws = ne.new_workspace(plan, B * P)
+    cache = ne.Cache.empty(B, C)
+    ne.ngram_cache_reset(plan, cache, ws)
+    ref = oracle.RingOracle(B, C, cfg.N)
+    ids, poff = ds.prompts()
+    # prompts longer than C are committed in chunks of at most C ids
+    for start in range(0, 17, C):
+        chunk = [ids[poff[b] + start: min(poff[b + 1], poff[b] + start + C)] for b in range(B)]
+        flat, off = csr(chunk)
+        ne.ngram_cache_append(plan, cache, dev_i32(flat) if len(flat) else dev_i32([0])[:0], dev_i32(off), ws)
+        for b in range(B):
+            ref.append(b, chunk[b])
+    off_step = dev_i32(ds.step_offsets())
+    idx = torch.empty((B * P, cfg.S), dtype=torch.int32, device="cuda")
+    for step in range(12):
+        tok = ds.step_tokens(step)
+        ne.ngram_hash_indices(plan, dev_i32(tok), off_step, idx, ws, cache=cache)
+        want = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk,
+                                   oracle.context_windows(cfg.N, tok, ds.step_offsets(), histories=ref.histories()))
+        np.testing.assert_array_equal(idx.cpu().numpy(), want)
+        a = ds.accept_lengths(step)
+        ne.ngram_cache_append(plan, cache, dev_i32(tok), off_step, ws)
+        ne.ngram_cache_rollback(plan, cache, dev_i32(P - 1 - a), ws)
+        for b in range(B):
+            assert ref.append(b, tok[b * P:(b + 1) * P]) and ref.rollback(b, int(P - 1 - a[b]))
+        assert ne.ngram_embed_get_status(ws) == 0
+    check_ring(ne, cache, ref)
+
+
+def test_evicted_context_is_flagged(ne):
+    N, C = 5, 4  # capacity exactly N-1
+    plan = ne.ngram_embed_plan_create(1000, 64, N, 1, [4099, 5003, 6007, 7001], ne.NGRAM_BF16)
+    ws = ne.new_workspace(plan, 16)
+    cache = ne.Cache.empty(1, C)
+    ne.ngram_cache_reset(plan, cache, ws)
+    ne.ngram_cache_append(plan, cache, dev_i32([1, 2, 3, 4]), dev_i32([0, 4]), ws)
+    ne.ngram_cache_append(plan, cache, dev_i32([5, 6]), dev_i32([0, 2]), ws)  # holds positions 2..5
+    idx = torch.empty((1, 4), dtype=torch.int32, device="cuda")
+    ne.ngram_hash_indices(plan, dev_i32([9]), dev_i32([0, 1]), idx, ws, cache=cache)
+    assert ne.ngram_embed_get_status(ws) == 0
+    want = oracle.hash_indices(1000, N, 1, [4099, 5003, 6007, 7001],
+                               oracle.context_windows(N, np.array([9], np.int32), [0, 1],
+                                                      histories=[[1, 2, 3, 4, 5, 6]]))
+    np.testing.assert_array_equal(idx.cpu().numpy(), want)
+    # a rollback that would need position 1 again is refused and changes nothing
+    ne.ngram_cache_rollback(plan, cache, dev_i32([1]), ws)
+    assert ne.status_names(ne.ngram_embed_get_status(ws)) == ["BAD_ROLLBACK"]
+    assert cache.len.item() == 6
+    ne.ngram_embed_clear_status(ws)
+    # a caller that corrupts valid_from makes the context read an evicted position
+    cache.valid_from.fill_(5)
+    ne.ngram_hash_indices(plan, dev_i32([9]), dev_i32([0, 1]), idx, ws, cache=cache)
+    assert ne.status_names(ne.ngram_embed_get_status(ws)) == ["EVICTED"]

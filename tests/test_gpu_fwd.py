@@ -1,0 +1,247 @@
+"""GPU parity of the whole layer (Eq. 3 of "Scaling Embeddings Outperforms Scaling
+Experts in Language Models", section 2) against the fp64 oracle.
+
+Tolerance (bf16 tables, fp32 accumulation, bf16 output): max|err| <= 2e-2 and
+rel-L2 <= 5e-3 vs fp64. Sizes span several 128-token tiles with a ragged tail;
+the full-size workloads are checked on sampled rows the oracle computes one by one,
+in the launch configuration the bench times.
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import configs, gen, workloads
+from tests.helpers import assert_close, device_tables, host_W, oracle_rows, to_device, to_host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ne():
+    import hashed_gram_embedding_horner_b200 as m
+    return m
+
+
+def dev_i32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+
+def plan_for(ne, cfg, variant=0, tile_n=None):
+    plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk,
+                                      ne.NGRAM_BF16 if cfg.dtype == "bf16" else ne.NGRAM_F32)
+    if variant:
+        ne.ngram_embed_plan_set_variant(plan, variant)
+    if tile_n:
+        ne.ngram_embed_plan_set_tile_n(plan, tile_n)
+    return plan
+
+
+def run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W, cache=None):
+    T = len(tokens)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    out = torch.full((T, cfg.D), float("nan"), dtype=dt, device="cuda")
+    ws = ne.new_workspace(plan, T)
+    ne.ngram_embed_fwd(plan, dev_i32(tokens), dev_i32(offsets), E0, E, W, out, ws, cache=cache)
+    return out, ne.ngram_embed_get_status(ws)
+
+
+def small_cfg(V0, D, N, K, seed=1, dtype="bf16"):
+    S = (N - 1) * K
+    V = tuple(configs.primes_from(1009 + 37 * s * s, 1)[0] for s in range(S))
+    return configs.NgramConfig(name=f"D{D}N{N}K{K}", V0=V0, D=D, N=N, K=K, V_nk=V, dtype=dtype, seed=seed)
+
+
+RAGGED = [1, 0, 37, 130, 133]   # T = 301: three 128-token tiles, the last one ragged
+
+
+def ragged_tokens(cfg, lengths=RAGGED):
+    off = gen.offsets_from_lengths(lengths)
+    return gen.zipf_tokens(cfg.seed + 17, int(off[-1]), cfg.V0), off
+
+
+# ---------------------------------------------------------------- small shapes, every kernel
+
+def test_tiny_fp32_config_full_parity(ne):
+    cfg = configs.TINY
+    tokens, offsets = workloads.prefill_tokens(cfg)
+    E0, E, W = device_tables(cfg, fill_on_device=False)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    plan = plan_for(ne, cfg)
+    assert not ne.ngram_embed_plan_uses_tensor_cores(plan)
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    ma, rl = assert_close(to_host_f64(out), want, what="tiny fp32")
+    assert rl < 1e-6  # fp32 tables and accumulation: far inside the bf16 tolerance
+
+
+SHAPES = [(5000, 256, 3, 2), (5000, 512, 5, 2), (3000, 1024, 3, 2), (5000, 384, 2, 3), (4000, 512, 3, 4)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "V0%d_D%d_N%d_K%d" % s)
+@pytest.mark.parametrize("variant,tile_n", [(1, 256), (1, 128), (2, 256), (2, 128), (3, None)],
+                         ids=["tc_gather4_n256", "tc_gather4_n128", "tc_cpasync_n256", "tc_cpasync_n128", "simt"])
+def test_small_shapes_all_kernels(ne, shape, variant, tile_n):
+    cfg = small_cfg(*shape)
+    if tile_n == 256 and cfg.D % 256:
+        pytest.skip("D not a multiple of 256")
+    tokens, offsets = ragged_tokens(cfg)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = plan_for(ne, cfg, variant, tile_n)
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    assert_close(to_host_f64(out), want, what=f"{cfg.name} variant {variant}")
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("D,N,K", [(384, 2, 3), (896, 8, 1)])  # S + 1 = 4 or 8: the scale is exact
+def test_gather_and_layout_bit_exact(ne, variant, D, N, K):
+    """W = I and E_0 = 0: out = concat_s E_s[idx_s] / (S+1) exactly (a product by 1 and a power
+    of two), so every gathered element must land in its place bit for bit. Then all E_s = 0:
+    out = E_0[t] / (S+1) exactly, which pins the E_0 gather of the epilogue."""
+    cfg = small_cfg(7000, D, N, K, seed=3)
+    S = cfg.S
+    tokens, offsets = ragged_tokens(cfg, [5, 128, 200, 3])
+    from tests.helpers import host_tables
+    E0h, Eh, _ = host_tables(cfg)
+    eye = gen.f32_to_bf16_bits(np.eye(D, dtype=np.float32))
+    idx = oracle.hash_indices(cfg.V0, N, K, cfg.V_nk, oracle.context_windows(N, tokens, offsets))
+    G = np.concatenate([gen.bf16_bits_to_f32(Eh[s][idx[:, s]]) for s in range(S)], axis=1)
+    plan = plan_for(ne, cfg, variant)
+    zeros0 = torch.zeros((cfg.V0, D), dtype=torch.bfloat16, device="cuda")
+    Ed = [to_device(e, torch.bfloat16) for e in Eh]
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, zeros0, Ed, to_device(eye, torch.bfloat16))
+    assert status == 0
+    got = out.float().cpu().numpy()
+    np.testing.assert_array_equal(got, G / (S + 1))
+    zeros = [torch.zeros_like(e) for e in Ed]
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, to_device(E0h, torch.bfloat16), zeros,
+                          to_device(eye, torch.bfloat16))
+    np.testing.assert_array_equal(out.float().cpu().numpy(), gen.bf16_bits_to_f32(E0h[tokens]) / (S + 1))
+
+
+def test_n1_is_base_embedding(ne):
+    cfg = configs.NgramConfig(name="n1", V0=3000, D=256, N=1, K=1, V_nk=(), dtype="bf16")
+    tokens, offsets = ragged_tokens(cfg)
+    E0h = gen.table_bf16(0, gen.TAG_E0, cfg.V0, cfg.D, 0.02)
+    plan = plan_for(ne, cfg)
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, to_device(E0h, torch.bfloat16), [], None)
+    assert status == 0
+    np.testing.assert_array_equal(out.float().cpu().numpy(), gen.bf16_bits_to_f32(E0h[tokens]))
+
+
+def test_gather_api_bit_exact(ne):
+    cfg = small_cfg(5000, 512, 5, 2)
+    tokens, offsets = ragged_tokens(cfg)
+    from tests.helpers import host_tables
+    _, Eh, _ = host_tables(cfg)
+    idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, oracle.context_windows(cfg.N, tokens, offsets))
+    plan = plan_for(ne, cfg)
+    ws = ne.new_workspace(plan, len(tokens))
+    G = torch.empty((len(tokens), cfg.D), dtype=torch.bfloat16, device="cuda")
+    ne.ngram_embed_gather(plan, dev_i32(idx), [to_device(e, torch.bfloat16) for e in Eh], G, ws)
+    want = oracle.gather_rows(Eh, idx).reshape(len(tokens), cfg.D)
+    np.testing.assert_array_equal(G.view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
+def test_project_api_flags_bad_indices(ne):
+    cfg = small_cfg(5000, 256, 3, 2)
+    tokens, offsets = ragged_tokens(cfg, [130])
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, oracle.context_windows(cfg.N, tokens, offsets))
+    plan = plan_for(ne, cfg)
+    ws = ne.new_workspace(plan, len(tokens))
+    out = torch.empty((len(tokens), cfg.D), dtype=torch.bfloat16, device="cuda")
+    args = (to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16))
+    ne.ngram_embed_project(plan, dev_i32(tokens), dev_i32(idx), *args, out, ws)
+    assert ne.ngram_embed_get_status(ws) == 0
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    assert_close(to_host_f64(out), want, what="project")
+    bad = idx.copy()
+    bad[3, 1] = cfg.V_nk[1]      # one past the end of sub-table 1
+    ne.ngram_embed_project(plan, dev_i32(tokens), dev_i32(bad), *args, out, ws)
+    assert "BAD_TOKEN" in ne.status_names(ne.ngram_embed_get_status(ws))
+
+
+# ---------------------------------------------------------------- full-size workloads (sampled)
+
+def sample_rows(offsets, T, n=192, seed=0):
+    rng = np.random.default_rng(seed)
+    edges = []
+    for b in range(len(offsets) - 1):
+        s, e = int(offsets[b]), int(offsets[b + 1])
+        edges += [x for x in (s, s + 1, s + 2, s + 3, e - 1) if s <= x < e]
+    rows = np.unique(np.concatenate([np.array(edges, np.int64), rng.integers(0, T, n), [T - 1]]))
+    return rows
+
+
+@pytest.mark.parametrize("cfg", [configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN, configs.FULL_SCALE],
+                         ids=lambda c: c.name)
+def test_full_size_prefill_sampled(ne, cfg):
+    tokens, offsets = workloads.prefill_tokens(cfg)
+    T = len(tokens)
+    E0, E, W = device_tables(cfg)
+    plan = plan_for(ne, cfg)
+    assert ne.ngram_embed_plan_uses_tensor_cores(plan)
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    assert not torch.isnan(out).any()
+    rows = sample_rows(offsets, T)
+    want = oracle_rows(cfg, tokens, offsets, rows, host_W(cfg))
+    assert_close(to_host_f64(out[torch.from_numpy(rows).cuda()]), want, what=cfg.name)
+    # the second A loader computes the same MMAs on the same shared-memory tiles
+    ne.ngram_embed_plan_set_variant(plan, 2)
+    out2, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0 and torch.equal(out, out2)
+    del E0, E, W, out, out2
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def test_spec_decode_forward_through_ring(ne):
+    """Spec-decode workload (B = 256, 5 ids per sequence per step): each step's outputs read
+    their context from the ring; sampled rows vs the oracle over the committed history."""
+    cfg = configs.SPEC_DECODE
+    ds = workloads.DecodeStream(cfg)
+    B, P, C = ds.B, ds.P, cfg.ring_capacity
+    E0, E, W = device_tables(cfg)
+    Wh = host_W(cfg)
+    plan = plan_for(ne, cfg)
+    ws = ne.new_workspace(plan, B * P)
+    cache = ne.Cache.empty(B, C)
+    ne.ngram_cache_reset(plan, cache, ws)
+    ref = oracle.RingOracle(B, C, cfg.N)
+    ids, poff = ds.prompts()
+    for start in range(0, cfg.prompt_max + 1, C):
+        chunk = [ids[poff[b] + start: min(poff[b + 1], poff[b] + start + C)] for b in range(B)]
+        off = gen.offsets_from_lengths([len(c) for c in chunk])
+        flat = np.concatenate(chunk).astype(np.int32) if off[-1] else np.zeros(1, np.int32)
+        ne.ngram_cache_append(plan, cache, dev_i32(flat), dev_i32(off), ws)
+        for b in range(B):
+            ref.append(b, chunk[b])
+    off_step = ds.step_offsets()
+    out = torch.empty((B * P, cfg.D), dtype=torch.bfloat16, device="cuda")
+    for step in range(4):
+        tok = ds.step_tokens(step)
+        ne.ngram_embed_fwd(plan, dev_i32(tok), dev_i32(off_step), E0, E, W, out, ws, cache=cache)
+        rows = sample_rows(off_step, B * P, n=48, seed=step)
+        want = oracle_rows(cfg, tok, off_step, rows, Wh, histories=ref.histories())
+        assert_close(to_host_f64(out[torch.from_numpy(rows).cuda()]), want, what=f"decode step {step}")
+        a = ds.accept_lengths(step)
+        ne.ngram_cache_append(plan, cache, dev_i32(tok), dev_i32(off_step), ws)
+        ne.ngram_cache_rollback(plan, cache, dev_i32(P - 1 - a), ws)
+        for b in range(B):
+            ref.append(b, tok[b * P:(b + 1) * P])
+            ref.rollback(b, int(P - 1 - a[b]))
+    assert ne.ngram_embed_get_status(ws) == 0
+    del E0, E, W
+    gc.collect()
+    torch.cuda.empty_cache()
