@@ -53,7 +53,7 @@ def test_append_rollback_match_history_model(ne):
         if rng.random() < 0.6:
             ids = [rng.integers(0, V0, rng.integers(0, C + 3)).tolist() for _ in slots]
             flat, off = csr(ids)
-            ne.ngram_cache_append(plan, cache, dev_i32(flat) if len(flat) else dev_i32([0])[:0], dev_i32(off), ws,
+            ne.ngram_cache_append(plan, cache, dev_i32(flat) if len(flat) else dev_i32([0]), dev_i32(off), ws,
                                   slots=dev_i32(slots))
             want_bad = False
             for s, x in zip(slots, ids):
@@ -113,7 +113,7 @@ def test_decode_hashes_through_ring(ne):
     for start in range(0, 17, C):
         chunk = [ids[poff[b] + start: min(poff[b + 1], poff[b] + start + C)] for b in range(B)]
         flat, off = csr(chunk)
-        ne.ngram_cache_append(plan, cache, dev_i32(flat) if len(flat) else dev_i32([0])[:0], dev_i32(off), ws)
+        ne.ngram_cache_append(plan, cache, dev_i32(flat) if len(flat) else dev_i32([0]), dev_i32(off), ws)
         for b in range(B):
             ref.append(b, chunk[b])
     off_step = dev_i32(ds.step_offsets())
