@@ -34,6 +34,11 @@ WORKLOADS = {
     "prefill_d2048": configs.PREFILL_D2048,
     "prefill_varlen_d4096": configs.PREFILL_D4096_VARLEN,
     "full_scale_prefill": configs.FULL_SCALE,
+    # small case of the prefill_d2048 kernel shape for profiler captures: ~1.1 GB of
+    # tables (still far above the 126 MB L2), 2 x 4096 tokens
+    "profile_d2048": configs.PREFILL_D2048.with_(
+        name="profile_bf16_D2048_N3_K2_small", num_seqs=2,
+        V_nk=tuple(configs.primes_from(270000 + 131072 // 2, 4))),
 }
 L2_FLUSH_BYTES = 256 << 20
 
@@ -108,7 +113,7 @@ def dist_env():
 
 # ------------------------------------------------------------------ reference arm: the oracle
 
-def oracle_sample_rate(cfg, budget_s: float = 15.0, max_tokens: int = 4096):
+def oracle_sample_rate(cfg, budget_s: float = 15.0, max_tokens: int = 32768):
     """Time the fp64 CPU oracle (exact hash + Eq. 3 combine) on a bounded sample of the
     workload's tokens; the table rows it reads are regenerated beforehand (not timed)."""
     import oracle
@@ -180,6 +185,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    ap.add_argument("--profile-only", action="store_true",
+                    help="warm up, run --steps forward calls back to back and exit (for profiler captures)")
     args = ap.parse_args()
     cfg = WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -219,6 +226,13 @@ def main():
     torch.cuda.synchronize()
     if ne.ngram_embed_get_status(ws) != 0:
         raise RuntimeError(f"device status {ne.status_names(ne.ngram_embed_get_status(ws))}")
+    if args.profile_only:
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_only": cfg.name, "steps": args.steps,
+                          "status": ne.ngram_embed_get_status(ws)}), flush=True)
+        return
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:

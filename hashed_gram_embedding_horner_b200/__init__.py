@@ -31,14 +31,15 @@ STATUS_BITS = {
     0x1: "BAD_TOKEN", 0x2: "BAD_OFFSETS", 0x4: "BAD_SLOT", 0x8: "BAD_APPEND",
     0x10: "BAD_ROLLBACK", 0x20: "EVICTED", 0x40: "TIMEOUT",
 }
-VARIANT_AUTO, VARIANT_TC_GATHER4, VARIANT_TC_CPASYNC, VARIANT_SIMT = 0, 1, 2, 3
+VARIANT_AUTO, VARIANT_TC_TMA_ROWS, VARIANT_TC_SPLIT_ROWS, VARIANT_SIMT = 0, 1, 2, 3
 
 EXPORTED = [
     "ngram_embed_plan_create", "ngram_embed_plan_destroy", "ngram_embed_workspace_bytes",
     "ngram_embed_fwd", "ngram_hash_indices", "ngram_embed_project", "ngram_embed_gather",
     "ngram_cache_reset", "ngram_cache_append", "ngram_cache_rollback", "ngram_embed_get_status",
     "ngram_embed_clear_status", "ngram_embed_error_string", "ngram_embed_plan_uses_tensor_cores",
-    "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_selftest_wait_timeout",
+    "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_plan_set_tma_rows",
+    "ngram_embed_selftest_wait_timeout",
 ]
 
 
@@ -72,6 +73,7 @@ _sig("ngram_embed_error_string", [ctypes.c_int], ctypes.c_char_p)
 _sig("ngram_embed_plan_uses_tensor_cores", [_P])
 _sig("ngram_embed_plan_set_variant", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tile_n", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
 
 
@@ -149,6 +151,10 @@ def ngram_embed_plan_set_variant(plan: Plan, variant: int):
 
 def ngram_embed_plan_set_tile_n(plan: Plan, tile_n: int):
     _check(_lib.ngram_embed_plan_set_tile_n(plan.handle, tile_n), "ngram_embed_plan_set_tile_n")
+
+
+def ngram_embed_plan_set_tma_rows(plan: Plan, rows: int):
+    _check(_lib.ngram_embed_plan_set_tma_rows(plan.handle, rows), "ngram_embed_plan_set_tma_rows")
 
 
 def ngram_embed_plan_uses_tensor_cores(plan: Plan) -> bool:

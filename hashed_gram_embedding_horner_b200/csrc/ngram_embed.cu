@@ -28,7 +28,8 @@ namespace {
 constexpr size_t kStatusBytes = 256;  // status word + padding; the index buffer follows
 constexpr int kStages = 4;
 
-enum Variant : int { kAuto = 0, kTcGather4 = 1, kTcCpAsync = 2, kSimt = 3 };
+enum Variant : int { kAuto = 0, kTcTmaRows = 1, kTcSplitRows = 2, kSimt = 3 };
+constexpr int kDefaultTmaRows = 0;  // A rows per tile gathered by TMA; the rest by cp.async (fastest measured)
 
 }  // namespace
 
@@ -41,7 +42,8 @@ struct ngram_embed_plan {
   uint64_t barrett[kMaxS];
   int device;
   int sms;
-  int variant;  // resolved: kTcGather4, kTcCpAsync or kSimt
+  int variant;  // resolved: kTcTmaRows, kTcSplitRows or kSimt
+  int tma_rows; // tensor-core kernel: A rows per tile gathered by TMA (multiple of 32)
   int bn;       // tensor-core tile width (256 or 128)
   bool tc_ok;   // the shape admits the tensor-core kernel
   // tensor-map cache (re-encoded when a table or W pointer changes)
@@ -49,7 +51,7 @@ struct ngram_embed_plan {
   const void* map_W = nullptr;
   const void* map_E[kMaxS] = {};
   bool maps_valid = false;
-  bool smem_attr_set[4] = {};  // per (tile width, A loader) kernel instance, on `device`
+  bool smem_attr_set[2] = {};  // per tile-width kernel instance, on `device`
 };
 
 namespace {
@@ -113,11 +115,11 @@ int refresh_maps(ngram_embed_plan* p, const void* const* E_nk, const void* W) {
   return NGRAM_OK;
 }
 
-template <int BN, int AMODE>
+template <int BN>
 int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
   using L = ProjSmem<BN, kStages>;
-  auto kern = proj_sm100_kernel<BN, kStages, AMODE>;
-  const int key = (BN == 256 ? 2 : 0) + AMODE;
+  auto kern = proj_sm100_kernel<BN, kStages>;
+  const int key = BN == 256 ? 1 : 0;
   if (!p->smem_attr_set[key]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess)
       return NGRAM_ERR_CUDA;
@@ -245,9 +247,8 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   prm.num_k_blocks = p->D / kBK;
   prm.scale = 1.0f / static_cast<float>(p->S + 1);
   prm.status = status_ptr(ws);
-  if (p->bn == 256)
-    return p->variant == kTcGather4 ? launch_tc<256, kGather4>(p, prm, st) : launch_tc<256, kCpAsync>(p, prm, st);
-  return p->variant == kTcGather4 ? launch_tc<128, kGather4>(p, prm, st) : launch_tc<128, kCpAsync>(p, prm, st);
+  prm.tma_rows = p->variant == kTcTmaRows ? kBM : p->tma_rows;
+  return p->bn == 256 ? launch_tc<256>(p, prm, st) : launch_tc<128>(p, prm, st);
 }
 
 int check_tables(const ngram_embed_plan* p, const void* E0, const void* const* E_nk, const void* W) {
@@ -319,7 +320,8 @@ int ngram_embed_plan_create(const ngram_embed_config* cfg, ngram_embed_plan** ou
   }
   p->tc_ok = cfg->dtype == NGRAM_BF16 && S > 0 && cfg->D % 128 == 0 && d % kBK == 0;
   p->bn = cfg->D % 256 == 0 ? 256 : 128;
-  p->variant = p->tc_ok ? kTcGather4 : kSimt;
+  p->variant = p->tc_ok ? kTcSplitRows : kSimt;
+  p->tma_rows = kDefaultTmaRows;
   *out = p;
   return NGRAM_OK;
 }
@@ -333,12 +335,20 @@ int ngram_embed_plan_uses_tensor_cores(const ngram_embed_plan* plan) {
   return plan && plan->variant != kSimt ? 1 : 0;
 }
 
-// Select the projection kernel: 0 = automatic, 1 = tensor cores with TMA row gathers,
-// 2 = tensor cores with cp.async row gathers, 3 = CUDA cores.
+// Select the projection kernel: 0 = automatic, 1 = tensor cores with every A row gathered by
+// TMA, 2 = tensor cores with the A rows split between TMA and cp.async, 3 = CUDA cores.
 int ngram_embed_plan_set_variant(ngram_embed_plan* plan, int variant) {
   if (!plan || variant < kAuto || variant > kSimt) return NGRAM_ERR_INVALID_ARG;
-  if ((variant == kTcGather4 || variant == kTcCpAsync) && !plan->tc_ok) return NGRAM_ERR_UNSUPPORTED;
-  plan->variant = variant == kAuto ? (plan->tc_ok ? kTcGather4 : kSimt) : variant;
+  if ((variant == kTcTmaRows || variant == kTcSplitRows) && !plan->tc_ok) return NGRAM_ERR_UNSUPPORTED;
+  plan->variant = variant == kAuto ? (plan->tc_ok ? kTcSplitRows : kSimt) : variant;
+  return NGRAM_OK;
+}
+
+// Tensor-core kernel, variant 2: how many of the 128 rows of each A tile TMA gathers
+// (0, 32, 64, 96 or 128); cp.async gathers the rest.
+int ngram_embed_plan_set_tma_rows(ngram_embed_plan* plan, int rows) {
+  if (!plan || rows < 0 || rows > kBM || rows % 32 != 0) return NGRAM_ERR_INVALID_ARG;
+  plan->tma_rows = rows;
   return NGRAM_OK;
 }
 

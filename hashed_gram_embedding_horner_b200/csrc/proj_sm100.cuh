@@ -6,18 +6,28 @@
 // The contraction G * W_stacked^T (G[i] = concat_s E_s[idx[i][s]]) runs on tcgen05.mma
 // (kind::f16, bf16 in, fp32 accumulate in TMEM). A k-block of 64 columns always lies
 // inside one sub-table (d % 64 == 0), so each A tile row is one 128-byte slice of one
-// gathered sub-table row: A tiles are gathered straight from HBM into shared memory in
-// the 128-byte-swizzled K-major layout, and G never exists in global memory.
+// gathered sub-table row: A tiles are gathered straight from HBM/L2 into shared memory
+// in the 128-byte-swizzled K-major layout, and G never exists in global memory.
 //
-// Persistent kernel, one CTA per SM, warp-specialised (12 warps):
-//   warps 0-3   A producers. Mode kGather4: warp 0 issues TMA tile::gather4 loads (each
-//               lane 4 rows of the 128-row tile). Mode kCpAsync: 128 threads each copy
-//               one row with 16-byte cp.async into the swizzled slot, then make the
-//               writes visible to the tensor core (wait, proxy fence, arrive).
-//   warp 4      W producer: one lane issues 2-D TMA loads of W_stacked tiles.
-//   warp 5      TMEM allocator; one lane issues the MMAs and commits.
-//   warps 8-11  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+// Gathering 128-byte row slices is the expensive part: per SM, a TMA tile::gather4
+// (four rows) and the load/store units each sustain only a fraction of the rate the
+// tensor core consumes. So the 128 rows of each A tile are split: the first `tma_rows`
+// rows arrive by TMA gather4, the rest by 16-byte cp.async, and both engines run in
+// parallel. cp.async writes through the generic proxy; their completion is tracked by
+// the stage's mbarrier (cp.async.mbarrier.arrive.noinc), and the MMA thread issues a
+// generic->async proxy fence after observing the barrier and before its tcgen05.mma.
+//
+// Persistent kernel, one CTA per SM, warp-specialised (16 warps):
+//   warps 0-7   A producers (256 threads): every thread copies its share of the cp.async
+//               rows (thread t: 16-byte chunk t % 8 of rows tma_rows + t/8 + 32 j) and
+//               arrives; tma_rows/4 lanes spread over the 8 warps each issue one gather4
+//               per stage; thread 0 posts the TMA byte count.
+//   warp 8      W producer: one lane issues 2-D TMA loads of W_stacked tiles.
+//   warp 9      TMEM allocator; one lane issues the MMAs and commits.
+//   warps 12-15 epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //               32*(w%4) ..+31), + E_0 row slice, * 1/(S+1), bf16 RNE, store.
+// Each tile walks its k-blocks starting at a tile-dependent rotation, so CTAs that share
+// a W column block (or an A row block) do not read the same lines at the same time.
 // Shared memory holds STAGES (A, B) stage pairs; TMEM holds two BN-column fp32
 // accumulators so the epilogue of one tile overlaps the main loop of the next.
 // Every wait is bounded (see mbar_wait); on a timeout all roles stop, drain what they
@@ -30,12 +40,12 @@ namespace ngram {
 
 constexpr int kBM = 128;  // tokens per tile (UMMA M, TMEM lanes)
 constexpr int kBK = 64;   // bf16 columns per k-block = one 128-byte swizzle row
-constexpr int kProjThreads = 384;
-constexpr int kWarpB = 4;
-constexpr int kWarpMma = 5;
-constexpr int kWarpEpi0 = 8;
-
-enum AMode : int { kGather4 = 0, kCpAsync = 1 };
+constexpr int kProjThreads = 512;
+constexpr int kAWarps = 8;
+constexpr int kAThreads = kAWarps * 32;
+constexpr int kWarpB = 8;
+constexpr int kWarpMma = 9;
+constexpr int kWarpEpi0 = 12;
 
 struct ProjParams {
   const int32_t* tokens;  // [T]
@@ -48,6 +58,7 @@ struct ProjParams {
   uint32_t V0;
   int D, S, d;
   int num_m_blocks, num_n_blocks, num_k_blocks;
+  int tma_rows;           // rows of each A tile gathered by TMA (multiple of 32, 0..128)
   float scale;
   int* status;
 };
@@ -77,7 +88,19 @@ __device__ __forceinline__ uint32_t clamp_row(int32_t r, uint32_t V, int* status
   return static_cast<uint32_t>(r);
 }
 
-template <int BN, int STAGES, int AMODE>
+// First k-block of a tile: a rotation that differs between tiles running side by side.
+__device__ __forceinline__ int k_rotation(int m_blk, int n_blk, int KB) { return (m_blk * 5 + n_blk * 3) % KB; }
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued before has landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <int BN, int STAGES>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_sm100_kernel(const __grid_constant__ ProjMaps maps, const __grid_constant__ ProjParams p) {
   using L = ProjSmem<BN, STAGES>;
@@ -99,10 +122,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    const uint32_t a_arrivals = AMODE == kGather4 ? 1u : 128u;
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), a_arrivals + 1u);  // A producer(s) + the W producer
-      mbar_init(empty_bar(s), 1u);              // one tcgen05.commit
+      // every A thread (cp.async completion), thread 0's TMA byte count, the W producer
+      mbar_init(full_bar(s), static_cast<uint32_t>(kAThreads) + 2u);
+      mbar_init(empty_bar(s), 1u);  // one tcgen05.commit
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1u);
@@ -113,9 +136,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == kWarpB && lane == 0) {
-    tma_prefetch_desc(&maps.W);
-  }
+  if (warp == kWarpB && lane == 0) tma_prefetch_desc(&maps.W);
   if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
     tmem_relinquish();
@@ -129,75 +150,68 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   const int KB = p.num_k_blocks;
   const int kb_per_sub = p.d / kBK;
 
-  if ((AMODE == kGather4 && warp == 0) || (AMODE == kCpAsync && warp < 4)) {
-    // ------------------------------------------------------------ A producer
+  if (warp < kAWarps) {
+    // ------------------------------------------------------------ A producers
+    const int t = threadIdx.x;                 // 0..255
+    const int chunk = t & 7;
+    const int rsub = t >> 3;                   // 0..31
+    const int n_cp = (kBM - p.tma_rows) >> 5;  // cp.async rows per thread: tma_rows + rsub + 32 j
+    const uint32_t swz = static_cast<uint32_t>((chunk ^ (rsub & 7)) << 4);
+    // TMA issuers: lanes 0 .. tma_rows/32 - 1 of every producer warp, 4 rows each.
+    const int lanes_tma = p.tma_rows >> 5;
+    const bool tma_issuer = lane < lanes_tma;
+    const int issuer = warp * lanes_tma + lane;  // rows 4*issuer .. +3
+    const uint32_t tma_bytes = static_cast<uint32_t>(p.tma_rows) * 128u;
     const uint64_t pol = l2_policy_evict_normal();
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    int prev_stage = -1;  // kCpAsync: stage whose arrival is still held back
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int m_blk = tile / p.num_n_blocks;
-      if constexpr (AMODE == kGather4) {
-        const int64_t row0 = static_cast<int64_t>(m_blk) * kBM + lane * 4;
-        int32_t r[4];
-        for (int kb = 0; kb < KB; ++kb) {
-          const int s = kb / kb_per_sub;
-          const int c0 = (kb - s * kb_per_sub) * kBK;
-          if (kb == s * kb_per_sub) {
+      const int rot = k_rotation(m_blk, tile % p.num_n_blocks, KB);
+      const int64_t row_base = static_cast<int64_t>(m_blk) * kBM;
+      int cur_s = -1;
+      int32_t r4[4] = {0, 0, 0, 0};
+      const uint16_t* src[4] = {nullptr, nullptr, nullptr, nullptr};
+      for (int i = 0; i < KB; ++i) {
+        int kb = i + rot;
+        if (kb >= KB) kb -= KB;
+        const int s = kb / kb_per_sub;
+        const int c0 = (kb - s * kb_per_sub) * kBK;
+        if (s != cur_s) {
+          const uint32_t V = p.Vs[s];
+          if (tma_issuer) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const int64_t gr = row0 + j;
-              r[j] = gr < p.T ? static_cast<int32_t>(clamp_row(p.idx[gr * p.S + s], p.Vs[s], p.status)) : 0;
+              const int64_t gr = row_base + issuer * 4 + j;
+              r4[j] = gr < p.T ? static_cast<int32_t>(clamp_row(p.idx[gr * p.S + s], V, p.status)) : 0;
             }
           }
-          // lane 0 waits for the slot and posts the byte count; the warp follows it.
-          bool got = false;
-          if (lane == 0) {
-            got = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status);
-            if (got) mbar_arrive_expect_tx(full_bar(stage), L::kABytes);
-          }
-          if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-          tma_gather4(a_tile(stage) + lane * 512, &maps.E[s], c0, r[0], r[1], r[2], r[3],
-                      full_bar(stage), pol);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-      } else {
-        const int row = threadIdx.x;  // 0..127
-        const int64_t gr = static_cast<int64_t>(m_blk) * kBM + row;
-        const bool valid = gr < p.T;
-        const uint16_t* src = nullptr;
-        for (int kb = 0; kb < KB; ++kb) {
-          const int s = kb / kb_per_sub;
-          const int c0 = (kb - s * kb_per_sub) * kBK;
-          if (kb == s * kb_per_sub) {
-            const uint32_t ix = valid ? clamp_row(p.idx[gr * p.S + s], p.Vs[s], p.status) : 0u;
-            src = p.E[s] + static_cast<int64_t>(ix) * p.d;
-          }
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          const uint32_t dst = a_tile(stage) + row * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) cp_async_16(dst + ((c ^ (row & 7)) << 4), src + c0 + c * 8);
-          cp_async_commit();
-          if (prev_stage >= 0) {
-            cp_async_wait<1>();        // the previous stage's copies have landed
-            fence_proxy_async_smem();  // make them visible to the tensor core
-            mbar_arrive(full_bar(prev_stage));
+          for (int j = 0; j < 4; ++j) {
+            if (j < n_cp) {
+              const int64_t gr = row_base + p.tma_rows + rsub + 32 * j;
+              const uint32_t ix = gr < p.T ? clamp_row(p.idx[gr * p.S + s], V, p.status) : 0u;
+              src[j] = p.E[s] + static_cast<int64_t>(ix) * p.d + chunk * 8;
+            }
           }
-          prev_stage = stage;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          cur_s = s;
         }
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        const uint32_t a = a_tile(stage);
+        if (t == 0) mbar_arrive_expect_tx(full_bar(stage), tma_bytes);
+        if (tma_issuer)
+          tma_gather4(a + issuer * 512, &maps.E[s], c0, r4[0], r4[1], r4[2], r4[3], full_bar(stage), pol);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (j < n_cp) cp_async_16(a + (p.tma_rows + rsub + 32 * j) * 128 + swz, src[j] + c0);
+        cp_async_arrive_noinc(full_bar(stage));
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
-    if constexpr (AMODE == kCpAsync) {
-      cp_async_wait<0>();
-      if (ok && prev_stage >= 0) {
-        fence_proxy_async_smem();
-        mbar_arrive(full_bar(prev_stage));
-      }
-    } else if (!ok) {
-      // Aborting: give the gathers this warp may still have in flight time to land
-      // (bounded) before the CTA exits.
+    cp_async_wait_all();
+    if (!ok) {
+      // Aborting: give the TMA gathers still in flight time to land (bounded) before exit.
       const uint64_t t0 = globaltimer_ns();
       while (globaltimer_ns() - t0 < 1000ull * 1000ull) __nanosleep(1000);
     }
@@ -210,7 +224,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int n_blk = tile % p.num_n_blocks;
-        for (int kb = 0; kb < KB; ++kb) {
+        const int rot = k_rotation(tile / p.num_n_blocks, n_blk, KB);
+        for (int i = 0; i < KB; ++i) {
+          int kb = i + rot;
+          if (kb >= KB) kb -= KB;
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), L::kBBytes);
           tma_load_2d(b_tile(stage), &maps.W, kb * kBK, n_blk * BN, full_bar(stage), pol);
@@ -232,15 +249,15 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         if (!mbar_wait(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int i = 0; i < KB; ++i) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
-          if constexpr (AMODE == kCpAsync) fence_proxy_async_smem();
+          fence_proxy_async_smem();  // the stage's cp.async rows were written by the generic proxy
           const uint64_t adesc = sw128_kmajor_desc(a_tile(stage));
           const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage));
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)  // K = 16 per instruction: +32 B = +2 in the address field
-            umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
           umma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }

@@ -191,11 +191,15 @@ int ngram_embed_plan_uses_tensor_cores(const ngram_embed_plan* plan);
 
 /* Choose the projection kernel of a plan (for testing one implementation against another):
  *   0 = automatic (tensor cores when the shape allows: bf16, D % 128 == 0, d % 64 == 0, N >= 2),
- *   1 = tensor cores, A rows gathered by TMA (tile::gather4),
- *   2 = tensor cores, A rows gathered by 16-byte cp.async,
+ *   1 = tensor cores, every gathered A row brought in by TMA (tile::gather4),
+ *   2 = tensor cores, A rows split between TMA gather4 and 16-byte cp.async (default),
  *   3 = CUDA cores.
  * Returns NGRAM_ERR_UNSUPPORTED if the shape does not admit the chosen kernel. */
 int ngram_embed_plan_set_variant(ngram_embed_plan* plan, int variant);
+
+/* Variant 2: how many of the 128 rows of each gathered tile TMA brings in (0, 32, 64, 96
+ * or 128; default 0); cp.async brings in the rest. A tuning knob: results do not change. */
+int ngram_embed_plan_set_tma_rows(ngram_embed_plan* plan, int rows);
 
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */
 int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);

@@ -83,9 +83,11 @@ SHAPES = [(5000, 256, 3, 2), (5000, 512, 5, 2), (3000, 1024, 3, 2), (5000, 384, 
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "V0%d_D%d_N%d_K%d" % s)
-@pytest.mark.parametrize("variant,tile_n", [(1, 256), (1, 128), (2, 256), (2, 128), (3, None)],
-                         ids=["tc_gather4_n256", "tc_gather4_n128", "tc_cpasync_n256", "tc_cpasync_n128", "simt"])
-def test_small_shapes_all_kernels(ne, shape, variant, tile_n):
+@pytest.mark.parametrize("variant,tile_n,tma_rows", [(1, 256, None), (1, 128, None), (2, 256, 64), (2, 128, 64),
+                                                     (2, 256, 0), (2, 128, 32), (2, 256, 96), (3, None, None)],
+                         ids=["tc_tma_n256", "tc_tma_n128", "tc_split64_n256", "tc_split64_n128",
+                              "tc_cpasync_n256", "tc_split32_n128", "tc_split96_n256", "simt"])
+def test_small_shapes_all_kernels(ne, shape, variant, tile_n, tma_rows):
     cfg = small_cfg(*shape)
     if tile_n == 256 and cfg.D % 256:
         pytest.skip("D not a multiple of 256")
@@ -94,15 +96,17 @@ def test_small_shapes_all_kernels(ne, shape, variant, tile_n):
     E0h, Eh, Wh = host_tables(cfg)
     E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
     plan = plan_for(ne, cfg, variant, tile_n)
+    if tma_rows is not None:
+        ne.ngram_embed_plan_set_tma_rows(plan, tma_rows)
     out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
     assert status == 0
     want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
     assert_close(to_host_f64(out), want, what=f"{cfg.name} variant {variant}")
 
 
-@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("variant,tma_rows", [(1, None), (2, 0), (2, 32), (2, 64), (2, 96)])
 @pytest.mark.parametrize("D,N,K", [(384, 2, 3), (896, 8, 1)])  # S + 1 = 4 or 8: the scale is exact
-def test_gather_and_layout_bit_exact(ne, variant, D, N, K):
+def test_gather_and_layout_bit_exact(ne, variant, tma_rows, D, N, K):
     """W = I and E_0 = 0: out = concat_s E_s[idx_s] / (S+1) exactly (a product by 1 and a power
     of two), so every gathered element must land in its place bit for bit. Then all E_s = 0:
     out = E_0[t] / (S+1) exactly, which pins the E_0 gather of the epilogue."""
@@ -115,6 +119,8 @@ def test_gather_and_layout_bit_exact(ne, variant, D, N, K):
     idx = oracle.hash_indices(cfg.V0, N, K, cfg.V_nk, oracle.context_windows(N, tokens, offsets))
     G = np.concatenate([gen.bf16_bits_to_f32(Eh[s][idx[:, s]]) for s in range(S)], axis=1)
     plan = plan_for(ne, cfg, variant)
+    if tma_rows is not None:
+        ne.ngram_embed_plan_set_tma_rows(plan, tma_rows)
     zeros0 = torch.zeros((cfg.V0, D), dtype=torch.bfloat16, device="cuda")
     Ed = [to_device(e, torch.bfloat16) for e in Eh]
     out, status = run_fwd(ne, plan, cfg, tokens, offsets, zeros0, Ed, to_device(eye, torch.bfloat16))
@@ -197,10 +203,11 @@ def test_full_size_prefill_sampled(ne, cfg):
     rows = sample_rows(offsets, T)
     want = oracle_rows(cfg, tokens, offsets, rows, host_W(cfg))
     assert_close(to_host_f64(out[torch.from_numpy(rows).cuda()]), want, what=cfg.name)
-    # the second A loader computes the same MMAs on the same shared-memory tiles
-    ne.ngram_embed_plan_set_variant(plan, 2)
-    out2, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
-    assert status == 0 and torch.equal(out, out2)
+    # other splits of the A rows between TMA and cp.async feed the MMAs the same tiles
+    for rows in (0, 128):
+        ne.ngram_embed_plan_set_tma_rows(plan, rows)
+        out2, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+        assert status == 0 and torch.equal(out, out2), rows
     del E0, E, W, out, out2
     gc.collect()
     torch.cuda.empty_cache()
