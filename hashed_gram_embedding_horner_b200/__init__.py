@@ -39,7 +39,7 @@ EXPORTED = [
     "ngram_cache_reset", "ngram_cache_append", "ngram_cache_rollback", "ngram_embed_get_status",
     "ngram_embed_clear_status", "ngram_embed_error_string", "ngram_embed_plan_uses_tensor_cores",
     "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_plan_set_tma_rows",
-    "ngram_embed_selftest_wait_timeout",
+    "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws",
 ]
 
 
@@ -75,6 +75,7 @@ _sig("ngram_embed_plan_set_variant", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tile_n", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
+_sig("ngram_embed_fwd_static_ws", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P])
 
 
 class NgramError(RuntimeError):

@@ -528,3 +528,65 @@ int ngram_embed_clear_status(void* workspace, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Forward pass with library-owned scratch, for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc: plugin hosts that hand a layer only its input and
+// output buffers, and latency-critical loops where cudaMalloc's implicit device-wide
+// synchronisation is not allowed. ngram_embed_fwd_static_ws runs the same forward pass as
+// ngram_embed_fwd, but its workspace (the status word and the per-token index buffer) is
+// the fixed array below, compiled into the library. Every GPU that loads the library holds
+// these kNoAllocScratchBytes until the process exits.
+//
+// In host code `g_noalloc_scratch` names a host-side stand-in, not a device address, so the
+// array's device address is looked up with cudaGetSymbolAddress once per device, with that
+// device current, by the first call made on that device (that first call should come
+// before any stream capture). All calls share the array and it keeps the last call's
+// contents: each call zeroes the status word before use, and calls that overlap on the GPU
+// (concurrent streams) race on the array.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB: status header + T*S indices
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::once_flag g_noalloc_once[kNoAllocMaxDevices];
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+cudaError_t g_noalloc_err[kNoAllocMaxDevices] = {};
+
+void* noalloc_scratch(int device) {
+  if (device < 0 || device >= kNoAllocMaxDevices) return nullptr;
+  std::call_once(g_noalloc_once[device], [device] {
+    void* p = nullptr;
+    g_noalloc_err[device] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    g_noalloc_ptr[device] = g_noalloc_err[device] == cudaSuccess ? p : nullptr;
+  });
+  return g_noalloc_ptr[device];
+}
+
+}  // namespace
+
+extern "C" int ngram_embed_fwd_static_ws(const ngram_embed_plan* plan, const int32_t* tokens,
+                                         const int32_t* seq_offsets, int32_t num_seqs, int64_t num_tokens,
+                                         const void* E0, const void* const* E_nk, const void* W_stacked,
+                                         const ngram_cache* cache, const int32_t* cache_slots, void* out,
+                                         int32_t* status_out, void* stream) {
+  if (!plan || num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
+  if (ws_bytes(plan, num_tokens) > kNoAllocScratchBytes) return NGRAM_ERR_WORKSPACE;  // above the fixed limit
+  int rc = set_device(plan);
+  if (rc) return rc;
+  void* ws = noalloc_scratch(plan->device);
+  if (!ws) return NGRAM_ERR_CUDA;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess) return NGRAM_ERR_CUDA;  // status word
+  rc = ngram_embed_fwd(plan, tokens, seq_offsets, num_seqs, num_tokens, E0, E_nk, W_stacked, cache, cache_slots,
+                       out, ws, kNoAllocScratchBytes, stream);
+  if (rc) return rc;
+  if (status_out &&
+      cudaMemcpyAsync(status_out, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return NGRAM_ERR_CUDA;
+  return NGRAM_OK;
+}

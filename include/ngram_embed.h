@@ -172,6 +172,24 @@ int ngram_cache_rollback(const ngram_embed_plan* plan, const ngram_cache* cache,
                          const int32_t* slots, const int32_t* counts, int32_t n,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* ngram_embed_fwd for callers that cannot allocate device memory (plugin hosts that pass a
+ * layer only its inputs and outputs; latency-critical loops where cudaMalloc's implicit
+ * device-wide synchronisation is not allowed). The paper has no counterpart: this is an
+ * interface convenience. Same arguments and results as ngram_embed_fwd, but the workspace
+ * is a fixed 4 MiB array inside the library (every GPU that loads the library holds it
+ * until exit), so calls need ngram_embed_workspace_bytes(plan, num_tokens) <= 4 MiB
+ * (about num_tokens * S * 4 bytes); larger calls return NGRAM_ERR_WORKSPACE and launch
+ * nothing. Allocates nothing. The first call on a device looks up the array's device
+ * address (once per device); make that first call before any stream capture. Each call
+ * zeroes the array's status word, then, if status_out (a device int32) is not NULL, copies
+ * the call's device status bits there on `stream`. All calls share the one array: calls
+ * that overlap on the GPU (for example on two streams) race and must be avoided. */
+int ngram_embed_fwd_static_ws(const ngram_embed_plan* plan, const int32_t* tokens,
+                              const int32_t* seq_offsets, int32_t num_seqs, int64_t num_tokens,
+                              const void* E0, const void* const* E_nk, const void* W_stacked,
+                              const ngram_cache* cache, const int32_t* cache_slots, void* out,
+                              int32_t* status_out, void* stream);
+
 /* Synchronise `stream` and copy the sticky status word to *status_out. */
 int ngram_embed_get_status(const void* workspace, void* stream, int32_t* status_out);
 /* Zero the status word (asynchronous on `stream`). */
