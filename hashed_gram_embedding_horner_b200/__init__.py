@@ -39,7 +39,7 @@ EXPORTED = [
     "ngram_cache_reset", "ngram_cache_append", "ngram_cache_rollback", "ngram_embed_get_status",
     "ngram_embed_clear_status", "ngram_embed_error_string", "ngram_embed_plan_uses_tensor_cores",
     "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_plan_set_tma_rows",
-    "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws",
+    "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws", "ngram_embed_plan_set_cta_pair",
 ]
 
 
@@ -74,6 +74,7 @@ _sig("ngram_embed_plan_uses_tensor_cores", [_P])
 _sig("ngram_embed_plan_set_variant", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tile_n", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
 _sig("ngram_embed_fwd_static_ws", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P])
 
@@ -156,6 +157,10 @@ def ngram_embed_plan_set_tile_n(plan: Plan, tile_n: int):
 
 def ngram_embed_plan_set_tma_rows(plan: Plan, rows: int):
     _check(_lib.ngram_embed_plan_set_tma_rows(plan.handle, rows), "ngram_embed_plan_set_tma_rows")
+
+
+def ngram_embed_plan_set_cta_pair(plan: Plan, on: bool):
+    _check(_lib.ngram_embed_plan_set_cta_pair(plan.handle, int(bool(on))), "ngram_embed_plan_set_cta_pair")
 
 
 def ngram_embed_plan_uses_tensor_cores(plan: Plan) -> bool:

@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "hash.cuh"
 #include "proj_sm100.cuh"
+#include "proj_sm100_pair.cuh"
 #include "simt.cuh"
 
 using namespace ngram;
@@ -26,7 +27,8 @@ using namespace ngram;
 namespace {
 
 constexpr size_t kStatusBytes = 256;  // status word + padding; the index buffer follows
-constexpr int kStages = 4;
+constexpr int kStages = 4;       // one-CTA kernel: 4 x (16 KB A + 32 KB W) at N = 256
+constexpr int kPairStages = 6;   // CTA-pair kernel: 6 x (16 KB A + 16 KB W) per CTA at N = 256
 
 enum Variant : int { kAuto = 0, kTcTmaRows = 1, kTcSplitRows = 2, kSimt = 3 };
 constexpr int kDefaultTmaRows = 0;  // A rows per tile gathered by TMA; the rest by cp.async (fastest measured)
@@ -51,7 +53,9 @@ struct ngram_embed_plan {
   const void* map_W = nullptr;
   const void* map_E[kMaxS] = {};
   bool maps_valid = false;
-  bool smem_attr_set[2] = {};  // per tile-width kernel instance, on `device`
+  bool smem_attr_set[4] = {};  // per (kernel form, tile width) instance, on `device`
+  bool cta_pair = true;        // use the CTA-pair (cta_group::2) kernel
+  int max_clusters[2] = {0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
 };
 
 namespace {
@@ -104,6 +108,9 @@ int refresh_maps(ngram_embed_plan* p, const void* const* E_nk, const void* W) {
   int rc = encode_2d(&p->maps.W, W, p->D, p->D, static_cast<uint64_t>(p->D) * 2, kBK, p->bn,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
   if (rc) return rc;
+  rc = encode_2d(&p->maps.Whalf, W, p->D, p->D, static_cast<uint64_t>(p->D) * 2, kBK, p->bn / 2,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (rc) return rc;
   for (int s = 0; s < p->S; ++s) {
     rc = encode_2d(&p->maps.E[s], E_nk[s], p->d, p->V[s], static_cast<uint64_t>(p->d) * 2, kBK, 1,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
@@ -128,6 +135,45 @@ int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
   const int tiles = prm.num_m_blocks * prm.num_n_blocks;
   const int grid = tiles < p->sms ? tiles : p->sms;
   kern<<<grid, kProjThreads, L::kLaunchBytes, st>>>(p->maps, prm);
+  return check_launch();
+}
+
+// CTA-pair kernel: clusters of two CTAs, one 256 x BN tile per pair per step.
+template <int BN>
+int launch_tc_pair(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t st) {
+  constexpr int kStg = BN == 256 ? kPairStages : 8;
+  using L = PairSmem<BN, kStg>;
+  auto kern = proj_sm100_pair_kernel<BN, kStg>;
+  const int key = 2 + (BN == 256 ? 1 : 0);
+  if (!p->smem_attr_set[key]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+      return NGRAM_ERR_CUDA;
+    p->smem_attr_set[key] = true;
+  }
+  prm.num_m_blocks = static_cast<int>((T + 2 * kBM - 1) / (2 * kBM));
+  const int tiles = prm.num_m_blocks * prm.num_n_blocks;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kProjThreads);
+  cfg.dynamicSmemBytes = L::kLaunchBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int& max_pairs = p->max_clusters[BN == 256 ? 1 : 0];
+  if (max_pairs == 0) {
+    cfg.gridDim = dim3(2 * (p->sms / 2));
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return NGRAM_ERR_CUDA;
+    max_pairs = n;
+  }
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  cfg.gridDim = dim3(2 * pairs);
+  if (cudaLaunchKernelEx(&cfg, kern, p->maps, prm) != cudaSuccess) return NGRAM_ERR_CUDA;
   return check_launch();
 }
 
@@ -248,6 +294,8 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   prm.scale = 1.0f / static_cast<float>(p->S + 1);
   prm.status = status_ptr(ws);
   prm.tma_rows = p->variant == kTcTmaRows ? kBM : p->tma_rows;
+  if (p->cta_pair)
+    return p->bn == 256 ? launch_tc_pair<256>(p, prm, T, st) : launch_tc_pair<128>(p, prm, T, st);
   return p->bn == 256 ? launch_tc<256>(p, prm, st) : launch_tc<128>(p, prm, st);
 }
 
@@ -321,7 +369,10 @@ int ngram_embed_plan_create(const ngram_embed_config* cfg, ngram_embed_plan** ou
   p->tc_ok = cfg->dtype == NGRAM_BF16 && S > 0 && cfg->D % 128 == 0 && d % kBK == 0;
   p->bn = cfg->D % 256 == 0 ? 256 : 128;
   p->variant = p->tc_ok ? kTcSplitRows : kSimt;
-  p->tma_rows = kDefaultTmaRows;
+  // Defaults from B200 measurements of the two kernel forms: at D = 2048 the CTA pair with
+  // every A row gathered by TMA is fastest; at D = 4096 one CTA per tile with cp.async rows.
+  p->cta_pair = cfg->D <= 2048;
+  p->tma_rows = p->cta_pair ? kBM : kDefaultTmaRows;
   *out = p;
   return NGRAM_OK;
 }
@@ -349,6 +400,14 @@ int ngram_embed_plan_set_variant(ngram_embed_plan* plan, int variant) {
 int ngram_embed_plan_set_tma_rows(ngram_embed_plan* plan, int rows) {
   if (!plan || rows < 0 || rows > kBM || rows % 32 != 0) return NGRAM_ERR_INVALID_ARG;
   plan->tma_rows = rows;
+  return NGRAM_OK;
+}
+
+// Tensor-core kernel form: 1 = CTA pairs (cta_group::2, 256-token tiles; default),
+// 0 = one CTA per tile (128-token tiles).
+int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on) {
+  if (!plan || (on != 0 && on != 1)) return NGRAM_ERR_INVALID_ARG;
+  plan->cta_pair = on != 0;
   return NGRAM_OK;
 }
 

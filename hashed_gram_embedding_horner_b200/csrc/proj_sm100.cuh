@@ -65,6 +65,7 @@ struct ProjParams {
 
 struct ProjMaps {
   CUtensorMap W;            // W_stacked, box {64, BN}, 128-byte swizzle
+  CUtensorMap Whalf;        // W_stacked, box {64, BN/2} (CTA-pair kernel: each CTA loads half)
   CUtensorMap E[kMaxS];     // sub-table s, box {64, 1}, 128-byte swizzle (gather4)
 };
 
@@ -90,6 +91,48 @@ __device__ __forceinline__ uint32_t clamp_row(int32_t r, uint32_t V, int* status
 
 // First k-block of a tile: a rotation that differs between tiles running side by side.
 __device__ __forceinline__ int k_rotation(int m_blk, int n_blk, int KB) { return (m_blk * 5 + n_blk * 3) % KB; }
+
+// The k-blocks a tile visits (from its rotation, wrapping) fall into runs that each use one
+// sub-table. Producers walk the CTA's (tile, k-block) sequence run by run and load the row
+// indices of the next run while the current one is being copied, so the dependent index
+// load never sits between a freed stage and its refill.
+struct KRun {
+  int tile;     // tile of the run (>= number of tiles: past the end)
+  int i;        // position of the run's first k-block in the tile's sequence
+  int s;        // sub-table
+  int c_first;  // k-block offset of the run's first k-block inside the sub-table
+  int len;      // k-blocks in the run
+};
+
+__device__ __forceinline__ KRun k_run_at(int tile, int i, int num_n_blocks, int KB, int kb_per_sub) {
+  KRun r;
+  r.tile = tile;
+  r.i = i;
+  int kb = i + k_rotation(tile / num_n_blocks, tile % num_n_blocks, KB);
+  if (kb >= KB) kb -= KB;
+  r.s = kb / kb_per_sub;
+  r.c_first = kb - r.s * kb_per_sub;
+  const int rem = kb_per_sub - r.c_first;
+  r.len = rem < KB - i ? rem : KB - i;
+  return r;
+}
+
+__device__ __forceinline__ KRun k_run_next(const KRun& r, int stride, int num_n_blocks, int KB, int kb_per_sub) {
+  int i = r.i + r.len, tile = r.tile;
+  if (i >= KB) {
+    i = 0;
+    tile += stride;
+  }
+  return k_run_at(tile, i, num_n_blocks, KB, kb_per_sub);
+}
+
+// A load issued where it stands in the program (volatile asm keeps its place among the
+// producer's other asm), consumed one run later.
+__device__ __forceinline__ int32_t ld_idx_early(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -163,51 +206,53 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     const int issuer = warp * lanes_tma + lane;  // rows 4*issuer .. +3
     const uint32_t tma_bytes = static_cast<uint32_t>(p.tma_rows) * 128u;
     const uint64_t pol = l2_policy_evict_normal();
+    const int stride = static_cast<int>(gridDim.x);
+    // raw row indices of the current and the next run: cp.async rows, then TMA rows
+    int32_t raw[8], nraw[8];
+    auto load_raw = [&](const KRun& r, int32_t (&dst)[8]) {
+      const int64_t row_base = static_cast<int64_t>(r.tile / p.num_n_blocks) * kBM;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t g1 = row_base + p.tma_rows + rsub + 32 * j;
+        dst[j] = (j < n_cp && g1 < p.T) ? ld_idx_early(p.idx + g1 * p.S + r.s) : 0;
+        const int64_t g2 = row_base + issuer * 4 + j;
+        dst[4 + j] = (tma_issuer && g2 < p.T) ? ld_idx_early(p.idx + g2 * p.S + r.s) : 0;
+      }
+    };
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int m_blk = tile / p.num_n_blocks;
-      const int rot = k_rotation(m_blk, tile % p.num_n_blocks, KB);
-      const int64_t row_base = static_cast<int64_t>(m_blk) * kBM;
-      int cur_s = -1;
-      int32_t r4[4] = {0, 0, 0, 0};
-      const uint16_t* src[4] = {nullptr, nullptr, nullptr, nullptr};
-      for (int i = 0; i < KB; ++i) {
-        int kb = i + rot;
-        if (kb >= KB) kb -= KB;
-        const int s = kb / kb_per_sub;
-        const int c0 = (kb - s * kb_per_sub) * kBK;
-        if (s != cur_s) {
-          const uint32_t V = p.Vs[s];
-          if (tma_issuer) {
+    KRun cur = k_run_at(blockIdx.x, 0, p.num_n_blocks, KB, kb_per_sub);
+    if (cur.tile < num_tiles) load_raw(cur, raw);
+    KRun nxt = k_run_next(cur, stride, p.num_n_blocks, KB, kb_per_sub);
+    if (nxt.tile < num_tiles) load_raw(nxt, nraw);
+    while (cur.tile < num_tiles && ok) {
+      const uint32_t V = p.Vs[cur.s];
+      const uint16_t* src[4];
+      int32_t r4[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int64_t gr = row_base + issuer * 4 + j;
-              r4[j] = gr < p.T ? static_cast<int32_t>(clamp_row(p.idx[gr * p.S + s], V, p.status)) : 0;
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j < n_cp) {
-              const int64_t gr = row_base + p.tma_rows + rsub + 32 * j;
-              const uint32_t ix = gr < p.T ? clamp_row(p.idx[gr * p.S + s], V, p.status) : 0u;
-              src[j] = p.E[s] + static_cast<int64_t>(ix) * p.d + chunk * 8;
-            }
-          }
-          cur_s = s;
-        }
+      for (int j = 0; j < 4; ++j) {
+        src[j] = p.E[cur.s] + static_cast<int64_t>(clamp_row(raw[j], V, p.status)) * p.d + chunk * 8;
+        r4[j] = static_cast<int32_t>(clamp_row(raw[4 + j], V, p.status));
+      }
+      for (int q = 0; q < cur.len; ++q) {
+        const int c0 = (cur.c_first + q) * kBK;
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
         const uint32_t a = a_tile(stage);
         if (t == 0) mbar_arrive_expect_tx(full_bar(stage), tma_bytes);
         if (tma_issuer)
-          tma_gather4(a + issuer * 512, &maps.E[s], c0, r4[0], r4[1], r4[2], r4[3], full_bar(stage), pol);
+          tma_gather4(a + issuer * 512, &maps.E[cur.s], c0, r4[0], r4[1], r4[2], r4[3], full_bar(stage), pol);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (j < n_cp) cp_async_16(a + (p.tma_rows + rsub + 32 * j) * 128 + swz, src[j] + c0);
         cp_async_arrive_noinc(full_bar(stage));
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
+      cur = nxt;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) raw[j] = nraw[j];
+      nxt = k_run_next(nxt, stride, p.num_n_blocks, KB, kb_per_sub);
+      if (nxt.tile < num_tiles) load_raw(nxt, nraw);
     }
     cp_async_wait_all();
     if (!ok) {

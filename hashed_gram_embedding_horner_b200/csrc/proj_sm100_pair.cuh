@@ -1,0 +1,316 @@
+// Two-CTA (cta_group::2) form of the fused gather + projection + epilogue kernel.
+//
+// Same arithmetic as proj_sm100_kernel (Eq. 3 of "Scaling Embeddings Outperforms Scaling
+// Experts in Language Models", section 2), on 256 x BN tiles computed by a pair of CTAs
+// (a cluster of two on neighbouring SMs): CTA r of the pair gathers rows r*128 .. +127 of
+// the tile's A rows and loads rows r*BN/2 .. +BN/2-1 of the tile's W block; one thread of
+// CTA 0 issues tcgen05.mma.cta_group::2 (M = 256, N = BN), which reads A and B from both
+// CTAs' shared memory and writes each CTA's 128 accumulator rows into its own TMEM. Per SM
+// and k-block this moves 16 KB of A + BN/2 * 128 B of W instead of 16 KB + BN * 128 B,
+// which is what limits the one-CTA kernel (on-chip bytes in flight, not DRAM).
+//
+// Cross-CTA signalling, all plain (no multicast):
+//   - W halves (and, with tma_rows = 128, the A rows: tile::gather4, 32 issuing lanes per
+//     CTA) are TMA loads in their .cta_group::2 form: the data lands in the issuing CTA's
+//     shared memory and the byte count completes on CTA 0's stage barrier;
+//   - with tma_rows = 0 (default) the A rows arrive by 16-byte cp.async, which can only
+//     signal the issuing CTA's own barrier: CTA 0's cp.async threads arrive on CTA 0's stage
+//     barrier; CTA 1's arrive on CTA 1's, and a relay lane of CTA 1 (one lane per stage, so
+//     the slow cluster-scope release of one stage overlaps the others) waits for it, fences
+//     generic->async proxy and arrives remotely on CTA 0's stage barrier;
+//   - CTA 0's MMA thread commits stage release and "accumulator ready" to the barriers of
+//     both CTAs (two tcgen05.commit, one per CTA address);
+//   - CTA 1's epilogue warps arrive remotely on CTA 0's "accumulator free" barrier.
+// Waits on barriers that receive remote arrivals use cluster-scope acquire. Every wait is
+// bounded; both CTAs meet at cluster barriers after set-up and before teardown.
+#pragma once
+
+#include "proj_sm100.cuh"
+
+namespace ngram {
+
+constexpr int kWarpRelay = 10;
+
+template <int BN, int STAGES>
+struct PairSmem {
+  static constexpr int kABytes = kBM * kBK * 2;         // this CTA's 128 A rows
+  static constexpr int kBBytes = (BN / 2) * kBK * 2;    // this CTA's BN/2 rows of W
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kBytes = kBarOffset + kNumBars * 8 + 16;
+  static constexpr int kLaunchBytes = kBytes + 1024;
+  static constexpr int kTmemCols = 2 * BN;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kProjThreads, 1)
+    proj_sm100_pair_kernel(const __grid_constant__ ProjMaps maps, const __grid_constant__ ProjParams p) {
+  using L = PairSmem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBarOffset;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + L::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto a_tile = [&](int s) { return sbase + s * L::kStageBytes; };
+  auto b_tile = [&](int s) { return sbase + s * L::kStageBytes + L::kABytes; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs and owns the stage barriers
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int num_pairs = static_cast<int>(gridDim.x >> 1);
+
+  const bool cp_rows = p.tma_rows == 0;  // A rows by cp.async (else all by TMA gather4)
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      // CTA 0: thread 0 posts the pair's TMA bytes (+ its 256 cp.async threads + CTA 1's relay);
+      // CTA 1: its 256 cp.async threads (unused in TMA-only mode)
+      const uint32_t arrivals = rank == 0 ? (cp_rows ? 1u + static_cast<uint32_t>(kAThreads) + 1u : 1u)
+                                          : static_cast<uint32_t>(kAThreads);
+      mbar_init(full_bar(s), arrivals);
+      mbar_init(empty_bar(s), 1u);  // one tcgen05.commit from CTA 0's MMA thread
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1u);
+      mbar_init(tempty_bar(a), 128u + 4u);  // CTA 0: its 128 epilogue threads + CTA 1's 4 epilogue warps
+    }
+    mbar_init(drain_bar, 1u);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpB && lane == 0) tma_prefetch_desc(&maps.Whalf);
+  if (warp == kWarpMma) {
+    tmem_alloc_pair(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.num_m_blocks * p.num_n_blocks;  // m blocks of 256 rows
+  const int KB = p.num_k_blocks;
+  const int kb_per_sub = p.d / kBK;
+
+  if (warp < kAWarps) {
+    // ------------------------------------------------------------ A producers (own 128 rows)
+    const int t = threadIdx.x;
+    const int chunk = t & 7, rsub = t >> 3;                         // cp.async mode
+    const uint32_t swz = static_cast<uint32_t>((chunk ^ (rsub & 7)) << 4);
+    const bool issuer = !cp_rows && lane < 4;                       // gather4 mode: 32 lanes x 4 rows
+    const int iss = warp * 4 + lane;
+    const uint32_t pair_tx = cp_rows ? 2u * L::kBBytes : 2u * (L::kABytes + L::kBBytes);
+    const uint64_t pol = l2_policy_evict_normal();
+    // raw row indices (this thread's 4 rows) of the current and the next run
+    int32_t raw[4], nraw[4];
+    auto load_raw = [&](const KRun& r, int32_t (&dst)[4]) {
+      const int64_t row_base = static_cast<int64_t>(r.tile / p.num_n_blocks) * (2 * kBM) + rank * kBM;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t gr = row_base + (cp_rows ? rsub + 32 * j : iss * 4 + j);
+        dst[j] = ((cp_rows || issuer) && gr < p.T) ? ld_idx_early(p.idx + gr * p.S + r.s) : 0;
+      }
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    KRun cur = k_run_at(pair, 0, p.num_n_blocks, KB, kb_per_sub);
+    if (cur.tile < num_tiles) load_raw(cur, raw);
+    KRun nxt = k_run_next(cur, num_pairs, p.num_n_blocks, KB, kb_per_sub);
+    if (nxt.tile < num_tiles) load_raw(nxt, nraw);
+    while (cur.tile < num_tiles && ok) {
+      const uint32_t V = p.Vs[cur.s];
+      const uint16_t* src[4];
+      int32_t r4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t ix = clamp_row(raw[j], V, p.status);
+        src[j] = p.E[cur.s] + static_cast<int64_t>(ix) * p.d + chunk * 8;
+        r4[j] = static_cast<int32_t>(ix);
+      }
+      for (int q = 0; q < cur.len; ++q) {
+        const int c0 = (cur.c_first + q) * kBK;
+        if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        const uint32_t a = a_tile(stage);
+        if (rank == 0 && t == 0) mbar_arrive_expect_tx(full_bar(stage), pair_tx);
+        if (cp_rows) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) cp_async_16(a + (rsub + 32 * j) * 128 + swz, src[j] + c0);
+          cp_async_arrive_noinc(full_bar(stage));
+        } else if (issuer) {
+          tma_gather4_pair(a + iss * 512, &maps.E[cur.s], c0, r4[0], r4[1], r4[2], r4[3],
+                           map_to_cta(full_bar(stage), 0), pol);
+        }
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      cur = nxt;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) raw[j] = nraw[j];
+      nxt = k_run_next(nxt, num_pairs, p.num_n_blocks, KB, kb_per_sub);
+      if (nxt.tile < num_tiles) load_raw(nxt, nraw);
+    }
+    cp_async_wait_all();
+    if (!ok) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 1000ull * 1000ull) __nanosleep(1000);
+    }
+  } else if (warp == kWarpB) {
+    // ------------------------------------------------------------ W producer (own BN/2 rows)
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        const int n_blk = tile % p.num_n_blocks;
+        const int rot = k_rotation(tile / p.num_n_blocks, n_blk, KB);
+        for (int i = 0; i < KB; ++i) {
+          int kb = i + rot;
+          if (kb >= KB) kb -= KB;
+          if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          tma_load_2d_pair(b_tile(stage), &maps.Whalf, kb * kBK, n_blk * BN + static_cast<int>(rank) * (BN / 2),
+                           map_to_cta(full_bar(stage), 0), pol);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer (CTA 0)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(2 * kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!mbar_wait_cluster(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int i = 0; i < KB; ++i) {
+          if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          if (cp_rows) fence_proxy_async_smem();  // this CTA's cp.async rows: generic proxy writes
+          const uint64_t adesc = sw128_kmajor_desc(a_tile(stage));
+          const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
+          umma_commit_pair(map_to_cta(empty_bar(stage), 0));
+          umma_commit_pair(map_to_cta(empty_bar(stage), 1));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) {
+          umma_commit_pair(map_to_cta(tfull_bar(acc), 0));
+          umma_commit_pair(map_to_cta(tfull_bar(acc), 1));
+        }
+      }
+      umma_commit_pair(map_to_cta(drain_bar, 0));
+      mbar_wait_drain(drain_bar, 0, 100ull * 1000 * 1000);
+    }
+  } else if (warp == kWarpRelay) {
+    // ------------------------------------------------------------ relay (CTA 1, cp.async mode)
+    // Lane l handles stages l, l + STAGES, ...: waits for CTA 1's cp.async rows of the stage,
+    // fences them for the async proxy and arrives on CTA 0's stage barrier.
+    if (cp_rows && rank == 1 && lane < STAGES) {
+      const int my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
+      const int total = my_tiles > 0 ? my_tiles * KB : 0;
+      const uint32_t remote = map_to_cta(full_bar(lane), 0);
+      uint32_t phase = 0;
+      for (int k = lane; k < total; k += STAGES) {
+        if (!mbar_wait(full_bar(lane), phase, abort_flag, p.status)) break;
+        fence_proxy_async_smem();
+        mbar_arrive_remote(remote);
+        phase ^= 1u;
+      }
+    }
+  } else if (warp >= kWarpEpi0) {
+    // ------------------------------------------------------------ epilogue (own 128 rows)
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t tempty_remote0 = map_to_cta(tempty_bar(0), 0);
+    const uint32_t tempty_remote1 = map_to_cta(tempty_bar(1), 0);
+    int local = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
+      const int m_blk = tile / p.num_n_blocks;
+      const int n_blk = tile % p.num_n_blocks;
+      const int acc = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const int64_t gr = static_cast<int64_t>(m_blk) * (2 * kBM) + rank * kBM + row_in_tile;
+      const bool valid = gr < p.T;
+      uint32_t t = 0;
+      if (valid) {
+        const int32_t tok = p.tokens[gr];
+        t = (tok >= 0 && static_cast<uint32_t>(tok) < p.V0) ? static_cast<uint32_t>(tok) : 0u;
+      }
+      const uint4* e0 = reinterpret_cast<const uint4*>(p.E0 + static_cast<int64_t>(t) * p.D + n_blk * BN);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + gr * p.D + n_blk * BN);
+      uint4 ecur[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) ecur[v] = valid ? __ldg(e0 + v) : make_uint4(0, 0, 0, 0);
+
+      bool got = false;
+      if (lane == 0) got = mbar_wait_cluster(tfull_bar(acc), use & 1u, abort_flag, p.status);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, v);
+        uint4 enext[4];
+        const bool has_next = c + 1 < BN / 32;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          enext[w] = (valid && has_next) ? __ldg(e0 + (c + 1) * 4 + w) : make_uint4(0, 0, 0, 0);
+        tmem_wait_ld();
+        if (c + 1 == BN / 32) {
+          tc_fence_before();
+          if (rank == 0) {
+            mbar_arrive(tempty_bar(acc));
+          } else {
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acc ? tempty_remote1 : tempty_remote0);
+          }
+        }
+        if (valid) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t ew[4] = {ecur[w].x, ecur[w].y, ecur[w].z, ecur[w].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const int col = w * 8 + h * 2;
+              const float x0 = (__uint_as_float(v[col]) + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale;
+              const float x1 = (__uint_as_float(v[col + 1]) + bf16_bits_to_float(ew[h] >> 16)) * p.scale;
+              o[h] = pack_bf16x2(x0, x1);
+            }
+            dst[c * 4 + w] = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) ecur[w] = enext[w];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no remote arrive or pair MMA is outstanding past this point
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace ngram

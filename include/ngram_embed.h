@@ -216,8 +216,16 @@ int ngram_embed_plan_uses_tensor_cores(const ngram_embed_plan* plan);
 int ngram_embed_plan_set_variant(ngram_embed_plan* plan, int variant);
 
 /* Variant 2: how many of the 128 rows of each gathered tile TMA brings in (0, 32, 64, 96
- * or 128; default 0); cp.async brings in the rest. A tuning knob: results do not change. */
+ * or 128; default 128 for the pair form, 0 for the one-CTA form); cp.async brings in the
+ * rest. A tuning knob: results do not change. */
 int ngram_embed_plan_set_tma_rows(ngram_embed_plan* plan, int rows);
+
+/* Tensor-core kernel form: 1 = pairs of CTAs on neighbouring SMs share each 256-token tile
+ * (tcgen05 cta_group::2; each CTA loads half of the W tile; A rows by cp.async when tma_rows
+ * is 0, else all by TMA gather4), 0 = one CTA per 128-token tile. Default: pairs with TMA rows
+ * when D <= 2048, else one CTA with cp.async rows. A tuning knob: results agree within the
+ * stated tolerance (the k-block order differs). */
+int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on);
 
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */
 int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);

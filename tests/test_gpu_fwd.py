@@ -29,13 +29,15 @@ def dev_i32(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
 
 
-def plan_for(ne, cfg, variant=0, tile_n=None):
+def plan_for(ne, cfg, variant=0, tile_n=None, pair=None):
     plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk,
                                       ne.NGRAM_BF16 if cfg.dtype == "bf16" else ne.NGRAM_F32)
     if variant:
         ne.ngram_embed_plan_set_variant(plan, variant)
     if tile_n:
         ne.ngram_embed_plan_set_tile_n(plan, tile_n)
+    if pair is not None:
+        ne.ngram_embed_plan_set_cta_pair(plan, pair)
     return plan
 
 
@@ -83,11 +85,12 @@ SHAPES = [(5000, 256, 3, 2), (5000, 512, 5, 2), (3000, 1024, 3, 2), (5000, 384, 
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "V0%d_D%d_N%d_K%d" % s)
-@pytest.mark.parametrize("variant,tile_n,tma_rows", [(1, 256, None), (1, 128, None), (2, 256, 64), (2, 128, 64),
-                                                     (2, 256, 0), (2, 128, 32), (2, 256, 96), (3, None, None)],
-                         ids=["tc_tma_n256", "tc_tma_n128", "tc_split64_n256", "tc_split64_n128",
-                              "tc_cpasync_n256", "tc_split32_n128", "tc_split96_n256", "simt"])
-def test_small_shapes_all_kernels(ne, shape, variant, tile_n, tma_rows):
+@pytest.mark.parametrize("variant,tile_n,tma_rows,pair", [
+    (1, 256, None, 0), (1, 128, None, 0), (2, 256, 64, 0), (2, 128, 64, 0), (2, 256, 0, 0), (2, 128, 32, 0),
+    (2, 256, 96, 0), (2, 256, 0, 1), (2, 128, 0, 1), (2, 256, 64, 1), (1, 256, None, 1), (3, None, None, None)],
+    ids=["tc_tma_n256", "tc_tma_n128", "tc_split64_n256", "tc_split64_n128", "tc_cpasync_n256", "tc_split32_n128",
+         "tc_split96_n256", "pair_cpasync_n256", "pair_cpasync_n128", "pair_split64_n256", "pair_tma_n256", "simt"])
+def test_small_shapes_all_kernels(ne, shape, variant, tile_n, tma_rows, pair):
     cfg = small_cfg(*shape)
     if tile_n == 256 and cfg.D % 256:
         pytest.skip("D not a multiple of 256")
@@ -95,7 +98,7 @@ def test_small_shapes_all_kernels(ne, shape, variant, tile_n, tma_rows):
     from tests.helpers import host_tables
     E0h, Eh, Wh = host_tables(cfg)
     E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
-    plan = plan_for(ne, cfg, variant, tile_n)
+    plan = plan_for(ne, cfg, variant, tile_n, pair)
     if tma_rows is not None:
         ne.ngram_embed_plan_set_tma_rows(plan, tma_rows)
     out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
@@ -104,9 +107,10 @@ def test_small_shapes_all_kernels(ne, shape, variant, tile_n, tma_rows):
     assert_close(to_host_f64(out), want, what=f"{cfg.name} variant {variant}")
 
 
-@pytest.mark.parametrize("variant,tma_rows", [(1, None), (2, 0), (2, 32), (2, 64), (2, 96)])
+@pytest.mark.parametrize("variant,tma_rows,pair", [(1, None, 0), (2, 0, 0), (2, 32, 0), (2, 64, 0), (2, 96, 0),
+                                                  (1, None, 1), (2, 0, 1), (2, 64, 1)])
 @pytest.mark.parametrize("D,N,K", [(384, 2, 3), (896, 8, 1)])  # S + 1 = 4 or 8: the scale is exact
-def test_gather_and_layout_bit_exact(ne, variant, tma_rows, D, N, K):
+def test_gather_and_layout_bit_exact(ne, variant, tma_rows, pair, D, N, K):
     """W = I and E_0 = 0: out = concat_s E_s[idx_s] / (S+1) exactly (a product by 1 and a power
     of two), so every gathered element must land in its place bit for bit. Then all E_s = 0:
     out = E_0[t] / (S+1) exactly, which pins the E_0 gather of the epilogue."""
@@ -118,7 +122,7 @@ def test_gather_and_layout_bit_exact(ne, variant, tma_rows, D, N, K):
     eye = gen.f32_to_bf16_bits(np.eye(D, dtype=np.float32))
     idx = oracle.hash_indices(cfg.V0, N, K, cfg.V_nk, oracle.context_windows(N, tokens, offsets))
     G = np.concatenate([gen.bf16_bits_to_f32(Eh[s][idx[:, s]]) for s in range(S)], axis=1)
-    plan = plan_for(ne, cfg, variant)
+    plan = plan_for(ne, cfg, variant, pair=pair)
     if tma_rows is not None:
         ne.ngram_embed_plan_set_tma_rows(plan, tma_rows)
     zeros0 = torch.zeros((cfg.V0, D), dtype=torch.bfloat16, device="cuda")
@@ -204,11 +208,17 @@ def test_full_size_prefill_sampled(ne, cfg):
     want = oracle_rows(cfg, tokens, offsets, rows, host_W(cfg))
     assert_close(to_host_f64(out[torch.from_numpy(rows).cuda()]), want, what=cfg.name)
     # other splits of the A rows between TMA and cp.async feed the MMAs the same tiles
-    for rows in (0, 128):
-        ne.ngram_embed_plan_set_tma_rows(plan, rows)
+    for tr in (64, 128):
+        ne.ngram_embed_plan_set_tma_rows(plan, tr)
         out2, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
-        assert status == 0 and torch.equal(out, out2), rows
-    del E0, E, W, out, out2
+        assert status == 0 and torch.equal(out, out2), tr
+    # the one-CTA kernel form (other tile order and k rotation) agrees with the oracle too
+    ne.ngram_embed_plan_set_tma_rows(plan, 0)
+    ne.ngram_embed_plan_set_cta_pair(plan, 0)
+    out1, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    assert_close(to_host_f64(out1[torch.from_numpy(rows).cuda()]), want, what=cfg.name + " one-CTA")
+    del E0, E, W, out, out2, out1
     gc.collect()
     torch.cuda.empty_cache()
 
