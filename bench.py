@@ -174,6 +174,103 @@ def config_block(cfg, args):
             "l2": "flushed between timed steps (256 MB write)"}
 
 
+# ------------------------------------------------------------------ decode (speculative, ring cache)
+
+def run_decode(ne, cfg, steps: int, warmup: int, dev, seed_offset: int = 0):
+    """Speculative decode: per step, every sequence brings 5 ids (x0 + 4 drafts); the layer
+    reads each sequence's context from the N-gram cache ring, then the accepted prefix
+    (1 + a ids, a ~ U{0..4}) is committed. `steps` steps are captured in one CUDA graph and
+    replayed; the L2 is not flushed between steps (steady state: W stays L2-resident, the
+    27 GB of sub-tables do not)."""
+    import torch
+    from synth.tables import device_tables
+    cfg = cfg.with_(seed=cfg.seed + seed_offset)
+    ds = workloads.DecodeStream(cfg)
+    B, P, C = ds.B, ds.P, cfg.ring_capacity
+    T = B * P
+    E0, E, W = device_tables(cfg)
+    plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
+    ws = ne.new_workspace(plan, T)
+    cache = ne.Cache.empty(B, C, device=dev)
+    ne.ngram_cache_reset(plan, cache, ws)
+    dev_i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+    ids, poff = ds.prompts()
+    for start in range(0, cfg.prompt_max + 1, C):
+        chunk = [ids[poff[b] + start: min(poff[b + 1], poff[b] + start + C)] for b in range(B)]
+        off = gen.offsets_from_lengths([len(c) for c in chunk])
+        flat = np.concatenate(chunk).astype(np.int32) if off[-1] else np.zeros(1, np.int32)
+        ne.ngram_cache_append(plan, cache, dev_i32(flat), dev_i32(off), ws)
+    n_total = warmup + 2 * steps
+    tok_all = dev_i32(np.stack([ds.step_tokens(i) for i in range(n_total)]))
+    cnt_all = dev_i32(np.stack([1 + ds.accept_lengths(i) for i in range(n_total)]))
+    offsets = dev_i32(ds.step_offsets())
+    out = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
+
+    def step(i, stream):
+        ne.ngram_embed_fwd(plan, tok_all[i], offsets, E0, E, W, out, ws, cache=cache, stream=stream)
+        ne.ngram_cache_commit(plan, cache, tok_all[i], P, cnt_all[i], ws, stream=stream)
+
+    cur = torch.cuda.current_stream()
+    for i in range(warmup):
+        step(i, cur)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    graphs = []
+    for rep in range(2):  # two graphs: one warm-up replay, one timed
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(warmup + rep * steps, warmup + (rep + 1) * steps):
+                step(i, s)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    graphs[0].replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        a.record(s)
+        graphs[1].replay()
+        b.record(s)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    status = ne.ngram_embed_get_status(ws)
+    # the projection alone at this shape, and the stand-alone hash + gather stage
+    idx = torch.empty((T, cfg.S), dtype=torch.int32, device=dev)
+    G = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
+    ne.ngram_hash_indices(plan, tok_all[0], offsets, idx, ws, cache=cache)
+
+    def timed(fn, n=50):
+        for _ in range(5):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for e0, e1 in ev:
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return float(np.median([e0.elapsed_time(e1) for e0, e1 in ev]))
+
+    proj_ms = timed(lambda: ne.ngram_embed_project(plan, tok_all[0], idx, E0, E, W, out, ws))
+    hash_ms = timed(lambda: ne.ngram_hash_indices(plan, tok_all[0], offsets, idx, ws, cache=cache))
+    gather_ms = timed(lambda: ne.ngram_embed_gather(plan, idx, E, G, ws))
+    gather_bytes = T * cfg.S * cfg.d * 2 * 2  # sub-rows read + G written
+    pk = peaks()
+    flops = 2.0 * T * cfg.D * cfg.D
+    res = {
+        "workload": cfg.name, "steps": steps, "tokens_per_step": T, "ms_per_step": ms / steps,
+        "value": steps * T / (ms / 1e3), "unit": UNIT, "graph": True, "gpu_launches_per_step": 3,
+        "layer_tflops": flops / (ms / steps / 1e3) / 1e12,
+        "projection": {"ms": proj_ms, "tflops": flops / (proj_ms / 1e3) / 1e12,
+                       "frac": flops / (proj_ms / 1e3) / 1e12 / pk["bf16_tflops"]},
+        "hash_ms": hash_ms,
+        "gather_stage": {"ms": gather_ms, "bytes": gather_bytes, "gbs": gather_bytes / (gather_ms / 1e3) / 1e9,
+                         "frac_hbm": gather_bytes / (gather_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+        "device_status": status,
+    }
+    del graphs, E0, E, W
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------ our arm
 
 def main():
@@ -185,6 +282,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    ap.add_argument("--no-decode", action="store_true", help="skip the speculative-decode measurement")
+    ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--profile-only", action="store_true",
                     help="warm up, run --steps forward calls back to back and exit (for profiler captures)")
     args = ap.parse_args()
@@ -301,6 +400,17 @@ def main():
         e2e_ms = float(t.item())
     status = ne.ngram_embed_get_status(ws)
 
+    del E0, E, W
+    torch.cuda.empty_cache()
+    decode = None
+    if not args.no_decode:
+        decode = run_decode(ne, configs.SPEC_DECODE, args.decode_steps, max(args.warmup, 3), dev, seed_offset=rank)
+        if world > 1:
+            t = torch.tensor([decode["ms_per_step"]], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            decode["ms_per_step"] = float(t.item())
+            decode["value"] = world * decode["tokens_per_step"] / (decode["ms_per_step"] / 1e3)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample_rate(cfg)
@@ -313,7 +423,9 @@ def main():
             "config": config_block(cfg, argparse.Namespace(gpus=world)),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16_tflops"], "traffic": None,
-                         "kernel": "proj_sm100_kernel (gather + tcgen05 projection + epilogue)",
+                         "kernel": ("proj_sm100_pair_kernel (CTA pairs, cta_group::2)" if cfg.D <= 2048 else
+                                    "proj_sm100_kernel (one CTA per tile)") +
+                                   ": fused sub-row gather + tcgen05 projection + E_0 add + scale",
                          "kernel_ms": proj_ms, "peak_source": pk["source"] + " (burst)",
                          "layer_frac": (flops / (ms_per_step / 1e3) / 1e12) / pk["bf16_tflops"],
                          "hash_kernel_ms": hash_ms,
@@ -323,6 +435,7 @@ def main():
                     "h2d_bytes_per_step": tokens.numel() * 4 + offsets.numel() * 4,
                     "d2h_bytes_per_step": out.numel() * 2},
             "gpu_launches": 2 * args.steps,
+            "decode": decode,
             "clocks": clk.summary(),
             "device_status": status,
             "impl": "ours",

@@ -40,6 +40,7 @@ EXPORTED = [
     "ngram_embed_clear_status", "ngram_embed_error_string", "ngram_embed_plan_uses_tensor_cores",
     "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_plan_set_tma_rows",
     "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws", "ngram_embed_plan_set_cta_pair",
+    "ngram_cache_commit",
 ]
 
 
@@ -67,6 +68,7 @@ _sig("ngram_embed_gather", [_P, _P, _I64, _P, _P, _P, _SZ, _P])
 _sig("ngram_cache_reset", [_P, _P, _P, _I32, _P, _SZ, _P])
 _sig("ngram_cache_append", [_P, _P, _P, _P, _P, _I32, _P, _SZ, _P])
 _sig("ngram_cache_rollback", [_P, _P, _P, _P, _I32, _P, _SZ, _P])
+_sig("ngram_cache_commit", [_P, _P, _P, _P, _I32, _P, _I32, _P, _SZ, _P])
 _sig("ngram_embed_get_status", [_P, _P, ctypes.POINTER(_I32)])
 _sig("ngram_embed_clear_status", [_P, _P])
 _sig("ngram_embed_error_string", [ctypes.c_int], ctypes.c_char_p)
@@ -224,6 +226,13 @@ def ngram_cache_append(plan: Plan, cache: Cache, tokens, tok_offsets, workspace,
                                  _i32(tokens, "tokens"), _i32(tok_offsets, "tok_offsets"), tok_offsets.numel() - 1,
                                  _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "ngram_cache_append")
+
+
+def ngram_cache_commit(plan: Plan, cache: Cache, tokens, stride: int, counts, workspace, slots=None, stream=None):
+    rc = _lib.ngram_cache_commit(plan.handle, ctypes.byref(cache.struct), _i32(slots, "slots"),
+                                 _i32(tokens, "tokens"), stride, _i32(counts, "counts"), counts.numel(),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_cache_commit")
 
 
 def ngram_cache_rollback(plan: Plan, cache: Cache, counts, workspace, slots=None, stream=None):

@@ -44,7 +44,10 @@ __device__ __forceinline__ uint32_t horner_step(uint32_t h, uint32_t V0, uint32_
   return static_cast<uint32_t>(r);
 }
 
+constexpr int kHashSmemOffsets = 4096;  // offsets staged in shared memory when B + 1 fits
+
 __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashParams p) {
+  __shared__ int32_t s_off[kHashSmemOffsets];
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
 
   // Offsets check (sticky status; the lookups below stay in bounds regardless).
@@ -54,15 +57,22 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashP
                      (i < p.num_seqs && p.offsets[i + 1] < o);
     if (bad) set_status(p.status, NGRAM_STATUS_BAD_OFFSETS);
   }
+  // Small batches: one coalesced pass brings every offset into shared memory, so the
+  // sequence search below costs no dependent global loads.
+  const bool staged = p.num_seqs + 1 <= kHashSmemOffsets;
+  if (staged) {
+    for (int k = threadIdx.x; k <= p.num_seqs; k += blockDim.x) s_off[k] = p.offsets[k];
+    __syncthreads();
+  }
   if (i >= p.T) return;
 
   // Sequence of token i: the largest b with offsets[b] <= i.
   int32_t lo = 0, hi = p.num_seqs;
   while (hi - lo > 1) {
     const int32_t mid = (lo + hi) >> 1;
-    if (p.offsets[mid] <= i) lo = mid; else hi = mid;
+    if ((staged ? s_off[mid] : p.offsets[mid]) <= i) lo = mid; else hi = mid;
   }
-  const int64_t start = p.offsets[lo];
+  const int64_t start = staged ? s_off[lo] : p.offsets[lo];
 
   int32_t slot = -1;
   int64_t hist_len = 0, hist_from = 0;

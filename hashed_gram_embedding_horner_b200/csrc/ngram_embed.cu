@@ -512,13 +512,14 @@ int ngram_embed_gather(const ngram_embed_plan* plan, const int32_t* idx, int64_t
 
 static int cache_launch(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots,
                         const int32_t* tokens, const int32_t* tok_offsets, const int32_t* counts, int32_t n,
-                        void* workspace, size_t workspace_bytes, void* stream, int which) {
+                        void* workspace, size_t workspace_bytes, void* stream, int which, int32_t stride = 0) {
   int rc = validate_common(plan, workspace, workspace_bytes, 0);
   if (rc) return rc;
   if (!cache || n < 0) return NGRAM_ERR_INVALID_ARG;
   if ((rc = validate_cache(plan, cache))) return rc;
   if (n == 0) return NGRAM_OK;
   if (which == 1 && (!tokens || !tok_offsets)) return NGRAM_ERR_INVALID_ARG;
+  if (which == 3 && (!tokens || !counts || stride < 1)) return NGRAM_ERR_INVALID_ARG;
   if (which == 2 && !counts) return NGRAM_ERR_INVALID_ARG;
   if ((rc = set_device(plan))) return rc;
   CacheParams c{};
@@ -533,12 +534,13 @@ static int cache_launch(const ngram_embed_plan* plan, const ngram_cache* cache, 
   c.tokens = tokens;
   c.tok_offsets = tok_offsets;
   c.counts = counts;
+  c.stride = stride;
   c.n = n;
   c.status = status_ptr(workspace);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (which == 0)
     cache_reset_kernel<<<(n + 255) / 256, 256, 0, st>>>(c);
-  else if (which == 1)
+  else if (which == 1 || which == 3)
     cache_append_kernel<<<(n + 7) / 8, 256, 0, st>>>(c);
   else
     cache_rollback_kernel<<<(n + 255) / 256, 256, 0, st>>>(c);
@@ -554,6 +556,12 @@ int ngram_cache_append(const ngram_embed_plan* plan, const ngram_cache* cache, c
                        const int32_t* tokens, const int32_t* tok_offsets, int32_t n, void* workspace,
                        size_t workspace_bytes, void* stream) {
   return cache_launch(plan, cache, slots, tokens, tok_offsets, nullptr, n, workspace, workspace_bytes, stream, 1);
+}
+
+int ngram_cache_commit(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots,
+                       const int32_t* tokens, int32_t stride, const int32_t* counts, int32_t n, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return cache_launch(plan, cache, slots, tokens, nullptr, counts, n, workspace, workspace_bytes, stream, 3, stride);
 }
 
 int ngram_cache_rollback(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots,

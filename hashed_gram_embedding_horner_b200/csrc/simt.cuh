@@ -150,7 +150,8 @@ struct CacheParams {
   const int32_t* slots;       // nullptr: entry i -> slot i
   const int32_t* tokens;      // append
   const int32_t* tok_offsets; // append
-  const int32_t* counts;      // rollback
+  const int32_t* counts;      // rollback; commit (ids per entry)
+  int32_t stride;             // commit: entry i's ids start at tokens[i * stride]
   int32_t n;
   int* status;
 };
@@ -183,9 +184,10 @@ __global__ void cache_append_kernel(const __grid_constant__ CacheParams p) {
   if (lane == 0) s = entry_slot(p, i);
   s = __shfl_sync(0xffffffffu, s, 0);
   if (s < 0) return;
-  const int32_t b = p.tok_offsets[i], e = p.tok_offsets[i + 1];
-  const int32_t m = e - b;
-  if (b < 0 || m < 0 || m > p.capacity) {
+  // CSR entries (tok_offsets) or fixed-stride entries with counts (commit of accepted ids)
+  const int32_t b = p.tok_offsets ? p.tok_offsets[i] : i * p.stride;
+  const int32_t m = p.tok_offsets ? p.tok_offsets[i + 1] - b : p.counts[i];
+  if (b < 0 || m < 0 || m > p.capacity || (!p.tok_offsets && m > p.stride)) {
     if (lane == 0) set_status(p.status, (b < 0 || m < 0) ? NGRAM_STATUS_BAD_OFFSETS : NGRAM_STATUS_BAD_APPEND);
     return;
   }

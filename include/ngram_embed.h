@@ -165,6 +165,15 @@ int ngram_cache_append(const ngram_embed_plan* plan, const ngram_cache* cache,
                        const int32_t* slots, const int32_t* tokens, const int32_t* tok_offsets,
                        int32_t n, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Commit the accepted prefix of a speculative step in one launch: entry i appends
+ * tokens[i*stride .. i*stride + counts[i]) (device int32; 0 <= counts[i] <= min(stride,
+ * capacity)) to slot slots[i]. Equivalent to ngram_cache_append of all `stride` ids followed
+ * by ngram_cache_rollback of stride - counts[i]. */
+int ngram_cache_commit(const ngram_embed_plan* plan, const ngram_cache* cache,
+                       const int32_t* slots, const int32_t* tokens, int32_t stride,
+                       const int32_t* counts, int32_t n, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
 /* Un-commit ids: entry i drops the newest counts[i] ids (device int32) of slot slots[i].
  * Rejected (status bit, slot unchanged) if counts[i] < 0, counts[i] > len, or the newest
  * N-1 remaining positions are no longer all held by the ring. */

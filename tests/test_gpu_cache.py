@@ -97,6 +97,39 @@ def test_commit_paths_agree_on_device(ne):
             assert r1[b, pos % C] == r2[b, pos % C]
 
 
+def test_commit_equals_append_then_rollback(ne):
+    """ngram_cache_commit(counts) leaves the same committed history as append(all P ids) +
+    rollback(P - counts), each matching the history model, and rejects counts above the
+    stride or the capacity."""
+    N, C, B, P = 3, 8, 6, 5
+    plan = ne.ngram_embed_plan_create(1000, 64, N, 2, [4099, 5003, 6007, 7001], ne.NGRAM_BF16)
+    ws = ne.new_workspace(plan, 64)
+    c1, c2 = ne.Cache.empty(B, C), ne.Cache.empty(B, C)
+    ref1, ref2 = oracle.RingOracle(B, C, N), oracle.RingOracle(B, C, N)
+    rng = np.random.default_rng(9)
+    for rnd in range(5):
+        step = rng.integers(0, 1000, B * P).astype(np.int32)
+        a = rng.integers(0, P, B).astype(np.int32)
+        ne.ngram_cache_commit(plan, c1, dev_i32(step), P, dev_i32(1 + a), ws)
+        ne.ngram_cache_append(plan, c2, dev_i32(step), dev_i32(np.arange(B + 1) * P), ws)
+        ne.ngram_cache_rollback(plan, c2, dev_i32(P - 1 - a), ws)
+        assert ne.ngram_embed_get_status(ws) == 0
+        for b in range(B):
+            assert ref1.append(b, step[b * P:b * P + 1 + a[b]])
+            assert ref2.append(b, step[b * P:(b + 1) * P]) and ref2.rollback(b, int(P - 1 - a[b]))
+        check_ring(ne, c1, ref1)
+        check_ring(ne, c2, ref2)
+        # same committed history; committing only the accepted ids evicts no more than append + rollback
+        assert torch.equal(c1.len, c2.len) and bool((c1.valid_from <= c2.valid_from).all())
+        ln = c1.len.cpu().numpy()
+        r1, r2 = c1.ring.cpu().numpy(), c2.ring.cpu().numpy()
+        for b in range(B):
+            for pos in range(int(ln[b]) - (N - 1), int(ln[b])):
+                assert r1[b, pos % C] == r2[b, pos % C]
+    ne.ngram_cache_commit(plan, c1, dev_i32(np.zeros(B * P)), P, dev_i32([P + 1] * B), ws)
+    assert ne.status_names(ne.ngram_embed_get_status(ws)) == ["BAD_APPEND"]
+
+
 def test_decode_hashes_through_ring(ne):
     """Spec-decode workload: per step, hashes of the 5 in-step ids read the ring's
     committed history; equal (bit-exact) to the oracle over the full history."""
