@@ -284,6 +284,8 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-decode", action="store_true", help="skip the speculative-decode measurement")
     ap.add_argument("--decode-steps", type=int, default=100)
+    ap.add_argument("--decode-only", action="store_true",
+                    help="only the speculative-decode measurement (one JSON line with the decode object)")
     ap.add_argument("--profile-only", action="store_true",
                     help="warm up, run --steps forward calls back to back and exit (for profiler captures)")
     args = ap.parse_args()
@@ -305,6 +307,14 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
+    if args.decode_only:
+        decode = run_decode(ne, configs.SPEC_DECODE, args.decode_steps, max(args.warmup, 3), dev, seed_offset=rank)
+        if rank == 0:
+            print(json.dumps({"decode_only": True, "decode": decode}), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     # each rank: its own batch of the same shape (seeded per rank), tables identical
     tokens_h, offsets_h = workloads.prefill_tokens(cfg.with_(seed=cfg.seed) if rank == 0 else cfg.with_(seed=rank))

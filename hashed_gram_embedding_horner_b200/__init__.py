@@ -40,7 +40,7 @@ EXPORTED = [
     "ngram_embed_clear_status", "ngram_embed_error_string", "ngram_embed_plan_uses_tensor_cores",
     "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_plan_set_tma_rows",
     "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws", "ngram_embed_plan_set_cta_pair",
-    "ngram_cache_commit",
+    "ngram_cache_commit", "ngram_embed_plan_set_stream_k",
 ]
 
 
@@ -77,6 +77,7 @@ _sig("ngram_embed_plan_set_variant", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tile_n", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
 _sig("ngram_embed_fwd_static_ws", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P])
 
@@ -118,8 +119,9 @@ class Plan:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
-            _lib.ngram_embed_plan_destroy(h)
+        lib = _lib  # None once the module is torn down at interpreter exit
+        if h and lib is not None:
+            lib.ngram_embed_plan_destroy(h)
             self.handle = None
 
 
@@ -163,6 +165,11 @@ def ngram_embed_plan_set_tma_rows(plan: Plan, rows: int):
 
 def ngram_embed_plan_set_cta_pair(plan: Plan, on: bool):
     _check(_lib.ngram_embed_plan_set_cta_pair(plan.handle, int(bool(on))), "ngram_embed_plan_set_cta_pair")
+
+
+def ngram_embed_plan_set_stream_k(plan: Plan, mode: int):
+    """0 automatic, 1 stream-K whenever the workspace and shape allow it, 2 never."""
+    _check(_lib.ngram_embed_plan_set_stream_k(plan.handle, int(mode)), "ngram_embed_plan_set_stream_k")
 
 
 def ngram_embed_plan_uses_tensor_cores(plan: Plan) -> bool:

@@ -26,7 +26,11 @@ using namespace ngram;
 
 namespace {
 
-constexpr size_t kStatusBytes = 256;  // status word + padding; the index buffer follows
+// Workspace: [status word + padding | stream-K arrival counters | T x S indices | stream-K partials]
+constexpr size_t kStatusBytes = 256;
+constexpr int kSkMaxTiles = 2048;                          // stream-K only for grids of at most this many tiles
+constexpr size_t kSkCounterBytes = size_t(kSkMaxTiles) * 4 * sizeof(int32_t);  // one per (tile, row quarter)
+constexpr size_t kHeadBytes = kStatusBytes + kSkCounterBytes;                   // zeroed by clear_status
 constexpr int kStages = 4;       // one-CTA kernel: 4 x (16 KB A + 32 KB W) at N = 256
 constexpr int kPairStages = 6;   // CTA-pair kernel: 6 x (16 KB A + 16 KB W) per CTA at N = 256
 
@@ -55,6 +59,7 @@ struct ngram_embed_plan {
   bool maps_valid = false;
   bool smem_attr_set[4] = {};  // per (kernel form, tile width) instance, on `device`
   bool cta_pair = true;        // use the CTA-pair (cta_group::2) kernel
+  int stream_k = 0;            // one-CTA kernel schedule: 0 automatic, 1 stream-K when possible, 2 never
   int max_clusters[2] = {0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
 };
 
@@ -77,12 +82,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int32_t* status_ptr(void* ws) { return static_cast<int32_t*>(ws); }
-int32_t* idx_ptr(void* ws) { return reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kStatusBytes); }
+int32_t* idx_ptr(void* ws) { return reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kHeadBytes); }
 
-size_t ws_bytes(const ngram_embed_plan* p, int64_t T) {
+// Bytes every call needs: the head and the index buffer.
+size_t ws_base(const ngram_embed_plan* p, int64_t T) {
   const size_t idx = static_cast<size_t>(T) * static_cast<size_t>(p->S) * sizeof(int32_t);
-  return kStatusBytes + ((idx + 255) & ~size_t(255));
+  return kHeadBytes + ((idx + 255) & ~size_t(255));
 }
+// Stream-K fp32 partial tiles: two 128 x 256 slots per SM.
+size_t sk_partial_bytes(const ngram_embed_plan* p) {
+  return p->tc_ok ? size_t(2) * static_cast<size_t>(p->sms) * kBM * 256 * sizeof(float) : 0;
+}
+// Bytes that let every call of up to T tokens take its fastest schedule.
+size_t ws_bytes(const ngram_embed_plan* p, int64_t T) { return ws_base(p, T) + sk_partial_bytes(p); }
 
 int check_launch() { return cudaGetLastError() == cudaSuccess ? NGRAM_OK : NGRAM_ERR_CUDA; }
 
@@ -122,6 +134,18 @@ int refresh_maps(ngram_embed_plan* p, const void* const* E_nk, const void* W) {
   return NGRAM_OK;
 }
 
+// Stream-K (every CTA takes an equal share of the (tile, k-block) units) instead of one
+// tile per CTA per wave: when the last wave of tiles would leave many SMs idle.
+bool use_stream_k(const ngram_embed_plan* p, const ProjParams& prm, int64_t T, size_t ws_size) {
+  const int tiles = prm.num_m_blocks * prm.num_n_blocks;
+  const int64_t units = static_cast<int64_t>(tiles) * prm.num_k_blocks;
+  if (p->stream_k == 2 || p->sms <= 0 || tiles > kSkMaxTiles || units < p->sms) return false;
+  if (ws_size < ws_bytes(p, T)) return false;
+  if (p->stream_k == 1) return true;
+  const int waves = (tiles + p->sms - 1) / p->sms;
+  return static_cast<double>(tiles) < 0.9 * waves * p->sms;  // data-parallel fill below 90%
+}
+
 template <int BN>
 int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
   using L = ProjSmem<BN, kStages>;
@@ -133,7 +157,7 @@ int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
     p->smem_attr_set[key] = true;
   }
   const int tiles = prm.num_m_blocks * prm.num_n_blocks;
-  const int grid = tiles < p->sms ? tiles : p->sms;
+  const int grid = (prm.stream_k || tiles > p->sms) ? p->sms : tiles;
   kern<<<grid, kProjThreads, L::kLaunchBytes, st>>>(p->maps, prm);
   return check_launch();
 }
@@ -180,7 +204,7 @@ int launch_tc_pair(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t 
 int validate_common(const ngram_embed_plan* p, void* ws, size_t ws_size, int64_t T) {
   if (!p || !ws || T < 0 || T > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
   if (!aligned16(ws)) return NGRAM_ERR_MISALIGNED;
-  if (ws_size < ws_bytes(p, T)) return NGRAM_ERR_WORKSPACE;
+  if (ws_size < ws_base(p, T)) return NGRAM_ERR_WORKSPACE;
   return NGRAM_OK;
 }
 
@@ -265,8 +289,11 @@ int launch_simt(const ngram_embed_plan* p, const int32_t* tokens, const int32_t*
   return check_launch();
 }
 
+// ws_T: the token count the workspace was validated for (its index buffer's length);
+// the stream-K partials, if the workspace holds them, follow that buffer.
 int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int64_t T, const void* E0,
-            const void* const* E_nk, const void* W, void* out, void* ws, cudaStream_t st) {
+            const void* const* E_nk, const void* W, void* out, void* ws, size_t ws_size, int64_t ws_T,
+            cudaStream_t st) {
   if (p->variant == kSimt) {
     return p->dtype == NGRAM_F32
                ? launch_simt<float>(p, tokens, idx, T, E0, E_nk, W, out, ws, st)
@@ -294,6 +321,11 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   prm.scale = 1.0f / static_cast<float>(p->S + 1);
   prm.status = status_ptr(ws);
   prm.tma_rows = p->variant == kTcTmaRows ? kBM : p->tma_rows;
+  if (!p->cta_pair && use_stream_k(p, prm, ws_T, ws_size)) {
+    prm.stream_k = 1;
+    prm.sk_counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+    prm.sk_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_base(p, ws_T));
+  }
   if (p->cta_pair)
     return p->bn == 256 ? launch_tc_pair<256>(p, prm, T, st) : launch_tc_pair<128>(p, prm, T, st);
   return p->bn == 256 ? launch_tc<256>(p, prm, st) : launch_tc<128>(p, prm, st);
@@ -419,6 +451,12 @@ int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int bn) {
   return NGRAM_OK;
 }
 
+int ngram_embed_plan_set_stream_k(ngram_embed_plan* plan, int mode) {
+  if (!plan || mode < 0 || mode > 2) return NGRAM_ERR_INVALID_ARG;
+  plan->stream_k = mode;
+  return NGRAM_OK;
+}
+
 size_t ngram_embed_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens) {
   if (!plan || max_tokens < 0) return 0;
   return ws_bytes(plan, max_tokens);
@@ -452,7 +490,7 @@ int ngram_embed_project(const ngram_embed_plan* plan_c, const int32_t* tokens, c
   if (!aligned16(out)) return NGRAM_ERR_MISALIGNED;
   if ((rc = check_tables(plan, E0, E_nk, W_stacked))) return rc;
   if ((rc = set_device(plan))) return rc;
-  return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace,
+  return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace, workspace_bytes, 0,
                  static_cast<cudaStream_t>(stream));
 }
 
@@ -476,7 +514,8 @@ int ngram_embed_fwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     rc = launch_hash(plan, tokens, seq_offsets, num_seqs, num_tokens, cache, cache_slots, idx, workspace, st);
     if (rc) return rc;
   }
-  return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace, st);
+  return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace, workspace_bytes, num_tokens,
+                 st);
 }
 
 int ngram_embed_gather(const ngram_embed_plan* plan, const int32_t* idx, int64_t num_tokens,
@@ -589,7 +628,7 @@ int ngram_embed_get_status(const void* workspace, void* stream, int32_t* status_
 
 int ngram_embed_clear_status(void* workspace, void* stream) {
   if (!workspace) return NGRAM_ERR_INVALID_ARG;
-  return cudaMemsetAsync(workspace, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) == cudaSuccess
+  return cudaMemsetAsync(workspace, 0, kHeadBytes, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? NGRAM_OK
              : NGRAM_ERR_CUDA;
 }
@@ -642,7 +681,7 @@ extern "C" int ngram_embed_fwd_static_ws(const ngram_embed_plan* plan, const int
                                          const ngram_cache* cache, const int32_t* cache_slots, void* out,
                                          int32_t* status_out, void* stream) {
   if (!plan || num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
-  if (ws_bytes(plan, num_tokens) > kNoAllocScratchBytes) return NGRAM_ERR_WORKSPACE;  // above the fixed limit
+  if (ws_base(plan, num_tokens) > kNoAllocScratchBytes) return NGRAM_ERR_WORKSPACE;  // above the fixed limit
   int rc = set_device(plan);
   if (rc) return rc;
   void* ws = noalloc_scratch(plan->device);

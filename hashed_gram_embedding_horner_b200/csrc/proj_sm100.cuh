@@ -61,6 +61,11 @@ struct ProjParams {
   int tma_rows;           // rows of each A tile gathered by TMA (multiple of 32, 0..128)
   float scale;
   int* status;
+  // stream-K (one-CTA kernel): per-tile arrival counters (zero between launches) and
+  // two fp32 partial slots of 128 x BN per CTA
+  int stream_k;
+  int* sk_counters;
+  float* sk_partials;
 };
 
 struct ProjMaps {
@@ -124,6 +129,99 @@ __device__ __forceinline__ KRun k_run_next(const KRun& r, int stride, int num_n_
     tile += stride;
   }
   return k_run_at(tile, i, num_n_blocks, KB, kb_per_sub);
+}
+
+// ---- work lists of the one-CTA kernel --------------------------------------------------
+// Data-parallel: CTA c takes whole tiles c, c + grid, ... Stream-K: the tiles' k-positions
+// form U = tiles * KB units in tile-major order and CTA c takes units [c*U/grid,
+// (c+1)*U/grid); a tile whose units straddle CTAs is computed in pieces ("segments")
+// whose fp32 partial sums are added by the last piece to finish.
+struct WorkPlan {
+  int num_tiles, KB, grid;
+  int sk;          // 1: stream-K
+  int64_t u_end;   // stream-K: end of this CTA's units
+};
+
+struct Seg {
+  int tile;        // >= num_tiles: past the end
+  int i0, i1;      // positions [i0, i1) of the tile's rotated k-block sequence
+  int64_t u_next;  // stream-K: first unit after this segment
+};
+
+__device__ __forceinline__ int64_t sk_first_unit(int64_t U, int grid, int cta) { return (int64_t(cta) * U) / grid; }
+// The CTA whose units contain unit u.
+__device__ __forceinline__ int sk_cta_of(int64_t u, int64_t U, int grid) {
+  return static_cast<int>(((u + 1) * grid + U - 1) / U) - 1;
+}
+
+__device__ __forceinline__ Seg seg_at_unit(const WorkPlan& w, int64_t u) {
+  Seg g;
+  if (u >= w.u_end) {
+    g.tile = w.num_tiles;
+    g.i0 = g.i1 = 0;
+    g.u_next = u;
+    return g;
+  }
+  g.tile = static_cast<int>(u / w.KB);
+  g.i0 = static_cast<int>(u - static_cast<int64_t>(g.tile) * w.KB);
+  const int64_t left = w.u_end - u;
+  g.i1 = left < w.KB - g.i0 ? g.i0 + static_cast<int>(left) : w.KB;
+  g.u_next = u + (g.i1 - g.i0);
+  return g;
+}
+
+__device__ __forceinline__ Seg seg_first(const WorkPlan& w, int cta) {
+  if (w.sk) return seg_at_unit(w, sk_first_unit(static_cast<int64_t>(w.num_tiles) * w.KB, w.grid, cta));
+  Seg g;
+  g.tile = cta;
+  g.i0 = 0;
+  g.i1 = w.KB;
+  g.u_next = 0;
+  return g;
+}
+
+__device__ __forceinline__ Seg seg_next(const WorkPlan& w, const Seg& g) {
+  if (w.sk) return seg_at_unit(w, g.u_next);
+  Seg n;
+  n.tile = g.tile + w.grid;
+  n.i0 = 0;
+  n.i1 = w.KB;
+  n.u_next = 0;
+  return n;
+}
+
+// A run of k-positions of one segment that use one sub-table.
+struct SRun {
+  Seg g;
+  int i, s, c_first, len;
+};
+
+__device__ __forceinline__ SRun srun_at(const Seg& g, int i, int num_n_blocks, int KB, int kb_per_sub) {
+  SRun r;
+  r.g = g;
+  r.i = i;
+  int kb = i + k_rotation(g.tile / num_n_blocks, g.tile % num_n_blocks, KB);
+  if (kb >= KB) kb -= KB;
+  r.s = kb / kb_per_sub;
+  r.c_first = kb - r.s * kb_per_sub;
+  const int rem = kb_per_sub - r.c_first;
+  r.len = rem < g.i1 - i ? rem : g.i1 - i;
+  return r;
+}
+
+__device__ __forceinline__ SRun srun_next(const WorkPlan& w, const SRun& r, int num_n_blocks, int kb_per_sub) {
+  const int i = r.i + r.len;
+  if (i >= r.g.i1) {
+    const Seg g = seg_next(w, r.g);
+    return srun_at(g, g.i0, num_n_blocks, w.KB, kb_per_sub);
+  }
+  return srun_at(r.g, i, num_n_blocks, w.KB, kb_per_sub);
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // A load issued where it stands in the program (volatile asm keeps its place among the
@@ -192,6 +290,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   const int num_tiles = p.num_m_blocks * p.num_n_blocks;
   const int KB = p.num_k_blocks;
   const int kb_per_sub = p.d / kBK;
+  WorkPlan wp;
+  wp.num_tiles = num_tiles;
+  wp.KB = KB;
+  wp.grid = static_cast<int>(gridDim.x);
+  wp.sk = p.stream_k;
+  wp.u_end = p.stream_k ? sk_first_unit(static_cast<int64_t>(num_tiles) * KB, wp.grid, blockIdx.x + 1) : 0;
 
   if (warp < kAWarps) {
     // ------------------------------------------------------------ A producers
@@ -206,11 +310,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     const int issuer = warp * lanes_tma + lane;  // rows 4*issuer .. +3
     const uint32_t tma_bytes = static_cast<uint32_t>(p.tma_rows) * 128u;
     const uint64_t pol = l2_policy_evict_normal();
-    const int stride = static_cast<int>(gridDim.x);
     // raw row indices of the current and the next run: cp.async rows, then TMA rows
     int32_t raw[8], nraw[8];
-    auto load_raw = [&](const KRun& r, int32_t (&dst)[8]) {
-      const int64_t row_base = static_cast<int64_t>(r.tile / p.num_n_blocks) * kBM;
+    auto load_raw = [&](const SRun& r, int32_t (&dst)[8]) {
+      const int64_t row_base = static_cast<int64_t>(r.g.tile / p.num_n_blocks) * kBM;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t g1 = row_base + p.tma_rows + rsub + 32 * j;
@@ -222,11 +325,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    KRun cur = k_run_at(blockIdx.x, 0, p.num_n_blocks, KB, kb_per_sub);
-    if (cur.tile < num_tiles) load_raw(cur, raw);
-    KRun nxt = k_run_next(cur, stride, p.num_n_blocks, KB, kb_per_sub);
-    if (nxt.tile < num_tiles) load_raw(nxt, nraw);
-    while (cur.tile < num_tiles && ok) {
+    const Seg g0 = seg_first(wp, blockIdx.x);
+    SRun cur = srun_at(g0, g0.i0, p.num_n_blocks, KB, kb_per_sub);
+    if (cur.g.tile < num_tiles) load_raw(cur, raw);
+    SRun nxt = srun_next(wp, cur, p.num_n_blocks, kb_per_sub);
+    if (nxt.g.tile < num_tiles) load_raw(nxt, nraw);
+    while (cur.g.tile < num_tiles && ok) {
       const uint32_t V = p.Vs[cur.s];
       const uint16_t* src[4];
       int32_t r4[4];
@@ -251,8 +355,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       cur = nxt;
 #pragma unroll
       for (int j = 0; j < 8; ++j) raw[j] = nraw[j];
-      nxt = k_run_next(nxt, stride, p.num_n_blocks, KB, kb_per_sub);
-      if (nxt.tile < num_tiles) load_raw(nxt, nraw);
+      nxt = srun_next(wp, nxt, p.num_n_blocks, kb_per_sub);
+      if (nxt.g.tile < num_tiles) load_raw(nxt, nraw);
     }
     cp_async_wait_all();
     if (!ok) {
@@ -267,10 +371,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int n_blk = tile % p.num_n_blocks;
-        const int rot = k_rotation(tile / p.num_n_blocks, n_blk, KB);
-        for (int i = 0; i < KB; ++i) {
+      for (Seg g = seg_first(wp, blockIdx.x); g.tile < num_tiles && ok; g = seg_next(wp, g)) {
+        const int n_blk = g.tile % p.num_n_blocks;
+        const int rot = k_rotation(g.tile / p.num_n_blocks, n_blk, KB);
+        for (int i = g.i0; i < g.i1; ++i) {
           int kb = i + rot;
           if (kb >= KB) kb -= KB;
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
@@ -288,13 +392,13 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int local = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+      for (Seg g = seg_first(wp, blockIdx.x); g.tile < num_tiles && ok; g = seg_next(wp, g), ++local) {
         const int acc = local & 1;
         const uint32_t use = static_cast<uint32_t>(local >> 1);
         if (!mbar_wait(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int i = 0; i < KB; ++i) {
+        for (int i = g.i0; i < g.i1; ++i) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           fence_proxy_async_smem();  // the stage's cp.async rows were written by the generic proxy
@@ -302,7 +406,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage));
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)  // K = 16 per instruction: +32 B = +2 in the address field
-            umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (i > g.i0 || k != 0) ? 1u : 0u);
           umma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -316,12 +420,15 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int row_in_tile = q * 32 + lane;  // == TMEM lane
+    const int64_t U = static_cast<int64_t>(num_tiles) * KB;
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+    for (Seg g = seg_first(wp, blockIdx.x); g.tile < num_tiles; g = seg_next(wp, g), ++local) {
+      const int tile = g.tile;
       const int m_blk = tile / p.num_n_blocks;
       const int n_blk = tile % p.num_n_blocks;
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const bool whole = g.i0 == 0 && g.i1 == KB;
       const int64_t gr = static_cast<int64_t>(m_blk) * kBM + row_in_tile;
       const bool valid = gr < p.T;
       uint32_t t = 0;
@@ -334,44 +441,135 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       // E_0 slice of chunk 0 before waiting on the accumulator.
       uint4 ecur[4];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) ecur[v] = valid ? __ldg(e0 + v) : make_uint4(0, 0, 0, 0);
+      for (int v = 0; v < 4; ++v) ecur[v] = (valid && whole) ? __ldg(e0 + v) : make_uint4(0, 0, 0, 0);
 
       bool got = false;
       if (lane == 0) got = mbar_wait(tfull_bar(acc), use & 1u, abort_flag, p.status);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;  // warp-uniform: tcgen05.ld is .aligned
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      if (whole) {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, v);
-        uint4 enext[4];
-        const bool has_next = c + 1 < BN / 32;
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v);
+          uint4 enext[4];
+          const bool has_next = c + 1 < BN / 32;
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
-          enext[w] = (valid && has_next) ? __ldg(e0 + (c + 1) * 4 + w) : make_uint4(0, 0, 0, 0);
-        tmem_wait_ld();
-        if (c + 1 == BN / 32) {
-          tc_fence_before();
-          mbar_arrive(tempty_bar(acc));  // accumulator fully read: MMA may reuse it
-        }
-        if (valid) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const uint32_t ew[4] = {ecur[w].x, ecur[w].y, ecur[w].z, ecur[w].w};
-            uint32_t o[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const int col = w * 8 + h * 2;
-              const float x0 = (__uint_as_float(v[col]) + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale;
-              const float x1 = (__uint_as_float(v[col + 1]) + bf16_bits_to_float(ew[h] >> 16)) * p.scale;
-              o[h] = pack_bf16x2(x0, x1);
-            }
-            dst[c * 4 + w] = make_uint4(o[0], o[1], o[2], o[3]);
+          for (int w = 0; w < 4; ++w)
+            enext[w] = (valid && has_next) ? __ldg(e0 + (c + 1) * 4 + w) : make_uint4(0, 0, 0, 0);
+          tmem_wait_ld();
+          if (c + 1 == BN / 32) {
+            tc_fence_before();
+            mbar_arrive(tempty_bar(acc));  // accumulator fully read: MMA may reuse it
           }
-        }
+          if (valid) {
 #pragma unroll
-        for (int w = 0; w < 4; ++w) ecur[w] = enext[w];
+            for (int w = 0; w < 4; ++w) {
+              const uint32_t ew[4] = {ecur[w].x, ecur[w].y, ecur[w].z, ecur[w].w};
+              uint32_t o[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const int col = w * 8 + h * 2;
+                const float x0 = (__uint_as_float(v[col]) + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale;
+                const float x1 = (__uint_as_float(v[col + 1]) + bf16_bits_to_float(ew[h] >> 16)) * p.scale;
+                o[h] = pack_bf16x2(x0, x1);
+              }
+              dst[c * 4 + w] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+#pragma unroll
+          for (int w = 0; w < 4; ++w) ecur[w] = enext[w];
+        }
+      } else {
+        // Stream-K piece of a tile. Per (tile, row quarter) an arrival counter counts the
+        // pieces published so far. The warp whose piece completes the tile sums it: its own
+        // piece straight from TMEM, every other piece from its owner's partial slot, then
+        // E_0 and the scale. A warp that finds all other pieces already counted skips
+        // publishing its own. Nobody waits for anybody.
+        const int64_t u_tile = static_cast<int64_t>(tile) * KB;
+        const int c_lo = sk_cta_of(u_tile, U, wp.grid), c_hi = sk_cta_of(u_tile + KB - 1, U, wp.grid);
+        const int others = c_hi - c_lo;  // pieces of the tile besides this one
+        int* cnt = p.sk_counters + tile * 4 + q;
+        int fin = 0;
+        if (lane == 0) fin = ld_acquire_gpu(cnt) == others;
+        fin = __shfl_sync(0xffffffffu, fin, 0);
+        if (!fin) {
+          // slot 0: the piece that starts this CTA's unit range; slot 1: the one that ends it
+          const int slot = (u_tile + g.i0 == sk_first_unit(U, wp.grid, blockIdx.x)) ? 0 : 1;
+          float4* mine = reinterpret_cast<float4*>(p.sk_partials) +
+                         (static_cast<size_t>(blockIdx.x) * 2 + slot) * (kBM * BN / 4) + row_in_tile;
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int w = 0; w < 8; ++w)  // column group major: a warp's store is 512 contiguous bytes
+              mine[(c * 8 + w) * kBM] = make_float4(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1]),
+                                                    __uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3]));
+          }
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) fin = atomicAdd(cnt, 1) == others;
+          fin = __shfl_sync(0xffffffffu, fin, 0);
+          if (fin) __threadfence();
+        }
+        if (fin) {
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint4 e[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) e[w] = valid ? __ldg(e0 + c * 4 + w) : make_uint4(0, 0, 0, 0);
+            // Pieces are added in CTA order whoever finishes, so the bits do not depend on
+            // arrival order: the pieces before this CTA's, its own (TMEM), those after.
+            float sum[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) sum[k] = 0.f;
+            auto add_piece = [&](int cc) {
+              const int sl = (sk_first_unit(U, wp.grid, cc) >= u_tile) ? 0 : 1;
+              const float4* part = reinterpret_cast<const float4*>(p.sk_partials) +
+                                   (static_cast<size_t>(cc) * 2 + sl) * (kBM * BN / 4) + row_in_tile;
+              float4 x[8];
+#pragma unroll
+              for (int w = 0; w < 8; ++w) x[w] = __ldcg(part + (c * 8 + w) * kBM);
+#pragma unroll
+              for (int w = 0; w < 8; ++w) {
+                sum[4 * w] += x[w].x;
+                sum[4 * w + 1] += x[w].y;
+                sum[4 * w + 2] += x[w].z;
+                sum[4 * w + 3] += x[w].w;
+              }
+            };
+            const int self = static_cast<int>(blockIdx.x);
+            for (int cc = c_lo; cc < self; ++cc) add_piece(cc);
+            {
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(taddr + c * 32, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) sum[k] += __uint_as_float(v[k]);
+            }
+            for (int cc = self + 1; cc <= c_hi; ++cc) add_piece(cc);
+            if (valid) {
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                const uint32_t ew[4] = {e[w].x, e[w].y, e[w].z, e[w].w};
+                uint32_t o[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  const int col = w * 8 + h * 2;
+                  o[h] = pack_bf16x2((sum[col] + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale,
+                                     (sum[col + 1] + bf16_bits_to_float(ew[h] >> 16)) * p.scale);
+                }
+                dst[c * 4 + w] = make_uint4(o[0], o[1], o[2], o[3]);
+              }
+            }
+          }
+          if (lane == 0) *cnt = 0;  // the tile is done: zero again for the next launch
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(acc));  // accumulator read for the last time: MMA may reuse it
       }
     }
   }

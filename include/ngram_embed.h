@@ -107,9 +107,14 @@ typedef struct {
 int ngram_embed_plan_create(const ngram_embed_config* cfg, ngram_embed_plan** out);
 int ngram_embed_plan_destroy(ngram_embed_plan* plan);
 
-/* Device workspace bytes needed for calls of up to max_tokens tokens (status word plus
- * the [max_tokens x S] int32 index buffer). Must be zeroed once before first use
- * (ngram_embed_clear_status does that for the status word; the rest needs no init). */
+/* Device workspace bytes for calls of up to max_tokens tokens: a 33,024-byte head (the
+ * status word, then the stream-K arrival counters), the [max_tokens x S] int32 index
+ * buffer, then, for plans that use the tensor-core kernel, 2 x (SM count) x 128 x 256 fp32
+ * stream-K partial tiles. A workspace without the partials (head + index buffer, rounded
+ * up to 256 bytes) is accepted too; the projection then never uses the stream-K schedule.
+ * The head must be zeroed once before first use (ngram_embed_clear_status does it); the
+ * rest needs no init. The kernels leave the counters zero after every call that did not
+ * set NGRAM_STATUS_TIMEOUT. */
 size_t ngram_embed_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens);
 
 /* The whole layer (section 2, Eq. 2 + Eq. 3) for num_tokens tokens in num_seqs sequences.
@@ -201,7 +206,7 @@ int ngram_embed_fwd_static_ws(const ngram_embed_plan* plan, const int32_t* token
 
 /* Synchronise `stream` and copy the sticky status word to *status_out. */
 int ngram_embed_get_status(const void* workspace, void* stream, int32_t* status_out);
-/* Zero the status word (asynchronous on `stream`). */
+/* Zero the workspace head: status word and stream-K counters (asynchronous on `stream`). */
 int ngram_embed_clear_status(void* workspace, void* stream);
 
 /* Self-test of the device-side bounded wait used by every pipeline barrier of the
@@ -238,6 +243,16 @@ int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on);
 
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */
 int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);
+
+/* Schedule of the one-CTA tensor-core kernel: 0 = automatic (stream-K when one tile per CTA
+ * would leave more than a tenth of the last wave's SMs idle), 1 = stream-K whenever possible,
+ * 2 = never. Stream-K gives every SM an equal run of (tile, k-block) units; a tile split
+ * between CTAs is summed in fp32 by whichever CTA finishes its piece last, so no CTA waits
+ * for another. It needs the workspace's partial tiles, at most 2048 tiles and at least
+ * one k-block per SM; otherwise, and with the CTA-pair form, the kernel takes one tile per
+ * CTA. A tuning knob: results agree within the stated tolerance (the summation order
+ * differs). */
+int ngram_embed_plan_set_stream_k(ngram_embed_plan* plan, int mode);
 
 #ifdef __cplusplus
 }

@@ -79,7 +79,8 @@ def test_plan_without_device_validates_then_fails_launch(ne):
     assert rc == 0 and h.value
     lib = ne._lib
     ws_need = lib.ngram_embed_workspace_bytes(h, 1000)
-    assert ws_need == 256 + ((1000 * 4 * 4 + 255) // 256) * 256
+    # head (status word + 2048 x 4 stream-K counters), indices; no SM count without a device
+    assert ws_need == 256 + 2048 * 4 * 4 + ((1000 * 4 * 4 + 255) // 256) * 256
     fake = ctypes.c_void_p(0x10000)           # never dereferenced
     odd = ctypes.c_void_p(0x10004)
     tabs = (ctypes.c_void_p * 4)(0x20000, 0x30000, 0x40000, 0x50000)
@@ -94,6 +95,7 @@ def test_plan_without_device_validates_then_fails_launch(ne):
     assert fwd(fake, ws_need) == -5            # would launch: no device
     assert lib.ngram_embed_plan_set_variant(h, 9) == -1
     assert lib.ngram_embed_plan_set_tile_n(h, 64) == -1
+    assert lib.ngram_embed_plan_set_stream_k(h, 3) == -1 and lib.ngram_embed_plan_set_stream_k(h, 2) == 0
     assert lib.ngram_embed_plan_uses_tensor_cores(h) == 1
     bad_cache = ne._Cache(0, 0, 0, 4, 8)
     assert lib.ngram_cache_rollback(h, ctypes.byref(bad_cache), None, fake, 3, fake, ws_need, None) == -1

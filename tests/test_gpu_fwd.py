@@ -137,6 +137,69 @@ def test_gather_and_layout_bit_exact(ne, variant, tma_rows, pair, D, N, K):
     np.testing.assert_array_equal(out.float().cpu().numpy(), gen.bf16_bits_to_f32(E0h[tokens]) / (S + 1))
 
 
+# ---------------------------------------------------------------- stream-K schedule
+
+SK_SHAPES = [(3000, 1024, 3, 2, 301), (5000, 2048, 3, 2, 301), (4000, 4096, 2, 2, 1000), (5000, 1536, 4, 1, 77)]
+
+
+@pytest.mark.parametrize("shape", SK_SHAPES, ids=lambda s: "V0%d_D%d_N%d_K%d_T%d" % s)
+@pytest.mark.parametrize("tile_n", [256, 128])
+def test_stream_k_matches_oracle_and_is_repeatable(ne, shape, tile_n):
+    """One-CTA kernel with every SM given an equal run of (tile, k-block) units, so tiles are
+    split over up to a dozen CTAs: parity with the oracle; a second call on the same
+    workspace gives the same bits (the fixup order is fixed and the arrival counters are
+    left at zero); data-parallel schedule agrees within the tolerance."""
+    V0, D, N, K, T = shape
+    cfg = small_cfg(V0, D, N, K, seed=5)
+    if D % tile_n:
+        pytest.skip("D not a multiple of the tile width")
+    lengths = [T // 3, 0, T - T // 3 - 5, 5]
+    tokens, offsets = ragged_tokens(cfg, lengths)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = plan_for(ne, cfg, 2, tile_n, pair=0)
+    ne.ngram_embed_plan_set_tma_rows(plan, 0)
+    ne.ngram_embed_plan_set_stream_k(plan, 1)
+    out = torch.full((T, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = ne.new_workspace(plan, T)
+    tk, of = dev_i32(tokens), dev_i32(offsets)
+    ne.ngram_embed_fwd(plan, tk, of, E0, E, W, out, ws)
+    assert ne.ngram_embed_get_status(ws) == 0
+    assert not ws[256:256 + 2048 * 16].any()  # every split tile's counters back at zero
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    assert_close(to_host_f64(out), want, what=f"{cfg.name} stream-K n{tile_n}")
+    again = torch.full_like(out, float("nan"))
+    ne.ngram_embed_fwd(plan, tk, of, E0, E, W, again, ws)
+    assert ne.ngram_embed_get_status(ws) == 0 and torch.equal(out, again)
+    ne.ngram_embed_plan_set_stream_k(plan, 2)
+    dp = torch.full_like(out, float("nan"))
+    ne.ngram_embed_fwd(plan, tk, of, E0, E, W, dp, ws)
+    assert ne.ngram_embed_get_status(ws) == 0
+    assert_close(to_host_f64(dp), want, what=f"{cfg.name} data-parallel n{tile_n}")
+
+
+def test_stream_k_bit_exact_with_identity_w(ne):
+    """W = I and E_0 = 0 under stream-K: each output element gets one nonzero product, so
+    the fp32 partials of a split tile add zeros to it and the result stays exact."""
+    cfg = small_cfg(7000, 1152, 2, 3, seed=3)   # S + 1 = 4: the scale is exact; 27 tiles of 128 x 128
+    S = cfg.S
+    tokens, offsets = ragged_tokens(cfg, [5, 128, 200, 3])
+    from tests.helpers import host_tables
+    _, Eh, _ = host_tables(cfg)
+    eye = gen.f32_to_bf16_bits(np.eye(cfg.D, dtype=np.float32))
+    idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, oracle.context_windows(cfg.N, tokens, offsets))
+    G = np.concatenate([gen.bf16_bits_to_f32(Eh[s][idx[:, s]]) for s in range(S)], axis=1)
+    plan = plan_for(ne, cfg, 2, 128, pair=0)
+    ne.ngram_embed_plan_set_tma_rows(plan, 0)
+    ne.ngram_embed_plan_set_stream_k(plan, 1)
+    zeros0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.bfloat16, device="cuda")
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, zeros0, [to_device(e, torch.bfloat16) for e in Eh],
+                          to_device(eye, torch.bfloat16))
+    assert status == 0
+    np.testing.assert_array_equal(out.float().cpu().numpy(), G / (S + 1))
+
+
 def test_n1_is_base_embedding(ne):
     cfg = configs.NgramConfig(name="n1", V0=3000, D=256, N=1, K=1, V_nk=(), dtype="bf16")
     tokens, offsets = ragged_tokens(cfg)
