@@ -40,6 +40,14 @@ WORKLOADS = {
         name="profile_bf16_D2048_N3_K2_small", num_seqs=2,
         V_nk=tuple(configs.primes_from(270000 + 131072 // 2, 4))),
 }
+DECODE_WORKLOADS = {
+    "spec_decode": configs.SPEC_DECODE,
+    # small case of the spec_decode kernel shapes for profiler captures: 8 sub-tables of
+    # ~300k rows (2.5 GB, still far above the 126 MB L2)
+    "profile_decode": configs.SPEC_DECODE.with_(
+        name="profile_spec_decode_bf16_D4096_N3_K4_small",
+        V_nk=tuple(configs.primes_from(300000 + 131072 // 2, 8))),
+}
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -233,25 +241,46 @@ def run_decode(ne, cfg, steps: int, warmup: int, dev, seed_offset: int = 0):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     status = ne.ngram_embed_get_status(ws)
-    # the projection alone at this shape, and the stand-alone hash + gather stage
-    idx = torch.empty((T, cfg.S), dtype=torch.int32, device=dev)
+    # The projection alone at this shape, and the stand-alone hash and gather stages. Each is
+    # timed as `n` launches on `n` different steps' inputs captured in one CUDA graph (so
+    # host launch overhead is not in the number and the sub-rows are not L2 hits from the
+    # launch before), averaged over the replay.
+    n_k = min(20, n_total)
+    idx_all = torch.empty((n_k, T, cfg.S), dtype=torch.int32, device=dev)
+    for i in range(n_k):
+        ne.ngram_hash_indices(plan, tok_all[i], offsets, idx_all[i], ws, cache=cache)
     G = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
-    ne.ngram_hash_indices(plan, tok_all[0], offsets, idx, ws, cache=cache)
 
-    def timed(fn, n=50):
-        for _ in range(5):
-            fn()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        for e0, e1 in ev:
-            e0.record()
-            fn()
-            e1.record()
+    def timed(fn):
+        gs = torch.cuda.Stream()
+        gs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(gs):
+            for i in range(3):
+                fn(i, gs)
+        torch.cuda.current_stream().wait_stream(gs)
+        gg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gg, stream=gs):
+            for i in range(n_k):
+                fn(i, gs)
         torch.cuda.synchronize()
-        return float(np.median([e0.elapsed_time(e1) for e0, e1 in ev]))
+        gg.replay()
+        torch.cuda.synchronize()
+        res_ms = []
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(gs):
+                e0.record(gs)
+                gg.replay()
+                e1.record(gs)
+            torch.cuda.synchronize()
+            res_ms.append(e0.elapsed_time(e1) / n_k)
+        del gg
+        return float(np.median(res_ms))
 
-    proj_ms = timed(lambda: ne.ngram_embed_project(plan, tok_all[0], idx, E0, E, W, out, ws))
-    hash_ms = timed(lambda: ne.ngram_hash_indices(plan, tok_all[0], offsets, idx, ws, cache=cache))
-    gather_ms = timed(lambda: ne.ngram_embed_gather(plan, idx, E, G, ws))
+    proj_ms = timed(lambda i, st: ne.ngram_embed_project(plan, tok_all[i], idx_all[i], E0, E, W, out, ws, stream=st))
+    hash_ms = timed(lambda i, st: ne.ngram_hash_indices(plan, tok_all[i], offsets, idx_all[n_k - 1 - i], ws,
+                                                        cache=cache, stream=st))
+    gather_ms = timed(lambda i, st: ne.ngram_embed_gather(plan, idx_all[i], E, G, ws, stream=st))
     gather_bytes = T * cfg.S * cfg.d * 2 * 2  # sub-rows read + G written
     pk = peaks()
     flops = 2.0 * T * cfg.D * cfg.D
@@ -284,6 +313,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-decode", action="store_true", help="skip the speculative-decode measurement")
     ap.add_argument("--decode-steps", type=int, default=100)
+    ap.add_argument("--decode-workload", default="spec_decode", choices=sorted(DECODE_WORKLOADS))
     ap.add_argument("--decode-only", action="store_true",
                     help="only the speculative-decode measurement (one JSON line with the decode object)")
     ap.add_argument("--profile-only", action="store_true",
@@ -308,7 +338,7 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     if args.decode_only:
-        decode = run_decode(ne, configs.SPEC_DECODE, args.decode_steps, max(args.warmup, 3), dev, seed_offset=rank)
+        decode = run_decode(ne, DECODE_WORKLOADS[args.decode_workload], args.decode_steps, max(args.warmup, 3), dev, seed_offset=rank)
         if rank == 0:
             print(json.dumps({"decode_only": True, "decode": decode}), flush=True)
         if world > 1:
@@ -414,7 +444,7 @@ def main():
     torch.cuda.empty_cache()
     decode = None
     if not args.no_decode:
-        decode = run_decode(ne, configs.SPEC_DECODE, args.decode_steps, max(args.warmup, 3), dev, seed_offset=rank)
+        decode = run_decode(ne, DECODE_WORKLOADS[args.decode_workload], args.decode_steps, max(args.warmup, 3), dev, seed_offset=rank)
         if world > 1:
             t = torch.tensor([decode["ms_per_step"]], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)

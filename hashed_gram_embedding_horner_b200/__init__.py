@@ -40,7 +40,7 @@ EXPORTED = [
     "ngram_embed_clear_status", "ngram_embed_error_string", "ngram_embed_plan_uses_tensor_cores",
     "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_plan_set_tma_rows",
     "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws", "ngram_embed_plan_set_cta_pair",
-    "ngram_cache_commit", "ngram_embed_plan_set_stream_k",
+    "ngram_cache_commit", "ngram_embed_plan_set_stream_k", "ngram_embed_plan_set_pdl",
 ]
 
 
@@ -78,6 +78,7 @@ _sig("ngram_embed_plan_set_tile_n", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
 _sig("ngram_embed_fwd_static_ws", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P])
 
@@ -170,6 +171,11 @@ def ngram_embed_plan_set_cta_pair(plan: Plan, on: bool):
 def ngram_embed_plan_set_stream_k(plan: Plan, mode: int):
     """0 automatic, 1 stream-K whenever the workspace and shape allow it, 2 never."""
     _check(_lib.ngram_embed_plan_set_stream_k(plan.handle, int(mode)), "ngram_embed_plan_set_stream_k")
+
+
+def ngram_embed_plan_set_pdl(plan: Plan, on: bool):
+    """Launch the plan's kernels as programmatic dependent launches (default on)."""
+    _check(_lib.ngram_embed_plan_set_pdl(plan.handle, int(bool(on))), "ngram_embed_plan_set_pdl")
 
 
 def ngram_embed_plan_uses_tensor_cores(plan: Plan) -> bool:

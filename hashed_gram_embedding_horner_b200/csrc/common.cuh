@@ -328,6 +328,17 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
 // Self-test of the bounded wait: one warp waits on an mbarrier that nothing ever
 // arrives at; mbar_wait must give up after limit_ns, raise NGRAM_STATUS_TIMEOUT
 // and let the kernel return normally.
+// Programmatic dependent launch (sm_90+): a kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream is still running.
+// pdl_wait() blocks until that kernel has completed and its memory is visible, so every
+// kernel here calls it before its first global memory access; what runs before it (barrier
+// init, TMEM allocation, descriptor prefetch) overlaps the previous kernel's tail.
+// pdl_launch_dependents() lets the next kernel be scheduled before this one ends; it only
+// moves scheduling earlier, never the next kernel's pdl_wait(). Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __global__ void selftest_wait_kernel(int* status, uint64_t limit_ns) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;

@@ -49,6 +49,8 @@ constexpr int kHashSmemOffsets = 4096;  // offsets staged in shared memory when 
 __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashParams p) {
   __shared__ int32_t s_off[kHashSmemOffsets];
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
 
   // Offsets check (sticky status; the lookups below stay in bounds regardless).
   if (i <= p.num_seqs) {

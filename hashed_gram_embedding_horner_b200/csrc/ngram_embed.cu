@@ -15,6 +15,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <utility>
 
 #include "common.cuh"
 #include "hash.cuh"
@@ -60,6 +61,7 @@ struct ngram_embed_plan {
   bool smem_attr_set[4] = {};  // per (kernel form, tile width) instance, on `device`
   bool cta_pair = true;        // use the CTA-pair (cta_group::2) kernel
   int stream_k = 0;            // one-CTA kernel schedule: 0 automatic, 1 stream-K when possible, 2 never
+  bool pdl = false;            // launch as programmatic dependent launches
   int max_clusters[2] = {0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
 };
 
@@ -98,6 +100,37 @@ size_t ws_bytes(const ngram_embed_plan* p, int64_t T) { return ws_base(p, T) + s
 
 int check_launch() { return cudaGetLastError() == cudaSuccess ? NGRAM_OK : NGRAM_ERR_CUDA; }
 
+// Every kernel launch: optionally as a programmatic dependent launch (the kernel may be
+// scheduled while the previous kernel on the stream finishes; its pdl_wait() orders
+// the memory), optionally in clusters of `cluster` CTAs.
+template <typename... KArgs, typename... Args>
+int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, int cluster,
+           Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = n ? attr : nullptr;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) return NGRAM_ERR_CUDA;
+  return check_launch();
+}
+
 int encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
               uint32_t box_inner, uint32_t box_outer, CUtensorMapL2promotion promo) {
   auto fn = encode_fn();
@@ -135,7 +168,9 @@ int refresh_maps(ngram_embed_plan* p, const void* const* E_nk, const void* W) {
 }
 
 // Stream-K (every CTA takes an equal share of the (tile, k-block) units) instead of one
-// tile per CTA per wave: when the last wave of tiles would leave many SMs idle.
+// tile per CTA per wave: when a grid of two or more waves ends in a wave that leaves many
+// SMs idle. Measured on B200 at D = 2048 and 4096: a unit costs about 1.3x as much under
+// stream-K (fixups, pieces that start mid-tile), and a single wave is never worth splitting.
 bool use_stream_k(const ngram_embed_plan* p, const ProjParams& prm, int64_t T, size_t ws_size) {
   const int tiles = prm.num_m_blocks * prm.num_n_blocks;
   const int64_t units = static_cast<int64_t>(tiles) * prm.num_k_blocks;
@@ -143,7 +178,7 @@ bool use_stream_k(const ngram_embed_plan* p, const ProjParams& prm, int64_t T, s
   if (ws_size < ws_bytes(p, T)) return false;
   if (p->stream_k == 1) return true;
   const int waves = (tiles + p->sms - 1) / p->sms;
-  return static_cast<double>(tiles) < 0.9 * waves * p->sms;  // data-parallel fill below 90%
+  return waves >= 2 && 1.3 * tiles < static_cast<double>(waves) * p->sms;
 }
 
 template <int BN>
@@ -158,8 +193,7 @@ int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
   }
   const int tiles = prm.num_m_blocks * prm.num_n_blocks;
   const int grid = (prm.stream_k || tiles > p->sms) ? p->sms : tiles;
-  kern<<<grid, kProjThreads, L::kLaunchBytes, st>>>(p->maps, prm);
-  return check_launch();
+  return launch(kern, dim3(grid), dim3(kProjThreads), L::kLaunchBytes, st, p->pdl, 1, p->maps, prm);
 }
 
 // CTA-pair kernel: clusters of two CTAs, one 256 x BN tile per pair per step.
@@ -196,9 +230,7 @@ int launch_tc_pair(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t 
     max_pairs = n;
   }
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  cfg.gridDim = dim3(2 * pairs);
-  if (cudaLaunchKernelEx(&cfg, kern, p->maps, prm) != cudaSuccess) return NGRAM_ERR_CUDA;
-  return check_launch();
+  return launch(kern, dim3(2 * pairs), dim3(kProjThreads), L::kLaunchBytes, st, p->pdl, 2, p->maps, prm);
 }
 
 int validate_common(const ngram_embed_plan* p, void* ws, size_t ws_size, int64_t T) {
@@ -244,8 +276,7 @@ int launch_hash(const ngram_embed_plan* p, const int32_t* tokens, const int32_t*
   h.status = status_ptr(ws);
   const int64_t work = T > num_seqs + 1 ? T : num_seqs + 1;
   const int64_t blocks = (work + 255) / 256;
-  hash_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(h);
-  return check_launch();
+  return launch(hash_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, p->pdl, 1, h);
 }
 
 int validate_cache(const ngram_embed_plan* p, const ngram_cache* c) {
@@ -285,8 +316,7 @@ int launch_simt(const ngram_embed_plan* p, const int32_t* tokens, const int32_t*
       return NGRAM_ERR_CUDA;
   }
   const int64_t blocks = (n_tok + tpb - 1) / tpb;
-  proj_simt_kernel<T><<<static_cast<unsigned>(blocks), 256, smem, st>>>(s);
-  return check_launch();
+  return launch(proj_simt_kernel<T>, dim3(static_cast<unsigned>(blocks)), dim3(256), smem, st, p->pdl, 1, s);
 }
 
 // ws_T: the token count the workspace was validated for (its index buffer's length);
@@ -451,6 +481,12 @@ int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int bn) {
   return NGRAM_OK;
 }
 
+int ngram_embed_plan_set_pdl(ngram_embed_plan* plan, int on) {
+  if (!plan || (on != 0 && on != 1)) return NGRAM_ERR_INVALID_ARG;
+  plan->pdl = on != 0;
+  return NGRAM_OK;
+}
+
 int ngram_embed_plan_set_stream_k(ngram_embed_plan* plan, int mode) {
   if (!plan || mode < 0 || mode > 2) return NGRAM_ERR_INVALID_ARG;
   plan->stream_k = mode;
@@ -541,12 +577,14 @@ int ngram_embed_gather(const ngram_embed_plan* plan, const int32_t* idx, int64_t
   g.S = plan->S;
   g.row_bytes = plan->d * plan->elt;
   g.status = status_ptr(workspace);
-  const int64_t rows = num_tokens * plan->S;
-  int64_t blocks = (rows + 7) / 8;
-  const int64_t cap = static_cast<int64_t>(plan->sms) * 16;
+  // every resident thread (8 blocks of 256 per SM, spread evenly over the SMs) takes an
+  // equal share of the 16-byte vectors; fewer blocks only when there are fewer vectors
+  const int64_t vecs = num_tokens * plan->S * (g.row_bytes / 16);
+  int64_t blocks = (vecs + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(plan->sms > 0 ? plan->sms : 1) * 8;
   if (blocks > cap) blocks = cap;
-  gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(g);
-  return check_launch();
+  return launch(gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                static_cast<cudaStream_t>(stream), plan->pdl, 1, g);
 }
 
 static int cache_launch(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots,
@@ -577,13 +615,10 @@ static int cache_launch(const ngram_embed_plan* plan, const ngram_cache* cache, 
   c.n = n;
   c.status = status_ptr(workspace);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (which == 0)
-    cache_reset_kernel<<<(n + 255) / 256, 256, 0, st>>>(c);
-  else if (which == 1 || which == 3)
-    cache_append_kernel<<<(n + 7) / 8, 256, 0, st>>>(c);
-  else
-    cache_rollback_kernel<<<(n + 255) / 256, 256, 0, st>>>(c);
-  return check_launch();
+  if (which == 0) return launch(cache_reset_kernel, dim3((n + 255) / 256), dim3(256), 0, st, plan->pdl, 1, c);
+  if (which == 1 || which == 3)
+    return launch(cache_append_kernel, dim3((n + 7) / 8), dim3(256), 0, st, plan->pdl, 1, c);
+  return launch(cache_rollback_kernel, dim3((n + 255) / 256), dim3(256), 0, st, plan->pdl, 1, c);
 }
 
 int ngram_cache_reset(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots, int32_t n,

@@ -286,6 +286,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();  // nothing above touched global memory
 
   const int num_tiles = p.num_m_blocks * p.num_n_blocks;
   const int KB = p.num_k_blocks;

@@ -48,6 +48,8 @@ struct SimtParams {
 template <typename T>
 __global__ void __launch_bounds__(256) proj_simt_kernel(const __grid_constant__ SimtParams<T> p) {
   extern __shared__ float g[];  // [tokens_per_block][D]
+  pdl_launch_dependents();
+  pdl_wait();
   const int TPB = p.tokens_per_block;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * TPB;
   const int64_t left = p.T_tokens - t0;
@@ -117,24 +119,51 @@ struct GatherParams {
   int* status;
 };
 
-// One warp per (token, sub-table) row: 16-byte vector copies of E_s[idx] into
-// G[i][s*d .. (s+1)*d). Grid-stride over rows.
+// 16-byte vectors of G, numbered row-major (row = token * S + s): vector v is copied by
+// thread v mod (threads in the grid), so a warp covers 512 contiguous bytes of one row and
+// the whole grid moves threads x 16 bytes per pass. Each thread issues the loads of
+// kGatherUnroll passes before any of their stores, so a grid of every resident thread has
+// all sub-rows of a decode step (1280 tokens x 8 x 1 KiB = 10 MiB) in flight at once.
+constexpr int kGatherUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ GatherParams p) {
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const int vec = p.row_bytes >> 4;
-  for (int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       w < p.T * p.S; w += warps) {
-    const int64_t i = w / p.S;
-    const int s = static_cast<int>(w - i * p.S);
-    int32_t r = p.idx[w];
-    if (static_cast<uint32_t>(r) >= p.Vs[s]) {
-      if (lane == 0) set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
-      r = 0;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int vec_per_row = p.row_bytes >> 4;
+  const int64_t total = p.T * p.S * vec_per_row;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
+       base += nthreads * kGatherUnroll) {
+    uint4 v[kGatherUnroll];
+    int64_t dst_off[kGatherUnroll];
+#pragma unroll
+    for (int j = 0; j < kGatherUnroll; ++j) {
+      const int64_t vi = base + j * nthreads;
+      dst_off[j] = -1;
+      if (vi < total) {
+        const int64_t row = vi / vec_per_row;
+        const int c = static_cast<int>(vi - row * vec_per_row);
+        const int s = static_cast<int>(row % p.S);
+        int32_t r = __ldg(p.idx + row);
+        if (static_cast<uint32_t>(r) >= p.Vs[s]) {
+          set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+          r = 0;
+        }
+        v[j] = ld_stream_v4(p.E[s] + static_cast<int64_t>(r) * p.row_bytes + c * 16);
+        dst_off[j] = vi * 16;
+      }
     }
-    const uint4* src = reinterpret_cast<const uint4*>(p.E[s] + static_cast<int64_t>(r) * p.row_bytes);
-    uint4* dst = reinterpret_cast<uint4*>(p.G + (i * p.S + s) * static_cast<int64_t>(p.row_bytes));
-    for (int v = lane; v < vec; v += 32) dst[v] = __ldg(src + v);
+#pragma unroll
+    for (int j = 0; j < kGatherUnroll; ++j)
+      if (dst_off[j] >= 0) *reinterpret_cast<uint4*>(p.G + dst_off[j]) = v[j];
   }
 }
 
@@ -166,6 +195,8 @@ __device__ __forceinline__ int32_t entry_slot(const CacheParams& p, int32_t i) {
 }
 
 __global__ void cache_reset_kernel(const __grid_constant__ CacheParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int32_t i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= p.n) return;
   const int32_t s = entry_slot(p, i);
@@ -177,6 +208,8 @@ __global__ void cache_reset_kernel(const __grid_constant__ CacheParams p) {
 // One warp per entry: write the ids at positions len .. len+m-1 (slot pos % C), then
 // len += m and valid_from = max(valid_from, len - C). Rejected entries change nothing.
 __global__ void cache_append_kernel(const __grid_constant__ CacheParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int32_t i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (i >= p.n) return;
@@ -215,6 +248,8 @@ __global__ void cache_append_kernel(const __grid_constant__ CacheParams p) {
 // One thread per entry: drop the newest counts[i] ids if the ring still holds the
 // newest N-1 positions that remain; otherwise flag and leave the slot unchanged.
 __global__ void cache_rollback_kernel(const __grid_constant__ CacheParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int32_t i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= p.n) return;
   const int32_t s = entry_slot(p, i);

@@ -244,8 +244,9 @@ int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on);
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */
 int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);
 
-/* Schedule of the one-CTA tensor-core kernel: 0 = automatic (stream-K when one tile per CTA
- * would leave more than a tenth of the last wave's SMs idle), 1 = stream-K whenever possible,
+/* Schedule of the one-CTA tensor-core kernel: 0 = automatic (stream-K when the grid takes two
+ * or more waves of one tile per CTA and the last wave leaves many SMs idle, e.g. 160 tiles of
+ * 128 x 256 on 148 SMs), 1 = stream-K whenever possible,
  * 2 = never. Stream-K gives every SM an equal run of (tile, k-block) units; a tile split
  * between CTAs is summed in fp32 by whichever CTA finishes its piece last, so no CTA waits
  * for another. It needs the workspace's partial tiles, at most 2048 tiles and at least
@@ -253,6 +254,14 @@ int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);
  * CTA. A tuning knob: results agree within the stated tolerance (the summation order
  * differs). */
 int ngram_embed_plan_set_stream_k(ngram_embed_plan* plan, int mode);
+
+/* 1 = launch every kernel of the plan as a programmatic dependent launch: it may be
+ * scheduled while the kernel before it on the stream finishes, and runs only its setup
+ * (barriers, tensor-memory allocation) until that kernel has completed and its writes are
+ * visible. 0 (default) = plain launches: measured on B200 inside CUDA graphs, the gap
+ * between launches is already about 1 us, and early-scheduled grids slowed the decode
+ * step's hash -> projection pair down. Results do not change. */
+int ngram_embed_plan_set_pdl(ngram_embed_plan* plan, int on);
 
 #ifdef __cplusplus
 }

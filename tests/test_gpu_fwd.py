@@ -325,3 +325,55 @@ def test_spec_decode_forward_through_ring(ne):
     del E0, E, W
     gc.collect()
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("pair", [0, 1])
+def test_pdl_and_graph_replay_match_plain_launches(ne, pair):
+    """Decode-like steps back to back (forward through the ring, then commit the accepted
+    ids), with no host sync in between: programmatic dependent launches, eagerly and
+    replayed from a CUDA graph, give the same bits and the same ring as plain launches."""
+    cfg = small_cfg(5000, 1024, 3, 2, seed=11)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    B, P, steps = 40, 5, 4
+    rng = np.random.default_rng(4)
+    toks = [dev_i32(rng.integers(0, cfg.V0, B * P)) for _ in range(steps)]
+    cnts = [dev_i32(1 + rng.integers(0, P, B)) for _ in range(steps)]
+    off = dev_i32(np.arange(B + 1) * P)
+
+    def run(pdl, graph):
+        plan = plan_for(ne, cfg, pair=pair)
+        ne.ngram_embed_plan_set_pdl(plan, pdl)
+        ws = ne.new_workspace(plan, B * P)
+        cache = ne.Cache.empty(B, 8)
+        ne.ngram_cache_reset(plan, cache, ws)
+        outs = [torch.full((B * P, cfg.D), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(steps)]
+
+        def body(st=None):
+            for i in range(steps):
+                ne.ngram_embed_fwd(plan, toks[i], off, E0, E, W, outs[i], ws, cache=cache, stream=st)
+                ne.ngram_cache_commit(plan, cache, toks[i], P, cnts[i], ws, stream=st)
+
+        if graph:
+            # first call outside the capture: it sets kernel attributes and encodes tensor maps
+            ne.ngram_embed_fwd(plan, toks[0], off, E0, E, W, outs[0], ws, cache=cache)
+            torch.cuda.synchronize()
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                body(s)
+            g.replay()
+            torch.cuda.synchronize()
+            del g
+        else:
+            body()
+        assert ne.ngram_embed_get_status(ws) == 0
+        return [o.clone() for o in outs], cache.ring.clone(), cache.len.clone()
+
+    ref = run(0, False)
+    for pdl, graph in ((1, False), (1, True)):
+        got = run(pdl, graph)
+        assert all(torch.equal(a, b) for a, b in zip(ref[0], got[0])), (pdl, graph)
+        assert torch.equal(ref[1], got[1]) and torch.equal(ref[2], got[2])
