@@ -280,8 +280,12 @@ def run_decode(ne, cfg, steps: int, warmup: int, dev, seed_offset: int = 0):
     proj_ms = timed(lambda i, st: ne.ngram_embed_project(plan, tok_all[i], idx_all[i], E0, E, W, out, ws, stream=st))
     hash_ms = timed(lambda i, st: ne.ngram_hash_indices(plan, tok_all[i], offsets, idx_all[n_k - 1 - i], ws,
                                                         cache=cache, stream=st))
-    gather_ms = timed(lambda i, st: ne.ngram_embed_gather(plan, idx_all[i], E, G, ws, stream=st))
-    gather_bytes = T * cfg.S * cfg.d * 2 * 2  # sub-rows read + G written
+    R0 = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
+    # the step's table lookups alone: its 8 sub-rows and E_0 row per token (the layer's HBM
+    # reads besides W, 16 KiB per token) copied to G and E0_out (written back, 16 KiB)
+    gather_ms = timed(lambda i, st: ne.ngram_embed_gather(plan, idx_all[i], E, G, ws, tokens=tok_all[i], E0=E0,
+                                                          E0_out=R0, stream=st))
+    gather_bytes = T * (cfg.S * cfg.d + cfg.D) * 2 * 2  # rows read + rows written
     pk = peaks()
     flops = 2.0 * T * cfg.D * cfg.D
     res = {

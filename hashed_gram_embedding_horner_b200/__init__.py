@@ -41,6 +41,7 @@ EXPORTED = [
     "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_plan_set_tma_rows",
     "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws", "ngram_embed_plan_set_cta_pair",
     "ngram_cache_commit", "ngram_embed_plan_set_stream_k", "ngram_embed_plan_set_pdl",
+    "ngram_embed_plan_set_a_stages",
 ]
 
 
@@ -64,7 +65,7 @@ _sig("ngram_embed_workspace_bytes", [_P, _I64], _SZ)
 _sig("ngram_embed_fwd", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P])
 _sig("ngram_hash_indices", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _SZ, _P])
 _sig("ngram_embed_project", [_P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P])
-_sig("ngram_embed_gather", [_P, _P, _I64, _P, _P, _P, _SZ, _P])
+_sig("ngram_embed_gather", [_P, _P, _I64, _P, _P, _P, _P, _P, _P, _SZ, _P])
 _sig("ngram_cache_reset", [_P, _P, _P, _I32, _P, _SZ, _P])
 _sig("ngram_cache_append", [_P, _P, _P, _P, _P, _I32, _P, _SZ, _P])
 _sig("ngram_cache_rollback", [_P, _P, _P, _P, _I32, _P, _SZ, _P])
@@ -79,6 +80,7 @@ _sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_a_stages", [_P, ctypes.c_int])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
 _sig("ngram_embed_fwd_static_ws", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P])
 
@@ -173,6 +175,11 @@ def ngram_embed_plan_set_stream_k(plan: Plan, mode: int):
     _check(_lib.ngram_embed_plan_set_stream_k(plan.handle, int(mode)), "ngram_embed_plan_set_stream_k")
 
 
+def ngram_embed_plan_set_a_stages(plan: Plan, stages: int):
+    """Depth of the one-CTA kernel's A ring (0 = default); the W ring takes the rest."""
+    _check(_lib.ngram_embed_plan_set_a_stages(plan.handle, int(stages)), "ngram_embed_plan_set_a_stages")
+
+
 def ngram_embed_plan_set_pdl(plan: Plan, on: bool):
     """Launch the plan's kernels as programmatic dependent launches (default on)."""
     _check(_lib.ngram_embed_plan_set_pdl(plan.handle, int(bool(on))), "ngram_embed_plan_set_pdl")
@@ -220,9 +227,14 @@ def ngram_embed_project(plan: Plan, tokens, idx, E0, E_nk, W_stacked, out, works
     _check(rc, "ngram_embed_project")
 
 
-def ngram_embed_gather(plan: Plan, idx, E_nk, G_out, workspace, stream=None):
+def ngram_embed_gather(plan: Plan, idx, E_nk, G_out, workspace, tokens=None, E0=None, E0_out=None, stream=None):
+    """Sub-rows E_s[idx[i, s]] into G_out [T x D]; with E0_out, also E_0[tokens[i]] rows."""
     tabs = _tables(E_nk)
+    if E0_out is not None and (tokens is None or E0 is None):
+        raise ValueError("E0_out needs tokens and E0")
     rc = _lib.ngram_embed_gather(plan.handle, _i32(idx, "idx"), idx.shape[0], tabs, _ptr(G_out),
+                                 None if tokens is None else _i32(tokens, "tokens"),
+                                 None if E0 is None else _ptr(E0), None if E0_out is None else _ptr(E0_out),
                                  _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "ngram_embed_gather")
 

@@ -32,8 +32,15 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kSkMaxTiles = 2048;                          // stream-K only for grids of at most this many tiles
 constexpr size_t kSkCounterBytes = size_t(kSkMaxTiles) * 4 * sizeof(int32_t);  // one per (tile, row quarter)
 constexpr size_t kHeadBytes = kStatusBytes + kSkCounterBytes;                   // zeroed by clear_status
-constexpr int kStages = 4;       // one-CTA kernel: 4 x (16 KB A + 32 KB W) at N = 256
-constexpr int kPairStages = 6;   // CTA-pair kernel: 6 x (16 KB A + 16 KB W) per CTA at N = 256
+// One-CTA kernel shared memory (224 KB): A stages of 16 KB, W stages of BN x 128 B and the
+// epilogue's 128 x BN bf16 tile. N = 256: A + W = 2 + 4, 4 + 3 or 6 + 2 stages;
+// N = 128: 6 + 6, 8 + 4 or 10 + 2.
+constexpr int kDefaultAStages256 = 4;
+constexpr int kDefaultAStages128 = 8;
+// CTA-pair kernel shared memory per CTA: A stages of 16 KB, W stages of BN/2 x 128 B.
+// N = 256: A + W = 6 + 6, 8 + 5 or 10 + 4 stages; N = 128: 8 + 8, 10 + 8 or 12 + 4.
+constexpr int kDefaultPairAStages256 = 8;
+constexpr int kDefaultPairAStages128 = 10;
 
 enum Variant : int { kAuto = 0, kTcTmaRows = 1, kTcSplitRows = 2, kSimt = 3 };
 constexpr int kDefaultTmaRows = 0;  // A rows per tile gathered by TMA; the rest by cp.async (fastest measured)
@@ -58,7 +65,10 @@ struct ngram_embed_plan {
   const void* map_W = nullptr;
   const void* map_E[kMaxS] = {};
   bool maps_valid = false;
-  bool smem_attr_set[4] = {};  // per (kernel form, tile width) instance, on `device`
+  const void* map_out = nullptr;  // the out map's pointer and row count
+  int64_t map_out_T = -1;
+  bool smem_attr_set[12] = {};  // per kernel instance (form, tile width, rings), on `device`
+  int a_stages = 0;            // one-CTA kernel: A ring depth (0 = default for the tile width)
   bool cta_pair = true;        // use the CTA-pair (cta_group::2) kernel
   int stream_k = 0;            // one-CTA kernel schedule: 0 automatic, 1 stream-K when possible, 2 never
   bool pdl = false;            // launch as programmatic dependent launches
@@ -145,7 +155,15 @@ int encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
   return r == CUDA_SUCCESS ? NGRAM_OK : NGRAM_ERR_CUDA;
 }
 
-int refresh_maps(ngram_embed_plan* p, const void* const* E_nk, const void* W) {
+int refresh_maps(ngram_embed_plan* p, const void* const* E_nk, const void* W, void* out, int64_t T) {
+  if (p->map_out != out || p->map_out_T != T) {
+    p->map_out = nullptr;
+    int rc = encode_2d(&p->maps.Out, out, p->D, static_cast<uint64_t>(T), static_cast<uint64_t>(p->D) * 2, kBK, 32,
+                       CU_TENSOR_MAP_L2_PROMOTION_NONE);
+    if (rc) return rc;
+    p->map_out = out;
+    p->map_out_T = T;
+  }
   bool same = p->maps_valid && p->map_W == W;
   for (int s = 0; same && s < p->S; ++s) same = p->map_E[s] == E_nk[s];
   if (same) return NGRAM_OK;
@@ -181,11 +199,11 @@ bool use_stream_k(const ngram_embed_plan* p, const ProjParams& prm, int64_t T, s
   return waves >= 2 && 1.3 * tiles < static_cast<double>(waves) * p->sms;
 }
 
-template <int BN>
-int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
-  using L = ProjSmem<BN, kStages>;
-  auto kern = proj_sm100_kernel<BN, kStages>;
-  const int key = BN == 256 ? 1 : 0;
+template <int BN, int AST, int WST>
+int launch_tc_rings(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st, int key) {
+  using L = ProjSmem<BN, AST, WST>;
+  static_assert(L::kLaunchBytes <= 232448, "one-CTA kernel rings exceed 227 KB of shared memory");
+  auto kern = proj_sm100_kernel<BN, AST, WST>;
   if (!p->smem_attr_set[key]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess)
       return NGRAM_ERR_CUDA;
@@ -196,13 +214,28 @@ int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
   return launch(kern, dim3(grid), dim3(kProjThreads), L::kLaunchBytes, st, p->pdl, 1, p->maps, prm);
 }
 
-// CTA-pair kernel: clusters of two CTAs, one 256 x BN tile per pair per step.
 template <int BN>
-int launch_tc_pair(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t st) {
-  constexpr int kStg = BN == 256 ? kPairStages : 8;
-  using L = PairSmem<BN, kStg>;
-  auto kern = proj_sm100_pair_kernel<BN, kStg>;
-  const int key = 2 + (BN == 256 ? 1 : 0);
+int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
+  if (BN == 256) {
+    switch (p->a_stages ? p->a_stages : kDefaultAStages256) {
+      case 2: return launch_tc_rings<256, 2, 4>(p, prm, st, 0);
+      case 6: return launch_tc_rings<256, 6, 2>(p, prm, st, 1);
+      default: return launch_tc_rings<256, 4, 3>(p, prm, st, 2);
+    }
+  }
+  switch (p->a_stages ? p->a_stages : kDefaultAStages128) {
+    case 6: return launch_tc_rings<128, 6, 6>(p, prm, st, 3);
+    case 10: return launch_tc_rings<128, 10, 2>(p, prm, st, 5);
+    default: return launch_tc_rings<128, 8, 4>(p, prm, st, 4);
+  }
+}
+
+// CTA-pair kernel: clusters of two CTAs, one 256 x BN tile per pair per step.
+template <int BN, int AST, int WST>
+int launch_tc_pair_rings(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t st, int key) {
+  using L = PairSmem<BN, AST, WST>;
+  static_assert(L::kLaunchBytes <= 232448, "CTA-pair kernel rings exceed 227 KB of shared memory");
+  auto kern = proj_sm100_pair_kernel<BN, AST, WST>;
   if (!p->smem_attr_set[key]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
@@ -231,6 +264,22 @@ int launch_tc_pair(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t 
   }
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   return launch(kern, dim3(2 * pairs), dim3(kProjThreads), L::kLaunchBytes, st, p->pdl, 2, p->maps, prm);
+}
+
+template <int BN>
+int launch_tc_pair(ngram_embed_plan* p, const ProjParams& prm, int64_t T, cudaStream_t st) {
+  if (BN == 256) {
+    switch (p->a_stages ? p->a_stages : kDefaultPairAStages256) {
+      case 6: return launch_tc_pair_rings<256, 6, 6>(p, prm, T, st, 6);
+      case 10: return launch_tc_pair_rings<256, 10, 4>(p, prm, T, st, 8);
+      default: return launch_tc_pair_rings<256, 8, 5>(p, prm, T, st, 7);
+    }
+  }
+  switch (p->a_stages ? p->a_stages : kDefaultPairAStages128) {
+    case 8: return launch_tc_pair_rings<128, 8, 8>(p, prm, T, st, 9);
+    case 12: return launch_tc_pair_rings<128, 12, 4>(p, prm, T, st, 11);
+    default: return launch_tc_pair_rings<128, 10, 8>(p, prm, T, st, 10);
+  }
 }
 
 int validate_common(const ngram_embed_plan* p, void* ws, size_t ws_size, int64_t T) {
@@ -329,7 +378,7 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
                ? launch_simt<float>(p, tokens, idx, T, E0, E_nk, W, out, ws, st)
                : launch_simt<uint16_t>(p, tokens, idx, T, E0, E_nk, W, out, ws, st);
   }
-  int rc = refresh_maps(p, E_nk, W);
+  int rc = refresh_maps(p, E_nk, W, out, T);
   if (rc) return rc;
   ProjParams prm{};
   prm.tokens = tokens;
@@ -481,6 +530,15 @@ int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int bn) {
   return NGRAM_OK;
 }
 
+int ngram_embed_plan_set_a_stages(ngram_embed_plan* plan, int stages) {
+  if (!plan) return NGRAM_ERR_INVALID_ARG;
+  // every depth some form takes; a form given a depth it does not take uses its default
+  const bool ok = stages == 0 || (stages % 2 == 0 && stages >= 2 && stages <= 12);
+  if (!ok) return NGRAM_ERR_INVALID_ARG;
+  plan->a_stages = stages;
+  return NGRAM_OK;
+}
+
 int ngram_embed_plan_set_pdl(ngram_embed_plan* plan, int on) {
   if (!plan || (on != 0 && on != 1)) return NGRAM_ERR_INVALID_ARG;
   plan->pdl = on != 0;
@@ -555,14 +613,16 @@ int ngram_embed_fwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
 }
 
 int ngram_embed_gather(const ngram_embed_plan* plan, const int32_t* idx, int64_t num_tokens,
-                       const void* const* E_nk, void* G_out, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+                       const void* const* E_nk, void* G_out, const int32_t* tokens, const void* E0,
+                       void* E0_out, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = validate_common(plan, workspace, workspace_bytes, 0);
   if (rc) return rc;
   if (num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
-  if (num_tokens == 0 || plan->S == 0) return NGRAM_OK;
-  if (!idx || !E_nk || !G_out) return NGRAM_ERR_INVALID_ARG;
-  if (!aligned16(G_out)) return NGRAM_ERR_MISALIGNED;
+  if (num_tokens == 0 || (plan->S == 0 && !E0_out)) return NGRAM_OK;
+  if (plan->S > 0 && (!idx || !E_nk || !G_out)) return NGRAM_ERR_INVALID_ARG;
+  if (E0_out && (!tokens || !E0)) return NGRAM_ERR_INVALID_ARG;
+  if ((G_out && !aligned16(G_out)) || (E0_out && (!aligned16(E0_out) || !aligned16(E0))))
+    return NGRAM_ERR_MISALIGNED;
   GatherParams g{};
   for (int s = 0; s < plan->S; ++s) {
     if (!E_nk[s]) return NGRAM_ERR_INVALID_ARG;
@@ -576,10 +636,25 @@ int ngram_embed_gather(const ngram_embed_plan* plan, const int32_t* idx, int64_t
   g.T = num_tokens;
   g.S = plan->S;
   g.row_bytes = plan->d * plan->elt;
+  g.tokens = tokens;
+  g.E0 = static_cast<const uint8_t*>(E0);
+  g.E0_out = static_cast<uint8_t*>(E0_out);
+  g.V0 = static_cast<uint32_t>(plan->V0);
+  g.e0_row_bytes = plan->D * plan->elt;
   g.status = status_ptr(workspace);
   // every resident thread (8 blocks of 256 per SM, spread evenly over the SMs) takes an
   // equal share of the 16-byte vectors; fewer blocks only when there are fewer vectors
-  const int64_t vecs = num_tokens * plan->S * (g.row_bytes / 16);
+  const int64_t vecs = num_tokens * plan->S * (g.row_bytes / 16) + (E0_out ? num_tokens * (g.e0_row_bytes / 16) : 0);
+  // the kernel numbers vectors (and its grid-stride steps) in 32 bits
+  if (vecs + static_cast<int64_t>(plan->sms > 0 ? plan->sms : 1) * 8 * 256 * kGatherUnroll > UINT32_MAX)
+    return NGRAM_ERR_UNSUPPORTED;
+  auto log2_or_neg = [](int v) {
+    int sh = 0;
+    while ((1 << sh) < v) ++sh;
+    return (1 << sh) == v ? sh : -1;
+  };
+  g.vshift = log2_or_neg(g.row_bytes / 16);
+  g.eshift = log2_or_neg(g.e0_row_bytes / 16);
   int64_t blocks = (vecs + 255) / 256;
   const int64_t cap = static_cast<int64_t>(plan->sms > 0 ? plan->sms : 1) * 8;
   if (blocks > cap) blocks = cap;

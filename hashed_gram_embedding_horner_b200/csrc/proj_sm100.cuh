@@ -28,8 +28,11 @@
 //               32*(w%4) ..+31), + E_0 row slice, * 1/(S+1), bf16 RNE, store.
 // Each tile walks its k-blocks starting at a tile-dependent rotation, so CTAs that share
 // a W column block (or an A row block) do not read the same lines at the same time.
-// Shared memory holds STAGES (A, B) stage pairs; TMEM holds two BN-column fp32
-// accumulators so the epilogue of one tile overlaps the main loop of the next.
+// Shared memory holds two rings with their own barriers: AST stages of gathered A rows and
+// WST stages of W tiles. A rows come from random table rows (often HBM misses, the longest
+// latency on the path) and W tiles from L2, so the A ring is the deeper one: decoupling the
+// rings lets more A bytes be in flight than a shared (A, W) stage would. TMEM holds two
+// BN-column fp32 accumulators so the epilogue of one tile overlaps the main loop of the next.
 // Every wait is bounded (see mbar_wait); on a timeout all roles stop, drain what they
 // have in flight, free TMEM and return with NGRAM_STATUS_TIMEOUT set.
 #pragma once
@@ -72,15 +75,18 @@ struct ProjMaps {
   CUtensorMap W;            // W_stacked, box {64, BN}, 128-byte swizzle
   CUtensorMap Whalf;        // W_stacked, box {64, BN/2} (CTA-pair kernel: each CTA loads half)
   CUtensorMap E[kMaxS];     // sub-table s, box {64, 1}, 128-byte swizzle (gather4)
+  CUtensorMap Out;          // out [T x D], box {64, 32}, 128-byte swizzle (epilogue TMA stores)
 };
 
-template <int BN, int STAGES>
+template <int BN, int AST, int WST>
 struct ProjSmem {
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBarOffset = STAGES * kStageBytes;
-  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kWOffset = AST * kABytes;  // A ring, then the W ring,
+  static constexpr int kEOffset = kWOffset + WST * kBBytes;  // then the epilogue's tile
+  static constexpr int kEBytes = kBM * BN * 2;  // E_0 slice in, bf16 output out (BN/64 boxes of 128 x 64)
+  static constexpr int kBarOffset = kEOffset + kEBytes;
+  static constexpr int kNumBars = 2 * AST + 2 * WST + 5;
   static constexpr int kBytes = kBarOffset + kNumBars * 8 + 16;
   static constexpr int kLaunchBytes = kBytes + 1024;  // slack for 1024-byte alignment
   static constexpr int kTmemCols = 2 * BN;
@@ -241,32 +247,39 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-template <int BN, int STAGES>
+template <int BN, int AST, int WST>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_sm100_kernel(const __grid_constant__ ProjMaps maps, const __grid_constant__ ProjParams p) {
-  using L = ProjSmem<BN, STAGES>;
+  using L = ProjSmem<BN, AST, WST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kBarOffset;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
-  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };                   // A ring
+  auto empty_bar = [&](int s) { return bar0 + 8u * (AST + s); };
+  auto wfull_bar = [&](int s) { return bar0 + 8u * (2 * AST + s); };      // W ring
+  auto wempty_bar = [&](int s) { return bar0 + 8u * (2 * AST + WST + s); };
+  constexpr int kT0 = 2 * AST + 2 * WST;
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (kT0 + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (kT0 + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (kT0 + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + L::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto a_tile = [&](int s) { return sbase + s * L::kStageBytes; };
-  auto b_tile = [&](int s) { return sbase + s * L::kStageBytes + L::kABytes; };
+  auto a_tile = [&](int s) { return sbase + s * L::kABytes; };
+  auto b_tile = [&](int s) { return sbase + L::kWOffset + s * L::kBBytes; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      // every A thread (cp.async completion), thread 0's TMA byte count, the W producer
-      mbar_init(full_bar(s), static_cast<uint32_t>(kAThreads) + 2u);
+    for (int s = 0; s < AST; ++s) {
+      // every A thread (cp.async completion) and thread 0's TMA byte count
+      mbar_init(full_bar(s), static_cast<uint32_t>(kAThreads) + 1u);
       mbar_init(empty_bar(s), 1u);  // one tcgen05.commit
+    }
+    for (int s = 0; s < WST; ++s) {
+      mbar_init(wfull_bar(s), 1u);   // the W producer's TMA byte count
+      mbar_init(wempty_bar(s), 1u);  // one tcgen05.commit
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1u);
@@ -352,7 +365,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         for (int j = 0; j < 4; ++j)
           if (j < n_cp) cp_async_16(a + (p.tma_rows + rsub + 32 * j) * 128 + swz, src[j] + c0);
         cp_async_arrive_noinc(full_bar(stage));
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++stage == AST) { stage = 0; phase ^= 1u; }
       }
       cur = nxt;
 #pragma unroll
@@ -379,10 +392,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         for (int i = g.i0; i < g.i1; ++i) {
           int kb = i + rot;
           if (kb >= KB) kb -= KB;
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_bar(stage), L::kBBytes);
-          tma_load_2d(b_tile(stage), &maps.W, kb * kBK, n_blk * BN, full_bar(stage), pol);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (!mbar_wait(wempty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(wfull_bar(stage), L::kBBytes);
+          tma_load_2d(b_tile(stage), &maps.W, kb * kBK, n_blk * BN, wfull_bar(stage), pol);
+          if (++stage == WST) { stage = 0; phase ^= 1u; }
         }
       }
     }
@@ -390,8 +403,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN);
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = 0, wstage = 0;
+      uint32_t phase = 0, wphase = 0;
       bool ok = true;
       int local = 0;
       for (Seg g = seg_first(wp, blockIdx.x); g.tile < num_tiles && ok; g = seg_next(wp, g), ++local) {
@@ -401,16 +414,19 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int i = g.i0; i < g.i1; ++i) {
+          if (!mbar_wait(wfull_bar(wstage), wphase, abort_flag, p.status)) { ok = false; break; }
           if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           fence_proxy_async_smem();  // the stage's cp.async rows were written by the generic proxy
           const uint64_t adesc = sw128_kmajor_desc(a_tile(stage));
-          const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage));
+          const uint64_t bdesc = sw128_kmajor_desc(b_tile(wstage));
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)  // K = 16 per instruction: +32 B = +2 in the address field
             umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (i > g.i0 || k != 0) ? 1u : 0u);
           umma_commit(empty_bar(stage));
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          umma_commit(wempty_bar(wstage));
+          if (++stage == AST) { stage = 0; phase ^= 1u; }
+          if (++wstage == WST) { wstage = 0; wphase ^= 1u; }
         }
         if (ok) umma_commit(tfull_bar(acc));
       }
@@ -422,6 +438,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int row_in_tile = q * 32 + lane;  // == TMEM lane
+    const uint32_t stage_q = sbase + L::kEOffset + q * 4096;  // this warp's rows of box 0
     const int64_t U = static_cast<int64_t>(num_tiles) * KB;
     int local = 0;
     for (Seg g = seg_first(wp, blockIdx.x); g.tile < num_tiles; g = seg_next(wp, g), ++local) {
@@ -440,10 +457,19 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       }
       const uint4* e0 = reinterpret_cast<const uint4*>(p.E0 + static_cast<int64_t>(t) * p.D + n_blk * BN);
       uint4* dst = reinterpret_cast<uint4*>(p.out + gr * p.D + n_blk * BN);
-      // E_0 slice of chunk 0 before waiting on the accumulator.
-      uint4 ecur[4];
-#pragma unroll
-      for (int v = 0; v < 4; ++v) ecur[v] = (valid && whole) ? __ldg(e0 + v) : make_uint4(0, 0, 0, 0);
+      if (whole) {
+        // Stage this row's E_0 slice now, a whole main loop ahead of its use: once the
+        // previous tile's TMA stores have read the rows, cp.async them into the tile buffer
+        // (box b holds columns 64b..64b+63; 16-byte chunk c of row r sits at c ^ (r % 8)).
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        if (valid) {
+          const uint16_t* e0row = p.E0 + static_cast<int64_t>(t) * p.D + n_blk * BN;
+#pragma unroll 8
+          for (int c = 0; c < BN / 8; ++c)
+            cp_async_16(stage_q + (c >> 3) * 16384 + lane * 128 + (((c & 7) ^ (lane & 7)) << 4), e0row + c * 8);
+        }
+      }
 
       bool got = false;
       if (lane == 0) got = mbar_wait(tfull_bar(acc), use & 1u, abort_flag, p.status);
@@ -451,37 +477,41 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
       if (whole) {
+        cp_async_wait_all();  // this lane's E_0 row
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + c * 32, v);
-          uint4 enext[4];
-          const bool has_next = c + 1 < BN / 32;
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            enext[w] = (valid && has_next) ? __ldg(e0 + (c + 1) * 4 + w) : make_uint4(0, 0, 0, 0);
           tmem_wait_ld();
           if (c + 1 == BN / 32) {
             tc_fence_before();
             mbar_arrive(tempty_bar(acc));  // accumulator fully read: MMA may reuse it
           }
-          if (valid) {
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const uint32_t ew[4] = {ecur[w].x, ecur[w].y, ecur[w].z, ecur[w].w};
-              uint32_t o[4];
+          for (int w = 0; w < 4; ++w) {  // columns 32c + 8w .. +7: chunk (4c + w) % 8 of box c / 2
+            const uint32_t sa = stage_q + (c >> 1) * 16384 + lane * 128 + (((((c & 1) << 2) | w) ^ (lane & 7)) << 4);
+            const uint4 e = ld_shared_v4(sa);
+            const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
+            uint32_t o[4];
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const int col = w * 8 + h * 2;
-                const float x0 = (__uint_as_float(v[col]) + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale;
-                const float x1 = (__uint_as_float(v[col + 1]) + bf16_bits_to_float(ew[h] >> 16)) * p.scale;
-                o[h] = pack_bf16x2(x0, x1);
-              }
-              dst[c * 4 + w] = make_uint4(o[0], o[1], o[2], o[3]);
+            for (int h = 0; h < 4; ++h) {
+              const int col = w * 8 + h * 2;
+              const float x0 = (__uint_as_float(v[col]) + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale;
+              const float x1 = (__uint_as_float(v[col + 1]) + bf16_bits_to_float(ew[h] >> 16)) * p.scale;
+              o[h] = pack_bf16x2(x0, x1);
             }
+            st_shared_v4(sa, make_uint4(o[0], o[1], o[2], o[3]));
           }
+        }
+        // The warp's 32 output rows go out as BN/64 TMA box stores (rows past T are clipped;
+        // a box that starts past T is not issued).
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && static_cast<int64_t>(m_blk) * kBM + q * 32 < p.T) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) ecur[w] = enext[w];
+          for (int b = 0; b < BN / 64; ++b)
+            tma_store_2d(&maps.Out, stage_q + b * 16384, n_blk * BN + b * 64, m_blk * kBM + q * 32);
+          bulk_commit_group();
         }
       } else {
         // Stream-K piece of a tile. Per (tile, row quarter) an arrival counter counts the
@@ -574,6 +604,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         mbar_arrive(tempty_bar(acc));  // accumulator read for the last time: MMA may reuse it
       }
     }
+    cp_async_wait_all();                   // E_0 rows still landing (after an abort)
+    if (lane == 0) bulk_wait_group<0>();  // output stores complete before the CTA exits
   }
 
   tc_fence_before();

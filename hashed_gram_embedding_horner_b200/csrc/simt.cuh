@@ -116,15 +116,23 @@ struct GatherParams {
   int64_t T;
   int S;
   int row_bytes;  // d * element size, a multiple of 16
+  // optional E_0 rows: E0_out[i] = E0[tokens[i]] (E0_out == nullptr: none)
+  const int32_t* tokens;
+  const uint8_t* E0;
+  uint8_t* E0_out;
+  uint32_t V0;
+  int e0_row_bytes;  // D * element size
+  int vshift, eshift;  // log2 of the 16-byte vectors per sub-row / per E_0 row, or -1
   int* status;
 };
 
-// 16-byte vectors of G, numbered row-major (row = token * S + s): vector v is copied by
-// thread v mod (threads in the grid), so a warp covers 512 contiguous bytes of one row and
-// the whole grid moves threads x 16 bytes per pass. Each thread issues the loads of
-// kGatherUnroll passes before any of their stores, so a grid of every resident thread has
-// all sub-rows of a decode step (1280 tokens x 8 x 1 KiB = 10 MiB) in flight at once.
-constexpr int kGatherUnroll = 4;
+// 16-byte vectors of G, numbered row-major (row = token * S + s), then (optionally) those
+// of the E_0 rows: vector v is copied by thread v mod (threads in the grid), so a warp
+// covers 512 contiguous bytes of one row and the grid moves threads x 16 bytes per pass.
+// Each thread issues the loads of kGatherUnroll passes before any of their stores, so a
+// grid of every resident thread has all rows of a decode step (1280 tokens x (8 sub-rows
+// of 1 KiB + one E_0 row of 8 KiB) = 20 MiB) in flight at once.
+constexpr int kGatherUnroll = 8;
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   uint4 v;
@@ -134,36 +142,59 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   return v;
 }
 
+// Vector index -> (row, vector in row): a shift when the row holds a power of two of
+// vectors (always, for d and D multiples of 8 that are powers of two), else a division.
+__device__ __forceinline__ uint32_t split_vec(uint32_t v, int shift, uint32_t per_row, uint32_t& c) {
+  const uint32_t row = shift >= 0 ? v >> shift : v / per_row;
+  c = v - row * per_row;
+  return row;
+}
+
 __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ GatherParams p) {
   pdl_launch_dependents();
   pdl_wait();
-  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int vec_per_row = p.row_bytes >> 4;
-  const int64_t total = p.T * p.S * vec_per_row;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
-       base += nthreads * kGatherUnroll) {
+  // 32-bit vector numbering (the host launches this kernel only when every index fits):
+  // the index arithmetic is per vector, and 64-bit division would cost more than the copy.
+  const uint32_t nthreads = gridDim.x * blockDim.x;
+  const uint32_t vec_per_row = static_cast<uint32_t>(p.row_bytes >> 4);
+  const uint32_t vec_per_e0 = static_cast<uint32_t>(p.e0_row_bytes >> 4);
+  const uint32_t S = static_cast<uint32_t>(p.S);
+  const uint32_t total_g = static_cast<uint32_t>(p.T) * S * vec_per_row;
+  const uint32_t total = total_g + (p.E0_out ? static_cast<uint32_t>(p.T) * vec_per_e0 : 0u);
+  for (uint32_t base = blockIdx.x * blockDim.x + threadIdx.x; base < total; base += nthreads * kGatherUnroll) {
     uint4 v[kGatherUnroll];
-    int64_t dst_off[kGatherUnroll];
+    uint8_t* dst[kGatherUnroll];
 #pragma unroll
     for (int j = 0; j < kGatherUnroll; ++j) {
-      const int64_t vi = base + j * nthreads;
-      dst_off[j] = -1;
-      if (vi < total) {
-        const int64_t row = vi / vec_per_row;
-        const int c = static_cast<int>(vi - row * vec_per_row);
-        const int s = static_cast<int>(row % p.S);
+      const uint32_t vi = base + j * nthreads;
+      dst[j] = nullptr;
+      if (vi < total_g) {
+        uint32_t c;
+        const uint32_t row = split_vec(vi, p.vshift, vec_per_row, c);
+        const uint32_t s = row % S;
         int32_t r = __ldg(p.idx + row);
         if (static_cast<uint32_t>(r) >= p.Vs[s]) {
           set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
           r = 0;
         }
         v[j] = ld_stream_v4(p.E[s] + static_cast<int64_t>(r) * p.row_bytes + c * 16);
-        dst_off[j] = vi * 16;
+        dst[j] = p.G + static_cast<int64_t>(vi) * 16;
+      } else if (vi < total) {
+        const uint32_t e = vi - total_g;
+        uint32_t c;
+        const uint32_t i = split_vec(e, p.eshift, vec_per_e0, c);
+        int32_t t = __ldg(p.tokens + i);
+        if (static_cast<uint32_t>(t) >= p.V0) {
+          set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+          t = 0;
+        }
+        v[j] = ld_stream_v4(p.E0 + static_cast<int64_t>(t) * p.e0_row_bytes + c * 16);
+        dst[j] = p.E0_out + static_cast<int64_t>(e) * 16;
       }
     }
 #pragma unroll
     for (int j = 0; j < kGatherUnroll; ++j)
-      if (dst_off[j] >= 0) *reinterpret_cast<uint4*>(p.G + dst_off[j]) = v[j];
+      if (dst[j]) *reinterpret_cast<uint4*>(dst[j]) = v[j];
   }
 }
 

@@ -149,11 +149,15 @@ int ngram_embed_project(const ngram_embed_plan* plan, const int32_t* tokens,
                         const void* const* E_nk, const void* W_stacked, void* out,
                         void* workspace, size_t workspace_bytes, void* stream);
 
-/* The sub-row lookup of Eq. 3 alone: G_out[i][s*d + c] = E_s[idx[i][s]][c], [T x D]
- * device, plan dtype (the concatenated gathered rows the projection multiplies). */
+/* The table lookups of Eq. 3 alone (the HBM-bound stage of a step, for callers that run
+ * their own projection): G_out[i][s*d + c] = E_s[idx[i][s]][c], [T x D] device, plan dtype
+ * (the concatenated sub-rows the projection multiplies). If E0_out is not NULL, also
+ * E0_out[i] = E_0[tokens[i]] ([T x D], plan dtype); tokens and E0 are then required and
+ * tokens outside [0, V0) read row 0 and set NGRAM_STATUS_BAD_TOKEN. Calls that copy 2^32
+ * 16-byte vectors or more (about 500k tokens at D = 4096) return NGRAM_ERR_UNSUPPORTED. */
 int ngram_embed_gather(const ngram_embed_plan* plan, const int32_t* idx, int64_t num_tokens,
-                       const void* const* E_nk, void* G_out, void* workspace,
-                       size_t workspace_bytes, void* stream);
+                       const void* const* E_nk, void* G_out, const int32_t* tokens, const void* E0,
+                       void* E0_out, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---- N-gram cache (section 4.2) ----
  * slots: [n] int32 device cache slots, distinct within one call (NULL: slot i for entry i).
@@ -243,6 +247,13 @@ int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on);
 
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */
 int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);
+
+/* Depth of the one-CTA tensor-core kernel's ring of gathered A stages (16 KB each); the
+ * rest of its 224 KB of shared memory holds the ring of W tiles and the epilogue's output
+ * tile. Tile width 256: 2, 4 or 6 (W ring 4, 3 or 2 deep); tile width 128: 6, 8 or 10 (W ring
+ * 6, 4 or 2 deep); 0 = default (4 at width 256, 8 at width 128). A tuning knob: results do
+ * not change. */
+int ngram_embed_plan_set_a_stages(ngram_embed_plan* plan, int stages);
 
 /* Schedule of the one-CTA tensor-core kernel: 0 = automatic (stream-K when the grid takes two
  * or more waves of one tile per CTA and the last wave leaves many SMs idle, e.g. 160 tiles of

@@ -222,6 +222,47 @@ def test_gather_api_bit_exact(ne):
     ne.ngram_embed_gather(plan, dev_i32(idx), [to_device(e, torch.bfloat16) for e in Eh], G, ws)
     want = oracle.gather_rows(Eh, idx).reshape(len(tokens), cfg.D)
     np.testing.assert_array_equal(G.view(torch.int16).cpu().numpy().view(np.uint16), want)
+    # with the E_0 rows of the tokens as well; one token out of range reads row 0 and is flagged
+    E0h = gen.table_bf16(cfg.seed, gen.TAG_E0, cfg.V0, cfg.D, cfg.e_std)
+    bad = tokens.copy()
+    bad[7] = cfg.V0 + 3
+    G2 = torch.empty_like(G)
+    R0 = torch.empty((len(tokens), cfg.D), dtype=torch.bfloat16, device="cuda")
+    ne.ngram_embed_gather(plan, dev_i32(idx), [to_device(e, torch.bfloat16) for e in Eh], G2, ws,
+                          tokens=dev_i32(bad), E0=to_device(E0h, torch.bfloat16), E0_out=R0)
+    assert ne.status_names(ne.ngram_embed_get_status(ws)) == ["BAD_TOKEN"]
+    assert torch.equal(G, G2)
+    want0 = E0h[np.where(bad < cfg.V0, bad, 0)]
+    np.testing.assert_array_equal(R0.view(torch.int16).cpu().numpy().view(np.uint16), want0)
+
+
+def test_gather_stage_at_decode_size_sampled(ne):
+    """The gather stage at the spec-decode shape (1280 tokens, 8 sub-tables of 3.3M rows):
+    sampled sub-rows and E_0 rows equal the generator's rows bit for bit."""
+    cfg = configs.SPEC_DECODE
+    ds = workloads.DecodeStream(cfg)
+    T = ds.B * ds.P
+    E0, E, W = device_tables(cfg)
+    tok = ds.step_tokens(3)
+    idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk,
+                              oracle.context_windows(cfg.N, tok, ds.step_offsets()))
+    plan = plan_for(ne, cfg)
+    ws = ne.new_workspace(plan, T)
+    G = torch.empty((T, cfg.D), dtype=torch.bfloat16, device="cuda")
+    R0 = torch.empty((T, cfg.D), dtype=torch.bfloat16, device="cuda")
+    ne.ngram_embed_gather(plan, dev_i32(idx), E, G, ws, tokens=dev_i32(tok), E0=E0, E0_out=R0)
+    assert ne.ngram_embed_get_status(ws) == 0
+    rows = np.unique(np.concatenate([[0, 1, T - 1], np.random.default_rng(2).integers(0, T, 40)]))
+    from tests.helpers import host_rows
+    Gh = G[torch.from_numpy(rows).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)
+    Rh = R0[torch.from_numpy(rows).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)
+    for s in range(cfg.S):
+        np.testing.assert_array_equal(Gh[:, s * cfg.d:(s + 1) * cfg.d],
+                                      host_rows(cfg, gen.TAG_SUBTABLE0 + s, idx[rows, s], cfg.d, cfg.e_std))
+    np.testing.assert_array_equal(Rh, host_rows(cfg, gen.TAG_E0, tok[rows], cfg.D, cfg.e_std))
+    del E0, E, W
+    gc.collect()
+    torch.cuda.empty_cache()
 
 
 def test_project_api_flags_bad_indices(ne):
@@ -377,3 +418,24 @@ def test_pdl_and_graph_replay_match_plain_launches(ne, pair):
         got = run(pdl, graph)
         assert all(torch.equal(a, b) for a, b in zip(ref[0], got[0])), (pdl, graph)
         assert torch.equal(ref[1], got[1]) and torch.equal(ref[2], got[2])
+
+
+@pytest.mark.parametrize("pair,tile_n,stages", [(1, 256, 6), (1, 256, 8), (1, 256, 10), (1, 128, 8), (1, 128, 12),
+                                                (0, 256, 2), (0, 256, 6), (0, 128, 6), (0, 128, 10)])
+@pytest.mark.parametrize("tma_rows", [0, 128])
+def test_ring_depths_agree(ne, pair, tile_n, stages, tma_rows):
+    """Every A/W ring split of both kernel forms feeds the MMAs the same tiles in the same
+    order: bits equal to the default split's."""
+    cfg = small_cfg(5000, 1024, 3, 2, seed=21)
+    tokens, offsets = ragged_tokens(cfg)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = plan_for(ne, cfg, 2, tile_n, pair)
+    ne.ngram_embed_plan_set_tma_rows(plan, tma_rows)
+    ne.ngram_embed_plan_set_stream_k(plan, 2)
+    ref, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    ne.ngram_embed_plan_set_a_stages(plan, stages)
+    got, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0 and torch.equal(ref, got)
