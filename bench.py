@@ -51,6 +51,37 @@ DECODE_WORKLOADS = {
 L2_FLUSH_BYTES = 256 << 20
 
 
+def kernel_source_hash() -> str:
+    """sha256 over the library's CUDA sources: a profile's counters describe the kernels of
+    the sources they were taken from, and only those."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hashed_gram_embedding_horner_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        h.update(os.path.basename(f).encode())
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) recorded in a
+    profiles/*.md summary for this kernel and workload, if it was taken from these sources;
+    else None."""
+    import glob
+    src = kernel_source_hash()
+    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for ln in open(f):
+            if ln.startswith("traffic_record:"):
+                try:
+                    rec = json.loads(ln.split(":", 1)[1])
+                except ValueError:
+                    continue
+                if rec.get("kernel") == kernel and rec.get("workload") == workload and rec.get("source_sha256") == src:
+                    return float(rec["bytes_per_launch"])
+    return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -419,6 +450,9 @@ def main():
     pk = peaks()
     flops = 2.0 * T * cfg.D * cfg.D
     achieved = flops / (proj_ms / 1e3) / 1e12
+    form = ne.ngram_embed_plan_kernel_form(plan, T)
+    kernel_name = {"cta_pair": "proj_sm100_pair_kernel", "one_cta": "proj_sm100_kernel",
+                   "one_cta_stream_k": "proj_sm100_kernel", "cuda_cores": "proj_simt_kernel"}[form]
     algo_bytes = T * (2 * cfg.D * 2 + 4) + cfg.D * cfg.D * 2
 
     # --- end to end through the C ABI with host buffers: H2D inputs, fwd, D2H output
@@ -466,10 +500,10 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_block(cfg, argparse.Namespace(gpus=world)),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / pk["bf16_tflops"], "traffic": None,
-                         "kernel": ("proj_sm100_pair_kernel (CTA pairs, cta_group::2)" if cfg.D <= 2048 else
-                                    "proj_sm100_kernel (one CTA per tile)") +
-                                   ": fused sub-row gather + tcgen05 projection + E_0 add + scale",
+                         "frac": achieved / pk["bf16_tflops"],
+                         "traffic": profiled_traffic(kernel_name, cfg.name),
+                         "kernel": kernel_name + " (" + form + "): fused sub-row gather + tcgen05 projection"
+                                   " + E_0 add + scale",
                          "kernel_ms": proj_ms, "peak_source": pk["source"] + " (burst)",
                          "layer_frac": (flops / (ms_per_step / 1e3) / 1e12) / pk["bf16_tflops"],
                          "hash_kernel_ms": hash_ms,

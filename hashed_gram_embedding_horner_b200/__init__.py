@@ -41,7 +41,7 @@ EXPORTED = [
     "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_plan_set_tma_rows",
     "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws", "ngram_embed_plan_set_cta_pair",
     "ngram_cache_commit", "ngram_embed_plan_set_stream_k", "ngram_embed_plan_set_pdl",
-    "ngram_embed_plan_set_a_stages",
+    "ngram_embed_plan_set_a_stages", "ngram_embed_plan_kernel_form",
 ]
 
 
@@ -81,6 +81,7 @@ _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_a_stages", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_kernel_form", [_P, _I64])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
 _sig("ngram_embed_fwd_static_ws", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P])
 
@@ -166,8 +167,10 @@ def ngram_embed_plan_set_tma_rows(plan: Plan, rows: int):
     _check(_lib.ngram_embed_plan_set_tma_rows(plan.handle, rows), "ngram_embed_plan_set_tma_rows")
 
 
-def ngram_embed_plan_set_cta_pair(plan: Plan, on: bool):
-    _check(_lib.ngram_embed_plan_set_cta_pair(plan.handle, int(bool(on))), "ngram_embed_plan_set_cta_pair")
+def ngram_embed_plan_set_cta_pair(plan: Plan, on):
+    """True/1: CTA pairs; False/0: one CTA per tile; None/-1: automatic (default)."""
+    v = -1 if on is None or on == -1 else int(bool(on))
+    _check(_lib.ngram_embed_plan_set_cta_pair(plan.handle, v), "ngram_embed_plan_set_cta_pair")
 
 
 def ngram_embed_plan_set_stream_k(plan: Plan, mode: int):
@@ -178,6 +181,16 @@ def ngram_embed_plan_set_stream_k(plan: Plan, mode: int):
 def ngram_embed_plan_set_a_stages(plan: Plan, stages: int):
     """Depth of the one-CTA kernel's A ring (0 = default); the W ring takes the rest."""
     _check(_lib.ngram_embed_plan_set_a_stages(plan.handle, int(stages)), "ngram_embed_plan_set_a_stages")
+
+
+KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair"}
+
+
+def ngram_embed_plan_kernel_form(plan: Plan, num_tokens: int) -> str:
+    """Which projection kernel a call of num_tokens tokens runs (with a full-size workspace)."""
+    rc = _lib.ngram_embed_plan_kernel_form(plan.handle, int(num_tokens))
+    _check(min(rc, 0), "ngram_embed_plan_kernel_form")
+    return KERNEL_FORMS[rc]
 
 
 def ngram_embed_plan_set_pdl(plan: Plan, on: bool):

@@ -37,13 +37,14 @@ constexpr size_t kHeadBytes = kStatusBytes + kSkCounterBytes;                   
 // N = 128: 6 + 6, 8 + 4 or 10 + 2.
 constexpr int kDefaultAStages256 = 4;
 constexpr int kDefaultAStages128 = 8;
-// CTA-pair kernel shared memory per CTA: A stages of 16 KB, W stages of BN/2 x 128 B.
-// N = 256: A + W = 6 + 6, 8 + 5 or 10 + 4 stages; N = 128: 8 + 8, 10 + 8 or 12 + 4.
-constexpr int kDefaultPairAStages256 = 8;
-constexpr int kDefaultPairAStages128 = 10;
+// CTA-pair kernel: stages of (16 KB of A + BN/2 x 128 B of W) per CTA, one barrier pair
+// per stage (measured ~2 % faster than separate A and W rings of the same bytes, which
+// double the barrier traffic of the cluster-scope waits and commits; a 7th stage gained
+// nothing).
+constexpr int kPairStages256 = 6;
+constexpr int kPairStages128 = 8;
 
 enum Variant : int { kAuto = 0, kTcTmaRows = 1, kTcSplitRows = 2, kSimt = 3 };
-constexpr int kDefaultTmaRows = 0;  // A rows per tile gathered by TMA; the rest by cp.async (fastest measured)
 
 }  // namespace
 
@@ -57,7 +58,7 @@ struct ngram_embed_plan {
   int device;
   int sms;
   int variant;  // resolved: kTcTmaRows, kTcSplitRows or kSimt
-  int tma_rows; // tensor-core kernel: A rows per tile gathered by TMA (multiple of 32)
+  int tma_rows; // tensor-core kernel: A rows per tile gathered by TMA (multiple of 32; -1 = per form)
   int bn;       // tensor-core tile width (256 or 128)
   bool tc_ok;   // the shape admits the tensor-core kernel
   // tensor-map cache (re-encoded when a table or W pointer changes)
@@ -69,7 +70,7 @@ struct ngram_embed_plan {
   int64_t map_out_T = -1;
   bool smem_attr_set[12] = {};  // per kernel instance (form, tile width, rings), on `device`
   int a_stages = 0;            // one-CTA kernel: A ring depth (0 = default for the tile width)
-  bool cta_pair = true;        // use the CTA-pair (cta_group::2) kernel
+  int cta_pair = -1;           // kernel form: 1 CTA pairs (cta_group::2), 0 one CTA per tile, -1 automatic
   int stream_k = 0;            // one-CTA kernel schedule: 0 automatic, 1 stream-K when possible, 2 never
   bool pdl = false;            // launch as programmatic dependent launches
   int max_clusters[2] = {0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
@@ -106,7 +107,9 @@ size_t sk_partial_bytes(const ngram_embed_plan* p) {
   return p->tc_ok ? size_t(2) * static_cast<size_t>(p->sms) * kBM * 256 * sizeof(float) : 0;
 }
 // Bytes that let every call of up to T tokens take its fastest schedule.
-size_t ws_bytes(const ngram_embed_plan* p, int64_t T) { return ws_base(p, T) + sk_partial_bytes(p); }
+size_t ws_bytes(const ngram_embed_plan* p, int64_t T) {
+  return ws_base(p, T) + sk_partial_bytes(p);
+}
 
 int check_launch() { return cudaGetLastError() == cudaSuccess ? NGRAM_OK : NGRAM_ERR_CUDA; }
 
@@ -231,11 +234,11 @@ int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
 }
 
 // CTA-pair kernel: clusters of two CTAs, one 256 x BN tile per pair per step.
-template <int BN, int AST, int WST>
-int launch_tc_pair_rings(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t st, int key) {
-  using L = PairSmem<BN, AST, WST>;
-  static_assert(L::kLaunchBytes <= 232448, "CTA-pair kernel rings exceed 227 KB of shared memory");
-  auto kern = proj_sm100_pair_kernel<BN, AST, WST>;
+template <int BN, int kStg>
+int launch_tc_pair_stages(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t st, int key) {
+  using L = PairSmem<BN, kStg>;
+  static_assert(L::kLaunchBytes <= 232448, "CTA-pair kernel stages exceed 227 KB of shared memory");
+  auto kern = proj_sm100_pair_kernel<BN, kStg>;
   if (!p->smem_attr_set[key]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
@@ -268,19 +271,10 @@ int launch_tc_pair_rings(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStr
 
 template <int BN>
 int launch_tc_pair(ngram_embed_plan* p, const ProjParams& prm, int64_t T, cudaStream_t st) {
-  if (BN == 256) {
-    switch (p->a_stages ? p->a_stages : kDefaultPairAStages256) {
-      case 6: return launch_tc_pair_rings<256, 6, 6>(p, prm, T, st, 6);
-      case 10: return launch_tc_pair_rings<256, 10, 4>(p, prm, T, st, 8);
-      default: return launch_tc_pair_rings<256, 8, 5>(p, prm, T, st, 7);
-    }
-  }
-  switch (p->a_stages ? p->a_stages : kDefaultPairAStages128) {
-    case 8: return launch_tc_pair_rings<128, 8, 8>(p, prm, T, st, 9);
-    case 12: return launch_tc_pair_rings<128, 12, 4>(p, prm, T, st, 11);
-    default: return launch_tc_pair_rings<128, 10, 8>(p, prm, T, st, 10);
-  }
+  if (BN == 256) return launch_tc_pair_stages<256, kPairStages256>(p, prm, T, st, 7);
+  return launch_tc_pair_stages<128, kPairStages128>(p, prm, T, st, 6);
 }
+
 
 int validate_common(const ngram_embed_plan* p, void* ws, size_t ws_size, int64_t T) {
   if (!p || !ws || T < 0 || T > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
@@ -399,14 +393,17 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   prm.num_k_blocks = p->D / kBK;
   prm.scale = 1.0f / static_cast<float>(p->S + 1);
   prm.status = status_ptr(ws);
-  prm.tma_rows = p->variant == kTcTmaRows ? kBM : p->tma_rows;
-  if (!p->cta_pair && use_stream_k(p, prm, ws_T, ws_size)) {
+  const bool sk = p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
+  const bool pair = p->cta_pair == 1 || (p->cta_pair == -1 && !sk);
+  // A rows by TMA gather4 in the pair form, by cp.async in the one-CTA form (measured
+  // fastest for each), unless the plan fixes the split.
+  prm.tma_rows = p->variant == kTcTmaRows ? kBM : (p->tma_rows >= 0 ? p->tma_rows : (pair ? kBM : 0));
+  if (pair) return p->bn == 256 ? launch_tc_pair<256>(p, prm, T, st) : launch_tc_pair<128>(p, prm, T, st);
+  if (sk) {
     prm.stream_k = 1;
     prm.sk_counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kStatusBytes);
     prm.sk_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_base(p, ws_T));
   }
-  if (p->cta_pair)
-    return p->bn == 256 ? launch_tc_pair<256>(p, prm, T, st) : launch_tc_pair<128>(p, prm, T, st);
   return p->bn == 256 ? launch_tc<256>(p, prm, st) : launch_tc<128>(p, prm, st);
 }
 
@@ -480,10 +477,11 @@ int ngram_embed_plan_create(const ngram_embed_config* cfg, ngram_embed_plan** ou
   p->tc_ok = cfg->dtype == NGRAM_BF16 && S > 0 && cfg->D % 128 == 0 && d % kBK == 0;
   p->bn = cfg->D % 256 == 0 ? 256 : 128;
   p->variant = p->tc_ok ? kTcSplitRows : kSimt;
-  // Defaults from B200 measurements of the two kernel forms: at D = 2048 the CTA pair with
-  // every A row gathered by TMA is fastest; at D = 4096 one CTA per tile with cp.async rows.
-  p->cta_pair = cfg->D <= 2048;
-  p->tma_rows = p->cta_pair ? kBM : kDefaultTmaRows;
+  // Defaults from B200 measurements: the CTA pair with every A row gathered by TMA, except
+  // where the one-CTA form's stream-K schedule applies (grids that end in a thin last wave,
+  // e.g. a 1280-token decode step at D = 4096), with cp.async rows.
+  p->cta_pair = -1;
+  p->tma_rows = -1;
   *out = p;
   return NGRAM_OK;
 }
@@ -509,7 +507,7 @@ int ngram_embed_plan_set_variant(ngram_embed_plan* plan, int variant) {
 // Tensor-core kernel, variant 2: how many of the 128 rows of each A tile TMA gathers
 // (0, 32, 64, 96 or 128); cp.async gathers the rest.
 int ngram_embed_plan_set_tma_rows(ngram_embed_plan* plan, int rows) {
-  if (!plan || rows < 0 || rows > kBM || rows % 32 != 0) return NGRAM_ERR_INVALID_ARG;
+  if (!plan || rows < -1 || rows > kBM || (rows >= 0 && rows % 32 != 0)) return NGRAM_ERR_INVALID_ARG;
   plan->tma_rows = rows;
   return NGRAM_OK;
 }
@@ -517,9 +515,21 @@ int ngram_embed_plan_set_tma_rows(ngram_embed_plan* plan, int rows) {
 // Tensor-core kernel form: 1 = CTA pairs (cta_group::2, 256-token tiles; default),
 // 0 = one CTA per tile (128-token tiles).
 int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on) {
-  if (!plan || (on != 0 && on != 1)) return NGRAM_ERR_INVALID_ARG;
-  plan->cta_pair = on != 0;
+  if (!plan || on < -1 || on > 1) return NGRAM_ERR_INVALID_ARG;
+  plan->cta_pair = on;
   return NGRAM_OK;
+}
+
+int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens) {
+  if (!plan || num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
+  if (plan->variant == kSimt) return 0;
+  ProjParams prm{};
+  prm.num_m_blocks = static_cast<int>((num_tokens + kBM - 1) / kBM);
+  prm.num_n_blocks = plan->D / plan->bn;
+  prm.num_k_blocks = plan->D / kBK;
+  const bool sk = plan->cta_pair != 1 && use_stream_k(plan, prm, num_tokens, ws_bytes(plan, num_tokens));
+  if (plan->cta_pair == 1 || (plan->cta_pair == -1 && !sk)) return 3;
+  return sk ? 2 : 1;
 }
 
 // Tensor-core tile width: 256 or 128 output columns per tile (D must divide).

@@ -31,38 +31,35 @@ namespace ngram {
 
 constexpr int kWarpRelay = 10;
 
-template <int BN, int AST, int WST>
+template <int BN, int STAGES>
 struct PairSmem {
   static constexpr int kABytes = kBM * kBK * 2;         // this CTA's 128 A rows
   static constexpr int kBBytes = (BN / 2) * kBK * 2;    // this CTA's BN/2 rows of W
-  static constexpr int kWOffset = AST * kABytes;        // A ring, then the W ring
-  static constexpr int kBarOffset = kWOffset + WST * kBBytes;
-  static constexpr int kNumBars = 2 * AST + 2 * WST + 5;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kBytes = kBarOffset + kNumBars * 8 + 16;
   static constexpr int kLaunchBytes = kBytes + 1024;
   static constexpr int kTmemCols = 2 * BN;
 };
 
-template <int BN, int AST, int WST>
+template <int BN, int STAGES>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_sm100_pair_kernel(const __grid_constant__ ProjMaps maps, const __grid_constant__ ProjParams p) {
-  using L = PairSmem<BN, AST, WST>;
+  using L = PairSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kBarOffset;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };                   // A ring
-  auto empty_bar = [&](int s) { return bar0 + 8u * (AST + s); };
-  auto wfull_bar = [&](int s) { return bar0 + 8u * (2 * AST + s); };      // W ring
-  auto wempty_bar = [&](int s) { return bar0 + 8u * (2 * AST + WST + s); };
-  constexpr int kT0 = 2 * AST + 2 * WST;
-  auto tfull_bar = [&](int a) { return bar0 + 8u * (kT0 + a); };
-  auto tempty_bar = [&](int a) { return bar0 + 8u * (kT0 + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (kT0 + 4);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + L::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto a_tile = [&](int s) { return sbase + s * L::kABytes; };
-  auto b_tile = [&](int s) { return sbase + L::kWOffset + s * L::kBBytes; };
+  auto a_tile = [&](int s) { return sbase + s * L::kStageBytes; };
+  auto b_tile = [&](int s) { return sbase + s * L::kStageBytes + L::kABytes; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -72,17 +69,13 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
   const bool cp_rows = p.tma_rows == 0;  // A rows by cp.async (else all by TMA gather4)
   if (threadIdx.x == 0) {
-    for (int s = 0; s < AST; ++s) {
-      // CTA 0: its 256 cp.async threads + CTA 1's relay (cp.async mode), or thread 0 posting
-      // the pair's gather4 bytes (TMA mode); CTA 1: its 256 cp.async threads (cp.async mode)
-      const uint32_t arrivals = rank == 0 ? (cp_rows ? static_cast<uint32_t>(kAThreads) + 1u : 1u)
+    for (int s = 0; s < STAGES; ++s) {
+      // CTA 0: thread 0 posts the pair's TMA bytes (+ its 256 cp.async threads + CTA 1's relay);
+      // CTA 1: its 256 cp.async threads (unused in TMA-only mode)
+      const uint32_t arrivals = rank == 0 ? (cp_rows ? 1u + static_cast<uint32_t>(kAThreads) + 1u : 1u)
                                           : static_cast<uint32_t>(kAThreads);
       mbar_init(full_bar(s), arrivals);
       mbar_init(empty_bar(s), 1u);  // one tcgen05.commit from CTA 0's MMA thread
-    }
-    for (int s = 0; s < WST; ++s) {
-      mbar_init(wfull_bar(s), 1u);   // CTA 0: its W producer posts both halves' bytes
-      mbar_init(wempty_bar(s), 1u);  // one tcgen05.commit from CTA 0's MMA thread
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1u);
@@ -117,7 +110,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     const uint32_t swz = static_cast<uint32_t>((chunk ^ (rsub & 7)) << 4);
     const bool issuer = !cp_rows && lane < 4;                       // gather4 mode: 32 lanes x 4 rows
     const int iss = warp * 4 + lane;
-    const uint32_t pair_tx = 2u * L::kABytes;  // TMA mode: both CTAs' gathered rows
+    const uint32_t pair_tx = cp_rows ? 2u * L::kBBytes : 2u * (L::kABytes + L::kBBytes);
     const uint64_t pol = l2_policy_evict_normal();
     // raw row indices (this thread's 4 rows) of the current and the next run
     int32_t raw[4], nraw[4];
@@ -150,7 +143,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const int c0 = (cur.c_first + q) * kBK;
         if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
         const uint32_t a = a_tile(stage);
-        if (!cp_rows && rank == 0 && t == 0) mbar_arrive_expect_tx(full_bar(stage), pair_tx);
+        if (rank == 0 && t == 0) mbar_arrive_expect_tx(full_bar(stage), pair_tx);
         if (cp_rows) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) cp_async_16(a + (rsub + 32 * j) * 128 + swz, src[j] + c0);
@@ -159,7 +152,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           tma_gather4_pair(a + iss * 512, &maps.E[cur.s], c0, r4[0], r4[1], r4[2], r4[3],
                            map_to_cta(full_bar(stage), 0), pol);
         }
-        if (++stage == AST) { stage = 0; phase ^= 1u; }
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       cur = nxt;
 #pragma unroll
@@ -185,11 +178,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         for (int i = 0; i < KB; ++i) {
           int kb = i + rot;
           if (kb >= KB) kb -= KB;
-          if (!mbar_wait_cluster(wempty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          if (rank == 0) mbar_arrive_expect_tx(wfull_bar(stage), 2u * L::kBBytes);
+          if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           tma_load_2d_pair(b_tile(stage), &maps.Whalf, kb * kBK, n_blk * BN + static_cast<int>(rank) * (BN / 2),
-                           map_to_cta(wfull_bar(stage), 0), pol);
-          if (++stage == WST) { stage = 0; phase ^= 1u; }
+                           map_to_cta(full_bar(stage), 0), pol);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
     }
@@ -197,8 +189,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     // ------------------------------------------------------------ MMA issuer (CTA 0)
     if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16(2 * kBM, BN);
-      int stage = 0, wstage = 0;
-      uint32_t phase = 0, wphase = 0;
+      int stage = 0;
+      uint32_t phase = 0;
       bool ok = true;
       int local = 0;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
@@ -208,21 +200,17 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int i = 0; i < KB; ++i) {
-          if (!mbar_wait_cluster(wfull_bar(wstage), wphase, abort_flag, p.status)) { ok = false; break; }
           if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           if (cp_rows) fence_proxy_async_smem();  // this CTA's cp.async rows: generic proxy writes
           const uint64_t adesc = sw128_kmajor_desc(a_tile(stage));
-          const uint64_t bdesc = sw128_kmajor_desc(b_tile(wstage));
+          const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage));
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
             umma_bf16_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
           umma_commit_pair(map_to_cta(empty_bar(stage), 0));
           umma_commit_pair(map_to_cta(empty_bar(stage), 1));
-          umma_commit_pair(map_to_cta(wempty_bar(wstage), 0));
-          umma_commit_pair(map_to_cta(wempty_bar(wstage), 1));
-          if (++stage == AST) { stage = 0; phase ^= 1u; }
-          if (++wstage == WST) { wstage = 0; wphase ^= 1u; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (ok) {
           umma_commit_pair(map_to_cta(tfull_bar(acc), 0));
@@ -234,14 +222,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     }
   } else if (warp == kWarpRelay) {
     // ------------------------------------------------------------ relay (CTA 1, cp.async mode)
-    // Lane l handles A stages l, l + AST, ...: waits for CTA 1's cp.async rows of the stage,
+    // Lane l handles stages l, l + STAGES, ...: waits for CTA 1's cp.async rows of the stage,
     // fences them for the async proxy and arrives on CTA 0's stage barrier.
-    if (cp_rows && rank == 1 && lane < AST) {
+    if (cp_rows && rank == 1 && lane < STAGES) {
       const int my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
       const int total = my_tiles > 0 ? my_tiles * KB : 0;
       const uint32_t remote = map_to_cta(full_bar(lane), 0);
       uint32_t phase = 0;
-      for (int k = lane; k < total; k += AST) {
+      for (int k = lane; k < total; k += STAGES) {
         if (!mbar_wait(full_bar(lane), phase, abort_flag, p.status)) break;
         fence_proxy_async_smem();
         mbar_arrive_remote(remote);

@@ -134,14 +134,6 @@ struct GatherParams {
 // of 1 KiB + one E_0 row of 8 KiB) = 20 MiB) in flight at once.
 constexpr int kGatherUnroll = 8;
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 // Vector index -> (row, vector in row): a shift when the row holds a power of two of
 // vectors (always, for d and D multiples of 8 that are powers of two), else a division.
 __device__ __forceinline__ uint32_t split_vec(uint32_t v, int shift, uint32_t per_row, uint32_t& c) {

@@ -234,25 +234,32 @@ int ngram_embed_plan_uses_tensor_cores(const ngram_embed_plan* plan);
 int ngram_embed_plan_set_variant(ngram_embed_plan* plan, int variant);
 
 /* Variant 2: how many of the 128 rows of each gathered tile TMA brings in (0, 32, 64, 96
- * or 128; default 128 for the pair form, 0 for the one-CTA form); cp.async brings in the
+ * or 128; -1 = default: 128 in the pair form, 0 in the one-CTA form); cp.async brings in the
  * rest. A tuning knob: results do not change. */
 int ngram_embed_plan_set_tma_rows(ngram_embed_plan* plan, int rows);
 
 /* Tensor-core kernel form: 1 = pairs of CTAs on neighbouring SMs share each 256-token tile
  * (tcgen05 cta_group::2; each CTA loads half of the W tile; A rows by cp.async when tma_rows
- * is 0, else all by TMA gather4), 0 = one CTA per 128-token tile. Default: pairs with TMA rows
- * when D <= 2048, else one CTA with cp.async rows. A tuning knob: results agree within the
- * stated tolerance (the k-block order differs). */
+ * is 0, else all by TMA gather4), 0 = one CTA per 128-token tile, -1 (default) = automatic:
+ * the pair form, except where the one-CTA form's stream-K schedule applies (see
+ * ngram_embed_plan_set_stream_k). A tuning knob: results agree within the stated tolerance
+ * (the k-block order differs). */
 int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on);
+
+/* The projection kernel a call of num_tokens tokens would run, given a workspace of
+ * ngram_embed_workspace_bytes(plan, num_tokens): 0 = CUDA cores, 1 = one CTA per tile,
+ * 2 = one CTA per SM with the stream-K schedule, 3 = CTA pairs; negative on bad arguments. */
+int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens);
 
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */
 int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);
 
-/* Depth of the one-CTA tensor-core kernel's ring of gathered A stages (16 KB each); the
- * rest of its 224 KB of shared memory holds the ring of W tiles and the epilogue's output
- * tile. Tile width 256: 2, 4 or 6 (W ring 4, 3 or 2 deep); tile width 128: 6, 8 or 10 (W ring
- * 6, 4 or 2 deep); 0 = default (4 at width 256, 8 at width 128). A tuning knob: results do
- * not change. */
+/* Depth of the one-CTA tensor-core kernel's ring of gathered A stages (16 KB each); the rest
+ * of its 224 KB of shared memory holds the ring of W tiles and the epilogue's output tile.
+ * Tile width 256: 2, 4 or 6 (W ring 4, 3 or 2 deep); width 128: 6, 8 or 10 (W 6, 4 or 2).
+ * Any other even depth up to 12 selects the default (4 at width 256, 8 at 128), as does 0.
+ * The CTA-pair form keeps one ring of combined (A, W) stages. A tuning knob: results do not
+ * change. */
 int ngram_embed_plan_set_a_stages(ngram_embed_plan* plan, int stages);
 
 /* Schedule of the one-CTA tensor-core kernel: 0 = automatic (stream-K when the grid takes two

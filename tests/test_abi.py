@@ -98,6 +98,10 @@ def test_plan_without_device_validates_then_fails_launch(ne):
     assert lib.ngram_embed_plan_set_stream_k(h, 3) == -1 and lib.ngram_embed_plan_set_stream_k(h, 2) == 0
     assert lib.ngram_embed_plan_set_pdl(h, 2) == -1 and lib.ngram_embed_plan_set_pdl(h, 1) == 0
     assert lib.ngram_embed_plan_set_a_stages(h, 5) == -1 and lib.ngram_embed_plan_set_a_stages(h, 6) == 0
+    # no device: the stream-K schedule (it needs the SM count) never applies, so the pair form
+    assert lib.ngram_embed_plan_kernel_form(h, 1280) == 3 and lib.ngram_embed_plan_kernel_form(h, -1) == -1
+    assert lib.ngram_embed_plan_set_cta_pair(h, 0) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 1
+    assert lib.ngram_embed_plan_set_cta_pair(h, -1) == 0 and lib.ngram_embed_plan_set_cta_pair(h, 2) == -1
     assert lib.ngram_embed_plan_uses_tensor_cores(h) == 1
     bad_cache = ne._Cache(0, 0, 0, 4, 8)
     assert lib.ngram_cache_rollback(h, ctypes.byref(bad_cache), None, fake, 3, fake, ws_need, None) == -1

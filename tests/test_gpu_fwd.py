@@ -311,6 +311,7 @@ def test_full_size_prefill_sampled(ne, cfg):
     rows = sample_rows(offsets, T)
     want = oracle_rows(cfg, tokens, offsets, rows, host_W(cfg))
     assert_close(to_host_f64(out[torch.from_numpy(rows).cuda()]), want, what=cfg.name)
+    assert ne.ngram_embed_plan_kernel_form(plan, T) == "cta_pair"
     # other splits of the A rows between TMA and cp.async feed the MMAs the same tiles
     for tr in (64, 128):
         ne.ngram_embed_plan_set_tma_rows(plan, tr)
@@ -325,6 +326,18 @@ def test_full_size_prefill_sampled(ne, cfg):
     del E0, E, W, out, out2, out1
     gc.collect()
     torch.cuda.empty_cache()
+
+
+def test_automatic_kernel_form(ne):
+    """Prefill grids run the CTA-pair form; a 1280-token decode step at D = 4096 (160 tiles of
+    128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule."""
+    for cfg in (configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN):
+        plan = plan_for(ne, cfg)
+        assert ne.ngram_embed_plan_kernel_form(plan, 32768) == "cta_pair"
+    plan = plan_for(ne, configs.SPEC_DECODE)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "one_cta_stream_k"
+    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"  # one wave: nothing to balance
+    assert ne.ngram_embed_plan_kernel_form(plan_for(ne, configs.TINY), 128) == "cuda_cores"
 
 
 def test_spec_decode_forward_through_ring(ne):
@@ -420,11 +433,10 @@ def test_pdl_and_graph_replay_match_plain_launches(ne, pair):
         assert torch.equal(ref[1], got[1]) and torch.equal(ref[2], got[2])
 
 
-@pytest.mark.parametrize("pair,tile_n,stages", [(1, 256, 6), (1, 256, 8), (1, 256, 10), (1, 128, 8), (1, 128, 12),
-                                                (0, 256, 2), (0, 256, 6), (0, 128, 6), (0, 128, 10)])
+@pytest.mark.parametrize("pair,tile_n,stages", [(0, 256, 2), (0, 256, 6), (0, 128, 6), (0, 128, 10)])
 @pytest.mark.parametrize("tma_rows", [0, 128])
 def test_ring_depths_agree(ne, pair, tile_n, stages, tma_rows):
-    """Every A/W ring split of both kernel forms feeds the MMAs the same tiles in the same
+    """Every A/W ring split of the one-CTA kernel feeds the MMAs the same tiles in the same
     order: bits equal to the default split's."""
     cfg = small_cfg(5000, 1024, 3, 2, seed=21)
     tokens, offsets = ragged_tokens(cfg)
@@ -439,3 +451,4 @@ def test_ring_depths_agree(ne, pair, tile_n, stages, tma_rows):
     ne.ngram_embed_plan_set_a_stages(plan, stages)
     got, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
     assert status == 0 and torch.equal(ref, got)
+
