@@ -143,6 +143,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def rank_config(cfg, rank: int):
+    """Rank r's batch under data parallelism: the same shape and tables, its own token
+    stream (rank 0 runs the configured workload)."""
+    return cfg if rank == 0 else cfg.with_(seed=cfg.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's number (device times are reduced with MAX over ranks)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -215,7 +232,7 @@ def config_block(cfg, args):
 
 # ------------------------------------------------------------------ decode (speculative, ring cache)
 
-def run_decode(ne, cfg, steps: int, warmup: int, dev, seed_offset: int = 0):
+def run_decode(ne, cfg, steps: int, warmup: int, dev, rank: int = 0):
     """Speculative decode: per step, every sequence brings 5 ids (x0 + 4 drafts); the layer
     reads each sequence's context from the N-gram cache ring, then the accepted prefix
     (1 + a ids, a ~ U{0..4}) is committed. `steps` steps are captured in one CUDA graph and
@@ -223,8 +240,7 @@ def run_decode(ne, cfg, steps: int, warmup: int, dev, seed_offset: int = 0):
     27 GB of sub-tables do not)."""
     import torch
     from synth.tables import device_tables
-    cfg = cfg.with_(seed=cfg.seed + seed_offset)
-    ds = workloads.DecodeStream(cfg)
+    ds = workloads.DecodeStream(rank_config(cfg, rank))  # this rank's streams; tables shared
     B, P, C = ds.B, ds.P, cfg.ring_capacity
     T = B * P
     E0, E, W = device_tables(cfg)
@@ -373,7 +389,10 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     if args.decode_only:
-        decode = run_decode(ne, DECODE_WORKLOADS[args.decode_workload], args.decode_steps, max(args.warmup, 3), dev, seed_offset=rank)
+        decode = run_decode(ne, DECODE_WORKLOADS[args.decode_workload], args.decode_steps, max(args.warmup, 3), dev,
+                            rank=rank)
+        decode["ms_per_step"] = max_over_ranks(decode["ms_per_step"], world, dev)
+        decode["value"] = world * decode["tokens_per_step"] / (decode["ms_per_step"] / 1e3)
         if rank == 0:
             print(json.dumps({"decode_only": True, "decode": decode}), flush=True)
         if world > 1:
@@ -382,7 +401,7 @@ def main():
         return
 
     # each rank: its own batch of the same shape (seeded per rank), tables identical
-    tokens_h, offsets_h = workloads.prefill_tokens(cfg.with_(seed=cfg.seed) if rank == 0 else cfg.with_(seed=rank))
+    tokens_h, offsets_h = workloads.prefill_tokens(rank_config(cfg, rank))
     T, B = len(tokens_h), len(offsets_h) - 1
     E0, E, W = device_tables(cfg)
     tokens = torch.from_numpy(tokens_h).to(dev)
@@ -421,11 +440,9 @@ def main():
         torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = float(np.sum(step_ms))
+    total_ms = max_over_ranks(total_ms, world, dev)
     if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.barrier()
-        total_ms = float(t.item())
     ms_per_step = total_ms / args.steps
     value = world * T / (ms_per_step / 1e3)
 
@@ -472,21 +489,17 @@ def main():
         ee[i][1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in ee]))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     status = ne.ngram_embed_get_status(ws)
 
     del E0, E, W
     torch.cuda.empty_cache()
     decode = None
     if not args.no_decode:
-        decode = run_decode(ne, DECODE_WORKLOADS[args.decode_workload], args.decode_steps, max(args.warmup, 3), dev, seed_offset=rank)
+        decode = run_decode(ne, DECODE_WORKLOADS[args.decode_workload], args.decode_steps, max(args.warmup, 3), dev,
+                            rank=rank)
         if world > 1:
-            t = torch.tensor([decode["ms_per_step"]], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            decode["ms_per_step"] = float(t.item())
+            decode["ms_per_step"] = max_over_ranks(decode["ms_per_step"], world, dev)
             decode["value"] = world * decode["tokens_per_step"] / (decode["ms_per_step"] / 1e3)
 
     cpu = None
