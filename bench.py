@@ -51,16 +51,19 @@ DECODE_WORKLOADS = {
 L2_FLUSH_BYTES = 256 << 20
 
 
+# the projection kernels' device code, stage counts and tile shapes
+PROJECTION_SOURCES = ("common.cuh", "proj_sm100.cuh", "proj_sm100_pair.cuh")
+
+
 def kernel_source_hash() -> str:
-    """sha256 over the library's CUDA sources: a profile's counters describe the kernels of
-    the sources they were taken from, and only those."""
-    import glob
+    """sha256 over the projection kernels' sources: a profile's counters describe the
+    kernels of the sources they were taken from, and only those."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hashed_gram_embedding_horner_b200", "csrc")
-    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
-        h.update(os.path.basename(f).encode())
-        h.update(open(f, "rb").read())
+    for name in PROJECTION_SOURCES:
+        h.update(name.encode())
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()
 
 

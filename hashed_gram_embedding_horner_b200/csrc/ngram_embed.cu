@@ -32,17 +32,6 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kSkMaxTiles = 2048;                          // stream-K only for grids of at most this many tiles
 constexpr size_t kSkCounterBytes = size_t(kSkMaxTiles) * 4 * sizeof(int32_t);  // one per (tile, row quarter)
 constexpr size_t kHeadBytes = kStatusBytes + kSkCounterBytes;                   // zeroed by clear_status
-// One-CTA kernel shared memory (224 KB): A stages of 16 KB, W stages of BN x 128 B and the
-// epilogue's 128 x BN bf16 tile. N = 256: A + W = 2 + 4, 4 + 3 or 6 + 2 stages;
-// N = 128: 6 + 6, 8 + 4 or 10 + 2.
-constexpr int kDefaultAStages256 = 4;
-constexpr int kDefaultAStages128 = 8;
-// CTA-pair kernel: stages of (16 KB of A + BN/2 x 128 B of W) per CTA, one barrier pair
-// per stage (measured ~2 % faster than separate A and W rings of the same bytes, which
-// double the barrier traffic of the cluster-scope waits and commits; a 7th stage gained
-// nothing).
-constexpr int kPairStages256 = 6;
-constexpr int kPairStages128 = 8;
 
 enum Variant : int { kAuto = 0, kTcTmaRows = 1, kTcSplitRows = 2, kSimt = 3 };
 

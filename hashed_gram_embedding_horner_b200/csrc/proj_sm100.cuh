@@ -78,6 +78,12 @@ struct ProjMaps {
   CUtensorMap Out;          // out [T x D], box {64, 32}, 128-byte swizzle (epilogue TMA stores)
 };
 
+// Shared memory (224 KB): A stages of 16 KB, W stages of BN x 128 B and the epilogue's
+// 128 x BN bf16 tile. N = 256: A + W = 2 + 4, 4 + 3 or 6 + 2 stages; N = 128: 6 + 6, 8 + 4
+// or 10 + 2. Defaults:
+constexpr int kDefaultAStages256 = 4;
+constexpr int kDefaultAStages128 = 8;
+
 template <int BN, int AST, int WST>
 struct ProjSmem {
   static constexpr int kABytes = kBM * kBK * 2;
