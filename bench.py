@@ -493,6 +493,18 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in ee]))
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
+
+    # --- embedding amplification by LayerNorm over the layer output (HBM-bound: the
+    # output read once from HBM, written once), in place, L2 flushed before each launch
+    ln_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ln_ev[i][0].record(stream)
+        ne.ngram_embed_layernorm(plan, out, out, ws, eps=1e-5, stream=stream)
+        ln_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ln_ms = float(np.mean([a.elapsed_time(b) for a, b in ln_ev]))
+    ln_bytes = 2 * out.numel() * out.element_size()
     status = ne.ngram_embed_get_status(ws)
 
     del E0, E, W
@@ -529,6 +541,8 @@ def main():
                     "h2d_bytes_per_step": tokens.numel() * 4 + offsets.numel() * 4,
                     "d2h_bytes_per_step": out.numel() * 2},
             "gpu_launches": 2 * args.steps,
+            "amplification": {"layernorm_ms": ln_ms, "bytes": ln_bytes, "gbs": ln_bytes / (ln_ms / 1e3) / 1e9,
+                              "frac_hbm": ln_bytes / (ln_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
             "decode": decode,
             "clocks": clk.summary(),
             "device_status": status,

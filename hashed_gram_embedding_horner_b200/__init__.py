@@ -42,6 +42,7 @@ EXPORTED = [
     "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws", "ngram_embed_plan_set_cta_pair",
     "ngram_cache_commit", "ngram_embed_plan_set_stream_k", "ngram_embed_plan_set_pdl",
     "ngram_embed_plan_set_a_stages", "ngram_embed_plan_kernel_form",
+    "ngram_embed_plan_set_output_scale", "ngram_embed_layernorm",
 ]
 
 
@@ -82,6 +83,8 @@ _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_a_stages", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_kernel_form", [_P, _I64])
+_sig("ngram_embed_plan_set_output_scale", [_P, ctypes.c_float])
+_sig("ngram_embed_layernorm", [_P, _P, _I64, _P, _P, ctypes.c_float, _P, _P, _SZ, _P])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
 _sig("ngram_embed_fwd_static_ws", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P])
 
@@ -181,6 +184,18 @@ def ngram_embed_plan_set_stream_k(plan: Plan, mode: int):
 def ngram_embed_plan_set_a_stages(plan: Plan, stages: int):
     """Depth of the one-CTA kernel's A ring (0 = default); the W ring takes the rest."""
     _check(_lib.ngram_embed_plan_set_a_stages(plan.handle, int(stages)), "ngram_embed_plan_set_a_stages")
+
+
+def ngram_embed_plan_set_output_scale(plan: Plan, scale: float):
+    """Embedding amplification by a constant, folded into the epilogue (default 1)."""
+    _check(_lib.ngram_embed_plan_set_output_scale(plan.handle, float(scale)), "ngram_embed_plan_set_output_scale")
+
+
+def ngram_embed_layernorm(plan: Plan, x, y, workspace, gamma=None, beta=None, eps: float = 1e-5, stream=None):
+    """Row LayerNorm of a [T, D] layer output (y may be x)."""
+    rc = _lib.ngram_embed_layernorm(plan.handle, _ptr(x), x.shape[0], _ptr(gamma), _ptr(beta), float(eps), _ptr(y),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_embed_layernorm")
 
 
 KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair"}

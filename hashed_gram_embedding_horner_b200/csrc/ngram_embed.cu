@@ -62,6 +62,7 @@ struct ngram_embed_plan {
   int cta_pair = -1;           // kernel form: 1 CTA pairs (cta_group::2), 0 one CTA per tile, -1 automatic
   int stream_k = 0;            // one-CTA kernel schedule: 0 automatic, 1 stream-K when possible, 2 never
   bool pdl = false;            // launch as programmatic dependent launches
+  float out_scale = 1.0f;      // embedding amplification factor folded into the 1/(S+1) scale
   int max_clusters[2] = {0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
 };
 
@@ -339,7 +340,7 @@ int launch_simt(const ngram_embed_plan* p, const int32_t* tokens, const int32_t*
   if (tpb > 8) tpb = 8;
   if (tpb < 1) tpb = 1;
   s.tokens_per_block = tpb;
-  s.scale = 1.0f / static_cast<float>(p->S + 1);
+  s.scale = p->out_scale / static_cast<float>(p->S + 1);
   s.status = status_ptr(ws);
   const size_t smem = static_cast<size_t>(tpb) * p->D * sizeof(float);
   if (smem > 48 * 1024) {
@@ -380,7 +381,7 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   prm.num_m_blocks = static_cast<int>((T + kBM - 1) / kBM);
   prm.num_n_blocks = p->D / p->bn;
   prm.num_k_blocks = p->D / kBK;
-  prm.scale = 1.0f / static_cast<float>(p->S + 1);
+  prm.scale = p->out_scale / static_cast<float>(p->S + 1);
   prm.status = status_ptr(ws);
   const bool sk = p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
   const bool pair = p->cta_pair == 1 || (p->cta_pair == -1 && !sk);
@@ -536,6 +537,39 @@ int ngram_embed_plan_set_a_stages(ngram_embed_plan* plan, int stages) {
   if (!ok) return NGRAM_ERR_INVALID_ARG;
   plan->a_stages = stages;
   return NGRAM_OK;
+}
+
+int ngram_embed_plan_set_output_scale(ngram_embed_plan* plan, float scale) {
+  if (!plan || !(scale == scale) || scale == 0.0f || scale > 3.0e38f || scale < -3.0e38f) return NGRAM_ERR_INVALID_ARG;
+  plan->out_scale = scale;
+  return NGRAM_OK;
+}
+
+int ngram_embed_layernorm(const ngram_embed_plan* plan, const void* x, int64_t num_tokens, const float* gamma,
+                          const float* beta, float eps, void* y, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  int rc = validate_common(plan, workspace, workspace_bytes, 0);
+  if (rc) return rc;
+  if (num_tokens < 0 || num_tokens > INT32_MAX || !(eps >= 0.0f) || eps > 1.0f) return NGRAM_ERR_INVALID_ARG;
+  if (num_tokens == 0) return NGRAM_OK;
+  if (!x || !y) return NGRAM_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return NGRAM_ERR_MISALIGNED;
+  if ((rc = set_device(plan))) return rc;
+  LayerNormParams l{};
+  l.x = x;
+  l.y = y;
+  l.gamma = gamma;
+  l.beta = beta;
+  l.eps = eps;
+  l.T = num_tokens;
+  l.D = plan->D;
+  constexpr int kRowsPerBlock = 8;  // one warp per row
+  const int64_t blocks = (num_tokens + kRowsPerBlock - 1) / kRowsPerBlock;
+  return plan->dtype == NGRAM_F32
+             ? launch(layernorm_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(32 * kRowsPerBlock), 0,
+                      static_cast<cudaStream_t>(stream), plan->pdl, 1, l)
+             : launch(layernorm_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(32 * kRowsPerBlock), 0,
+                      static_cast<cudaStream_t>(stream), plan->pdl, 1, l);
 }
 
 int ngram_embed_plan_set_pdl(ngram_embed_plan* plan, int on) {

@@ -190,6 +190,86 @@ __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ Gat
   }
 }
 
+// ------------------------------------------------------------------ embedding amplification
+// LayerNorm over each output row (section 3.2.4 of "Scaling Embeddings Outperforms
+// Scaling Experts in Language Models": normalising the N-gram embedding output before it
+// joins the residual stream amplifies it early in training). One warp per row; the row
+// is read three times (mean, centred second moment, write), the second and third from
+// L1/L2; fp32 arithmetic; y may alias x.
+
+struct LayerNormParams {
+  const void* x;
+  void* y;
+  const float* gamma;  // [D] or nullptr (1)
+  const float* beta;   // [D] or nullptr (0)
+  float eps;
+  int64_t T;
+  int D;
+};
+
+// 16 bytes of a row: 4 fp32 or 8 bf16 values.
+template <bool F32>
+__device__ __forceinline__ void ln_load(const LayerNormParams& p, int64_t row, int c, float (&v)[F32 ? 4 : 8]) {
+  if constexpr (F32) {
+    const float4 a = reinterpret_cast<const float4*>(static_cast<const float*>(p.x) + row * p.D)[c];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  } else {
+    const uint4 u = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + row * p.D)[c];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      v[2 * h] = __uint_as_float(w[h] << 16);
+      v[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+    }
+  }
+}
+
+template <bool F32>
+__global__ void __launch_bounds__(256) layernorm_kernel(const __grid_constant__ LayerNormParams p) {
+  constexpr int VW = F32 ? 4 : 8;  // values per 16-byte vector
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= p.T) return;
+  const int nv = p.D / VW;  // D * element size is a multiple of 16 for every plan
+  float sum = 0.f;
+  for (int c = lane; c < nv; c += 32) {
+    float v[VW];
+    ln_load<F32>(p, row, c, v);
+#pragma unroll
+    for (int k = 0; k < VW; ++k) sum += v[k];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float mean = sum / static_cast<float>(p.D);
+  float sq = 0.f;
+  for (int c = lane; c < nv; c += 32) {
+    float v[VW];
+    ln_load<F32>(p, row, c, v);
+#pragma unroll
+    for (int k = 0; k < VW; ++k) sq += (v[k] - mean) * (v[k] - mean);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  const float rstd = rsqrtf(sq / static_cast<float>(p.D) + p.eps);
+  for (int c = lane; c < nv; c += 32) {
+    float v[VW];
+    ln_load<F32>(p, row, c, v);
+#pragma unroll
+    for (int k = 0; k < VW; ++k) {
+      const int col = c * VW + k;
+      v[k] = (v[k] - mean) * rstd * (p.gamma ? p.gamma[col] : 1.f) + (p.beta ? p.beta[col] : 0.f);
+    }
+    if constexpr (F32) {
+      reinterpret_cast<float4*>(static_cast<float*>(p.y) + row * p.D)[c] = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+      reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.y) + row * p.D)[c] =
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    }
+  }
+}
+
 // ------------------------------------------------------------------ N-gram cache ring
 
 struct CacheParams {

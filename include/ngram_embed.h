@@ -208,6 +208,25 @@ int ngram_embed_fwd_static_ws(const ngram_embed_plan* plan, const int32_t* token
                               const ngram_cache* cache, const int32_t* cache_slots, void* out,
                               int32_t* status_out, void* stream);
 
+/* ---- embedding amplification (section 3.2.4) ----
+ * The pages amplify the N-gram embedding output early in training, either by a constant
+ * factor or by a LayerNorm before it joins the residual stream (the factor is garbled in
+ * the text: a sqrt(D)-like constant; the caller chooses it).
+ *
+ * Multiply every output of ngram_embed_fwd / ngram_embed_project by `scale` (folded into
+ * the 1/((N-1)K+1) factor of the epilogue: no extra pass). Default 1. Rejects 0 and
+ * non-finite values. */
+int ngram_embed_plan_set_output_scale(ngram_embed_plan* plan, float scale);
+
+/* y[i] = (x[i] - mean(x[i])) / sqrt(var(x[i]) + eps) * gamma + beta over each row of D
+ * values (population variance; fp32 arithmetic; plan dtype in and out).
+ *   x, y   [num_tokens x D] device, 16-byte aligned; y may equal x (in place)
+ *   gamma, beta  [D] fp32 device, or NULL for 1 and 0
+ *   eps    in [0, 1] */
+int ngram_embed_layernorm(const ngram_embed_plan* plan, const void* x, int64_t num_tokens,
+                          const float* gamma, const float* beta, float eps, void* y,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronise `stream` and copy the sticky status word to *status_out. */
 int ngram_embed_get_status(const void* workspace, void* stream, int32_t* status_out);
 /* Zero the workspace head: status word and stream-K counters (asynchronous on `stream`). */

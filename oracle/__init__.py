@@ -206,3 +206,26 @@ class RingOracle:
 
     def histories(self, slots=None):
         return [list(self.hist[b]) for b in (range(len(self.hist)) if slots is None else slots)]
+
+
+# ---------------------------------------------------------------- embedding amplification
+# Section 3.2.4 ("effective training through embedding amplification"): the N-gram
+# embedding output is amplified before it joins the residual stream, by a constant factor
+# or by a LayerNorm. Plain definitions in fp64.
+
+def amplify(e: np.ndarray, scale: float) -> np.ndarray:
+    """Constant amplification: e * scale."""
+    return np.asarray(e, dtype=np.float64) * float(scale)
+
+
+def layernorm(x: np.ndarray, gamma=None, beta=None, eps: float = 0.0) -> np.ndarray:
+    """Row LayerNorm: (x - mean) / sqrt(population variance + eps) * gamma + beta."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    y = (x - mu) / np.sqrt(var + eps)
+    if gamma is not None:
+        y = y * np.asarray(gamma, dtype=np.float64)
+    if beta is not None:
+        y = y + np.asarray(beta, dtype=np.float64)
+    return y

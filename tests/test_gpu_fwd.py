@@ -452,3 +452,55 @@ def test_ring_depths_agree(ne, pair, tile_n, stages, tma_rows):
     got, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
     assert status == 0 and torch.equal(ref, got)
 
+
+
+# ---------------------------------------------------------------- embedding amplification
+
+@pytest.mark.parametrize("pair", [0, 1])
+def test_output_scale_amplifies_the_layer(ne, pair):
+    """A constant amplification (here sqrt(D)) folded into the epilogue equals the oracle's
+    layer output times that constant."""
+    cfg = small_cfg(5000, 1024, 3, 2, seed=41)
+    tokens, offsets = ragged_tokens(cfg)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = plan_for(ne, cfg, pair=pair)
+    amp = float(np.sqrt(cfg.D))
+    ne.ngram_embed_plan_set_output_scale(plan, amp)
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    want = oracle.amplify(oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh), amp)
+    assert_close(to_host_f64(out), want, max_abs=2e-2 * amp, what="amplified")
+
+
+@pytest.mark.parametrize("dtype,D,N,K", [("bf16", 2048, 3, 1), ("bf16", 384, 2, 3), ("fp32", 64, 3, 1),
+                                         ("fp32", 36, 2, 3)])
+def test_layernorm_matches_oracle(ne, dtype, D, N, K):
+    """LayerNorm amplification of a layer output (bf16: the prefill D; an odd width; fp32 tiny
+    widths incl. one not a multiple of 8), in place and out of place, with and without
+    gamma/beta."""
+    rng = np.random.default_rng(7)
+    T = 301
+    S = (N - 1) * K
+    plan = ne.ngram_embed_plan_create(1000, D, N, K, [4099, 5003, 6007][:S], ne.NGRAM_BF16 if dtype == "bf16" else ne.NGRAM_F32)
+    ws = ne.new_workspace(plan, T)
+    x32 = rng.normal(0.01, 0.007, (T, D)).astype(np.float32)
+    if dtype == "bf16":
+        xb = gen.f32_to_bf16_bits(x32)
+        x = to_device(xb, torch.bfloat16)
+        xin = gen.bf16_bits_to_f32(xb)
+        tol = dict(max_abs=2e-2, rel_l2=5e-3)
+    else:
+        x = torch.from_numpy(x32).cuda()
+        xin = x32
+        tol = dict(max_abs=1e-4, rel_l2=1e-5)
+    g = torch.from_numpy(rng.normal(1, 0.1, D).astype(np.float32)).cuda()
+    b = torch.from_numpy(rng.normal(0, 0.1, D).astype(np.float32)).cuda()
+    y = torch.empty_like(x)
+    ne.ngram_embed_layernorm(plan, x, y, ws, gamma=g, beta=b, eps=1e-5)
+    want = oracle.layernorm(xin, g.cpu().numpy(), b.cpu().numpy(), eps=1e-5)
+    assert_close(to_host_f64(y), want, what=f"layernorm {dtype} D{D}", **tol)
+    ne.ngram_embed_layernorm(plan, x, x, ws, eps=1e-5)  # in place, no affine
+    assert_close(to_host_f64(x), oracle.layernorm(xin, eps=1e-5), what="in place", **tol)
+    assert ne.ngram_embed_get_status(ws) == 0

@@ -262,3 +262,35 @@ def test_history_context_equals_prefill_over_full_history():
         full = np.array(hist[b] + step[off[b]:off[b + 1]].tolist(), np.int32)
         pre = oracle.hash_indices(V0, N, K, V, oracle.context_windows(N, full, [0, len(full)]))
         np.testing.assert_array_equal(dec[off[b]:off[b + 1]], pre[len(hist[b]):])
+
+
+# ---------------------------------------------------------------- amplification (section 3.2.4)
+
+def test_layernorm_worked_example():
+    """[1, 2, 3, 4]: mean 2.5, population variance 1.25, so (x - 2.5) / sqrt(1.25)."""
+    got = oracle.layernorm(np.array([[1.0, 2.0, 3.0, 4.0]]))
+    want = np.array([[-1.5, -0.5, 0.5, 1.5]]) / np.sqrt(1.25)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(got, [[-1.3416407864998738, -0.4472135954999579, 0.4472135954999579,
+                                      1.3416407864998738]], rtol=0, atol=1e-15)
+
+
+def test_layernorm_invariants_and_affine():
+    rng = np.random.default_rng(5)
+    x = rng.normal(3.0, 0.02, (7, 96))
+    y = oracle.layernorm(x, eps=1e-12)
+    np.testing.assert_allclose(y.mean(axis=1), 0, atol=1e-12)
+    np.testing.assert_allclose((y ** 2).mean(axis=1), 1, atol=1e-6)
+    # shift and positive scale of a row leave it unchanged; gamma/beta act per column
+    np.testing.assert_allclose(oracle.layernorm(5 * x + 11, eps=0), oracle.layernorm(x, eps=0), atol=1e-10)
+    g, b = rng.normal(size=96), rng.normal(size=96)
+    np.testing.assert_allclose(oracle.layernorm(x, g, b, eps=1e-12), y * g + b, atol=1e-12)
+    # eps bounds the gain of a constant row: output 0, not a division by zero
+    np.testing.assert_array_equal(oracle.layernorm(np.full((1, 8), 2.0), eps=1e-5), np.zeros((1, 8)))
+
+
+def test_amplify_is_a_scalar_on_eq3():
+    rng = np.random.default_rng(6)
+    e = rng.normal(size=(3, 16))
+    np.testing.assert_array_equal(oracle.amplify(e, 1.0), e)
+    np.testing.assert_allclose(oracle.amplify(e, np.sqrt(16.0)), 4.0 * e, rtol=1e-15)
