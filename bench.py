@@ -366,6 +366,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-decode", action="store_true", help="skip the speculative-decode measurement")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward (training) measurement")
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--decode-workload", default="spec_decode", choices=sorted(DECODE_WORKLOADS))
     ap.add_argument("--decode-only", action="store_true",
@@ -507,6 +508,35 @@ def main():
     ln_bytes = 2 * out.numel() * out.element_size()
     status = ne.ngram_embed_get_status(ws)
 
+    # --- backward (training): parameter gradients for a random bf16 dL/de, fp32 gradient
+    # tables accumulated in place; two tcgen05 GEMMs of 2 T D^2 FLOPs each dominate
+    backward = None
+    if not args.no_backward:
+        g_out = (torch.randn((T, cfg.D), device=dev) * 0.01).to(torch.bfloat16)
+        dE0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.float32, device=dev)
+        dE = [torch.zeros((v, cfg.d), dtype=torch.float32, device=dev) for v in cfg.V_nk]
+        dW = torch.zeros((cfg.D, cfg.D), dtype=torch.float32, device=dev)
+        bws = ne.new_bwd_workspace(plan, T, device=dev)
+        bwd = lambda: ne.ngram_embed_bwd(plan, tokens, idx, g_out, bws, E_nk=E, W_stacked=W, dE0=dE0, dE_nk=dE,
+                                         dW=dW, stream=stream)
+        for _ in range(2):
+            bwd()
+        torch.cuda.synchronize()
+        bw_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(max(3, args.steps // 4))]
+        for i, (e0, e1) in enumerate(bw_ev):
+            flush.fill_(i & 0xFF)
+            e0.record(stream)
+            bwd()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        bw_ms = float(np.mean([a.elapsed_time(b) for a, b in bw_ev]))
+        bw_flops = 4.0 * T * cfg.D * cfg.D
+        backward = {"ms": bw_ms, "tokens_per_s": T / (bw_ms / 1e3), "tflops": bw_flops / (bw_ms / 1e3) / 1e12,
+                    "frac": bw_flops / (bw_ms / 1e3) / 1e12 / pk["bf16_tflops"],
+                    "device_status": ne.ngram_embed_get_status(bws)}
+        del g_out, dE0, dE, dW, bws
+
     del E0, E, W
     torch.cuda.empty_cache()
     decode = None
@@ -541,6 +571,7 @@ def main():
                     "h2d_bytes_per_step": tokens.numel() * 4 + offsets.numel() * 4,
                     "d2h_bytes_per_step": out.numel() * 2},
             "gpu_launches": 2 * args.steps,
+            "backward": backward,
             "amplification": {"layernorm_ms": ln_ms, "bytes": ln_bytes, "gbs": ln_bytes / (ln_ms / 1e3) / 1e9,
                               "frac_hbm": ln_bytes / (ln_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
             "decode": decode,

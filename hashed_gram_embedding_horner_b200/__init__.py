@@ -43,6 +43,7 @@ EXPORTED = [
     "ngram_cache_commit", "ngram_embed_plan_set_stream_k", "ngram_embed_plan_set_pdl",
     "ngram_embed_plan_set_a_stages", "ngram_embed_plan_kernel_form",
     "ngram_embed_plan_set_output_scale", "ngram_embed_layernorm",
+    "ngram_embed_bwd_workspace_bytes", "ngram_embed_bwd",
 ]
 
 
@@ -84,6 +85,8 @@ _sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_a_stages", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_kernel_form", [_P, _I64])
 _sig("ngram_embed_plan_set_output_scale", [_P, ctypes.c_float])
+_sig("ngram_embed_bwd_workspace_bytes", [_P, _I64], _SZ)
+_sig("ngram_embed_bwd", [_P, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P])
 _sig("ngram_embed_layernorm", [_P, _P, _I64, _P, _P, ctypes.c_float, _P, _P, _SZ, _P])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
 _sig("ngram_embed_fwd_static_ws", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P])
@@ -196,6 +199,25 @@ def ngram_embed_layernorm(plan: Plan, x, y, workspace, gamma=None, beta=None, ep
     rc = _lib.ngram_embed_layernorm(plan.handle, _ptr(x), x.shape[0], _ptr(gamma), _ptr(beta), float(eps), _ptr(y),
                                     _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "ngram_embed_layernorm")
+
+
+def new_bwd_workspace(plan: Plan, max_tokens: int, device="cuda"):
+    """A zeroed uint8 workspace tensor of ngram_embed_bwd_workspace_bytes(plan, max_tokens)."""
+    import torch
+    return torch.zeros(_lib.ngram_embed_bwd_workspace_bytes(plan.handle, int(max_tokens)), dtype=torch.uint8,
+                       device=device)
+
+
+def ngram_embed_bwd(plan: Plan, tokens, idx, grad_out, workspace, E_nk=None, W_stacked=None, dE0=None, dE_nk=None,
+                    dW=None, stream=None):
+    """Accumulate the layer's parameter gradients (fp32 tensors, += semantics) from
+    grad_out = dL/de and the forward's indices. Pass None to skip a gradient."""
+    tabs = _tables(E_nk) if E_nk is not None else None
+    grads = (ctypes.c_void_p * len(dE_nk))(*[t.data_ptr() for t in dE_nk]) if dE_nk is not None else None
+    rc = _lib.ngram_embed_bwd(plan.handle, _i32(tokens, "tokens"), _i32(idx, "idx"), tokens.numel(), tabs,
+                              _ptr(W_stacked), _ptr(grad_out), _ptr(dE0), grads, _ptr(dW), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_embed_bwd")
 
 
 KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair"}

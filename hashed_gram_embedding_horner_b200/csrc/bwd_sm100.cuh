@@ -1,0 +1,342 @@
+// Backward of the N-gram embedding layer (Eq. 3 of "Scaling Embeddings Outperforms Scaling
+// Experts in Language Models", section 2), for training from scratch (section 6).
+//
+// With c = (output scale) / ((N-1)K + 1) and g = dL/de [T x D]:
+//   dE_0[t_i]              += c g_i                                   (scatter over tokens)
+//   dG                      = c g W_stacked                 [T x D]   (tcgen05 GEMM, K = D)
+//   dE_s[idx_s(i)][j]      += dG[i][s d + j]                          (scatter, fused in the
+//                                                                      GEMM's epilogue)
+//   dW_stacked             += c g^T G,  G[i][s d + j] = E_s[idx_s(i)][j]   (tcgen05 GEMM, K = T)
+// Colliding rows (several tokens, one table row) add up: every scatter is an fp32 atomic
+// add, so the summation order (not the set of terms) varies between runs.
+//
+// Both GEMMs run on one kernel, `dense_gemm_sm100_kernel`: A [M x K] and B [N x K], both
+// K-major bf16 tiles brought in by 2-D TMA (the operands that are not K-major in memory —
+// W for dG, g and G for dW — are first transposed into the workspace), fp32 accumulators
+// in TMEM, work units of (128 x BN tile, k range) handed out round-robin to persistent
+// CTAs (split-K where tiles are few), and an epilogue that atomically adds the scaled
+// partial tile into its destination: sub-table gradient rows (dG) or dW.
+#pragma once
+
+#include "proj_sm100.cuh"
+
+namespace ngram {
+
+// ------------------------------------------------------------------ transposes
+
+// dst[c][r] = src[r][c] for r < R, and 0 for R <= r < R_pad (dst rows are R_pad long, a
+// multiple of 8 so the rows of dst stay 16-byte aligned for TMA). bf16, 32 x 32 tiles.
+struct TransposeParams {
+  const uint16_t* src;
+  uint16_t* dst;
+  int64_t R, R_pad;
+  int C;
+};
+
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __grid_constant__ TransposeParams p) {
+  __shared__ uint16_t tile[32][33];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int c0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t r = r0 + ty + 8 * k;
+    const int c = c0 + tx;
+    tile[ty + 8 * k][tx] = (r < p.R && c < p.C) ? p.src[r * p.C + c] : uint16_t(0);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int c = c0 + ty + 8 * k;
+    const int64_t r = r0 + tx;
+    if (c < p.C && r < p.R_pad) p.dst[static_cast<int64_t>(c) * p.R_pad + r] = tile[tx][ty + 8 * k];
+  }
+}
+
+// GT[c][i] = G[i][c] = E_s[idx[i][s]][c - s d] (s = c / d) for i < T, 0 for T <= i < T_pad.
+struct GatherTParams {
+  const int32_t* idx;
+  const uint16_t* E[kMaxS];
+  uint32_t Vs[kMaxS];
+  uint16_t* dst;
+  int64_t T, T_pad;
+  int S, d, D;
+  int* status;
+};
+
+__global__ void __launch_bounds__(256) gather_transpose_kernel(const __grid_constant__ GatherTParams p) {
+  __shared__ uint16_t tile[32][33];
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int c0 = blockIdx.y * 32;  // 32 columns never straddle two sub-tables (d % 64 == 0)
+  const int s = c0 / p.d;
+  const int j0 = c0 - s * p.d;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t i = i0 + ty + 8 * k;
+    uint16_t v = 0;
+    if (i < p.T) {
+      int32_t r = p.idx[i * p.S + s];
+      if (static_cast<uint32_t>(r) >= p.Vs[s]) {
+        if (tx == 0) set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+        r = 0;
+      }
+      v = p.E[s][static_cast<int64_t>(r) * p.d + j0 + tx];
+    }
+    tile[ty + 8 * k][tx] = v;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int c = c0 + ty + 8 * k;
+    const int64_t i = i0 + tx;
+    if (i < p.T_pad) p.dst[static_cast<int64_t>(c) * p.T_pad + i] = tile[tx][ty + 8 * k];
+  }
+}
+
+// ------------------------------------------------------------------ dE_0 scatter
+
+struct ScatterE0Params {
+  const int32_t* tokens;
+  const uint16_t* g;  // [T x D] bf16
+  float* dE0;         // [V0 x D] fp32
+  int64_t T;
+  int D;
+  uint32_t V0;
+  float scale;
+  int* status;
+};
+
+// One warp per token: dE0[t_i] += scale * g_i, 16-byte vector atomics.
+__global__ void __launch_bounds__(256) scatter_e0_kernel(const __grid_constant__ ScatterE0Params p) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= p.T) return;
+  int32_t t = p.tokens[i];
+  if (static_cast<uint32_t>(t) >= p.V0) {
+    if (lane == 0) set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+    t = 0;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(p.g + i * p.D);
+  float4* dst = reinterpret_cast<float4*>(p.dE0 + static_cast<int64_t>(t) * p.D);
+  for (int v = lane; v < (p.D >> 3); v += 32) {
+    const uint4 u = src[v];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float f[8];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      f[2 * h] = bf16_bits_to_float(w[h] & 0xFFFFu) * p.scale;
+      f[2 * h + 1] = bf16_bits_to_float(w[h] >> 16) * p.scale;
+    }
+    atomicAdd(dst + 2 * v, make_float4(f[0], f[1], f[2], f[3]));
+    atomicAdd(dst + 2 * v + 1, make_float4(f[4], f[5], f[6], f[7]));
+  }
+}
+
+// ------------------------------------------------------------------ dense tcgen05 GEMM
+
+enum GemmEpi : int { kEpiScatterSub = 0, kEpiAccumDense = 1 };
+
+struct DenseMaps {
+  CUtensorMap A;  // [M x K] bf16, K-major, box {64, 128}, 128-byte swizzle
+  CUtensorMap B;  // [N x K] bf16, K-major, box {64, BN}, 128-byte swizzle
+};
+
+struct DenseParams {
+  int M, N;            // rows of A (tokens, or D) and of B (D)
+  int num_m_blocks, num_n_blocks, num_k_blocks;
+  int splits;          // k ranges per tile (split-K): unit u = tile * splits + k range
+  int kb_per_split;
+  float scale;
+  int epi;             // GemmEpi
+  // kEpiScatterSub: row i of the tile -> dE_s[idx[i][s]][c - s d] for column c (s = c / d)
+  const int32_t* idx;
+  float* dE[kMaxS];
+  uint32_t Vs[kMaxS];
+  int S, d;
+  // kEpiAccumDense: out[row][col] (row stride N)
+  float* out;
+  int* status;
+};
+
+constexpr int kGemmThreads = 256;  // warp 0: TMA producer, warp 1: MMA + TMEM, warps 4-7: epilogue
+
+template <int BN, int STAGES>
+struct DenseSmem {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kBytes = kBarOffset + kNumBars * 8 + 16;
+  static constexpr int kLaunchBytes = kBytes + 1024;
+  static constexpr int kTmemCols = 2 * BN;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    dense_gemm_sm100_kernel(const __grid_constant__ DenseMaps maps, const __grid_constant__ DenseParams p) {
+  using L = DenseSmem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBarOffset;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + L::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto a_tile = [&](int s) { return sbase + s * L::kStageBytes; };
+  auto b_tile = [&](int s) { return sbase + s * L::kStageBytes + L::kABytes; };
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1u);   // the producer's byte count
+      mbar_init(empty_bar(s), 1u);  // one tcgen05.commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1u);
+      mbar_init(tempty_bar(a), 128u);
+    }
+    mbar_init(drain_bar, 1u);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.A);
+    tma_prefetch_desc(&maps.B);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
+
+  const int num_units = p.num_m_blocks * p.num_n_blocks * p.splits;
+  auto unit_k = [&](int u, int& kb0, int& kb1) {
+    const int ks = u % p.splits;
+    kb0 = ks * p.kb_per_split;
+    kb1 = kb0 + p.kb_per_split < p.num_k_blocks ? kb0 + p.kb_per_split : p.num_k_blocks;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (A and B)
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const int tile = u / p.splits;
+        const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
+        int kb0, kb1;
+        unit_k(u, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_bar(stage), L::kStageBytes);
+          tma_load_2d(a_tile(stage), &maps.A, kb * kBK, m_blk * kBM, full_bar(stage), pol);
+          tma_load_2d(b_tile(stage), &maps.B, kb * kBK, n_blk * BN, full_bar(stage), pol);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!mbar_wait(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        int kb0, kb1;
+        unit_k(u, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = sw128_kmajor_desc(a_tile(stage));
+          const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb > kb0 || k != 0) ? 1u : 0u);
+          umma_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) umma_commit(tfull_bar(acc));
+      }
+      umma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0, 100ull * 1000 * 1000);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue: atomic adds
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    int local = 0;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++local) {
+      const int tile = u / p.splits;
+      const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
+      const int acc = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const int64_t row = static_cast<int64_t>(m_blk) * kBM + row_in_tile;
+      const bool valid = row < p.M;
+      bool got = false;
+      if (lane == 0) got = mbar_wait(tfull_bar(acc), use & 1u, abort_flag, p.status);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, v);
+        tmem_wait_ld();
+        if (c + 1 == BN / 32) {
+          tc_fence_before();
+          mbar_arrive(tempty_bar(acc));
+        }
+        if (!valid) continue;
+        const int col0 = n_blk * BN + c * 32;
+        float4* dst;
+        if (p.epi == kEpiScatterSub) {
+          const int s = col0 / p.d;  // 32 columns never straddle two sub-tables
+          int32_t r = p.idx[row * p.S + s];
+          if (static_cast<uint32_t>(r) >= p.Vs[s]) {
+            set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+            r = 0;
+          }
+          dst = reinterpret_cast<float4*>(p.dE[s] + static_cast<int64_t>(r) * p.d + (col0 - s * p.d));
+        } else {
+          dst = reinterpret_cast<float4*>(p.out + row * p.N + col0);
+        }
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+          atomicAdd(dst + w, make_float4(__uint_as_float(v[4 * w]) * p.scale, __uint_as_float(v[4 * w + 1]) * p.scale,
+                                         __uint_as_float(v[4 * w + 2]) * p.scale,
+                                         __uint_as_float(v[4 * w + 3]) * p.scale));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace ngram

@@ -334,9 +334,6 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
 }
 
-// Self-test of the bounded wait: one warp waits on an mbarrier that nothing ever
-// arrives at; mbar_wait must give up after limit_ns, raise NGRAM_STATUS_TIMEOUT
-// and let the kernel return normally.
 // 2-D TMA store of a shared-memory box (bulk-group completion). x (innermost) in elements.
 __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int32_t x, int32_t y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
@@ -375,6 +372,9 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Self-test of the bounded wait: one warp waits on an mbarrier that nothing ever
+// arrives at; mbar_wait must give up after limit_ns, raise NGRAM_STATUS_TIMEOUT
+// and let the kernel return normally.
 __global__ void selftest_wait_kernel(int* status, uint64_t limit_ns) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;

@@ -22,6 +22,7 @@
 #include "proj_sm100.cuh"
 #include "proj_sm100_pair.cuh"
 #include "simt.cuh"
+#include "bwd_sm100.cuh"
 
 using namespace ngram;
 
@@ -265,6 +266,70 @@ int launch_tc_pair(ngram_embed_plan* p, const ProjParams& prm, int64_t T, cudaSt
   return launch_tc_pair_stages<128, kPairStages128>(p, prm, T, st, 6);
 }
 
+
+// ---- backward -------------------------------------------------------------------------
+// Workspace: the head (status word, ...), then W^T [D x D], g^T [D x T8] and G^T [D x T8]
+// bf16 (T8 = T rounded up to 8, zero-filled), each 256-byte aligned.
+constexpr int kBwdStages = 4;  // x (16 KB A + BN x 128 B B)
+
+int64_t pad8(int64_t T) { return (T + 7) & ~int64_t(7); }
+size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+size_t bwd_ws_bytes(const ngram_embed_plan* p, int64_t T) {
+  const size_t D = static_cast<size_t>(p->D);
+  return kHeadBytes + round256(D * D * 2) + 2 * round256(D * static_cast<size_t>(pad8(T)) * 2);
+}
+
+// Split-K factor for a GEMM of `tiles` output tiles and KB k-blocks: the one, up to KB / 16
+// k-blocks per unit, whose units best fill whole waves of the SMs (ties: fewer splits).
+int choose_splits(int tiles, int KB, int sms) {
+  int best = 1;
+  double best_fill = -1.0;
+  const int max_s = KB / 16 > 1 ? (KB / 16 < 64 ? KB / 16 : 64) : 1;
+  for (int s = 1; s <= max_s; ++s) {
+    const int kbps = (KB + s - 1) / s;
+    const int units = tiles * ((KB + kbps - 1) / kbps);
+    const int waves = (units + sms - 1) / sms;
+    const double fill = static_cast<double>(units) / (static_cast<double>(waves) * sms);
+    if (fill > best_fill + 0.01) {
+      best_fill = fill;
+      best = s;
+    }
+  }
+  return best;
+}
+
+template <int BN>
+int launch_dense_gemm(ngram_embed_plan* p, DenseParams prm, const void* A, int64_t a_rows, const void* B,
+                      int64_t b_rows, int64_t K, int64_t row_elems, bool split, cudaStream_t st) {
+  using L = DenseSmem<BN, kBwdStages>;
+  auto kern = dense_gemm_sm100_kernel<BN, kBwdStages>;
+  const int key = BN == 256 ? 10 : 11;
+  if (!p->smem_attr_set[key]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess)
+      return NGRAM_ERR_CUDA;
+    p->smem_attr_set[key] = true;
+  }
+  DenseMaps maps;
+  int rc = encode_2d(&maps.A, A, static_cast<uint64_t>(row_elems), static_cast<uint64_t>(a_rows),
+                     static_cast<uint64_t>(row_elems) * 2, kBK, kBM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (rc) return rc;
+  rc = encode_2d(&maps.B, B, static_cast<uint64_t>(row_elems), static_cast<uint64_t>(b_rows),
+                 static_cast<uint64_t>(row_elems) * 2, kBK, BN, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (rc) return rc;
+  prm.M = static_cast<int>(a_rows);
+  prm.N = static_cast<int>(b_rows);
+  prm.num_m_blocks = static_cast<int>((a_rows + kBM - 1) / kBM);
+  prm.num_n_blocks = static_cast<int>(b_rows / BN);
+  prm.num_k_blocks = static_cast<int>((K + kBK - 1) / kBK);
+  const int tiles = prm.num_m_blocks * prm.num_n_blocks;
+  const int sms = p->sms > 0 ? p->sms : 1;
+  const int s = split ? choose_splits(tiles, prm.num_k_blocks, sms) : 1;
+  prm.kb_per_split = (prm.num_k_blocks + s - 1) / s;
+  prm.splits = (prm.num_k_blocks + prm.kb_per_split - 1) / prm.kb_per_split;  // every split non-empty
+  const int units = tiles * prm.splits;
+  const int grid = units < sms ? units : sms;
+  return launch(kern, dim3(grid), dim3(kGemmThreads), L::kLaunchBytes, st, p->pdl, 1, maps, prm);
+}
 
 int validate_common(const ngram_embed_plan* p, void* ws, size_t ws_size, int64_t T) {
   if (!p || !ws || T < 0 || T > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
@@ -542,6 +607,119 @@ int ngram_embed_plan_set_a_stages(ngram_embed_plan* plan, int stages) {
 int ngram_embed_plan_set_output_scale(ngram_embed_plan* plan, float scale) {
   if (!plan || !(scale == scale) || scale == 0.0f || scale > 3.0e38f || scale < -3.0e38f) return NGRAM_ERR_INVALID_ARG;
   plan->out_scale = scale;
+  return NGRAM_OK;
+}
+
+size_t ngram_embed_bwd_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens) {
+  if (!plan || max_tokens < 0) return 0;
+  return bwd_ws_bytes(plan, max_tokens);
+}
+
+int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const int32_t* idx, int64_t num_tokens,
+                    const void* const* E_nk, const void* W_stacked, const void* grad_out, float* dE0,
+                    float* const* dE_nk, float* dW, void* workspace, size_t workspace_bytes, void* stream) {
+  auto* p = const_cast<ngram_embed_plan*>(plan_c);
+  if (!p || !workspace || num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
+  if (!p->tc_ok) return NGRAM_ERR_UNSUPPORTED;  // bf16 tensor-core shapes only
+  if (!aligned16(workspace)) return NGRAM_ERR_MISALIGNED;
+  if (workspace_bytes < bwd_ws_bytes(p, num_tokens)) return NGRAM_ERR_WORKSPACE;
+  if (num_tokens == 0 || (!dE0 && !dE_nk && !dW)) return NGRAM_OK;
+  if (!tokens || !idx || !grad_out || (dE_nk && !W_stacked) || (dW && !E_nk))
+    return NGRAM_ERR_INVALID_ARG;
+  if (!aligned16(grad_out) || (dE0 && !aligned16(dE0)) || (dW && !aligned16(dW)) ||
+      (W_stacked && !aligned16(W_stacked)))
+    return NGRAM_ERR_MISALIGNED;
+  for (int s = 0; s < p->S; ++s) {
+    if (dE_nk && (!dE_nk[s] || !aligned16(dE_nk[s]))) return dE_nk[s] ? NGRAM_ERR_MISALIGNED : NGRAM_ERR_INVALID_ARG;
+    if (dW && (!E_nk[s] || !aligned16(E_nk[s]))) return E_nk[s] ? NGRAM_ERR_MISALIGNED : NGRAM_ERR_INVALID_ARG;
+  }
+  int rc = set_device(p);
+  if (rc) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t T = num_tokens, T8 = pad8(T);
+  const int D = p->D;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint16_t* Wt = reinterpret_cast<uint16_t*>(base + kHeadBytes);
+  uint16_t* gT = reinterpret_cast<uint16_t*>(base + kHeadBytes + round256(size_t(D) * D * 2));
+  uint16_t* GT = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(gT) + round256(size_t(D) * T8 * 2));
+  const float scale = p->out_scale / static_cast<float>(p->S + 1);
+  const auto* g = static_cast<const uint16_t*>(grad_out);
+
+  if (dE0) {
+    ScatterE0Params e{};
+    e.tokens = tokens;
+    e.g = g;
+    e.dE0 = dE0;
+    e.T = T;
+    e.D = D;
+    e.V0 = static_cast<uint32_t>(p->V0);
+    e.scale = scale;
+    e.status = status_ptr(workspace);
+    if ((rc = launch(scatter_e0_kernel, dim3(static_cast<unsigned>((T + 7) / 8)), dim3(256), 0, st, p->pdl, 1, e)))
+      return rc;
+  }
+  if (dE_nk) {
+    // dG = c g W_stacked, i.e. A = g [T x D] and B = W^T [D x D] (both K-major over D);
+    // the epilogue adds each 32-column piece into its sub-table's gradient row.
+    TransposeParams tp{};
+    tp.src = static_cast<const uint16_t*>(W_stacked);
+    tp.dst = Wt;
+    tp.R = D;
+    tp.R_pad = D;
+    tp.C = D;
+    if ((rc = launch(transpose_bf16_kernel, dim3(D / 32, D / 32), dim3(256), 0, st, p->pdl, 1, tp))) return rc;
+    DenseParams dp{};
+    dp.scale = scale;
+    dp.epi = kEpiScatterSub;
+    dp.idx = idx;
+    for (int s = 0; s < p->S; ++s) {
+      dp.dE[s] = dE_nk[s];
+      dp.Vs[s] = static_cast<uint32_t>(p->V[s]);
+    }
+    dp.S = p->S;
+    dp.d = p->d;
+    dp.status = status_ptr(workspace);
+    if ((rc = p->D % 256 == 0 ? launch_dense_gemm<256>(p, dp, g, T, Wt, D, D, D, false, st)
+                              : launch_dense_gemm<128>(p, dp, g, T, Wt, D, D, D, false, st)))
+      return rc;
+  }
+  if (dW) {
+    // dW += c g^T G: A = g^T [D x T8] and B = G^T [D x T8] (K-major over tokens), split-K
+    // units adding into dW.
+    TransposeParams tp{};
+    tp.src = g;
+    tp.dst = gT;
+    tp.R = T;
+    tp.R_pad = T8;
+    tp.C = D;
+    if ((rc = launch(transpose_bf16_kernel, dim3(static_cast<unsigned>((T8 + 31) / 32), D / 32), dim3(256), 0, st,
+                     p->pdl, 1, tp)))
+      return rc;
+    GatherTParams gp{};
+    gp.idx = idx;
+    for (int s = 0; s < p->S; ++s) {
+      gp.E[s] = static_cast<const uint16_t*>(E_nk[s]);
+      gp.Vs[s] = static_cast<uint32_t>(p->V[s]);
+    }
+    gp.dst = GT;
+    gp.T = T;
+    gp.T_pad = T8;
+    gp.S = p->S;
+    gp.d = p->d;
+    gp.D = D;
+    gp.status = status_ptr(workspace);
+    if ((rc = launch(gather_transpose_kernel, dim3(static_cast<unsigned>((T8 + 31) / 32), D / 32), dim3(256), 0, st,
+                     p->pdl, 1, gp)))
+      return rc;
+    DenseParams dp{};
+    dp.scale = scale;
+    dp.epi = kEpiAccumDense;
+    dp.out = dW;
+    dp.status = status_ptr(workspace);
+    if ((rc = p->D % 256 == 0 ? launch_dense_gemm<256>(p, dp, gT, D, GT, D, T8, T8, true, st)
+                              : launch_dense_gemm<128>(p, dp, gT, D, GT, D, T8, T8, true, st)))
+      return rc;
+  }
   return NGRAM_OK;
 }
 

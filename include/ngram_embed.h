@@ -208,6 +208,26 @@ int ngram_embed_fwd_static_ws(const ngram_embed_plan* plan, const int32_t* token
                               const ngram_cache* cache, const int32_t* cache_slots, void* out,
                               int32_t* status_out, void* stream);
 
+/* ---- backward (training; the pages train the layer from scratch, section 6) ----
+ * Gradients of Eq. 3 given g = dL/de (bf16 [num_tokens x D]) and the forward's indices
+ * (idx from ngram_hash_indices, [num_tokens x S]); c = output scale / ((N-1)K+1):
+ *   dE0[t_i]            += c g_i
+ *   dE_nk[s][idx[i][s]] += (c g W_stacked)[i][s d .. s d + d)     (rows that collide add up)
+ *   dW                  += c g^T G,  G[i] = the concatenated sub-rows of token i
+ * All gradients are fp32 device arrays of their parameter's shape (dE0 [V0 x D], dE_nk[s]
+ * [V_nk[s] x d], dW [D x D]), accumulated with atomic adds (the summation order varies
+ * between runs; the terms do not). Any of dE0, dE_nk (HOST array of S device pointers) and
+ * dW may be NULL to skip that gradient; W_stacked is needed for dE_nk, E_nk for dW.
+ * bf16 tensor-core plans only (else NGRAM_ERR_UNSUPPORTED). Index values outside
+ * [0, V_nk) read/write row 0 and set NGRAM_STATUS_BAD_TOKEN.
+ *   workspace  >= ngram_embed_bwd_workspace_bytes(plan, num_tokens): W^T and the transposed
+ *              g and G (about 4 D num_tokens + 2 D^2 bytes); its head is the status word */
+size_t ngram_embed_bwd_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens);
+int ngram_embed_bwd(const ngram_embed_plan* plan, const int32_t* tokens, const int32_t* idx,
+                    int64_t num_tokens, const void* const* E_nk, const void* W_stacked,
+                    const void* grad_out, float* dE0, float* const* dE_nk, float* dW,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- embedding amplification (section 3.2.4) ----
  * The pages amplify the N-gram embedding output early in training, either by a constant
  * factor or by a LayerNorm before it joins the residual stream (the factor is garbled in

@@ -229,3 +229,44 @@ def layernorm(x: np.ndarray, gamma=None, beta=None, eps: float = 0.0) -> np.ndar
     if beta is not None:
         y = y + np.asarray(beta, dtype=np.float64)
     return y
+
+
+# ---------------------------------------------------------------- backward (training)
+# Gradients of Eq. 3 (section 2) w.r.t. its parameters, given g = dL/de. The layer is
+# linear in E_0, in each E_{n,k} (for fixed indices) and in W, so each gradient is the
+# plain definition below, written with numpy fp64 primitives (matmul, scatter-add).
+
+def backward(V0: int, D: int, N: int, K: int, V_nk, tokens, seq_offsets, E_nk, W, g, scale: float = 1.0,
+             histories=None):
+    """-> (dE0 [V0, D], [dE_s [V_s, d]], dW [D, D]) in float64 for grad_out g [T, D].
+
+    c = scale / ((N-1)K + 1); dE0[t_i] += c g_i; dG = c g W; dE_s[idx_s(i)] += dG[i, s-block];
+    dW = c g^T G with G the concatenated looked-up sub-rows. Tables as uint16 bf16 bits or
+    float32."""
+    S = (N - 1) * K
+    d = D // S if S else 0
+    c = float(scale) / (S + 1)
+    tokens = np.asarray(tokens)
+    g64 = _to_f64(g)
+    dE0 = np.zeros((V0, D), np.float64)
+    np.add.at(dE0, tokens.astype(np.int64), c * g64)
+    dE = []
+    dW = np.zeros((D, D), np.float64)
+    if S:
+        idx = hash_indices(V0, N, K, V_nk, context_windows(N, tokens, seq_offsets, histories=histories))
+        W64 = _to_f64(W)
+        dG = c * (g64 @ W64)
+        G = np.concatenate([_to_f64(np.asarray(E_nk[s])[idx[:, s]]) for s in range(S)], axis=1)
+        for s in range(S):
+            gs = np.zeros((V_nk[s], d), np.float64)
+            np.add.at(gs, idx[:, s].astype(np.int64), dG[:, s * d:(s + 1) * d])
+            dE.append(gs)
+        dW = c * (g64.T @ G)
+    return dE0, dE, dW
+
+
+def _to_f64(a) -> np.ndarray:
+    a = np.asarray(a)
+    if a.dtype == np.uint16:  # bf16 bit patterns
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)

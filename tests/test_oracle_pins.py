@@ -294,3 +294,60 @@ def test_amplify_is_a_scalar_on_eq3():
     e = rng.normal(size=(3, 16))
     np.testing.assert_array_equal(oracle.amplify(e, 1.0), e)
     np.testing.assert_allclose(oracle.amplify(e, np.sqrt(16.0)), 4.0 * e, rtol=1e-15)
+
+
+# ---------------------------------------------------------------- backward
+
+def test_backward_is_the_exact_directional_derivative():
+    """L(params) = <g, e(params)>. e is linear in E_0, in each sub-table (indices fixed) and
+    in W, so for any direction X of one parameter, L(p + X) - L(p) = <dL/dp, X> exactly (up
+    to fp64 rounding). Both sides from independent code: the left from the C forward
+    oracle, the right from the numpy backward."""
+    rng = np.random.default_rng(11)
+    V0, D, N, K = 200, 48, 3, 2
+    V = [101, 103, 107, 109]
+    S, d = 4, 12
+    lengths = [7, 1, 0, 13]
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    T = int(off[-1])
+    tok = rng.integers(0, 12, T).astype(np.int32)  # few distinct ids: E_0 rows collide
+    # small integers everywhere: every sum and product below is exact in fp32 and fp64,
+    # so the identity must hold to the last bit
+    ints = lambda shape: rng.integers(-8, 9, shape).astype(np.float32)
+    E0 = ints((V0, D))
+    E = [ints((V[s], d)) for s in range(S)]
+    W = ints((D, D))
+    g = ints((T, D)).astype(np.float64)
+    scale = 2.5  # c = 2.5 / 5 = 0.5: exact
+    L = lambda E0_, E_, W_: float(np.sum(g * scale * oracle.forward(V0, D, N, K, V, tok, off, E0_, E_, W_)))
+    dE0, dE, dW = oracle.backward(V0, D, N, K, V, tok, off, E, W, g, scale=scale)
+    base = L(E0, E, W)
+    X = ints(E0.shape)
+    assert L(E0 + X, E, W) - base == np.sum(dE0 * X.astype(np.float64))
+    for s in range(S):
+        X = ints(E[s].shape)
+        E2 = [e.copy() for e in E]
+        E2[s] = E[s] + X
+        assert L(E0, E2, W) - base == np.sum(dE[s] * X.astype(np.float64))
+    X = ints(W.shape)
+    assert L(E0, E, W + X) - base == np.sum(dW * X.astype(np.float64))
+    # a wrong scale, a transposed dW or a dropped collision would each fail one of the above;
+    # negative control: the transpose of dW is not the gradient
+    assert L(E0, E, W + X) - base != np.sum(dW.T * X.astype(np.float64))
+
+
+def test_backward_collisions_add_up():
+    """Two tokens with the same id (and so the same context and rows) double the row grad."""
+    V0, D, N, K = 50, 16, 2, 1
+    V = [53]
+    tok = np.array([5, 5], np.int32)
+    off = np.array([0, 1, 2], np.int32)  # two one-token sequences: both contexts (0, 5)
+    E = [np.ones((53, 16), np.float32)]
+    W = np.eye(16, dtype=np.float32)
+    g = np.ones((2, 16))
+    dE0, dE, dW = oracle.backward(V0, D, N, K, V, tok, off, E, W, g)
+    np.testing.assert_array_equal(dE0[5], np.full(16, 2 * 0.5))
+    r = oracle.hash_indices(V0, N, K, V, oracle.context_windows(N, tok, off))[0, 0]
+    np.testing.assert_array_equal(dE[0][r], np.full(16, 2 * 0.5))
+    assert np.count_nonzero(dE[0]) == 16
+    np.testing.assert_array_equal(dW, np.full((16, 16), 2 * 0.5))
