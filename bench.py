@@ -367,6 +367,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-decode", action="store_true", help="skip the speculative-decode measurement")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward (training) measurement")
+    ap.add_argument("--no-stats", action="store_true", help="skip the hash-statistics sweep")
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--decode-workload", default="spec_decode", choices=sorted(DECODE_WORKLOADS))
     ap.add_argument("--decode-only", action="store_true",
@@ -508,6 +509,31 @@ def main():
     ln_bytes = 2 * out.numel() * out.element_size()
     status = ne.ngram_embed_get_status(ws)
 
+    # --- hash statistics (section 3.2.2, Fig. 3b): collisions of the 2-gram hash for table
+    # sizes swept over [30, 33] V0 (denser next to the multiples of V0), on 100 Zipf
+    # sequences of 4096 tokens
+    stats = None
+    if not args.no_stats and rank == 0:
+        V0 = cfg.V0
+        s_tok = torch.from_numpy(gen.zipf_tokens(cfg.seed + 99, 100 * 4096, V0).astype(np.int32)).to(dev)
+        s_off = torch.from_numpy(gen.offsets_from_lengths([4096] * 100)).to(dev)
+        moduli = sorted({int(V0 * (30 + k * 0.05)) for k in range(61)} |
+                        {m * V0 + dd for m in (30, 31, 32, 33) for dd in (-3, -1, 1, 3)})
+        ne.ngram_hash_stats(V0, 2, s_tok, s_off, moduli[:2])  # warm-up
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        distinct, rows = ne.ngram_hash_stats(V0, 2, s_tok, s_off, moduli, stream=stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        st_ms = t0.elapsed_time(t1)
+        coll = np.array([distinct - r for r in rows])
+        near = np.array([min(abs(v - m * V0) for m in (30, 31, 32, 33)) <= 3 for v in moduli])
+        stats = {"ms": st_ms, "windows": int(s_tok.numel()), "moduli": len(moduli),
+                 "windows_per_s": s_tok.numel() * len(moduli) / (st_ms / 1e3), "distinct_2grams": distinct,
+                 "collisions_near_multiples_median": float(np.median(coll[near])),
+                 "collisions_elsewhere_median": float(np.median(coll[~near]))}
+
     # --- backward (training): parameter gradients for a random bf16 dL/de, fp32 gradient
     # tables accumulated in place; two tcgen05 GEMMs of 2 T D^2 FLOPs each dominate
     backward = None
@@ -572,6 +598,7 @@ def main():
                     "d2h_bytes_per_step": out.numel() * 2},
             "gpu_launches": 2 * args.steps,
             "backward": backward,
+            "hash_stats": stats,
             "amplification": {"layernorm_ms": ln_ms, "bytes": ln_bytes, "gbs": ln_bytes / (ln_ms / 1e3) / 1e9,
                               "frac_hbm": ln_bytes / (ln_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
             "decode": decode,

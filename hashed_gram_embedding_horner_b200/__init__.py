@@ -44,6 +44,7 @@ EXPORTED = [
     "ngram_embed_plan_set_a_stages", "ngram_embed_plan_kernel_form",
     "ngram_embed_plan_set_output_scale", "ngram_embed_layernorm",
     "ngram_embed_bwd_workspace_bytes", "ngram_embed_bwd",
+    "ngram_hash_stats_workspace_bytes", "ngram_hash_stats",
 ]
 
 
@@ -86,6 +87,8 @@ _sig("ngram_embed_plan_set_a_stages", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_kernel_form", [_P, _I64])
 _sig("ngram_embed_plan_set_output_scale", [_P, ctypes.c_float])
 _sig("ngram_embed_bwd_workspace_bytes", [_P, _I64], _SZ)
+_sig("ngram_hash_stats_workspace_bytes", [_I64, _I64, ctypes.c_int], _SZ)
+_sig("ngram_hash_stats", [_I64, ctypes.c_int, _P, _P, _I32, _I64, _P, ctypes.c_int, _P, _P, _P, _SZ, _P])
 _sig("ngram_embed_bwd", [_P, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P])
 _sig("ngram_embed_layernorm", [_P, _P, _I64, _P, _P, ctypes.c_float, _P, _P, _SZ, _P])
 _sig("ngram_embed_selftest_wait_timeout", [_P, _I64, _P])
@@ -218,6 +221,23 @@ def ngram_embed_bwd(plan: Plan, tokens, idx, grad_out, workspace, E_nk=None, W_s
                               _ptr(W_stacked), _ptr(grad_out), _ptr(dE0), grads, _ptr(dW), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "ngram_embed_bwd")
+
+
+def ngram_hash_stats(V0: int, n: int, tokens, seq_offsets, moduli, workspace=None, stream=None):
+    """Hit counts and collisions of the n-gram hash X_n mod V for each V in `moduli`:
+    returns (distinct_ngrams or None, [rows_hit per modulus])."""
+    import torch
+    mods = (_I64 * len(moduli))(*[int(v) for v in moduli])
+    hits = (_I64 * len(moduli))()
+    dist = _I64()
+    need = _lib.ngram_hash_stats_workspace_bytes(tokens.numel(), max(int(v) for v in moduli), len(moduli))
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=tokens.device)
+    rc = _lib.ngram_hash_stats(int(V0), int(n), _i32(tokens, "tokens"), _i32(seq_offsets, "seq_offsets"),
+                               seq_offsets.numel() - 1, tokens.numel(), mods, len(moduli), hits, ctypes.byref(dist),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_hash_stats")
+    return (None if dist.value < 0 else int(dist.value)), [int(h) for h in hits]
 
 
 KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair"}

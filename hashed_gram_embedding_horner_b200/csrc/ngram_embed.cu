@@ -23,6 +23,7 @@
 #include "proj_sm100_pair.cuh"
 #include "simt.cuh"
 #include "bwd_sm100.cuh"
+#include "stats.cuh"
 
 using namespace ngram;
 
@@ -607,6 +608,95 @@ int ngram_embed_plan_set_a_stages(ngram_embed_plan* plan, int stages) {
 int ngram_embed_plan_set_output_scale(ngram_embed_plan* plan, float scale) {
   if (!plan || !(scale == scale) || scale == 0.0f || scale > 3.0e38f || scale < -3.0e38f) return NGRAM_ERR_INVALID_ARG;
   plan->out_scale = scale;
+  return NGRAM_OK;
+}
+
+// ---- hash statistics -----------------------------------------------------------------
+namespace {
+uint64_t stats_set_cap(int64_t T) {
+  uint64_t cap = 1024;
+  while (cap < 2 * static_cast<uint64_t>(T)) cap <<= 1;
+  return cap;
+}
+size_t stats_ws_bytes(int64_t T, int64_t max_modulus, int num_moduli) {
+  return kHeadBytes + round256(static_cast<size_t>(T) * 8) + round256(stats_set_cap(T) * 8) + 256 +
+         round256((static_cast<size_t>(max_modulus) / 32 + 1) * 4) + round256(static_cast<size_t>(num_moduli) * 8);
+}
+}  // namespace
+
+size_t ngram_hash_stats_workspace_bytes(int64_t max_tokens, int64_t max_modulus, int num_moduli) {
+  if (max_tokens < 0 || max_modulus < 1 || num_moduli < 1) return 0;
+  return stats_ws_bytes(max_tokens, max_modulus, num_moduli);
+}
+
+int ngram_hash_stats(int64_t V0, int n, const int32_t* tokens, const int32_t* seq_offsets, int32_t num_seqs,
+                     int64_t num_tokens, const int64_t* moduli, int num_moduli, int64_t* rows_hit,
+                     int64_t* distinct_ngrams, void* workspace, size_t workspace_bytes, void* stream) {
+  if (V0 < 1 || V0 >= (int64_t(1) << 31) || n < 1 || n > kMaxN || num_tokens < 0 || num_tokens > INT32_MAX ||
+      num_seqs < 1 || !moduli || num_moduli < 1 || !rows_hit || !distinct_ngrams || !workspace ||
+      (num_tokens > 0 && (!tokens || !seq_offsets)))
+    return NGRAM_ERR_INVALID_ARG;
+  int64_t max_v = 0;
+  for (int j = 0; j < num_moduli; ++j) {
+    if (moduli[j] < 1 || moduli[j] >= (int64_t(1) << 31)) return NGRAM_ERR_INVALID_ARG;
+    max_v = moduli[j] > max_v ? moduli[j] : max_v;
+  }
+  if (!aligned16(workspace)) return NGRAM_ERR_MISALIGNED;
+  if (workspace_bytes < stats_ws_bytes(num_tokens, max_v, num_moduli)) return NGRAM_ERR_WORKSPACE;
+  // V0^n < 2^64: the window's exact integer fits a 64-bit key
+  unsigned __int128 pw = 1;
+  bool exact64 = true;
+  for (int j = 0; j < n && exact64; ++j) {
+    pw *= static_cast<unsigned __int128>(V0);
+    exact64 = pw < (static_cast<unsigned __int128>(1) << 64);
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NGRAM_ERR_CUDA;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  const uint64_t cap = stats_set_cap(num_tokens);
+  auto* keys = reinterpret_cast<unsigned long long*>(base + kHeadBytes);
+  auto* set = reinterpret_cast<unsigned long long*>(base + kHeadBytes + round256(size_t(num_tokens) * 8));
+  auto* distinct = reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(set) + round256(cap * 8));
+  auto* bitmap = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(distinct) + 256);
+  auto* hits = reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(bitmap) +
+                                                     round256((size_t(max_v) / 32 + 1) * 4));
+  if (cudaMemsetAsync(distinct, 0, 8, st) != cudaSuccess ||
+      cudaMemsetAsync(hits, 0, size_t(num_moduli) * 8, st) != cudaSuccess)
+    return NGRAM_ERR_CUDA;
+  StatsParams sp{};
+  sp.tokens = tokens;
+  sp.offsets = seq_offsets;
+  sp.num_seqs = num_seqs;
+  sp.T = num_tokens;
+  sp.V0 = static_cast<uint32_t>(V0);
+  sp.n = n;
+  sp.exact64 = exact64;
+  sp.keys = keys;
+  sp.set = set;
+  sp.set_mask = cap - 1;
+  sp.distinct = distinct;
+  sp.status = status_ptr(workspace);
+  const unsigned blocks = static_cast<unsigned>((num_tokens + 255) / 256);
+  int rc = NGRAM_OK;
+  if (num_tokens > 0 && exact64) {
+    if (cudaMemsetAsync(set, 0xFF, cap * 8, st) != cudaSuccess) return NGRAM_ERR_CUDA;
+    if ((rc = launch(stats_keys_kernel, dim3(blocks), dim3(256), 0, st, false, 1, sp))) return rc;
+  }
+  for (int j = 0; j < num_moduli && num_tokens > 0; ++j) {
+    sp.V = static_cast<uint32_t>(moduli[j]);
+    sp.barrett = ~uint64_t(0) / static_cast<uint64_t>(moduli[j]);
+    sp.bitmap = bitmap;
+    sp.rows_hit = hits + j;
+    if (cudaMemsetAsync(bitmap, 0, (size_t(moduli[j]) / 32 + 1) * 4, st) != cudaSuccess) return NGRAM_ERR_CUDA;
+    if ((rc = launch(stats_rows_kernel, dim3(blocks), dim3(256), 0, st, false, 1, sp))) return rc;
+  }
+  unsigned long long d_host = 0;
+  if (cudaMemcpyAsync(&d_host, distinct, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(rows_hit, hits, size_t(num_moduli) * 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return NGRAM_ERR_CUDA;
+  *distinct_ngrams = exact64 ? static_cast<int64_t>(d_host) : -1;
   return NGRAM_OK;
 }
 

@@ -228,6 +228,23 @@ int ngram_embed_bwd(const ngram_embed_plan* plan, const int32_t* tokens, const i
                     const void* grad_out, float* dE0, float* const* dE_nk, float* dW,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- hash statistics (section 3.2.2, Fig. 3): choosing table sizes ----
+ * For the n-gram hash H = X_n mod V (Eq. 2, the layer's context rule: pad 0 before a
+ * sequence start) over a token stream:
+ *   rows_hit[j]       number of distinct rows (X_n mod moduli[j]) hit by the stream
+ *                     (hit rate = rows_hit[j] / moduli[j]);
+ *   *distinct_ngrams  number of distinct n-gram windows in the stream, or -1 when
+ *                     V0^n >= 2^64 (windows are then not counted);
+ *   collisions at moduli[j] = *distinct_ngrams - rows_hit[j].
+ * tokens / seq_offsets as for ngram_embed_fwd (device); moduli, rows_hit, distinct_ngrams
+ * are HOST arrays. Analysis, not the hot path: the call synchronises `stream`.
+ *   workspace  >= ngram_hash_stats_workspace_bytes(num_tokens, max modulus, num_moduli) */
+size_t ngram_hash_stats_workspace_bytes(int64_t max_tokens, int64_t max_modulus, int num_moduli);
+int ngram_hash_stats(int64_t V0, int n, const int32_t* tokens, const int32_t* seq_offsets,
+                     int32_t num_seqs, int64_t num_tokens, const int64_t* moduli, int num_moduli,
+                     int64_t* rows_hit, int64_t* distinct_ngrams, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
 /* ---- embedding amplification (section 3.2.4) ----
  * The pages amplify the N-gram embedding output early in training, either by a constant
  * factor or by a LayerNorm before it joins the residual stream (the factor is garbled in

@@ -270,3 +270,20 @@ def _to_f64(a) -> np.ndarray:
     if a.dtype == np.uint16:  # bf16 bit patterns
         return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     return a.astype(np.float64)
+
+
+# ---------------------------------------------------------------- hash statistics
+# Section 3.2.2 (Fig. 3): the vocabulary hit rate (table rows hit at least once by the
+# stream) and hash collisions (distinct n-gram windows minus distinct rows they map to).
+# Plain definitions: Python sets over the windows of the layer's context rule.
+
+def hash_stats(V0: int, n: int, tokens, seq_offsets, moduli):
+    """-> (distinct windows, [distinct rows per modulus]) for the n-gram hash X_n mod V."""
+    win = context_windows(n, tokens, seq_offsets)  # [T, n]: column j is t_{i-j}, pad 0
+    keys = set()
+    xs = []
+    for w in win.tolist():
+        x = sum(int(t) * int(V0) ** j for j, t in enumerate(w))  # Eq. 2's X_n, exact
+        keys.add(x)
+        xs.append(x)
+    return len(keys), [len({x % int(V) for x in xs}) for V in moduli]

@@ -351,3 +351,35 @@ def test_backward_collisions_add_up():
     np.testing.assert_array_equal(dE[0][r], np.full(16, 2 * 0.5))
     assert np.count_nonzero(dE[0]) == 16
     np.testing.assert_array_equal(dW, np.full((16, 16), 2 * 0.5))
+
+
+# ---------------------------------------------------------------- hash statistics (section 3.2.2)
+
+def test_hash_stats_worked_example():
+    """[7, 42, 999, 0, 500], V0 = 1000, 2-grams: the golden indices mod 4099 are 7, 2943, 2009,
+    2943, 500 (positions 1 and 3 collide): 5 windows, 4 rows, 1 collision; mod V0 the row is
+    the newest id (5 rows); a modulus above every X_n loses nothing."""
+    tok = np.array([7, 42, 999, 0, 500], np.int32)
+    off = np.array([0, 5], np.int32)
+    golden = [7, 2943, 2009, 2943, 500]
+    assert len(set(golden)) == 4
+    assert oracle.hash_stats(1000, 2, tok, off, [4099, 1000, 10 ** 7]) == (5, [4, 5, 5])
+
+
+def test_hash_stats_multiple_of_v0_closed_form():
+    """V = m V0 for 2-grams: X_2 mod m V0 = (t_{i-1} mod m) V0 + t_i, so the rows hit are the
+    distinct pairs (t_{i-1} mod m, t_i) — counted here from the pairs, not from X."""
+    rng = np.random.default_rng(12)
+    V0 = 997
+    lengths = [50, 1, 200, 77]
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    tok = rng.integers(0, V0, int(off[-1])).astype(np.int32)
+    prev = np.zeros_like(tok)
+    for b in range(len(lengths)):
+        s, e = off[b], off[b + 1]
+        prev[s + 1:e] = tok[s:e - 1]  # pad 0 before each start
+    for m in (1, 2, 5, 31):
+        want = len({(int(p) % m, int(t)) for p, t in zip(prev, tok)})
+        windows, rows = oracle.hash_stats(V0, 2, tok, off, [m * V0])
+        assert rows == [want] and windows == len({(int(p), int(t)) for p, t in zip(prev, tok)})
+    assert oracle.hash_stats(V0, 2, tok, off, [1])[1] == [1]
