@@ -45,6 +45,7 @@ EXPORTED = [
     "ngram_embed_plan_set_output_scale", "ngram_embed_layernorm",
     "ngram_embed_bwd_workspace_bytes", "ngram_embed_bwd",
     "ngram_hash_stats_workspace_bytes", "ngram_hash_stats",
+    "ngram_draft_cache_reset", "ngram_embed_draft_workspace_bytes", "ngram_embed_fwd_draft",
 ]
 
 
@@ -55,6 +56,10 @@ class _Config(ctypes.Structure):
 
 class _Cache(ctypes.Structure):
     _fields_ = [("ring", _P), ("len", _P), ("valid_from", _P), ("capacity", _I32), ("max_seqs", _I32)]
+
+
+class _DraftCache(ctypes.Structure):
+    _fields_ = [("keys", _P), ("emb", _P), ("positions", _I32), ("max_seqs", _I32)]
 
 
 def _sig(name, args, res=ctypes.c_int):
@@ -88,6 +93,9 @@ _sig("ngram_embed_plan_kernel_form", [_P, _I64])
 _sig("ngram_embed_plan_set_output_scale", [_P, ctypes.c_float])
 _sig("ngram_embed_bwd_workspace_bytes", [_P, _I64], _SZ)
 _sig("ngram_hash_stats_workspace_bytes", [_I64, _I64, ctypes.c_int], _SZ)
+_sig("ngram_draft_cache_reset", [_P, _P, _P, _I32, _P, _SZ, _P])
+_sig("ngram_embed_draft_workspace_bytes", [_P, _I64], _SZ)
+_sig("ngram_embed_fwd_draft", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P])
 _sig("ngram_hash_stats", [_I64, ctypes.c_int, _P, _P, _I32, _I64, _P, ctypes.c_int, _P, _P, _P, _SZ, _P])
 _sig("ngram_embed_bwd", [_P, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P])
 _sig("ngram_embed_layernorm", [_P, _P, _I64, _P, _P, ctypes.c_float, _P, _P, _SZ, _P])
@@ -153,6 +161,47 @@ class Cache:
         return cls(torch.zeros((max_seqs, capacity), dtype=torch.int32, device=device),
                    torch.zeros(max_seqs, dtype=torch.int64, device=device),
                    torch.zeros(max_seqs, dtype=torch.int64, device=device))
+
+
+class DraftCache:
+    """Draft-phase embedding cache (caller-owned torch tensors): keys int32
+    [max_seqs, positions, N], emb [max_seqs, positions, D] in the plan's dtype."""
+
+    def __init__(self, keys, emb):
+        self.keys, self.emb = keys, emb
+        self.struct = _DraftCache(keys.data_ptr(), emb.data_ptr(), keys.shape[1], keys.shape[0])
+
+    @classmethod
+    def empty(cls, plan: "Plan", max_seqs: int, positions: int, device="cuda"):
+        import torch
+        dt = torch.bfloat16 if plan.dtype == NGRAM_BF16 else torch.float32
+        return cls(torch.full((max_seqs, positions, plan.N), -1, dtype=torch.int32, device=device),
+                   torch.zeros((max_seqs, positions, plan.D), dtype=dt, device=device))
+
+
+def ngram_draft_cache_reset(plan: "Plan", dc: DraftCache, workspace, slots=None, stream=None):
+    n = slots.numel() if slots is not None else dc.keys.shape[0]
+    rc = _lib.ngram_draft_cache_reset(plan.handle, ctypes.byref(dc.struct), _i32(slots, "slots"), n, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_draft_cache_reset")
+
+
+def new_draft_workspace(plan: "Plan", max_tokens: int, device="cuda"):
+    import torch
+    return torch.zeros(_lib.ngram_embed_draft_workspace_bytes(plan.handle, int(max_tokens)), dtype=torch.uint8,
+                       device=device)
+
+
+def ngram_embed_fwd_draft(plan: "Plan", tokens, seq_offsets, E0, E_nk, W_stacked, out, workspace, cache: "Cache",
+                          dc: DraftCache, hits=None, cache_slots=None, stream=None):
+    """The layer through the N-gram cache and the draft-phase embedding cache."""
+    tabs = _tables(E_nk)
+    rc = _lib.ngram_embed_fwd_draft(plan.handle, _i32(tokens, "tokens"), _i32(seq_offsets, "seq_offsets"),
+                                    seq_offsets.numel() - 1, tokens.numel(), _ptr(E0), tabs, _ptr(W_stacked),
+                                    ctypes.byref(cache.struct), _i32(cache_slots, "cache_slots"),
+                                    ctypes.byref(dc.struct), _ptr(out), _i32(hits, "hits"), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_embed_fwd_draft")
 
 
 def ngram_embed_plan_create(V0: int, D: int, N: int, K: int, V_nk, dtype: int = NGRAM_BF16) -> Plan:

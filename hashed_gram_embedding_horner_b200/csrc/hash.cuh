@@ -31,6 +31,11 @@ struct HashParams {
   int32_t capacity;
   int32_t max_seqs;
   int32_t* idx_out;  // [T * S]
+  // draft-phase embedding cache: the window ids (oldest first) of every token, [T * N], and
+  // its cache entry slot * positions + (i - sequence start), or -1 past `positions`
+  int32_t* win_out;
+  int32_t* entry_out;
+  int32_t positions;
   int* status;
 };
 
@@ -115,6 +120,11 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashP
     u[j] = static_cast<uint32_t>(t);
   }
 
+  if (p.win_out) {
+    for (int j = 0; j < p.N; ++j) p.win_out[i * p.N + j] = static_cast<int32_t>(u[p.N - 1 - j]);
+    const int64_t jpos = i - start;
+    p.entry_out[i] = (slot >= 0 && jpos < p.positions) ? static_cast<int32_t>(slot * p.positions + jpos) : -1;
+  }
   int32_t* out = p.idx_out + i * p.S;
   for (int n = 2; n <= p.N; ++n) {
     for (int k = 0; k < p.K; ++k) {

@@ -24,6 +24,7 @@
 #include "simt.cuh"
 #include "bwd_sm100.cuh"
 #include "stats.cuh"
+#include "draft.cuh"
 
 using namespace ngram;
 
@@ -349,7 +350,7 @@ int set_device(const ngram_embed_plan* p) {
 
 int launch_hash(const ngram_embed_plan* p, const int32_t* tokens, const int32_t* offsets, int32_t num_seqs,
                 int64_t T, const ngram_cache* cache, const int32_t* slots, int32_t* idx_out, void* ws,
-                cudaStream_t st) {
+                cudaStream_t st, int32_t* win_out = nullptr, int32_t* entry_out = nullptr, int32_t positions = 0) {
   HashParams h{};
   h.tokens = tokens;
   h.offsets = offsets;
@@ -372,6 +373,9 @@ int launch_hash(const ngram_embed_plan* p, const int32_t* tokens, const int32_t*
     h.slots = slots;
   }
   h.idx_out = idx_out;
+  h.win_out = win_out;
+  h.entry_out = entry_out;
+  h.positions = positions;
   h.status = status_ptr(ws);
   const int64_t work = T > num_seqs + 1 ? T : num_seqs + 1;
   const int64_t blocks = (work + 255) / 256;
@@ -386,8 +390,10 @@ int validate_cache(const ngram_embed_plan* p, const ngram_cache* c) {
 
 template <typename T>
 int launch_simt(const ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int64_t n_tok,
-                const void* E0, const void* const* E_nk, const void* W, void* out, void* ws, cudaStream_t st) {
+                const void* E0, const void* const* E_nk, const void* W, void* out, void* ws, cudaStream_t st,
+                const int32_t* T_dev = nullptr) {
   SimtParams<T> s{};
+  s.T_dev = T_dev;
   s.tokens = tokens;
   s.idx = idx;
   s.E0 = static_cast<const T*>(E0);
@@ -420,13 +426,14 @@ int launch_simt(const ngram_embed_plan* p, const int32_t* tokens, const int32_t*
 
 // ws_T: the token count the workspace was validated for (its index buffer's length);
 // the stream-K partials, if the workspace holds them, follow that buffer.
+// T_dev (optional): the kernels take min(*T_dev, T) tokens, a count known only on the device.
 int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int64_t T, const void* E0,
             const void* const* E_nk, const void* W, void* out, void* ws, size_t ws_size, int64_t ws_T,
-            cudaStream_t st) {
+            cudaStream_t st, const int32_t* T_dev = nullptr) {
   if (p->variant == kSimt) {
     return p->dtype == NGRAM_F32
-               ? launch_simt<float>(p, tokens, idx, T, E0, E_nk, W, out, ws, st)
-               : launch_simt<uint16_t>(p, tokens, idx, T, E0, E_nk, W, out, ws, st);
+               ? launch_simt<float>(p, tokens, idx, T, E0, E_nk, W, out, ws, st, T_dev)
+               : launch_simt<uint16_t>(p, tokens, idx, T, E0, E_nk, W, out, ws, st, T_dev);
   }
   int rc = refresh_maps(p, E_nk, W, out, T);
   if (rc) return rc;
@@ -449,7 +456,9 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   prm.num_k_blocks = p->D / kBK;
   prm.scale = p->out_scale / static_cast<float>(p->S + 1);
   prm.status = status_ptr(ws);
-  const bool sk = p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
+  prm.T_dev = T_dev;
+  // stream-K needs every CTA to hold a unit, which a device-side count cannot promise
+  const bool sk = !T_dev && p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
   const bool pair = p->cta_pair == 1 || (p->cta_pair == -1 && !sk);
   // A rows by TMA gather4 in the pair form, by cp.async in the one-CTA form (measured
   // fastest for each), unless the plan fixes the split.
@@ -698,6 +707,120 @@ int ngram_hash_stats(int64_t V0, int n, const int32_t* tokens, const int32_t* se
     return NGRAM_ERR_CUDA;
   *distinct_ngrams = exact64 ? static_cast<int64_t>(d_host) : -1;
   return NGRAM_OK;
+}
+
+// ---- draft-phase embedding cache ----------------------------------------------------
+namespace {
+struct DraftWs {
+  int32_t *idx, *win, *entry, *miss_count, *miss_token, *miss_idx, *miss_pos, *miss_entry;
+  uint8_t* miss_out;
+  size_t bytes;
+};
+DraftWs draft_ws(const ngram_embed_plan* p, int64_t T, void* ws) {
+  DraftWs w{};
+  size_t off = kHeadBytes;
+  auto take = [&](size_t b) {
+    const size_t at = off;
+    off += round256(b);
+    return at;
+  };
+  const size_t t = static_cast<size_t>(T);
+  const size_t a_idx = take(t * p->S * 4), a_win = take(t * p->N * 4), a_entry = take(t * 4), a_cnt = take(4),
+               a_tok = take(t * 4), a_midx = take(t * p->S * 4), a_pos = take(t * 4), a_ment = take(t * 4),
+               a_out = take(t * static_cast<size_t>(p->D) * p->elt);
+  w.bytes = off;
+  if (ws) {
+    auto* b = static_cast<uint8_t*>(ws);
+    w.idx = reinterpret_cast<int32_t*>(b + a_idx);
+    w.win = reinterpret_cast<int32_t*>(b + a_win);
+    w.entry = reinterpret_cast<int32_t*>(b + a_entry);
+    w.miss_count = reinterpret_cast<int32_t*>(b + a_cnt);
+    w.miss_token = reinterpret_cast<int32_t*>(b + a_tok);
+    w.miss_idx = reinterpret_cast<int32_t*>(b + a_midx);
+    w.miss_pos = reinterpret_cast<int32_t*>(b + a_pos);
+    w.miss_entry = reinterpret_cast<int32_t*>(b + a_ment);
+    w.miss_out = b + a_out;
+  }
+  return w;
+}
+}  // namespace
+
+size_t ngram_embed_draft_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens) {
+  if (!plan || max_tokens < 0) return 0;
+  return draft_ws(plan, max_tokens, nullptr).bytes;
+}
+
+int ngram_draft_cache_reset(const ngram_embed_plan* plan, const ngram_draft_cache* dc, const int32_t* slots,
+                            int32_t n, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = validate_common(plan, workspace, workspace_bytes, 0);
+  if (rc) return rc;
+  if (!dc || !dc->keys || !dc->emb || dc->positions < 1 || dc->max_seqs < 0 || n < 0 || n > dc->max_seqs)
+    return NGRAM_ERR_INVALID_ARG;
+  if (n == 0) return NGRAM_OK;
+  if ((rc = set_device(plan))) return rc;
+  DraftResetParams r{};
+  r.keys = dc->keys;
+  r.slots = slots;
+  r.n = n;
+  r.positions = dc->positions;
+  r.N = plan->N;
+  r.max_seqs = dc->max_seqs;
+  r.status = status_ptr(workspace);
+  const int64_t work = static_cast<int64_t>(n) * dc->positions;
+  return launch(draft_reset_kernel, dim3(static_cast<unsigned>((work + 255) / 256)), dim3(256), 0,
+                static_cast<cudaStream_t>(stream), plan->pdl, 1, r);
+}
+
+int ngram_embed_fwd_draft(const ngram_embed_plan* plan_c, const int32_t* tokens, const int32_t* seq_offsets,
+                          int32_t num_seqs, int64_t num_tokens, const void* E0, const void* const* E_nk,
+                          const void* W_stacked, const ngram_cache* cache, const int32_t* cache_slots,
+                          const ngram_draft_cache* dc, void* out, int32_t* hits_out, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  auto* plan = const_cast<ngram_embed_plan*>(plan_c);
+  if (!plan || !workspace || num_tokens < 0 || num_tokens > INT32_MAX || num_seqs < 0) return NGRAM_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return NGRAM_ERR_MISALIGNED;
+  const DraftWs w = draft_ws(plan, num_tokens, workspace);
+  if (workspace_bytes < w.bytes) return NGRAM_ERR_WORKSPACE;
+  if (num_tokens == 0) return NGRAM_OK;
+  if (!tokens || !seq_offsets || num_seqs == 0 || !out || !cache || !dc || !dc->keys || !dc->emb ||
+      dc->positions < 1 || dc->max_seqs < cache->max_seqs)
+    return NGRAM_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(dc->emb)) return NGRAM_ERR_MISALIGNED;
+  int rc;
+  if ((rc = check_tables(plan, E0, E_nk, W_stacked))) return rc;
+  if ((rc = validate_cache(plan, cache))) return rc;
+  if ((rc = set_device(plan))) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(w.miss_count, 0, 4, st) != cudaSuccess) return NGRAM_ERR_CUDA;
+  if ((rc = launch_hash(plan, tokens, seq_offsets, num_seqs, num_tokens, cache, cache_slots, w.idx, workspace, st,
+                        w.win, w.entry, dc->positions)))
+    return rc;
+  DraftParams d{};
+  d.tokens = tokens;
+  d.idx = w.idx;
+  d.win = w.win;
+  d.entry = w.entry;
+  d.keys = dc->keys;
+  d.emb = static_cast<uint8_t*>(dc->emb);
+  d.T = num_tokens;
+  d.N = plan->N;
+  d.S = plan->S;
+  d.row_bytes = plan->D * plan->elt;
+  d.out = static_cast<uint8_t*>(out);
+  d.miss_count = w.miss_count;
+  d.miss_token = w.miss_token;
+  d.miss_idx = w.miss_idx;
+  d.miss_pos = w.miss_pos;
+  d.miss_entry = w.miss_entry;
+  d.miss_out = w.miss_out;
+  d.hits = hits_out;
+  const unsigned warps_blocks = static_cast<unsigned>((num_tokens + 7) / 8);
+  if ((rc = launch(draft_probe_kernel, dim3(warps_blocks), dim3(256), 0, st, plan->pdl, 1, d))) return rc;
+  // the misses' rows (at most num_tokens; the kernels read the count)
+  if ((rc = project(plan, w.miss_token, w.miss_idx, num_tokens, E0, E_nk, W_stacked, w.miss_out, workspace,
+                    workspace_bytes, 0, st, w.miss_count)))
+    return rc;
+  return launch(draft_scatter_kernel, dim3(warps_blocks), dim3(256), 0, st, plan->pdl, 1, d);
 }
 
 size_t ngram_embed_bwd_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens) {

@@ -69,6 +69,9 @@ struct ProjParams {
   int stream_k;
   int* sk_counters;
   float* sk_partials;
+  // if set, the token count is min(*T_dev, T), read by the kernel (a count produced on the
+  // device, e.g. the cache misses of a draft-phase call); num_m_blocks then covers T
+  const int32_t* T_dev;
 };
 
 struct ProjMaps {
@@ -308,7 +311,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   pdl_launch_dependents();
   pdl_wait();  // nothing above touched global memory
 
-  const int num_tiles = p.num_m_blocks * p.num_n_blocks;
+  const int64_t T = p.T_dev ? (*p.T_dev < p.T ? *p.T_dev : p.T) : p.T;
+  const int num_tiles = static_cast<int>((T + kBM - 1) / kBM) * p.num_n_blocks;
   const int KB = p.num_k_blocks;
   const int kb_per_sub = p.d / kBK;
   WorkPlan wp;
@@ -338,9 +342,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t g1 = row_base + p.tma_rows + rsub + 32 * j;
-        dst[j] = (j < n_cp && g1 < p.T) ? ld_idx_early(p.idx + g1 * p.S + r.s) : 0;
+        dst[j] = (j < n_cp && g1 < T) ? ld_idx_early(p.idx + g1 * p.S + r.s) : 0;
         const int64_t g2 = row_base + issuer * 4 + j;
-        dst[4 + j] = (tma_issuer && g2 < p.T) ? ld_idx_early(p.idx + g2 * p.S + r.s) : 0;
+        dst[4 + j] = (tma_issuer && g2 < T) ? ld_idx_early(p.idx + g2 * p.S + r.s) : 0;
       }
     };
     int stage = 0;
@@ -455,7 +459,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       const bool whole = g.i0 == 0 && g.i1 == KB;
       const int64_t gr = static_cast<int64_t>(m_blk) * kBM + row_in_tile;
-      const bool valid = gr < p.T;
+      const bool valid = gr < T;
       uint32_t t = 0;
       if (valid) {
         const int32_t tok = p.tokens[gr];
@@ -513,7 +517,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         // a box that starts past T is not issued).
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && static_cast<int64_t>(m_blk) * kBM + q * 32 < p.T) {
+        if (lane == 0 && static_cast<int64_t>(m_blk) * kBM + q * 32 < T) {
 #pragma unroll
           for (int b = 0; b < BN / 64; ++b)
             tma_store_2d(&maps.Out, stage_q + b * 16384, n_blk * BN + b * 64, m_blk * kBM + q * 32);

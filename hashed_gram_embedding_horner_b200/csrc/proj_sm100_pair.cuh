@@ -105,7 +105,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   pdl_launch_dependents();
   pdl_wait();  // nothing above touched global memory
 
-  const int num_tiles = p.num_m_blocks * p.num_n_blocks;  // m blocks of 256 rows
+  const int64_t T = p.T_dev ? (*p.T_dev < p.T ? *p.T_dev : p.T) : p.T;
+  const int num_tiles = static_cast<int>((T + 2 * kBM - 1) / (2 * kBM)) * p.num_n_blocks;  // m blocks of 256 rows
   const int KB = p.num_k_blocks;
   const int kb_per_sub = p.d / kBK;
 
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t gr = row_base + (cp_rows ? rsub + 32 * j : iss * 4 + j);
-        dst[j] = ((cp_rows || issuer) && gr < p.T) ? ld_idx_early(p.idx + gr * p.S + r.s) : 0;
+        dst[j] = ((cp_rows || issuer) && gr < T) ? ld_idx_early(p.idx + gr * p.S + r.s) : 0;
       }
     };
     int stage = 0;
@@ -255,7 +256,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       const int64_t gr = static_cast<int64_t>(m_blk) * (2 * kBM) + rank * kBM + row_in_tile;
-      const bool valid = gr < p.T;
+      const bool valid = gr < T;
       uint32_t t = 0;
       if (valid) {
         const int32_t tok = p.tokens[gr];

@@ -39,6 +39,7 @@ struct SimtParams {
   int D, S, d;
   int tokens_per_block;
   float scale;
+  const int32_t* T_dev;  // if set, the token count is min(*T_dev, T_tokens)
   int* status;
 };
 
@@ -52,7 +53,8 @@ __global__ void __launch_bounds__(256) proj_simt_kernel(const __grid_constant__ 
   pdl_wait();
   const int TPB = p.tokens_per_block;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * TPB;
-  const int64_t left = p.T_tokens - t0;
+  const int64_t T_eff = p.T_dev ? (*p.T_dev < p.T_tokens ? *p.T_dev : p.T_tokens) : p.T_tokens;
+  const int64_t left = T_eff - t0;
   const int nt = static_cast<int>(left < TPB ? left : TPB);
   if (nt <= 0) return;
 

@@ -208,6 +208,40 @@ int ngram_embed_fwd_static_ws(const ngram_embed_plan* plan, const int32_t* token
                               const ngram_cache* cache, const int32_t* cache_slots, void* out,
                               int32_t* status_out, void* stream);
 
+/* ---- draft-phase embedding cache (section 4.2, optimisations for speculative decoding) ----
+ * Embeddings computed while drafting are kept so that verification does not compute them
+ * again. Entry (slot, j) holds the embedding of the token at in-step position j of the
+ * sequence in cache slot `slot`, with the N ids of its window as the key. A token's output
+ * depends only on its window, so a token whose window equals its entry's key takes the
+ * stored row (bit-identical to what was computed), and nothing needs invalidating when
+ * drafts are rejected or the history moves on. Caller-owned device arrays:
+ *   keys [max_seqs x positions x N] int32 (reset before first use), emb [max_seqs x
+ *   positions x D] in the plan dtype, 16-byte aligned. */
+typedef struct {
+  int32_t* keys;
+  void* emb;
+  int32_t positions;  /* entries per slot: the in-step positions (e.g. 1 + drafts) */
+  int32_t max_seqs;   /* slots; must be >= the N-gram cache's max_seqs */
+} ngram_draft_cache;
+
+/* Empty the entries of slots[0..n) (of slots 0..n-1 if slots is NULL). */
+int ngram_draft_cache_reset(const ngram_embed_plan* plan, const ngram_draft_cache* dc,
+                            const int32_t* slots, int32_t n, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* ngram_embed_fwd through the N-gram cache ring (cache required) and the draft cache: hits
+ * are copied, misses computed (projection over the misses only, their count read on the
+ * device) and stored. In-step positions beyond dc->positions are computed, not cached.
+ *   hits_out   device int32 (may be NULL): incremented by the number of hits
+ *   workspace  >= ngram_embed_draft_workspace_bytes(plan, num_tokens) */
+size_t ngram_embed_draft_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens);
+int ngram_embed_fwd_draft(const ngram_embed_plan* plan, const int32_t* tokens,
+                          const int32_t* seq_offsets, int32_t num_seqs, int64_t num_tokens,
+                          const void* E0, const void* const* E_nk, const void* W_stacked,
+                          const ngram_cache* cache, const int32_t* cache_slots,
+                          const ngram_draft_cache* dc, void* out, int32_t* hits_out,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- backward (training; the pages train the layer from scratch, section 6) ----
  * Gradients of Eq. 3 given g = dL/de (bf16 [num_tokens x D]) and the forward's indices
  * (idx from ngram_hash_indices, [num_tokens x S]); c = output scale / ((N-1)K+1):
