@@ -336,6 +336,27 @@ def run_decode(ne, cfg, steps: int, warmup: int, dev, rank: int = 0):
     gather_ms = timed(lambda i, st: ne.ngram_embed_gather(plan, idx_all[i], E, G, ws, tokens=tok_all[i], E0=E0,
                                                           E0_out=R0, stream=st))
     gather_bytes = T * (cfg.S * cfg.d + cfg.D) * 2 * 2  # rows read + rows written
+    # Draft-phase embedding cache: a verify call whose 5 in-step embeddings were all
+    # computed while drafting (all hits), and the last draft call of a step (4 hits and the
+    # new draft's miss per sequence), against the plain forward of the same 1280 tokens.
+    dc = ne.DraftCache.empty(plan, B, P, device=dev)
+    ne.ngram_draft_cache_reset(plan, dc, ws)
+    dws = ne.new_draft_workspace(plan, T, device=dev)
+    tok_v = tok_all[0]
+    tok_alt = tok_all[0].clone().view(B, P)
+    tok_alt[:, P - 1] = (tok_alt[:, P - 1] + 1) % cfg.V0
+    tok_alt = tok_alt.view(-1)
+    ne.ngram_embed_fwd_draft(plan, tok_v, offsets, E0, E, W, out, dws, cache, dc)
+    hits_d = torch.zeros(1, dtype=torch.int32, device=dev)
+    verify_ms = timed(lambda i, st: ne.ngram_embed_fwd_draft(plan, tok_v, offsets, E0, E, W, out, dws, cache, dc,
+                                                             hits=hits_d, stream=st))
+    alt = [tok_v, tok_alt]
+    draft_ms = timed(lambda i, st: ne.ngram_embed_fwd_draft(plan, alt[i & 1], offsets, E0, E, W, out, dws, cache, dc,
+                                                            stream=st))
+    plain_ms = timed(lambda i, st: ne.ngram_embed_fwd(plan, tok_all[i], offsets, E0, E, W, out, ws, cache=cache,
+                                                      stream=st))
+    hit_rate = hits_d.item() / (T * (3 + 4 * n_k))  # timed(): 3 eager calls, then 1 + 3 replays of n_k
+
     pk = peaks()
     flops = 2.0 * T * cfg.D * cfg.D
     res = {
@@ -347,6 +368,8 @@ def run_decode(ne, cfg, steps: int, warmup: int, dev, rank: int = 0):
         "hash_ms": hash_ms,
         "gather_stage": {"ms": gather_ms, "bytes": gather_bytes, "gbs": gather_bytes / (gather_ms / 1e3) / 1e9,
                          "frac_hbm": gather_bytes / (gather_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+        "draft_cache": {"verify_all_hits_ms": verify_ms, "draft_step_4_of_5_hits_ms": draft_ms,
+                        "plain_forward_ms": plain_ms, "verify_hit_rate": hit_rate},
         "device_status": status,
     }
     del graphs, E0, E, W

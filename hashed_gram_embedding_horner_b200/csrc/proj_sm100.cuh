@@ -318,7 +318,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   WorkPlan wp;
   wp.num_tiles = num_tiles;
   wp.KB = KB;
-  wp.grid = static_cast<int>(gridDim.x);
+  // stream-K partitions the units over at most as many CTAs as there are units (the count
+  // may be known only here, on the device); CTAs past that hold none
+  const int64_t units_total = static_cast<int64_t>(num_tiles) * KB;
+  wp.grid = (p.stream_k && units_total < gridDim.x) ? static_cast<int>(units_total) : static_cast<int>(gridDim.x);
   wp.sk = p.stream_k;
   wp.u_end = p.stream_k ? sk_first_unit(static_cast<int64_t>(num_tiles) * KB, wp.grid, blockIdx.x + 1) : 0;
 

@@ -27,7 +27,7 @@ def dev_i32(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
 
 
-@pytest.mark.parametrize("pair", [None, 0])
+@pytest.mark.parametrize("pair", [None, 0])  # misses by CTA pairs (automatic), or one CTA per tile
 def test_draft_then_verify(ne, pair):
     from synth import configs
     V0, D, N, K = 5000, 1024, 3, 2
