@@ -95,42 +95,156 @@ __global__ void __launch_bounds__(256) gather_transpose_kernel(const __grid_cons
 }
 
 // ------------------------------------------------------------------ dE_0 scatter
+// dE0[v] += c * sum_{i : t_i = v} g_i. Token streams repeat ids heavily (Zipf: the commonest
+// id is ~10 % of a batch), so adding each row atomically into dE0 would serialise on the
+// hot rows. Instead: a counting sort of the positions by token id (histogram, exclusive scan
+// over V0, scatter), then each warp sums a run of kSegRows consecutive sorted positions and
+// adds one partial row per distinct id in its run — a hot id costs one add per run.
+
+constexpr int kSegRows = 16;
 
 struct ScatterE0Params {
   const int32_t* tokens;
-  const uint16_t* g;  // [T x D] bf16
-  float* dE0;         // [V0 x D] fp32
+  const uint16_t* g;   // [T x D] bf16
+  float* dE0;          // [V0 x D] fp32
   int64_t T;
   int D;
   uint32_t V0;
   float scale;
+  int32_t* counts;     // [V0 + 1]: histogram, then exclusive prefix (bin starts)
+  int32_t* cursor;     // [V0]: fill positions
+  int32_t* order;      // [T]: positions sorted by token id
+  int32_t* sorted_tok; // [T]: their ids
+  int32_t* block_sums; // [num_blocks]: scan totals of 1024-bin blocks, then their prefixes
+  int num_blocks;
   int* status;
 };
 
-// One warp per token: dE0[t_i] += scale * g_i, 16-byte vector atomics.
-__global__ void __launch_bounds__(256) scatter_e0_kernel(const __grid_constant__ ScatterE0Params p) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (i >= p.T) return;
-  int32_t t = p.tokens[i];
+__device__ __forceinline__ uint32_t e0_token(const ScatterE0Params& p, int64_t i) {
+  const int32_t t = p.tokens[i];
   if (static_cast<uint32_t>(t) >= p.V0) {
-    if (lane == 0) set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
-    t = 0;
+    set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+    return 0;
   }
-  const uint4* src = reinterpret_cast<const uint4*>(p.g + i * p.D);
-  float4* dst = reinterpret_cast<float4*>(p.dE0 + static_cast<int64_t>(t) * p.D);
-  for (int v = lane; v < (p.D >> 3); v += 32) {
-    const uint4 u = src[v];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    float f[8];
+  return static_cast<uint32_t>(t);
+}
+
+__global__ void __launch_bounds__(256) e0_hist_kernel(const __grid_constant__ ScatterE0Params p) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < p.T) atomicAdd(p.counts + e0_token(p, i), 1);
+}
+
+// Exclusive scan of counts[0..V0) in place, in three launches: each block of 1024 bins
+// scans itself and records its total; one block scans the totals (in chunks of 1024 when
+// there are more); each block adds its prefix.
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t c, int32_t* warp_sums, int32_t& total) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  int32_t x = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int32_t t = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    warp_sums[lane] = t;
+  }
+  __syncthreads();
+  total = warp_sums[31];
+  const int32_t r = (w > 0 ? warp_sums[w - 1] : 0) + x - c;
+  __syncthreads();  // warp_sums may be reused by the caller's next scan
+  return r;
+}
+
+__global__ void __launch_bounds__(1024) e0_scan_blocks_kernel(const __grid_constant__ ScatterE0Params p) {
+  __shared__ int32_t warp_sums[32];
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x;
+  const int32_t c = b < p.V0 ? p.counts[b] : 0;
+  int32_t total;
+  const int32_t ex = block_exclusive_scan(c, warp_sums, total);
+  if (b < p.V0) p.counts[b] = ex;
+  if (threadIdx.x == 0) p.block_sums[blockIdx.x] = total;
+}
+
+__global__ void __launch_bounds__(1024) e0_scan_top_kernel(const __grid_constant__ ScatterE0Params p) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < p.num_blocks; base += 1024) {
+    const int k = base + threadIdx.x;
+    const int32_t c = k < p.num_blocks ? p.block_sums[k] : 0;
+    int32_t total;
+    const int32_t ex = block_exclusive_scan(c, warp_sums, total);
+    if (k < p.num_blocks) p.block_sums[k] = carry + ex;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += total;
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(1024) e0_scan_add_kernel(const __grid_constant__ ScatterE0Params p) {
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x;
+  if (b < p.V0) p.counts[b] += p.block_sums[blockIdx.x];
+}
+
+__global__ void __launch_bounds__(256) e0_place_kernel(const __grid_constant__ ScatterE0Params p) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= p.T) return;
+  const uint32_t t = e0_token(p, i);
+  const int32_t at = p.counts[t] + atomicAdd(p.cursor + t, 1);
+  p.order[at] = static_cast<int32_t>(i);
+  p.sorted_tok[at] = static_cast<int32_t>(t);
+}
+
+// One warp per (run of kSegRows sorted positions, 256 columns): each lane loads its 8
+// columns (16 bytes) of all kSegRows rows first, then sums them in order, adding one
+// partial row into dE0 per distinct id in the run.
+__global__ void __launch_bounds__(256) e0_reduce_kernel(const __grid_constant__ ScatterE0Params p) {
+  const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int chunks = (p.D + 255) / 256;
+  const int64_t seg = item / chunks;
+  const int c = static_cast<int>(item - seg * chunks) * 256 + lane * 8;
+  const int64_t k0 = seg * kSegRows;
+  if (k0 >= p.T || c >= p.D) return;
+  const int n = static_cast<int>(p.T - k0 < kSegRows ? p.T - k0 : kSegRows);
+  uint4 rows[kSegRows];
+#pragma unroll
+  for (int r = 0; r < kSegRows; ++r)
+    if (r < n) rows[r] = *reinterpret_cast<const uint4*>(p.g + static_cast<int64_t>(p.order[k0 + r]) * p.D + c);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int32_t cur = p.sorted_tok[k0];
+  auto flush = [&](int32_t tok) {
+    float4* dst = reinterpret_cast<float4*>(p.dE0 + static_cast<int64_t>(tok) * p.D + c);
+    atomicAdd(dst, make_float4(acc[0] * p.scale, acc[1] * p.scale, acc[2] * p.scale, acc[3] * p.scale));
+    atomicAdd(dst + 1, make_float4(acc[4] * p.scale, acc[5] * p.scale, acc[6] * p.scale, acc[7] * p.scale));
+#pragma unroll
+    for (int h = 0; h < 8; ++h) acc[h] = 0.f;
+  };
+#pragma unroll
+  for (int r = 0; r < kSegRows; ++r) {
+    if (r >= n) break;
+    const int32_t tok = p.sorted_tok[k0 + r];
+    if (tok != cur) {
+      flush(cur);
+      cur = tok;
+    }
+    const uint32_t wds[4] = {rows[r].x, rows[r].y, rows[r].z, rows[r].w};
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      f[2 * h] = bf16_bits_to_float(w[h] & 0xFFFFu) * p.scale;
-      f[2 * h + 1] = bf16_bits_to_float(w[h] >> 16) * p.scale;
+      acc[2 * h] += bf16_bits_to_float(wds[h] & 0xFFFFu);
+      acc[2 * h + 1] += bf16_bits_to_float(wds[h] >> 16);
     }
-    atomicAdd(dst + 2 * v, make_float4(f[0], f[1], f[2], f[3]));
-    atomicAdd(dst + 2 * v + 1, make_float4(f[4], f[5], f[6], f[7]));
   }
+  flush(cur);
 }
 
 // ------------------------------------------------------------------ dense tcgen05 GEMM

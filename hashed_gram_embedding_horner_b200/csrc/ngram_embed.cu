@@ -276,9 +276,14 @@ constexpr int kBwdStages = 4;  // x (16 KB A + BN x 128 B B)
 
 int64_t pad8(int64_t T) { return (T + 7) & ~int64_t(7); }
 size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+// dE0's counting sort: counts [V0 + 1], cursor [V0], order [T], sorted ids [T] (int32).
+size_t bwd_sort_bytes(const ngram_embed_plan* p, int64_t T) {
+  return round256((static_cast<size_t>(p->V0) + 1) * 4) + round256(static_cast<size_t>(p->V0) * 4) +
+         2 * round256(static_cast<size_t>(T) * 4) + round256((static_cast<size_t>(p->V0) + 1023) / 1024 * 4);
+}
 size_t bwd_ws_bytes(const ngram_embed_plan* p, int64_t T) {
   const size_t D = static_cast<size_t>(p->D);
-  return kHeadBytes + round256(D * D * 2) + 2 * round256(D * static_cast<size_t>(pad8(T)) * 2);
+  return kHeadBytes + round256(D * D * 2) + 2 * round256(D * static_cast<size_t>(pad8(T)) * 2) + bwd_sort_bytes(p, T);
 }
 
 // Split-K factor for a GEMM of `tiles` output tiles and KB k-blocks: the one, up to KB / 16
@@ -861,6 +866,7 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
   const auto* g = static_cast<const uint16_t*>(grad_out);
 
   if (dE0) {
+    uint8_t* sort = reinterpret_cast<uint8_t*>(GT) + round256(size_t(D) * T8 * 2);
     ScatterE0Params e{};
     e.tokens = tokens;
     e.g = g;
@@ -869,8 +875,24 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     e.D = D;
     e.V0 = static_cast<uint32_t>(p->V0);
     e.scale = scale;
+    e.counts = reinterpret_cast<int32_t*>(sort);
+    e.cursor = reinterpret_cast<int32_t*>(sort + round256((size_t(p->V0) + 1) * 4));
+    e.order = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(e.cursor) + round256(size_t(p->V0) * 4));
+    e.sorted_tok = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(e.order) + round256(size_t(T) * 4));
+    e.block_sums = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(e.sorted_tok) + round256(size_t(T) * 4));
+    e.num_blocks = static_cast<int>((p->V0 + 1023) / 1024);
     e.status = status_ptr(workspace);
-    if ((rc = launch(scatter_e0_kernel, dim3(static_cast<unsigned>((T + 7) / 8)), dim3(256), 0, st, p->pdl, 1, e)))
+    const unsigned tb = static_cast<unsigned>((T + 255) / 256);
+    if (cudaMemsetAsync(e.counts, 0, (size_t(p->V0) + 1) * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(e.cursor, 0, size_t(p->V0) * 4, st) != cudaSuccess)
+      return NGRAM_ERR_CUDA;
+    if ((rc = launch(e0_hist_kernel, dim3(tb), dim3(256), 0, st, p->pdl, 1, e))) return rc;
+    if ((rc = launch(e0_scan_blocks_kernel, dim3(e.num_blocks), dim3(1024), 0, st, p->pdl, 1, e))) return rc;
+    if ((rc = launch(e0_scan_top_kernel, dim3(1), dim3(1024), 0, st, p->pdl, 1, e))) return rc;
+    if ((rc = launch(e0_scan_add_kernel, dim3(e.num_blocks), dim3(1024), 0, st, p->pdl, 1, e))) return rc;
+    if ((rc = launch(e0_place_kernel, dim3(tb), dim3(256), 0, st, p->pdl, 1, e))) return rc;
+    const int64_t items = (T + kSegRows - 1) / kSegRows * ((D + 255) / 256);  // one warp each
+    if ((rc = launch(e0_reduce_kernel, dim3(static_cast<unsigned>((items + 7) / 8)), dim3(256), 0, st, p->pdl, 1, e)))
       return rc;
   }
   if (dE_nk) {
