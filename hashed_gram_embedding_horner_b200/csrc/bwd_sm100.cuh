@@ -23,9 +23,44 @@
 namespace ngram {
 
 // ------------------------------------------------------------------ transposes
+// 64 x 64 bf16 tiles through shared memory, 16-byte loads and stores on both sides: 256
+// threads read the tile's 64 source rows (128 bytes each) and write its 64 destination rows.
 
-// dst[c][r] = src[r][c] for r < R, and 0 for R <= r < R_pad (dst rows are R_pad long, a
-// multiple of 8 so the rows of dst stay 16-byte aligned for TMA). bf16, 32 x 32 tiles.
+constexpr int kTT = 64;        // tile edge
+constexpr int kTTPad = 8;      // bf16 of padding per shared row (rows 144 bytes apart)
+
+// src_row(r) -> pointer to the 64 source values of tile row r (or nullptr: zeros).
+template <typename SrcRow>
+__device__ __forceinline__ void transpose_tile(uint16_t (*tile)[kTT + kTTPad], SrcRow src_row, uint16_t* dst,
+                                               int64_t dst_stride, int64_t dst_col0, int dst_rows,
+                                               int64_t dst_cols) {
+  const int t = threadIdx.x;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {  // 64 rows x 8 vectors
+    const int v = t + 256 * k;
+    const int r = v >> 3, c8 = (v & 7) * 8;
+    const uint16_t* src = src_row(r);
+    const uint4 u = src ? *reinterpret_cast<const uint4*>(src + c8) : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint2*>(&tile[r][c8]) = make_uint2(u.x, u.y);
+    *reinterpret_cast<uint2*>(&tile[r][c8 + 4]) = make_uint2(u.z, u.w);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {  // 64 destination rows (source columns) x 8 vectors
+    const int v = t + 256 * k;
+    const int c = v >> 3, r8 = (v & 7) * 8;
+    if (c >= dst_rows || dst_col0 + r8 >= dst_cols) continue;
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      w[h] = static_cast<uint32_t>(tile[r8 + 2 * h][c]) | (static_cast<uint32_t>(tile[r8 + 2 * h + 1][c]) << 16);
+    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(c) * dst_stride + dst_col0 + r8) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// dst[c][r] = src[r][c] for r < R, 0 for R <= r < R_pad (dst rows are R_pad long, a multiple
+// of 8, so they stay 16-byte aligned for TMA). C a multiple of 64.
 struct TransposeParams {
   const uint16_t* src;
   uint16_t* dst;
@@ -34,23 +69,12 @@ struct TransposeParams {
 };
 
 __global__ void __launch_bounds__(256) transpose_bf16_kernel(const __grid_constant__ TransposeParams p) {
-  __shared__ uint16_t tile[32][33];
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 32;
-  const int c0 = blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int64_t r = r0 + ty + 8 * k;
-    const int c = c0 + tx;
-    tile[ty + 8 * k][tx] = (r < p.R && c < p.C) ? p.src[r * p.C + c] : uint16_t(0);
-  }
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int c = c0 + ty + 8 * k;
-    const int64_t r = r0 + tx;
-    if (c < p.C && r < p.R_pad) p.dst[static_cast<int64_t>(c) * p.R_pad + r] = tile[tx][ty + 8 * k];
-  }
+  __shared__ __align__(16) uint16_t tile[kTT][kTT + kTTPad];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kTT;
+  const int c0 = blockIdx.y * kTT;
+  transpose_tile(
+      tile, [&](int r) { return r0 + r < p.R ? p.src + (r0 + r) * p.C + c0 : nullptr; },
+      p.dst + static_cast<int64_t>(c0) * p.R_pad, p.R_pad, r0, kTT, p.R_pad);
 }
 
 // GT[c][i] = G[i][c] = E_s[idx[i][s]][c - s d] (s = c / d) for i < T, 0 for T <= i < T_pad.
@@ -65,33 +89,24 @@ struct GatherTParams {
 };
 
 __global__ void __launch_bounds__(256) gather_transpose_kernel(const __grid_constant__ GatherTParams p) {
-  __shared__ uint16_t tile[32][33];
-  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * 32;
-  const int c0 = blockIdx.y * 32;  // 32 columns never straddle two sub-tables (d % 64 == 0)
+  __shared__ __align__(16) uint16_t tile[kTT][kTT + kTTPad];
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kTT;
+  const int c0 = blockIdx.y * kTT;  // 64 columns never straddle two sub-tables (d % 64 == 0)
   const int s = c0 / p.d;
   const int j0 = c0 - s * p.d;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int64_t i = i0 + ty + 8 * k;
-    uint16_t v = 0;
-    if (i < p.T) {
-      int32_t r = p.idx[i * p.S + s];
-      if (static_cast<uint32_t>(r) >= p.Vs[s]) {
-        if (tx == 0) set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
-        r = 0;
-      }
-      v = p.E[s][static_cast<int64_t>(r) * p.d + j0 + tx];
-    }
-    tile[ty + 8 * k][tx] = v;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int c = c0 + ty + 8 * k;
-    const int64_t i = i0 + tx;
-    if (i < p.T_pad) p.dst[static_cast<int64_t>(c) * p.T_pad + i] = tile[tx][ty + 8 * k];
-  }
+  transpose_tile(
+      tile,
+      [&](int r) -> const uint16_t* {
+        const int64_t i = i0 + r;
+        if (i >= p.T) return nullptr;
+        int32_t row = p.idx[i * p.S + s];
+        if (static_cast<uint32_t>(row) >= p.Vs[s]) {
+          set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+          row = 0;
+        }
+        return p.E[s] + static_cast<int64_t>(row) * p.d + j0;
+      },
+      p.dst + static_cast<int64_t>(c0) * p.T_pad, p.T_pad, i0, kTT, p.T_pad);
 }
 
 // ------------------------------------------------------------------ dE_0 scatter

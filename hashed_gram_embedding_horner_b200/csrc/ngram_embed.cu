@@ -904,7 +904,7 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     tp.R = D;
     tp.R_pad = D;
     tp.C = D;
-    if ((rc = launch(transpose_bf16_kernel, dim3(D / 32, D / 32), dim3(256), 0, st, p->pdl, 1, tp))) return rc;
+    if ((rc = launch(transpose_bf16_kernel, dim3(D / kTT, D / kTT), dim3(256), 0, st, p->pdl, 1, tp))) return rc;
     DenseParams dp{};
     dp.scale = scale;
     dp.epi = kEpiScatterSub;
@@ -929,8 +929,8 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     tp.R = T;
     tp.R_pad = T8;
     tp.C = D;
-    if ((rc = launch(transpose_bf16_kernel, dim3(static_cast<unsigned>((T8 + 31) / 32), D / 32), dim3(256), 0, st,
-                     p->pdl, 1, tp)))
+    if ((rc = launch(transpose_bf16_kernel, dim3(static_cast<unsigned>((T8 + kTT - 1) / kTT), D / kTT), dim3(256), 0,
+                     st, p->pdl, 1, tp)))
       return rc;
     GatherTParams gp{};
     gp.idx = idx;
@@ -945,8 +945,8 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     gp.d = p->d;
     gp.D = D;
     gp.status = status_ptr(workspace);
-    if ((rc = launch(gather_transpose_kernel, dim3(static_cast<unsigned>((T8 + 31) / 32), D / 32), dim3(256), 0, st,
-                     p->pdl, 1, gp)))
+    if ((rc = launch(gather_transpose_kernel, dim3(static_cast<unsigned>((T8 + kTT - 1) / kTT), D / kTT), dim3(256),
+                     0, st, p->pdl, 1, gp)))
       return rc;
     DenseParams dp{};
     dp.scale = scale;
