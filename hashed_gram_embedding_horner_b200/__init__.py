@@ -46,6 +46,7 @@ EXPORTED = [
     "ngram_embed_bwd_workspace_bytes", "ngram_embed_bwd",
     "ngram_hash_stats_workspace_bytes", "ngram_hash_stats",
     "ngram_draft_cache_reset", "ngram_embed_draft_workspace_bytes", "ngram_embed_fwd_draft",
+    "ngram_embed_fwd_step",
 ]
 
 
@@ -94,6 +95,7 @@ _sig("ngram_embed_plan_set_output_scale", [_P, ctypes.c_float])
 _sig("ngram_embed_bwd_workspace_bytes", [_P, _I64], _SZ)
 _sig("ngram_hash_stats_workspace_bytes", [_I64, _I64, ctypes.c_int], _SZ)
 _sig("ngram_draft_cache_reset", [_P, _P, _P, _I32, _P, _SZ, _P])
+_sig("ngram_embed_fwd_step", [_P, _P, _I32, _P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P])
 _sig("ngram_embed_draft_workspace_bytes", [_P, _I64], _SZ)
 _sig("ngram_embed_fwd_draft", [_P, _P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P])
 _sig("ngram_hash_stats", [_I64, ctypes.c_int, _P, _P, _I32, _I64, _P, ctypes.c_int, _P, _P, _P, _SZ, _P])
@@ -177,6 +179,21 @@ class DraftCache:
         dt = torch.bfloat16 if plan.dtype == NGRAM_BF16 else torch.float32
         return cls(torch.full((max_seqs, positions, plan.N), -1, dtype=torch.int32, device=device),
                    torch.zeros((max_seqs, positions, plan.D), dtype=dt, device=device))
+
+
+def ngram_embed_fwd_step(plan: "Plan", tokens, seq_offsets, E0, E_nk, W_stacked, out, workspace, cache: "Cache",
+                         commit_tokens=None, commit_stride: int = 0, commit_counts=None, cache_slots=None,
+                         stream=None):
+    """Commit the previous step's accepted ids (if commit_counts is given), then the layer
+    for this step's ids through the N-gram cache: two launches."""
+    tabs = _tables(E_nk)
+    rc = _lib.ngram_embed_fwd_step(plan.handle, _i32(commit_tokens, "commit_tokens"), int(commit_stride),
+                                   _i32(commit_counts, "commit_counts"), _i32(tokens, "tokens"),
+                                   _i32(seq_offsets, "seq_offsets"), seq_offsets.numel() - 1, tokens.numel(),
+                                   _ptr(E0), tabs, _ptr(W_stacked), ctypes.byref(cache.struct),
+                                   _i32(cache_slots, "cache_slots"), _ptr(out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "ngram_embed_fwd_step")
 
 
 def ngram_draft_cache_reset(plan: "Plan", dc: DraftCache, workspace, slots=None, stream=None):

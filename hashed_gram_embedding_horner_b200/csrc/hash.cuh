@@ -49,6 +49,54 @@ __device__ __forceinline__ uint32_t horner_step(uint32_t h, uint32_t V0, uint32_
   return static_cast<uint32_t>(r);
 }
 
+// Eq. 2 for token i of a sequence starting at `start`, with the sequence's committed
+// history (slot >= 0: hist_len ids, those before hist_from evicted) before it.
+__device__ __forceinline__ void hash_one(const HashParams& p, int64_t i, int64_t start, int32_t slot,
+                                         int64_t hist_len, int64_t hist_from) {
+  // u[j] = t_{i-j}, newest first.
+  uint32_t u[kMaxN];
+#pragma unroll
+  for (int j = 0; j < kMaxN; ++j) {
+    if (j >= p.N) break;
+    const int64_t a = i - j;  // absolute token position if inside this call's sequence
+    int64_t t = 0;
+    if (a >= start && a >= 0) {
+      t = p.tokens[a];
+    } else if (slot >= 0) {
+      const int64_t pos = hist_len + (a - start);  // position in the committed history
+      if (pos >= 0) {
+        if (pos < hist_from) {
+          set_status(p.status, NGRAM_STATUS_EVICTED);
+        } else {
+          t = p.ring[static_cast<int64_t>(slot) * p.capacity + (pos % p.capacity)];
+        }
+      }
+    }
+    if (t < 0 || t >= p.V0) {
+      set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+      t = 0;
+    }
+    u[j] = static_cast<uint32_t>(t);
+  }
+
+  if (p.win_out) {
+    for (int j = 0; j < p.N; ++j) p.win_out[i * p.N + j] = static_cast<int32_t>(u[p.N - 1 - j]);
+    const int64_t jpos = i - start;
+    p.entry_out[i] = (slot >= 0 && jpos < p.positions) ? static_cast<int32_t>(slot * p.positions + jpos) : -1;
+  }
+  int32_t* out = p.idx_out + i * p.S;
+  for (int n = 2; n <= p.N; ++n) {
+    for (int k = 0; k < p.K; ++k) {
+      const int s = (n - 2) * p.K + k;
+      const uint32_t V = p.V[s];
+      const uint64_t m = p.barrett[s];
+      uint32_t h = 0;
+      for (int j = n - 1; j >= 0; --j) h = horner_step(h, p.V0, u[j], V, m);
+      out[s] = static_cast<int32_t>(h);
+    }
+  }
+}
+
 constexpr int kHashSmemOffsets = 4096;  // offsets staged in shared memory when B + 1 fits
 
 __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashParams p) {
@@ -94,48 +142,7 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashP
     }
   }
 
-  // u[j] = t_{i-j}, newest first.
-  uint32_t u[kMaxN];
-#pragma unroll
-  for (int j = 0; j < kMaxN; ++j) {
-    if (j >= p.N) break;
-    const int64_t a = i - j;  // absolute token position if inside this call's sequence
-    int64_t t = 0;
-    if (a >= start && a >= 0) {
-      t = p.tokens[a];
-    } else if (slot >= 0) {
-      const int64_t pos = hist_len + (a - start);  // position in the committed history
-      if (pos >= 0) {
-        if (pos < hist_from) {
-          set_status(p.status, NGRAM_STATUS_EVICTED);
-        } else {
-          t = p.ring[static_cast<int64_t>(slot) * p.capacity + (pos % p.capacity)];
-        }
-      }
-    }
-    if (t < 0 || t >= p.V0) {
-      set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
-      t = 0;
-    }
-    u[j] = static_cast<uint32_t>(t);
-  }
-
-  if (p.win_out) {
-    for (int j = 0; j < p.N; ++j) p.win_out[i * p.N + j] = static_cast<int32_t>(u[p.N - 1 - j]);
-    const int64_t jpos = i - start;
-    p.entry_out[i] = (slot >= 0 && jpos < p.positions) ? static_cast<int32_t>(slot * p.positions + jpos) : -1;
-  }
-  int32_t* out = p.idx_out + i * p.S;
-  for (int n = 2; n <= p.N; ++n) {
-    for (int k = 0; k < p.K; ++k) {
-      const int s = (n - 2) * p.K + k;
-      const uint32_t V = p.V[s];
-      const uint64_t m = p.barrett[s];
-      uint32_t h = 0;
-      for (int j = n - 1; j >= 0; --j) h = horner_step(h, p.V0, u[j], V, m);
-      out[s] = static_cast<int32_t>(h);
-    }
-  }
+  hash_one(p, i, start, slot, hist_len, hist_from);
 }
 
 }  // namespace ngram

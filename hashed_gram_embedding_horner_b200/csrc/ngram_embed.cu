@@ -25,6 +25,7 @@
 #include "bwd_sm100.cuh"
 #include "stats.cuh"
 #include "draft.cuh"
+#include "decode.cuh"
 
 using namespace ngram;
 
@@ -1056,6 +1057,66 @@ int ngram_embed_fwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     rc = launch_hash(plan, tokens, seq_offsets, num_seqs, num_tokens, cache, cache_slots, idx, workspace, st);
     if (rc) return rc;
   }
+  return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace, workspace_bytes, num_tokens,
+                 st);
+}
+
+int ngram_embed_fwd_step(const ngram_embed_plan* plan_c, const int32_t* commit_tokens, int32_t commit_stride,
+                         const int32_t* commit_counts, const int32_t* tokens, const int32_t* seq_offsets,
+                         int32_t num_seqs, int64_t num_tokens, const void* E0, const void* const* E_nk,
+                         const void* W_stacked, const ngram_cache* cache, const int32_t* cache_slots, void* out,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  auto* plan = const_cast<ngram_embed_plan*>(plan_c);
+  int rc = validate_common(plan, workspace, workspace_bytes, num_tokens);
+  if (rc) return rc;
+  if (num_seqs < 1 || !cache || !tokens || !seq_offsets || (num_tokens > 0 && !out)) return NGRAM_ERR_INVALID_ARG;
+  if (commit_counts && (!commit_tokens || commit_stride < 1)) return NGRAM_ERR_INVALID_ARG;
+  if (num_tokens > 0 && !aligned16(out)) return NGRAM_ERR_MISALIGNED;
+  if ((rc = check_tables(plan, E0, E_nk, W_stacked))) return rc;
+  if ((rc = validate_cache(plan, cache))) return rc;
+  if (num_seqs > cache->max_seqs && !cache_slots) return NGRAM_ERR_INVALID_ARG;
+  if ((rc = set_device(plan))) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* idx = idx_ptr(workspace);
+  CacheParams c{};
+  c.ring = cache->ring;
+  c.len = cache->len;
+  c.valid_from = cache->valid_from;
+  c.capacity = cache->capacity;
+  c.max_seqs = cache->max_seqs;
+  c.N = plan->N;
+  c.V0 = static_cast<uint32_t>(plan->V0);
+  c.slots = cache_slots;
+  c.tokens = commit_tokens;
+  c.counts = commit_counts;
+  c.stride = commit_stride;
+  c.n = num_seqs;
+  c.status = status_ptr(workspace);
+  HashParams h{};
+  h.tokens = tokens;
+  h.offsets = seq_offsets;
+  h.num_seqs = num_seqs;
+  h.T = num_tokens;
+  h.V0 = static_cast<uint32_t>(plan->V0);
+  h.N = plan->N;
+  h.K = plan->K;
+  h.S = plan->S;
+  for (int s = 0; s < plan->S; ++s) {
+    h.V[s] = static_cast<uint32_t>(plan->V[s]);
+    h.barrett[s] = plan->barrett[s];
+  }
+  h.ring = cache->ring;
+  h.len = cache->len;
+  h.valid_from = cache->valid_from;
+  h.capacity = cache->capacity;
+  h.max_seqs = cache->max_seqs;
+  h.slots = cache_slots;
+  h.idx_out = idx;
+  h.status = status_ptr(workspace);
+  if ((rc = launch(commit_hash_kernel, dim3(static_cast<unsigned>((num_seqs + 7) / 8)), dim3(256), 0, st,
+                   plan->pdl, 1, c, h)))
+    return rc;
+  if (num_tokens == 0) return NGRAM_OK;
   return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace, workspace_bytes, num_tokens,
                  st);
 }

@@ -312,12 +312,9 @@ __global__ void cache_reset_kernel(const __grid_constant__ CacheParams p) {
 
 // One warp per entry: write the ids at positions len .. len+m-1 (slot pos % C), then
 // len += m and valid_from = max(valid_from, len - C). Rejected entries change nothing.
-__global__ void cache_append_kernel(const __grid_constant__ CacheParams p) {
-  pdl_launch_dependents();
-  pdl_wait();
-  const int32_t i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (i >= p.n) return;
+// One warp appends entry i's ids (CSR entries, or the first counts[i] of a fixed stride)
+// to its slot's ring: the N-gram cache update of a commit.
+__device__ __forceinline__ void append_entry(const CacheParams& p, int32_t i, int lane) {
   int32_t s = -1;
   if (lane == 0) s = entry_slot(p, i);
   s = __shfl_sync(0xffffffffu, s, 0);
@@ -348,6 +345,15 @@ __global__ void cache_append_kernel(const __grid_constant__ CacheParams p) {
     const int64_t vf = nl - p.capacity;
     if (vf > p.valid_from[s]) p.valid_from[s] = vf;
   }
+}
+
+__global__ void cache_append_kernel(const __grid_constant__ CacheParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int32_t i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (i >= p.n) return;
+  append_entry(p, i, lane);
 }
 
 // One thread per entry: drop the newest counts[i] ids if the ring still holds the

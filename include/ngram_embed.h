@@ -135,6 +135,18 @@ int ngram_embed_fwd(const ngram_embed_plan* plan, const int32_t* tokens,
                     const ngram_cache* cache, const int32_t* cache_slots, void* out,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* One speculative-decode step in two launches instead of three: the commit of the previous
+ * step's accepted ids (exactly ngram_cache_commit(commit_tokens, commit_stride,
+ * commit_counts), skipped if commit_counts is NULL) fused with this step's context hashing,
+ * then the projection — the same results as ngram_cache_commit followed by ngram_embed_fwd
+ * with the cache. Sequence b's slot is cache_slots[b] (or b) for both parts. */
+int ngram_embed_fwd_step(const ngram_embed_plan* plan, const int32_t* commit_tokens,
+                         int32_t commit_stride, const int32_t* commit_counts, const int32_t* tokens,
+                         const int32_t* seq_offsets, int32_t num_seqs, int64_t num_tokens,
+                         const void* E0, const void* const* E_nk, const void* W_stacked,
+                         const ngram_cache* cache, const int32_t* cache_slots, void* out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* Eq. 2 alone (context assembly + hash): idx_out[i * S + s] = H_{n,k}(...) as int32,
  * bit-exact. Arguments as for ngram_embed_fwd; idx_out is [num_tokens x S] device. */
 int ngram_hash_indices(const ngram_embed_plan* plan, const int32_t* tokens,

@@ -190,3 +190,37 @@ def test_evicted_context_is_flagged(ne):
     cache.valid_from.fill_(5)
     ne.ngram_hash_indices(plan, dev_i32([9]), dev_i32([0, 1]), idx, ws, cache=cache)
     assert ne.status_names(ne.ngram_embed_get_status(ws)) == ["EVICTED"]
+
+
+def test_fused_commit_and_step_equals_separate_calls(ne):
+    """ngram_embed_fwd_step (commit of the previous step fused with this step's hashing) gives
+    the same outputs, bit for bit, and the same ring as ngram_cache_commit + ngram_embed_fwd."""
+    from tests.helpers import host_tables, to_device
+    N, K, D, B, P, C = 3, 2, 512, 24, 5, 8
+    V0, V = 3000, [4099, 5003, 6007, 7001]
+    cfg = configs.NgramConfig(name="step", V0=V0, D=D, N=N, K=K, V_nk=tuple(V), dtype="bf16", seed=13)
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = ne.ngram_embed_plan_create(V0, D, N, K, V, ne.NGRAM_BF16)
+    ws1, ws2 = ne.new_workspace(plan, B * P), ne.new_workspace(plan, B * P)
+    c1, c2 = ne.Cache.empty(B, C), ne.Cache.empty(B, C)
+    for c, w in ((c1, ws1), (c2, ws2)):
+        ne.ngram_cache_reset(plan, c, w)
+    rng = np.random.default_rng(21)
+    off = dev_i32(np.arange(B + 1) * P)
+    prev = None
+    for step in range(6):
+        tok = dev_i32(rng.integers(0, V0, B * P))
+        cnt = dev_i32(1 + rng.integers(0, P, B))
+        o1 = torch.empty((B * P, D), dtype=torch.bfloat16, device="cuda")
+        o2 = torch.empty_like(o1)
+        if prev is not None:
+            ne.ngram_cache_commit(plan, c1, prev[0], P, prev[1], ws1)
+        ne.ngram_embed_fwd(plan, tok, off, E0, E, W, o1, ws1, cache=c1)
+        ne.ngram_embed_fwd_step(plan, tok, off, E0, E, W, o2, ws2, c2,
+                                commit_tokens=None if prev is None else prev[0], commit_stride=P,
+                                commit_counts=None if prev is None else prev[1])
+        assert torch.equal(o1, o2), step
+        assert torch.equal(c1.ring, c2.ring) and torch.equal(c1.len, c2.len) and torch.equal(c1.valid_from, c2.valid_from)
+        prev = (tok, cnt)
+    assert ne.ngram_embed_get_status(ws1) == 0 and ne.ngram_embed_get_status(ws2) == 0
