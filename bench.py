@@ -498,7 +498,8 @@ def main():
     flops = 2.0 * T * cfg.D * cfg.D
     achieved = flops / (proj_ms / 1e3) / 1e12
     form = ne.ngram_embed_plan_kernel_form(plan, T)
-    kernel_name = {"cta_pair": "proj_sm100_pair_kernel", "one_cta": "proj_sm100_kernel",
+    kernel_name = {"cta_pair": "proj_sm100_pair_kernel", "cta_pair_wide": "proj_sm100_pair_kernel",
+                   "one_cta": "proj_sm100_kernel",
                    "one_cta_stream_k": "proj_sm100_kernel", "cuda_cores": "proj_simt_kernel"}[form]
     algo_bytes = T * (2 * cfg.D * 2 + 4) + cfg.D * cfg.D * 2
 

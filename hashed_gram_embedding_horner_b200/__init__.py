@@ -41,7 +41,7 @@ EXPORTED = [
     "ngram_embed_plan_set_variant", "ngram_embed_plan_set_tile_n", "ngram_embed_plan_set_tma_rows",
     "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws", "ngram_embed_plan_set_cta_pair",
     "ngram_cache_commit", "ngram_embed_plan_set_stream_k", "ngram_embed_plan_set_pdl",
-    "ngram_embed_plan_set_a_stages", "ngram_embed_plan_kernel_form",
+    "ngram_embed_plan_set_a_stages", "ngram_embed_plan_kernel_form", "ngram_embed_plan_set_pair_wide",
     "ngram_embed_plan_set_output_scale", "ngram_embed_layernorm",
     "ngram_embed_bwd_workspace_bytes", "ngram_embed_bwd",
     "ngram_hash_stats_workspace_bytes", "ngram_hash_stats",
@@ -87,6 +87,7 @@ _sig("ngram_embed_plan_set_variant", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tile_n", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_pair_wide", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_a_stages", [_P, ctypes.c_int])
@@ -248,6 +249,12 @@ def ngram_embed_plan_set_cta_pair(plan: Plan, on):
     _check(_lib.ngram_embed_plan_set_cta_pair(plan.handle, v), "ngram_embed_plan_set_cta_pair")
 
 
+def ngram_embed_plan_set_pair_wide(plan: Plan, on):
+    """True/1: the pair form's 512-column tiles; False/0: 256-column; None/-1: automatic."""
+    v = -1 if on is None or on == -1 else int(bool(on))
+    _check(_lib.ngram_embed_plan_set_pair_wide(plan.handle, v), "ngram_embed_plan_set_pair_wide")
+
+
 def ngram_embed_plan_set_stream_k(plan: Plan, mode: int):
     """0 automatic, 1 stream-K whenever the workspace and shape allow it, 2 never."""
     _check(_lib.ngram_embed_plan_set_stream_k(plan.handle, int(mode)), "ngram_embed_plan_set_stream_k")
@@ -306,7 +313,7 @@ def ngram_hash_stats(V0: int, n: int, tokens, seq_offsets, moduli, workspace=Non
     return (None if dist.value < 0 else int(dist.value)), [int(h) for h in hits]
 
 
-KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair"}
+KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair", 4: "cta_pair_wide"}
 
 
 def ngram_embed_plan_kernel_form(plan: Plan, num_tokens: int) -> str:

@@ -67,7 +67,8 @@ struct ngram_embed_plan {
   int stream_k = 0;            // one-CTA kernel schedule: 0 automatic, 1 stream-K when possible, 2 never
   bool pdl = false;            // launch as programmatic dependent launches
   float out_scale = 1.0f;      // embedding amplification factor folded into the 1/(S+1) scale
-  int max_clusters[2] = {0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
+  int pair_wide = -1;          // pair form with 512-column tiles: 1 on, 0 off, -1 automatic
+  int max_clusters[3] = {0, 0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
 };
 
 namespace {
@@ -252,7 +253,7 @@ int launch_tc_pair_stages(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaSt
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int& max_pairs = p->max_clusters[BN == 256 ? 1 : 0];
+  int& max_pairs = p->max_clusters[BN == 512 ? 2 : (BN == 256 ? 1 : 0)];
   if (max_pairs == 0) {
     cfg.gridDim = dim3(2 * (p->sms / 2));
     int n = 0;
@@ -267,6 +268,23 @@ template <int BN>
 int launch_tc_pair(ngram_embed_plan* p, const ProjParams& prm, int64_t T, cudaStream_t st) {
   if (BN == 256) return launch_tc_pair_stages<256, kPairStages256>(p, prm, T, st, 7);
   return launch_tc_pair_stages<128, kPairStages128>(p, prm, T, st, 6);
+}
+
+// The pair form's 512-column tiles (two N = 256 MMAs per A stage): needs 256-column W
+// halves and D % 512 == 0. Automatic: whichever width finishes its whole waves of tiles
+// sooner, a 256-column tile costing 0.57 of a 512-column one (measured on B200 at T = 32768
+// and 65536: 0.54 at D = 2048, 0.61 at D = 4096), so small grids keep the narrow tiles
+// that occupy more SMs. Not automatic when the token count is known only on the device (a
+// draft call's misses: usually a few tiles, for which the narrow tiles keep more SMs busy).
+bool use_pair_wide(const ngram_embed_plan* p, int64_t T, bool count_on_device = false) {
+  if (p->bn != 256 || p->D % 512 != 0 || p->pair_wide == 0) return false;
+  if (p->pair_wide == 1) return true;
+  if (p->sms < 2 || count_on_device) return false;  // no device: the SM count is unknown
+  const int64_t pairs = p->sms / 2;
+  const int64_t wide_tiles = (T + 2 * kBM - 1) / (2 * kBM) * (p->D / 512);
+  const int64_t waves_wide = (wide_tiles + pairs - 1) / pairs;
+  const int64_t waves_narrow = (2 * wide_tiles + pairs - 1) / pairs;
+  return static_cast<double>(waves_wide) <= 0.57 * static_cast<double>(waves_narrow);
 }
 
 
@@ -471,6 +489,11 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   // A rows by TMA gather4 in the pair form, by cp.async in the one-CTA form (measured
   // fastest for each), unless the plan fixes the split.
   prm.tma_rows = p->variant == kTcTmaRows ? kBM : (p->tma_rows >= 0 ? p->tma_rows : (pair ? kBM : 0));
+  if (pair && use_pair_wide(p, T, T_dev != nullptr)) {
+    prm.num_n_blocks = p->D / 512;
+    prm.tma_rows = kBM;  // A rows by gather4 only
+    return launch_tc_pair_stages<512, kPairStagesWide>(p, prm, T, st, 8);
+  }
   if (pair) return p->bn == 256 ? launch_tc_pair<256>(p, prm, T, st) : launch_tc_pair<128>(p, prm, T, st);
   if (sk) {
     prm.stream_k = 1;
@@ -601,8 +624,14 @@ int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_token
   prm.num_n_blocks = plan->D / plan->bn;
   prm.num_k_blocks = plan->D / kBK;
   const bool sk = plan->cta_pair != 1 && use_stream_k(plan, prm, num_tokens, ws_bytes(plan, num_tokens));
-  if (plan->cta_pair == 1 || (plan->cta_pair == -1 && !sk)) return 3;
+  if (plan->cta_pair == 1 || (plan->cta_pair == -1 && !sk)) return use_pair_wide(plan, num_tokens) ? 4 : 3;
   return sk ? 2 : 1;
+}
+
+int ngram_embed_plan_set_pair_wide(ngram_embed_plan* plan, int on) {
+  if (!plan || on < -1 || on > 1) return NGRAM_ERR_INVALID_ARG;
+  plan->pair_wide = on;
+  return NGRAM_OK;
 }
 
 // Tensor-core tile width: 256 or 128 output columns per tile (D must divide).

@@ -36,17 +36,30 @@ constexpr int kWarpRelay = 10;
 // barrier traffic of the cluster-scope waits and commits; a 7th stage gained nothing).
 constexpr int kPairStages256 = 6;
 constexpr int kPairStages128 = 8;
+constexpr int kPairStagesWide = 4;  // BN = 512: 16 KB of A + 32 KB of W per stage
 
+// BN <= 256: one MMA of N = BN per k-step, two accumulators (2 x BN TMEM columns) so the
+// epilogue of one tile overlaps the main loop of the next.
+// BN = 512 ("wide"): two MMAs of N = 256 per k-step (halves h = 0, 1 of the tile's columns)
+// on the same A stage, so every gathered A row feeds twice the columns; the accumulator
+// takes all 512 TMEM columns, each half drained by its own four epilogue warps (warps 12-15
+// and 4-7; the A rows come by gather4 from warps 0-3) and freed on its own barrier, so the
+// next tile's MMAs into half h wait only for that half.
 template <int BN, int STAGES>
 struct PairSmem {
+  static constexpr bool kWide = BN > 256;
+  static constexpr int kHalves = kWide ? 2 : 1;
+  static constexpr int kMmaN = BN / kHalves;            // N of one MMA
   static constexpr int kABytes = kBM * kBK * 2;         // this CTA's 128 A rows
-  static constexpr int kBBytes = (BN / 2) * kBK * 2;    // this CTA's BN/2 rows of W
+  static constexpr int kBSubBytes = (kMmaN / 2) * kBK * 2;  // this CTA's rows of one MMA's B
+  static constexpr int kBBytes = kHalves * kBSubBytes;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarOffset = STAGES * kStageBytes;
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kBytes = kBarOffset + kNumBars * 8 + 16;
   static constexpr int kLaunchBytes = kBytes + 1024;
-  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kTmemCols = kWide ? 512 : 2 * BN;
+  static_assert(kTmemCols <= 512, "accumulators exceed TMEM");
 };
 
 template <int BN, int STAGES>
@@ -73,7 +86,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int num_pairs = static_cast<int>(gridDim.x >> 1);
 
-  const bool cp_rows = p.tma_rows == 0;  // A rows by cp.async (else all by TMA gather4)
+  constexpr bool kWide = L::kWide;
+  constexpr int kMmaN = L::kMmaN;
+  const bool cp_rows = !kWide && p.tma_rows == 0;  // A rows by cp.async (else all by TMA gather4)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       // CTA 0: thread 0 posts the pair's TMA bytes (+ its 256 cp.async threads + CTA 1's relay);
@@ -110,13 +125,15 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   const int KB = p.num_k_blocks;
   const int kb_per_sub = p.d / kBK;
 
-  if (warp < kAWarps) {
+  const bool epi_warp = warp >= kWarpEpi0 || (kWide && warp >= kAWarps / 2 && warp < kAWarps);
+  if (warp < kAWarps && !epi_warp) {
     // ------------------------------------------------------------ A producers (own 128 rows)
     const int t = threadIdx.x;
     const int chunk = t & 7, rsub = t >> 3;                         // cp.async mode
     const uint32_t swz = static_cast<uint32_t>((chunk ^ (rsub & 7)) << 4);
-    const bool issuer = !cp_rows && lane < 4;                       // gather4 mode: 32 lanes x 4 rows
-    const int iss = warp * 4 + lane;
+    // gather4 mode: 32 issuing lanes x 4 rows (wide: lanes 0-7 of warps 0-3, else 0-3 of 0-7)
+    const bool issuer = !cp_rows && lane < (kWide ? 8 : 4);
+    const int iss = kWide ? warp * 8 + lane : warp * 4 + lane;
     const uint32_t pair_tx = cp_rows ? 2u * L::kBBytes : 2u * (L::kABytes + L::kBBytes);
     const uint64_t pol = l2_policy_evict_normal();
     // raw row indices (this thread's 4 rows) of the current and the next run
@@ -186,8 +203,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           int kb = i + rot;
           if (kb >= KB) kb -= KB;
           if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          tma_load_2d_pair(b_tile(stage), &maps.Whalf, kb * kBK, n_blk * BN + static_cast<int>(rank) * (BN / 2),
-                           map_to_cta(full_bar(stage), 0), pol);
+#pragma unroll
+          for (int h = 0; h < L::kHalves; ++h)
+            tma_load_2d_pair(b_tile(stage) + h * L::kBSubBytes, &maps.Whalf, kb * kBK,
+                             n_blk * BN + h * kMmaN + static_cast<int>(rank) * (kMmaN / 2),
+                             map_to_cta(full_bar(stage), 0), pol);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -195,31 +215,46 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer (CTA 0)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(2 * kBM, BN);
+      constexpr uint32_t idesc = umma_idesc_bf16(2 * kBM, kMmaN);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int local = 0;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
-        const int acc = local & 1;
-        const uint32_t use = static_cast<uint32_t>(local >> 1);
-        if (!mbar_wait_cluster(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
+        // one accumulator of both halves (wide), else two alternating ones
+        const int acc = kWide ? 0 : (local & 1);
+        const uint32_t use = static_cast<uint32_t>(kWide ? local : local >> 1);
+        if (!kWide) {
+          if (!mbar_wait_cluster(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+        }
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int i = 0; i < KB; ++i) {
+        for (int i = 0; i < KB && ok; ++i) {
           if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           if (cp_rows) fence_proxy_async_smem();  // this CTA's cp.async rows: generic proxy writes
           const uint64_t adesc = sw128_kmajor_desc(a_tile(stage));
-          const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage));
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
+          for (int h = 0; h < L::kHalves; ++h) {
+            if (kWide && i == 0) {  // half h of the previous tile drained
+              if (!mbar_wait_cluster(tempty_bar(h), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+              tc_fence_after();
+            }
+            const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage) + h * L::kBSubBytes);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+              umma_bf16_pair(d_tmem + h * kMmaN, adesc + 2u * k, bdesc + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
+            if (kWide && i + 1 == KB) {  // half h complete: its epilogue may start
+              umma_commit_pair(map_to_cta(tfull_bar(h), 0));
+              umma_commit_pair(map_to_cta(tfull_bar(h), 1));
+            }
+          }
+          if (!ok) break;
           umma_commit_pair(map_to_cta(empty_bar(stage), 0));
           umma_commit_pair(map_to_cta(empty_bar(stage), 1));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (ok) {
+        if (ok && !kWide) {
           umma_commit_pair(map_to_cta(tfull_bar(acc), 0));
           umma_commit_pair(map_to_cta(tfull_bar(acc), 1));
         }
@@ -243,9 +278,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         phase ^= 1u;
       }
     }
-  } else if (warp >= kWarpEpi0) {
+  } else if (epi_warp) {
     // ------------------------------------------------------------ epilogue (own 128 rows)
-    const int q = warp & 3;
+    const int q = warp & 3;  // TMEM lanes q*32 .. q*32+31 (warp w reaches quadrant w % 4)
+    const int half = kWide && warp < kWarpEpi0 ? 1 : 0;  // wide: warps 4-7 drain columns 256-511
     const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_remote0 = map_to_cta(tempty_bar(0), 0);
     const uint32_t tempty_remote1 = map_to_cta(tempty_bar(1), 0);
@@ -253,8 +289,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
       const int m_blk = tile / p.num_n_blocks;
       const int n_blk = tile % p.num_n_blocks;
-      const int acc = local & 1;
-      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const int acc = kWide ? half : (local & 1);
+      const uint32_t use = static_cast<uint32_t>(kWide ? local : local >> 1);
+      const int col0 = n_blk * BN + half * kMmaN;
       const int64_t gr = static_cast<int64_t>(m_blk) * (2 * kBM) + rank * kBM + row_in_tile;
       const bool valid = gr < T;
       uint32_t t = 0;
@@ -262,8 +299,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const int32_t tok = p.tokens[gr];
         t = (tok >= 0 && static_cast<uint32_t>(tok) < p.V0) ? static_cast<uint32_t>(tok) : 0u;
       }
-      const uint4* e0 = reinterpret_cast<const uint4*>(p.E0 + static_cast<int64_t>(t) * p.D + n_blk * BN);
-      uint4* dst = reinterpret_cast<uint4*>(p.out + gr * p.D + n_blk * BN);
+      const uint4* e0 = reinterpret_cast<const uint4*>(p.E0 + static_cast<int64_t>(t) * p.D + col0);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + gr * p.D + col0);
       uint4 ecur[4];
 #pragma unroll
       for (int v = 0; v < 4; ++v) ecur[v] = valid ? __ldg(e0 + v) : make_uint4(0, 0, 0, 0);
@@ -272,18 +309,18 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       if (lane == 0) got = mbar_wait_cluster(tfull_bar(acc), use & 1u, abort_flag, p.status);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kMmaN);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < kMmaN / 32; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + c * 32, v);
         uint4 enext[4];
-        const bool has_next = c + 1 < BN / 32;
+        const bool has_next = c + 1 < kMmaN / 32;
 #pragma unroll
         for (int w = 0; w < 4; ++w)
           enext[w] = (valid && has_next) ? __ldg(e0 + (c + 1) * 4 + w) : make_uint4(0, 0, 0, 0);
         tmem_wait_ld();
-        if (c + 1 == BN / 32) {
+        if (c + 1 == kMmaN / 32) {
           tc_fence_before();
           if (rank == 0) {
             mbar_arrive(tempty_bar(acc));

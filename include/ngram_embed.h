@@ -348,9 +348,18 @@ int ngram_embed_plan_set_tma_rows(ngram_embed_plan* plan, int rows);
  * (the k-block order differs). */
 int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on);
 
+/* CTA-pair form with 512-column tiles: each pair gathers a 256-row A block once per k-block
+ * and issues two tcgen05 MMAs of N = 256 on it (half the gathered rows per FLOP of the
+ * 256-column tiles); the accumulator fills all 512 TMEM columns and each half is drained and
+ * freed separately. Applies when the tile width is 256 and D % 512 == 0, with A rows by TMA
+ * gather4. 1 = on, 0 = off, -1 (default) = automatic. A tuning knob: results agree within
+ * the stated tolerance. NGRAM_ERR_INVALID_ARG for other values. */
+int ngram_embed_plan_set_pair_wide(ngram_embed_plan* plan, int on);
+
 /* The projection kernel a call of num_tokens tokens would run, given a workspace of
  * ngram_embed_workspace_bytes(plan, num_tokens): 0 = CUDA cores, 1 = one CTA per tile,
- * 2 = one CTA per SM with the stream-K schedule, 3 = CTA pairs; negative on bad arguments. */
+ * 2 = one CTA per SM with the stream-K schedule, 3 = CTA pairs, 4 = CTA pairs with
+ * 512-column tiles; negative on bad arguments. */
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens);
 
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */

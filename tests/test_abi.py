@@ -102,6 +102,12 @@ def test_plan_without_device_validates_then_fails_launch(ne):
     assert lib.ngram_embed_plan_kernel_form(h, 1280) == 3 and lib.ngram_embed_plan_kernel_form(h, -1) == -1
     assert lib.ngram_embed_plan_set_cta_pair(h, 0) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 1
     assert lib.ngram_embed_plan_set_cta_pair(h, -1) == 0 and lib.ngram_embed_plan_set_cta_pair(h, 2) == -1
+    # 512-column pair tiles (D = 2048 here): on when forced, automatic needs the SM count
+    assert lib.ngram_embed_plan_set_pair_wide(h, 2) == -1 and lib.ngram_embed_plan_set_pair_wide(h, -2) == -1
+    assert lib.ngram_embed_plan_set_pair_wide(h, 1) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 4
+    assert lib.ngram_embed_plan_set_tile_n(h, 128) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 3
+    assert lib.ngram_embed_plan_set_tile_n(h, 256) == 0
+    assert lib.ngram_embed_plan_set_pair_wide(h, -1) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 3
     assert lib.ngram_embed_plan_uses_tensor_cores(h) == 1
     bad_cache = ne._Cache(0, 0, 0, 4, 8)
     assert lib.ngram_cache_rollback(h, ctypes.byref(bad_cache), None, fake, 3, fake, ws_need, None) == -1

@@ -311,7 +311,17 @@ def test_full_size_prefill_sampled(ne, cfg):
     rows = sample_rows(offsets, T)
     want = oracle_rows(cfg, tokens, offsets, rows, host_W(cfg))
     assert_close(to_host_f64(out[torch.from_numpy(rows).cuda()]), want, what=cfg.name)
-    assert ne.ngram_embed_plan_kernel_form(plan, T) == "cta_pair"
+    assert ne.ngram_embed_plan_kernel_form(plan, T).startswith("cta_pair")
+    # the other pair tile width (256 or 512 columns) agrees with the oracle too
+    wide = ne.ngram_embed_plan_kernel_form(plan, T) == "cta_pair_wide"
+    ne.ngram_embed_plan_set_pair_wide(plan, 0 if wide else 1)
+    outw, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    assert_close(to_host_f64(outw[torch.from_numpy(rows).cuda()]), want, what=cfg.name + " other pair width")
+    del outw
+    ne.ngram_embed_plan_set_pair_wide(plan, 0)
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
     # other splits of the A rows between TMA and cp.async feed the MMAs the same tiles
     for tr in (64, 128):
         ne.ngram_embed_plan_set_tma_rows(plan, tr)
@@ -328,15 +338,59 @@ def test_full_size_prefill_sampled(ne, cfg):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("shape,lengths", [
+    ((5000, 512, 5, 2), RAGGED),                     # one m-block pair of tiles, ragged tail
+    ((4000, 512, 3, 4), RAGGED),
+    ((3000, 1536, 2, 3), [1, 0, 4096, 3000, 77]),    # 3 column tiles of 512
+    ((5000, 1024, 3, 2), [9000, 1, 7000, 5001, 3]),  # 166 tiles: pairs take several tiles each
+], ids=["D512N5K2", "D512N3K4", "D1536N2K3", "D1024N3K2_multi"])
+def test_pair_wide_matches_oracle(ne, shape, lengths):
+    """The pair form's 512-column tiles (two N = 256 MMAs per A stage, TMEM halves drained
+    and freed separately) against the oracle on every row, and against the 256-column pair
+    form (same products, other k-block rotation)."""
+    cfg = small_cfg(*shape)
+    tokens, offsets = ragged_tokens(cfg, lengths)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = plan_for(ne, cfg, pair=1)
+    ne.ngram_embed_plan_set_pair_wide(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == "cta_pair_wide"
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    assert_close(to_host_f64(out), want, what=cfg.name + " wide pair")
+    again, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0 and torch.equal(out, again)  # fixed order: repeatable bits
+    ne.ngram_embed_plan_set_pair_wide(plan, 0)
+    assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == "cta_pair"
+    narrow, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    assert (out.float() - narrow.float()).abs().max().item() <= 2e-2
+
+
+def test_pair_wide_not_for_narrow_tiles(ne):
+    """512-column tiles need D % 512 == 0 and 256-column W halves; otherwise the knob leaves
+    the 256- or 128-column pair form in place."""
+    plan = plan_for(ne, small_cfg(5000, 768, 3, 2), pair=1)
+    ne.ngram_embed_plan_set_pair_wide(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, 4096) == "cta_pair"
+    plan = plan_for(ne, small_cfg(5000, 1024, 3, 2), tile_n=128, pair=1)
+    ne.ngram_embed_plan_set_pair_wide(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, 4096) == "cta_pair"
+
+
 def test_automatic_kernel_form(ne):
-    """Prefill grids run the CTA-pair form; a 1280-token decode step at D = 4096 (160 tiles of
-    128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule."""
+    """Prefill grids run the CTA-pair form with 512-column tiles; a 1280-token decode step at
+    D = 4096 (160 tiles of 128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule;
+    a grid of one wave keeps the 256-column pair tiles (more SMs busy)."""
     for cfg in (configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN):
         plan = plan_for(ne, cfg)
-        assert ne.ngram_embed_plan_kernel_form(plan, 32768) == "cta_pair"
+        assert ne.ngram_embed_plan_kernel_form(plan, 32768) == "cta_pair_wide"
     plan = plan_for(ne, configs.SPEC_DECODE)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "one_cta_stream_k"
     assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"  # one wave: nothing to balance
+    assert ne.ngram_embed_plan_kernel_form(plan, 5120) == "cta_pair"   # 160 wide tiles: a thin 3rd wave
     assert ne.ngram_embed_plan_kernel_form(plan_for(ne, configs.TINY), 128) == "cuda_cores"
 
 
