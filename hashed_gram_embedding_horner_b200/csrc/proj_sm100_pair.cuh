@@ -56,7 +56,11 @@ struct PairSmem {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarOffset = STAGES * kStageBytes;
   static constexpr int kNumBars = 2 * STAGES + 5;
-  static constexpr int kBytes = kBarOffset + kNumBars * 8 + 16;
+  // epilogue staging: 32 rows x 32 fp32 columns per epilogue warp (8 warps wide, else 4)
+  static constexpr int kEpiWarps = kWide ? 8 : 4;
+  static constexpr int kEpiWarpBytes = 32 * 32 * 4;
+  static constexpr int kEpiOffset = (kBarOffset + kNumBars * 8 + 16 + 127) / 128 * 128;
+  static constexpr int kBytes = kEpiOffset + kEpiWarps * kEpiWarpBytes;
   static constexpr int kLaunchBytes = kBytes + 1024;
   static constexpr int kTmemCols = kWide ? 512 : 2 * BN;
   static_assert(kTmemCols <= 512, "accumulators exceed TMEM");
@@ -280,9 +284,21 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     }
   } else if (epi_warp) {
     // ------------------------------------------------------------ epilogue (own 128 rows)
+    // Per 32-column chunk: each lane reads its row's fp32 accumulators from TMEM (32x32b
+    // shape: lane = row) and writes them to this warp's staging area in shared memory; then
+    // four lanes per row read them back 8 columns each, add the E_0 slice, scale, round and
+    // store, so each global access instruction covers 8 rows x 64 contiguous bytes instead
+    // of 32 rows x 16 bytes (a quarter of the lines through L1 for the E_0 reads and the
+    // output writes). Same arithmetic per element: (acc + E_0) * scale, rounded once.
     const int q = warp & 3;  // TMEM lanes q*32 .. q*32+31 (warp w reaches quadrant w % 4)
     const int half = kWide && warp < kWarpEpi0 ? 1 : 0;  // wide: warps 4-7 drain columns 256-511
-    const int row_in_tile = q * 32 + lane;
+    const uint32_t stg = sbase + L::kEpiOffset + static_cast<uint32_t>(half * 4 + q) * L::kEpiWarpBytes;
+    const int rsub = lane >> 2, u2 = lane & 3;  // read-back: rows i*8 + rsub, columns u2*8 .. u2*8+7
+    // staging layout: row r at r*128 bytes, 16-byte unit w at ((w ^ (r & 7)) << 4): conflict-free
+    // for both the row-per-lane writes and the 4-lanes-per-row reads
+    const uint32_t row_w = stg + static_cast<uint32_t>(lane) * 128u;
+    const uint32_t rd_lo = stg + static_cast<uint32_t>(rsub) * 128u + (static_cast<uint32_t>((2 * u2) ^ rsub) << 4);
+    const uint32_t rd_hi = stg + static_cast<uint32_t>(rsub) * 128u + (static_cast<uint32_t>((2 * u2 + 1) ^ rsub) << 4);
     const uint32_t tempty_remote0 = map_to_cta(tempty_bar(0), 0);
     const uint32_t tempty_remote1 = map_to_cta(tempty_bar(1), 0);
     int local = 0;
@@ -292,35 +308,51 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       const int acc = kWide ? half : (local & 1);
       const uint32_t use = static_cast<uint32_t>(kWide ? local : local >> 1);
       const int col0 = n_blk * BN + half * kMmaN;
-      const int64_t gr = static_cast<int64_t>(m_blk) * (2 * kBM) + rank * kBM + row_in_tile;
-      const bool valid = gr < T;
-      uint32_t t = 0;
-      if (valid) {
-        const int32_t tok = p.tokens[gr];
-        t = (tok >= 0 && static_cast<uint32_t>(tok) < p.V0) ? static_cast<uint32_t>(tok) : 0u;
-      }
-      const uint4* e0 = reinterpret_cast<const uint4*>(p.E0 + static_cast<int64_t>(t) * p.D + col0);
-      uint4* dst = reinterpret_cast<uint4*>(p.out + gr * p.D + col0);
-      uint4 ecur[4];
+      const int64_t row0 = static_cast<int64_t>(m_blk) * (2 * kBM) + rank * kBM + q * 32;
+      // this lane's four read-back rows: E_0 and output addresses of its 8 columns
+      const uint4* e0r[4];
+      // output rows i*8 + rsub: row i is i * D / 8 vectors of 8 columns past row 0
+      uint4* dst0 = reinterpret_cast<uint4*>(p.out + (row0 + rsub) * p.D + col0 + u2 * 8);
+      bool valid[4];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) ecur[v] = valid ? __ldg(e0 + v) : make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 4; ++i) {
+        const int64_t gr = row0 + i * 8 + rsub;
+        valid[i] = gr < T;
+        uint32_t t = 0;
+        if (valid[i]) {
+          const int32_t tok = p.tokens[gr];
+          t = (tok >= 0 && static_cast<uint32_t>(tok) < p.V0) ? static_cast<uint32_t>(tok) : 0u;
+        }
+        e0r[i] = reinterpret_cast<const uint4*>(p.E0 + static_cast<int64_t>(t) * p.D + col0 + u2 * 8);
+        // the row's E_0 slice (kMmaN * 2 bytes) toward L2 while the tile's main loop runs
+        if (valid[i]) {
+#pragma unroll
+          for (int l = u2; l < kMmaN * 2 / 128; l += 4)
+            prefetch_l2(reinterpret_cast<const uint8_t*>(p.E0 + static_cast<int64_t>(t) * p.D + col0) + l * 128);
+        }
+      }
+      constexpr int kChunks = kMmaN / 32;
+      uint4 e[kChunks][4];  // E_0 of chunk c, row i: loaded two chunks ahead
+#pragma unroll
+      for (int c = 0; c < 2 && c < kChunks; ++c)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) e[c][i] = valid[i] ? __ldg(e0r[i] + c * 4) : make_uint4(0, 0, 0, 0);
 
       bool got = false;
       if (lane == 0) got = mbar_wait_cluster(tfull_bar(acc), use & 1u, abort_flag, p.status);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kMmaN);
-#pragma unroll 1
-      for (int c = 0; c < kMmaN / 32; ++c) {
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + c * 32, v);
-        uint4 enext[4];
-        const bool has_next = c + 1 < kMmaN / 32;
+        if (c + 2 < kChunks) {
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
-          enext[w] = (valid && has_next) ? __ldg(e0 + (c + 1) * 4 + w) : make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 4; ++i) e[c + 2][i] = valid[i] ? __ldg(e0r[i] + (c + 2) * 4) : make_uint4(0, 0, 0, 0);
+        }
         tmem_wait_ld();
-        if (c + 1 == kMmaN / 32) {
+        if (c + 1 == kChunks) {
           tc_fence_before();
           if (rank == 0) {
             mbar_arrive(tempty_bar(acc));
@@ -329,23 +361,30 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             if (lane == 0) mbar_arrive_remote(acc ? tempty_remote1 : tempty_remote0);
           }
         }
-        if (valid) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const uint32_t ew[4] = {ecur[w].x, ecur[w].y, ecur[w].z, ecur[w].w};
+        for (int w = 0; w < 8; ++w)
+          st_shared_v4(row_w + (static_cast<uint32_t>(w ^ (lane & 7)) << 4),
+                       make_uint4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]));
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 lo = ld_shared_v4(rd_lo + i * 8 * 128);
+          const uint4 hi = ld_shared_v4(rd_hi + i * 8 * 128);
+          if (valid[i]) {
+            const float a[8] = {__uint_as_float(lo.x), __uint_as_float(lo.y), __uint_as_float(lo.z), __uint_as_float(lo.w),
+                                __uint_as_float(hi.x), __uint_as_float(hi.y), __uint_as_float(hi.z), __uint_as_float(hi.w)};
+            const uint32_t ew[4] = {e[c][i].x, e[c][i].y, e[c][i].z, e[c][i].w};
             uint32_t o[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              const int col = w * 8 + h * 2;
-              const float x0 = (__uint_as_float(v[col]) + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale;
-              const float x1 = (__uint_as_float(v[col + 1]) + bf16_bits_to_float(ew[h] >> 16)) * p.scale;
+              const float x0 = (a[2 * h] + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale;
+              const float x1 = (a[2 * h + 1] + bf16_bits_to_float(ew[h] >> 16)) * p.scale;
               o[h] = pack_bf16x2(x0, x1);
             }
-            dst[c * 4 + w] = make_uint4(o[0], o[1], o[2], o[3]);
+            dst0[static_cast<int64_t>(i) * p.D + c * 4] = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
-#pragma unroll
-        for (int w = 0; w < 4; ++w) ecur[w] = enext[w];
+        __syncwarp();  // the staging area is rewritten by the next chunk
       }
     }
   }
