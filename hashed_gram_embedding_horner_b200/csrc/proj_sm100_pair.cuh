@@ -104,7 +104,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1u);
-      mbar_init(tempty_bar(a), 128u + 4u);  // CTA 0: its 128 epilogue threads + CTA 1's 4 epilogue warps
+      // CTA 0: the threads of its epilogue warps + one remote arrive per CTA 1 epilogue warp
+      mbar_init(tempty_bar(a), kWide ? 256u + 8u : 128u + 4u);
     }
     mbar_init(drain_bar, 1u);
     *abort_flag = 0;
@@ -224,39 +225,65 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int local = 0;
+      auto advance = [&](int& st, uint32_t& ph) { if (++st == STAGES) { st = 0; ph ^= 1u; } };
+      // the MMAs of half h (all of the tile when not wide) on stage st, k-block i of the tile
+      auto issue = [&](int st, int h, int i, uint32_t d_tmem) {
+        const uint64_t adesc = sw128_kmajor_desc(a_tile(st));
+        const uint64_t bdesc = sw128_kmajor_desc(b_tile(st) + h * L::kBSubBytes);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k)
+          umma_bf16_pair(d_tmem + h * kMmaN, adesc + 2u * k, bdesc + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
+        if (kWide && i + 1 == KB) {  // half h complete: its epilogue may start
+          umma_commit_pair(map_to_cta(tfull_bar(h), 0));
+          umma_commit_pair(map_to_cta(tfull_bar(h), 1));
+        }
+      };
+      auto release = [&](int st) {
+        umma_commit_pair(map_to_cta(empty_bar(st), 0));
+        umma_commit_pair(map_to_cta(empty_bar(st), 1));
+      };
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
         // one accumulator of both halves (wide), else two alternating ones
         const int acc = kWide ? 0 : (local & 1);
         const uint32_t use = static_cast<uint32_t>(kWide ? local : local >> 1);
-        if (!kWide) {
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        int i0 = 0;
+        if (kWide) {
+          // The epilogue frees half 0 of the previous tile first: the MMAs of half 0 run on
+          // the stages already loaded while half 1 is still being drained; those stages'
+          // half-1 MMAs (same per-element order) and releases follow once it is free.
+          const int pre = KB < STAGES ? KB : STAGES;
+          if (!mbar_wait_cluster(tempty_bar(0), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          int st = stage;
+          uint32_t ph = phase;
+          for (int i = 0; i < pre; ++i) {
+            if (!mbar_wait_cluster(full_bar(st), ph, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+            issue(st, 0, i, d_tmem);
+            advance(st, ph);
+          }
+          if (!ok) break;
+          if (!mbar_wait_cluster(tempty_bar(1), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          for (int i = 0; i < pre; ++i) {
+            issue(stage, 1, i, d_tmem);
+            release(stage);
+            advance(stage, phase);
+          }
+          i0 = pre;
+        } else {
           if (!mbar_wait_cluster(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
         }
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int i = 0; i < KB && ok; ++i) {
+        for (int i = i0; i < KB; ++i) {
           if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           if (cp_rows) fence_proxy_async_smem();  // this CTA's cp.async rows: generic proxy writes
-          const uint64_t adesc = sw128_kmajor_desc(a_tile(stage));
 #pragma unroll
-          for (int h = 0; h < L::kHalves; ++h) {
-            if (kWide && i == 0) {  // half h of the previous tile drained
-              if (!mbar_wait_cluster(tempty_bar(h), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
-              tc_fence_after();
-            }
-            const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage) + h * L::kBSubBytes);
-#pragma unroll
-            for (int k = 0; k < kBK / 16; ++k)
-              umma_bf16_pair(d_tmem + h * kMmaN, adesc + 2u * k, bdesc + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
-            if (kWide && i + 1 == KB) {  // half h complete: its epilogue may start
-              umma_commit_pair(map_to_cta(tfull_bar(h), 0));
-              umma_commit_pair(map_to_cta(tfull_bar(h), 1));
-            }
-          }
-          if (!ok) break;
-          umma_commit_pair(map_to_cta(empty_bar(stage), 0));
-          umma_commit_pair(map_to_cta(empty_bar(stage), 1));
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          for (int h = 0; h < L::kHalves; ++h) issue(stage, h, i, d_tmem);
+          release(stage);
+          advance(stage, phase);
         }
         if (ok && !kWide) {
           umma_commit_pair(map_to_cta(tfull_bar(acc), 0));
@@ -290,9 +317,15 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     // store, so each global access instruction covers 8 rows x 64 contiguous bytes instead
     // of 32 rows x 16 bytes (a quarter of the lines through L1 for the E_0 reads and the
     // output writes). Same arithmetic per element: (acc + E_0) * scale, rounded once.
+    // Wide tiles: all eight warps drain half 0 first (warps 12-15 its columns 0-127, warps
+    // 4-7 columns 128-255), free it, then half 1 the same way, so half 0 is free for the
+    // next tile's MMAs after half of the drain.
+    constexpr int kSegs = kWide ? 2 : 1;                 // accumulator halves, in drain order
+    constexpr int kSegChunks = (kWide ? 128 : kMmaN) / 32;
+    constexpr int kChunks = kSegs * kSegChunks;
     const int q = warp & 3;  // TMEM lanes q*32 .. q*32+31 (warp w reaches quadrant w % 4)
-    const int half = kWide && warp < kWarpEpi0 ? 1 : 0;  // wide: warps 4-7 drain columns 256-511
-    const uint32_t stg = sbase + L::kEpiOffset + static_cast<uint32_t>(half * 4 + q) * L::kEpiWarpBytes;
+    const int g = kWide && warp < kWarpEpi0 ? 1 : 0;    // wide: column group of each half
+    const uint32_t stg = sbase + L::kEpiOffset + static_cast<uint32_t>(g * 4 + q) * L::kEpiWarpBytes;
     const int rsub = lane >> 2, u2 = lane & 3;  // read-back: rows i*8 + rsub, columns u2*8 .. u2*8+7
     // staging layout: row r at r*128 bytes, 16-byte unit w at ((w ^ (r & 7)) << 4): conflict-free
     // for both the row-per-lane writes and the 4-lanes-per-row reads
@@ -301,13 +334,15 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     const uint32_t rd_hi = stg + static_cast<uint32_t>(rsub) * 128u + (static_cast<uint32_t>((2 * u2 + 1) ^ rsub) << 4);
     const uint32_t tempty_remote0 = map_to_cta(tempty_bar(0), 0);
     const uint32_t tempty_remote1 = map_to_cta(tempty_bar(1), 0);
+    // chunk cc: its first column relative to col0 (output / E_0) and within the accumulator
+    auto chunk_col = [&](int cc) { return (kWide ? (cc / kSegChunks) * kMmaN : 0) + (cc % kSegChunks) * 32; };
     int local = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
       const int m_blk = tile / p.num_n_blocks;
       const int n_blk = tile % p.num_n_blocks;
-      const int acc = kWide ? half : (local & 1);
+      const int acc = kWide ? 0 : (local & 1);
       const uint32_t use = static_cast<uint32_t>(kWide ? local : local >> 1);
-      const int col0 = n_blk * BN + half * kMmaN;
+      const int col0 = n_blk * BN + g * 128;
       const int64_t row0 = static_cast<int64_t>(m_blk) * (2 * kBM) + rank * kBM + q * 32;
       // this lane's four read-back rows: E_0 and output addresses of its 8 columns
       const uint4* e0r[4];
@@ -323,42 +358,48 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           const int32_t tok = p.tokens[gr];
           t = (tok >= 0 && static_cast<uint32_t>(tok) < p.V0) ? static_cast<uint32_t>(tok) : 0u;
         }
-        e0r[i] = reinterpret_cast<const uint4*>(p.E0 + static_cast<int64_t>(t) * p.D + col0 + u2 * 8);
-        // the row's E_0 slice (kMmaN * 2 bytes) toward L2 while the tile's main loop runs
-        if (valid[i]) {
-#pragma unroll
-          for (int l = u2; l < kMmaN * 2 / 128; l += 4)
-            prefetch_l2(reinterpret_cast<const uint8_t*>(p.E0 + static_cast<int64_t>(t) * p.D + col0) + l * 128);
-        }
+        const uint16_t* row_e0 = p.E0 + static_cast<int64_t>(t) * p.D + col0;
+        e0r[i] = reinterpret_cast<const uint4*>(row_e0 + u2 * 8);
+        // the row's E_0 columns of this warp toward L2 while the tile's main loop runs: line
+        // u2 of them (wide: 2 lines in each half, else kMmaN * 2 / 128 lines)
+        constexpr int kLines = kWide ? 4 : kMmaN * 2 / 128;
+        if (valid[i] && u2 < kLines)
+          prefetch_l2(reinterpret_cast<const uint8_t*>(row_e0) +
+                      (kWide ? (u2 >> 1) * kMmaN * 2 + (u2 & 1) * 128 : u2 * 128));
       }
-      constexpr int kChunks = kMmaN / 32;
       uint4 e[kChunks][4];  // E_0 of chunk c, row i: loaded two chunks ahead
 #pragma unroll
       for (int c = 0; c < 2 && c < kChunks; ++c)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) e[c][i] = valid[i] ? __ldg(e0r[i] + c * 4) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 4; ++i) e[c][i] = valid[i] ? __ldg(e0r[i] + chunk_col(c) / 8) : make_uint4(0, 0, 0, 0);
 
-      bool got = false;
-      if (lane == 0) got = mbar_wait_cluster(tfull_bar(acc), use & 1u, abort_flag, p.status);
-      if (!__shfl_sync(0xffffffffu, got, 0)) break;
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kMmaN);
+      bool alive = true;
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) {
+      for (int cc = 0; cc < kChunks; ++cc) {
+        const int seg = cc / kSegChunks;
+        const int bar = kWide ? seg : acc;
+        if (cc % kSegChunks == 0) {
+          bool got = false;
+          if (lane == 0) got = mbar_wait_cluster(tfull_bar(bar), use & 1u, abort_flag, p.status);
+          if (!__shfl_sync(0xffffffffu, got, 0)) { alive = false; break; }
+          tc_fence_after();
+        }
+        const uint32_t tcol = (kWide ? static_cast<uint32_t>(seg * kMmaN + g * 128) : static_cast<uint32_t>(acc * kMmaN)) +
+                              static_cast<uint32_t>((cc % kSegChunks) * 32);
         uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, v);
-        if (c + 2 < kChunks) {
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + tcol, v);
+        if (cc + 2 < kChunks) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) e[c + 2][i] = valid[i] ? __ldg(e0r[i] + (c + 2) * 4) : make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 4; ++i) e[cc + 2][i] = valid[i] ? __ldg(e0r[i] + chunk_col(cc + 2) / 8) : make_uint4(0, 0, 0, 0);
         }
         tmem_wait_ld();
-        if (c + 1 == kChunks) {
+        if (cc % kSegChunks == kSegChunks - 1) {  // this warp's last read of the segment
           tc_fence_before();
           if (rank == 0) {
-            mbar_arrive(tempty_bar(acc));
+            mbar_arrive(tempty_bar(bar));
           } else {
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(acc ? tempty_remote1 : tempty_remote0);
+            if (lane == 0) mbar_arrive_remote(bar ? tempty_remote1 : tempty_remote0);
           }
         }
 #pragma unroll
@@ -373,7 +414,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           if (valid[i]) {
             const float a[8] = {__uint_as_float(lo.x), __uint_as_float(lo.y), __uint_as_float(lo.z), __uint_as_float(lo.w),
                                 __uint_as_float(hi.x), __uint_as_float(hi.y), __uint_as_float(hi.z), __uint_as_float(hi.w)};
-            const uint32_t ew[4] = {e[c][i].x, e[c][i].y, e[c][i].z, e[c][i].w};
+            const uint32_t ew[4] = {e[cc][i].x, e[cc][i].y, e[cc][i].z, e[cc][i].w};
             uint32_t o[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
@@ -381,11 +422,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
               const float x1 = (a[2 * h + 1] + bf16_bits_to_float(ew[h] >> 16)) * p.scale;
               o[h] = pack_bf16x2(x0, x1);
             }
-            dst0[static_cast<int64_t>(i) * p.D + c * 4] = make_uint4(o[0], o[1], o[2], o[3]);
+            dst0[static_cast<int64_t>(i) * p.D + chunk_col(cc) / 8] = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
         __syncwarp();  // the staging area is rewritten by the next chunk
       }
+      if (!alive) break;
     }
   }
 
