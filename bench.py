@@ -499,6 +499,7 @@ def main():
     achieved = flops / (proj_ms / 1e3) / 1e12
     form = ne.ngram_embed_plan_kernel_form(plan, T)
     kernel_name = {"cta_pair": "proj_sm100_pair_kernel", "cta_pair_wide": "proj_sm100_pair_kernel",
+                   "cta_pair_stream_k": "proj_sm100_pair_kernel",
                    "one_cta": "proj_sm100_kernel",
                    "one_cta_stream_k": "proj_sm100_kernel", "cuda_cores": "proj_simt_kernel"}[form]
     algo_bytes = T * (2 * cfg.D * 2 + 4) + cfg.D * cfg.D * 2

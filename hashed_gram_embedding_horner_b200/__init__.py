@@ -313,7 +313,8 @@ def ngram_hash_stats(V0: int, n: int, tokens, seq_offsets, moduli, workspace=Non
     return (None if dist.value < 0 else int(dist.value)), [int(h) for h in hits]
 
 
-KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair", 4: "cta_pair_wide"}
+KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair", 4: "cta_pair_wide",
+                5: "cta_pair_stream_k"}
 
 
 def ngram_embed_plan_kernel_form(plan: Plan, num_tokens: int) -> str:

@@ -228,6 +228,21 @@ int launch_tc(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st) {
   }
 }
 
+// Stream-K for the CTA-pair kernel's 256 x 256 tiles, over the co-resident pairs (one per
+// two SMs); pieces are counted per (tile, CTA, row quarter) in the workspace head, and each
+// CTA has two partial slots of 128 x 256 fp32. Only when the plan asks for both the pair
+// form and stream-K: at the 1280-token decode step (D = 4096) it measured 69.9 us against
+// 56.2 us for the one-CTA form's stream-K, whose cp.async row gather keeps more DRAM misses
+// in flight than TMA gather4.
+bool use_pair_stream_k(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws_T) {
+  if (p->stream_k != 1 || p->cta_pair != 1 || p->sms < 2 || p->bn != 256) return false;
+  const int64_t pairs = p->sms / 2;
+  const int64_t tiles = (T + 2 * kBM - 1) / (2 * kBM) * (p->D / p->bn);
+  const int64_t units = tiles * (p->D / kBK);
+  if (tiles > kSkMaxTiles / 2 || units < pairs) return false;
+  return ws_size >= ws_bytes(p, ws_T);
+}
+
 // CTA-pair kernel: clusters of two CTAs, one 256 x BN tile per pair per step.
 template <int BN, int kStg>
 int launch_tc_pair_stages(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t st, int key) {
@@ -260,7 +275,7 @@ int launch_tc_pair_stages(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaSt
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return NGRAM_ERR_CUDA;
     max_pairs = n;
   }
-  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  const int pairs = (prm.stream_k || tiles > max_pairs) ? max_pairs : tiles;
   return launch(kern, dim3(2 * pairs), dim3(kProjThreads), L::kLaunchBytes, st, p->pdl, 2, p->maps, prm);
 }
 
@@ -484,15 +499,25 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   // Not stream-K when the count is known only on the device: for the few tiles of a draft
   // call's misses its fix-ups cost more than they balance (measured: 256 misses at D = 4096,
   // 79 us stream-K vs 64 us CTA pairs).
-  const bool sk = !T_dev && p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
+  // the one-CTA form's stream-K where its grid ends in a thin wave, else the pair form
+  // (512-column tiles where they fill their waves)
+  const bool psk = !T_dev && p->cta_pair != 0 && p->pair_wide != 1 && use_pair_stream_k(p, T, ws_size, ws_T);
+  const bool sk = !psk && !T_dev && p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
   const bool pair = p->cta_pair == 1 || (p->cta_pair == -1 && !sk);
   // A rows by TMA gather4 in the pair form, by cp.async in the one-CTA form (measured
   // fastest for each), unless the plan fixes the split.
   prm.tma_rows = p->variant == kTcTmaRows ? kBM : (p->tma_rows >= 0 ? p->tma_rows : (pair ? kBM : 0));
-  if (pair && use_pair_wide(p, T, T_dev != nullptr)) {
+  if (pair && !psk && use_pair_wide(p, T, T_dev != nullptr)) {
     prm.num_n_blocks = p->D / 512;
     prm.tma_rows = kBM;  // A rows by gather4 only
     return launch_tc_pair_stages<512, kPairStagesWide>(p, prm, T, st, 8);
+  }
+  if (pair && psk) {
+    prm.stream_k = 1;
+    prm.tma_rows = kBM;  // A rows by gather4 only
+    prm.sk_counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+    prm.sk_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_base(p, ws_T));
+    return launch_tc_pair<256>(p, prm, T, st);
   }
   if (pair) return p->bn == 256 ? launch_tc_pair<256>(p, prm, T, st) : launch_tc_pair<128>(p, prm, T, st);
   if (sk) {
@@ -623,8 +648,10 @@ int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_token
   prm.num_m_blocks = static_cast<int>((num_tokens + kBM - 1) / kBM);
   prm.num_n_blocks = plan->D / plan->bn;
   prm.num_k_blocks = plan->D / kBK;
-  const bool sk = plan->cta_pair != 1 && use_stream_k(plan, prm, num_tokens, ws_bytes(plan, num_tokens));
-  if (plan->cta_pair == 1 || (plan->cta_pair == -1 && !sk)) return use_pair_wide(plan, num_tokens) ? 4 : 3;
+  const size_t ws = ws_bytes(plan, num_tokens);
+  const bool psk = plan->cta_pair != 0 && plan->pair_wide != 1 && use_pair_stream_k(plan, num_tokens, ws, num_tokens);
+  const bool sk = !psk && plan->cta_pair != 1 && use_stream_k(plan, prm, num_tokens, ws);
+  if (plan->cta_pair == 1 || (plan->cta_pair == -1 && !sk)) return psk ? 5 : (use_pair_wide(plan, num_tokens) ? 4 : 3);
   return sk ? 2 : 1;
 }
 

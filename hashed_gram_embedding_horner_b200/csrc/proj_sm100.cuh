@@ -112,45 +112,13 @@ __device__ __forceinline__ uint32_t clamp_row(int32_t r, uint32_t V, int* status
 // First k-block of a tile: a rotation that differs between tiles running side by side.
 __device__ __forceinline__ int k_rotation(int m_blk, int n_blk, int KB) { return (m_blk * 5 + n_blk * 3) % KB; }
 
-// The k-blocks a tile visits (from its rotation, wrapping) fall into runs that each use one
-// sub-table. Producers walk the CTA's (tile, k-block) sequence run by run and load the row
-// indices of the next run while the current one is being copied, so the dependent index
-// load never sits between a freed stage and its refill.
-struct KRun {
-  int tile;     // tile of the run (>= number of tiles: past the end)
-  int i;        // position of the run's first k-block in the tile's sequence
-  int s;        // sub-table
-  int c_first;  // k-block offset of the run's first k-block inside the sub-table
-  int len;      // k-blocks in the run
-};
-
-__device__ __forceinline__ KRun k_run_at(int tile, int i, int num_n_blocks, int KB, int kb_per_sub) {
-  KRun r;
-  r.tile = tile;
-  r.i = i;
-  int kb = i + k_rotation(tile / num_n_blocks, tile % num_n_blocks, KB);
-  if (kb >= KB) kb -= KB;
-  r.s = kb / kb_per_sub;
-  r.c_first = kb - r.s * kb_per_sub;
-  const int rem = kb_per_sub - r.c_first;
-  r.len = rem < KB - i ? rem : KB - i;
-  return r;
-}
-
-__device__ __forceinline__ KRun k_run_next(const KRun& r, int stride, int num_n_blocks, int KB, int kb_per_sub) {
-  int i = r.i + r.len, tile = r.tile;
-  if (i >= KB) {
-    i = 0;
-    tile += stride;
-  }
-  return k_run_at(tile, i, num_n_blocks, KB, kb_per_sub);
-}
-
-// ---- work lists of the one-CTA kernel --------------------------------------------------
-// Data-parallel: CTA c takes whole tiles c, c + grid, ... Stream-K: the tiles' k-positions
-// form U = tiles * KB units in tile-major order and CTA c takes units [c*U/grid,
-// (c+1)*U/grid); a tile whose units straddle CTAs is computed in pieces ("segments")
-// whose fp32 partial sums are added by the last piece to finish.
+// ---- work lists (one-CTA kernel: a worker is a CTA; pair kernel: a CTA pair) ------------
+// Data-parallel: worker c takes whole tiles c, c + grid, ... Stream-K: the tiles' k-positions
+// form U = tiles * KB units in tile-major order and worker c takes units [c*U/grid,
+// (c+1)*U/grid); a tile whose units straddle workers is computed in pieces ("segments")
+// whose fp32 partial sums are added by the last piece to finish. Producers walk a worker's
+// sequence run by run (a run: consecutive k-blocks of one segment that use one sub-table)
+// and load the row indices of the next run while the current one is being copied.
 struct WorkPlan {
   int num_tiles, KB, grid;
   int sk;          // 1: stream-K

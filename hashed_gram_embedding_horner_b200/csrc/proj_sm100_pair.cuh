@@ -66,6 +66,134 @@ struct PairSmem {
   static_assert(kTmemCols <= 512, "accumulators exceed TMEM");
 };
 
+// One stream-K piece of a 256-column pair tile (this CTA's 128 rows), as in the one-CTA
+// kernel: per (tile, CTA rank, row quarter) an arrival counter counts the pieces published
+// so far; the warp whose piece completes the tile sums every piece in pair order (its own
+// from TMEM, the others from their owners' partial slots), adds E_0 and scales. A warp
+// that finds all other pieces already counted skips publishing its own. Nobody waits for
+// anybody. Out of line: the fixup is rare, and inlined its registers press on the
+// whole-tile epilogue. Returns false if the accumulator never became ready (abort).
+struct PairPiece {
+  Seg sg;
+  int acc;
+  uint32_t use;
+  int64_t T, units_total;
+  int KB, grid, pair, q, lane;
+  uint32_t rank, tmem_base;
+  uint32_t tfull, tempty;  // this accumulator's barriers (tempty: CTA 0's, as a cluster address on CTA 1)
+  volatile int* abort_flag;
+};
+
+template <int BN>
+__device__ __noinline__ bool pair_sk_piece(const ProjParams& p, const PairPiece a) {
+  const int tile = a.sg.tile;
+  const int m_blk = tile / p.num_n_blocks;
+  const int n_blk = tile % p.num_n_blocks;
+  const int row_in_tile = a.q * 32 + a.lane;
+  const int64_t gr = static_cast<int64_t>(m_blk) * (2 * kBM) + a.rank * kBM + row_in_tile;
+  const bool valid = gr < a.T;
+  uint32_t t = 0;
+  if (valid) {
+    const int32_t tok = p.tokens[gr];
+    t = (tok >= 0 && static_cast<uint32_t>(tok) < p.V0) ? static_cast<uint32_t>(tok) : 0u;
+  }
+  const uint4* e0 = reinterpret_cast<const uint4*>(p.E0 + static_cast<int64_t>(t) * p.D + n_blk * BN);
+  uint4* dst = reinterpret_cast<uint4*>(p.out + gr * p.D + n_blk * BN);
+  bool got = false;
+  if (a.lane == 0) got = mbar_wait_cluster(a.tfull, a.use & 1u, a.abort_flag, p.status);
+  if (!__shfl_sync(0xffffffffu, got, 0)) return false;
+  tc_fence_after();
+  const uint32_t taddr = a.tmem_base + (static_cast<uint32_t>(a.q * 32) << 16) + static_cast<uint32_t>(a.acc * BN);
+  const int64_t u_tile = static_cast<int64_t>(tile) * a.KB;
+  const int c_lo = sk_cta_of(u_tile, a.units_total, a.grid), c_hi = sk_cta_of(u_tile + a.KB - 1, a.units_total, a.grid);
+  const int others = c_hi - c_lo;  // pieces of the tile besides this one
+  int* cnt = p.sk_counters + (tile * 2 + static_cast<int>(a.rank)) * 4 + a.q;
+  // partial slots: [pair][rank][slot] x (128 rows x BN columns), column-group major
+  auto slot_of = [&](int pr, int sl) {
+    return reinterpret_cast<float4*>(p.sk_partials) +
+           ((static_cast<size_t>(pr) * 2 + a.rank) * 2 + sl) * (kBM * BN / 4) + row_in_tile;
+  };
+  int fin = 0;
+  if (a.lane == 0) fin = ld_acquire_gpu(cnt) == others;
+  fin = __shfl_sync(0xffffffffu, fin, 0);
+  if (!fin) {
+    // slot 0: the piece that starts this pair's unit range; slot 1: the one that ends it
+    float4* mine = slot_of(a.pair, (u_tile + a.sg.i0 == sk_first_unit(a.units_total, a.grid, a.pair)) ? 0 : 1);
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int w = 0; w < 8; ++w)  // a warp's store is 512 contiguous bytes
+        mine[(c * 8 + w) * kBM] = make_float4(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1]),
+                                              __uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3]));
+    }
+    __threadfence();
+    __syncwarp();
+    if (a.lane == 0) fin = atomicAdd(cnt, 1) == others;
+    fin = __shfl_sync(0xffffffffu, fin, 0);
+    if (fin) __threadfence();
+  }
+  if (fin) {
+    // 16 columns at a time (register pressure): pieces before this pair's, its own
+    // (TMEM), those after, in pair order whoever finishes, so the bits do not depend on
+    // arrival order
+#pragma unroll 1
+    for (int c = 0; c < BN / 16; ++c) {
+      float sum[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) sum[k] = 0.f;
+      auto add_piece = [&](int pr) {
+        const float4* part = slot_of(pr, sk_first_unit(a.units_total, a.grid, pr) >= u_tile ? 0 : 1);
+        float4 x[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) x[w] = __ldcg(part + (c * 4 + w) * kBM);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          sum[4 * w] += x[w].x;
+          sum[4 * w + 1] += x[w].y;
+          sum[4 * w + 2] += x[w].z;
+          sum[4 * w + 3] += x[w].w;
+        }
+      };
+      for (int pr = c_lo; pr < a.pair; ++pr) add_piece(pr);
+      {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(taddr + c * 16, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) sum[k] += __uint_as_float(v[k]);
+      }
+      for (int pr = a.pair + 1; pr <= c_hi; ++pr) add_piece(pr);
+      if (valid) {
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const uint4 ev = __ldg(e0 + c * 2 + w);
+          const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int col = w * 8 + h * 2;
+            o[h] = pack_bf16x2((sum[col] + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale,
+                               (sum[col + 1] + bf16_bits_to_float(ew[h] >> 16)) * p.scale);
+          }
+          dst[c * 2 + w] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+    if (a.lane == 0) *cnt = 0;  // the tile is done: zero again for the next launch
+  }
+  tc_fence_before();  // accumulator read for the last time: the MMA may reuse it
+  if (a.rank == 0) {
+    mbar_arrive(a.tempty);
+  } else {
+    __syncwarp();
+    if (a.lane == 0) mbar_arrive_remote(a.tempty);
+  }
+  return true;
+}
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_sm100_pair_kernel(const __grid_constant__ ProjMaps maps, const __grid_constant__ ProjParams p) {
@@ -92,7 +220,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
   constexpr bool kWide = L::kWide;
   constexpr int kMmaN = L::kMmaN;
-  const bool cp_rows = !kWide && p.tma_rows == 0;  // A rows by cp.async (else all by TMA gather4)
+  // stream-K (256-column tiles only): the (tile, k-block) units split evenly over the pairs
+  const bool sk = !kWide && p.stream_k != 0;
+  const bool cp_rows = !kWide && !sk && p.tma_rows == 0;  // A rows by cp.async (else all by TMA gather4)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       // CTA 0: thread 0 posts the pair's TMA bytes (+ its 256 cp.async threads + CTA 1's relay);
@@ -129,6 +259,15 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   const int num_tiles = static_cast<int>((T + 2 * kBM - 1) / (2 * kBM)) * p.num_n_blocks;  // m blocks of 256 rows
   const int KB = p.num_k_blocks;
   const int kb_per_sub = p.d / kBK;
+  // Work list of this pair: whole tiles pair, pair + num_pairs, ...; or, under stream-K, an
+  // equal run of units (pairs past the unit count, known only here, hold none).
+  const int64_t units_total = static_cast<int64_t>(num_tiles) * KB;
+  WorkPlan wp;
+  wp.num_tiles = num_tiles;
+  wp.KB = KB;
+  wp.grid = (sk && units_total < num_pairs) ? static_cast<int>(units_total) : num_pairs;
+  wp.sk = sk ? 1 : 0;
+  wp.u_end = sk ? sk_first_unit(units_total, wp.grid, pair + 1) : 0;
 
   const bool epi_warp = warp >= kWarpEpi0 || (kWide && warp >= kAWarps / 2 && warp < kAWarps);
   if (warp < kAWarps && !epi_warp) {
@@ -143,8 +282,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     const uint64_t pol = l2_policy_evict_normal();
     // raw row indices (this thread's 4 rows) of the current and the next run
     int32_t raw[4], nraw[4];
-    auto load_raw = [&](const KRun& r, int32_t (&dst)[4]) {
-      const int64_t row_base = static_cast<int64_t>(r.tile / p.num_n_blocks) * (2 * kBM) + rank * kBM;
+    auto load_raw = [&](const SRun& r, int32_t (&dst)[4]) {
+      const int64_t row_base = static_cast<int64_t>(r.g.tile / p.num_n_blocks) * (2 * kBM) + rank * kBM;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t gr = row_base + (cp_rows ? rsub + 32 * j : iss * 4 + j);
@@ -154,11 +293,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    KRun cur = k_run_at(pair, 0, p.num_n_blocks, KB, kb_per_sub);
-    if (cur.tile < num_tiles) load_raw(cur, raw);
-    KRun nxt = k_run_next(cur, num_pairs, p.num_n_blocks, KB, kb_per_sub);
-    if (nxt.tile < num_tiles) load_raw(nxt, nraw);
-    while (cur.tile < num_tiles && ok) {
+    const Seg g0 = seg_first(wp, pair);
+    SRun cur = srun_at(g0, g0.i0, p.num_n_blocks, KB, kb_per_sub);
+    if (cur.g.tile < num_tiles) load_raw(cur, raw);
+    SRun nxt = srun_next(wp, cur, p.num_n_blocks, kb_per_sub);
+    if (nxt.g.tile < num_tiles) load_raw(nxt, nraw);
+    while (cur.g.tile < num_tiles && ok) {
       const uint32_t V = p.Vs[cur.s];
       const uint16_t* src[4];
       int32_t r4[4];
@@ -186,8 +326,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       cur = nxt;
 #pragma unroll
       for (int j = 0; j < 4; ++j) raw[j] = nraw[j];
-      nxt = k_run_next(nxt, num_pairs, p.num_n_blocks, KB, kb_per_sub);
-      if (nxt.tile < num_tiles) load_raw(nxt, nraw);
+      nxt = srun_next(wp, nxt, p.num_n_blocks, kb_per_sub);
+      if (nxt.g.tile < num_tiles) load_raw(nxt, nraw);
     }
     cp_async_wait_all();
     if (!ok) {
@@ -201,10 +341,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int n_blk = tile % p.num_n_blocks;
-        const int rot = k_rotation(tile / p.num_n_blocks, n_blk, KB);
-        for (int i = 0; i < KB; ++i) {
+      for (Seg g = seg_first(wp, pair); g.tile < num_tiles && ok; g = seg_next(wp, g)) {
+        const int n_blk = g.tile % p.num_n_blocks;
+        const int rot = k_rotation(g.tile / p.num_n_blocks, n_blk, KB);
+        for (int i = g.i0; i < g.i1; ++i) {
           int kb = i + rot;
           if (kb >= KB) kb -= KB;
           if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
@@ -242,12 +382,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         umma_commit_pair(map_to_cta(empty_bar(st), 0));
         umma_commit_pair(map_to_cta(empty_bar(st), 1));
       };
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
+      for (Seg g = seg_first(wp, pair); g.tile < num_tiles && ok; g = seg_next(wp, g), ++local) {
         // one accumulator of both halves (wide), else two alternating ones
         const int acc = kWide ? 0 : (local & 1);
         const uint32_t use = static_cast<uint32_t>(kWide ? local : local >> 1);
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        int i0 = 0;
+        int i0 = g.i0;  // wide tiles are always whole (i0 = 0, i1 = KB)
         if (kWide) {
           // The epilogue frees half 0 of the previous tile first: the MMAs of half 0 run on
           // the stages already loaded while half 1 is still being drained; those stages'
@@ -276,12 +416,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           if (!mbar_wait_cluster(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
         }
-        for (int i = i0; i < KB; ++i) {
+        for (int i = i0; i < g.i1; ++i) {
           if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           if (cp_rows) fence_proxy_async_smem();  // this CTA's cp.async rows: generic proxy writes
 #pragma unroll
-          for (int h = 0; h < L::kHalves; ++h) issue(stage, h, i, d_tmem);
+          for (int h = 0; h < L::kHalves; ++h) issue(stage, h, i - g.i0, d_tmem);  // a segment starts a fresh sum
           release(stage);
           advance(stage, phase);
         }
@@ -337,11 +477,32 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     // chunk cc: its first column relative to col0 (output / E_0) and within the accumulator
     auto chunk_col = [&](int cc) { return (kWide ? (cc / kSegChunks) * kMmaN : 0) + (cc % kSegChunks) * 32; };
     int local = 0;
-    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
+    for (Seg sg = seg_first(wp, pair); sg.tile < num_tiles; sg = seg_next(wp, sg), ++local) {
+      const int tile = sg.tile;
       const int m_blk = tile / p.num_n_blocks;
       const int n_blk = tile % p.num_n_blocks;
       const int acc = kWide ? 0 : (local & 1);
       const uint32_t use = static_cast<uint32_t>(kWide ? local : local >> 1);
+      if (!kWide && (sg.i0 != 0 || sg.i1 != KB)) {
+        PairPiece pc;
+        pc.sg = sg;
+        pc.acc = acc;
+        pc.use = use;
+        pc.T = T;
+        pc.units_total = units_total;
+        pc.KB = KB;
+        pc.grid = wp.grid;
+        pc.pair = pair;
+        pc.q = q;
+        pc.lane = lane;
+        pc.rank = rank;
+        pc.tmem_base = tmem_base;
+        pc.tfull = tfull_bar(acc);
+        pc.tempty = rank == 0 ? tempty_bar(acc) : (acc ? tempty_remote1 : tempty_remote0);
+        pc.abort_flag = abort_flag;
+        if (!pair_sk_piece<BN>(p, pc)) break;
+        continue;
+      }
       const int col0 = n_blk * BN + g * 128;
       const int64_t row0 = static_cast<int64_t>(m_blk) * (2 * kBM) + rank * kBM + q * 32;
       // this lane's four read-back rows: E_0 and output addresses of its 8 columns

@@ -359,7 +359,7 @@ int ngram_embed_plan_set_pair_wide(ngram_embed_plan* plan, int on);
 /* The projection kernel a call of num_tokens tokens would run, given a workspace of
  * ngram_embed_workspace_bytes(plan, num_tokens): 0 = CUDA cores, 1 = one CTA per tile,
  * 2 = one CTA per SM with the stream-K schedule, 3 = CTA pairs, 4 = CTA pairs with
- * 512-column tiles; negative on bad arguments. */
+ * 512-column tiles, 5 = CTA pairs with the stream-K schedule; negative on bad arguments. */
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens);
 
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */
@@ -373,14 +373,17 @@ int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);
  * change. */
 int ngram_embed_plan_set_a_stages(ngram_embed_plan* plan, int stages);
 
-/* Schedule of the one-CTA tensor-core kernel: 0 = automatic (stream-K when the grid takes two
- * or more waves of one tile per CTA and the last wave leaves many SMs idle, e.g. 160 tiles of
- * 128 x 256 on 148 SMs), 1 = stream-K whenever possible,
- * 2 = never. Stream-K gives every SM an equal run of (tile, k-block) units; a tile split
- * between CTAs is summed in fp32 by whichever CTA finishes its piece last, so no CTA waits
- * for another. It needs the workspace's partial tiles, at most 2048 tiles and at least
- * one k-block per SM; otherwise, and with the CTA-pair form, the kernel takes one tile per
- * CTA. A tuning knob: results agree within the stated tolerance (the summation order
+/* Schedule of the tensor-core kernels: 0 = automatic (the one-CTA form with stream-K when
+ * its grid takes two or more waves of one tile per CTA and the last wave leaves many SMs
+ * idle, e.g. 160 tiles of 128 x 256 on 148 SMs), 1 = stream-K whenever possible (for the
+ * CTA-pair form too when ngram_embed_plan_set_cta_pair(plan, 1) also fixes that form and
+ * the tiles are 256 columns wide), 2 = never. Stream-K gives every worker (a CTA, or a CTA
+ * pair) an equal run of (tile, k-block) units; a tile split between workers is summed in
+ * fp32, in worker order, by whichever finishes its piece last, so no worker waits for
+ * another. It needs the workspace's partial tiles, at most 2048 one-CTA tiles (1024 pair
+ * tiles) and at least one k-block per worker, and is not used with 512-column pair tiles or
+ * when the token count is read on the device; otherwise the kernel takes one tile per
+ * worker. A tuning knob: results agree within the stated tolerance (the summation order
  * differs). */
 int ngram_embed_plan_set_stream_k(ngram_embed_plan* plan, int mode);
 

@@ -179,20 +179,63 @@ def test_stream_k_matches_oracle_and_is_repeatable(ne, shape, tile_n):
     assert_close(to_host_f64(dp), want, what=f"{cfg.name} data-parallel n{tile_n}")
 
 
-def test_stream_k_bit_exact_with_identity_w(ne):
-    """W = I and E_0 = 0 under stream-K: each output element gets one nonzero product, so
-    the fp32 partials of a split tile add zeros to it and the result stays exact."""
-    cfg = small_cfg(7000, 1152, 2, 3, seed=3)   # S + 1 = 4: the scale is exact; 27 tiles of 128 x 128
+@pytest.mark.parametrize("shape", SK_SHAPES, ids=lambda s: "V0%d_D%d_N%d_K%d_T%d" % s)
+def test_pair_stream_k_matches_oracle_and_is_repeatable(ne, shape):
+    """CTA-pair kernel (256 x 256 tiles) with every pair given an equal run of units: tiles
+    split over up to a dozen pairs, each CTA of a pair summing its own 128 rows' pieces;
+    parity with the oracle, repeatable bits, counters back at zero, and agreement with the
+    pairs' data-parallel schedule."""
+    V0, D, N, K, T = shape
+    cfg = small_cfg(V0, D, N, K, seed=7)
+    lengths = [T // 3, 0, T - T // 3 - 5, 5]
+    tokens, offsets = ragged_tokens(cfg, lengths)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = plan_for(ne, cfg, 0, 256, pair=1)
+    ne.ngram_embed_plan_set_pair_wide(plan, 0)
+    ne.ngram_embed_plan_set_stream_k(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, T) == "cta_pair_stream_k"
+    out = torch.full((T, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = ne.new_workspace(plan, T)
+    tk, of = dev_i32(tokens), dev_i32(offsets)
+    ne.ngram_embed_fwd(plan, tk, of, E0, E, W, out, ws)
+    assert ne.ngram_embed_get_status(ws) == 0
+    assert not ws[256:256 + 2048 * 16].any()  # every split tile's counters back at zero
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    assert_close(to_host_f64(out), want, what=f"{cfg.name} pair stream-K")
+    again = torch.full_like(out, float("nan"))
+    ne.ngram_embed_fwd(plan, tk, of, E0, E, W, again, ws)
+    assert ne.ngram_embed_get_status(ws) == 0 and torch.equal(out, again)
+    ne.ngram_embed_plan_set_stream_k(plan, 2)
+    assert ne.ngram_embed_plan_kernel_form(plan, T) == "cta_pair"
+    dp = torch.full_like(out, float("nan"))
+    ne.ngram_embed_fwd(plan, tk, of, E0, E, W, dp, ws)
+    assert ne.ngram_embed_get_status(ws) == 0
+    assert_close(to_host_f64(dp), want, what=f"{cfg.name} pair data-parallel")
+
+
+@pytest.mark.parametrize("pair", [0, 1])
+def test_stream_k_bit_exact_with_identity_w(ne, pair):
+    """W = I and E_0 = 0 under stream-K (one-CTA or CTA-pair form): each output element gets
+    one nonzero product, so the fp32 partials of a split tile add zeros to it and the
+    result stays exact."""
+    # S + 1 = 4: the scale is exact; one-CTA: 27 tiles of 128 x 128; pairs: 9 of 256 x 256
+    # (108 units of a k-block on 74 pairs)
+    cfg = small_cfg(7000, 1152 if pair == 0 else 768, 2, 3, seed=3)
     S = cfg.S
-    tokens, offsets = ragged_tokens(cfg, [5, 128, 200, 3])
+    tokens, offsets = ragged_tokens(cfg, [5, 128, 200, 3] if pair == 0 else [5, 300, 400, 3])
     from tests.helpers import host_tables
     _, Eh, _ = host_tables(cfg)
     eye = gen.f32_to_bf16_bits(np.eye(cfg.D, dtype=np.float32))
     idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, oracle.context_windows(cfg.N, tokens, offsets))
     G = np.concatenate([gen.bf16_bits_to_f32(Eh[s][idx[:, s]]) for s in range(S)], axis=1)
-    plan = plan_for(ne, cfg, 2, 128, pair=0)
-    ne.ngram_embed_plan_set_tma_rows(plan, 0)
+    plan = plan_for(ne, cfg, 2 if pair == 0 else 0, 128 if pair == 0 else 256, pair=pair)
+    if pair == 0:
+        ne.ngram_embed_plan_set_tma_rows(plan, 0)
+    ne.ngram_embed_plan_set_pair_wide(plan, 0)
     ne.ngram_embed_plan_set_stream_k(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == ("one_cta_stream_k" if pair == 0 else "cta_pair_stream_k")
     zeros0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.bfloat16, device="cuda")
     out, status = run_fwd(ne, plan, cfg, tokens, offsets, zeros0, [to_device(e, torch.bfloat16) for e in Eh],
                           to_device(eye, torch.bfloat16))
@@ -383,14 +426,20 @@ def test_pair_wide_not_for_narrow_tiles(ne):
 def test_automatic_kernel_form(ne):
     """Prefill grids run the CTA-pair form with 512-column tiles; a 1280-token decode step at
     D = 4096 (160 tiles of 128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule;
-    a grid of one wave keeps the 256-column pair tiles (more SMs busy)."""
+    a grid of one wave keeps the 256-column pair tiles (more SMs busy). The pairs' stream-K
+    schedule is taken only when both the pair form and stream-K are asked for."""
     for cfg in (configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN):
         plan = plan_for(ne, cfg)
         assert ne.ngram_embed_plan_kernel_form(plan, 32768) == "cta_pair_wide"
     plan = plan_for(ne, configs.SPEC_DECODE)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "one_cta_stream_k"
     assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"  # one wave: nothing to balance
-    assert ne.ngram_embed_plan_kernel_form(plan, 5120) == "cta_pair"   # 160 wide tiles: a thin 3rd wave
+    ne.ngram_embed_plan_set_cta_pair(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_wide"
+    ne.ngram_embed_plan_set_stream_k(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_stream_k"
+    ne.ngram_embed_plan_set_cta_pair(plan, None)
+    ne.ngram_embed_plan_set_stream_k(plan, 0)
     assert ne.ngram_embed_plan_kernel_form(plan_for(ne, configs.TINY), 128) == "cuda_cores"
 
 
