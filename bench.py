@@ -55,15 +55,26 @@ L2_FLUSH_BYTES = 256 << 20
 PROJECTION_SOURCES = ("common.cuh", "proj_sm100.cuh", "proj_sm100_pair.cuh")
 
 
-def kernel_source_hash() -> str:
-    """sha256 over the projection kernels' sources: a profile's counters describe the
-    kernels of the sources they were taken from, and only those."""
+def code_only(text: str) -> str:
+    """C++ source with its comments and blank lines removed and trailing spaces cut: what
+    the compiler sees of it (these sources hold no comment markers inside string literals)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
+def kernel_source_hash(read=None) -> str:
+    """sha256 over the projection kernels' sources, comments removed: a profile's counters
+    describe the kernels of the code they were taken from, and only those. `read(name)`
+    returns a source's text (default: the working tree)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hashed_gram_embedding_horner_b200", "csrc")
     for name in PROJECTION_SOURCES:
+        text = read(name) if read else open(os.path.join(csrc, name), encoding="utf-8").read()
         h.update(name.encode())
-        h.update(open(os.path.join(csrc, name), "rb").read())
+        h.update(code_only(text).encode())
     return h.hexdigest()
 
 

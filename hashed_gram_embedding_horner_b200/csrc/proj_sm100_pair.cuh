@@ -10,14 +10,15 @@
 // which is what limits the one-CTA kernel (on-chip bytes in flight, not DRAM).
 //
 // Cross-CTA signalling, all plain (no multicast):
-//   - W halves (and, with tma_rows = 128, the A rows: tile::gather4, 32 issuing lanes per
-//     CTA) are TMA loads in their .cta_group::2 form: the data lands in the issuing CTA's
-//     shared memory and the byte count completes on CTA 0's stage barrier;
-//   - with tma_rows = 0 (default) the A rows arrive by 16-byte cp.async, which can only
-//     signal the issuing CTA's own barrier: CTA 0's cp.async threads arrive on CTA 0's stage
-//     barrier; CTA 1's arrive on CTA 1's, and a relay lane of CTA 1 (one lane per stage, so
-//     the slow cluster-scope release of one stage overlaps the others) waits for it, fences
-//     generic->async proxy and arrives remotely on CTA 0's stage barrier;
+//   - W halves (and, with tma_rows = 128, the default, the A rows: tile::gather4, 32
+//     issuing lanes per CTA) are TMA loads in their .cta_group::2 form: the data lands in
+//     the issuing CTA's shared memory and the byte count completes on CTA 0's stage barrier;
+//   - with tma_rows = 0 (256- and 128-column tiles only) the A rows arrive by 16-byte
+//     cp.async, which can only signal the issuing CTA's own barrier: CTA 0's cp.async
+//     threads arrive on CTA 0's stage barrier; CTA 1's arrive on CTA 1's, and a relay lane
+//     of CTA 1 (one lane per stage, so the slow cluster-scope release of one stage overlaps
+//     the others) waits for it, fences generic->async proxy and arrives remotely on CTA 0's
+//     stage barrier;
 //   - CTA 0's MMA thread commits stage release and "accumulator ready" to the barriers of
 //     both CTAs (two tcgen05.commit, one per CTA address);
 //   - CTA 1's epilogue warps arrive remotely on CTA 0's "accumulator free" barrier.
@@ -42,9 +43,10 @@ constexpr int kPairStagesWide = 4;  // BN = 512: 16 KB of A + 32 KB of W per sta
 // epilogue of one tile overlaps the main loop of the next.
 // BN = 512 ("wide"): two MMAs of N = 256 per k-step (halves h = 0, 1 of the tile's columns)
 // on the same A stage, so every gathered A row feeds twice the columns; the accumulator
-// takes all 512 TMEM columns, each half drained by its own four epilogue warps (warps 12-15
-// and 4-7; the A rows come by gather4 from warps 0-3) and freed on its own barrier, so the
-// next tile's MMAs into half h wait only for that half.
+// takes all 512 TMEM columns. Eight epilogue warps (12-15 and 4-7; the A rows come by
+// gather4 from warps 0-3) drain half 0 first and free it on its own barrier, then half 1,
+// and the next tile's half-0 MMAs start on the loaded stages as soon as half 0 is free.
+// Stream-K (BN = 256, on request): as in the one-CTA kernel, over pairs instead of CTAs.
 template <int BN, int STAGES>
 struct PairSmem {
   static constexpr bool kWide = BN > 256;
