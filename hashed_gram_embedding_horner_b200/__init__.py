@@ -42,6 +42,7 @@ EXPORTED = [
     "ngram_embed_selftest_wait_timeout", "ngram_embed_fwd_static_ws", "ngram_embed_plan_set_cta_pair",
     "ngram_cache_commit", "ngram_embed_plan_set_stream_k", "ngram_embed_plan_set_pdl",
     "ngram_embed_plan_set_a_stages", "ngram_embed_plan_kernel_form", "ngram_embed_plan_set_pair_wide",
+    "ngram_embed_plan_set_sm_count",
     "ngram_embed_plan_set_output_scale", "ngram_embed_layernorm",
     "ngram_embed_bwd_workspace_bytes", "ngram_embed_bwd",
     "ngram_hash_stats_workspace_bytes", "ngram_hash_stats",
@@ -88,6 +89,7 @@ _sig("ngram_embed_plan_set_tile_n", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pair_wide", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_sm_count", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_a_stages", [_P, ctypes.c_int])
@@ -253,6 +255,11 @@ def ngram_embed_plan_set_pair_wide(plan: Plan, on):
     """True/1: the pair form's 512-column tiles; False/0: 256-column; None/-1: automatic."""
     v = -1 if on is None or on == -1 else int(bool(on))
     _check(_lib.ngram_embed_plan_set_pair_wide(plan.handle, v), "ngram_embed_plan_set_pair_wide")
+
+
+def ngram_embed_plan_set_sm_count(plan: Plan, sms: int):
+    """SMs the plan's kernels use: 0 = all of the device's; else 2 .. the device's count."""
+    _check(_lib.ngram_embed_plan_set_sm_count(plan.handle, int(sms)), "ngram_embed_plan_set_sm_count")
 
 
 def ngram_embed_plan_set_stream_k(plan: Plan, mode: int):

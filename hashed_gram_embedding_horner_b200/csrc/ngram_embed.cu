@@ -49,7 +49,8 @@ struct ngram_embed_plan {
   int64_t V[kMaxS];
   uint64_t barrett[kMaxS];
   int device;
-  int sms;
+  int sms;         // SMs the plan's kernels use (grids, stream-K shares, partial slots)
+  int sms_device;  // SMs of the device (0 without one)
   int variant;  // resolved: kTcTmaRows, kTcSplitRows or kSimt
   int tma_rows; // tensor-core kernel: A rows per tile gathered by TMA (multiple of 32; -1 = per form)
   int bn;       // tensor-core tile width (256 or 128)
@@ -275,7 +276,10 @@ int launch_tc_pair_stages(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaSt
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return NGRAM_ERR_CUDA;
     max_pairs = n;
   }
-  const int pairs = (prm.stream_k || tiles > max_pairs) ? max_pairs : tiles;
+  // co-resident pairs, within the plan's SM count (which also sizes the stream-K slots)
+  const int cap = max_pairs < p->sms / 2 ? max_pairs : p->sms / 2;
+  if (cap < 1) return NGRAM_ERR_CUDA;
+  const int pairs = (prm.stream_k || tiles > cap) ? cap : tiles;
   return launch(kern, dim3(2 * pairs), dim3(kProjThreads), L::kLaunchBytes, st, p->pdl, 2, p->maps, prm);
 }
 
@@ -595,6 +599,7 @@ int ngram_embed_plan_create(const ngram_embed_config* cfg, ngram_embed_plan** ou
     p->device = -1;
     p->sms = 0;
   }
+  p->sms_device = p->sms;
   p->tc_ok = cfg->dtype == NGRAM_BF16 && S > 0 && cfg->D % 128 == 0 && d % kBK == 0;
   p->bn = cfg->D % 256 == 0 ? 256 : 128;
   p->variant = p->tc_ok ? kTcSplitRows : kSimt;
@@ -653,6 +658,12 @@ int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_token
   const bool sk = !psk && plan->cta_pair != 1 && use_stream_k(plan, prm, num_tokens, ws);
   if (plan->cta_pair == 1 || (plan->cta_pair == -1 && !sk)) return psk ? 5 : (use_pair_wide(plan, num_tokens) ? 4 : 3);
   return sk ? 2 : 1;
+}
+
+int ngram_embed_plan_set_sm_count(ngram_embed_plan* plan, int sms) {
+  if (!plan || sms < 0 || sms == 1 || (plan->sms_device > 0 && sms > plan->sms_device)) return NGRAM_ERR_INVALID_ARG;
+  plan->sms = sms == 0 ? plan->sms_device : sms;
+  return NGRAM_OK;
 }
 
 int ngram_embed_plan_set_pair_wide(ngram_embed_plan* plan, int on) {

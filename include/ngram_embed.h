@@ -348,6 +348,13 @@ int ngram_embed_plan_set_tma_rows(ngram_embed_plan* plan, int rows);
  * (the k-block order differs). */
 int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on);
 
+/* How many SMs the plan's kernels use: 0 = all of the device's (default), else 2 ..
+ * the device's count. Grids, stream-K shares and the workspace's partial tiles follow it
+ * (ngram_embed_workspace_bytes shrinks with it), so other work can keep the remaining SMs.
+ * Without a device any count >= 2 is accepted, which lets ngram_embed_plan_kernel_form
+ * report the choice a device of that size would make. NGRAM_ERR_INVALID_ARG otherwise. */
+int ngram_embed_plan_set_sm_count(ngram_embed_plan* plan, int sms);
+
 /* CTA-pair form with 512-column tiles: each pair gathers a 256-row A block once per k-block
  * and issues two tcgen05 MMAs of N = 256 on it (half the gathered rows per FLOP of the
  * 256-column tiles); the accumulator fills all 512 TMEM columns and each half is drained and

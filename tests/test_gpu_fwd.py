@@ -423,6 +423,29 @@ def test_pair_wide_not_for_narrow_tiles(ne):
     assert ne.ngram_embed_plan_kernel_form(plan, 4096) == "cta_pair"
 
 
+@pytest.mark.parametrize("sms", [40, 9])
+def test_reduced_sm_count_every_form(ne, sms):
+    """A plan limited to fewer SMs than the device has (grids, pairs and stream-K shares
+    shrink, and so does the workspace): every kernel form still matches the oracle."""
+    cfg = small_cfg(5000, 1024, 3, 2, seed=13)
+    tokens, offsets = ragged_tokens(cfg, [700, 1, 2000, 301, 3])
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    forms = set()
+    for pair, wide, sk in ((None, None, 0), (1, 1, 0), (1, 0, 1), (1, 0, 2), (0, 0, 1), (0, 0, 2)):
+        plan = plan_for(ne, cfg, pair=pair)
+        ne.ngram_embed_plan_set_sm_count(plan, sms)
+        ne.ngram_embed_plan_set_pair_wide(plan, wide)
+        ne.ngram_embed_plan_set_stream_k(plan, sk)
+        forms.add(ne.ngram_embed_plan_kernel_form(plan, len(tokens)))
+        out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+        assert status == 0
+        assert_close(to_host_f64(out), want, what=f"{sms} SMs, pair={pair} wide={wide} stream-K={sk}")
+    assert {"cta_pair_wide", "cta_pair_stream_k", "cta_pair", "one_cta_stream_k", "one_cta"} <= forms
+
+
 def test_automatic_kernel_form(ne):
     """Prefill grids run the CTA-pair form with 512-column tiles; a 1280-token decode step at
     D = 4096 (160 tiles of 128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule;
