@@ -110,7 +110,7 @@ int ngram_embed_plan_destroy(ngram_embed_plan* plan);
 /* Device workspace bytes for calls of up to max_tokens tokens: a 33,024-byte head (the
  * status word, then the stream-K arrival counters), the [max_tokens x S] int32 index
  * buffer, then, for plans that use the tensor-core kernel, 2 x (SM count) x 128 x 256 fp32
- * stream-K partial tiles. A workspace without the partials (head + index buffer, rounded
+ * stream-K partial tiles (the plan's SM count: see ngram_embed_plan_set_sm_count). A workspace without the partials (head + index buffer, rounded
  * up to 256 bytes) is accepted too; the projection then never uses the stream-K schedule.
  * The head must be zeroed once before first use (ngram_embed_clear_status does it); the
  * rest needs no init. The kernels leave the counters zero after every call that did not
