@@ -41,3 +41,22 @@ def test_traffic_record_follows_the_code_not_the_comments(tmp_path, monkeypatch)
     # a code edit drops it
     _tree(tmp_path, {name: texts[name].replace("return", "return 1 +")})
     assert bench.profiled_traffic("k", "w") is None
+
+
+def test_reference_arm_line_on_the_host():
+    """`bench.py --impl reference` times the fp64 oracle on the host cores and prints the
+    contract's line: the same metric, unit and workload as the GPU arm, `impl` reference,
+    a cpu_baseline describing this run and an e2e object with no device copies."""
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0", "--ref-step-seconds", "0.2"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["metric"].startswith("N-gram embed tokens/s")
+    assert line["config"]["workload"] == "prefill_bf16_D2048_N3_K2" and line["steps"] == 1
+    assert line["value"] > 0 and line["n_gpus"] == 1 and line["vs_baseline"] is None
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and "sampled" in cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
