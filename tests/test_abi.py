@@ -183,3 +183,76 @@ def test_sm_count_sizes_the_stream_k_workspace(ne):
     assert lib.ngram_embed_workspace_bytes(h, 1000) == base
     assert lib.ngram_embed_plan_kernel_form(h, 32768) == 3
     lib.ngram_embed_plan_destroy(h)
+
+
+def test_next_row_entry_points_validate_on_the_host(ne):
+    """Backward, draft cache, fused decode step, amplification and hash statistics reject
+    bad arguments on the host, before any device work (no device is needed to check)."""
+    lib = ne._lib
+    rc, h = _create(ne)  # bf16, D = 2048, N = 3, K = 2: S = 4
+    assert rc == 0
+    ws, big = ctypes.c_void_p(0x10000), ctypes.c_size_t(1 << 40)
+    odd = ctypes.c_void_p(0x10008)  # 8-byte aligned only
+    fake = ctypes.c_void_p(0x20000)
+    tabs = (ctypes.c_void_p * 4)(*([0x30000] * 4))
+    E_nk = ctypes.cast(tabs, ctypes.c_void_p)
+    # amplification factor: finite and non-zero
+    for bad in (0.0, float("nan"), float("inf"), -float("inf")):
+        assert lib.ngram_embed_plan_set_output_scale(h, bad) == -1
+    assert lib.ngram_embed_plan_set_output_scale(h, -1.5) == 0 and lib.ngram_embed_plan_set_output_scale(h, 1.0) == 0
+    # LayerNorm: eps in [0, 1], sizes, pointers, alignment; nothing to do for 0 rows
+    for eps in (-0.1, 2.0, float("nan")):
+        assert lib.ngram_embed_layernorm(h, fake, 8, None, None, eps, fake, ws, big, None) == -1
+    assert lib.ngram_embed_layernorm(h, fake, -1, None, None, 1e-5, fake, ws, big, None) == -1
+    assert lib.ngram_embed_layernorm(h, None, 8, None, None, 1e-5, fake, ws, big, None) == -1
+    assert lib.ngram_embed_layernorm(h, odd, 8, None, None, 1e-5, fake, ws, big, None) == -3
+    assert lib.ngram_embed_layernorm(h, None, 0, None, None, 1e-5, None, ws, big, None) == 0
+    # backward: sizes, workspace, pointers, alignment; nothing to do without outputs or rows
+    need = lib.ngram_embed_bwd_workspace_bytes(h, 1000)
+    assert need > 0 and lib.ngram_embed_bwd_workspace_bytes(h, -1) == 0
+    assert lib.ngram_embed_bwd(h, fake, fake, -1, E_nk, fake, fake, fake, None, None, ws, big, None) == -1
+    assert lib.ngram_embed_bwd(h, fake, fake, 1000, E_nk, fake, fake, fake, None, None, ws, need - 1, None) == -4
+    assert lib.ngram_embed_bwd(h, fake, fake, 1000, E_nk, fake, fake, fake, None, None, odd, need, None) == -3
+    assert lib.ngram_embed_bwd(h, fake, None, 1000, E_nk, fake, fake, fake, None, None, ws, need, None) == -1
+    assert lib.ngram_embed_bwd(h, fake, fake, 1000, E_nk, fake, odd, fake, None, None, ws, need, None) == -3
+    assert lib.ngram_embed_bwd(h, fake, fake, 0, E_nk, fake, fake, fake, None, None, ws, need, None) == 0
+    assert lib.ngram_embed_bwd(h, fake, fake, 1000, E_nk, fake, fake, None, None, None, ws, need, None) == 0
+    rc, h32 = _create(ne, V0=1000, D=64, N=3, K=2, V=(4099, 5003, 6007, 7001), dtype=1)
+    assert lib.ngram_embed_bwd(h32, fake, fake, 10, E_nk, fake, fake, fake, None, None, ws, big, None) == -2
+    lib.ngram_embed_plan_destroy(h32)
+    # draft-phase cache
+    cache = ne._Cache(0x40000, 0x50000, 0x60000, 8, 256)
+    dc = ne._DraftCache(0x70000, 0x80000, 5, 256)
+    dneed = lib.ngram_embed_draft_workspace_bytes(h, 1280)
+    assert dneed > 0
+    assert lib.ngram_draft_cache_reset(h, None, None, 1, ws, big, None) == -1
+    assert lib.ngram_draft_cache_reset(h, ctypes.byref(dc), None, 257, ws, big, None) == -1
+    assert lib.ngram_draft_cache_reset(h, ctypes.byref(dc), None, 0, ws, big, None) == 0
+    args = lambda d, c, n, w: (h, fake, fake, 256, n, fake, E_nk, fake, ctypes.byref(c), None, ctypes.byref(d), fake,
+                               None, ws, w, None)
+    assert lib.ngram_embed_fwd_draft(*args(dc, cache, 1280, dneed - 1)) == -4
+    assert lib.ngram_embed_fwd_draft(*args(dc, cache, 0, dneed)) == 0
+    assert lib.ngram_embed_fwd_draft(*args(ne._DraftCache(0x70000, 0x80000, 0, 256), cache, 1280, dneed)) == -1
+    assert lib.ngram_embed_fwd_draft(*args(ne._DraftCache(0x70000, 0x80000, 5, 255), cache, 1280, dneed)) == -1
+    assert lib.ngram_embed_fwd_draft(*args(ne._DraftCache(0x70000, 0x80008, 5, 256), cache, 1280, dneed)) == -3
+    # fused decode step: sequences, cache, commit arguments
+    step = lambda ct, stride, cnt, n_seqs, c: (h, ct, stride, cnt, fake, fake, n_seqs, 1280, fake, E_nk, fake, c, None,
+                                              fake, ws, big, None)
+    assert lib.ngram_embed_fwd_step(*step(fake, 5, fake, 0, ctypes.byref(cache))) == -1
+    assert lib.ngram_embed_fwd_step(*step(fake, 5, fake, 256, None)) == -1
+    assert lib.ngram_embed_fwd_step(*step(None, 5, fake, 256, ctypes.byref(cache))) == -1
+    assert lib.ngram_embed_fwd_step(*step(fake, 0, fake, 256, ctypes.byref(cache))) == -1
+    lib.ngram_embed_plan_destroy(h)
+    # hash statistics (no plan): n-gram order, V0, moduli, workspace
+    moduli = (ctypes.c_int64 * 2)(1009, 262147)
+    hits, distinct = (ctypes.c_int64 * 2)(), ctypes.c_int64()
+    sneed = lib.ngram_hash_stats_workspace_bytes(1000, 262147, 2)
+    assert sneed > 0 and lib.ngram_hash_stats_workspace_bytes(-1, 10, 1) == 0
+    assert lib.ngram_hash_stats_workspace_bytes(10, 0, 1) == 0 and lib.ngram_hash_stats_workspace_bytes(10, 10, 0) == 0
+    st = lambda V0, n, mod, nm, w, wb: lib.ngram_hash_stats(V0, n, fake, fake, 4, 1000, mod, nm, hits,
+                                                          ctypes.byref(distinct), w, wb, None)
+    assert st(0, 2, moduli, 2, ws, sneed) == -1 and st(1 << 31, 2, moduli, 2, ws, sneed) == -1
+    assert st(131072, 0, moduli, 2, ws, sneed) == -1 and st(131072, 9, moduli, 2, ws, sneed) == -1
+    assert st(131072, 2, moduli, 0, ws, sneed) == -1
+    assert st(131072, 2, (ctypes.c_int64 * 2)(1009, 0), 2, ws, sneed) == -1
+    assert st(131072, 2, moduli, 2, odd, sneed) == -3 and st(131072, 2, moduli, 2, ws, sneed - 1) == -4
