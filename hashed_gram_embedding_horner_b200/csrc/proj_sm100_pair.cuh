@@ -461,7 +461,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     // output writes). Same arithmetic per element: (acc + E_0) * scale, rounded once.
     // Wide tiles: all eight warps drain half 0 first (warps 12-15 its columns 0-127, warps
     // 4-7 columns 128-255), free it, then half 1 the same way, so half 0 is free for the
-    // next tile's MMAs after half of the drain.
+    // next tile's MMAs after half of the drain. A stream-K segment that covers only part of
+    // a tile is handed to pair_sk_piece.
     constexpr int kSegs = kWide ? 2 : 1;                 // accumulator halves, in drain order
     constexpr int kSegChunks = (kWide ? 128 : kMmaN) / 32;
     constexpr int kChunks = kSegs * kSegChunks;
