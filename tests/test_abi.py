@@ -15,8 +15,6 @@ HEADER = os.path.join(ROOT, "include", "ngram_embed.h")
 
 @pytest.fixture(scope="module")
 def ne():
-    from hashed_gram_embedding_horner_b200 import build
-    build.build()
     import hashed_gram_embedding_horner_b200 as m
     return m
 
