@@ -1327,35 +1327,42 @@ int ngram_embed_clear_status(void* workspace, void* stream) {
 // Some callers cannot call cudaMalloc: plugin hosts that hand a layer only its input and
 // output buffers, and latency-critical loops where cudaMalloc's implicit device-wide
 // synchronisation is not allowed. ngram_embed_fwd_static_ws runs the same forward pass as
-// ngram_embed_fwd, but its workspace (the status word and the per-token index buffer) is
-// the fixed array below, compiled into the library. Every GPU that loads the library holds
-// these kNoAllocScratchBytes until the process exits.
+// ngram_embed_fwd, but its workspace (the head with the status word and the stream-K
+// arrival counters, the per-token index buffer and, when they fit, the stream-K partial
+// tiles) is the fixed array below, compiled into the library. Every GPU that loads the
+// library holds these kNoAllocScratchBytes until the process exits.
 //
 // In host code `g_noalloc_scratch` names a host-side stand-in, not a device address, so the
 // array's device address is looked up with cudaGetSymbolAddress once per device, with that
 // device current, by the first call made on that device (that first call should come
-// before any stream capture). All calls share the array and it keeps the last call's
-// contents: each call zeroes the status word before use, and calls that overlap on the GPU
-// (concurrent streams) race on the array.
+// before any stream capture). A failed lookup is not remembered: the next call tries again.
+// All calls share the array and it keeps the last call's contents: each call zeroes the
+// whole head (status word and arrival counters, which a call that stopped at a bounded-wait
+// timeout may leave non-zero) before use, and calls that overlap on the GPU (concurrent
+// streams) race on the array.
 // ---------------------------------------------------------------------------------------
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB: status header + T*S indices
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
 constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::once_flag g_noalloc_once[kNoAllocMaxDevices];
+std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
-cudaError_t g_noalloc_err[kNoAllocMaxDevices] = {};
 
+// The array's device address on `device` (current), or nullptr if the lookup failed.
 void* noalloc_scratch(int device) {
   if (device < 0 || device >= kNoAllocMaxDevices) return nullptr;
-  std::call_once(g_noalloc_once[device], [device] {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[device]) {
     void* p = nullptr;
-    g_noalloc_err[device] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    g_noalloc_ptr[device] = g_noalloc_err[device] == cudaSuccess ? p : nullptr;
-  });
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess) {
+      g_noalloc_ptr[device] = p;
+    } else {
+      cudaGetLastError();  // clear the error; a later call retries the lookup
+    }
+  }
   return g_noalloc_ptr[device];
 }
 
@@ -1373,7 +1380,7 @@ extern "C" int ngram_embed_fwd_static_ws(const ngram_embed_plan* plan, const int
   void* ws = noalloc_scratch(plan->device);
   if (!ws) return NGRAM_ERR_CUDA;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess) return NGRAM_ERR_CUDA;  // status word
+  if (cudaMemsetAsync(ws, 0, kHeadBytes, st) != cudaSuccess) return NGRAM_ERR_CUDA;  // status word + counters
   rc = ngram_embed_fwd(plan, tokens, seq_offsets, num_seqs, num_tokens, E0, E_nk, W_stacked, cache, cache_slots,
                        out, ws, kNoAllocScratchBytes, stream);
   if (rc) return rc;

@@ -207,13 +207,18 @@ int ngram_cache_rollback(const ngram_embed_plan* plan, const ngram_cache* cache,
  * device-wide synchronisation is not allowed). The paper has no counterpart: this is an
  * interface convenience. Same arguments and results as ngram_embed_fwd, but the workspace
  * is a fixed 4 MiB array inside the library (every GPU that loads the library holds it
- * until exit), so calls need ngram_embed_workspace_bytes(plan, num_tokens) <= 4 MiB
- * (about num_tokens * S * 4 bytes); larger calls return NGRAM_ERR_WORKSPACE and launch
- * nothing. Allocates nothing. The first call on a device looks up the array's device
- * address (once per device); make that first call before any stream capture. Each call
- * zeroes the array's status word, then, if status_out (a device int32) is not NULL, copies
- * the call's device status bits there on `stream`. All calls share the one array: calls
- * that overlap on the GPU (for example on two streams) race and must be avoided. */
+ * until exit). A call needs the workspace head and its index buffer to fit:
+ * 33,024 + num_tokens * S * 4 bytes (rounded up to 256) <= 4 MiB, about 131,000 tokens at
+ * S = 8; larger calls return NGRAM_ERR_WORKSPACE and launch nothing. The stream-K schedule
+ * runs only when its partial tiles fit too (2 x SMs x 128 x 256 x 4 bytes: a plan limited
+ * to a few SMs by ngram_embed_plan_set_sm_count). Allocates nothing. The first call on a
+ * device looks up the array's device address (once per device; a failed lookup returns
+ * NGRAM_ERR_CUDA and is retried by the next call); make that first call before any stream
+ * capture. Each call zeroes the array's whole head (the status word and the stream-K
+ * arrival counters) on `stream`, then, if status_out (a device int32) is not NULL, copies
+ * the call's device status bits there on `stream`. All calls share the one array and it
+ * keeps the last call's contents: calls that overlap on the GPU (for example on two
+ * streams) race and must be avoided. */
 int ngram_embed_fwd_static_ws(const ngram_embed_plan* plan, const int32_t* tokens,
                               const int32_t* seq_offsets, int32_t num_seqs, int64_t num_tokens,
                               const void* E0, const void* const* E_nk, const void* W_stacked,

@@ -4,8 +4,11 @@ cudaMalloc's device-wide synchronisation is not allowed). Its workspace is a fix
 inside the library, so the caller passes only inputs and outputs.
 
 Checked through the C ABI against ngram_embed_fwd (caller-provided workspace) on two
-calls in a row, within the tolerance the other parity tests use. This file is collected
-last so that a failure here comes after every other test has run.
+calls in a row: the same kernels run on the same inputs, so the bits must be equal (which
+also puts them within the tolerance the other parity tests use). Also covered: the stream-K
+schedule running inside the fixed array (a plan limited to 8 SMs, whose partial tiles fit),
+and the status word that each call clears and reports through status_out. This file is
+collected last so that a failure here comes after every other test has run.
 """
 import ctypes
 
@@ -63,6 +66,62 @@ def test_static_workspace_forward_matches_fwd(ne):
         assert status.item() == 0
         assert ne.ngram_embed_get_status(ws) == 0
         _close(got, want)
+        assert torch.equal(got, want)
+
+
+def _noalloc_cfg():
+    return configs.NgramConfig(name="noalloc", V0=6000, D=512, N=5, K=2,
+                               V_nk=tuple(configs.primes_from(20000, 8)), dtype="bf16", seed=5)
+
+
+def test_static_workspace_stream_k_matches_fwd(ne):
+    """With 8 SMs the stream-K partial tiles (2 x 8 x 128 KB) fit the fixed array, so the
+    schedule whose arrival counters and partials live in it runs; two calls in a row equal
+    ngram_embed_fwd with its own workspace (same schedule) bit for bit."""
+    cfg = _noalloc_cfg()
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
+    ne.ngram_embed_plan_set_sm_count(plan, 8)
+    ne.ngram_embed_plan_set_stream_k(plan, 1)
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    for call, lengths in enumerate(([3, 330, 97], [129, 1, 0, 300])):
+        off_h = gen.offsets_from_lengths(lengths)
+        T = int(off_h[-1])
+        assert ne.ngram_embed_plan_kernel_form(plan, T) == "one_cta_stream_k"
+        assert ne.ngram_embed_workspace_bytes(plan, T) <= 4 << 20  # the partials fit the fixed array
+        tokens = torch.from_numpy(gen.zipf_tokens(60 + call, T, cfg.V0)).cuda()
+        offsets = torch.from_numpy(off_h).cuda()
+        want = torch.empty((T, cfg.D), dtype=torch.bfloat16, device="cuda")
+        ws = ne.new_workspace(plan, T)
+        ne.ngram_embed_fwd(plan, tokens, offsets, E0, E, W, want, ws)
+        got = torch.full_like(want, float("nan"))
+        assert _static_ws_fwd(ne, plan, tokens, offsets, E0, E, W, got, status) == 0
+        torch.cuda.synchronize()
+        assert status.item() == 0 and ne.ngram_embed_get_status(ws) == 0
+        assert torch.equal(got, want)
+
+
+def test_static_workspace_reports_and_clears_device_status(ne):
+    """A token id outside [0, V0) sets BAD_TOKEN in the call's status (written to status_out);
+    the next, clean call starts from a cleared head and reports 0."""
+    cfg = _noalloc_cfg()
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
+    off_h = gen.offsets_from_lengths([40, 90])
+    tok_h = gen.zipf_tokens(7, int(off_h[-1]), cfg.V0)
+    offsets = torch.from_numpy(off_h).cuda()
+    out = torch.empty((len(tok_h), cfg.D), dtype=torch.bfloat16, device="cuda")
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    bad = tok_h.copy()
+    bad[17] = cfg.V0  # one past the last id
+    assert _static_ws_fwd(ne, plan, torch.from_numpy(bad).cuda(), offsets, E0, E, W, out, status) == 0
+    torch.cuda.synchronize()
+    assert ne.status_names(status.item()) == ["BAD_TOKEN"]
+    assert _static_ws_fwd(ne, plan, torch.from_numpy(tok_h).cuda(), offsets, E0, E, W, out, status) == 0
+    torch.cuda.synchronize()
+    assert status.item() == 0
 
 
 def test_static_workspace_rejects_calls_above_its_size(ne):
