@@ -1,10 +1,17 @@
 """Benchmark of the hashed N-gram embedding forward on B200: one JSON line.
 
-Workload (default): prefill, V0 = 131072, D = 2048, N = 3, K = 2 (4 sub-tables of width
-512, V_{n,k} ~ 2.16M primes), 8 sequences x 4096 Zipf(1.1) tokens, bf16 tables (8.9 GB).
-A step is one call of the C ABI's ngram_embed_fwd over the whole batch (context + hash,
-gather, projection, E_0 add, scale), inputs resident in HBM; the L2 is flushed (a
-256 MB write) between timed steps, outside the timed events.
+Headline workload: the full-scale layer, V0 = 131072, D = 4096, N = 5, K = 2 (8 sub-tables of
+width 512, V_{n,k} ~ 7.27M primes: 59.6 GB of bf16 sub-tables + 1.07 GB E_0 + 33.5 MB W),
+prefill of 8 sequences x 4096 Zipf(1.1) tokens. A step is one call of the C ABI's
+ngram_embed_fwd over the whole batch (context + hash, gather, projection, E_0 add, scale),
+inputs resident in HBM; the L2 is flushed (a 256 MB write) between timed steps, outside
+the timed events.
+
+The same line carries, as sub-objects: the other prefill workloads (D = 2048, N = 3, K = 2;
+D = 4096, N = 5, K = 2 with varied lengths), each with its own roofline; speculative decode
+(1000 steps of 256 sequences x 5 ids through the N-gram cache) on the full-scale layer and
+on the D = 4096, N = 3, K = 4 layer; the backward pass (D = 2048 layer); the LayerNorm
+amplification; the hash statistics sweep; and the fp64 CPU oracle's rate on the host cores.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -31,16 +38,23 @@ from synth import configs, gen, workloads  # noqa: E402
 METRIC = "N-gram embed tokens/s (prefill & decode) + % of tensor/HBM roofline, 1 B200"
 UNIT = "tokens/s"
 WORKLOADS = {
+    "full_scale_prefill": configs.FULL_SCALE,
     "prefill_d2048": configs.PREFILL_D2048,
     "prefill_varlen_d4096": configs.PREFILL_D4096_VARLEN,
-    "full_scale_prefill": configs.FULL_SCALE,
-    # small case of the prefill_d2048 kernel shape for profiler captures: ~1.1 GB of
-    # tables (still far above the 126 MB L2), 2 x 4096 tokens
+    # small cases of the prefill kernel shapes for profiler captures: the same tokens and
+    # layer widths over ~1-3.5 GB of tables (still far above the 126 MB L2)
     "profile_d2048": configs.PREFILL_D2048.with_(
-        name="profile_bf16_D2048_N3_K2_small", num_seqs=2,
+        name="profile_bf16_D2048_N3_K2_small",
         V_nk=tuple(configs.primes_from(270000 + 131072 // 2, 4))),
+    "profile_full_scale": configs.FULL_SCALE.with_(
+        name="profile_full_scale_bf16_D4096_N5_K2_small",
+        V_nk=tuple(configs.primes_from(300000 + 131072 // 2, 8))),
 }
+HEADLINE = "full_scale_prefill"
+# the other prefill workloads, measured in the same run (each with its own roofline)
+SUB_PREFILL = ("prefill_varlen_d4096", "prefill_d2048")
 DECODE_WORKLOADS = {
+    "full_scale_decode": configs.FULL_SCALE_DECODE,
     "spec_decode": configs.SPEC_DECODE,
     # small case of the spec_decode kernel shapes for profiler captures: 8 sub-tables of
     # ~300k rows (2.5 GB, still far above the 126 MB L2)
@@ -49,6 +63,7 @@ DECODE_WORKLOADS = {
         V_nk=tuple(configs.primes_from(300000 + 131072 // 2, 8))),
 }
 L2_FLUSH_BYTES = 256 << 20
+TRAFFIC_RECORDS = os.path.join("profiles", "traffic_records.json")
 
 
 # the projection kernels' device code, stage counts and tile shapes
@@ -79,20 +94,21 @@ def kernel_source_hash(read=None) -> str:
 
 
 def profiled_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) recorded in a
-    profiles/*.md summary for this kernel and workload, if it was taken from these sources;
-    else None."""
-    import glob
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of `kernel` at
+    `workload`, from the committed record of ncu captures, if it was taken from these
+    sources; else None. A record taken on a smaller case of the same kernel shape carries
+    the factor that scales it to one launch of `workload` (the units the launches process)."""
+    path = os.path.join(ROOT, TRAFFIC_RECORDS)
+    if not os.path.exists(path):
+        return None
+    try:
+        records = json.load(open(path))["records"]
+    except (ValueError, KeyError):
+        return None
     src = kernel_source_hash()
-    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
-        for ln in open(f):
-            if ln.startswith("traffic_record:"):
-                try:
-                    rec = json.loads(ln.split(":", 1)[1])
-                except ValueError:
-                    continue
-                if rec.get("kernel") == kernel and rec.get("workload") == workload and rec.get("source_sha256") == src:
-                    return float(rec["bytes_per_launch"])
+    for rec in records:
+        if rec.get("kernel") == kernel and rec.get("workload") == workload and rec.get("source_sha256") == src:
+            return float(rec["bytes_per_launch"]) * float(rec.get("scale_to_workload", 1.0))
     return None
 
 
@@ -181,83 +197,241 @@ def dist_env():
     return ws, rank, local
 
 
+def tokens_per_step(cfg) -> int:
+    return cfg.num_seqs * cfg.seq_len if cfg.seq_len else cfg.extras.get("total_tokens")
+
+
 # ------------------------------------------------------------------ reference arm: the oracle
 
-def oracle_sample_rate(cfg, budget_s: float = 15.0, max_tokens: int = 32768):
-    """Time the fp64 CPU oracle (exact hash + Eq. 3 combine) on a bounded sample of the
-    workload's tokens; the table rows it reads are regenerated beforehand (not timed)."""
-    import oracle
-    from synth.tables import host_W, host_rows
-    tokens, offsets = workloads.prefill_tokens(cfg)
-    W = host_W(cfg)
-    rng = np.random.default_rng(0)
+class OracleSampler:
+    """Times the fp64 CPU oracle (exact hash + Eq. 3 combine) on bounded samples of a
+    prefill workload's tokens; the table rows a sample reads are regenerated beforehand,
+    outside the timed part."""
 
-    def run(n):
-        rows = np.sort(rng.choice(len(tokens), size=n, replace=False))
-        win = oracle.context_windows(cfg.N, tokens, offsets)[rows]
+    def __init__(self, cfg):
+        import oracle
+        from synth.tables import host_W
+        self.oracle, self.cfg = oracle, cfg
+        self.tokens, self.offsets = workloads.prefill_tokens(cfg)
+        self.windows = oracle.context_windows(cfg.N, self.tokens, self.offsets)
+        self.W = host_W(cfg)
+        self.rng = np.random.default_rng(0)
+
+    def run(self, n: int) -> float:
+        """Seconds of oracle work for n sampled tokens (hash + combine)."""
+        from synth.tables import host_rows
+        cfg, o = self.cfg, self.oracle
+        rows = np.sort(self.rng.choice(len(self.tokens), size=n, replace=False))
+        win = self.windows[rows]
         t0 = time.perf_counter()
-        idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, win)
+        idx = o.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, win)
         t_hash = time.perf_counter() - t0
-        e0 = host_rows(cfg, gen.TAG_E0, tokens[rows], cfg.D, cfg.e_std)
+        e0 = host_rows(cfg, gen.TAG_E0, self.tokens[rows], cfg.D, cfg.e_std)
         sub = np.stack([host_rows(cfg, gen.TAG_SUBTABLE0 + s, idx[:, s], cfg.d, cfg.e_std) for s in range(cfg.S)], 1)
         t1 = time.perf_counter()
-        oracle.combine(cfg.D, cfg.S, e0, sub, W)
+        o.combine(cfg.D, cfg.S, e0, sub, self.W)
         return t_hash + time.perf_counter() - t1
 
-    n = max(oracle.num_threads(), 8)
-    dt = run(n)
-    n2 = int(min(max_tokens, max(n, n * budget_s / max(dt, 1e-6) * 0.8)))
-    dt2 = run(n2)
-    return {"value": n2 / dt2, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{n2} tokens sampled from the workload (exact hash + fp64 Eq. 3), {dt2:.1f} s"}
+    def size_for(self, budget_s: float, max_tokens: int) -> int:
+        """Tokens that take about `budget_s` of oracle time (from a short calibration run)."""
+        n = max(self.oracle.num_threads(), 8)
+        dt = self.run(n)
+        return int(min(max_tokens, max(n, n * budget_s / max(dt, 1e-6) * 0.8)))
+
+
+def oracle_sample_rate(cfg, budget_s: float = 15.0, max_tokens: int = 32768):
+    """The oracle's tokens/s on one bounded sample of the workload (the cpu_baseline)."""
+    s = OracleSampler(cfg)
+    n = s.size_for(budget_s, max_tokens)
+    dt = s.run(n)
+    return {"value": n / dt, "unit": UNIT, "cores": s.oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} tokens sampled from the workload (exact hash + fp64 Eq. 3), {dt:.1f} s"}
 
 
 def run_reference(args, cfg):
     ws, rank, _ = dist_env()
     if rank != 0:
         return
-    steps = []
-    per = None
+    s = OracleSampler(cfg)
+    n = s.size_for(args.ref_step_seconds, 2048)
+    times = []
     for i in range(args.warmup + args.steps):
-        r = oracle_sample_rate(cfg, budget_s=args.ref_step_seconds, max_tokens=2048)
+        dt = s.run(n)
         if i >= args.warmup:
-            steps.append(r)
-        per = r
-    value = float(np.mean([s["value"] for s in steps]))
+            times.append(dt)
+    sec = float(np.mean(times))
+    value = n / sec
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * cfg.num_seqs * cfg.seq_len / value
-        if cfg.seq_len else None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "steps": args.steps, "warmup": args.warmup,
+        # each step is one timed sample of `sample_tokens_per_step` tokens of the workload
+        "ms_per_step": 1e3 * sec, "sample_tokens_per_step": n,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_block(cfg, args),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": per["cores"], "kind": "oracle",
-                         "sample": per["sample"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": s.oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{n} tokens sampled from the workload per step (exact hash + fp64 Eq. 3), "
+                                   f"{sec:.2f} s per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 def config_block(cfg, args):
-    T = cfg.num_seqs * cfg.seq_len if cfg.seq_len else cfg.extras.get("total_tokens")
     return {"workload": cfg.name, "V0": cfg.V0, "D": cfg.D, "N": cfg.N, "K": cfg.K, "V_nk": list(cfg.V_nk),
-            "tokens_per_step": T, "num_seqs": cfg.num_seqs, "token_dist": f"zipf({cfg.zipf_alpha})",
+            "tokens_per_step": tokens_per_step(cfg), "num_seqs": cfg.num_seqs, "token_dist": f"zipf({cfg.zipf_alpha})",
             "tables_gb": round(cfg.table_bytes() / 1e9, 2), "parallelism": f"dp{args.gpus}",
             "l2": "flushed between timed steps (256 MB write)"}
 
 
+def events(n):
+    import torch
+    return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+
+
+def kernel_of_form(form: str) -> str:
+    return {"cta_pair": "proj_sm100_pair_kernel", "cta_pair_wide": "proj_sm100_pair_kernel",
+            "cta_pair_stream_k": "proj_sm100_pair_kernel", "one_cta": "proj_sm100_kernel",
+            "one_cta_stream_k": "proj_sm100_kernel", "cuda_cores": "proj_simt_kernel"}[form]
+
+
+# ------------------------------------------------------------------ prefill
+
+def run_prefill(ne, cfg, tables, args, dev, flush, world, rank, clock_gpu=None, e2e=True):
+    """Time `args.steps` whole-layer steps of a prefill workload (L2 flushed between steps),
+    then its dominant kernel alone (the projection) and the hash, and, if `e2e`, the same
+    call with host buffers (H2D of the inputs and D2H of the output inside the timed region).
+    Returns (result dict, output tensor, workspace, plan)."""
+    import torch
+    E0, E, W = tables
+    stream = torch.cuda.current_stream()
+    tokens_h, offsets_h = workloads.prefill_tokens(rank_config(cfg, rank))
+    T = len(tokens_h)
+    tokens = torch.from_numpy(tokens_h).to(dev)
+    offsets = torch.from_numpy(offsets_h).to(dev)
+    plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
+    ws = ne.new_workspace(plan, T)
+    out = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        ne.ngram_embed_fwd(plan, tokens, offsets, E0, E, W, out, ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if ne.ngram_embed_get_status(ws) != 0:
+        raise RuntimeError(f"device status {ne.status_names(ne.ngram_embed_get_status(ws))}")
+
+    clk = ClockSampler(clock_gpu) if clock_gpu is not None else None
+    if clk:
+        clk.__enter__()
+    ev = events(args.steps)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    total_ms = float(np.sum([a.elapsed_time(b) for a, b in ev]))
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_per_step = total_ms / args.steps
+
+    # the dominant kernel alone: the projection (gather + tcgen05 GEMM + epilogue) from
+    # precomputed indices; and the hash alone. CUDA events on the launching stream.
+    idx = torch.empty((T, cfg.S), dtype=torch.int32, device=dev)
+    ne.ngram_hash_indices(plan, tokens, offsets, idx, ws, stream=stream)
+    pe, hs = events(args.steps), events(args.steps)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        hs[i][0].record(stream)
+        ne.ngram_hash_indices(plan, tokens, offsets, idx, ws, stream=stream)
+        hs[i][1].record(stream)
+        flush.fill_((i + 1) & 0xFF)
+        pe[i][0].record(stream)
+        ne.ngram_embed_project(plan, tokens, idx, E0, E, W, out, ws, stream=stream)
+        pe[i][1].record(stream)
+    torch.cuda.synchronize()
+    if clk:
+        clk.__exit__(None, None, None)
+    proj_ms = float(np.mean([a.elapsed_time(b) for a, b in pe]))
+    hash_ms = float(np.mean([a.elapsed_time(b) for a, b in hs]))
+    pk = peaks()
+    flops = 2.0 * T * cfg.D * cfg.D
+    achieved = flops / (proj_ms / 1e3) / 1e12
+    form = ne.ngram_embed_plan_kernel_form(plan, T)
+    kernel = kernel_of_form(form)
+    algo_bytes = T * (2 * cfg.D * 2 + 4) + cfg.D * cfg.D * 2
+    res = {
+        "workload": cfg.name, "tokens_per_step": T, "steps": args.steps, "ms_per_step": ms_per_step,
+        "value": world * T / (ms_per_step / 1e3), "unit": UNIT, "tables_gb": round(cfg.table_bytes() / 1e9, 2),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_tflops"], "traffic": profiled_traffic(kernel, cfg.name),
+                     "kernel": kernel + " (" + form + "): fused sub-row gather + tcgen05 projection + E_0 add + scale",
+                     "kernel_ms": proj_ms, "peak_source": pk["source"] + " (burst)",
+                     "layer_frac": (flops / (ms_per_step / 1e3) / 1e12) / pk["bf16_tflops"],
+                     "hash_kernel_ms": hash_ms, "flops_per_launch": flops, "algorithmic_bytes": algo_bytes},
+    }
+    if clk:
+        res["clocks"] = clk.summary()
+    if e2e:
+        # end to end through the C ABI with host buffers: H2D inputs, fwd, D2H output
+        tok_pin = torch.from_numpy(tokens_h).pin_memory()
+        off_pin = torch.from_numpy(offsets_h).pin_memory()
+        out_pin = torch.empty((T, cfg.D), dtype=torch.bfloat16).pin_memory()
+        tok_d, off_d = torch.empty_like(tokens), torch.empty_like(offsets)
+        ee = events(args.steps)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ee[i][0].record(stream)
+            tok_d.copy_(tok_pin, non_blocking=True)
+            off_d.copy_(off_pin, non_blocking=True)
+            ne.ngram_embed_fwd(plan, tok_d, off_d, E0, E, W, out, ws, stream=stream)
+            out_pin.copy_(out, non_blocking=True)
+            ee[i][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ee])), world, dev)
+        res["e2e"] = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
+                      "h2d_bytes_per_step": tokens.numel() * 4 + offsets.numel() * 4,
+                      "d2h_bytes_per_step": out.numel() * 2}
+    res["device_status"] = ne.ngram_embed_get_status(ws)
+    return res, out, ws, plan, (tokens, idx)
+
+
+def run_layernorm(ne, plan, out, ws, args, flush):
+    """Embedding amplification by LayerNorm over the layer output (HBM-bound: the output read
+    once from HBM, written once), in place, L2 flushed before each launch."""
+    import torch
+    stream = torch.cuda.current_stream()
+    ln_ev = events(args.steps)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ln_ev[i][0].record(stream)
+        ne.ngram_embed_layernorm(plan, out, out, ws, eps=1e-5, stream=stream)
+        ln_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ln_ms = float(np.mean([a.elapsed_time(b) for a, b in ln_ev]))
+    ln_bytes = 2 * out.numel() * out.element_size()
+    pk = peaks()
+    return {"layernorm_ms": ln_ms, "bytes": ln_bytes, "gbs": ln_bytes / (ln_ms / 1e3) / 1e9,
+            "frac_hbm": ln_bytes / (ln_ms / 1e3) / 1e9 / pk["hbm_gbs"], "tokens": out.shape[0], "D": out.shape[1]}
+
+
 # ------------------------------------------------------------------ decode (speculative, ring cache)
 
-def run_decode(ne, cfg, steps: int, warmup: int, dev, rank: int = 0):
+def run_decode(ne, cfg, tables, steps: int, warmup: int, dev, rank: int = 0, extras: bool = True):
     """Speculative decode: per step, every sequence brings 5 ids (x0 + 4 drafts); the layer
     reads each sequence's context from the N-gram cache ring, then the accepted prefix
     (1 + a ids, a ~ U{0..4}) is committed. `steps` steps are captured in one CUDA graph and
     replayed; the L2 is not flushed between steps (steady state: W stays L2-resident, the
-    27 GB of sub-tables do not)."""
+    tens of GB of sub-tables do not)."""
     import torch
-    from synth.tables import device_tables
+    E0, E, W = tables
     ds = workloads.DecodeStream(rank_config(cfg, rank))  # this rank's streams; tables shared
     B, P, C = ds.B, ds.P, cfg.ring_capacity
     T = B * P
-    E0, E, W = device_tables(cfg)
     plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
     ws = ne.new_workspace(plan, T)
     cache = ne.Cache.empty(B, C, device=dev)
@@ -304,6 +478,19 @@ def run_decode(ne, cfg, steps: int, warmup: int, dev, rank: int = 0):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     status = ne.ngram_embed_get_status(ws)
+    del graphs
+    pk = peaks()
+    flops = 2.0 * T * cfg.D * cfg.D
+    res = {
+        "workload": cfg.name, "steps": steps, "tokens_per_step": T, "ms_per_step": ms / steps,
+        "value": steps * T / (ms / 1e3), "unit": UNIT, "graph": True, "gpu_launches_per_step": 2,
+        "layer_tflops": flops / (ms / steps / 1e3) / 1e12,
+        "layer_frac": flops / (ms / steps / 1e3) / 1e12 / pk["bf16_tflops"],
+        "kernel_form": ne.ngram_embed_plan_kernel_form(plan, T),
+    }
+    if not extras:
+        res["device_status"] = status
+        return res
     # The projection alone at this shape, and the stand-alone hash and gather stages. Each is
     # timed as `n` launches on `n` different steps' inputs captured in one CUDA graph (so
     # host launch overhead is not in the number and the sub-rows are not L2 hits from the
@@ -369,25 +556,34 @@ def run_decode(ne, cfg, steps: int, warmup: int, dev, rank: int = 0):
     plain_ms = timed(lambda i, st: ne.ngram_embed_fwd(plan, tok_all[i], offsets, E0, E, W, out, ws, cache=cache,
                                                       stream=st))
     hit_rate = hits_d.item() / (T * (3 + 4 * n_k))  # timed(): 3 eager calls, then 1 + 3 replays of n_k
-
-    pk = peaks()
-    flops = 2.0 * T * cfg.D * cfg.D
-    res = {
-        "workload": cfg.name, "steps": steps, "tokens_per_step": T, "ms_per_step": ms / steps,
-        "value": steps * T / (ms / 1e3), "unit": UNIT, "graph": True, "gpu_launches_per_step": 2,
-        "layer_tflops": flops / (ms / steps / 1e3) / 1e12,
+    res.update({
         "projection": {"ms": proj_ms, "tflops": flops / (proj_ms / 1e3) / 1e12,
                        "frac": flops / (proj_ms / 1e3) / 1e12 / pk["bf16_tflops"]},
         "hash_ms": hash_ms,
-        "gather_stage": {"ms": gather_ms, "bytes": gather_bytes, "gbs": gather_bytes / (gather_ms / 1e3) / 1e9,
-                         "frac_hbm": gather_bytes / (gather_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+        "gather_stage_standalone": {
+            "what": "ngram_embed_gather alone (the step's sub-rows and E_0 rows copied out); not a kernel of the "
+                    "timed step, whose projection gathers its rows itself",
+            "ms": gather_ms, "bytes": gather_bytes, "gbs": gather_bytes / (gather_ms / 1e3) / 1e9,
+            "frac_hbm": gather_bytes / (gather_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
         "draft_cache": {"verify_all_hits_ms": verify_ms, "draft_step_4_of_5_hits_ms": draft_ms,
                         "plain_forward_ms": plain_ms, "verify_hit_rate": hit_rate},
         "device_status": status,
-    }
-    del graphs, E0, E, W
-    torch.cuda.empty_cache()
+    })
     return res
+
+
+def tables_for(cfg, held):
+    """The device tables of `cfg`: the ones already held when they are identical, else freshly
+    filled ones (the held ones are released first)."""
+    import torch
+    from synth.tables import device_tables
+    if held[0] is not None and configs.same_tables(held[0], cfg):
+        return held[1]
+    held[0] = held[1] = None
+    torch.cuda.empty_cache()
+    t = device_tables(cfg)
+    held[0], held[1] = cfg, t
+    return t
 
 
 # ------------------------------------------------------------------ our arm
@@ -397,15 +593,17 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="prefill_d2048", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-step-seconds", type=float, default=8.0)
-    ap.add_argument("--no-decode", action="store_true", help="skip the speculative-decode measurement")
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--no-decode", action="store_true", help="skip the speculative-decode measurements")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward (training) measurement")
     ap.add_argument("--no-stats", action="store_true", help="skip the hash-statistics sweep")
-    ap.add_argument("--decode-steps", type=int, default=100)
-    ap.add_argument("--decode-workload", default="spec_decode", choices=sorted(DECODE_WORKLOADS))
+    ap.add_argument("--no-sub", action="store_true", help="skip the other prefill workloads")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--decode-workload", default=None, choices=sorted(DECODE_WORKLOADS),
+                    help="with --decode-only: the one decode workload to run")
     ap.add_argument("--decode-only", action="store_true",
                     help="only the speculative-decode measurement (one JSON line with the decode object)")
     ap.add_argument("--profile-only", action="store_true",
@@ -429,187 +627,79 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
+    held = [None, None]  # (config, tables) currently on the device
+
     if args.decode_only:
-        decode = run_decode(ne, DECODE_WORKLOADS[args.decode_workload], args.decode_steps, max(args.warmup, 3), dev,
-                            rank=rank)
-        decode["ms_per_step"] = max_over_ranks(decode["ms_per_step"], world, dev)
-        decode["value"] = world * decode["tokens_per_step"] / (decode["ms_per_step"] / 1e3)
+        names = [args.decode_workload] if args.decode_workload else ["full_scale_decode", "spec_decode"]
+        dec = {}
+        for name in names:
+            dcfg = DECODE_WORKLOADS[name]
+            d = run_decode(ne, dcfg, tables_for(dcfg, held), args.decode_steps, max(args.warmup, 3), dev, rank=rank)
+            d["ms_per_step"] = max_over_ranks(d["ms_per_step"], world, dev)
+            d["value"] = world * d["tokens_per_step"] / (d["ms_per_step"] / 1e3)
+            dec[dcfg.name] = d
         if rank == 0:
-            print(json.dumps({"decode_only": True, "decode": decode}), flush=True)
+            print(json.dumps({"decode_only": True, "decode": dec}), flush=True)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
         return
 
-    # each rank: its own batch of the same shape (seeded per rank), tables identical
-    tokens_h, offsets_h = workloads.prefill_tokens(rank_config(cfg, rank))
-    T, B = len(tokens_h), len(offsets_h) - 1
-    E0, E, W = device_tables(cfg)
-    tokens = torch.from_numpy(tokens_h).to(dev)
-    offsets = torch.from_numpy(offsets_h).to(dev)
-    plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
-    ws = ne.new_workspace(plan, T)
-    out = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    def step():
-        ne.ngram_embed_fwd(plan, tokens, offsets, E0, E, W, out, ws, stream=stream)
-
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
-    if ne.ngram_embed_get_status(ws) != 0:
-        raise RuntimeError(f"device status {ne.status_names(ne.ngram_embed_get_status(ws))}")
     if args.profile_only:
-        for _ in range(args.steps):
-            step()
+        E0, E, W = device_tables(cfg)
+        tokens_h, offsets_h = workloads.prefill_tokens(cfg)
+        tokens, offsets = torch.from_numpy(tokens_h).to(dev), torch.from_numpy(offsets_h).to(dev)
+        plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
+        ws = ne.new_workspace(plan, len(tokens_h))
+        out = torch.empty((len(tokens_h), cfg.D), dtype=torch.bfloat16, device=dev)
+        for _ in range(max(args.warmup, 3) + args.steps):
+            ne.ngram_embed_fwd(plan, tokens, offsets, E0, E, W, out, ws, stream=stream)
         torch.cuda.synchronize()
         print(json.dumps({"profile_only": cfg.name, "steps": args.steps,
                           "status": ne.ngram_embed_get_status(ws)}), flush=True)
         return
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = float(np.sum(step_ms))
-    total_ms = max_over_ranks(total_ms, world, dev)
-    if world > 1:
-        dist.barrier()
-    ms_per_step = total_ms / args.steps
-    value = world * T / (ms_per_step / 1e3)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    # --- dominant kernel alone: the projection (gather + tcgen05 GEMM + epilogue) from
-    # precomputed indices, CUDA events on the launching stream.
-    idx = torch.empty((T, cfg.S), dtype=torch.int32, device=dev)
-    ne.ngram_hash_indices(plan, tokens, offsets, idx, ws, stream=stream)
-    pe = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    hs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        hs[i][0].record(stream)
-        ne.ngram_hash_indices(plan, tokens, offsets, idx, ws, stream=stream)
-        hs[i][1].record(stream)
-        flush.fill_((i + 1) & 0xFF)
-        pe[i][0].record(stream)
-        ne.ngram_embed_project(plan, tokens, idx, E0, E, W, out, ws, stream=stream)
-        pe[i][1].record(stream)
-    torch.cuda.synchronize()
-    proj_ms = float(np.mean([a.elapsed_time(b) for a, b in pe]))
-    hash_ms = float(np.mean([a.elapsed_time(b) for a, b in hs]))
-    pk = peaks()
-    flops = 2.0 * T * cfg.D * cfg.D
-    achieved = flops / (proj_ms / 1e3) / 1e12
-    form = ne.ngram_embed_plan_kernel_form(plan, T)
-    kernel_name = {"cta_pair": "proj_sm100_pair_kernel", "cta_pair_wide": "proj_sm100_pair_kernel",
-                   "cta_pair_stream_k": "proj_sm100_pair_kernel",
-                   "one_cta": "proj_sm100_kernel",
-                   "one_cta_stream_k": "proj_sm100_kernel", "cuda_cores": "proj_simt_kernel"}[form]
-    algo_bytes = T * (2 * cfg.D * 2 + 4) + cfg.D * cfg.D * 2
+    # --- the headline workload: the whole layer, its dominant kernel, end to end, LayerNorm
+    head, out, ws, plan, _ = run_prefill(ne, cfg, tables_for(cfg, held), args, dev, flush, world, rank,
+                                         clock_gpu=local)
+    amplification = run_layernorm(ne, plan, out, ws, args, flush)
+    del out, ws
 
-    # --- end to end through the C ABI with host buffers: H2D inputs, fwd, D2H output
-    tok_pin = torch.from_numpy(tokens_h).pin_memory()
-    off_pin = torch.from_numpy(offsets_h).pin_memory()
-    out_pin = torch.empty((T, cfg.D), dtype=torch.bfloat16).pin_memory()
-    tok_d = torch.empty_like(tokens)
-    off_d = torch.empty_like(offsets)
-    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        ee[i][0].record(stream)
-        tok_d.copy_(tok_pin, non_blocking=True)
-        off_d.copy_(off_pin, non_blocking=True)
-        ne.ngram_embed_fwd(plan, tok_d, off_d, E0, E, W, out, ws, stream=stream)
-        out_pin.copy_(out, non_blocking=True)
-        ee[i][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in ee]))
-    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    # --- speculative decode: the headline layer's decode half first (its tables are held)
+    decode = None
+    if not args.no_decode:
+        decode = {}
+        for name in ("full_scale_decode", "spec_decode"):
+            dcfg = DECODE_WORKLOADS[name]
+            d = run_decode(ne, dcfg, tables_for(dcfg, held), args.decode_steps, max(args.warmup, 3), dev, rank=rank)
+            d["ms_per_step"] = max_over_ranks(d["ms_per_step"], world, dev)
+            d["value"] = world * d["tokens_per_step"] / (d["ms_per_step"] / 1e3)
+            decode[dcfg.name] = d
 
-    # --- embedding amplification by LayerNorm over the layer output (HBM-bound: the
-    # output read once from HBM, written once), in place, L2 flushed before each launch
-    ln_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        ln_ev[i][0].record(stream)
-        ne.ngram_embed_layernorm(plan, out, out, ws, eps=1e-5, stream=stream)
-        ln_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    ln_ms = float(np.mean([a.elapsed_time(b) for a, b in ln_ev]))
-    ln_bytes = 2 * out.numel() * out.element_size()
-    status = ne.ngram_embed_get_status(ws)
+    # --- the other prefill workloads, each with its own roofline (the varlen D = 4096 layer
+    # draws the same tables as the spec-decode layer above, so they are not filled again)
+    sub = {}
+    backward = None
+    if not args.no_sub:
+        for name in SUB_PREFILL:
+            scfg = WORKLOADS[name]
+            r, sout, sws, splan, (stok, sidx) = run_prefill(ne, scfg, tables_for(scfg, held), args, dev, flush,
+                                                            world, rank, e2e=False)
+            sub[scfg.name] = r
+            del sout, sws
+            if name == "prefill_d2048" and not args.no_backward:
+                backward = run_backward(ne, scfg, held[1], splan, stok, sidx, args, dev, flush)
+    held[0] = held[1] = None
+    torch.cuda.empty_cache()
 
     # --- hash statistics (section 3.2.2, Fig. 3b): collisions of the 2-gram hash for table
     # sizes swept over [30, 33] V0 (denser next to the multiples of V0), on 100 Zipf
     # sequences of 4096 tokens
     stats = None
     if not args.no_stats and rank == 0:
-        V0 = cfg.V0
-        s_tok = torch.from_numpy(gen.zipf_tokens(cfg.seed + 99, 100 * 4096, V0).astype(np.int32)).to(dev)
-        s_off = torch.from_numpy(gen.offsets_from_lengths([4096] * 100)).to(dev)
-        moduli = sorted({int(V0 * (30 + k * 0.05)) for k in range(61)} |
-                        {m * V0 + dd for m in (30, 31, 32, 33) for dd in (-3, -1, 1, 3)})
-        ne.ngram_hash_stats(V0, 2, s_tok, s_off, moduli[:2])  # warm-up
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        distinct, rows = ne.ngram_hash_stats(V0, 2, s_tok, s_off, moduli, stream=stream)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        st_ms = t0.elapsed_time(t1)
-        coll = np.array([distinct - r for r in rows])
-        near = np.array([min(abs(v - m * V0) for m in (30, 31, 32, 33)) <= 3 for v in moduli])
-        stats = {"ms": st_ms, "windows": int(s_tok.numel()), "moduli": len(moduli),
-                 "windows_per_s": s_tok.numel() * len(moduli) / (st_ms / 1e3), "distinct_2grams": distinct,
-                 "collisions_near_multiples_median": float(np.median(coll[near])),
-                 "collisions_elsewhere_median": float(np.median(coll[~near]))}
-
-    # --- backward (training): parameter gradients for a random bf16 dL/de, fp32 gradient
-    # tables accumulated in place; two tcgen05 GEMMs of 2 T D^2 FLOPs each dominate
-    backward = None
-    if not args.no_backward:
-        g_out = (torch.randn((T, cfg.D), device=dev) * 0.01).to(torch.bfloat16)
-        dE0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.float32, device=dev)
-        dE = [torch.zeros((v, cfg.d), dtype=torch.float32, device=dev) for v in cfg.V_nk]
-        dW = torch.zeros((cfg.D, cfg.D), dtype=torch.float32, device=dev)
-        bws = ne.new_bwd_workspace(plan, T, device=dev)
-        bwd = lambda: ne.ngram_embed_bwd(plan, tokens, idx, g_out, bws, E_nk=E, W_stacked=W, dE0=dE0, dE_nk=dE,
-                                         dW=dW, stream=stream)
-        for _ in range(2):
-            bwd()
-        torch.cuda.synchronize()
-        bw_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(max(3, args.steps // 4))]
-        for i, (e0, e1) in enumerate(bw_ev):
-            flush.fill_(i & 0xFF)
-            e0.record(stream)
-            bwd()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        bw_ms = float(np.mean([a.elapsed_time(b) for a, b in bw_ev]))
-        bw_flops = 4.0 * T * cfg.D * cfg.D
-        backward = {"ms": bw_ms, "tokens_per_s": T / (bw_ms / 1e3), "tflops": bw_flops / (bw_ms / 1e3) / 1e12,
-                    "frac": bw_flops / (bw_ms / 1e3) / 1e12 / pk["bf16_tflops"],
-                    "device_status": ne.ngram_embed_get_status(bws)}
-        del g_out, dE0, dE, dW, bws
-
-    del E0, E, W
-    torch.cuda.empty_cache()
-    decode = None
-    if not args.no_decode:
-        decode = run_decode(ne, DECODE_WORKLOADS[args.decode_workload], args.decode_steps, max(args.warmup, 3), dev,
-                            rank=rank)
-        if world > 1:
-            decode["ms_per_step"] = max_over_ranks(decode["ms_per_step"], world, dev)
-            decode["value"] = world * decode["tokens_per_step"] / (decode["ms_per_step"] / 1e3)
+        stats = run_hash_stats(ne, cfg, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -617,37 +707,86 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_block(cfg, argparse.Namespace(gpus=world)),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / pk["bf16_tflops"],
-                         "traffic": profiled_traffic(kernel_name, cfg.name),
-                         "kernel": kernel_name + " (" + form + "): fused sub-row gather + tcgen05 projection"
-                                   " + E_0 add + scale",
-                         "kernel_ms": proj_ms, "peak_source": pk["source"] + " (burst)",
-                         "layer_frac": (flops / (ms_per_step / 1e3) / 1e12) / pk["bf16_tflops"],
-                         "hash_kernel_ms": hash_ms,
-                         "algorithmic_bytes": algo_bytes},
+            "roofline": head["roofline"],
             "cpu_baseline": cpu,
-            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": tokens.numel() * 4 + offsets.numel() * 4,
-                    "d2h_bytes_per_step": out.numel() * 2},
+            "e2e": head["e2e"],
             "gpu_launches": 2 * args.steps,
+            "prefill_other_workloads": sub,
+            "decode": decode,
             "backward": backward,
             "hash_stats": stats,
-            "amplification": {"layernorm_ms": ln_ms, "bytes": ln_bytes, "gbs": ln_bytes / (ln_ms / 1e3) / 1e9,
-                              "frac_hbm": ln_bytes / (ln_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
-            "decode": decode,
-            "clocks": clk.summary(),
-            "device_status": status,
+            "amplification": amplification,
+            "clocks": head.get("clocks"),
+            "device_status": head["device_status"],
             "impl": "ours",
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_backward(ne, cfg, tables, plan, tokens, idx, args, dev, flush):
+    """Parameter gradients for a random bf16 dL/de, fp32 gradient tables accumulated in
+    place; two tcgen05 GEMMs of 2 T D^2 FLOPs each dominate."""
+    import torch
+    E0, E, W = tables
+    stream = torch.cuda.current_stream()
+    T = tokens.numel()
+    g_out = (torch.randn((T, cfg.D), device=dev) * 0.01).to(torch.bfloat16)
+    dE0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.float32, device=dev)
+    dE = [torch.zeros((v, cfg.d), dtype=torch.float32, device=dev) for v in cfg.V_nk]
+    dW = torch.zeros((cfg.D, cfg.D), dtype=torch.float32, device=dev)
+    bws = ne.new_bwd_workspace(plan, T, device=dev)
+    bwd = lambda: ne.ngram_embed_bwd(plan, tokens, idx, g_out, bws, E_nk=E, W_stacked=W, dE0=dE0, dE_nk=dE,
+                                     dW=dW, stream=stream)
+    for _ in range(2):
+        bwd()
+    torch.cuda.synchronize()
+    bw_ev = events(max(3, args.steps // 4))
+    for i, (e0, e1) in enumerate(bw_ev):
+        flush.fill_(i & 0xFF)
+        e0.record(stream)
+        bwd()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    bw_ms = float(np.mean([a.elapsed_time(b) for a, b in bw_ev]))
+    bw_flops = 4.0 * T * cfg.D * cfg.D
+    pk = peaks()
+    res = {"workload": cfg.name, "ms": bw_ms, "tokens_per_s": T / (bw_ms / 1e3),
+           "tflops": bw_flops / (bw_ms / 1e3) / 1e12, "frac": bw_flops / (bw_ms / 1e3) / 1e12 / pk["bf16_tflops"],
+           "device_status": ne.ngram_embed_get_status(bws)}
+    del g_out, dE0, dE, dW, bws
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_hash_stats(ne, cfg, dev):
+    import torch
+    stream = torch.cuda.current_stream()
+    V0 = cfg.V0
+    s_tok = torch.from_numpy(gen.zipf_tokens(cfg.seed + 99, 100 * 4096, V0).astype(np.int32)).to(dev)
+    s_off = torch.from_numpy(gen.offsets_from_lengths([4096] * 100)).to(dev)
+    moduli = sorted({int(V0 * (30 + k * 0.05)) for k in range(61)} |
+                    {m * V0 + dd for m in (30, 31, 32, 33) for dd in (-3, -1, 1, 3)})
+    ne.ngram_hash_stats(V0, 2, s_tok, s_off, moduli[:2])  # warm-up
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    distinct, rows = ne.ngram_hash_stats(V0, 2, s_tok, s_off, moduli, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    st_ms = t0.elapsed_time(t1)
+    coll = np.array([distinct - r for r in rows])
+    near = np.array([min(abs(v - m * V0) for m in (30, 31, 32, 33)) <= 3 for v in moduli])
+    return {"ms": st_ms, "windows": int(s_tok.numel()), "moduli": len(moduli),
+            "windows_per_s": s_tok.numel() * len(moduli) / (st_ms / 1e3), "distinct_2grams": distinct,
+            "collisions_near_multiples_median": float(np.median(coll[near])),
+            "collisions_elsewhere_median": float(np.median(coll[~near]))}
 
 
 if __name__ == "__main__":

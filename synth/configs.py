@@ -121,5 +121,15 @@ FULL_SCALE = NgramConfig(
     V_nk=tuple(mid_multiple_primes(V0_BIG, 55, 8)), dtype="bf16", num_seqs=8, seq_len=4096,
     decode_steps=1000, extras={"decode_seqs": 256})
 
+# The decode half of the full-scale workload: the same layer and tables, 256 sequences x 5
+# ids per step through a ring of the last N - 1 = 4 ids (capacity 16).
+FULL_SCALE_DECODE = FULL_SCALE.with_(name="full_scale_decode_bf16_D4096_N5_K2", num_seqs=256, seq_len=0)
+
 CONFIGS = [TINY, PREFILL_D2048, PREFILL_D4096_VARLEN, SPEC_DECODE, FULL_SCALE]
-BY_NAME = {c.name: c for c in CONFIGS}
+BY_NAME = {c.name: c for c in CONFIGS + [FULL_SCALE_DECODE]}
+
+
+def same_tables(a: NgramConfig, b: NgramConfig) -> bool:
+    """True when two workloads draw identical tables (same seed, shapes and value scales)."""
+    return (a.seed, a.V0, a.D, a.V_nk, a.dtype, a.e_std, a.d, a.S > 0) == \
+        (b.seed, b.V0, b.D, b.V_nk, b.dtype, b.e_std, b.d, b.S > 0)

@@ -31,8 +31,10 @@ def test_traffic_record_follows_the_code_not_the_comments(tmp_path, monkeypatch)
     monkeypatch.setattr(bench, "ROOT", str(root))
     (root / "profiles").mkdir()
     rec = {"kernel": "k", "workload": "w", "bytes_per_launch": 1234, "source_sha256": bench.kernel_source_hash()}
-    (root / "profiles" / "k_w.md").write_text("# k\n\ntraffic_record: " + json.dumps(rec) + "\n")
+    scaled = dict(rec, workload="w2", measured_on="w2_small", scale_to_workload=2.0)
+    (root / bench.TRAFFIC_RECORDS).write_text(json.dumps({"records": [rec, scaled]}))
     assert bench.profiled_traffic("k", "w") == 1234.0
+    assert bench.profiled_traffic("k", "w2") == 2468.0  # a smaller case's capture, scaled by units
     assert bench.profiled_traffic("k", "other") is None
     # a comment edit keeps the record
     name = bench.PROJECTION_SOURCES[-1]
@@ -55,8 +57,12 @@ def test_reference_arm_line_on_the_host():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["higher_is_better"] is True
     assert line["metric"].startswith("N-gram embed tokens/s")
-    assert line["config"]["workload"] == "prefill_bf16_D2048_N3_K2" and line["steps"] == 1
+    assert line["config"]["workload"] == "full_scale_bf16_D4096_N5_K2" and line["steps"] == 1
+    assert line["config"]["tokens_per_step"] == 32768 and line["config"]["tables_gb"] > 59
     assert line["value"] > 0 and line["n_gpus"] == 1 and line["vs_baseline"] is None
+    # each step is the timed sample: its own tokens and milliseconds, not an extrapolation
+    n = line["sample_tokens_per_step"]
+    assert 1 <= n <= 2048 and abs(line["value"] * line["ms_per_step"] / 1e3 - n) < 1e-6 * n
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and "sampled" in cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

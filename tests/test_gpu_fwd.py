@@ -340,20 +340,40 @@ def sample_rows(offsets, T, n=192, seed=0):
     return rows
 
 
+def tile_rows(offsets, T, tile=256, per=2, seed=0):
+    """Rows to check at full size: `per` random rows in every `tile`-token block (every pair
+    tile of the projection, the last partial one included), every sequence's first four and
+    last rows, and the last token."""
+    rng = np.random.default_rng(seed)
+    starts = np.arange(0, T, tile)
+    ends = np.minimum(starts + tile, T)
+    picks = [rng.integers(a, b, per) for a, b in zip(starts, ends)]
+    return np.unique(np.concatenate([sample_rows(offsets, T, n=0, seed=seed)] + picks))
+
+
 @pytest.mark.parametrize("cfg", [configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN, configs.FULL_SCALE],
                          ids=lambda c: c.name)
-def test_full_size_prefill_sampled(ne, cfg):
+def test_full_size_prefill(ne, cfg):
+    """The full-size prefill workloads in the launch configuration the bench times (default
+    plan, full workspace): every output row of the D = 2048 layer against the oracle, and at
+    least two rows of every 256-token tile (plus sequence edges) of the D = 4096 layers.
+    Then the other kernel forms at the same size on sampled rows."""
     tokens, offsets = workloads.prefill_tokens(cfg)
     T = len(tokens)
     E0, E, W = device_tables(cfg)
+    Wh = host_W(cfg)
     plan = plan_for(ne, cfg)
     assert ne.ngram_embed_plan_uses_tensor_cores(plan)
     out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
     assert status == 0
     assert not torch.isnan(out).any()
+    rows = np.arange(T) if cfg is configs.PREFILL_D2048 else tile_rows(offsets, T)
+    for a in range(0, len(rows), 8192):  # in slices: host memory for the fp64 rows stays bounded
+        r = rows[a:a + 8192]
+        want = oracle_rows(cfg, tokens, offsets, r, Wh)
+        assert_close(to_host_f64(out[torch.from_numpy(r).cuda()]), want, what=f"{cfg.name} rows {r[0]}..{r[-1]}")
     rows = sample_rows(offsets, T)
-    want = oracle_rows(cfg, tokens, offsets, rows, host_W(cfg))
-    assert_close(to_host_f64(out[torch.from_numpy(rows).cuda()]), want, what=cfg.name)
+    want = oracle_rows(cfg, tokens, offsets, rows, Wh)
     assert ne.ngram_embed_plan_kernel_form(plan, T).startswith("cta_pair")
     # the other pair tile width (256 or 512 columns) agrees with the oracle too
     wide = ne.ngram_embed_plan_kernel_form(plan, T) == "cta_pair_wide"

@@ -145,6 +145,27 @@ def test_forward_matches_library_matmul(D, N, K):
         assert np.abs(wrong - got).max() > 1e-3
 
 
+def test_gather_rows_by_hand():
+    """The row lookup E_s[idx[i, s]] -> [T, S, d]: tables whose every entry encodes its own
+    (table, row, column), so each looked-up value names where it came from. A transposed
+    stack axis, a swapped index column or a row/column mix-up fails here."""
+    S, d = 3, 4
+    V = [5, 7, 6]
+    tables = [np.array([[1000 * s + 10 * r + c for c in range(d)] for r in range(V[s])], dtype=np.int64)
+              for s in range(S)]
+    idx = np.array([[0, 6, 5], [4, 0, 2], [2, 3, 0]], dtype=np.int32)  # T = 3 tokens
+    got = oracle.gather_rows(tables, idx)
+    assert got.shape == (3, S, d)
+    for i in range(3):
+        for s in range(S):
+            assert got[i, s].tolist() == [1000 * s + 10 * int(idx[i, s]) + c for c in range(d)]
+    # token 1's block for sub-table 2 is row 2 of table 2, written out
+    assert got[1, 2].tolist() == [2020, 2021, 2022, 2023]
+    # concatenated along the feature axis it is G's layout: column s * d + c
+    G = got.reshape(3, S * d)
+    assert G[2, 1 * d + 3] == 1000 * 1 + 10 * 3 + 3
+
+
 def test_combine_bf16_exact_conversion():
     rng = np.random.default_rng(1)
     D, S = 8, 2
