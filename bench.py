@@ -481,12 +481,16 @@ def run_decode(ne, cfg, tables, steps: int, warmup: int, dev, rank: int = 0, ext
     del graphs
     pk = peaks()
     flops = 2.0 * T * cfg.D * cfg.D
+    form = ne.ngram_embed_plan_kernel_form(plan, T)
+    dense = form.startswith("cta_pair_dense") or form == "cta_pair_wide_dense"
     res = {
         "workload": cfg.name, "steps": steps, "tokens_per_step": T, "ms_per_step": ms / steps,
-        "value": steps * T / (ms / 1e3), "unit": UNIT, "graph": True, "gpu_launches_per_step": 2,
+        "value": steps * T / (ms / 1e3), "unit": UNIT, "graph": True,
+        # commit + hash, (the sub-row gather of the dense-A form,) the projection
+        "gpu_launches_per_step": 3 if dense else 2,
         "layer_tflops": flops / (ms / steps / 1e3) / 1e12,
         "layer_frac": flops / (ms / steps / 1e3) / 1e12 / pk["bf16_tflops"],
-        "kernel_form": ne.ngram_embed_plan_kernel_form(plan, T),
+        "kernel_form": form,
     }
     if not extras:
         res["device_status"] = status
@@ -530,12 +534,11 @@ def run_decode(ne, cfg, tables, steps: int, warmup: int, dev, rank: int = 0, ext
     proj_ms = timed(lambda i, st: ne.ngram_embed_project(plan, tok_all[i], idx_all[i], E0, E, W, out, ws, stream=st))
     hash_ms = timed(lambda i, st: ne.ngram_hash_indices(plan, tok_all[i], offsets, idx_all[n_k - 1 - i], ws,
                                                         cache=cache, stream=st))
-    R0 = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
-    # the step's table lookups alone: its 8 sub-rows and E_0 row per token (the layer's HBM
-    # reads besides W, 16 KiB per token) copied to G and E0_out (written back, 16 KiB)
-    gather_ms = timed(lambda i, st: ne.ngram_embed_gather(plan, idx_all[i], E, G, ws, tokens=tok_all[i], E0=E0,
-                                                          E0_out=R0, stream=st))
-    gather_bytes = T * (cfg.S * cfg.d + cfg.D) * 2 * 2  # rows read + rows written
+    # the step's table lookups as the dense-A form runs them: its 8 sub-rows per token (8 KiB)
+    # copied from the sub-tables into G (written back, 8 KiB); the E_0 rows are read by the
+    # projection's epilogue
+    gather_ms = timed(lambda i, st: ne.ngram_embed_gather(plan, idx_all[i], E, G, ws, stream=st))
+    gather_bytes = T * cfg.S * cfg.d * 2 * 2  # rows read + rows written
     # Draft-phase embedding cache: a verify call whose 5 in-step embeddings were all
     # computed while drafting (all hits), and the last draft call of a step (4 hits and the
     # new draft's miss per sequence), against the plain forward of the same 1280 tokens.
@@ -558,11 +561,14 @@ def run_decode(ne, cfg, tables, steps: int, warmup: int, dev, rank: int = 0, ext
     hit_rate = hits_d.item() / (T * (3 + 4 * n_k))  # timed(): 3 eager calls, then 1 + 3 replays of n_k
     res.update({
         "projection": {"ms": proj_ms, "tflops": flops / (proj_ms / 1e3) / 1e12,
-                       "frac": flops / (proj_ms / 1e3) / 1e12 / pk["bf16_tflops"]},
+                       "frac": flops / (proj_ms / 1e3) / 1e12 / pk["bf16_tflops"],
+                       "what": "ngram_embed_project: " + ("sub-row gather into G + dense-A tcgen05 projection"
+                                                          if dense else "fused row gather + tcgen05 projection")},
         "hash_ms": hash_ms,
-        "gather_stage_standalone": {
-            "what": "ngram_embed_gather alone (the step's sub-rows and E_0 rows copied out); not a kernel of the "
-                    "timed step, whose projection gathers its rows itself",
+        "gather_stage": {
+            "what": ("gather_kernel, as the step runs it: the sub-rows copied into G" if dense else
+                     "gather_kernel alone (the sub-rows copied into G); not a kernel of this step, whose "
+                     "projection gathers its rows itself"),
             "ms": gather_ms, "bytes": gather_bytes, "gbs": gather_bytes / (gather_ms / 1e3) / 1e9,
             "frac_hbm": gather_bytes / (gather_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
         "draft_cache": {"verify_all_hits_ms": verify_ms, "draft_step_4_of_5_hits_ms": draft_ms,

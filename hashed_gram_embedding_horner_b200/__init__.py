@@ -47,7 +47,7 @@ EXPORTED = [
     "ngram_embed_bwd_workspace_bytes", "ngram_embed_bwd",
     "ngram_hash_stats_workspace_bytes", "ngram_hash_stats",
     "ngram_draft_cache_reset", "ngram_embed_draft_workspace_bytes", "ngram_embed_fwd_draft",
-    "ngram_embed_fwd_step",
+    "ngram_embed_fwd_step", "ngram_embed_plan_set_dense_a",
 ]
 
 
@@ -89,6 +89,7 @@ _sig("ngram_embed_plan_set_tile_n", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pair_wide", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_dense_a", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_sm_count", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
@@ -321,7 +322,13 @@ def ngram_hash_stats(V0: int, n: int, tokens, seq_offsets, moduli, workspace=Non
 
 
 KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair", 4: "cta_pair_wide",
-                5: "cta_pair_stream_k"}
+                5: "cta_pair_stream_k", 6: "cta_pair_dense", 7: "cta_pair_dense_stream_k", 8: "cta_pair_wide_dense"}
+
+
+def ngram_embed_plan_set_dense_a(plan: "Plan", mode: int):
+    """Dense-A form (sub-rows gathered into G first, A by dense TMA): 0 automatic (small
+    calls), 1 whenever the workspace holds G, 2 never."""
+    _check(_lib.ngram_embed_plan_set_dense_a(plan.handle, int(mode)), "ngram_embed_plan_set_dense_a")
 
 
 def ngram_embed_plan_kernel_form(plan: Plan, num_tokens: int) -> str:

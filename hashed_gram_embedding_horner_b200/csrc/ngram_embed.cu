@@ -69,6 +69,9 @@ struct ngram_embed_plan {
   bool pdl = false;            // launch as programmatic dependent launches
   float out_scale = 1.0f;      // embedding amplification factor folded into the 1/(S+1) scale
   int pair_wide = -1;          // pair form with 512-column tiles: 1 on, 0 off, -1 automatic
+  int dense_a = 0;             // sub-rows gathered into G first, A by dense TMA: 0 automatic, 1 on, 2 off
+  const void* map_A = nullptr;  // the dense-A map's pointer and row count
+  int64_t map_A_T = -1;
   int max_clusters[3] = {0, 0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
 };
 
@@ -102,9 +105,26 @@ size_t ws_base(const ngram_embed_plan* p, int64_t T) {
 size_t sk_partial_bytes(const ngram_embed_plan* p) {
   return p->tc_ok ? size_t(2) * static_cast<size_t>(p->sms) * kBM * 256 * sizeof(float) : 0;
 }
+// The dense-A form: the call's sub-rows gathered into G [T x D] bf16 first (a stand-alone
+// gather kernel with every resident thread copying), then the CTA-pair projection reads A as
+// dense TMA boxes of G. Automatic for calls whose G is at most this many bytes: G then stays
+// in L2 between the two launches, and such calls (decode steps: 1280 tokens x 8 KiB = 10.5 MB
+// at D = 4096) are too small for the fused row gather to keep enough DRAM misses in flight.
+constexpr size_t kDenseAutoBytes = size_t(24) << 20;
+size_t dense_g_bytes(const ngram_embed_plan* p, int64_t T) {
+  return (static_cast<size_t>(T) * static_cast<size_t>(p->D) * 2 + 255) & ~size_t(255);
+}
+// Whether calls of T tokens may take the dense-A form at all (its kernel needs 256-column W
+// halves: tile width 256, D % 256 == 0).
+bool dense_capable(const ngram_embed_plan* p) { return p->tc_ok && p->bn == 256 && p->dense_a != 2; }
+bool dense_wanted(const ngram_embed_plan* p, int64_t T) {
+  return dense_capable(p) && (p->dense_a == 1 || dense_g_bytes(p, T) <= kDenseAutoBytes);
+}
+// Workspace: [head | T x S indices | stream-K partials | G (dense-A form)]
+size_t dense_g_offset(const ngram_embed_plan* p, int64_t ws_T) { return ws_base(p, ws_T) + sk_partial_bytes(p); }
 // Bytes that let every call of up to T tokens take its fastest schedule.
 size_t ws_bytes(const ngram_embed_plan* p, int64_t T) {
-  return ws_base(p, T) + sk_partial_bytes(p);
+  return ws_base(p, T) + sk_partial_bytes(p) + (dense_wanted(p, T) ? dense_g_bytes(p, T) : 0);
 }
 
 int check_launch() { return cudaGetLastError() == cudaSuccess ? NGRAM_OK : NGRAM_ERR_CUDA; }
@@ -192,7 +212,7 @@ bool use_stream_k(const ngram_embed_plan* p, const ProjParams& prm, int64_t T, s
   const int tiles = prm.num_m_blocks * prm.num_n_blocks;
   const int64_t units = static_cast<int64_t>(tiles) * prm.num_k_blocks;
   if (p->stream_k == 2 || p->sms <= 0 || tiles > kSkMaxTiles || units < p->sms) return false;
-  if (ws_size < ws_bytes(p, T)) return false;
+  if (ws_size < ws_base(p, T) + sk_partial_bytes(p)) return false;
   if (p->stream_k == 1) return true;
   const int waves = (tiles + p->sms - 1) / p->sms;
   return waves >= 2 && 1.3 * tiles < static_cast<double>(waves) * p->sms;
@@ -241,7 +261,7 @@ bool use_pair_stream_k(const ngram_embed_plan* p, int64_t T, size_t ws_size, int
   const int64_t tiles = (T + 2 * kBM - 1) / (2 * kBM) * (p->D / p->bn);
   const int64_t units = tiles * (p->D / kBK);
   if (tiles > kSkMaxTiles / 2 || units < pairs) return false;
-  return ws_size >= ws_bytes(p, ws_T);
+  return ws_size >= ws_base(p, ws_T) + sk_partial_bytes(p);
 }
 
 // CTA-pair kernel: clusters of two CTAs, one 256 x BN tile per pair per step.
@@ -467,8 +487,98 @@ int launch_simt(const ngram_embed_plan* p, const int32_t* tokens, const int32_t*
   return launch(proj_simt_kernel<T>, dim3(static_cast<unsigned>(blocks)), dim3(256), smem, st, p->pdl, 1, s);
 }
 
-// ws_T: the token count the workspace was validated for (its index buffer's length);
-// the stream-K partials, if the workspace holds them, follow that buffer.
+// The projection kernel a call runs (ngram_embed_plan_kernel_form reports the same codes).
+enum Form : int {
+  kFormSimt = 0,       // CUDA cores
+  kFormOne = 1,        // one CTA per 128 x BN tile, fused row gather
+  kFormOneSk = 2,      // one CTA per SM, stream-K, fused row gather
+  kFormPair = 3,       // CTA pairs, 256 x BN tiles, fused row gather
+  kFormPairWide = 4,   // CTA pairs, 256 x 512 tiles, fused row gather
+  kFormPairSk = 5,     // CTA pairs, stream-K, fused row gather (opt-in)
+  kFormDense = 6,      // rows gathered into G first; CTA pairs, 256 x 256 tiles, A by dense TMA
+  kFormDenseSk = 7,    // the same with the pairs' stream-K schedule
+  kFormDenseWide = 8,  // the same with 256 x 512 tiles
+};
+
+// Stream-K for the dense-A pair form: automatic where a grid of whole 256 x 256 tiles would
+// take two or more waves of pairs and leave many pairs idle in the last (a decode step of
+// 1280 tokens at D = 4096: 80 tiles on 74 pairs), as for the one-CTA form.
+bool dense_stream_k(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws_T) {
+  if (p->stream_k == 2 || p->sms < 2 || p->pair_wide == 1) return false;
+  const int64_t pairs = p->sms / 2;
+  const int64_t tiles = (T + 2 * kBM - 1) / (2 * kBM) * (p->D / 256);
+  const int64_t units = tiles * (p->D / kBK);
+  if (tiles > kSkMaxTiles / 2 || units < pairs) return false;
+  if (ws_size < ws_base(p, ws_T) + sk_partial_bytes(p)) return false;
+  if (p->stream_k == 1) return true;
+  const int64_t waves = (tiles + pairs - 1) / pairs;
+  return waves >= 2 && 1.3 * static_cast<double>(tiles) < static_cast<double>(waves * pairs);
+}
+
+// ws_T: the token count the workspace was validated for (its index buffer's length); the
+// stream-K partials and the dense-A G buffer, if the workspace holds them, follow that buffer.
+// count_on_device: the token count is known only on the device (a draft call's misses).
+int choose_form(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws_T, bool count_on_device) {
+  if (p->variant == kSimt) return kFormSimt;
+  if (!count_on_device && p->cta_pair != 0 && dense_wanted(p, T) &&
+      ws_size >= dense_g_offset(p, ws_T) + dense_g_bytes(p, T)) {
+    if (dense_stream_k(p, T, ws_size, ws_T)) return kFormDenseSk;
+    return use_pair_wide(p, T) ? kFormDenseWide : kFormDense;
+  }
+  // Not stream-K when the count is known only on the device: for the few tiles of a draft
+  // call's misses its fix-ups cost more than they balance (measured: 256 misses at D = 4096,
+  // 79 us stream-K vs 64 us CTA pairs). Otherwise the one-CTA form's stream-K where its grid
+  // ends in a thin wave, else the pair form (512-column tiles where they fill their waves).
+  ProjParams prm{};
+  prm.num_m_blocks = static_cast<int>((T + kBM - 1) / kBM);
+  prm.num_n_blocks = p->D / p->bn;
+  prm.num_k_blocks = p->D / kBK;
+  const bool psk = !count_on_device && p->cta_pair != 0 && p->pair_wide != 1 && use_pair_stream_k(p, T, ws_size, ws_T);
+  const bool sk = !psk && !count_on_device && p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
+  const bool pair = p->cta_pair == 1 || (p->cta_pair == -1 && !sk);
+  if (pair) return psk ? kFormPairSk : (use_pair_wide(p, T, count_on_device) ? kFormPairWide : kFormPair);
+  return sk ? kFormOneSk : kFormOne;
+}
+
+// The stand-alone gather kernel: G[i][s*d + c] = E_s[idx[i][s]][c] and, if E0_out is given,
+// E0_out[i] = E_0[tokens[i]]. Arguments already checked.
+int launch_gather(const ngram_embed_plan* p, const int32_t* idx, int64_t T, const void* const* E_nk, void* G,
+                  const int32_t* tokens, const void* E0, void* E0_out, void* ws, cudaStream_t st) {
+  GatherParams g{};
+  for (int s = 0; s < p->S; ++s) {
+    g.E[s] = static_cast<const uint8_t*>(E_nk[s]);
+    g.Vs[s] = static_cast<uint32_t>(p->V[s]);
+  }
+  g.idx = idx;
+  g.G = static_cast<uint8_t*>(G);
+  g.T = T;
+  g.S = p->S;
+  g.row_bytes = p->d * p->elt;
+  g.tokens = tokens;
+  g.E0 = static_cast<const uint8_t*>(E0);
+  g.E0_out = static_cast<uint8_t*>(E0_out);
+  g.V0 = static_cast<uint32_t>(p->V0);
+  g.e0_row_bytes = p->D * p->elt;
+  g.status = status_ptr(ws);
+  // every resident thread (8 blocks of 256 per SM, spread evenly over the SMs) takes an
+  // equal share of the 16-byte vectors; fewer blocks only when there are fewer vectors
+  const int64_t vecs = T * p->S * (g.row_bytes / 16) + (E0_out ? T * (g.e0_row_bytes / 16) : 0);
+  // the kernel numbers vectors (and its grid-stride steps) in 32 bits
+  if (vecs + static_cast<int64_t>(p->sms > 0 ? p->sms : 1) * 8 * 256 * kGatherUnroll > UINT32_MAX)
+    return NGRAM_ERR_UNSUPPORTED;
+  auto log2_or_neg = [](int v) {
+    int sh = 0;
+    while ((1 << sh) < v) ++sh;
+    return (1 << sh) == v ? sh : -1;
+  };
+  g.vshift = log2_or_neg(g.row_bytes / 16);
+  g.eshift = log2_or_neg(g.e0_row_bytes / 16);
+  int64_t blocks = (vecs + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(p->sms > 0 ? p->sms : 1) * 8;
+  if (blocks > cap) blocks = cap;
+  return launch(gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, p->pdl, 1, g);
+}
+
 // T_dev (optional): the kernels take min(*T_dev, T) tokens, a count known only on the device.
 int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int64_t T, const void* E0,
             const void* const* E_nk, const void* W, void* out, void* ws, size_t ws_size, int64_t ws_T,
@@ -500,35 +610,50 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   prm.scale = p->out_scale / static_cast<float>(p->S + 1);
   prm.status = status_ptr(ws);
   prm.T_dev = T_dev;
-  // Not stream-K when the count is known only on the device: for the few tiles of a draft
-  // call's misses its fix-ups cost more than they balance (measured: 256 misses at D = 4096,
-  // 79 us stream-K vs 64 us CTA pairs).
-  // the one-CTA form's stream-K where its grid ends in a thin wave, else the pair form
-  // (512-column tiles where they fill their waves)
-  const bool psk = !T_dev && p->cta_pair != 0 && p->pair_wide != 1 && use_pair_stream_k(p, T, ws_size, ws_T);
-  const bool sk = !psk && !T_dev && p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
-  const bool pair = p->cta_pair == 1 || (p->cta_pair == -1 && !sk);
+  auto* wsb = static_cast<uint8_t*>(ws);
+  auto stream_k_buffers = [&] {
+    prm.stream_k = 1;
+    prm.sk_counters = reinterpret_cast<int*>(wsb + kStatusBytes);
+    prm.sk_partials = reinterpret_cast<float*>(wsb + ws_base(p, ws_T));
+  };
+  const int form = choose_form(p, T, ws_size, ws_T, T_dev != nullptr);
+  if (form == kFormDense || form == kFormDenseSk || form == kFormDenseWide) {
+    // the call's sub-rows into G (workspace), then A tiles as dense TMA boxes of G
+    void* G = wsb + dense_g_offset(p, ws_T);
+    if ((rc = launch_gather(p, idx, T, E_nk, G, nullptr, nullptr, nullptr, ws, st))) return rc;
+    if (p->map_A != G || p->map_A_T != T) {
+      p->map_A = nullptr;
+      if ((rc = encode_2d(&p->maps.A, G, p->D, static_cast<uint64_t>(T), static_cast<uint64_t>(p->D) * 2, kBK, kBM,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B)))
+        return rc;
+      p->map_A = G;
+      p->map_A_T = T;
+    }
+    prm.dense_a = 1;
+    prm.tma_rows = 0;
+    if (form == kFormDenseWide) {
+      prm.num_n_blocks = p->D / 512;
+      return launch_tc_pair_stages<512, kPairStagesWide>(p, prm, T, st, 8);
+    }
+    if (form == kFormDenseSk) stream_k_buffers();
+    return launch_tc_pair<256>(p, prm, T, st);
+  }
+  const bool pair = form == kFormPair || form == kFormPairWide || form == kFormPairSk;
   // A rows by TMA gather4 in the pair form, by cp.async in the one-CTA form (measured
   // fastest for each), unless the plan fixes the split.
   prm.tma_rows = p->variant == kTcTmaRows ? kBM : (p->tma_rows >= 0 ? p->tma_rows : (pair ? kBM : 0));
-  if (pair && !psk && use_pair_wide(p, T, T_dev != nullptr)) {
+  if (form == kFormPairWide) {
     prm.num_n_blocks = p->D / 512;
     prm.tma_rows = kBM;  // A rows by gather4 only
     return launch_tc_pair_stages<512, kPairStagesWide>(p, prm, T, st, 8);
   }
-  if (pair && psk) {
-    prm.stream_k = 1;
+  if (form == kFormPairSk) {
+    stream_k_buffers();
     prm.tma_rows = kBM;  // A rows by gather4 only
-    prm.sk_counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kStatusBytes);
-    prm.sk_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_base(p, ws_T));
     return launch_tc_pair<256>(p, prm, T, st);
   }
   if (pair) return p->bn == 256 ? launch_tc_pair<256>(p, prm, T, st) : launch_tc_pair<128>(p, prm, T, st);
-  if (sk) {
-    prm.stream_k = 1;
-    prm.sk_counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kStatusBytes);
-    prm.sk_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_base(p, ws_T));
-  }
+  if (form == kFormOneSk) stream_k_buffers();
   return p->bn == 256 ? launch_tc<256>(p, prm, st) : launch_tc<128>(p, prm, st);
 }
 
@@ -648,16 +773,13 @@ int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on) {
 
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens) {
   if (!plan || num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
-  if (plan->variant == kSimt) return 0;
-  ProjParams prm{};
-  prm.num_m_blocks = static_cast<int>((num_tokens + kBM - 1) / kBM);
-  prm.num_n_blocks = plan->D / plan->bn;
-  prm.num_k_blocks = plan->D / kBK;
-  const size_t ws = ws_bytes(plan, num_tokens);
-  const bool psk = plan->cta_pair != 0 && plan->pair_wide != 1 && use_pair_stream_k(plan, num_tokens, ws, num_tokens);
-  const bool sk = !psk && plan->cta_pair != 1 && use_stream_k(plan, prm, num_tokens, ws);
-  if (plan->cta_pair == 1 || (plan->cta_pair == -1 && !sk)) return psk ? 5 : (use_pair_wide(plan, num_tokens) ? 4 : 3);
-  return sk ? 2 : 1;
+  return choose_form(plan, num_tokens, ws_bytes(plan, num_tokens), num_tokens, false);
+}
+
+int ngram_embed_plan_set_dense_a(ngram_embed_plan* plan, int mode) {
+  if (!plan || mode < 0 || mode > 2) return NGRAM_ERR_INVALID_ARG;
+  plan->dense_a = mode;
+  return NGRAM_OK;
 }
 
 int ngram_embed_plan_set_sm_count(ngram_embed_plan* plan, int sms) {
@@ -1199,43 +1321,13 @@ int ngram_embed_gather(const ngram_embed_plan* plan, const int32_t* idx, int64_t
   if (E0_out && (!tokens || !E0)) return NGRAM_ERR_INVALID_ARG;
   if ((G_out && !aligned16(G_out)) || (E0_out && (!aligned16(E0_out) || !aligned16(E0))))
     return NGRAM_ERR_MISALIGNED;
-  GatherParams g{};
   for (int s = 0; s < plan->S; ++s) {
     if (!E_nk[s]) return NGRAM_ERR_INVALID_ARG;
     if (!aligned16(E_nk[s])) return NGRAM_ERR_MISALIGNED;
-    g.E[s] = static_cast<const uint8_t*>(E_nk[s]);
-    g.Vs[s] = static_cast<uint32_t>(plan->V[s]);
   }
   if ((rc = set_device(plan))) return rc;
-  g.idx = idx;
-  g.G = static_cast<uint8_t*>(G_out);
-  g.T = num_tokens;
-  g.S = plan->S;
-  g.row_bytes = plan->d * plan->elt;
-  g.tokens = tokens;
-  g.E0 = static_cast<const uint8_t*>(E0);
-  g.E0_out = static_cast<uint8_t*>(E0_out);
-  g.V0 = static_cast<uint32_t>(plan->V0);
-  g.e0_row_bytes = plan->D * plan->elt;
-  g.status = status_ptr(workspace);
-  // every resident thread (8 blocks of 256 per SM, spread evenly over the SMs) takes an
-  // equal share of the 16-byte vectors; fewer blocks only when there are fewer vectors
-  const int64_t vecs = num_tokens * plan->S * (g.row_bytes / 16) + (E0_out ? num_tokens * (g.e0_row_bytes / 16) : 0);
-  // the kernel numbers vectors (and its grid-stride steps) in 32 bits
-  if (vecs + static_cast<int64_t>(plan->sms > 0 ? plan->sms : 1) * 8 * 256 * kGatherUnroll > UINT32_MAX)
-    return NGRAM_ERR_UNSUPPORTED;
-  auto log2_or_neg = [](int v) {
-    int sh = 0;
-    while ((1 << sh) < v) ++sh;
-    return (1 << sh) == v ? sh : -1;
-  };
-  g.vshift = log2_or_neg(g.row_bytes / 16);
-  g.eshift = log2_or_neg(g.e0_row_bytes / 16);
-  int64_t blocks = (vecs + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(plan->sms > 0 ? plan->sms : 1) * 8;
-  if (blocks > cap) blocks = cap;
-  return launch(gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
-                static_cast<cudaStream_t>(stream), plan->pdl, 1, g);
+  return launch_gather(plan, idx, num_tokens, E_nk, G_out, tokens, E0, E0_out, workspace,
+                       static_cast<cudaStream_t>(stream));
 }
 
 static int cache_launch(const ngram_embed_plan* plan, const ngram_cache* cache, const int32_t* slots,

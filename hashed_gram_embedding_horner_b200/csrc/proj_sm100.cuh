@@ -72,6 +72,9 @@ struct ProjParams {
   // if set, the token count is min(*T_dev, T), read by the kernel (a count produced on the
   // device, e.g. the cache misses of a draft-phase call); num_m_blocks then covers T
   const int32_t* T_dev;
+  // CTA-pair kernel: 1 = A tiles are dense 2-D TMA boxes of an already gathered G [T x D]
+  // (maps.A), not rows gathered from the sub-tables
+  int dense_a;
 };
 
 struct ProjMaps {
@@ -79,6 +82,7 @@ struct ProjMaps {
   CUtensorMap Whalf;        // W_stacked, box {64, BN/2} (CTA-pair kernel: each CTA loads half)
   CUtensorMap E[kMaxS];     // sub-table s, box {64, 1}, 128-byte swizzle (gather4)
   CUtensorMap Out;          // out [T x D], box {64, 32}, 128-byte swizzle (epilogue TMA stores)
+  CUtensorMap A;            // gathered G [T x D], box {64, 128}, 128-byte swizzle (dense-A pair form)
 };
 
 // Shared memory (224 KB): A stages of 16 KB, W stages of BN x 128 B and the epilogue's

@@ -19,6 +19,10 @@
 //     of CTA 1 (one lane per stage, so the slow cluster-scope release of one stage overlaps
 //     the others) waits for it, fences generic->async proxy and arrives remotely on CTA 0's
 //     stage barrier;
+//   - with dense_a (a call whose sub-rows were gathered into G beforehand, small enough for
+//     G to stay in L2), each CTA's W producer thread also brings in its 128 A rows as one
+//     2-D TMA box of G per stage (.cta_group::2 form, byte count on CTA 0's barrier), and
+//     CTA 0's W producer posts the pair's byte count; the A producer warps stay idle;
 //   - CTA 0's MMA thread commits stage release and "accumulator ready" to the barriers of
 //     both CTAs (two tcgen05.commit, one per CTA address);
 //   - CTA 1's epilogue warps arrive remotely on CTA 0's "accumulator free" barrier.
@@ -224,7 +228,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   constexpr int kMmaN = L::kMmaN;
   // stream-K (256-column tiles only): the (tile, k-block) units split evenly over the pairs
   const bool sk = !kWide && p.stream_k != 0;
-  const bool cp_rows = !kWide && !sk && p.tma_rows == 0;  // A rows by cp.async (else all by TMA gather4)
+  const bool dense = p.dense_a != 0;                                // A by 2-D TMA boxes of G
+  const bool cp_rows = !kWide && !sk && !dense && p.tma_rows == 0;  // A rows by cp.async (else all by TMA gather4)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       // CTA 0: thread 0 posts the pair's TMA bytes (+ its 256 cp.async threads + CTA 1's relay);
@@ -244,7 +249,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == kWarpB && lane == 0) tma_prefetch_desc(&maps.Whalf);
+  if (warp == kWarpB && lane == 0) {
+    tma_prefetch_desc(&maps.Whalf);
+    if (p.dense_a) tma_prefetch_desc(&maps.A);
+  }
   if (warp == kWarpMma) {
     tmem_alloc_pair(smem_u32(tmem_slot), L::kTmemCols);
     tmem_relinquish_pair();
@@ -272,7 +280,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   wp.u_end = sk ? sk_first_unit(units_total, wp.grid, pair + 1) : 0;
 
   const bool epi_warp = warp >= kWarpEpi0 || (kWide && warp >= kAWarps / 2 && warp < kAWarps);
-  if (warp < kAWarps && !epi_warp) {
+  if (warp < kAWarps && !epi_warp && !dense) {
     // ------------------------------------------------------------ A producers (own 128 rows)
     const int t = threadIdx.x;
     const int chunk = t & 7, rsub = t >> 3;                         // cp.async mode
@@ -343,13 +351,21 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      const uint64_t pol_a = l2_policy_evict_normal();
       for (Seg g = seg_first(wp, pair); g.tile < num_tiles && ok; g = seg_next(wp, g)) {
         const int n_blk = g.tile % p.num_n_blocks;
-        const int rot = k_rotation(g.tile / p.num_n_blocks, n_blk, KB);
+        const int m_blk = g.tile / p.num_n_blocks;
+        const int rot = k_rotation(m_blk, n_blk, KB);
         for (int i = g.i0; i < g.i1; ++i) {
           int kb = i + rot;
           if (kb >= KB) kb -= KB;
           if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          if (dense) {
+            // this CTA's 128 rows of the k-block as one box of G (rows past T read zeros)
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2u * (L::kABytes + L::kBBytes));
+            tma_load_2d_pair(a_tile(stage), &maps.A, kb * kBK, m_blk * (2 * kBM) + static_cast<int>(rank) * kBM,
+                             map_to_cta(full_bar(stage), 0), pol_a);
+          }
 #pragma unroll
           for (int h = 0; h < L::kHalves; ++h)
             tma_load_2d_pair(b_tile(stage) + h * L::kBSubBytes, &maps.Whalf, kb * kBK,

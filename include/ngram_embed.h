@@ -110,11 +110,13 @@ int ngram_embed_plan_destroy(ngram_embed_plan* plan);
 /* Device workspace bytes for calls of up to max_tokens tokens: a 33,024-byte head (the
  * status word, then the stream-K arrival counters), the [max_tokens x S] int32 index
  * buffer, then, for plans that use the tensor-core kernel, 2 x (SM count) x 128 x 256 fp32
- * stream-K partial tiles (the plan's SM count: see ngram_embed_plan_set_sm_count). A workspace without the partials (head + index buffer, rounded
- * up to 256 bytes) is accepted too; the projection then never uses the stream-K schedule.
- * The head must be zeroed once before first use (ngram_embed_clear_status does it); the
- * rest needs no init. The kernels leave the counters zero after every call that did not
- * set NGRAM_STATUS_TIMEOUT. */
+ * stream-K partial tiles (the plan's SM count: see ngram_embed_plan_set_sm_count), then,
+ * for calls that the dense-A form would take (ngram_embed_plan_set_dense_a), the
+ * [max_tokens x D] bf16 G buffer, each region rounded up to 256 bytes. A workspace without
+ * the partials or G (head + index buffer) is accepted too; the projection then takes the
+ * forms that fit. The head must be zeroed once before first use (ngram_embed_clear_status
+ * does it); the rest needs no init. The kernels leave the counters zero after every call
+ * that did not set NGRAM_STATUS_TIMEOUT. */
 size_t ngram_embed_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens);
 
 /* The whole layer (section 2, Eq. 2 + Eq. 3) for num_tokens tokens in num_seqs sequences.
@@ -371,8 +373,26 @@ int ngram_embed_plan_set_pair_wide(ngram_embed_plan* plan, int on);
 /* The projection kernel a call of num_tokens tokens would run, given a workspace of
  * ngram_embed_workspace_bytes(plan, num_tokens): 0 = CUDA cores, 1 = one CTA per tile,
  * 2 = one CTA per SM with the stream-K schedule, 3 = CTA pairs, 4 = CTA pairs with
- * 512-column tiles, 5 = CTA pairs with the stream-K schedule; negative on bad arguments. */
+ * 512-column tiles, 5 = CTA pairs with the stream-K schedule (these gather the A rows from
+ * the sub-tables inside the projection); 6 = the call's sub-rows gathered into G first by a
+ * stand-alone gather kernel, then CTA pairs reading A as dense TMA boxes of G, 7 = the same
+ * with the pairs' stream-K schedule, 8 = the same with 512-column tiles (see
+ * ngram_embed_plan_set_dense_a); negative on bad arguments. */
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens);
+
+/* Dense-A form of the tensor-core projection: the call's sub-rows are first copied into a
+ * G buffer [num_tokens x D] (bf16) in the workspace by a gather kernel that keeps every
+ * resident thread's loads in flight, then the CTA-pair kernel reads its A tiles as dense
+ * 2-D TMA boxes of G (from L2, where G stays between the two launches) instead of gathering
+ * rows itself. 0 (default) = automatic: calls whose G takes at most 24 MiB (up to 3072
+ * tokens at D = 4096: decode steps, whose fused row gather leaves the tensor cores waiting on
+ * DRAM misses), when the workspace holds G and the plan allows the pair form with 256-column
+ * tiles; 1 = whenever the workspace holds G; 2 = never. ngram_embed_workspace_bytes includes G
+ * for the calls this setting selects. The stream-K schedule applies to it automatically
+ * where whole tiles would leave a thin last wave of pairs. A tuning knob: results agree
+ * within the stated tolerance (the k-block order differs). NGRAM_ERR_INVALID_ARG for other
+ * values. */
+int ngram_embed_plan_set_dense_a(ngram_embed_plan* plan, int mode);
 
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */
 int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);

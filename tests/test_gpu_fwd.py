@@ -454,29 +454,36 @@ def test_reduced_sm_count_every_form(ne, sms):
     E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
     want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
     forms = set()
-    for pair, wide, sk in ((None, None, 0), (1, 1, 0), (1, 0, 1), (1, 0, 2), (0, 0, 1), (0, 0, 2)):
+    for pair, wide, sk, dense in ((None, None, 0, 2), (1, 1, 0, 2), (1, 0, 1, 2), (1, 0, 2, 2), (0, 0, 1, 2),
+                                  (0, 0, 2, 2), (None, 0, 1, 1), (None, 0, 2, 1), (None, 1, 2, 1)):
         plan = plan_for(ne, cfg, pair=pair)
         ne.ngram_embed_plan_set_sm_count(plan, sms)
         ne.ngram_embed_plan_set_pair_wide(plan, wide)
         ne.ngram_embed_plan_set_stream_k(plan, sk)
+        ne.ngram_embed_plan_set_dense_a(plan, dense)
         forms.add(ne.ngram_embed_plan_kernel_form(plan, len(tokens)))
         out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
         assert status == 0
-        assert_close(to_host_f64(out), want, what=f"{sms} SMs, pair={pair} wide={wide} stream-K={sk}")
-    assert {"cta_pair_wide", "cta_pair_stream_k", "cta_pair", "one_cta_stream_k", "one_cta"} <= forms
+        assert_close(to_host_f64(out), want, what=f"{sms} SMs, pair={pair} wide={wide} stream-K={sk} dense={dense}")
+    assert {"cta_pair_wide", "cta_pair_stream_k", "cta_pair", "one_cta_stream_k", "one_cta", "cta_pair_dense",
+            "cta_pair_dense_stream_k", "cta_pair_wide_dense"} <= forms
 
 
 def test_automatic_kernel_form(ne):
     """Prefill grids run the CTA-pair form with 512-column tiles; a 1280-token decode step at
-    D = 4096 (160 tiles of 128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule;
-    a grid of one wave keeps the 256-column pair tiles (more SMs busy). The pairs' stream-K
-    schedule is taken only when both the pair form and stream-K are asked for."""
+    D = 4096 (10.5 MB of gathered sub-rows) runs the dense-A pair form with the pairs'
+    stream-K schedule (80 tiles of 256 x 256 on 74 pairs); a grid of one wave keeps the
+    256-column tiles (more SMs busy). Without the dense-A form, the decode step runs the
+    one-CTA stream-K schedule."""
     for cfg in (configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN):
         plan = plan_for(ne, cfg)
         assert ne.ngram_embed_plan_kernel_form(plan, 32768) == "cta_pair_wide"
     plan = plan_for(ne, configs.SPEC_DECODE)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_dense_stream_k"
+    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair_dense"  # one wave: nothing to balance
+    ne.ngram_embed_plan_set_dense_a(plan, 2)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "one_cta_stream_k"
-    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"  # one wave: nothing to balance
+    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"
     ne.ngram_embed_plan_set_cta_pair(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_wide"
     ne.ngram_embed_plan_set_stream_k(plan, 1)
@@ -484,6 +491,70 @@ def test_automatic_kernel_form(ne):
     ne.ngram_embed_plan_set_cta_pair(plan, None)
     ne.ngram_embed_plan_set_stream_k(plan, 0)
     assert ne.ngram_embed_plan_kernel_form(plan_for(ne, configs.TINY), 128) == "cuda_cores"
+
+
+@pytest.mark.parametrize("shape,lengths", [
+    ((5000, 512, 5, 2), RAGGED),                     # one m-block pair, ragged tail
+    ((4000, 1024, 3, 4), [1, 0, 1100, 3, 77]),        # several tiles, sequences of 1 and 3
+    ((3000, 2048, 3, 2), [640, 640]),                # T = 1280: decode-sized, 2 waves of pairs
+], ids=["D512N5K2", "D1024N3K4", "D2048N3K2_T1280"])
+@pytest.mark.parametrize("knobs,form", [
+    ({"stream_k": 2, "pair_wide": 0}, "cta_pair_dense"),
+    ({"stream_k": 1}, "cta_pair_dense_stream_k"),
+    ({"stream_k": 2, "pair_wide": 1}, "cta_pair_wide_dense"),
+], ids=["dense", "dense_stream_k", "dense_wide"])
+def test_dense_a_forms_match_oracle(ne, shape, lengths, knobs, form):
+    """The dense-A form (sub-rows gathered into G in the workspace, A by 2-D TMA boxes of G)
+    in each of its schedules against the oracle on every row; repeatable bits; and the same
+    products as the fused pair form within the tolerance."""
+    cfg = small_cfg(*shape)
+    tokens, offsets = ragged_tokens(cfg, lengths)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = plan_for(ne, cfg)
+    ne.ngram_embed_plan_set_dense_a(plan, 1)
+    ne.ngram_embed_plan_set_stream_k(plan, knobs["stream_k"])
+    if "pair_wide" in knobs:
+        ne.ngram_embed_plan_set_pair_wide(plan, knobs["pair_wide"])
+    assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == form
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    assert_close(to_host_f64(out), want, what=f"{cfg.name} {form}")
+    again, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0 and torch.equal(out, again)
+    ne.ngram_embed_plan_set_dense_a(plan, 2)
+    fused, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    assert (out.float() - fused.float()).abs().max().item() <= 2e-2
+
+
+@pytest.mark.parametrize("stream_k", [1, 2])
+def test_dense_a_gather_and_layout_bit_exact(ne, stream_k):
+    """W = I and E_0 = 0 through the dense-A form: out = concat_s E_s[idx_s] / (S + 1)
+    exactly, so every sub-row the gather kernel copied into G must reach its place in the
+    output bit for bit (stream-K pieces add zeros exactly)."""
+    cfg = small_cfg(7000, 768, 2, 3, seed=5)  # S + 1 = 4: the scale is exact
+    tokens, offsets = ragged_tokens(cfg, [5, 1300, 900, 3])  # 27 tiles of 256 x 256
+    from tests.helpers import host_tables
+    _, Eh, _ = host_tables(cfg)
+    E0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.bfloat16, device="cuda")
+    E = [to_device(e, torch.bfloat16) for e in Eh]
+    W = torch.eye(cfg.D, dtype=torch.bfloat16, device="cuda")
+    plan = plan_for(ne, cfg)
+    ne.ngram_embed_plan_set_dense_a(plan, 1)
+    ne.ngram_embed_plan_set_stream_k(plan, stream_k)
+    ne.ngram_embed_plan_set_pair_wide(plan, 0)
+    assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == \
+        ("cta_pair_dense_stream_k" if stream_k == 1 else "cta_pair_dense")
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, oracle.context_windows(cfg.N, tokens, offsets))
+    G = oracle.gather_rows(Eh, idx).reshape(len(tokens), cfg.D)
+    want = gen.f32_to_bf16_bits(gen.bf16_bits_to_f32(G) / np.float32(cfg.S + 1))
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, want)
 
 
 def test_spec_decode_forward_through_ring(ne):

@@ -74,22 +74,25 @@ def _noalloc_cfg():
                                V_nk=tuple(configs.primes_from(20000, 8)), dtype="bf16", seed=5)
 
 
-def test_static_workspace_stream_k_matches_fwd(ne):
+@pytest.mark.parametrize("dense_a,form", [(2, "one_cta_stream_k"), (1, "cta_pair_dense_stream_k")])
+def test_static_workspace_stream_k_matches_fwd(ne, dense_a, form):
     """With 8 SMs the stream-K partial tiles (2 x 8 x 128 KB) fit the fixed array, so the
-    schedule whose arrival counters and partials live in it runs; two calls in a row equal
-    ngram_embed_fwd with its own workspace (same schedule) bit for bit."""
+    schedules whose arrival counters and partials (and, in the dense-A form, the gathered
+    sub-rows) live in it run; two calls in a row equal ngram_embed_fwd with its own workspace
+    (same schedule) bit for bit."""
     cfg = _noalloc_cfg()
     E0h, Eh, Wh = host_tables(cfg)
     E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
     plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
     ne.ngram_embed_plan_set_sm_count(plan, 8)
     ne.ngram_embed_plan_set_stream_k(plan, 1)
+    ne.ngram_embed_plan_set_dense_a(plan, dense_a)
     status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     for call, lengths in enumerate(([3, 330, 97], [129, 1, 0, 300])):
         off_h = gen.offsets_from_lengths(lengths)
         T = int(off_h[-1])
-        assert ne.ngram_embed_plan_kernel_form(plan, T) == "one_cta_stream_k"
-        assert ne.ngram_embed_workspace_bytes(plan, T) <= 4 << 20  # the partials fit the fixed array
+        assert ne.ngram_embed_plan_kernel_form(plan, T) == form
+        assert ne.ngram_embed_workspace_bytes(plan, T) <= 4 << 20  # everything fits the fixed array
         tokens = torch.from_numpy(gen.zipf_tokens(60 + call, T, cfg.V0)).cuda()
         offsets = torch.from_numpy(off_h).cuda()
         want = torch.empty((T, cfg.D), dtype=torch.bfloat16, device="cuda")
