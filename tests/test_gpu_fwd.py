@@ -500,9 +500,10 @@ def test_automatic_kernel_form(ne):
 ], ids=["D512N5K2", "D1024N3K4", "D2048N3K2_T1280"])
 @pytest.mark.parametrize("knobs,form", [
     ({"stream_k": 2, "pair_wide": 0}, "cta_pair_dense"),
-    ({"stream_k": 1}, "cta_pair_dense_stream_k"),
+    ({"stream_k": 1, "sms": 10}, "cta_pair_dense_stream_k"),  # 5 pairs: tiles split into pieces
+    ({"stream_k": 1}, None),  # stream-K where the units outnumber the device's pairs
     ({"stream_k": 2, "pair_wide": 1}, "cta_pair_wide_dense"),
-], ids=["dense", "dense_stream_k", "dense_wide"])
+], ids=["dense", "dense_stream_k_10sms", "dense_stream_k", "dense_wide"])
 def test_dense_a_forms_match_oracle(ne, shape, lengths, knobs, form):
     """The dense-A form (sub-rows gathered into G in the workspace, A by 2-D TMA boxes of G)
     in each of its schedules against the oracle on every row; repeatable bits; and the same
@@ -517,6 +518,12 @@ def test_dense_a_forms_match_oracle(ne, shape, lengths, knobs, form):
     ne.ngram_embed_plan_set_stream_k(plan, knobs["stream_k"])
     if "pair_wide" in knobs:
         ne.ngram_embed_plan_set_pair_wide(plan, knobs["pair_wide"])
+    if "sms" in knobs:
+        ne.ngram_embed_plan_set_sm_count(plan, knobs["sms"])
+    if form is None:
+        units = -(-len(tokens) // 256) * (cfg.D // 256) * (cfg.D // 64)
+        pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+        form = "cta_pair_dense_stream_k" if units >= pairs else "cta_pair_dense"
     assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == form
     out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
     assert status == 0
