@@ -580,9 +580,11 @@ int launch_gather(const ngram_embed_plan* p, const int32_t* idx, int64_t T, cons
 }
 
 // T_dev (optional): the kernels take min(*T_dev, T) tokens, a count known only on the device.
+// g_ready: in the dense-A form, G already holds the call's sub-rows (the decode step's fused
+// commit + hash + gather launch wrote it).
 int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int64_t T, const void* E0,
             const void* const* E_nk, const void* W, void* out, void* ws, size_t ws_size, int64_t ws_T,
-            cudaStream_t st, const int32_t* T_dev = nullptr) {
+            cudaStream_t st, const int32_t* T_dev = nullptr, bool g_ready = false) {
   if (p->variant == kSimt) {
     return p->dtype == NGRAM_F32
                ? launch_simt<float>(p, tokens, idx, T, E0, E_nk, W, out, ws, st, T_dev)
@@ -620,7 +622,7 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   if (form == kFormDense || form == kFormDenseSk || form == kFormDenseWide) {
     // the call's sub-rows into G (workspace), then A tiles as dense TMA boxes of G
     void* G = wsb + dense_g_offset(p, ws_T);
-    if ((rc = launch_gather(p, idx, T, E_nk, G, nullptr, nullptr, nullptr, ws, st))) return rc;
+    if (!g_ready && (rc = launch_gather(p, idx, T, E_nk, G, nullptr, nullptr, nullptr, ws, st))) return rc;
     if (p->map_A != G || p->map_A_T != T) {
       p->map_A = nullptr;
       if ((rc = encode_2d(&p->maps.A, G, p->D, static_cast<uint64_t>(T), static_cast<uint64_t>(p->D) * 2, kBK, kBM,
@@ -1302,6 +1304,30 @@ int ngram_embed_fwd_step(const ngram_embed_plan* plan_c, const int32_t* commit_t
   h.slots = cache_slots;
   h.idx_out = idx;
   h.status = status_ptr(workspace);
+  const int form = num_tokens > 0 ? choose_form(plan, num_tokens, workspace_bytes, num_tokens, false) : kFormSimt;
+  if (form == kFormDense || form == kFormDenseSk || form == kFormDenseWide) {
+    // commit + hash + the sub-row gather into G in one launch (a block per sequence), then
+    // the dense-A projection
+    GatherParams g{};
+    for (int s = 0; s < plan->S; ++s) {
+      g.E[s] = static_cast<const uint8_t*>(E_nk[s]);
+      g.Vs[s] = static_cast<uint32_t>(plan->V[s]);
+    }
+    g.G = static_cast<uint8_t*>(workspace) + dense_g_offset(plan, num_tokens);
+    g.T = num_tokens;
+    g.S = plan->S;
+    g.row_bytes = plan->d * plan->elt;
+    int sh = 0;
+    while ((1 << sh) < g.row_bytes / 16) ++sh;
+    g.vshift = (1 << sh) == g.row_bytes / 16 ? sh : -1;
+    g.eshift = -1;
+    g.status = status_ptr(workspace);
+    if ((rc = launch(commit_hash_gather_kernel, dim3(static_cast<unsigned>(num_seqs)), dim3(256), 0, st, plan->pdl,
+                     1, c, h, g)))
+      return rc;
+    return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace, workspace_bytes, num_tokens,
+                   st, nullptr, true);
+  }
   if ((rc = launch(commit_hash_kernel, dim3(static_cast<unsigned>((num_seqs + 7) / 8)), dim3(256), 0, st,
                    plan->pdl, 1, c, h)))
     return rc;
