@@ -306,7 +306,7 @@ def ngram_embed_bwd(plan: Plan, tokens, idx, grad_out, workspace, E_nk=None, W_s
 
 def ngram_hash_stats(V0: int, n: int, tokens, seq_offsets, moduli, workspace=None, stream=None):
     """Hit counts and collisions of the n-gram hash X_n mod V for each V in `moduli`:
-    returns (distinct_ngrams or None, [rows_hit per modulus])."""
+    returns (distinct_ngrams, [rows_hit per modulus])."""
     import torch
     mods = (_I64 * len(moduli))(*[int(v) for v in moduli])
     hits = (_I64 * len(moduli))()

@@ -827,7 +827,7 @@ uint64_t stats_set_cap(int64_t T) {
   return cap;
 }
 size_t stats_ws_bytes(int64_t T, int64_t max_modulus, int num_moduli) {
-  return kHeadBytes + round256(static_cast<size_t>(T) * 8) + round256(stats_set_cap(T) * 8) + 256 +
+  return kHeadBytes + round256(static_cast<size_t>(T) * 8 * kWinWords) + round256(stats_set_cap(T) * 8) + 256 +
          round256((static_cast<size_t>(max_modulus) / 32 + 1) * 4) + round256(static_cast<size_t>(num_moduli) * 8);
 }
 }  // namespace
@@ -864,7 +864,7 @@ int ngram_hash_stats(int64_t V0, int n, const int32_t* tokens, const int32_t* se
   uint8_t* base = static_cast<uint8_t*>(workspace);
   const uint64_t cap = stats_set_cap(num_tokens);
   auto* keys = reinterpret_cast<unsigned long long*>(base + kHeadBytes);
-  auto* set = reinterpret_cast<unsigned long long*>(base + kHeadBytes + round256(size_t(num_tokens) * 8));
+  auto* set = reinterpret_cast<unsigned long long*>(base + kHeadBytes + round256(size_t(num_tokens) * 8 * kWinWords));
   auto* distinct = reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(set) + round256(cap * 8));
   auto* bitmap = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(distinct) + 256);
   auto* hits = reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(bitmap) +
@@ -887,9 +887,14 @@ int ngram_hash_stats(int64_t V0, int n, const int32_t* tokens, const int32_t* se
   sp.status = status_ptr(workspace);
   const unsigned blocks = static_cast<unsigned>((num_tokens + 255) / 256);
   int rc = NGRAM_OK;
-  if (num_tokens > 0 && exact64) {
+  if (num_tokens > 0) {
     if (cudaMemsetAsync(set, 0xFF, cap * 8, st) != cudaSuccess) return NGRAM_ERR_CUDA;
-    if ((rc = launch(stats_keys_kernel, dim3(blocks), dim3(256), 0, st, false, 1, sp))) return rc;
+    if (exact64) {
+      if ((rc = launch(stats_keys_kernel, dim3(blocks), dim3(256), 0, st, false, 1, sp))) return rc;
+    } else {
+      if ((rc = launch(stats_window_keys_kernel, dim3(blocks), dim3(256), 0, st, false, 1, sp))) return rc;
+      if ((rc = launch(stats_window_insert_kernel, dim3(blocks), dim3(256), 0, st, false, 1, sp))) return rc;
+    }
   }
   for (int j = 0; j < num_moduli && num_tokens > 0; ++j) {
     sp.V = static_cast<uint32_t>(moduli[j]);
@@ -904,7 +909,7 @@ int ngram_hash_stats(int64_t V0, int n, const int32_t* tokens, const int32_t* se
       cudaMemcpyAsync(rows_hit, hits, size_t(num_moduli) * 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return NGRAM_ERR_CUDA;
-  *distinct_ngrams = exact64 ? static_cast<int64_t>(d_host) : -1;
+  *distinct_ngrams = static_cast<int64_t>(d_host);
   return NGRAM_OK;
 }
 

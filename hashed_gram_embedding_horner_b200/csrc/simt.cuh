@@ -226,6 +226,11 @@ __device__ __forceinline__ void ln_load(const LayerNormParams& p, int64_t row, i
   }
 }
 
+// Rows of up to kLnRegVectors x 32 16-byte vectors (bf16: D <= 4096) are read from memory
+// once: each lane keeps its vectors in registers (all loads in flight together), and the
+// mean, the centred second moment and the output are computed from them.
+constexpr int kLnRegVectors = 16;
+
 template <bool F32>
 __global__ void __launch_bounds__(256) layernorm_kernel(const __grid_constant__ LayerNormParams p) {
   constexpr int VW = F32 ? 4 : 8;  // values per 16-byte vector
@@ -235,6 +240,70 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __grid_constant__ 
   const int lane = threadIdx.x & 31;
   if (row >= p.T) return;
   const int nv = p.D / VW;  // D * element size is a multiple of 16 for every plan
+  if (nv <= 32 * kLnRegVectors) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x) + row * p.D * (F32 ? 4 : 2));
+    uint4 u[kLnRegVectors];
+#pragma unroll
+    for (int j = 0; j < kLnRegVectors; ++j)
+      if (lane + 32 * j < nv) u[j] = src[lane + 32 * j];
+    auto values = [&](int j, float (&v)[VW]) {
+      const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+      if constexpr (F32) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) v[h] = __uint_as_float(w[h]);
+      } else {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          v[2 * h] = __uint_as_float(w[h] << 16);
+          v[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+        }
+      }
+    };
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < kLnRegVectors; ++j) {
+      if (lane + 32 * j >= nv) break;
+      float v[VW];
+      values(j, v);
+#pragma unroll
+      for (int k = 0; k < VW; ++k) sum += v[k];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float mean = sum / static_cast<float>(p.D);
+    float sq = 0.f;
+#pragma unroll
+    for (int j = 0; j < kLnRegVectors; ++j) {
+      if (lane + 32 * j >= nv) break;
+      float v[VW];
+      values(j, v);
+#pragma unroll
+      for (int k = 0; k < VW; ++k) sq += (v[k] - mean) * (v[k] - mean);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    const float rstd = rsqrtf(sq / static_cast<float>(p.D) + p.eps);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.y) + row * p.D * (F32 ? 4 : 2));
+#pragma unroll
+    for (int j = 0; j < kLnRegVectors; ++j) {
+      const int c = lane + 32 * j;
+      if (c >= nv) break;
+      float v[VW];
+      values(j, v);
+#pragma unroll
+      for (int k = 0; k < VW; ++k) {
+        const int col = c * VW + k;
+        v[k] = (v[k] - mean) * rstd * (p.gamma ? p.gamma[col] : 1.f) + (p.beta ? p.beta[col] : 0.f);
+      }
+      if constexpr (F32) {
+        dst[c] = make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]));
+      } else {
+        dst[c] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                            pack_bf16x2(v[6], v[7]));
+      }
+    }
+    return;
+  }
   float sum = 0.f;
   for (int c = lane; c < nv; c += 32) {
     float v[VW];

@@ -286,8 +286,8 @@ int ngram_embed_bwd(const ngram_embed_plan* plan, const int32_t* tokens, const i
  * sequence start) over a token stream:
  *   rows_hit[j]       number of distinct rows (X_n mod moduli[j]) hit by the stream
  *                     (hit rate = rows_hit[j] / moduli[j]);
- *   *distinct_ngrams  number of distinct n-gram windows in the stream, or -1 when
- *                     V0^n >= 2^64 (windows are then not counted);
+ *   *distinct_ngrams  number of distinct n-gram windows in the stream (exact: windows
+ *                     compared as integers X_n when V0^n < 2^64, else id by id);
  *   collisions at moduli[j] = *distinct_ngrams - rows_hit[j].
  * tokens / seq_offsets as for ngram_embed_fwd (device); moduli, rows_hit, distinct_ngrams
  * are HOST arrays. Analysis, not the hot path: the call synchronises `stream`.

@@ -699,15 +699,15 @@ def test_output_scale_amplifies_the_layer(ne, pair):
 
 
 @pytest.mark.parametrize("dtype,D,N,K", [("bf16", 2048, 3, 1), ("bf16", 384, 2, 3), ("fp32", 64, 3, 1),
-                                         ("fp32", 36, 2, 3)])
+                                         ("fp32", 36, 2, 3), ("bf16", 4096, 5, 2), ("bf16", 8192, 2, 2)])
 def test_layernorm_matches_oracle(ne, dtype, D, N, K):
-    """LayerNorm amplification of a layer output (bf16: the prefill D; an odd width; fp32 tiny
-    widths incl. one not a multiple of 8), in place and out of place, with and without
-    gamma/beta."""
+    """LayerNorm amplification of a layer output (bf16: the prefill widths, an odd width, and
+    D = 8192, above the rows kept in registers; fp32 tiny widths incl. one not a multiple of
+    8), in place and out of place, with and without gamma/beta."""
     rng = np.random.default_rng(7)
     T = 301
     S = (N - 1) * K
-    plan = ne.ngram_embed_plan_create(1000, D, N, K, [4099, 5003, 6007][:S], ne.NGRAM_BF16 if dtype == "bf16" else ne.NGRAM_F32)
+    plan = ne.ngram_embed_plan_create(1000, D, N, K, configs.primes_from(4099, 8)[:S], ne.NGRAM_BF16 if dtype == "bf16" else ne.NGRAM_F32)
     ws = ne.new_workspace(plan, T)
     x32 = rng.normal(0.01, 0.007, (T, D)).astype(np.float32)
     if dtype == "bf16":

@@ -29,7 +29,8 @@ def test_worked_example(ne):
 @pytest.mark.parametrize("n", [2, 3, 4, 5])
 def test_zipf_stream_matches_oracle(ne, n):
     """100 Zipf(1.1) sequences over V0 = 131072 (n <= 3: exact 64-bit window keys; n >= 4:
-    V0^n >= 2^64, rows only), moduli on and off multiples of V0, a ragged length mix."""
+    V0^n >= 2^64, windows compared id by id), moduli on and off multiples of V0, a ragged
+    length mix."""
     V0 = 131072
     rng = np.random.default_rng(n)
     lengths = rng.integers(0, 700, 100)
@@ -40,4 +41,18 @@ def test_zipf_stream_matches_oracle(ne, n):
     got = ne.ngram_hash_stats(V0, n, dev_i32(tok), dev_i32(off), moduli)
     windows, rows = oracle.hash_stats(V0, n, tok, off, moduli)
     assert got[1] == rows
-    assert got[0] == (windows if n <= 3 else None)
+    assert got[0] == windows
+
+
+def test_eight_gram_windows_over_the_largest_vocabulary(ne):
+    """n = 8 with V0 = 2^31 - 1 (all four packed words in use; X_8 < 2^248): distinct windows
+    and rows against the oracle's exact integers, including repeated windows."""
+    V0 = 2 ** 31 - 1
+    rng = np.random.default_rng(8)
+    base = rng.integers(0, V0, 300).astype(np.int32)
+    tok = np.concatenate([base, base[:120], rng.integers(0, 3, 200).astype(np.int32), base[50:90]])
+    off = gen.offsets_from_lengths([300, 120, 200, 40])
+    moduli = [7274513, 2 ** 31 - 3, 1]
+    got = ne.ngram_hash_stats(V0, 8, dev_i32(tok), dev_i32(off), moduli)
+    windows, rows = oracle.hash_stats(V0, 8, tok, off, moduli)
+    assert got == (windows, rows)
