@@ -326,8 +326,7 @@ KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pa
 
 
 def ngram_embed_plan_set_dense_a(plan: "Plan", mode: int):
-    """Dense-A form (sub-rows gathered into G first, A by dense TMA): 0 automatic (small
-    calls), 1 whenever the workspace holds G, 2 never."""
+    """Dense-A form (sub-rows gathered into G first, A by dense TMA): 1 on, 0 off (default)."""
     _check(_lib.ngram_embed_plan_set_dense_a(plan.handle, int(mode)), "ngram_embed_plan_set_dense_a")
 
 

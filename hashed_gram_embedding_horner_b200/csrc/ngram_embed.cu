@@ -69,7 +69,7 @@ struct ngram_embed_plan {
   bool pdl = false;            // launch as programmatic dependent launches
   float out_scale = 1.0f;      // embedding amplification factor folded into the 1/(S+1) scale
   int pair_wide = -1;          // pair form with 512-column tiles: 1 on, 0 off, -1 automatic
-  int dense_a = 0;             // sub-rows gathered into G first, A by dense TMA: 0 automatic, 1 on, 2 off
+  int dense_a = 0;             // sub-rows gathered into G first, A by dense TMA: 1 on, 0 off
   const void* map_A = nullptr;  // the dense-A map's pointer and row count
   int64_t map_A_T = -1;
   int max_clusters[3] = {0, 0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
@@ -107,24 +107,21 @@ size_t sk_partial_bytes(const ngram_embed_plan* p) {
 }
 // The dense-A form: the call's sub-rows gathered into G [T x D] bf16 first (a stand-alone
 // gather kernel with every resident thread copying), then the CTA-pair projection reads A as
-// dense TMA boxes of G. Automatic for calls whose G is at most this many bytes: G then stays
-// in L2 between the two launches, and such calls (decode steps: 1280 tokens x 8 KiB = 10.5 MB
-// at D = 4096) are too small for the fused row gather to keep enough DRAM misses in flight.
-constexpr size_t kDenseAutoBytes = size_t(24) << 20;
+// dense TMA boxes of G. Only on request: measured on B200 at the 1280-token decode step
+// (D = 4096) it took 78 us a step against 70 us for the fused one-CTA stream-K form, because
+// the tensor-core kernels there are limited by the rate at which an SM's shared memory fills
+// from L2 (about 55 GB/s per SM), not by the latency of the row gather, and the dense form
+// moves the same A bytes plus its own copy.
 size_t dense_g_bytes(const ngram_embed_plan* p, int64_t T) {
   return (static_cast<size_t>(T) * static_cast<size_t>(p->D) * 2 + 255) & ~size_t(255);
 }
-// Whether calls of T tokens may take the dense-A form at all (its kernel needs 256-column W
-// halves: tile width 256, D % 256 == 0).
-bool dense_capable(const ngram_embed_plan* p) { return p->tc_ok && p->bn == 256 && p->dense_a != 2; }
-bool dense_wanted(const ngram_embed_plan* p, int64_t T) {
-  return dense_capable(p) && (p->dense_a == 1 || dense_g_bytes(p, T) <= kDenseAutoBytes);
-}
+// The dense-A form needs 256-column W halves: tile width 256, D % 256 == 0.
+bool dense_wanted(const ngram_embed_plan* p) { return p->tc_ok && p->bn == 256 && p->dense_a == 1; }
 // Workspace: [head | T x S indices | stream-K partials | G (dense-A form)]
 size_t dense_g_offset(const ngram_embed_plan* p, int64_t ws_T) { return ws_base(p, ws_T) + sk_partial_bytes(p); }
 // Bytes that let every call of up to T tokens take its fastest schedule.
 size_t ws_bytes(const ngram_embed_plan* p, int64_t T) {
-  return ws_base(p, T) + sk_partial_bytes(p) + (dense_wanted(p, T) ? dense_g_bytes(p, T) : 0);
+  return ws_base(p, T) + sk_partial_bytes(p) + (dense_wanted(p) ? dense_g_bytes(p, T) : 0);
 }
 
 int check_launch() { return cudaGetLastError() == cudaSuccess ? NGRAM_OK : NGRAM_ERR_CUDA; }
@@ -500,9 +497,9 @@ enum Form : int {
   kFormDenseWide = 8,  // the same with 256 x 512 tiles
 };
 
-// Stream-K for the dense-A pair form: automatic where a grid of whole 256 x 256 tiles would
-// take two or more waves of pairs and leave many pairs idle in the last (a decode step of
-// 1280 tokens at D = 4096: 80 tiles on 74 pairs), as for the one-CTA form.
+// Stream-K for the dense-A pair form: where a grid of whole 256 x 256 tiles would take two or
+// more waves of pairs and leave many pairs idle in the last (a decode step of 1280 tokens at
+// D = 4096: 80 tiles on 74 pairs), as for the one-CTA form.
 bool dense_stream_k(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws_T) {
   if (p->stream_k == 2 || p->sms < 2 || p->pair_wide == 1) return false;
   const int64_t pairs = p->sms / 2;
@@ -520,7 +517,7 @@ bool dense_stream_k(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_
 // count_on_device: the token count is known only on the device (a draft call's misses).
 int choose_form(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws_T, bool count_on_device) {
   if (p->variant == kSimt) return kFormSimt;
-  if (!count_on_device && p->cta_pair != 0 && dense_wanted(p, T) &&
+  if (!count_on_device && p->cta_pair != 0 && dense_wanted(p) &&
       ws_size >= dense_g_offset(p, ws_T) + dense_g_bytes(p, T)) {
     if (dense_stream_k(p, T, ws_size, ws_T)) return kFormDenseSk;
     return use_pair_wide(p, T) ? kFormDenseWide : kFormDense;
@@ -779,7 +776,7 @@ int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_token
 }
 
 int ngram_embed_plan_set_dense_a(ngram_embed_plan* plan, int mode) {
-  if (!plan || mode < 0 || mode > 2) return NGRAM_ERR_INVALID_ARG;
+  if (!plan || mode < 0 || mode > 1) return NGRAM_ERR_INVALID_ARG;
   plan->dense_a = mode;
   return NGRAM_OK;
 }

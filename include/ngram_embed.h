@@ -111,8 +111,8 @@ int ngram_embed_plan_destroy(ngram_embed_plan* plan);
  * status word, then the stream-K arrival counters), the [max_tokens x S] int32 index
  * buffer, then, for plans that use the tensor-core kernel, 2 x (SM count) x 128 x 256 fp32
  * stream-K partial tiles (the plan's SM count: see ngram_embed_plan_set_sm_count), then,
- * for calls that the dense-A form would take (ngram_embed_plan_set_dense_a), the
- * [max_tokens x D] bf16 G buffer, each region rounded up to 256 bytes. A workspace without
+ * while the dense-A form is on (ngram_embed_plan_set_dense_a), the [max_tokens x D] bf16
+ * G buffer, each region rounded up to 256 bytes. A workspace without
  * the partials or G (head + index buffer) is accepted too; the projection then takes the
  * forms that fit. The head must be zeroed once before first use (ngram_embed_clear_status
  * does it); the rest needs no init. The kernels leave the counters zero after every call
@@ -383,15 +383,15 @@ int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_token
 /* Dense-A form of the tensor-core projection: the call's sub-rows are first copied into a
  * G buffer [num_tokens x D] (bf16) in the workspace by a gather kernel that keeps every
  * resident thread's loads in flight, then the CTA-pair kernel reads its A tiles as dense
- * 2-D TMA boxes of G (from L2, where G stays between the two launches) instead of gathering
- * rows itself. 0 (default) = automatic: calls whose G takes at most 24 MiB (up to 3072
- * tokens at D = 4096: decode steps, whose fused row gather leaves the tensor cores waiting on
- * DRAM misses), when the workspace holds G and the plan allows the pair form with 256-column
- * tiles; 1 = whenever the workspace holds G; 2 = never. ngram_embed_workspace_bytes includes G
- * for the calls this setting selects. The stream-K schedule applies to it automatically
- * where whole tiles would leave a thin last wave of pairs. A tuning knob: results agree
- * within the stated tolerance (the k-block order differs). NGRAM_ERR_INVALID_ARG for other
- * values. */
+ * 2-D TMA boxes of G instead of gathering rows itself; in ngram_embed_fwd_step the commit,
+ * the hash and this gather are one launch. 1 = on (whenever the workspace holds G and the
+ * plan allows the pair form with 256-column tiles), 0 = off (default: measured on B200 at a
+ * 1280-token decode step, 78 us against 70 us for the fused forms, whose limit there is the
+ * rate at which shared memory fills from L2, not the row gather). ngram_embed_workspace_bytes
+ * includes G while it is on. The stream-K schedule applies to it where whole tiles would
+ * leave a thin last wave of pairs, 512-column tiles where they fill their waves. A tuning
+ * knob: results agree within the stated tolerance (the k-block order differs).
+ * NGRAM_ERR_INVALID_ARG for other values. */
 int ngram_embed_plan_set_dense_a(ngram_embed_plan* plan, int mode);
 
 /* Tensor-core tile width in output columns: 256 (default when D % 256 == 0) or 128. */

@@ -77,9 +77,8 @@ def test_plan_without_device_validates_then_fails_launch(ne):
     assert rc == 0 and h.value
     lib = ne._lib
     ws_need = lib.ngram_embed_workspace_bytes(h, 1000)
-    # head (status word + 2048 x 4 stream-K counters), indices; no SM count without a device,
-    # so no stream-K partials; G for the dense-A form (1000 x 2048 bf16: a small call)
-    assert ws_need == 256 + 2048 * 4 * 4 + ((1000 * 4 * 4 + 255) // 256) * 256 + 1000 * 2048 * 2
+    # head (status word + 2048 x 4 stream-K counters), indices; no SM count without a device
+    assert ws_need == 256 + 2048 * 4 * 4 + ((1000 * 4 * 4 + 255) // 256) * 256
     fake = ctypes.c_void_p(0x10000)           # never dereferenced
     odd = ctypes.c_void_p(0x10004)
     tabs = (ctypes.c_void_p * 4)(0x20000, 0x30000, 0x40000, 0x50000)
@@ -97,27 +96,24 @@ def test_plan_without_device_validates_then_fails_launch(ne):
     assert lib.ngram_embed_plan_set_stream_k(h, 3) == -1 and lib.ngram_embed_plan_set_stream_k(h, 2) == 0
     assert lib.ngram_embed_plan_set_pdl(h, 2) == -1 and lib.ngram_embed_plan_set_pdl(h, 1) == 0
     assert lib.ngram_embed_plan_set_a_stages(h, 5) == -1 and lib.ngram_embed_plan_set_a_stages(h, 6) == 0
-    # no device: the stream-K schedule (it needs the SM count) never applies. 1280 tokens at
-    # D = 2048 (5.2 MB of G) take the dense-A pair form; with it off, the fused pair form
-    assert lib.ngram_embed_plan_kernel_form(h, 1280) == 6 and lib.ngram_embed_plan_kernel_form(h, -1) == -1
-    assert lib.ngram_embed_plan_set_dense_a(h, 3) == -1 and lib.ngram_embed_plan_set_dense_a(h, -1) == -1
-    assert lib.ngram_embed_plan_set_dense_a(h, 2) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 3
+    # no device: the stream-K schedule (it needs the SM count) never applies, so the pair form
+    assert lib.ngram_embed_plan_kernel_form(h, 1280) == 3 and lib.ngram_embed_plan_kernel_form(h, -1) == -1
+    assert lib.ngram_embed_plan_set_dense_a(h, 2) == -1 and lib.ngram_embed_plan_set_dense_a(h, -1) == -1
     assert lib.ngram_embed_plan_set_cta_pair(h, 0) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 1
     assert lib.ngram_embed_plan_set_dense_a(h, 1) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 1
     assert lib.ngram_embed_plan_set_cta_pair(h, -1) == 0 and lib.ngram_embed_plan_set_cta_pair(h, 2) == -1
-    # forced: the dense-A form at any size whose G the workspace holds (it grows by T x D x 2)
-    assert lib.ngram_embed_plan_kernel_form(h, 32768) == 6
+    # the dense-A form when asked for: at any size whose G the workspace holds (it grows by T x D x 2)
+    assert lib.ngram_embed_plan_kernel_form(h, 1280) == 6 and lib.ngram_embed_plan_kernel_form(h, 32768) == 6
     with_g = lib.ngram_embed_workspace_bytes(h, 32768)
     assert lib.ngram_embed_plan_set_dense_a(h, 0) == 0 and lib.ngram_embed_plan_kernel_form(h, 32768) == 3
     assert with_g - lib.ngram_embed_workspace_bytes(h, 32768) == 32768 * 2048 * 2
-    assert lib.ngram_embed_plan_set_dense_a(h, 2) == 0
     # 512-column pair tiles (D = 2048 here): on when forced, automatic needs the SM count
     assert lib.ngram_embed_plan_set_pair_wide(h, 2) == -1 and lib.ngram_embed_plan_set_pair_wide(h, -2) == -1
     assert lib.ngram_embed_plan_set_pair_wide(h, 1) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 4
-    assert lib.ngram_embed_plan_set_dense_a(h, 0) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 8
+    assert lib.ngram_embed_plan_set_dense_a(h, 1) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 8
     assert lib.ngram_embed_plan_set_tile_n(h, 128) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 3
-    assert lib.ngram_embed_plan_set_tile_n(h, 256) == 0
-    assert lib.ngram_embed_plan_set_pair_wide(h, -1) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 6
+    assert lib.ngram_embed_plan_set_tile_n(h, 256) == 0 and lib.ngram_embed_plan_set_dense_a(h, 0) == 0
+    assert lib.ngram_embed_plan_set_pair_wide(h, -1) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 3
     assert lib.ngram_embed_plan_uses_tensor_cores(h) == 1
     bad_cache = ne._Cache(0, 0, 0, 4, 8)
     assert lib.ngram_cache_rollback(h, ctypes.byref(bad_cache), None, fake, 3, fake, ws_need, None) == -1
@@ -148,18 +144,21 @@ V25 = (3342341, 3342371, 3342379, 3342413, 3342419, 3342439, 3342457, 3342473)
 @pytest.mark.parametrize("kw,T,sms,knobs,form", [
     (dict(), 32768, 148, {}, 4),                                  # prefill D = 2048: 512-column pair tiles
     (dict(D=4096, N=5, K=2, V=V25), 65536, 148, {}, 4),           # varlen prefill D = 4096
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {}, 7),            # decode step: dense A, pairs' stream-K
-    (dict(D=4096, N=3, K=4, V=V25), 128, 148, {}, 6),             # one wave: dense A, 256-column tiles
-    (dict(D=4096, N=3, K=4, V=V25), 5120, 148, {}, 3),            # 42 MB of G: fused; 160 wide tiles, a thin 3rd wave
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 40, {}, 8),             # 20 pairs: 40 wide tiles fill 2 waves
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"dense_a": 2}, 2),  # fused: one-CTA stream-K
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"dense_a": 2, "cta_pair": 1}, 4),
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"dense_a": 2, "cta_pair": 1, "stream_k": 1}, 5),
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {}, 2),            # decode step: one-CTA stream-K
+    (dict(D=4096, N=3, K=4, V=V25), 128, 148, {}, 3),             # one wave: 256-column pair tiles
+    (dict(D=4096, N=3, K=4, V=V25), 5120, 148, {}, 3),            # 160 wide tiles: a thin third wave
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 1}, 4),
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 1, "stream_k": 1}, 5),
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 0, "stream_k": 2}, 1),
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"stream_k": 2}, 8),  # dense A without stream-K: wide tiles
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 40, {"dense_a": 2}, 4),
-    (dict(), 32768, 148, {"tile_n": 128}, 3),                     # 128-column W halves: never wide, never dense
-    (dict(), 32768, 148, {"dense_a": 1}, 8),                      # forced dense A at prefill: wide tiles
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 40, {}, 4),             # 20 pairs: 40 wide tiles fill 2 waves
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"dense_a": 1}, 7),  # dense A: the pairs' stream-K
+    (dict(D=4096, N=3, K=4, V=V25), 128, 148, {"dense_a": 1}, 6),
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 40, {"dense_a": 1}, 8),  # 20 pairs: wide tiles fill 2 waves
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"dense_a": 1, "stream_k": 2}, 8),
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"dense_a": 1, "cta_pair": 0}, 2),  # dense A needs pairs
+    (dict(), 32768, 148, {"tile_n": 128}, 3),                     # 128-column W halves: never wide
+    (dict(), 32768, 148, {"tile_n": 128, "dense_a": 1}, 3),       # ... nor dense A
+    (dict(), 32768, 148, {"dense_a": 1}, 8),                      # dense A at prefill: wide tiles
     (dict(D=768, N=2, K=3, V=V25[:3]), 32768, 148, {}, 3),        # D % 512 != 0
 ])
 def test_kernel_form_choice_for_a_device_size(ne, kw, T, sms, knobs, form):

@@ -192,9 +192,11 @@ def test_evicted_context_is_flagged(ne):
     assert ne.status_names(ne.ngram_embed_get_status(ws)) == ["EVICTED"]
 
 
-def test_fused_commit_and_step_equals_separate_calls(ne):
-    """ngram_embed_fwd_step (commit of the previous step fused with this step's hashing) gives
-    the same outputs, bit for bit, and the same ring as ngram_cache_commit + ngram_embed_fwd."""
+@pytest.mark.parametrize("dense_a", [0, 1])
+def test_fused_commit_and_step_equals_separate_calls(ne, dense_a):
+    """ngram_embed_fwd_step (commit of the previous step fused with this step's hashing; with
+    the dense-A form also with the sub-row gather into G, one launch) gives the same outputs,
+    bit for bit, the same indices and the same ring as ngram_cache_commit + ngram_embed_fwd."""
     from tests.helpers import host_tables, to_device
     N, K, D, B, P, C = 3, 2, 512, 24, 5, 8
     V0, V = 3000, [4099, 5003, 6007, 7001]
@@ -202,6 +204,8 @@ def test_fused_commit_and_step_equals_separate_calls(ne):
     E0h, Eh, Wh = host_tables(cfg)
     E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
     plan = ne.ngram_embed_plan_create(V0, D, N, K, V, ne.NGRAM_BF16)
+    ne.ngram_embed_plan_set_dense_a(plan, dense_a)
+    assert ne.ngram_embed_plan_kernel_form(plan, B * P) == ("cta_pair_dense" if dense_a else "cta_pair")
     ws1, ws2 = ne.new_workspace(plan, B * P), ne.new_workspace(plan, B * P)
     c1, c2 = ne.Cache.empty(B, C), ne.Cache.empty(B, C)
     for c, w in ((c1, ws1), (c2, ws2)):
@@ -221,6 +225,8 @@ def test_fused_commit_and_step_equals_separate_calls(ne):
                                 commit_tokens=None if prev is None else prev[0], commit_stride=P,
                                 commit_counts=None if prev is None else prev[1])
         assert torch.equal(o1, o2), step
+        head = 33024  # the workspace's index buffer follows its head
+        assert torch.equal(ws1[head:head + B * P * 16], ws2[head:head + B * P * 16])  # [T x S] int32 indices
         assert torch.equal(c1.ring, c2.ring) and torch.equal(c1.len, c2.len) and torch.equal(c1.valid_from, c2.valid_from)
         prev = (tok, cnt)
     assert ne.ngram_embed_get_status(ws1) == 0 and ne.ngram_embed_get_status(ws2) == 0

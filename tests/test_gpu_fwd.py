@@ -454,8 +454,8 @@ def test_reduced_sm_count_every_form(ne, sms):
     E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
     want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
     forms = set()
-    for pair, wide, sk, dense in ((None, None, 0, 2), (1, 1, 0, 2), (1, 0, 1, 2), (1, 0, 2, 2), (0, 0, 1, 2),
-                                  (0, 0, 2, 2), (None, 0, 1, 1), (None, 0, 2, 1), (None, 1, 2, 1)):
+    for pair, wide, sk, dense in ((None, None, 0, 0), (1, 1, 0, 0), (1, 0, 1, 0), (1, 0, 2, 0), (0, 0, 1, 0),
+                                  (0, 0, 2, 0), (None, 0, 1, 1), (None, 0, 2, 1), (None, 1, 2, 1)):
         plan = plan_for(ne, cfg, pair=pair)
         ne.ngram_embed_plan_set_sm_count(plan, sms)
         ne.ngram_embed_plan_set_pair_wide(plan, wide)
@@ -471,25 +471,25 @@ def test_reduced_sm_count_every_form(ne, sms):
 
 def test_automatic_kernel_form(ne):
     """Prefill grids run the CTA-pair form with 512-column tiles; a 1280-token decode step at
-    D = 4096 (10.5 MB of gathered sub-rows) runs the dense-A pair form with the pairs'
-    stream-K schedule (80 tiles of 256 x 256 on 74 pairs); a grid of one wave keeps the
-    256-column tiles (more SMs busy). Without the dense-A form, the decode step runs the
-    one-CTA stream-K schedule."""
+    D = 4096 (160 tiles of 128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule;
+    a grid of one wave keeps the 256-column pair tiles (more SMs busy). The pairs' stream-K
+    schedule is taken only when both the pair form and stream-K are asked for. With the
+    dense-A form on, the decode step runs it with the pairs' stream-K schedule."""
     for cfg in (configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN):
         plan = plan_for(ne, cfg)
         assert ne.ngram_embed_plan_kernel_form(plan, 32768) == "cta_pair_wide"
     plan = plan_for(ne, configs.SPEC_DECODE)
-    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_dense_stream_k"
-    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair_dense"  # one wave: nothing to balance
-    ne.ngram_embed_plan_set_dense_a(plan, 2)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "one_cta_stream_k"
-    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"
+    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"  # one wave: nothing to balance
     ne.ngram_embed_plan_set_cta_pair(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_wide"
     ne.ngram_embed_plan_set_stream_k(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_stream_k"
     ne.ngram_embed_plan_set_cta_pair(plan, None)
     ne.ngram_embed_plan_set_stream_k(plan, 0)
+    ne.ngram_embed_plan_set_dense_a(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_dense_stream_k"
+    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair_dense"
     assert ne.ngram_embed_plan_kernel_form(plan_for(ne, configs.TINY), 128) == "cuda_cores"
 
 
@@ -531,7 +531,7 @@ def test_dense_a_forms_match_oracle(ne, shape, lengths, knobs, form):
     assert_close(to_host_f64(out), want, what=f"{cfg.name} {form}")
     again, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
     assert status == 0 and torch.equal(out, again)
-    ne.ngram_embed_plan_set_dense_a(plan, 2)
+    ne.ngram_embed_plan_set_dense_a(plan, 0)
     fused, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
     assert status == 0
     assert (out.float() - fused.float()).abs().max().item() <= 2e-2

@@ -74,7 +74,7 @@ def _noalloc_cfg():
                                V_nk=tuple(configs.primes_from(20000, 8)), dtype="bf16", seed=5)
 
 
-@pytest.mark.parametrize("dense_a,form", [(2, "one_cta_stream_k"), (1, "cta_pair_dense_stream_k")])
+@pytest.mark.parametrize("dense_a,form", [(0, "one_cta_stream_k"), (1, "cta_pair_dense_stream_k")])
 def test_static_workspace_stream_k_matches_fwd(ne, dense_a, form):
     """With 8 SMs the stream-K partial tiles (2 x 8 x 128 KB) fit the fixed array, so the
     schedules whose arrival counters and partials (and, in the dense-A form, the gathered
