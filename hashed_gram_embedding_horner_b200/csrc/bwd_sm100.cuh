@@ -10,104 +10,19 @@
 // Colliding rows (several tokens, one table row) add up: every scatter is an fp32 atomic
 // add, so the summation order (not the set of terms) varies between runs.
 //
-// Both GEMMs run on one kernel, `dense_gemm_sm100_kernel`: A [M x K] and B [N x K], both
-// K-major bf16 tiles brought in by 2-D TMA (the operands that are not K-major in memory —
-// W for dG, g and G for dW — are first transposed into the workspace), fp32 accumulators
+// Both GEMMs run on one kernel, `dense_gemm_sm100_kernel`: bf16 A (M x K) and B (N x K)
+// tiles brought in by 2-D TMA straight from the tensors as they lie in memory — K-major
+// (K contiguous: g for dG) or MN-major (M or N contiguous: W for dG, g and G for dW), the
+// tensor cores reading either layout from its shared-memory descriptor — fp32 accumulators
 // in TMEM, work units of (128 x BN tile, k range) handed out round-robin to persistent
 // CTAs (split-K where tiles are few), and an epilogue that atomically adds the scaled
-// partial tile into its destination: sub-table gradient rows (dG) or dW.
+// partial tile into its destination: sub-table gradient rows (dG) or dW. The only copy is
+// G itself, gathered row by row from the sub-tables into the workspace for dW.
 #pragma once
 
 #include "proj_sm100.cuh"
 
 namespace ngram {
-
-// ------------------------------------------------------------------ transposes
-// 64 x 64 bf16 tiles through shared memory, 16-byte loads and stores on both sides: 256
-// threads read the tile's 64 source rows (128 bytes each) and write its 64 destination rows.
-
-constexpr int kTT = 64;        // tile edge
-constexpr int kTTPad = 8;      // bf16 of padding per shared row (rows 144 bytes apart)
-
-// src_row(r) -> pointer to the 64 source values of tile row r (or nullptr: zeros).
-template <typename SrcRow>
-__device__ __forceinline__ void transpose_tile(uint16_t (*tile)[kTT + kTTPad], SrcRow src_row, uint16_t* dst,
-                                               int64_t dst_stride, int64_t dst_col0, int dst_rows,
-                                               int64_t dst_cols) {
-  const int t = threadIdx.x;
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {  // 64 rows x 8 vectors
-    const int v = t + 256 * k;
-    const int r = v >> 3, c8 = (v & 7) * 8;
-    const uint16_t* src = src_row(r);
-    const uint4 u = src ? *reinterpret_cast<const uint4*>(src + c8) : make_uint4(0, 0, 0, 0);
-    *reinterpret_cast<uint2*>(&tile[r][c8]) = make_uint2(u.x, u.y);
-    *reinterpret_cast<uint2*>(&tile[r][c8 + 4]) = make_uint2(u.z, u.w);
-  }
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {  // 64 destination rows (source columns) x 8 vectors
-    const int v = t + 256 * k;
-    const int c = v >> 3, r8 = (v & 7) * 8;
-    if (c >= dst_rows || dst_col0 + r8 >= dst_cols) continue;
-    uint32_t w[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h)
-      w[h] = static_cast<uint32_t>(tile[r8 + 2 * h][c]) | (static_cast<uint32_t>(tile[r8 + 2 * h + 1][c]) << 16);
-    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(c) * dst_stride + dst_col0 + r8) =
-        make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
-// dst[c][r] = src[r][c] for r < R, 0 for R <= r < R_pad (dst rows are R_pad long, a multiple
-// of 8, so they stay 16-byte aligned for TMA). C a multiple of 64.
-struct TransposeParams {
-  const uint16_t* src;
-  uint16_t* dst;
-  int64_t R, R_pad;
-  int C;
-};
-
-__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __grid_constant__ TransposeParams p) {
-  __shared__ __align__(16) uint16_t tile[kTT][kTT + kTTPad];
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kTT;
-  const int c0 = blockIdx.y * kTT;
-  transpose_tile(
-      tile, [&](int r) { return r0 + r < p.R ? p.src + (r0 + r) * p.C + c0 : nullptr; },
-      p.dst + static_cast<int64_t>(c0) * p.R_pad, p.R_pad, r0, kTT, p.R_pad);
-}
-
-// GT[c][i] = G[i][c] = E_s[idx[i][s]][c - s d] (s = c / d) for i < T, 0 for T <= i < T_pad.
-struct GatherTParams {
-  const int32_t* idx;
-  const uint16_t* E[kMaxS];
-  uint32_t Vs[kMaxS];
-  uint16_t* dst;
-  int64_t T, T_pad;
-  int S, d, D;
-  int* status;
-};
-
-__global__ void __launch_bounds__(256) gather_transpose_kernel(const __grid_constant__ GatherTParams p) {
-  __shared__ __align__(16) uint16_t tile[kTT][kTT + kTTPad];
-  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kTT;
-  const int c0 = blockIdx.y * kTT;  // 64 columns never straddle two sub-tables (d % 64 == 0)
-  const int s = c0 / p.d;
-  const int j0 = c0 - s * p.d;
-  transpose_tile(
-      tile,
-      [&](int r) -> const uint16_t* {
-        const int64_t i = i0 + r;
-        if (i >= p.T) return nullptr;
-        int32_t row = p.idx[i * p.S + s];
-        if (static_cast<uint32_t>(row) >= p.Vs[s]) {
-          set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
-          row = 0;
-        }
-        return p.E[s] + static_cast<int64_t>(row) * p.d + j0;
-      },
-      p.dst + static_cast<int64_t>(c0) * p.T_pad, p.T_pad, i0, kTT, p.T_pad);
-}
 
 // ------------------------------------------------------------------ dE_0 scatter
 // dE0[v] += c * sum_{i : t_i = v} g_i. Token streams repeat ids heavily (Zipf: the commonest
@@ -267,8 +182,11 @@ __global__ void __launch_bounds__(256) e0_reduce_kernel(const __grid_constant__ 
 enum GemmEpi : int { kEpiScatterSub = 0, kEpiAccumDense = 1 };
 
 struct DenseMaps {
-  CUtensorMap A;  // [M x K] bf16, K-major, box {64, 128}, 128-byte swizzle
-  CUtensorMap B;  // [N x K] bf16, K-major, box {64, BN}, 128-byte swizzle
+  // K-major operand: [rows x K] bf16, box {64, 128 (A) or BN (B)}; MN-major operand:
+  // [K x rows] bf16 (rows contiguous), box {64, 64}: a tile is rows / 64 such boxes. All
+  // with the 128-byte swizzle.
+  CUtensorMap A;
+  CUtensorMap B;
 };
 
 struct DenseParams {
@@ -286,9 +204,24 @@ struct DenseParams {
   // kEpiAccumDense: out[row][col] (row stride N)
   float* out;
   int* status;
+  int a_mn, b_mn;      // 1: the operand is MN-major in memory (see DenseMaps)
 };
 
-constexpr int kGemmThreads = 256;  // warp 0: TMA producer, warp 1: MMA + TMEM, warps 4-7: epilogue
+constexpr int kGemmThreads = 256;
+
+// Shared-memory descriptor of an MN-major bf16 tile in the canonical 128-byte-swizzle layout
+// as 2-D TMA writes it from boxes of 64 (M or N) x 64 (K): within a box, K row r holds 64
+// consecutive M/N elements at r * 128 bytes (16-byte chunks XOR-swizzled by r mod 8), so
+// groups of 8 K rows are 1024 bytes apart (stride byte offset); consecutive boxes, i.e. the
+// next 64 M/N elements, are 8192 bytes apart (leading byte offset). Advancing K by 16 rows
+// adds 2048 bytes to the start address.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu)     // start address, bits [0,14)
+         | (static_cast<uint64_t>(8192 >> 4) << 16)          // leading byte offset: next 64 M/N
+         | (static_cast<uint64_t>(1024 >> 4) << 32)          // stride byte offset: next 8 K rows
+         | (static_cast<uint64_t>(1) << 46)                  // descriptor version for sm_100
+         | (static_cast<uint64_t>(2) << 61);                 // layout: 128-byte swizzle
+}  // warp 0: TMA producer, warp 1: MMA + TMEM, warps 4-7: epilogue
 
 template <int BN, int STAGES>
 struct DenseSmem {
@@ -373,8 +306,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), L::kStageBytes);
-          tma_load_2d(a_tile(stage), &maps.A, kb * kBK, m_blk * kBM, full_bar(stage), pol);
-          tma_load_2d(b_tile(stage), &maps.B, kb * kBK, n_blk * BN, full_bar(stage), pol);
+          if (p.a_mn) {
+#pragma unroll
+            for (int j = 0; j < kBM / 64; ++j)
+              tma_load_2d(a_tile(stage) + j * 8192, &maps.A, m_blk * kBM + j * 64, kb * kBK, full_bar(stage), pol);
+          } else {
+            tma_load_2d(a_tile(stage), &maps.A, kb * kBK, m_blk * kBM, full_bar(stage), pol);
+          }
+          if (p.b_mn) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(b_tile(stage) + j * 8192, &maps.B, n_blk * BN + j * 64, kb * kBK, full_bar(stage), pol);
+          } else {
+            tma_load_2d(b_tile(stage), &maps.B, kb * kBK, n_blk * BN, full_bar(stage), pol);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -382,7 +327,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN);
+      // operand majors: bit 15 (A), bit 16 (B) of the instruction descriptor, 1 = MN-major
+      const uint32_t idesc = umma_idesc_bf16(kBM, BN) | (p.a_mn ? 1u << 15 : 0u) | (p.b_mn ? 1u << 16 : 0u);
+      const uint32_t a_step = p.a_mn ? 2048u >> 4 : 32u >> 4;  // K += 16 in the descriptor's address field
+      const uint32_t b_step = p.b_mn ? 2048u >> 4 : 32u >> 4;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -398,11 +346,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = sw128_kmajor_desc(a_tile(stage));
-          const uint64_t bdesc = sw128_kmajor_desc(b_tile(stage));
+          const uint64_t adesc = p.a_mn ? sw128_mnmajor_desc(a_tile(stage)) : sw128_kmajor_desc(a_tile(stage));
+          const uint64_t bdesc = p.b_mn ? sw128_mnmajor_desc(b_tile(stage)) : sw128_kmajor_desc(b_tile(stage));
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb > kb0 || k != 0) ? 1u : 0u);
+            umma_bf16(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, (kb > kb0 || k != 0) ? 1u : 0u);
           umma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }

@@ -325,20 +325,21 @@ bool use_pair_wide(const ngram_embed_plan* p, int64_t T, bool count_on_device = 
 
 
 // ---- backward -------------------------------------------------------------------------
-// Workspace: the head (status word, ...), then W^T [D x D], g^T [D x T8] and G^T [D x T8]
-// bf16 (T8 = T rounded up to 8, zero-filled), each 256-byte aligned.
+// Workspace: the head (status word, ...), then G [T x D] bf16 (the concatenated sub-rows of
+// every token, the B operand of dW), then the dE0 sort buffers, each 256-byte aligned.
 constexpr int kBwdStages = 4;  // x (16 KB A + BN x 128 B B)
 
-int64_t pad8(int64_t T) { return (T + 7) & ~int64_t(7); }
 size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
 // dE0's counting sort: counts [V0 + 1], cursor [V0], order [T], sorted ids [T] (int32).
 size_t bwd_sort_bytes(const ngram_embed_plan* p, int64_t T) {
   return round256((static_cast<size_t>(p->V0) + 1) * 4) + round256(static_cast<size_t>(p->V0) * 4) +
          2 * round256(static_cast<size_t>(T) * 4) + round256((static_cast<size_t>(p->V0) + 1023) / 1024 * 4);
 }
+size_t bwd_g_bytes(const ngram_embed_plan* p, int64_t T) {
+  return round256(static_cast<size_t>(T) * static_cast<size_t>(p->D) * 2);
+}
 size_t bwd_ws_bytes(const ngram_embed_plan* p, int64_t T) {
-  const size_t D = static_cast<size_t>(p->D);
-  return kHeadBytes + round256(D * D * 2) + 2 * round256(D * static_cast<size_t>(pad8(T)) * 2) + bwd_sort_bytes(p, T);
+  return kHeadBytes + bwd_g_bytes(p, T) + bwd_sort_bytes(p, T);
 }
 
 // Split-K factor for a GEMM of `tiles` output tiles and KB k-blocks: the one, up to KB / 16
@@ -360,9 +361,17 @@ int choose_splits(int tiles, int KB, int sms) {
   return best;
 }
 
+// A GEMM operand as it lies in memory: K-major ([rows x K], rows K elements apart) or
+// MN-major ([K x rows], K rows of `rows` elements).
+struct GemmOperand {
+  const void* base;
+  int64_t rows;  // M (A) or N (B)
+  bool mn;
+};
+
 template <int BN>
-int launch_dense_gemm(ngram_embed_plan* p, DenseParams prm, const void* A, int64_t a_rows, const void* B,
-                      int64_t b_rows, int64_t K, int64_t row_elems, bool split, cudaStream_t st) {
+int launch_dense_gemm(ngram_embed_plan* p, DenseParams prm, GemmOperand A, GemmOperand B, int64_t K, bool split,
+                      cudaStream_t st) {
   using L = DenseSmem<BN, kBwdStages>;
   auto kern = dense_gemm_sm100_kernel<BN, kBwdStages>;
   const int key = BN == 256 ? 10 : 11;
@@ -371,17 +380,22 @@ int launch_dense_gemm(ngram_embed_plan* p, DenseParams prm, const void* A, int64
       return NGRAM_ERR_CUDA;
     p->smem_attr_set[key] = true;
   }
+  auto encode = [&](CUtensorMap* m, const GemmOperand& o, uint32_t box_rows) {
+    return o.mn ? encode_2d(m, o.base, static_cast<uint64_t>(o.rows), static_cast<uint64_t>(K),
+                            static_cast<uint64_t>(o.rows) * 2, 64, 64, CU_TENSOR_MAP_L2_PROMOTION_L2_256B)
+                : encode_2d(m, o.base, static_cast<uint64_t>(K), static_cast<uint64_t>(o.rows),
+                            static_cast<uint64_t>(K) * 2, kBK, box_rows, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  };
   DenseMaps maps;
-  int rc = encode_2d(&maps.A, A, static_cast<uint64_t>(row_elems), static_cast<uint64_t>(a_rows),
-                     static_cast<uint64_t>(row_elems) * 2, kBK, kBM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  int rc = encode(&maps.A, A, kBM);
   if (rc) return rc;
-  rc = encode_2d(&maps.B, B, static_cast<uint64_t>(row_elems), static_cast<uint64_t>(b_rows),
-                 static_cast<uint64_t>(row_elems) * 2, kBK, BN, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
-  if (rc) return rc;
-  prm.M = static_cast<int>(a_rows);
-  prm.N = static_cast<int>(b_rows);
-  prm.num_m_blocks = static_cast<int>((a_rows + kBM - 1) / kBM);
-  prm.num_n_blocks = static_cast<int>(b_rows / BN);
+  if ((rc = encode(&maps.B, B, BN))) return rc;
+  prm.a_mn = A.mn ? 1 : 0;
+  prm.b_mn = B.mn ? 1 : 0;
+  prm.M = static_cast<int>(A.rows);
+  prm.N = static_cast<int>(B.rows);
+  prm.num_m_blocks = static_cast<int>((A.rows + kBM - 1) / kBM);
+  prm.num_n_blocks = static_cast<int>(B.rows / BN);
   prm.num_k_blocks = static_cast<int>((K + kBK - 1) / kBK);
   const int tiles = prm.num_m_blocks * prm.num_n_blocks;
   const int sms = p->sms > 0 ? p->sms : 1;
@@ -1050,17 +1064,15 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
   int rc = set_device(p);
   if (rc) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t T = num_tokens, T8 = pad8(T);
+  const int64_t T = num_tokens;
   const int D = p->D;
   uint8_t* base = static_cast<uint8_t*>(workspace);
-  uint16_t* Wt = reinterpret_cast<uint16_t*>(base + kHeadBytes);
-  uint16_t* gT = reinterpret_cast<uint16_t*>(base + kHeadBytes + round256(size_t(D) * D * 2));
-  uint16_t* GT = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(gT) + round256(size_t(D) * T8 * 2));
+  uint16_t* G = reinterpret_cast<uint16_t*>(base + kHeadBytes);
   const float scale = p->out_scale / static_cast<float>(p->S + 1);
   const auto* g = static_cast<const uint16_t*>(grad_out);
 
   if (dE0) {
-    uint8_t* sort = reinterpret_cast<uint8_t*>(GT) + round256(size_t(D) * T8 * 2);
+    uint8_t* sort = base + kHeadBytes + bwd_g_bytes(p, T);
     ScatterE0Params e{};
     e.tokens = tokens;
     e.g = g;
@@ -1090,15 +1102,8 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
       return rc;
   }
   if (dE_nk) {
-    // dG = c g W_stacked, i.e. A = g [T x D] and B = W^T [D x D] (both K-major over D);
-    // the epilogue adds each 32-column piece into its sub-table's gradient row.
-    TransposeParams tp{};
-    tp.src = static_cast<const uint16_t*>(W_stacked);
-    tp.dst = Wt;
-    tp.R = D;
-    tp.R_pad = D;
-    tp.C = D;
-    if ((rc = launch(transpose_bf16_kernel, dim3(D / kTT, D / kTT), dim3(256), 0, st, p->pdl, 1, tp))) return rc;
+    // dG = c g W_stacked: A = g [T x D] (K-major over D), B[n][k] = W_stacked[k][n] (W as it
+    // lies: MN-major); the epilogue adds each 32-column piece into its sub-table's gradient row.
     DenseParams dp{};
     dp.scale = scale;
     dp.epi = kEpiScatterSub;
@@ -1110,45 +1115,24 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     dp.S = p->S;
     dp.d = p->d;
     dp.status = status_ptr(workspace);
-    if ((rc = p->D % 256 == 0 ? launch_dense_gemm<256>(p, dp, g, T, Wt, D, D, D, false, st)
-                              : launch_dense_gemm<128>(p, dp, g, T, Wt, D, D, D, false, st)))
+    const GemmOperand A{g, T, false}, B{W_stacked, D, true};
+    if ((rc = p->D % 256 == 0 ? launch_dense_gemm<256>(p, dp, A, B, D, false, st)
+                              : launch_dense_gemm<128>(p, dp, A, B, D, false, st)))
       return rc;
   }
   if (dW) {
-    // dW += c g^T G: A = g^T [D x T8] and B = G^T [D x T8] (K-major over tokens), split-K
-    // units adding into dW.
-    TransposeParams tp{};
-    tp.src = g;
-    tp.dst = gT;
-    tp.R = T;
-    tp.R_pad = T8;
-    tp.C = D;
-    if ((rc = launch(transpose_bf16_kernel, dim3(static_cast<unsigned>((T8 + kTT - 1) / kTT), D / kTT), dim3(256), 0,
-                     st, p->pdl, 1, tp)))
-      return rc;
-    GatherTParams gp{};
-    gp.idx = idx;
-    for (int s = 0; s < p->S; ++s) {
-      gp.E[s] = static_cast<const uint16_t*>(E_nk[s]);
-      gp.Vs[s] = static_cast<uint32_t>(p->V[s]);
-    }
-    gp.dst = GT;
-    gp.T = T;
-    gp.T_pad = T8;
-    gp.S = p->S;
-    gp.d = p->d;
-    gp.D = D;
-    gp.status = status_ptr(workspace);
-    if ((rc = launch(gather_transpose_kernel, dim3(static_cast<unsigned>((T8 + kTT - 1) / kTT), D / kTT), dim3(256),
-                     0, st, p->pdl, 1, gp)))
-      return rc;
+    // dW += c g^T G: A[m][t] = g[t][m] and B[n][t] = G[t][n], both MN-major as they lie
+    // (G gathered row by row into the workspace first), K = T with split-K units adding
+    // into dW.
+    if ((rc = launch_gather(p, idx, T, E_nk, G, nullptr, nullptr, nullptr, workspace, st))) return rc;
     DenseParams dp{};
     dp.scale = scale;
     dp.epi = kEpiAccumDense;
     dp.out = dW;
     dp.status = status_ptr(workspace);
-    if ((rc = p->D % 256 == 0 ? launch_dense_gemm<256>(p, dp, gT, D, GT, D, T8, T8, true, st)
-                              : launch_dense_gemm<128>(p, dp, gT, D, GT, D, T8, T8, true, st)))
+    const GemmOperand A{g, D, true}, B{G, D, true};
+    if ((rc = p->D % 256 == 0 ? launch_dense_gemm<256>(p, dp, A, B, T, true, st)
+                              : launch_dense_gemm<128>(p, dp, A, B, T, true, st)))
       return rc;
   }
   return NGRAM_OK;

@@ -273,8 +273,11 @@ int ngram_embed_fwd_draft(const ngram_embed_plan* plan, const int32_t* tokens,
  * dW may be NULL to skip that gradient; W_stacked is needed for dE_nk, E_nk for dW.
  * bf16 tensor-core plans only (else NGRAM_ERR_UNSUPPORTED). Index values outside
  * [0, V_nk) read/write row 0 and set NGRAM_STATUS_BAD_TOKEN.
- *   workspace  >= ngram_embed_bwd_workspace_bytes(plan, num_tokens): W^T and the transposed
- *              g and G (about 4 D num_tokens + 2 D^2 bytes); its head is the status word */
+ *   workspace  >= ngram_embed_bwd_workspace_bytes(plan, num_tokens): G, the gathered
+ *              sub-rows [num_tokens x D] bf16, and the dE0 sort buffers (about
+ *              2 D num_tokens + 8 V0 + 8 num_tokens bytes); its head is the status word.
+ * The GEMMs read g and W_stacked where they lie (the tensor cores take the operands that are
+ * not K-major in memory as MN-major tiles): nothing is transposed. */
 size_t ngram_embed_bwd_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens);
 int ngram_embed_bwd(const ngram_embed_plan* plan, const int32_t* tokens, const int32_t* idx,
                     int64_t num_tokens, const void* const* E_nk, const void* W_stacked,
