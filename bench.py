@@ -289,9 +289,10 @@ def events(n):
 
 
 def kernel_of_form(form: str) -> str:
-    return {"cta_pair": "proj_sm100_pair_kernel", "cta_pair_wide": "proj_sm100_pair_kernel",
-            "cta_pair_stream_k": "proj_sm100_pair_kernel", "one_cta": "proj_sm100_kernel",
-            "one_cta_stream_k": "proj_sm100_kernel", "cuda_cores": "proj_simt_kernel"}[form]
+    if form.startswith("cta_pair"):
+        return "proj_sm100_pair_kernel"
+    return {"one_cta": "proj_sm100_kernel", "one_cta_stream_k": "proj_sm100_kernel",
+            "cuda_cores": "proj_simt_kernel"}[form]
 
 
 # ------------------------------------------------------------------ prefill

@@ -322,7 +322,8 @@ def ngram_hash_stats(V0: int, n: int, tokens, seq_offsets, moduli, workspace=Non
 
 
 KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair", 4: "cta_pair_wide",
-                5: "cta_pair_stream_k", 6: "cta_pair_dense", 7: "cta_pair_dense_stream_k", 8: "cta_pair_wide_dense"}
+                5: "cta_pair_stream_k", 6: "cta_pair_dense", 7: "cta_pair_dense_stream_k", 8: "cta_pair_wide_dense",
+                9: "cta_pair_wide_stream_k"}
 
 
 def ngram_embed_plan_set_dense_a(plan: "Plan", mode: int):

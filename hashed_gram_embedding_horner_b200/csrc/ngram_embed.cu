@@ -72,7 +72,7 @@ struct ngram_embed_plan {
   int dense_a = 0;             // sub-rows gathered into G first, A by dense TMA: 1 on, 0 off
   const void* map_A = nullptr;  // the dense-A map's pointer and row count
   int64_t map_A_T = -1;
-  int max_clusters[3] = {0, 0, 0};  // co-resident CTA pairs, per tile width (0 = not queried)
+  int max_clusters[4] = {0, 0, 0, 0};  // co-resident CTA pairs, per kernel instance (0 = not queried)
 };
 
 namespace {
@@ -101,9 +101,12 @@ size_t ws_base(const ngram_embed_plan* p, int64_t T) {
   const size_t idx = static_cast<size_t>(T) * static_cast<size_t>(p->S) * sizeof(int32_t);
   return kHeadBytes + ((idx + 255) & ~size_t(255));
 }
-// Stream-K fp32 partial tiles: two 128 x 256 slots per SM.
+// Whether the plan's shape admits the CTA-pair form's 512-column tiles (256-column W halves).
+bool wide_capable(const ngram_embed_plan* p) { return p->tc_ok && p->bn == 256 && p->D % 512 == 0; }
+// Stream-K fp32 partial tiles: two slots per SM of 128 rows x the widest tile a stream-K
+// schedule of the plan can split (512 columns where the 512-column pair tiles apply, else 256).
 size_t sk_partial_bytes(const ngram_embed_plan* p) {
-  return p->tc_ok ? size_t(2) * static_cast<size_t>(p->sms) * kBM * 256 * sizeof(float) : 0;
+  return p->tc_ok ? size_t(2) * static_cast<size_t>(p->sms) * kBM * (wide_capable(p) ? 512 : 256) * sizeof(float) : 0;
 }
 // The dense-A form: the call's sub-rows gathered into G [T x D] bf16 first (a stand-alone
 // gather kernel with every resident thread copying), then the CTA-pair projection reads A as
@@ -261,12 +264,13 @@ bool use_pair_stream_k(const ngram_embed_plan* p, int64_t T, size_t ws_size, int
   return ws_size >= ws_base(p, ws_T) + sk_partial_bytes(p);
 }
 
-// CTA-pair kernel: clusters of two CTAs, one 256 x BN tile per pair per step.
-template <int BN, int kStg>
+// CTA-pair kernel: clusters of two CTAs, one 256 x BN tile per pair per step (WSK: the
+// 512-column tiles' stream-K instance).
+template <int BN, int kStg, bool WSK = false>
 int launch_tc_pair_stages(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaStream_t st, int key) {
   using L = PairSmem<BN, kStg>;
   static_assert(L::kLaunchBytes <= 232448, "CTA-pair kernel stages exceed 227 KB of shared memory");
-  auto kern = proj_sm100_pair_kernel<BN, kStg>;
+  auto kern = proj_sm100_pair_kernel<BN, kStg, WSK>;
   if (!p->smem_attr_set[key]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
@@ -286,7 +290,7 @@ int launch_tc_pair_stages(ngram_embed_plan* p, ProjParams prm, int64_t T, cudaSt
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int& max_pairs = p->max_clusters[BN == 512 ? 2 : (BN == 256 ? 1 : 0)];
+  int& max_pairs = p->max_clusters[WSK ? 3 : (BN == 512 ? 2 : (BN == 256 ? 1 : 0))];
   if (max_pairs == 0) {
     cfg.gridDim = dim3(2 * (p->sms / 2));
     int n = 0;
@@ -323,6 +327,25 @@ bool use_pair_wide(const ngram_embed_plan* p, int64_t T, bool count_on_device = 
   return static_cast<double>(waves_wide) <= 0.57 * static_cast<double>(waves_narrow);
 }
 
+
+// Stream-K for the pair form's 512-column tiles: where whole tiles would leave pairs idle
+// (fewer tiles than pairs, or a thin last wave: a 1280-token decode step at D = 4096 has 40
+// tiles for 74 pairs) and every pair still covers at least half a tile (so a tile is split
+// into a few pieces, not many). These tiles move the fewest bytes per FLOP from L2 into
+// shared memory (48 KB per pair-SM and k-block for 8.4 MFLOP), the limit at this shape.
+// Needs the workspace's partial tiles and 16 arrival counters per tile (row quarter x
+// column group, per CTA of the pair).
+bool use_wide_stream_k(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws_T) {
+  if (!wide_capable(p) || p->stream_k == 2 || p->pair_wide == 0 || p->cta_pair == 0 || p->sms < 2) return false;
+  const int64_t pairs = p->sms / 2;
+  const int64_t tiles = (T + 2 * kBM - 1) / (2 * kBM) * (p->D / 512);
+  const int64_t units = tiles * (p->D / kBK);
+  if (tiles * 16 > static_cast<int64_t>(kSkMaxTiles) * 4 || units < pairs || 2 * tiles < pairs) return false;
+  if (ws_size < ws_base(p, ws_T) + sk_partial_bytes(p)) return false;
+  if (p->stream_k == 1) return true;
+  const int64_t waves = (tiles + pairs - 1) / pairs;
+  return 1.3 * static_cast<double>(tiles) < static_cast<double>(waves * pairs);
+}
 
 // ---- backward -------------------------------------------------------------------------
 // Workspace: the head (status word, ...), then G [T x D] bf16 (the concatenated sub-rows of
@@ -509,6 +532,7 @@ enum Form : int {
   kFormDense = 6,      // rows gathered into G first; CTA pairs, 256 x 256 tiles, A by dense TMA
   kFormDenseSk = 7,    // the same with the pairs' stream-K schedule
   kFormDenseWide = 8,  // the same with 256 x 512 tiles
+  kFormPairWideSk = 9, // CTA pairs, 256 x 512 tiles, stream-K, fused row gather
 };
 
 // Stream-K for the dense-A pair form: where a grid of whole 256 x 256 tiles would take two or
@@ -545,6 +569,7 @@ int choose_form(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws
   prm.num_n_blocks = p->D / p->bn;
   prm.num_k_blocks = p->D / kBK;
   const bool psk = !count_on_device && p->cta_pair != 0 && p->pair_wide != 1 && use_pair_stream_k(p, T, ws_size, ws_T);
+  if (!psk && !count_on_device && use_wide_stream_k(p, T, ws_size, ws_T)) return kFormPairWideSk;
   const bool sk = !psk && !count_on_device && p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
   const bool pair = p->cta_pair == 1 || (p->cta_pair == -1 && !sk);
   if (pair) return psk ? kFormPairSk : (use_pair_wide(p, T, count_on_device) ? kFormPairWide : kFormPair);
@@ -650,6 +675,12 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
     }
     if (form == kFormDenseSk) stream_k_buffers();
     return launch_tc_pair<256>(p, prm, T, st);
+  }
+  if (form == kFormPairWideSk) {
+    prm.num_n_blocks = p->D / 512;
+    prm.tma_rows = kBM;  // A rows by gather4 only
+    stream_k_buffers();
+    return launch_tc_pair_stages<512, kPairStagesWide, true>(p, prm, T, st, 9);
   }
   const bool pair = form == kFormPair || form == kFormPairWide || form == kFormPairSk;
   // A rows by TMA gather4 in the pair form, by cp.async in the one-CTA form (measured

@@ -50,7 +50,8 @@ constexpr int kPairStagesWide = 4;  // BN = 512: 16 KB of A + 32 KB of W per sta
 // takes all 512 TMEM columns. Eight epilogue warps (12-15 and 4-7; the A rows come by
 // gather4 from warps 0-3) drain half 0 first and free it on its own barrier, then half 1,
 // and the next tile's half-0 MMAs start on the loaded stages as soon as half 0 is free.
-// Stream-K (BN = 256, on request): as in the one-CTA kernel, over pairs instead of CTAs.
+// Stream-K: as in the one-CTA kernel, over pairs instead of CTAs; for 256-column tiles on
+// request, for 512-column tiles where whole tiles would leave pairs idle (a decode step).
 template <int BN, int STAGES>
 struct PairSmem {
   static constexpr bool kWide = BN > 256;
@@ -200,7 +201,164 @@ __device__ __noinline__ bool pair_sk_piece(const ProjParams& p, const PairPiece 
   return true;
 }
 
-template <int BN, int STAGES>
+// One stream-K piece of a 256 x 512 pair tile (the 512-column form): this warp's 32 rows
+// (TMEM lane quarter q) and its 256 columns (columns g*128 .. +127 of each accumulator half),
+// with an arrival counter per (tile, CTA rank, row quarter, column group). As pair_sk_piece,
+// but the warp waits for both accumulator halves, and the finished sum of a 32-column chunk
+// goes out through the warp's shared-memory staging area like a whole tile's (four lanes per
+// row read it back, add E_0, scale and store 64-byte row segments). Partial slots hold
+// 128 x 512 fp32. Returns false if the accumulator never became ready (abort).
+struct WidePiece {
+  Seg sg;
+  uint32_t use;
+  int64_t T, units_total;
+  int KB, grid, pair, q, g, lane;
+  uint32_t rank, tmem_base;
+  uint32_t tfull0, tfull1, tempty0, tempty1;  // tempty: CTA 0's barriers (cluster addresses on CTA 1)
+  uint32_t row_w, rd_lo, rd_hi;                // this warp's staging addresses (see the epilogue)
+  volatile int* abort_flag;
+};
+
+__device__ __noinline__ bool pair_sk_piece_wide(const ProjParams& p, const WidePiece a) {
+  constexpr int kCols = 512;
+  const int tile = a.sg.tile;
+  const int m_blk = tile / p.num_n_blocks;
+  const int n_blk = tile % p.num_n_blocks;
+  const int row_in_tile = a.q * 32 + a.lane;
+  for (int h = 0; h < 2; ++h) {
+    bool got = false;
+    if (a.lane == 0) got = mbar_wait_cluster(h ? a.tfull1 : a.tfull0, a.use & 1u, a.abort_flag, p.status);
+    if (!__shfl_sync(0xffffffffu, got, 0)) return false;
+  }
+  tc_fence_after();
+  const uint32_t tlane = a.tmem_base + (static_cast<uint32_t>(a.q * 32) << 16);
+  // chunk c (0..7) of this warp: tile column (= accumulator column) (c / 4) * 256 + g * 128 + (c % 4) * 32
+  auto chunk_col = [&](int c) { return (c >> 2) * 256 + a.g * 128 + (c & 3) * 32; };
+  const int64_t u_tile = static_cast<int64_t>(tile) * a.KB;
+  const int c_lo = sk_cta_of(u_tile, a.units_total, a.grid), c_hi = sk_cta_of(u_tile + a.KB - 1, a.units_total, a.grid);
+  const int others = c_hi - c_lo;  // pieces of the tile besides this one
+  int* cnt = p.sk_counters + ((tile * 2 + static_cast<int>(a.rank)) * 4 + a.q) * 2 + a.g;
+  // partial slots: [pair][rank][slot] x (128 rows x 512 columns), column-group major
+  auto slot_of = [&](int pr, int sl) {
+    return reinterpret_cast<float4*>(p.sk_partials) +
+           ((static_cast<size_t>(pr) * 2 + a.rank) * 2 + sl) * (kBM * kCols / 4) + row_in_tile;
+  };
+  int fin = 0;
+  if (a.lane == 0) fin = ld_acquire_gpu(cnt) == others;
+  fin = __shfl_sync(0xffffffffu, fin, 0);
+  if (!fin) {
+    // slot 0: the piece that starts this pair's unit range; slot 1: the one that ends it
+    float4* mine = slot_of(a.pair, (u_tile + a.sg.i0 == sk_first_unit(a.units_total, a.grid, a.pair)) ? 0 : 1);
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      const int col = chunk_col(c);
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tlane + col, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int w = 0; w < 8; ++w)  // a warp's store is 512 contiguous bytes
+        mine[((col >> 5) * 8 + w) * kBM] = make_float4(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1]),
+                                                      __uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3]));
+    }
+    __threadfence();
+    __syncwarp();
+    if (a.lane == 0) fin = atomicAdd(cnt, 1) == others;
+    fin = __shfl_sync(0xffffffffu, fin, 0);
+    if (fin) __threadfence();
+  }
+  if (fin) {
+    const int rsub = a.lane >> 2, u2 = a.lane & 3;  // read-back: rows i*8 + rsub, columns u2*8 .. +7
+    const int col0 = n_blk * kCols;
+    const int64_t row0 = static_cast<int64_t>(m_blk) * (2 * kBM) + a.rank * kBM + a.q * 32;
+    const uint16_t* e0row[4];
+    bool valid[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t gr = row0 + i * 8 + rsub;
+      valid[i] = gr < a.T;
+      uint32_t t = 0;
+      if (valid[i]) {
+        const int32_t tok = p.tokens[gr];
+        t = (tok >= 0 && static_cast<uint32_t>(tok) < p.V0) ? static_cast<uint32_t>(tok) : 0u;
+      }
+      e0row[i] = p.E0 + static_cast<int64_t>(t) * p.D + col0 + u2 * 8;
+    }
+    uint4* dst0 = reinterpret_cast<uint4*>(p.out + (row0 + rsub) * p.D + col0 + u2 * 8);
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      const int col = chunk_col(c);
+      // pieces in pair order, whoever finishes: those before this pair's, its own (TMEM),
+      // those after, so the bits do not depend on arrival order
+      float sum[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) sum[k] = 0.f;
+      auto add_piece = [&](int pr) {
+        const float4* part = slot_of(pr, sk_first_unit(a.units_total, a.grid, pr) >= u_tile ? 0 : 1);
+        float4 x[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) x[w] = __ldcg(part + ((col >> 5) * 8 + w) * kBM);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          sum[4 * w] += x[w].x;
+          sum[4 * w + 1] += x[w].y;
+          sum[4 * w + 2] += x[w].z;
+          sum[4 * w + 3] += x[w].w;
+        }
+      };
+      for (int pr = c_lo; pr < a.pair; ++pr) add_piece(pr);
+      {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tlane + col, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) sum[k] += __uint_as_float(v[k]);
+      }
+      for (int pr = a.pair + 1; pr <= c_hi; ++pr) add_piece(pr);
+      // stage the 32 x 32 chunk (row per lane), read it back four lanes per row
+#pragma unroll
+      for (int w = 0; w < 8; ++w)
+        st_shared_v4(a.row_w + (static_cast<uint32_t>(w ^ (a.lane & 7)) << 4),
+                     make_uint4(__float_as_uint(sum[4 * w]), __float_as_uint(sum[4 * w + 1]),
+                                __float_as_uint(sum[4 * w + 2]), __float_as_uint(sum[4 * w + 3])));
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 lo = ld_shared_v4(a.rd_lo + i * 8 * 128);
+        const uint4 hi = ld_shared_v4(a.rd_hi + i * 8 * 128);
+        if (valid[i]) {
+          const uint4 ev = __ldg(reinterpret_cast<const uint4*>(e0row[i] + col));
+          const float x[8] = {__uint_as_float(lo.x), __uint_as_float(lo.y), __uint_as_float(lo.z), __uint_as_float(lo.w),
+                              __uint_as_float(hi.x), __uint_as_float(hi.y), __uint_as_float(hi.z), __uint_as_float(hi.w)};
+          const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h)
+            o[h] = pack_bf16x2((x[2 * h] + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale,
+                               (x[2 * h + 1] + bf16_bits_to_float(ew[h] >> 16)) * p.scale);
+          dst0[static_cast<int64_t>(i) * p.D + col / 8] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      __syncwarp();  // the staging area is rewritten by the next chunk
+    }
+    if (a.lane == 0) *cnt = 0;  // the tile is done: zero again for the next launch
+  }
+  tc_fence_before();  // both halves read for the last time: the MMA may reuse them
+  if (a.rank == 0) {
+    mbar_arrive(a.tempty0);
+    mbar_arrive(a.tempty1);
+  } else {
+    __syncwarp();
+    if (a.lane == 0) {
+      mbar_arrive_remote(a.tempty0);
+      mbar_arrive_remote(a.tempty1);
+    }
+  }
+  return true;
+}
+
+// WSK: 512-column tiles under the stream-K schedule (a separate instance, so that the
+// whole-tile kernel of the prefill carries none of the piece code's registers).
+template <int BN, int STAGES, bool WSK = false>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_sm100_pair_kernel(const __grid_constant__ ProjMaps maps, const __grid_constant__ ProjParams p) {
   using L = PairSmem<BN, STAGES>;
@@ -226,8 +384,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
   constexpr bool kWide = L::kWide;
   constexpr int kMmaN = L::kMmaN;
-  // stream-K (256-column tiles only): the (tile, k-block) units split evenly over the pairs
-  const bool sk = !kWide && p.stream_k != 0;
+  // stream-K: the (tile, k-block) units split evenly over the pairs
+  const bool sk = (!L::kWide || WSK) && p.stream_k != 0;
   const bool dense = p.dense_a != 0;                                // A by 2-D TMA boxes of G
   const bool cp_rows = !kWide && !sk && !dense && p.tma_rows == 0;  // A rows by cp.async (else all by TMA gather4)
   if (threadIdx.x == 0) {
@@ -384,14 +542,15 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       bool ok = true;
       int local = 0;
       auto advance = [&](int& st, uint32_t& ph) { if (++st == STAGES) { st = 0; ph ^= 1u; } };
-      // the MMAs of half h (all of the tile when not wide) on stage st, k-block i of the tile
-      auto issue = [&](int st, int h, int i, uint32_t d_tmem) {
+      // the MMAs of half h (all of the tile when not wide) on stage st: k-block j of a segment
+      // of nj k-blocks (a segment starts a fresh sum)
+      auto issue = [&](int st, int h, int j, int nj, uint32_t d_tmem) {
         const uint64_t adesc = sw128_kmajor_desc(a_tile(st));
         const uint64_t bdesc = sw128_kmajor_desc(b_tile(st) + h * L::kBSubBytes);
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k)
-          umma_bf16_pair(d_tmem + h * kMmaN, adesc + 2u * k, bdesc + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
-        if (kWide && i + 1 == KB) {  // half h complete: its epilogue may start
+          umma_bf16_pair(d_tmem + h * kMmaN, adesc + 2u * k, bdesc + 2u * k, idesc, (j | k) != 0 ? 1u : 0u);
+        if (kWide && j + 1 == nj) {  // half h complete: its epilogue may start
           umma_commit_pair(map_to_cta(tfull_bar(h), 0));
           umma_commit_pair(map_to_cta(tfull_bar(h), 1));
         }
@@ -405,41 +564,42 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const int acc = kWide ? 0 : (local & 1);
         const uint32_t use = static_cast<uint32_t>(kWide ? local : local >> 1);
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        int i0 = g.i0;  // wide tiles are always whole (i0 = 0, i1 = KB)
+        const int nj = g.i1 - g.i0;  // k-blocks of this segment (the whole tile unless stream-K)
+        int j0 = 0;
         if (kWide) {
           // The epilogue frees half 0 of the previous tile first: the MMAs of half 0 run on
           // the stages already loaded while half 1 is still being drained; those stages'
           // half-1 MMAs (same per-element order) and releases follow once it is free.
-          const int pre = KB < STAGES ? KB : STAGES;
+          const int pre = nj < STAGES ? nj : STAGES;
           if (!mbar_wait_cluster(tempty_bar(0), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           int st = stage;
           uint32_t ph = phase;
-          for (int i = 0; i < pre; ++i) {
+          for (int j = 0; j < pre; ++j) {
             if (!mbar_wait_cluster(full_bar(st), ph, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            issue(st, 0, i, d_tmem);
+            issue(st, 0, j, nj, d_tmem);
             advance(st, ph);
           }
           if (!ok) break;
           if (!mbar_wait_cluster(tempty_bar(1), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
-          for (int i = 0; i < pre; ++i) {
-            issue(stage, 1, i, d_tmem);
+          for (int j = 0; j < pre; ++j) {
+            issue(stage, 1, j, nj, d_tmem);
             release(stage);
             advance(stage, phase);
           }
-          i0 = pre;
+          j0 = pre;
         } else {
           if (!mbar_wait_cluster(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
         }
-        for (int i = i0; i < g.i1; ++i) {
+        for (int j = j0; j < nj; ++j) {
           if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           if (cp_rows) fence_proxy_async_smem();  // this CTA's cp.async rows: generic proxy writes
 #pragma unroll
-          for (int h = 0; h < L::kHalves; ++h) issue(stage, h, i - g.i0, d_tmem);  // a segment starts a fresh sum
+          for (int h = 0; h < L::kHalves; ++h) issue(stage, h, j, nj, d_tmem);
           release(stage);
           advance(stage, phase);
         }
@@ -502,6 +662,31 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       const int n_blk = tile % p.num_n_blocks;
       const int acc = kWide ? 0 : (local & 1);
       const uint32_t use = static_cast<uint32_t>(kWide ? local : local >> 1);
+      if (WSK && kWide && (sg.i0 != 0 || sg.i1 != KB)) {
+        WidePiece pc;
+        pc.sg = sg;
+        pc.use = use;
+        pc.T = T;
+        pc.units_total = units_total;
+        pc.KB = KB;
+        pc.grid = wp.grid;
+        pc.pair = pair;
+        pc.q = q;
+        pc.g = g;
+        pc.lane = lane;
+        pc.rank = rank;
+        pc.tmem_base = tmem_base;
+        pc.tfull0 = tfull_bar(0);
+        pc.tfull1 = tfull_bar(1);
+        pc.tempty0 = rank == 0 ? tempty_bar(0) : tempty_remote0;
+        pc.tempty1 = rank == 0 ? tempty_bar(1) : tempty_remote1;
+        pc.row_w = row_w;
+        pc.rd_lo = rd_lo;
+        pc.rd_hi = rd_hi;
+        pc.abort_flag = abort_flag;
+        if (!pair_sk_piece_wide(p, pc)) break;
+        continue;
+      }
       if (!kWide && (sg.i0 != 0 || sg.i1 != KB)) {
         PairPiece pc;
         pc.sg = sg;

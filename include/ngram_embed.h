@@ -109,8 +109,9 @@ int ngram_embed_plan_destroy(ngram_embed_plan* plan);
 
 /* Device workspace bytes for calls of up to max_tokens tokens: a 33,024-byte head (the
  * status word, then the stream-K arrival counters), the [max_tokens x S] int32 index
- * buffer, then, for plans that use the tensor-core kernel, 2 x (SM count) x 128 x 256 fp32
- * stream-K partial tiles (the plan's SM count: see ngram_embed_plan_set_sm_count), then,
+ * buffer, then, for plans that use the tensor-core kernel, 2 x (SM count) x 128 x W fp32
+ * stream-K partial tiles, W = 512 where the 512-column pair tiles apply (D % 512 == 0, tile
+ * width 256), else 256 (the plan's SM count: see ngram_embed_plan_set_sm_count), then,
  * while the dense-A form is on (ngram_embed_plan_set_dense_a), the [max_tokens x D] bf16
  * G buffer, each region rounded up to 256 bytes. A workspace without
  * the partials or G (head + index buffer) is accepted too; the projection then takes the
@@ -369,18 +370,20 @@ int ngram_embed_plan_set_sm_count(ngram_embed_plan* plan, int sms);
  * and issues two tcgen05 MMAs of N = 256 on it (half the gathered rows per FLOP of the
  * 256-column tiles); the accumulator fills all 512 TMEM columns and each half is drained and
  * freed separately. Applies when the tile width is 256 and D % 512 == 0, with A rows by TMA
- * gather4. 1 = on, 0 = off, -1 (default) = automatic. A tuning knob: results agree within
- * the stated tolerance. NGRAM_ERR_INVALID_ARG for other values. */
+ * gather4. 1 = on, 0 = off, -1 (default) = automatic (with the stream-K schedule where whole
+ * tiles would leave pairs idle, see ngram_embed_plan_set_stream_k). A tuning knob: results
+ * agree within the stated tolerance. NGRAM_ERR_INVALID_ARG for other values. */
 int ngram_embed_plan_set_pair_wide(ngram_embed_plan* plan, int on);
 
 /* The projection kernel a call of num_tokens tokens would run, given a workspace of
  * ngram_embed_workspace_bytes(plan, num_tokens): 0 = CUDA cores, 1 = one CTA per tile,
  * 2 = one CTA per SM with the stream-K schedule, 3 = CTA pairs, 4 = CTA pairs with
- * 512-column tiles, 5 = CTA pairs with the stream-K schedule (these gather the A rows from
- * the sub-tables inside the projection); 6 = the call's sub-rows gathered into G first by a
- * stand-alone gather kernel, then CTA pairs reading A as dense TMA boxes of G, 7 = the same
- * with the pairs' stream-K schedule, 8 = the same with 512-column tiles (see
- * ngram_embed_plan_set_dense_a); negative on bad arguments. */
+ * 512-column tiles, 5 = CTA pairs with the stream-K schedule, 9 = CTA pairs with 512-column
+ * tiles and the stream-K schedule (these gather the A rows from the sub-tables inside the
+ * projection); 6 = the call's sub-rows gathered into G first by a stand-alone gather kernel,
+ * then CTA pairs reading A as dense TMA boxes of G, 7 = the same with the pairs' stream-K
+ * schedule, 8 = the same with 512-column tiles (see ngram_embed_plan_set_dense_a); negative
+ * on bad arguments. */
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens);
 
 /* Dense-A form of the tensor-core projection: the call's sub-rows are first copied into a
@@ -408,18 +411,19 @@ int ngram_embed_plan_set_tile_n(ngram_embed_plan* plan, int tile_n);
  * change. */
 int ngram_embed_plan_set_a_stages(ngram_embed_plan* plan, int stages);
 
-/* Schedule of the tensor-core kernels: 0 = automatic (the one-CTA form with stream-K when
- * its grid takes two or more waves of one tile per CTA and the last wave leaves many SMs
- * idle, e.g. 160 tiles of 128 x 256 on 148 SMs), 1 = stream-K whenever possible (for the
- * CTA-pair form too when ngram_embed_plan_set_cta_pair(plan, 1) also fixes that form and
- * the tiles are 256 columns wide), 2 = never. Stream-K gives every worker (a CTA, or a CTA
- * pair) an equal run of (tile, k-block) units; a tile split between workers is summed in
- * fp32, in worker order, by whichever finishes its piece last, so no worker waits for
- * another. It needs the workspace's partial tiles, at most 2048 one-CTA tiles (1024 pair
- * tiles) and at least one k-block per worker, and is not used with 512-column pair tiles or
- * when the token count is read on the device; otherwise the kernel takes one tile per
- * worker. A tuning knob: results agree within the stated tolerance (the summation order
- * differs). */
+/* Schedule of the tensor-core kernels: 0 = automatic, 1 = stream-K whenever possible (for
+ * the pairs' 256-column tiles only when ngram_embed_plan_set_cta_pair(plan, 1) also fixes
+ * the pair form and 512-column tiles are off), 2 = never. Stream-K gives every worker (a
+ * CTA, or a CTA pair) an equal run of (tile, k-block) units; a tile split between workers is
+ * summed in fp32, in worker order, by whichever finishes its piece last, so no worker waits
+ * for another. Automatic: the pairs' 512-column tiles under stream-K where whole tiles would
+ * leave pairs idle and every pair still covers at least half a tile (a 1280-token decode
+ * step at D = 4096: 40 tiles for 74 pairs); else the one-CTA form with stream-K when its
+ * grid takes two or more waves of one tile per CTA and the last wave leaves many SMs idle.
+ * It needs the workspace's partial tiles, at most 2048 one-CTA tiles (1024 pair tiles, 512
+ * 512-column tiles) and at least one k-block per worker, and is not used when the token
+ * count is read on the device; otherwise the kernel takes one tile per worker. A tuning
+ * knob: results agree within the stated tolerance (the summation order differs). */
 int ngram_embed_plan_set_stream_k(ngram_embed_plan* plan, int mode);
 
 /* 1 = launch every kernel of the plan as a programmatic dependent launch: it may be

@@ -144,10 +144,12 @@ V25 = (3342341, 3342371, 3342379, 3342413, 3342419, 3342439, 3342457, 3342473)
 @pytest.mark.parametrize("kw,T,sms,knobs,form", [
     (dict(), 32768, 148, {}, 4),                                  # prefill D = 2048: 512-column pair tiles
     (dict(D=4096, N=5, K=2, V=V25), 65536, 148, {}, 4),           # varlen prefill D = 4096
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {}, 2),            # decode step: one-CTA stream-K
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {}, 9),            # decode step: 40 wide tiles, stream-K
     (dict(D=4096, N=3, K=4, V=V25), 128, 148, {}, 3),             # one wave: 256-column pair tiles
-    (dict(D=4096, N=3, K=4, V=V25), 5120, 148, {}, 3),            # 160 wide tiles: a thin third wave
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 1}, 4),
+    (dict(D=4096, N=3, K=4, V=V25), 5120, 148, {}, 9),            # 160 wide tiles: a thin third wave
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"pair_wide": 0}, 2),  # without wide tiles: one-CTA stream-K
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"stream_k": 2}, 4),   # no stream-K: whole wide tiles
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 1}, 9),
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 1, "stream_k": 1}, 5),
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 0, "stream_k": 2}, 1),
     (dict(D=4096, N=3, K=4, V=V25), 1280, 40, {}, 4),             # 20 pairs: 40 wide tiles fill 2 waves
@@ -169,7 +171,8 @@ def test_kernel_form_choice_for_a_device_size(ne, kw, T, sms, knobs, form):
     assert rc == 0
     assert lib.ngram_embed_plan_set_sm_count(h, sms) == 0  # a B200 has 148: also valid on one
     setters = {"cta_pair": lib.ngram_embed_plan_set_cta_pair, "stream_k": lib.ngram_embed_plan_set_stream_k,
-               "tile_n": lib.ngram_embed_plan_set_tile_n, "dense_a": lib.ngram_embed_plan_set_dense_a}
+               "tile_n": lib.ngram_embed_plan_set_tile_n, "dense_a": lib.ngram_embed_plan_set_dense_a,
+               "pair_wide": lib.ngram_embed_plan_set_pair_wide}
     for k, v in knobs.items():
         assert setters[k](h, v) == 0
     assert lib.ngram_embed_plan_kernel_form(h, T) == form
@@ -177,8 +180,10 @@ def test_kernel_form_choice_for_a_device_size(ne, kw, T, sms, knobs, form):
 
 
 def test_sm_count_sizes_the_stream_k_workspace(ne):
-    """Two fp32 partial tiles of 128 x 256 per SM the plan uses; 0 restores the device's
-    count (none here: no partial tiles, no stream-K, no automatic 512-column tiles)."""
+    """Two fp32 partial tiles per SM the plan uses, of 128 x 512 (the widest tile its
+    stream-K schedules split: D = 2048 admits the 512-column pair tiles); 0 restores the
+    device's count (none here: no partial tiles, no stream-K, no automatic 512-column
+    tiles)."""
     import torch
     lib = ne._lib
     rc, h = _create(ne)
@@ -188,9 +193,9 @@ def test_sm_count_sizes_the_stream_k_workspace(ne):
     base = lib.ngram_embed_workspace_bytes(h, 1000)
     assert lib.ngram_embed_plan_set_sm_count(h, 1) == -1 and lib.ngram_embed_plan_set_sm_count(h, -3) == -1
     assert lib.ngram_embed_plan_set_sm_count(h, 148) == 0
-    assert lib.ngram_embed_workspace_bytes(h, 1000) == base + 2 * 148 * 128 * 256 * 4
+    assert lib.ngram_embed_workspace_bytes(h, 1000) == base + 2 * 148 * 128 * 512 * 4
     assert lib.ngram_embed_plan_set_sm_count(h, 40) == 0
-    assert lib.ngram_embed_workspace_bytes(h, 1000) == base + 2 * 40 * 128 * 256 * 4
+    assert lib.ngram_embed_workspace_bytes(h, 1000) == base + 2 * 40 * 128 * 512 * 4
     assert lib.ngram_embed_plan_kernel_form(h, 32768) == 4
     assert lib.ngram_embed_plan_set_sm_count(h, 0) == 0
     assert lib.ngram_embed_workspace_bytes(h, 1000) == base

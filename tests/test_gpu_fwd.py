@@ -215,14 +215,58 @@ def test_pair_stream_k_matches_oracle_and_is_repeatable(ne, shape):
     assert_close(to_host_f64(dp), want, what=f"{cfg.name} pair data-parallel")
 
 
-@pytest.mark.parametrize("pair", [0, 1])
+WSK_SHAPES = [((3000, 1024, 3, 2, 301), 6), ((5000, 2048, 3, 2, 301), 10), ((4000, 4096, 2, 2, 1280), 0),
+              ((5000, 1536, 4, 1, 77), 4)]
+
+
+@pytest.mark.parametrize("shape,sms", WSK_SHAPES, ids=lambda s: "V0%d_D%d_N%d_K%d_T%d" % s if isinstance(s, tuple)
+                         else f"sms{s}")
+def test_wide_stream_k_matches_oracle_and_is_repeatable(ne, shape, sms):
+    """CTA pairs with 512-column tiles under stream-K (pieces of a tile summed per row quarter
+    and column group by the last piece, through the epilogue's staging): a plan limited to a
+    few SMs splits the small shapes' tiles; the 1280-token D = 4096 shape takes this form by
+    itself. Parity with the oracle, repeatable bits, counters back at zero, and agreement
+    with whole 512-column tiles."""
+    V0, D, N, K, T = shape
+    cfg = small_cfg(V0, D, N, K, seed=9)
+    lengths = [T // 3, 0, T - T // 3 - 5, 5]
+    tokens, offsets = ragged_tokens(cfg, lengths)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = plan_for(ne, cfg)
+    if sms:
+        ne.ngram_embed_plan_set_sm_count(plan, sms)
+        ne.ngram_embed_plan_set_stream_k(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, T) == "cta_pair_wide_stream_k"
+    out = torch.full((T, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = ne.new_workspace(plan, T)
+    tk, of = dev_i32(tokens), dev_i32(offsets)
+    ne.ngram_embed_fwd(plan, tk, of, E0, E, W, out, ws)
+    assert ne.ngram_embed_get_status(ws) == 0
+    assert not ws[256:256 + 2048 * 16].any()  # every split tile's counters back at zero
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    assert_close(to_host_f64(out), want, what=f"{cfg.name} wide stream-K")
+    again = torch.full_like(out, float("nan"))
+    ne.ngram_embed_fwd(plan, tk, of, E0, E, W, again, ws)
+    assert ne.ngram_embed_get_status(ws) == 0 and torch.equal(out, again)
+    ne.ngram_embed_plan_set_stream_k(plan, 2)
+    ne.ngram_embed_plan_set_pair_wide(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, T) == "cta_pair_wide"
+    whole = torch.full_like(out, float("nan"))
+    ne.ngram_embed_fwd(plan, tk, of, E0, E, W, whole, ws)
+    assert ne.ngram_embed_get_status(ws) == 0
+    assert_close(to_host_f64(whole), want, what=f"{cfg.name} whole wide tiles")
+
+
+@pytest.mark.parametrize("pair", [0, 1, 2], ids=["one_cta", "pair", "pair_wide"])
 def test_stream_k_bit_exact_with_identity_w(ne, pair):
     """W = I and E_0 = 0 under stream-K (one-CTA or CTA-pair form): each output element gets
     one nonzero product, so the fp32 partials of a split tile add zeros to it and the
     result stays exact."""
     # S + 1 = 4: the scale is exact; one-CTA: 27 tiles of 128 x 128; pairs: 9 of 256 x 256
-    # (108 units of a k-block on 74 pairs)
-    cfg = small_cfg(7000, 1152 if pair == 0 else 768, 2, 3, seed=3)
+    # (108 units of a k-block on 74 pairs); wide: 9 of 256 x 512 on 3 pairs (72 units each)
+    cfg = small_cfg(7000, {0: 1152, 1: 768, 2: 1536}[pair], 2, 3, seed=3)
     S = cfg.S
     tokens, offsets = ragged_tokens(cfg, [5, 128, 200, 3] if pair == 0 else [5, 300, 400, 3])
     from tests.helpers import host_tables
@@ -230,12 +274,15 @@ def test_stream_k_bit_exact_with_identity_w(ne, pair):
     eye = gen.f32_to_bf16_bits(np.eye(cfg.D, dtype=np.float32))
     idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, oracle.context_windows(cfg.N, tokens, offsets))
     G = np.concatenate([gen.bf16_bits_to_f32(Eh[s][idx[:, s]]) for s in range(S)], axis=1)
-    plan = plan_for(ne, cfg, 2 if pair == 0 else 0, 128 if pair == 0 else 256, pair=pair)
+    plan = plan_for(ne, cfg, 2 if pair == 0 else 0, 128 if pair == 0 else 256, pair=min(pair, 1))
     if pair == 0:
         ne.ngram_embed_plan_set_tma_rows(plan, 0)
-    ne.ngram_embed_plan_set_pair_wide(plan, 0)
+    ne.ngram_embed_plan_set_pair_wide(plan, 1 if pair == 2 else 0)
+    if pair == 2:
+        ne.ngram_embed_plan_set_sm_count(plan, 6)
     ne.ngram_embed_plan_set_stream_k(plan, 1)
-    assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == ("one_cta_stream_k" if pair == 0 else "cta_pair_stream_k")
+    assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == \
+        ("one_cta_stream_k", "cta_pair_stream_k", "cta_pair_wide_stream_k")[pair]
     zeros0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.bfloat16, device="cuda")
     out, status = run_fwd(ne, plan, cfg, tokens, offsets, zeros0, [to_device(e, torch.bfloat16) for e in Eh],
                           to_device(eye, torch.bfloat16))
@@ -455,7 +502,8 @@ def test_reduced_sm_count_every_form(ne, sms):
     want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
     forms = set()
     for pair, wide, sk, dense in ((None, None, 0, 0), (1, 1, 0, 0), (1, 0, 1, 0), (1, 0, 2, 0), (0, 0, 1, 0),
-                                  (0, 0, 2, 0), (None, 0, 1, 1), (None, 0, 2, 1), (None, 1, 2, 1)):
+                                  (0, 0, 2, 0), (None, 0, 1, 1), (None, 0, 2, 1), (None, 1, 2, 1), (None, 1, 1, 0),
+                                  (1, 1, 2, 0)):
         plan = plan_for(ne, cfg, pair=pair)
         ne.ngram_embed_plan_set_sm_count(plan, sms)
         ne.ngram_embed_plan_set_pair_wide(plan, wide)
@@ -466,27 +514,31 @@ def test_reduced_sm_count_every_form(ne, sms):
         assert status == 0
         assert_close(to_host_f64(out), want, what=f"{sms} SMs, pair={pair} wide={wide} stream-K={sk} dense={dense}")
     assert {"cta_pair_wide", "cta_pair_stream_k", "cta_pair", "one_cta_stream_k", "one_cta", "cta_pair_dense",
-            "cta_pair_dense_stream_k", "cta_pair_wide_dense"} <= forms
+            "cta_pair_dense_stream_k", "cta_pair_wide_dense", "cta_pair_wide_stream_k"} <= forms
 
 
 def test_automatic_kernel_form(ne):
     """Prefill grids run the CTA-pair form with 512-column tiles; a 1280-token decode step at
-    D = 4096 (160 tiles of 128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule;
-    a grid of one wave keeps the 256-column pair tiles (more SMs busy). The pairs' stream-K
-    schedule is taken only when both the pair form and stream-K are asked for. With the
-    dense-A form on, the decode step runs it with the pairs' stream-K schedule."""
+    D = 4096 (40 such tiles for 74 pairs) runs them under the stream-K schedule; a grid of
+    one wave of 256-column tiles keeps those (more SMs busy than 8 wide tiles split many
+    ways). Without 512-column tiles the decode step runs the one-CTA form's stream-K
+    schedule; the pairs' 256-column stream-K is taken only when both the pair form and
+    stream-K are asked for. With the dense-A form on, the decode step runs it with the
+    pairs' stream-K schedule."""
     for cfg in (configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN):
         plan = plan_for(ne, cfg)
         assert ne.ngram_embed_plan_kernel_form(plan, 32768) == "cta_pair_wide"
     plan = plan_for(ne, configs.SPEC_DECODE)
-    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "one_cta_stream_k"
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_wide_stream_k"
     assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"  # one wave: nothing to balance
+    ne.ngram_embed_plan_set_pair_wide(plan, 0)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "one_cta_stream_k"
     ne.ngram_embed_plan_set_cta_pair(plan, 1)
-    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_wide"
     ne.ngram_embed_plan_set_stream_k(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_stream_k"
     ne.ngram_embed_plan_set_cta_pair(plan, None)
     ne.ngram_embed_plan_set_stream_k(plan, 0)
+    ne.ngram_embed_plan_set_pair_wide(plan, None)
     ne.ngram_embed_plan_set_dense_a(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_dense_stream_k"
     assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair_dense"

@@ -74,19 +74,21 @@ def _noalloc_cfg():
                                V_nk=tuple(configs.primes_from(20000, 8)), dtype="bf16", seed=5)
 
 
-@pytest.mark.parametrize("dense_a,form", [(0, "one_cta_stream_k"), (1, "cta_pair_dense_stream_k")])
-def test_static_workspace_stream_k_matches_fwd(ne, dense_a, form):
-    """With 8 SMs the stream-K partial tiles (2 x 8 x 128 KB) fit the fixed array, so the
+@pytest.mark.parametrize("dense_a,wide,form", [(0, 0, "one_cta_stream_k"), (1, -1, "cta_pair_dense_stream_k"),
+                                                (0, -1, "cta_pair_wide_stream_k")])
+def test_static_workspace_stream_k_matches_fwd(ne, dense_a, wide, form):
+    """With 6 SMs the stream-K partial tiles (2 x 6 x 256 KB) fit the fixed array, so the
     schedules whose arrival counters and partials (and, in the dense-A form, the gathered
-    sub-rows) live in it run; two calls in a row equal ngram_embed_fwd with its own workspace
-    (same schedule) bit for bit."""
+    sub-rows) live in it run, with tiles split between CTAs or pairs; two calls in a row
+    equal ngram_embed_fwd with its own workspace (same schedule) bit for bit."""
     cfg = _noalloc_cfg()
     E0h, Eh, Wh = host_tables(cfg)
     E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
     plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
-    ne.ngram_embed_plan_set_sm_count(plan, 8)
+    ne.ngram_embed_plan_set_sm_count(plan, 6)
     ne.ngram_embed_plan_set_stream_k(plan, 1)
     ne.ngram_embed_plan_set_dense_a(plan, dense_a)
+    ne.ngram_embed_plan_set_pair_wide(plan, wide)
     status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     for call, lengths in enumerate(([3, 330, 97], [129, 1, 0, 300])):
         off_h = gen.offsets_from_lengths(lengths)
