@@ -560,11 +560,21 @@ def run_decode(ne, cfg, tables, steps: int, warmup: int, dev, rank: int = 0, ext
     plain_ms = timed(lambda i, st: ne.ngram_embed_fwd(plan, tok_all[i], offsets, E0, E, W, out, ws, cache=cache,
                                                       stream=st))
     hit_rate = hits_d.item() / (T * (3 + 4 * n_k))  # timed(): 3 eager calls, then 1 + 3 replays of n_k
+    kernel = kernel_of_form(form)
+    traffic = profiled_traffic(kernel, cfg.name)
     res.update({
         "projection": {"ms": proj_ms, "tflops": flops / (proj_ms / 1e3) / 1e12,
                        "frac": flops / (proj_ms / 1e3) / 1e12 / pk["bf16_tflops"],
                        "what": "ngram_embed_project: " + ("sub-row gather into G + dense-A tcgen05 projection"
                                                           if dense else "fused row gather + tcgen05 projection")},
+        # the step's dominant kernel against both rooflines: its FLOPs at the bf16 peak, and the
+        # DRAM bytes an ncu capture of it moved (one launch at this shape) over its time here
+        "roofline": {"bound": "tensor", "kernel": kernel + " (" + form + ")", "kernel_ms": proj_ms,
+                     "achieved": flops / (proj_ms / 1e3) / 1e12, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": flops / (proj_ms / 1e3) / 1e12 / pk["bf16_tflops"], "traffic": traffic,
+                     "dram_gbs": None if traffic is None else traffic / (proj_ms / 1e3) / 1e9,
+                     "dram_frac_hbm": None if traffic is None else traffic / (proj_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                     "algorithmic_bytes": T * (2 * cfg.D * 2 + 4) + cfg.D * cfg.D * 2},
         "hash_ms": hash_ms,
         "gather_stage": {
             "what": ("gather_kernel, as the step runs it: the sub-rows copied into G" if dense else

@@ -328,23 +328,22 @@ bool use_pair_wide(const ngram_embed_plan* p, int64_t T, bool count_on_device = 
 }
 
 
-// Stream-K for the pair form's 512-column tiles: where whole tiles would leave pairs idle
-// (fewer tiles than pairs, or a thin last wave: a 1280-token decode step at D = 4096 has 40
-// tiles for 74 pairs) and every pair still covers at least half a tile (so a tile is split
-// into a few pieces, not many). These tiles move the fewest bytes per FLOP from L2 into
-// shared memory (48 KB per pair-SM and k-block for 8.4 MFLOP), the limit at this shape.
-// Needs the workspace's partial tiles and 16 arrival counters per tile (row quarter x
-// column group, per CTA of the pair).
+// Stream-K for the pair form's 512-column tiles: only when the plan asks for both the
+// 512-column tiles and stream-K (ngram_embed_plan_set_pair_wide(plan, 1) and
+// ngram_embed_plan_set_stream_k(plan, 1)). Measured on B200 at the 1280-token decode step
+// (D = 4096, 40 tiles for 74 pairs): 101 us a step against 71 us for the one-CTA form's
+// stream-K and 72 us for whole 512-column tiles. With one 512-column accumulator per CTA a
+// piece's epilogue (publishing or summing 256 KB of fp32 partials per CTA) cannot overlap
+// the MMAs of the pair's next piece, and each pair runs two pieces. Needs the workspace's
+// partial tiles and 16 arrival counters per tile (row quarter x column group, per CTA of
+// the pair), and at least half a tile per pair.
 bool use_wide_stream_k(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws_T) {
-  if (!wide_capable(p) || p->stream_k == 2 || p->pair_wide == 0 || p->cta_pair == 0 || p->sms < 2) return false;
+  if (!wide_capable(p) || p->stream_k != 1 || p->pair_wide != 1 || p->cta_pair == 0 || p->sms < 2) return false;
   const int64_t pairs = p->sms / 2;
   const int64_t tiles = (T + 2 * kBM - 1) / (2 * kBM) * (p->D / 512);
   const int64_t units = tiles * (p->D / kBK);
   if (tiles * 16 > static_cast<int64_t>(kSkMaxTiles) * 4 || units < pairs || 2 * tiles < pairs) return false;
-  if (ws_size < ws_base(p, ws_T) + sk_partial_bytes(p)) return false;
-  if (p->stream_k == 1) return true;
-  const int64_t waves = (tiles + pairs - 1) / pairs;
-  return 1.3 * static_cast<double>(tiles) < static_cast<double>(waves * pairs);
+  return ws_size >= ws_base(p, ws_T) + sk_partial_bytes(p);
 }
 
 // ---- backward -------------------------------------------------------------------------

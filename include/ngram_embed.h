@@ -370,9 +370,9 @@ int ngram_embed_plan_set_sm_count(ngram_embed_plan* plan, int sms);
  * and issues two tcgen05 MMAs of N = 256 on it (half the gathered rows per FLOP of the
  * 256-column tiles); the accumulator fills all 512 TMEM columns and each half is drained and
  * freed separately. Applies when the tile width is 256 and D % 512 == 0, with A rows by TMA
- * gather4. 1 = on, 0 = off, -1 (default) = automatic (with the stream-K schedule where whole
- * tiles would leave pairs idle, see ngram_embed_plan_set_stream_k). A tuning knob: results
- * agree within the stated tolerance. NGRAM_ERR_INVALID_ARG for other values. */
+ * gather4. 1 = on (with the stream-K schedule if ngram_embed_plan_set_stream_k(plan, 1)),
+ * 0 = off, -1 (default) = automatic. A tuning knob: results agree within the stated
+ * tolerance. NGRAM_ERR_INVALID_ARG for other values. */
 int ngram_embed_plan_set_pair_wide(ngram_embed_plan* plan, int on);
 
 /* The projection kernel a call of num_tokens tokens would run, given a workspace of
@@ -416,14 +416,16 @@ int ngram_embed_plan_set_a_stages(ngram_embed_plan* plan, int stages);
  * the pair form and 512-column tiles are off), 2 = never. Stream-K gives every worker (a
  * CTA, or a CTA pair) an equal run of (tile, k-block) units; a tile split between workers is
  * summed in fp32, in worker order, by whichever finishes its piece last, so no worker waits
- * for another. Automatic: the pairs' 512-column tiles under stream-K where whole tiles would
- * leave pairs idle and every pair still covers at least half a tile (a 1280-token decode
- * step at D = 4096: 40 tiles for 74 pairs); else the one-CTA form with stream-K when its
- * grid takes two or more waves of one tile per CTA and the last wave leaves many SMs idle.
+ * for another. Automatic: the one-CTA form with stream-K when its grid takes two or more
+ * waves of one tile per CTA and the last wave leaves many SMs idle (a 1280-token decode step
+ * at D = 4096). The pairs' 512-column tiles take it only when both are asked for
+ * (ngram_embed_plan_set_pair_wide(plan, 1) too; measured slower at the decode step: a
+ * piece's epilogue cannot overlap the next piece's MMAs with one 512-column accumulator).
  * It needs the workspace's partial tiles, at most 2048 one-CTA tiles (1024 pair tiles, 512
- * 512-column tiles) and at least one k-block per worker, and is not used when the token
- * count is read on the device; otherwise the kernel takes one tile per worker. A tuning
- * knob: results agree within the stated tolerance (the summation order differs). */
+ * 512-column tiles) and at least one k-block per worker (half a tile per pair for the
+ * 512-column tiles), and is not used when the token count is read on the device; otherwise
+ * the kernel takes one tile per worker. A tuning knob: results agree within the stated
+ * tolerance (the summation order differs). */
 int ngram_embed_plan_set_stream_k(ngram_embed_plan* plan, int mode);
 
 /* 1 = launch every kernel of the plan as a programmatic dependent launch: it may be

@@ -144,12 +144,15 @@ V25 = (3342341, 3342371, 3342379, 3342413, 3342419, 3342439, 3342457, 3342473)
 @pytest.mark.parametrize("kw,T,sms,knobs,form", [
     (dict(), 32768, 148, {}, 4),                                  # prefill D = 2048: 512-column pair tiles
     (dict(D=4096, N=5, K=2, V=V25), 65536, 148, {}, 4),           # varlen prefill D = 4096
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {}, 9),            # decode step: 40 wide tiles, stream-K
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {}, 2),            # decode step: one-CTA stream-K
     (dict(D=4096, N=3, K=4, V=V25), 128, 148, {}, 3),             # one wave: 256-column pair tiles
-    (dict(D=4096, N=3, K=4, V=V25), 5120, 148, {}, 9),            # 160 wide tiles: a thin third wave
+    (dict(D=4096, N=3, K=4, V=V25), 5120, 148, {}, 3),            # 160 wide tiles: a thin third wave
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"pair_wide": 0}, 2),  # without wide tiles: one-CTA stream-K
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"stream_k": 2}, 4),   # no stream-K: whole wide tiles
-    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 1}, 9),
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 1}, 4),
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"pair_wide": 1, "stream_k": 1}, 9),  # wide tiles, stream-K
+    (dict(D=4096, N=3, K=4, V=V25), 128, 148, {"pair_wide": 1, "stream_k": 1}, 2),   # 8 wide tiles: too few
+                                                                                     # to split; one-CTA stream-K
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 1, "stream_k": 1}, 5),
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 0, "stream_k": 2}, 1),
     (dict(D=4096, N=3, K=4, V=V25), 1280, 40, {}, 4),             # 20 pairs: 40 wide tiles fill 2 waves

@@ -224,9 +224,9 @@ WSK_SHAPES = [((3000, 1024, 3, 2, 301), 6), ((5000, 2048, 3, 2, 301), 10), ((400
 def test_wide_stream_k_matches_oracle_and_is_repeatable(ne, shape, sms):
     """CTA pairs with 512-column tiles under stream-K (pieces of a tile summed per row quarter
     and column group by the last piece, through the epilogue's staging): a plan limited to a
-    few SMs splits the small shapes' tiles; the 1280-token D = 4096 shape takes this form by
-    itself. Parity with the oracle, repeatable bits, counters back at zero, and agreement
-    with whole 512-column tiles."""
+    few SMs splits the small shapes' tiles; the 1280-token D = 4096 shape splits its 40
+    tiles over the device's pairs. Parity with the oracle, repeatable bits, counters back at
+    zero, and agreement with whole 512-column tiles."""
     V0, D, N, K, T = shape
     cfg = small_cfg(V0, D, N, K, seed=9)
     lengths = [T // 3, 0, T - T // 3 - 5, 5]
@@ -237,7 +237,8 @@ def test_wide_stream_k_matches_oracle_and_is_repeatable(ne, shape, sms):
     plan = plan_for(ne, cfg)
     if sms:
         ne.ngram_embed_plan_set_sm_count(plan, sms)
-        ne.ngram_embed_plan_set_stream_k(plan, 1)
+    ne.ngram_embed_plan_set_pair_wide(plan, 1)
+    ne.ngram_embed_plan_set_stream_k(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, T) == "cta_pair_wide_stream_k"
     out = torch.full((T, D), float("nan"), dtype=torch.bfloat16, device="cuda")
     ws = ne.new_workspace(plan, T)
@@ -519,23 +520,23 @@ def test_reduced_sm_count_every_form(ne, sms):
 
 def test_automatic_kernel_form(ne):
     """Prefill grids run the CTA-pair form with 512-column tiles; a 1280-token decode step at
-    D = 4096 (40 such tiles for 74 pairs) runs them under the stream-K schedule; a grid of
-    one wave of 256-column tiles keeps those (more SMs busy than 8 wide tiles split many
-    ways). Without 512-column tiles the decode step runs the one-CTA form's stream-K
-    schedule; the pairs' 256-column stream-K is taken only when both the pair form and
-    stream-K are asked for. With the dense-A form on, the decode step runs it with the
-    pairs' stream-K schedule."""
+    D = 4096 (160 tiles of 128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule;
+    a grid of one wave keeps the 256-column pair tiles (more SMs busy). The pairs' stream-K
+    schedules are taken only when the pair form (or the 512-column tiles) and stream-K are
+    both asked for. With the dense-A form on, the decode step runs it with the pairs'
+    stream-K schedule."""
     for cfg in (configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN):
         plan = plan_for(ne, cfg)
         assert ne.ngram_embed_plan_kernel_form(plan, 32768) == "cta_pair_wide"
     plan = plan_for(ne, configs.SPEC_DECODE)
-    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_wide_stream_k"
-    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"  # one wave: nothing to balance
-    ne.ngram_embed_plan_set_pair_wide(plan, 0)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "one_cta_stream_k"
+    assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"  # one wave: nothing to balance
     ne.ngram_embed_plan_set_cta_pair(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_wide"
     ne.ngram_embed_plan_set_stream_k(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_stream_k"
+    ne.ngram_embed_plan_set_pair_wide(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_wide_stream_k"
     ne.ngram_embed_plan_set_cta_pair(plan, None)
     ne.ngram_embed_plan_set_stream_k(plan, 0)
     ne.ngram_embed_plan_set_pair_wide(plan, None)

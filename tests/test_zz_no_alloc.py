@@ -75,7 +75,7 @@ def _noalloc_cfg():
 
 
 @pytest.mark.parametrize("dense_a,wide,form", [(0, 0, "one_cta_stream_k"), (1, -1, "cta_pair_dense_stream_k"),
-                                                (0, -1, "cta_pair_wide_stream_k")])
+                                                (0, 1, "cta_pair_wide_stream_k")])
 def test_static_workspace_stream_k_matches_fwd(ne, dense_a, wide, form):
     """With 6 SMs the stream-K partial tiles (2 x 6 x 256 KB) fit the fixed array, so the
     schedules whose arrival counters and partials (and, in the dense-A form, the gathered
