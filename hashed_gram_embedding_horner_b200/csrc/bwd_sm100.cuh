@@ -230,7 +230,9 @@ struct DenseSmem {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarOffset = STAGES * kStageBytes;
   static constexpr int kNumBars = 2 * STAGES + 5;
-  static constexpr int kBytes = kBarOffset + kNumBars * 8 + 16;
+  // epilogue staging: 32 rows x 32 fp32 columns per epilogue warp (4 warps)
+  static constexpr int kEpiOffset = (kBarOffset + kNumBars * 8 + 16 + 127) / 128 * 128;
+  static constexpr int kBytes = kEpiOffset + 4 * 32 * 32 * 4;
   static constexpr int kLaunchBytes = kBytes + 1024;
   static constexpr int kTmemCols = 2 * BN;
 };
@@ -361,21 +363,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue: atomic adds
+    // Per 32-column chunk: each lane reads its row's fp32 accumulators from TMEM (row per
+    // lane) into the warp's staging area; then eight lanes per row read them back, 16 bytes
+    // each, and add the scaled values into the row's destination, so every reduction
+    // instruction covers 4 rows x 128 contiguous bytes (whole 32-byte sectors) instead of
+    // 32 rows x 16 bytes. Staging layout: row r at r * 128 bytes, 16-byte unit w at
+    // ((w ^ (r & 7)) << 4): conflict-free both ways.
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
+    const uint32_t stg = sbase + L::kEpiOffset + static_cast<uint32_t>(q) * 4096u;
+    const uint32_t row_w = stg + static_cast<uint32_t>(lane) * 128u;
+    const int wv = lane & 7;   // read-back: 16-byte unit of the row
+    const int rq = lane >> 3;  // read-back: rows i * 4 + rq
     int local = 0;
     for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++local) {
       const int tile = u / p.splits;
       const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
-      const int64_t row = static_cast<int64_t>(m_blk) * kBM + row_in_tile;
-      const bool valid = row < p.M;
+      const int64_t row0 = static_cast<int64_t>(m_blk) * kBM + q * 32;  // this warp's first row
       bool got = false;
       if (lane == 0) got = mbar_wait(tfull_bar(acc), use & 1u, abort_flag, p.status);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      int s_cur = -1;
+      int32_t my_target = 0;  // scatter: this lane's row's table row in sub-table s_cur
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
@@ -385,25 +398,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_before();
           mbar_arrive(tempty_bar(acc));
         }
-        if (!valid) continue;
         const int col0 = n_blk * BN + c * 32;
-        float4* dst;
-        if (p.epi == kEpiScatterSub) {
-          const int s = col0 / p.d;  // 32 columns never straddle two sub-tables
-          int32_t r = p.idx[row * p.S + s];
-          if (static_cast<uint32_t>(r) >= p.Vs[s]) {
-            set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
-            r = 0;
+        const int s = p.epi == kEpiScatterSub ? col0 / p.d : 0;  // 32 columns never straddle two sub-tables
+        if (p.epi == kEpiScatterSub && s != s_cur) {
+          s_cur = s;
+          my_target = 0;
+          if (row0 + lane < p.M) {
+            my_target = p.idx[(row0 + lane) * p.S + s];
+            if (static_cast<uint32_t>(my_target) >= p.Vs[s]) {
+              set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+              my_target = 0;
+            }
           }
-          dst = reinterpret_cast<float4*>(p.dE[s] + static_cast<int64_t>(r) * p.d + (col0 - s * p.d));
-        } else {
-          dst = reinterpret_cast<float4*>(p.out + row * p.N + col0);
         }
 #pragma unroll
         for (int w = 0; w < 8; ++w)
-          atomicAdd(dst + w, make_float4(__uint_as_float(v[4 * w]) * p.scale, __uint_as_float(v[4 * w + 1]) * p.scale,
-                                         __uint_as_float(v[4 * w + 2]) * p.scale,
-                                         __uint_as_float(v[4 * w + 3]) * p.scale));
+          st_shared_v4(row_w + (static_cast<uint32_t>(w ^ (lane & 7)) << 4),
+                       make_uint4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]));
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = i * 4 + rq;  // row of the warp's 32
+          const uint4 x = ld_shared_v4(stg + static_cast<uint32_t>(r) * 128u + (static_cast<uint32_t>(wv ^ (r & 7)) << 4));
+          const int32_t target = __shfl_sync(0xffffffffu, my_target, r);
+          const int64_t grow = row0 + r;
+          if (grow < p.M) {
+            float* dst = p.epi == kEpiScatterSub
+                             ? p.dE[s] + static_cast<int64_t>(target) * p.d + (col0 - s * p.d) + wv * 4
+                             : p.out + grow * p.N + col0 + wv * 4;
+            atomicAdd(reinterpret_cast<float4*>(dst),
+                      make_float4(__uint_as_float(x.x) * p.scale, __uint_as_float(x.y) * p.scale,
+                                  __uint_as_float(x.z) * p.scale, __uint_as_float(x.w) * p.scale));
+          }
+        }
+        __syncwarp();  // the staging area is rewritten by the next chunk
       }
     }
   }
