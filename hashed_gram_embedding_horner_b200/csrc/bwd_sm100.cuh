@@ -370,7 +370,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // 32 rows x 16 bytes. Staging layout: row r at r * 128 bytes, 16-byte unit w at
     // ((w ^ (r & 7)) << 4): conflict-free both ways.
     const int q = warp & 3;
-    const int row_in_tile = q * 32 + lane;
     const uint32_t stg = sbase + L::kEpiOffset + static_cast<uint32_t>(q) * 4096u;
     const uint32_t row_w = stg + static_cast<uint32_t>(lane) * 128u;
     const int wv = lane & 7;   // read-back: 16-byte unit of the row
