@@ -440,8 +440,6 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const int32_t tok = p.tokens[gr];
         t = (tok >= 0 && static_cast<uint32_t>(tok) < p.V0) ? static_cast<uint32_t>(tok) : 0u;
       }
-      const uint4* e0 = reinterpret_cast<const uint4*>(p.E0 + static_cast<int64_t>(t) * p.D + n_blk * BN);
-      uint4* dst = reinterpret_cast<uint4*>(p.out + gr * p.D + n_blk * BN);
       if (whole) {
         // Stage this row's E_0 slice now, a whole main loop ahead of its use: once the
         // previous tile's TMA stores have read the rows, cp.async them into the tile buffer
@@ -502,8 +500,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         // Stream-K piece of a tile. Per (tile, row quarter) an arrival counter counts the
         // pieces published so far. The warp whose piece completes the tile sums it: its own
         // piece straight from TMEM, every other piece from its owner's partial slot, then
-        // E_0 and the scale. A warp that finds all other pieces already counted skips
-        // publishing its own. Nobody waits for anybody.
+        // E_0 and the scale, and stores the rows as a whole tile does. A warp that finds all
+        // other pieces already counted skips publishing its own. Nobody waits for anybody.
         const int64_t u_tile = static_cast<int64_t>(tile) * KB;
         const int c_lo = sk_cta_of(u_tile, U, wp.grid), c_hi = sk_cta_of(u_tile + KB - 1, U, wp.grid);
         const int others = c_hi - c_lo;  // pieces of the tile besides this one
@@ -533,11 +531,20 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           if (fin) __threadfence();
         }
         if (fin) {
+          // As for a whole tile: the rows' E_0 slice into this warp's staging rows (the
+          // previous TMA stores have read them), the finished sums written back there in
+          // bf16, and the rows leave by TMA box stores (rows past T clipped).
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+          if (valid) {
+            const uint16_t* e0row = p.E0 + static_cast<int64_t>(t) * p.D + n_blk * BN;
+#pragma unroll 8
+            for (int c = 0; c < BN / 8; ++c)
+              cp_async_16(stage_q + (c >> 3) * 16384 + lane * 128 + (((c & 7) ^ (lane & 7)) << 4), e0row + c * 8);
+          }
+          cp_async_wait_all();  // this lane's E_0 row
 #pragma unroll 1
           for (int c = 0; c < BN / 32; ++c) {
-            uint4 e[4];
-#pragma unroll
-            for (int w = 0; w < 4; ++w) e[w] = valid ? __ldg(e0 + c * 4 + w) : make_uint4(0, 0, 0, 0);
             // Pieces are added in CTA order whoever finishes, so the bits do not depend on
             // arrival order: the pieces before this CTA's, its own (TMEM), those after.
             float sum[32];
@@ -568,20 +575,28 @@ __global__ void __launch_bounds__(kProjThreads, 1)
               for (int k = 0; k < 32; ++k) sum[k] += __uint_as_float(v[k]);
             }
             for (int cc = self + 1; cc <= c_hi; ++cc) add_piece(cc);
-            if (valid) {
 #pragma unroll
-              for (int w = 0; w < 4; ++w) {
-                const uint32_t ew[4] = {e[w].x, e[w].y, e[w].z, e[w].w};
-                uint32_t o[4];
+            for (int w = 0; w < 4; ++w) {  // columns 32c + 8w .. +7: chunk (4c + w) % 8 of box c / 2
+              const uint32_t sa = stage_q + (c >> 1) * 16384 + lane * 128 + (((((c & 1) << 2) | w) ^ (lane & 7)) << 4);
+              const uint4 e = ld_shared_v4(sa);
+              const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
+              uint32_t o[4];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  const int col = w * 8 + h * 2;
-                  o[h] = pack_bf16x2((sum[col] + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale,
-                                     (sum[col + 1] + bf16_bits_to_float(ew[h] >> 16)) * p.scale);
-                }
-                dst[c * 4 + w] = make_uint4(o[0], o[1], o[2], o[3]);
+              for (int h = 0; h < 4; ++h) {
+                const int col = w * 8 + h * 2;
+                o[h] = pack_bf16x2((sum[col] + bf16_bits_to_float(ew[h] & 0xFFFFu)) * p.scale,
+                                   (sum[col + 1] + bf16_bits_to_float(ew[h] >> 16)) * p.scale);
               }
+              st_shared_v4(sa, make_uint4(o[0], o[1], o[2], o[3]));
             }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && static_cast<int64_t>(m_blk) * kBM + q * 32 < T) {
+#pragma unroll
+            for (int b = 0; b < BN / 64; ++b)
+              tma_store_2d(&maps.Out, stage_q + b * 16384, n_blk * BN + b * 64, m_blk * kBM + q * 32);
+            bulk_commit_group();
           }
           if (lane == 0) *cnt = 0;  // the tile is done: zero again for the next launch
         }
