@@ -289,6 +289,8 @@ def events(n):
 
 
 def kernel_of_form(form: str) -> str:
+    if form.startswith("cta_pair_columns"):
+        return "proj_sm100_cols_kernel"
     if form.startswith("cta_pair"):
         return "proj_sm100_pair_kernel"
     return {"one_cta": "proj_sm100_kernel", "one_cta_stream_k": "proj_sm100_kernel",
@@ -483,12 +485,12 @@ def run_decode(ne, cfg, tables, steps: int, warmup: int, dev, rank: int = 0, ext
     pk = peaks()
     flops = 2.0 * T * cfg.D * cfg.D
     form = ne.ngram_embed_plan_kernel_form(plan, T)
-    dense = form.startswith("cta_pair_dense") or form == "cta_pair_wide_dense"
+    dense = "dense" in form
     res = {
         "workload": cfg.name, "steps": steps, "tokens_per_step": T, "ms_per_step": ms / steps,
         "value": steps * T / (ms / 1e3), "unit": UNIT, "graph": True,
-        # commit + hash, (the sub-row gather of the dense-A form,) the projection
-        "gpu_launches_per_step": 3 if dense else 2,
+        # commit + hash (+ the dense-A forms' sub-row gather into G) in one launch, the projection
+        "gpu_launches_per_step": 2,
         "layer_tflops": flops / (ms / steps / 1e3) / 1e12,
         "layer_frac": flops / (ms / steps / 1e3) / 1e12 / pk["bf16_tflops"],
         "kernel_form": form,

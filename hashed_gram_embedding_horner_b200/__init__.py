@@ -47,7 +47,7 @@ EXPORTED = [
     "ngram_embed_bwd_workspace_bytes", "ngram_embed_bwd",
     "ngram_hash_stats_workspace_bytes", "ngram_hash_stats",
     "ngram_draft_cache_reset", "ngram_embed_draft_workspace_bytes", "ngram_embed_fwd_draft",
-    "ngram_embed_fwd_step", "ngram_embed_plan_set_dense_a",
+    "ngram_embed_fwd_step", "ngram_embed_plan_set_dense_a", "ngram_embed_plan_set_pair_columns",
 ]
 
 
@@ -90,6 +90,7 @@ _sig("ngram_embed_plan_set_tma_rows", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pair_wide", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_dense_a", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_pair_columns", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_sm_count", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
@@ -258,6 +259,12 @@ def ngram_embed_plan_set_pair_wide(plan: Plan, on):
     _check(_lib.ngram_embed_plan_set_pair_wide(plan.handle, v), "ngram_embed_plan_set_pair_wide")
 
 
+def ngram_embed_plan_set_pair_columns(plan: Plan, on):
+    """True/1: the pair form over column ranges whenever possible; False/0: never; None/-1: automatic."""
+    v = -1 if on is None or on == -1 else int(bool(on))
+    _check(_lib.ngram_embed_plan_set_pair_columns(plan.handle, v), "ngram_embed_plan_set_pair_columns")
+
+
 def ngram_embed_plan_set_sm_count(plan: Plan, sms: int):
     """SMs the plan's kernels use: 0 = all of the device's; else 2 .. the device's count."""
     _check(_lib.ngram_embed_plan_set_sm_count(plan.handle, int(sms)), "ngram_embed_plan_set_sm_count")
@@ -323,7 +330,8 @@ def ngram_hash_stats(V0: int, n: int, tokens, seq_offsets, moduli, workspace=Non
 
 KERNEL_FORMS = {0: "cuda_cores", 1: "one_cta", 2: "one_cta_stream_k", 3: "cta_pair", 4: "cta_pair_wide",
                 5: "cta_pair_stream_k", 6: "cta_pair_dense", 7: "cta_pair_dense_stream_k", 8: "cta_pair_wide_dense",
-                9: "cta_pair_wide_stream_k"}
+                9: "cta_pair_wide_stream_k", 10: "cta_pair_columns",
+                11: "cta_pair_columns_dense"}
 
 
 def ngram_embed_plan_set_dense_a(plan: "Plan", mode: int):

@@ -21,6 +21,7 @@
 #include "hash.cuh"
 #include "proj_sm100.cuh"
 #include "proj_sm100_pair.cuh"
+#include "proj_sm100_cols.cuh"
 #include "simt.cuh"
 #include "bwd_sm100.cuh"
 #include "stats.cuh"
@@ -62,7 +63,7 @@ struct ngram_embed_plan {
   bool maps_valid = false;
   const void* map_out = nullptr;  // the out map's pointer and row count
   int64_t map_out_T = -1;
-  bool smem_attr_set[12] = {};  // per kernel instance (form, tile width, rings), on `device`
+  bool smem_attr_set[16] = {};  // per kernel instance (form, tile width, rings), on `device`
   int a_stages = 0;            // one-CTA kernel: A ring depth (0 = default for the tile width)
   int cta_pair = -1;           // kernel form: 1 CTA pairs (cta_group::2), 0 one CTA per tile, -1 automatic
   int stream_k = 0;            // one-CTA kernel schedule: 0 automatic, 1 stream-K when possible, 2 never
@@ -72,7 +73,8 @@ struct ngram_embed_plan {
   int dense_a = 0;             // sub-rows gathered into G first, A by dense TMA: 1 on, 0 off
   const void* map_A = nullptr;  // the dense-A map's pointer and row count
   int64_t map_A_T = -1;
-  int max_clusters[4] = {0, 0, 0, 0};  // co-resident CTA pairs, per kernel instance (0 = not queried)
+  int max_clusters[5] = {0, 0, 0, 0, 0};  // co-resident CTA pairs, per kernel instance (0 = not queried)
+  int pair_cols = 0;           // pair form over column ranges: 1 whenever possible, 0 off
 };
 
 namespace {
@@ -191,6 +193,12 @@ int refresh_maps(ngram_embed_plan* p, const void* const* E_nk, const void* W, vo
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
   if (rc) return rc;
   rc = encode_2d(&p->maps.Whalf, W, p->D, p->D, static_cast<uint64_t>(p->D) * 2, kBK, p->bn / 2,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (rc) return rc;
+  rc = encode_2d(&p->maps.W16, W, p->D, p->D, static_cast<uint64_t>(p->D) * 2, kBK, 16,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (rc) return rc;
+  rc = encode_2d(&p->maps.W64, W, p->D, p->D, static_cast<uint64_t>(p->D) * 2, kBK, 64,
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
   if (rc) return rc;
   for (int s = 0; s < p->S; ++s) {
@@ -344,6 +352,77 @@ bool use_wide_stream_k(const ngram_embed_plan* p, int64_t T, size_t ws_size, int
   const int64_t units = tiles * (p->D / kBK);
   if (tiles * 16 > static_cast<int64_t>(kSkMaxTiles) * 4 || units < pairs || 2 * tiles < pairs) return false;
   return ws_size >= ws_base(p, ws_T) + sk_partial_bytes(p);
+}
+
+// Column ranges for the pair form (proj_sm100_cols.cuh): every pair computes the full K of
+// a range of columns of a 256-row block, so pairs a call's tiles would leave idle share the
+// work without stream-K's partial sums. Only with the token count known on the host, and only
+// on request (ngram_embed_plan_set_pair_columns(plan, 1)): measured on B200 at the 1280-token
+// decode step (D = 4096, 74 pairs, ranges of 256-320 columns), 61 us for the projection with
+// the rows copied in the kernel and 57 us reading them from G, against 55 us for the one-CTA
+// form's stream-K, whose fix-ups it avoids but whose stage rate (0.55 us per 48 KB stage) the
+// pairs' stages do not reach (0.8 us).
+bool use_pair_cols(const ngram_embed_plan* p, int64_t T, bool count_on_device) {
+  if (!p->tc_ok || p->bn != 256 || p->sms < 2 || count_on_device || T <= 0 || p->cta_pair == 0) return false;
+  return p->pair_cols == 1;
+}
+
+template <int HROWS, int STAGES>
+int set_cols_smem(ngram_embed_plan* p, int key) {
+  using L = ColsSmem<HROWS, STAGES>;
+  static_assert(L::kLaunchBytes <= 232448, "column-range kernel stages exceed 227 KB of shared memory");
+  if (!p->smem_attr_set[key]) {
+    if (cudaFuncSetAttribute(proj_sm100_cols_kernel<HROWS, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::kLaunchBytes) != cudaSuccess)
+      return NGRAM_ERR_CUDA;
+    p->smem_attr_set[key] = true;
+  }
+  return NGRAM_OK;
+}
+
+// The pairs are as many as fit (one per two SMs); the ranges are cut for that count. Ranges of
+// at most 320 columns (80 W rows per half and CTA) take the instance with 5 stages of 36 KB,
+// wider ones the instance with 4 stages of 48 KB.
+int launch_cols(ngram_embed_plan* p, const ProjParams& prm, int64_t T, cudaStream_t st) {
+  int rc;
+  if ((rc = set_cols_smem<128, 4>(p, 13))) return rc;
+  int& max_pairs = p->max_clusters[4];
+  if (max_pairs == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (p->sms / 2));
+    cfg.blockDim = dim3(kProjThreads);
+    cfg.dynamicSmemBytes = ColsSmem<128, 4>::kLaunchBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, proj_sm100_cols_kernel<128, 4>, &cfg) != cudaSuccess || n < 1)
+      return NGRAM_ERR_CUDA;
+    max_pairs = n;
+  }
+  const int pairs = max_pairs < p->sms / 2 ? max_pairs : p->sms / 2;
+  if (pairs < 1) return NGRAM_ERR_CUDA;
+  const int64_t mblocks = (T + 2 * kBM - 1) / (2 * kBM);
+  int widest = 0;
+  for (int pr = 0; pr < pairs; ++pr) {
+    const ColWork w = col_work(pr, pairs, mblocks, p->D / 64);
+    for (int k = 0; k < (w.m1 - w.m0) * w.nseg; ++k) {
+      const ColSeg sg = col_seg(w, k);
+      if (sg.ncols > widest) widest = sg.ncols;
+    }
+  }
+  if (widest <= 320) {
+    if ((rc = set_cols_smem<80, 5>(p, 12))) return rc;
+    return launch(proj_sm100_cols_kernel<80, 5>, dim3(2 * pairs), dim3(kProjThreads), ColsSmem<80, 5>::kLaunchBytes, st,
+                  p->pdl, 2, p->maps, prm);
+  }
+  return launch(proj_sm100_cols_kernel<128, 4>, dim3(2 * pairs), dim3(kProjThreads), ColsSmem<128, 4>::kLaunchBytes, st,
+                p->pdl, 2, p->maps, prm);
 }
 
 // ---- backward -------------------------------------------------------------------------
@@ -532,6 +611,8 @@ enum Form : int {
   kFormDenseSk = 7,    // the same with the pairs' stream-K schedule
   kFormDenseWide = 8,  // the same with 256 x 512 tiles
   kFormPairWideSk = 9, // CTA pairs, 256 x 512 tiles, stream-K, fused row gather
+  kFormPairCols = 10,  // CTA pairs, each a range of columns of a 256-row block, fused row gather
+  kFormDenseCols = 11, // rows gathered into G first; CTA pairs over column ranges, A by dense TMA
 };
 
 // Stream-K for the dense-A pair form: where a grid of whole 256 x 256 tiles would take two or
@@ -556,6 +637,7 @@ int choose_form(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws
   if (p->variant == kSimt) return kFormSimt;
   if (!count_on_device && p->cta_pair != 0 && dense_wanted(p) &&
       ws_size >= dense_g_offset(p, ws_T) + dense_g_bytes(p, T)) {
+    if (use_pair_cols(p, T, count_on_device)) return kFormDenseCols;
     if (dense_stream_k(p, T, ws_size, ws_T)) return kFormDenseSk;
     return use_pair_wide(p, T) ? kFormDenseWide : kFormDense;
   }
@@ -567,6 +649,7 @@ int choose_form(const ngram_embed_plan* p, int64_t T, size_t ws_size, int64_t ws
   prm.num_m_blocks = static_cast<int>((T + kBM - 1) / kBM);
   prm.num_n_blocks = p->D / p->bn;
   prm.num_k_blocks = p->D / kBK;
+  if (use_pair_cols(p, T, count_on_device)) return kFormPairCols;
   const bool psk = !count_on_device && p->cta_pair != 0 && p->pair_wide != 1 && use_pair_stream_k(p, T, ws_size, ws_T);
   if (!psk && !count_on_device && use_wide_stream_k(p, T, ws_size, ws_T)) return kFormPairWideSk;
   const bool sk = !psk && !count_on_device && p->cta_pair != 1 && use_stream_k(p, prm, ws_T, ws_size);
@@ -654,7 +737,7 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
     prm.sk_partials = reinterpret_cast<float*>(wsb + ws_base(p, ws_T));
   };
   const int form = choose_form(p, T, ws_size, ws_T, T_dev != nullptr);
-  if (form == kFormDense || form == kFormDenseSk || form == kFormDenseWide) {
+  if (form == kFormDense || form == kFormDenseSk || form == kFormDenseWide || form == kFormDenseCols) {
     // the call's sub-rows into G (workspace), then A tiles as dense TMA boxes of G
     void* G = wsb + dense_g_offset(p, ws_T);
     if (!g_ready && (rc = launch_gather(p, idx, T, E_nk, G, nullptr, nullptr, nullptr, ws, st))) return rc;
@@ -668,6 +751,7 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
     }
     prm.dense_a = 1;
     prm.tma_rows = 0;
+    if (form == kFormDenseCols) return launch_cols(p, prm, T, st);
     if (form == kFormDenseWide) {
       prm.num_n_blocks = p->D / 512;
       return launch_tc_pair_stages<512, kPairStagesWide>(p, prm, T, st, 8);
@@ -675,6 +759,7 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
     if (form == kFormDenseSk) stream_k_buffers();
     return launch_tc_pair<256>(p, prm, T, st);
   }
+  if (form == kFormPairCols) return launch_cols(p, prm, T, st);
   if (form == kFormPairWideSk) {
     prm.num_n_blocks = p->D / 512;
     prm.tma_rows = kBM;  // A rows by gather4 only
@@ -817,6 +902,12 @@ int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on) {
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens) {
   if (!plan || num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
   return choose_form(plan, num_tokens, ws_bytes(plan, num_tokens), num_tokens, false);
+}
+
+int ngram_embed_plan_set_pair_columns(ngram_embed_plan* plan, int mode) {
+  if (!plan || mode < -1 || mode > 1) return NGRAM_ERR_INVALID_ARG;
+  plan->pair_cols = mode == 1 ? 1 : 0;
+  return NGRAM_OK;
 }
 
 int ngram_embed_plan_set_dense_a(ngram_embed_plan* plan, int mode) {
@@ -1321,7 +1412,7 @@ int ngram_embed_fwd_step(const ngram_embed_plan* plan_c, const int32_t* commit_t
   h.idx_out = idx;
   h.status = status_ptr(workspace);
   const int form = num_tokens > 0 ? choose_form(plan, num_tokens, workspace_bytes, num_tokens, false) : kFormSimt;
-  if (form == kFormDense || form == kFormDenseSk || form == kFormDenseWide) {
+  if (form == kFormDense || form == kFormDenseSk || form == kFormDenseWide || form == kFormDenseCols) {
     // commit + hash + the sub-row gather into G in one launch (a block per sequence), then
     // the dense-A projection
     GatherParams g{};

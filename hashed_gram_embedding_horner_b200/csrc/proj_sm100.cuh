@@ -83,6 +83,8 @@ struct ProjMaps {
   CUtensorMap E[kMaxS];     // sub-table s, box {64, 1}, 128-byte swizzle (gather4)
   CUtensorMap Out;          // out [T x D], box {64, 32}, 128-byte swizzle (epilogue TMA stores)
   CUtensorMap A;            // gathered G [T x D], box {64, 128}, 128-byte swizzle (dense-A pair form)
+  CUtensorMap W16;          // W_stacked, box {64, 16} (column-range pair form: partial halves)
+  CUtensorMap W64;          // W_stacked, box {64, 64} (column-range pair form: partial halves)
 };
 
 // Shared memory (224 KB): A stages of 16 KB, W stages of BN x 128 B and the epilogue's

@@ -382,9 +382,24 @@ int ngram_embed_plan_set_pair_wide(ngram_embed_plan* plan, int on);
  * tiles and the stream-K schedule (these gather the A rows from the sub-tables inside the
  * projection); 6 = the call's sub-rows gathered into G first by a stand-alone gather kernel,
  * then CTA pairs reading A as dense TMA boxes of G, 7 = the same with the pairs' stream-K
- * schedule, 8 = the same with 512-column tiles (see ngram_embed_plan_set_dense_a); negative
- * on bad arguments. */
+ * schedule, 8 = the same with 512-column tiles (see ngram_embed_plan_set_dense_a); 10 = CTA
+ * pairs over column ranges (see ngram_embed_plan_set_pair_columns), 11 = the same reading A
+ * as dense TMA boxes of G; negative on bad arguments. */
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens);
+
+/* CTA-pair form over column ranges (Eq. 3 of "Scaling Embeddings Outperforms Scaling Experts
+ * in Language Models", section 2, partitioned by output columns): the pairs are spread evenly
+ * over the 256-token row blocks and each pair computes the full sum over K for a contiguous
+ * range of columns (a multiple of 64; two MMAs of N = half the range per k-step), so a call
+ * whose 256 x 512 tiles are fewer than the pairs keeps every pair busy without stream-K's
+ * partial sums. Ranges wider than 512 columns run as several passes over K. With the dense-A
+ * form on (ngram_embed_plan_set_dense_a) it reads A as dense boxes of G. 1 = whenever the
+ * plan's tile width is 256, the pair form is allowed and the token count is known on the
+ * host; 0 = never (default: measured on B200 at a 1280-token decode step at D = 4096, 61 us
+ * for the projection, 57 us reading G, against 55 us for the one-CTA form's stream-K; -1 is
+ * accepted as 0). A tuning knob: results agree within the stated tolerance (the k-block order
+ * differs). NGRAM_ERR_INVALID_ARG for other values. */
+int ngram_embed_plan_set_pair_columns(ngram_embed_plan* plan, int mode);
 
 /* Dense-A form of the tensor-core projection: the call's sub-rows are first copied into a
  * G buffer [num_tokens x D] (bf16) in the workspace by a gather kernel that keeps every

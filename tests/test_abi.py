@@ -145,6 +145,10 @@ V25 = (3342341, 3342371, 3342379, 3342413, 3342419, 3342439, 3342457, 3342473)
     (dict(), 32768, 148, {}, 4),                                  # prefill D = 2048: 512-column pair tiles
     (dict(D=4096, N=5, K=2, V=V25), 65536, 148, {}, 4),           # varlen prefill D = 4096
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {}, 2),            # decode step: one-CTA stream-K
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"pair_columns": 1}, 10),  # pairs over column ranges
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"pair_columns": 1, "cta_pair": 0}, 2),  # they need pairs
+    (dict(), 32768, 148, {"pair_columns": 1}, 10),                # at any size: 128 row blocks on 74 pairs
+    (dict(), 32768, 148, {"pair_columns": 1, "tile_n": 128}, 3),  # but not with 128-column W halves
     (dict(D=4096, N=3, K=4, V=V25), 128, 148, {}, 3),             # one wave: 256-column pair tiles
     (dict(D=4096, N=3, K=4, V=V25), 5120, 148, {}, 3),            # 160 wide tiles: a thin third wave
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"pair_wide": 0}, 2),  # without wide tiles: one-CTA stream-K
@@ -157,6 +161,7 @@ V25 = (3342341, 3342371, 3342379, 3342413, 3342419, 3342439, 3342457, 3342473)
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"cta_pair": 0, "stream_k": 2}, 1),
     (dict(D=4096, N=3, K=4, V=V25), 1280, 40, {}, 4),             # 20 pairs: 40 wide tiles fill 2 waves
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"dense_a": 1}, 7),  # dense A: the pairs' stream-K
+    (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"dense_a": 1, "pair_columns": 1}, 11),  # or column ranges
     (dict(D=4096, N=3, K=4, V=V25), 128, 148, {"dense_a": 1}, 6),
     (dict(D=4096, N=3, K=4, V=V25), 1280, 40, {"dense_a": 1}, 8),  # 20 pairs: wide tiles fill 2 waves
     (dict(D=4096, N=3, K=4, V=V25), 1280, 148, {"dense_a": 1, "stream_k": 2}, 8),
@@ -175,7 +180,8 @@ def test_kernel_form_choice_for_a_device_size(ne, kw, T, sms, knobs, form):
     assert lib.ngram_embed_plan_set_sm_count(h, sms) == 0  # a B200 has 148: also valid on one
     setters = {"cta_pair": lib.ngram_embed_plan_set_cta_pair, "stream_k": lib.ngram_embed_plan_set_stream_k,
                "tile_n": lib.ngram_embed_plan_set_tile_n, "dense_a": lib.ngram_embed_plan_set_dense_a,
-               "pair_wide": lib.ngram_embed_plan_set_pair_wide}
+               "pair_wide": lib.ngram_embed_plan_set_pair_wide,
+               "pair_columns": lib.ngram_embed_plan_set_pair_columns}
     for k, v in knobs.items():
         assert setters[k](h, v) == 0
     assert lib.ngram_embed_plan_kernel_form(h, T) == form

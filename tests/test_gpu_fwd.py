@@ -480,6 +480,67 @@ def test_pair_wide_matches_oracle(ne, shape, lengths):
     assert (out.float() - narrow.float()).abs().max().item() <= 2e-2
 
 
+@pytest.mark.parametrize("shape,lengths,sms", [
+    ((5000, 1024, 3, 2), RAGGED, None),                 # 2 row blocks, 37 pairs each: most hold no columns
+    ((4000, 2048, 3, 4), [256] * 5, None),              # 1280 tokens at D = 2048: ranges of 128-160 columns
+    ((5000, 4096, 3, 4), [5] * 256, None),              # the decode step's shape: ranges of 256-320 columns
+    ((3000, 1536, 2, 3), [300, 1, 399], 6),             # 3 pairs, 3 row blocks: 1536 columns in 3 passes
+    ((5000, 512, 5, 2), [1, 480, 19, 333, 167], 4),     # 2 pairs, 4 row blocks: whole blocks per pair
+    ((4000, 768, 3, 2), [3, 250, 7], 40),               # D % 512 != 0, one ragged block on 20 pairs
+], ids=["D1024_idle_pairs", "D2048_T1280", "D4096_T1280", "D1536_three_passes", "D512_blocks_per_pair",
+        "D768_ragged"])
+@pytest.mark.parametrize("dense", [0, 1], ids=["fused_rows", "dense_a"])
+def test_pair_columns_matches_oracle(ne, shape, lengths, sms, dense):
+    """The pair form over column ranges (every pair the full K of a range of columns of one
+    256-row block; two MMAs of N = half the range per k-step; wider ranges in several
+    passes), with the A rows copied by the kernel or read as dense boxes of G, against the
+    oracle on every row, twice for repeatable bits."""
+    cfg = small_cfg(*shape)
+    tokens, offsets = ragged_tokens(cfg, lengths)
+    from tests.helpers import host_tables
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = plan_for(ne, cfg)
+    if sms:
+        ne.ngram_embed_plan_set_sm_count(plan, sms)
+    ne.ngram_embed_plan_set_pair_columns(plan, 1)
+    ne.ngram_embed_plan_set_dense_a(plan, dense)
+    assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == ("cta_pair_columns", "cta_pair_columns_dense")[dense]
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0
+    want = oracle.forward(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, tokens, offsets, E0h, Eh, Wh)
+    assert_close(to_host_f64(out), want, what=cfg.name + " column ranges")
+    again, status = run_fwd(ne, plan, cfg, tokens, offsets, E0, E, W)
+    assert status == 0 and torch.equal(out, again)
+
+
+@pytest.mark.parametrize("D,N,K,sms", [(768, 2, 3, None), (1024, 2, 1, None), (1024, 2, 1, 6), (768, 2, 3, 12)])
+@pytest.mark.parametrize("dense", [0, 1], ids=["fused_rows", "dense_a"])
+def test_pair_columns_gather_and_layout_bit_exact(ne, D, N, K, sms, dense):
+    """W = I and E_0 = 0 (S + 1 a power of two): every output element is one gathered
+    element divided exactly, so each column range must put every column in its place bit for
+    bit, whatever the range widths (partial W halves by 16-row boxes, second passes)."""
+    cfg = small_cfg(7000, D, N, K, seed=3)
+    S = cfg.S
+    tokens, offsets = ragged_tokens(cfg, [5, 128, 200, 3, 311])
+    from tests.helpers import host_tables
+    _, Eh, _ = host_tables(cfg)
+    eye = gen.f32_to_bf16_bits(np.eye(cfg.D, dtype=np.float32))
+    idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, oracle.context_windows(cfg.N, tokens, offsets))
+    G = np.concatenate([gen.bf16_bits_to_f32(Eh[s][idx[:, s]]) for s in range(S)], axis=1)
+    plan = plan_for(ne, cfg)
+    if sms:
+        ne.ngram_embed_plan_set_sm_count(plan, sms)
+    ne.ngram_embed_plan_set_pair_columns(plan, 1)
+    ne.ngram_embed_plan_set_dense_a(plan, dense)
+    assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == ("cta_pair_columns", "cta_pair_columns_dense")[dense]
+    zeros0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.bfloat16, device="cuda")
+    out, status = run_fwd(ne, plan, cfg, tokens, offsets, zeros0, [to_device(e, torch.bfloat16) for e in Eh],
+                          to_device(eye, torch.bfloat16))
+    assert status == 0
+    np.testing.assert_array_equal(out.float().cpu().numpy(), G / (S + 1))
+
+
 def test_pair_wide_not_for_narrow_tiles(ne):
     """512-column tiles need D % 512 == 0 and 256-column W halves; otherwise the knob leaves
     the 256- or 128-column pair form in place."""
@@ -520,16 +581,20 @@ def test_reduced_sm_count_every_form(ne, sms):
 
 def test_automatic_kernel_form(ne):
     """Prefill grids run the CTA-pair form with 512-column tiles; a 1280-token decode step at
-    D = 4096 (160 tiles of 128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule;
+    D = 4096 (160 tiles of 128 x 256 on 148 SMs) runs the one-CTA form's stream-K schedule, or
+    the pairs over column ranges when asked for;
     a grid of one wave keeps the 256-column pair tiles (more SMs busy). The pairs' stream-K
     schedules are taken only when the pair form (or the 512-column tiles) and stream-K are
     both asked for. With the dense-A form on, the decode step runs it with the pairs'
-    stream-K schedule."""
+    stream-K schedule (or over column ranges when asked for)."""
     for cfg in (configs.PREFILL_D2048, configs.PREFILL_D4096_VARLEN):
         plan = plan_for(ne, cfg)
         assert ne.ngram_embed_plan_kernel_form(plan, 32768) == "cta_pair_wide"
     plan = plan_for(ne, configs.SPEC_DECODE)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "one_cta_stream_k"
+    ne.ngram_embed_plan_set_pair_columns(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_columns"
+    ne.ngram_embed_plan_set_pair_columns(plan, 0)
     assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair"  # one wave: nothing to balance
     ne.ngram_embed_plan_set_cta_pair(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_wide"
@@ -543,6 +608,9 @@ def test_automatic_kernel_form(ne):
     ne.ngram_embed_plan_set_dense_a(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_dense_stream_k"
     assert ne.ngram_embed_plan_kernel_form(plan, 128) == "cta_pair_dense"
+    ne.ngram_embed_plan_set_pair_columns(plan, 1)
+    assert ne.ngram_embed_plan_kernel_form(plan, 1280) == "cta_pair_columns_dense"
+    ne.ngram_embed_plan_set_pair_columns(plan, 0)
     assert ne.ngram_embed_plan_kernel_form(plan_for(ne, configs.TINY), 128) == "cuda_cores"
 
 
