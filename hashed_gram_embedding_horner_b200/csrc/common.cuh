@@ -149,6 +149,19 @@ __device__ __forceinline__ void fence_barrier_init() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Global-memory writes seen through the generic proxy (another CTA's stores, acquired) are
+// ordered before this thread's later async-proxy reads of them (a bulk copy).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Untiled bulk copy global -> this CTA's shared memory (16-byte aligned addresses, size a
+// multiple of 16), completing `bytes` on the mbarrier `bar`.
+__device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
 
 // 16-byte global load that bypasses L1 (rows read once per CTA).
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {

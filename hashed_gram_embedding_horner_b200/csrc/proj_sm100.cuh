@@ -101,10 +101,12 @@ struct ProjSmem {
   static constexpr int kEOffset = kWOffset + WST * kBBytes;  // then the epilogue's tile
   static constexpr int kEBytes = kBM * BN * 2;  // E_0 slice in, bf16 output out (BN/64 boxes of 128 x 64)
   static constexpr int kBarOffset = kEOffset + kEBytes;
-  static constexpr int kNumBars = 2 * AST + 2 * WST + 5;
+  static constexpr int kNumBars = 2 * AST + 2 * WST + 5 + 4;  // + one per epilogue warp (end fix-up)
   static constexpr int kBytes = kBarOffset + kNumBars * 8 + 16;
   static constexpr int kLaunchBytes = kBytes + 1024;  // slack for 1024-byte alignment
   static constexpr int kTmemCols = 2 * BN;
+  // the last stream-K fix-up stages one partial region per epilogue warp in the rings
+  static_assert(4 * BN * 128 <= kEOffset, "rings smaller than four partial regions");
 };
 
 __device__ __forceinline__ uint32_t clamp_row(int32_t r, uint32_t V, int* status) {
@@ -246,6 +248,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   auto tfull_bar = [&](int a) { return bar0 + 8u * (kT0 + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (kT0 + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (kT0 + 4);
+  auto fix_bar = [&](int q) { return bar0 + 8u * (kT0 + 5 + q); };  // epilogue warp q's last fix-up
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + L::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto a_tile = [&](int s) { return sbase + s * L::kABytes; };
@@ -269,6 +272,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       mbar_init(tempty_bar(a), 128u);  // every epilogue thread
     }
     mbar_init(drain_bar, 1u);
+    for (int q = 0; q < 4; ++q) mbar_init(fix_bar(q), 1u);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -514,17 +518,19 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         if (!fin) {
           // slot 0: the piece that starts this CTA's unit range; slot 1: the one that ends it
           const int slot = (u_tile + g.i0 == sk_first_unit(U, wp.grid, blockIdx.x)) ? 0 : 1;
+          // a slot holds 4 warp regions of 32 rows x BN columns (BN * 128 contiguous bytes
+          // each), column group major within a region: a warp's store is 512 contiguous bytes
           float4* mine = reinterpret_cast<float4*>(p.sk_partials) +
-                         (static_cast<size_t>(blockIdx.x) * 2 + slot) * (kBM * BN / 4) + row_in_tile;
+                         (static_cast<size_t>(blockIdx.x) * 2 + slot) * (kBM * BN / 4) + q * (BN / 4) * 32 + lane;
 #pragma unroll 1
           for (int c = 0; c < BN / 32; ++c) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(taddr + c * 32, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int w = 0; w < 8; ++w)  // column group major: a warp's store is 512 contiguous bytes
-              mine[(c * 8 + w) * kBM] = make_float4(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1]),
-                                                    __uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3]));
+            for (int w = 0; w < 8; ++w)
+              mine[(c * 8 + w) * 32] = make_float4(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1]),
+                                                   __uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3]));
           }
           __threadfence();
           __syncwarp();
@@ -544,6 +550,27 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             for (int c = 0; c < BN / 8; ++c)
               cp_async_16(stage_q + (c >> 3) * 16384 + lane * 128 + (((c & 7) ^ (lane & 7)) << 4), e0row + c * 8);
           }
+          // The CTA's last segment with one other piece: every stage has been consumed and
+          // none will be loaded again, so the rings are free, and the other piece's region
+          // for this warp comes in as one bulk copy into ring bytes [q * BN * 128, +BN * 128)
+          // instead of BN / 32 rounds of dependent loads at the very end of the launch.
+          const int self = static_cast<int>(blockIdx.x);
+          const bool staged = others == 1 && seg_next(wp, g).tile >= num_tiles;
+          const uint32_t ring_q = sbase + static_cast<uint32_t>(q * BN * 128);
+          auto region = [&](int cc) {  // this warp's region of CTA cc's piece of the tile
+            const int sl = (sk_first_unit(U, wp.grid, cc) >= u_tile) ? 0 : 1;
+            return reinterpret_cast<const float4*>(p.sk_partials) +
+                   (static_cast<size_t>(cc) * 2 + sl) * (kBM * BN / 4) + q * (BN / 4) * 32;
+          };
+          if (staged) {
+            if (lane == 0) {
+              fence_proxy_async_global();  // the acquired partial, read by the async proxy
+              mbar_arrive_expect_tx(fix_bar(q), BN * 128);
+              bulk_load_g2s(ring_q, region(c_lo == self ? c_hi : c_lo), BN * 128, fix_bar(q));
+              mbar_wait(fix_bar(q), 0, abort_flag, p.status);  // a timeout sets the status word
+            }
+            __syncwarp();
+          }
           cp_async_wait_all();  // this lane's E_0 row
 #pragma unroll 1
           for (int c = 0; c < BN / 32; ++c) {
@@ -553,12 +580,18 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 #pragma unroll
             for (int k = 0; k < 32; ++k) sum[k] = 0.f;
             auto add_piece = [&](int cc) {
-              const int sl = (sk_first_unit(U, wp.grid, cc) >= u_tile) ? 0 : 1;
-              const float4* part = reinterpret_cast<const float4*>(p.sk_partials) +
-                                   (static_cast<size_t>(cc) * 2 + sl) * (kBM * BN / 4) + row_in_tile;
               float4 x[8];
+              if (staged) {
 #pragma unroll
-              for (int w = 0; w < 8; ++w) x[w] = __ldcg(part + (c * 8 + w) * kBM);
+                for (int w = 0; w < 8; ++w) {
+                  const uint4 r = ld_shared_v4(ring_q + static_cast<uint32_t>(((c * 8 + w) * 32 + lane) * 16));
+                  x[w] = make_float4(__uint_as_float(r.x), __uint_as_float(r.y), __uint_as_float(r.z), __uint_as_float(r.w));
+                }
+              } else {
+                const float4* part = region(cc) + lane;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) x[w] = __ldcg(part + (c * 8 + w) * 32);
+              }
 #pragma unroll
               for (int w = 0; w < 8; ++w) {
                 sum[4 * w] += x[w].x;
@@ -567,7 +600,6 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 sum[4 * w + 3] += x[w].w;
               }
             };
-            const int self = static_cast<int>(blockIdx.x);
             for (int cc = c_lo; cc < self; ++cc) add_piece(cc);
             {
               uint32_t v[32];

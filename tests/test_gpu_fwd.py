@@ -144,10 +144,12 @@ SK_SHAPES = [(3000, 1024, 3, 2, 301), (5000, 2048, 3, 2, 301), (4000, 4096, 2, 2
 
 @pytest.mark.parametrize("shape", SK_SHAPES, ids=lambda s: "V0%d_D%d_N%d_K%d_T%d" % s)
 @pytest.mark.parametrize("tile_n", [256, 128])
-def test_stream_k_matches_oracle_and_is_repeatable(ne, shape, tile_n):
+@pytest.mark.parametrize("sms", [None, 10], ids=["all_sms", "10_sms"])
+def test_stream_k_matches_oracle_and_is_repeatable(ne, shape, tile_n, sms):
     """One-CTA kernel with every SM given an equal run of (tile, k-block) units, so tiles are
-    split over up to a dozen CTAs: parity with the oracle; a second call on the same
-    workspace gives the same bits (the fixup order is fixed and the arrival counters are
+    split over up to a dozen CTAs (on 10 SMs over at most two, whose last piece is summed
+    from a partial staged in the free rings): parity with the oracle; a second call on the
+    same workspace gives the same bits (the fixup order is fixed and the arrival counters are
     left at zero); data-parallel schedule agrees within the tolerance."""
     V0, D, N, K, T = shape
     cfg = small_cfg(V0, D, N, K, seed=5)
@@ -161,6 +163,8 @@ def test_stream_k_matches_oracle_and_is_repeatable(ne, shape, tile_n):
     plan = plan_for(ne, cfg, 2, tile_n, pair=0)
     ne.ngram_embed_plan_set_tma_rows(plan, 0)
     ne.ngram_embed_plan_set_stream_k(plan, 1)
+    if sms:
+        ne.ngram_embed_plan_set_sm_count(plan, sms)
     out = torch.full((T, D), float("nan"), dtype=torch.bfloat16, device="cuda")
     ws = ne.new_workspace(plan, T)
     tk, of = dev_i32(tokens), dev_i32(offsets)
@@ -260,30 +264,33 @@ def test_wide_stream_k_matches_oracle_and_is_repeatable(ne, shape, sms):
     assert_close(to_host_f64(whole), want, what=f"{cfg.name} whole wide tiles")
 
 
-@pytest.mark.parametrize("pair", [0, 1, 2], ids=["one_cta", "pair", "pair_wide"])
+@pytest.mark.parametrize("pair", [0, 1, 2, 3], ids=["one_cta", "pair", "pair_wide", "one_cta_10_sms"])
 def test_stream_k_bit_exact_with_identity_w(ne, pair):
     """W = I and E_0 = 0 under stream-K (one-CTA or CTA-pair form): each output element gets
     one nonzero product, so the fp32 partials of a split tile add zeros to it and the
     result stays exact."""
     # S + 1 = 4: the scale is exact; one-CTA: 27 tiles of 128 x 128; pairs: 9 of 256 x 256
-    # (108 units of a k-block on 74 pairs); wide: 9 of 256 x 512 on 3 pairs (72 units each)
-    cfg = small_cfg(7000, {0: 1152, 1: 768, 2: 1536}[pair], 2, 3, seed=3)
+    # (108 units of a k-block on 74 pairs); wide: 9 of 256 x 512 on 3 pairs (72 units each);
+    # one-CTA on 10 SMs: 48.6 units per CTA, a tile over at most two CTAs (the last piece's
+    # partial staged in the rings)
+    one = pair in (0, 3)
+    cfg = small_cfg(7000, {0: 1152, 1: 768, 2: 1536, 3: 1152}[pair], 2, 3, seed=3)
     S = cfg.S
-    tokens, offsets = ragged_tokens(cfg, [5, 128, 200, 3] if pair == 0 else [5, 300, 400, 3])
+    tokens, offsets = ragged_tokens(cfg, [5, 128, 200, 3] if one else [5, 300, 400, 3])
     from tests.helpers import host_tables
     _, Eh, _ = host_tables(cfg)
     eye = gen.f32_to_bf16_bits(np.eye(cfg.D, dtype=np.float32))
     idx = oracle.hash_indices(cfg.V0, cfg.N, cfg.K, cfg.V_nk, oracle.context_windows(cfg.N, tokens, offsets))
     G = np.concatenate([gen.bf16_bits_to_f32(Eh[s][idx[:, s]]) for s in range(S)], axis=1)
-    plan = plan_for(ne, cfg, 2 if pair == 0 else 0, 128 if pair == 0 else 256, pair=min(pair, 1))
-    if pair == 0:
+    plan = plan_for(ne, cfg, 2 if one else 0, 128 if one else 256, pair=0 if one else 1)
+    if one:
         ne.ngram_embed_plan_set_tma_rows(plan, 0)
     ne.ngram_embed_plan_set_pair_wide(plan, 1 if pair == 2 else 0)
-    if pair == 2:
-        ne.ngram_embed_plan_set_sm_count(plan, 6)
+    if pair in (2, 3):
+        ne.ngram_embed_plan_set_sm_count(plan, 6 if pair == 2 else 10)
     ne.ngram_embed_plan_set_stream_k(plan, 1)
     assert ne.ngram_embed_plan_kernel_form(plan, len(tokens)) == \
-        ("one_cta_stream_k", "cta_pair_stream_k", "cta_pair_wide_stream_k")[pair]
+        ("one_cta_stream_k", "cta_pair_stream_k", "cta_pair_wide_stream_k", "one_cta_stream_k")[pair]
     zeros0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.bfloat16, device="cuda")
     out, status = run_fwd(ne, plan, cfg, tokens, offsets, zeros0, [to_device(e, torch.bfloat16) for e in Eh],
                           to_device(eye, torch.bfloat16))
