@@ -49,6 +49,28 @@ __device__ __forceinline__ uint32_t horner_step(uint32_t h, uint32_t V0, uint32_
   return static_cast<uint32_t>(r);
 }
 
+// Eq. 2 for token i from its window u (u[j] = t_{i-j}, newest first, ids already checked),
+// and the draft-phase records of the window when asked for.
+__device__ __forceinline__ void hash_window(const HashParams& p, int64_t i, int64_t start, int32_t slot,
+                                            const uint32_t (&u)[kMaxN]) {
+  if (p.win_out) {
+    for (int j = 0; j < p.N; ++j) p.win_out[i * p.N + j] = static_cast<int32_t>(u[p.N - 1 - j]);
+    const int64_t jpos = i - start;
+    p.entry_out[i] = (slot >= 0 && jpos < p.positions) ? static_cast<int32_t>(slot * p.positions + jpos) : -1;
+  }
+  int32_t* out = p.idx_out + i * p.S;
+  for (int n = 2; n <= p.N; ++n) {
+    for (int k = 0; k < p.K; ++k) {
+      const int s = (n - 2) * p.K + k;
+      const uint32_t V = p.V[s];
+      const uint64_t m = p.barrett[s];
+      uint32_t h = 0;
+      for (int j = n - 1; j >= 0; --j) h = horner_step(h, p.V0, u[j], V, m);
+      out[s] = static_cast<int32_t>(h);
+    }
+  }
+}
+
 // Eq. 2 for token i of a sequence starting at `start`, with the sequence's committed
 // history (slot >= 0: hist_len ids, those before hist_from evicted) before it.
 __device__ __forceinline__ void hash_one(const HashParams& p, int64_t i, int64_t start, int32_t slot,
@@ -78,23 +100,7 @@ __device__ __forceinline__ void hash_one(const HashParams& p, int64_t i, int64_t
     }
     u[j] = static_cast<uint32_t>(t);
   }
-
-  if (p.win_out) {
-    for (int j = 0; j < p.N; ++j) p.win_out[i * p.N + j] = static_cast<int32_t>(u[p.N - 1 - j]);
-    const int64_t jpos = i - start;
-    p.entry_out[i] = (slot >= 0 && jpos < p.positions) ? static_cast<int32_t>(slot * p.positions + jpos) : -1;
-  }
-  int32_t* out = p.idx_out + i * p.S;
-  for (int n = 2; n <= p.N; ++n) {
-    for (int k = 0; k < p.K; ++k) {
-      const int s = (n - 2) * p.K + k;
-      const uint32_t V = p.V[s];
-      const uint64_t m = p.barrett[s];
-      uint32_t h = 0;
-      for (int j = n - 1; j >= 0; --j) h = horner_step(h, p.V0, u[j], V, m);
-      out[s] = static_cast<int32_t>(h);
-    }
-  }
+  hash_window(p, i, start, slot, u);
 }
 
 constexpr int kHashSmemOffsets = 4096;  // offsets staged in shared memory when B + 1 fits

@@ -446,6 +446,13 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const int32_t tok = p.tokens[gr];
         t = (tok >= 0 && static_cast<uint32_t>(tok) < p.V0) ? static_cast<uint32_t>(tok) : 0u;
       }
+      if (!whole && valid) {
+        // A stream-K piece may be the one that finishes the tile: its rows' E_0 slice toward
+        // L2 while the piece's main loop runs (the fix-up copies it in only once it knows).
+        const uint16_t* e0row = p.E0 + static_cast<int64_t>(t) * p.D + n_blk * BN;
+#pragma unroll
+        for (int l = 0; l < BN / 64; ++l) prefetch_l2(e0row + l * 64);
+      }
       if (whole) {
         // Stage this row's E_0 slice now, a whole main loop ahead of its use: once the
         // previous tile's TMA stores have read the rows, cp.async them into the tile buffer

@@ -230,3 +230,55 @@ def test_fused_commit_and_step_equals_separate_calls(ne, dense_a):
         assert torch.equal(c1.ring, c2.ring) and torch.equal(c1.len, c2.len) and torch.equal(c1.valid_from, c2.valid_from)
         prev = (tok, cnt)
     assert ne.ngram_embed_get_status(ws1) == 0 and ne.ngram_embed_get_status(ws2) == 0
+
+
+def test_fused_step_edge_cases_match_separate_calls(ne):
+    """The fused step's per-sequence path (loads in three rounds, committed ids taken from the
+    commit buffer) against ngram_cache_commit + ngram_embed_fwd where it matters: a sequence
+    of 40 ids (more than a warp's lanes: the one-load-at-a-time path), empty sequences,
+    nothing to commit, a count above the stride (BAD_APPEND), an id outside the vocabulary
+    in the commit buffer (BAD_TOKEN: that entry is not committed), and a history cut by
+    valid_from (EVICTED). Outputs, indices, ring, lengths and status bits agree."""
+    from tests.helpers import host_tables, to_device
+    N, K, D, B, P, C = 4, 1, 384, 6, 6, 8
+    V0, V = 3000, [4099, 5003, 6007]
+    cfg = configs.NgramConfig(name="edges", V0=V0, D=D, N=N, K=K, V_nk=tuple(V), dtype="bf16", seed=17)
+    E0h, Eh, Wh = host_tables(cfg)
+    E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
+    plan = ne.ngram_embed_plan_create(V0, D, N, K, V, ne.NGRAM_BF16)
+    lengths = [1, 40, 0, 6, 3, 2]
+    off_h = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    T = int(off_h[-1])
+    off = dev_i32(off_h)
+    ws1, ws2 = ne.new_workspace(plan, T), ne.new_workspace(plan, T)
+    c1, c2 = ne.Cache.empty(B, C), ne.Cache.empty(B, C)
+    for c, w in ((c1, ws1), (c2, ws2)):
+        ne.ngram_cache_reset(plan, c, w)
+    rng = np.random.default_rng(5)
+    prev = None
+    for step in range(5):
+        tok = dev_i32(rng.integers(0, V0, T))
+        commit = rng.integers(0, V0, B * P).astype(np.int32)
+        counts = np.array([1, 6, 0, 7 if step == 2 else 3, 2, 6], np.int32)
+        if step == 3:
+            commit[4 * P + 1] = V0 + 5  # entry 4 holds an id outside the vocabulary
+        if step == 4:
+            for c in (c1, c2):  # history of sequence 0 cut right below its newest position
+                c.valid_from[0] = c.len[0] - 1
+        o1 = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+        o2 = torch.empty_like(o1)
+        if prev is not None:
+            ne.ngram_cache_commit(plan, c1, prev[0], P, prev[1], ws1)
+        ne.ngram_embed_fwd(plan, tok, off, E0, E, W, o1, ws1, cache=c1)
+        ne.ngram_embed_fwd_step(plan, tok, off, E0, E, W, o2, ws2, c2,
+                                commit_tokens=None if prev is None else prev[0], commit_stride=P,
+                                commit_counts=None if prev is None else prev[1])
+        s1, s2 = ne.ngram_embed_get_status(ws1), ne.ngram_embed_get_status(ws2)
+        assert s1 == s2, (step, ne.status_names(s1), ne.status_names(s2))
+        assert torch.equal(o1, o2), step
+        head = 33024
+        assert torch.equal(ws1[head:head + T * 12], ws2[head:head + T * 12])  # [T x S] int32 indices
+        assert torch.equal(c1.ring, c2.ring) and torch.equal(c1.len, c2.len) and torch.equal(c1.valid_from, c2.valid_from)
+        prev = (dev_i32(commit), dev_i32(counts))
+    # the edge cases did occur
+    assert set(ne.status_names(ne.ngram_embed_get_status(ws2))) == {"BAD_APPEND", "BAD_TOKEN", "EVICTED"}
