@@ -13,8 +13,9 @@
 //
 // A range of c columns (a multiple of 64) runs as two MMAs of N = c/2 per k-step on the same
 // A stage (M = 256, tcgen05.mma.cta_group::2), the halves' accumulators at TMEM columns
-// [0, c/2) and [256, 256 + c/2). Equal halves, because an MMA costs a minimum time whatever
-// its N (measured on B200: a k-step of N = 256 + 32 took as long as 256 + 150). Each CTA
+// [0, c/2) and [256, 256 + c/2). Equal halves, because an MMA's time does not shrink below
+// that of N = 128 (measured on B200: a k-block of N = 32, 64 or 128 took 453 cycles, one of
+// N = 256 518-541), so a small second MMA would cost as much as a 128-column one. Each CTA
 // holds its 128 A rows (16-byte cp.async from the sub-tables) and c/4 rows of W per half
 // (2-D TMA: one 128-row box for a 256-column half, else boxes of 64 and 16 rows). A range wider
 // than 512 columns (fewer pairs than row blocks times D / 512) is cut into segments of at
