@@ -48,6 +48,7 @@ EXPORTED = [
     "ngram_hash_stats_workspace_bytes", "ngram_hash_stats",
     "ngram_draft_cache_reset", "ngram_embed_draft_workspace_bytes", "ngram_embed_fwd_draft",
     "ngram_embed_fwd_step", "ngram_embed_plan_set_dense_a", "ngram_embed_plan_set_pair_columns",
+    "ngram_embed_plan_set_fused_step",
 ]
 
 
@@ -91,6 +92,7 @@ _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pair_wide", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_dense_a", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pair_columns", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_fused_step", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_sm_count", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pdl", [_P, ctypes.c_int])
@@ -257,6 +259,11 @@ def ngram_embed_plan_set_pair_wide(plan: Plan, on):
     """True/1: the pair form's 512-column tiles; False/0: 256-column; None/-1: automatic."""
     v = -1 if on is None or on == -1 else int(bool(on))
     _check(_lib.ngram_embed_plan_set_pair_wide(plan.handle, v), "ngram_embed_plan_set_pair_wide")
+
+
+def ngram_embed_plan_set_fused_step(plan: Plan, on: bool):
+    """ngram_embed_fwd_step in one launch where the one-CTA form runs it (default False)."""
+    _check(_lib.ngram_embed_plan_set_fused_step(plan.handle, int(bool(on))), "ngram_embed_plan_set_fused_step")
 
 
 def ngram_embed_plan_set_pair_columns(plan: Plan, on):

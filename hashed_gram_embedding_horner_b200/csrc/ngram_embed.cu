@@ -34,6 +34,7 @@ namespace {
 
 // Workspace: [status word + padding | stream-K arrival counters | T x S indices | stream-K partials]
 constexpr size_t kStatusBytes = 256;
+constexpr size_t kStepCountOffset = 128;  // in the status header: the fused decode step's two counts
 constexpr int kSkMaxTiles = 2048;                          // stream-K only for grids of at most this many tiles
 constexpr size_t kSkCounterBytes = size_t(kSkMaxTiles) * 4 * sizeof(int32_t);  // one per (tile, row quarter)
 constexpr size_t kHeadBytes = kStatusBytes + kSkCounterBytes;                   // zeroed by clear_status
@@ -75,6 +76,7 @@ struct ngram_embed_plan {
   int64_t map_A_T = -1;
   int max_clusters[5] = {0, 0, 0, 0, 0};  // co-resident CTA pairs, per kernel instance (0 = not queried)
   int pair_cols = 0;           // pair form over column ranges: 1 whenever possible, 0 off
+  int fused_step = 0;          // decode step committed and hashed inside the one-CTA projection
 };
 
 namespace {
@@ -238,6 +240,22 @@ int launch_tc_rings(ngram_embed_plan* p, const ProjParams& prm, cudaStream_t st,
   }
   const int tiles = prm.num_m_blocks * prm.num_n_blocks;
   const int grid = (prm.stream_k || tiles > p->sms) ? p->sms : tiles;
+  if (prm.sh.on) {
+    // a fused decode step: its gather warps wait for the sequences every CTA hashes, so all
+    // CTAs must be resident at once (one per SM)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kProjThreads);
+    cfg.dynamicSmemBytes = L::kLaunchBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, p->maps, prm) != cudaSuccess) return NGRAM_ERR_CUDA;
+    return check_launch();
+  }
   return launch(kern, dim3(grid), dim3(kProjThreads), L::kLaunchBytes, st, p->pdl, 1, p->maps, prm);
 }
 
@@ -702,7 +720,8 @@ int launch_gather(const ngram_embed_plan* p, const int32_t* idx, int64_t T, cons
 // commit + hash + gather launch wrote it).
 int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int64_t T, const void* E0,
             const void* const* E_nk, const void* W, void* out, void* ws, size_t ws_size, int64_t ws_T,
-            cudaStream_t st, const int32_t* T_dev = nullptr, bool g_ready = false) {
+            cudaStream_t st, const int32_t* T_dev = nullptr, bool g_ready = false,
+            const StepHash* sh = nullptr) {
   if (p->variant == kSimt) {
     return p->dtype == NGRAM_F32
                ? launch_simt<float>(p, tokens, idx, T, E0, E_nk, W, out, ws, st, T_dev)
@@ -782,6 +801,7 @@ int project(ngram_embed_plan* p, const int32_t* tokens, const int32_t* idx, int6
   }
   if (pair) return p->bn == 256 ? launch_tc_pair<256>(p, prm, T, st) : launch_tc_pair<128>(p, prm, T, st);
   if (form == kFormOneSk) stream_k_buffers();
+  if (sh && (form == kFormOne || form == kFormOneSk)) prm.sh = *sh;  // the decode step's commit and hashing
   return p->bn == 256 ? launch_tc<256>(p, prm, st) : launch_tc<128>(p, prm, st);
 }
 
@@ -902,6 +922,12 @@ int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on) {
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens) {
   if (!plan || num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
   return choose_form(plan, num_tokens, ws_bytes(plan, num_tokens), num_tokens, false);
+}
+
+int ngram_embed_plan_set_fused_step(ngram_embed_plan* plan, int on) {
+  if (!plan || on < 0 || on > 1) return NGRAM_ERR_INVALID_ARG;
+  plan->fused_step = on;
+  return NGRAM_OK;
 }
 
 int ngram_embed_plan_set_pair_columns(ngram_embed_plan* plan, int mode) {
@@ -1434,6 +1460,18 @@ int ngram_embed_fwd_step(const ngram_embed_plan* plan_c, const int32_t* commit_t
       return rc;
     return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace, workspace_bytes, num_tokens,
                    st, nullptr, true);
+  }
+  if ((form == kFormOne || form == kFormOneSk) && plan->fused_step && plan->S <= 8 && num_tokens > 0) {
+    // One launch: warps 10-11 of every CTA of the one-CTA projection commit and hash a share
+    // of the sequences; its gather warps start once all are done.
+    StepHash sh{};
+    sh.on = 1;
+    sh.c = c;
+    sh.h = h;
+    sh.ready = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + kStepCountOffset);
+    sh.passed = sh.ready + 1;
+    return project(plan, tokens, idx, num_tokens, E0, E_nk, W_stacked, out, workspace, workspace_bytes, num_tokens,
+                   st, nullptr, false, &sh);
   }
   if ((rc = launch(commit_hash_kernel, dim3(static_cast<unsigned>((num_seqs + 7) / 8)), dim3(256), 0, st,
                    plan->pdl, 1, c, h)))

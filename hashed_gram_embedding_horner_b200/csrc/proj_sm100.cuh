@@ -38,6 +38,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "decode.cuh"
 
 namespace ngram {
 
@@ -49,6 +50,19 @@ constexpr int kAThreads = kAWarps * 32;
 constexpr int kWarpB = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpEpi0 = 12;
+
+// A decode step fused into the one-CTA projection (ngram_embed_fwd_step in one launch): the
+// otherwise idle warps 10 and 11 of every CTA commit and hash a share of the sequences
+// (commit_hash_warp_fast, section 4.2 N-gram Cache, Eq. 2) into the index buffer, and the
+// gather warps start once the count of sequences done reaches num_seqs. The launch is
+// cooperative, so every CTA is resident and the wait ends; it is bounded all the same.
+struct StepHash {
+  int on;
+  CacheParams c;
+  HashParams h;
+  int* ready;   // sequences hashed so far (zero between launches)
+  int* passed;  // CTAs past the wait (the last re-arms both counts)
+};
 
 struct ProjParams {
   const int32_t* tokens;  // [T]
@@ -75,7 +89,14 @@ struct ProjParams {
   // CTA-pair kernel: 1 = A tiles are dense 2-D TMA boxes of an already gathered G [T x D]
   // (maps.A), not rows gathered from the sub-tables
   int dense_a;
+  StepHash sh;  // one-CTA kernel: the decode step's commit and hashing, when sh.on
 };
+
+__device__ __forceinline__ int32_t ld_cg_b32(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.global.cg.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
 struct ProjMaps {
   CUtensorMap W;            // W_stacked, box {64, BN}, 128-byte swizzle
@@ -316,6 +337,33 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     const int issuer = warp * lanes_tma + lane;  // rows 4*issuer .. +3
     const uint32_t tma_bytes = static_cast<uint32_t>(p.tma_rows) * 128u;
     const uint64_t pol = l2_policy_evict_normal();
+    // A fused decode step: the indices are written during this launch (by warps 10-11 of
+    // every CTA): wait until all sequences are done, then read them coherently.
+    const bool fused = p.sh.on != 0;
+    if (fused) {
+      int go = 1;
+      if (t == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(p.sh.ready) < p.sh.h.num_seqs) {
+          if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+            set_status(p.status, NGRAM_STATUS_TIMEOUT);
+            *abort_flag = 1;
+            go = 0;
+            break;
+          }
+          __nanosleep(64);
+        }
+        __threadfence();
+        if (atomicAdd(p.sh.passed, 1) == static_cast<int>(gridDim.x) - 1) {  // the last CTA re-arms
+          *p.sh.ready = 0;
+          *p.sh.passed = 0;
+        }
+        *reinterpret_cast<volatile int*>(tmem_slot + 2) = go;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // the gather warps
+    }
+    const bool go = !fused || *reinterpret_cast<volatile int*>(tmem_slot + 2) != 0;
+    auto ld_idx = [&](const int32_t* q) { return fused ? ld_cg_b32(q) : ld_idx_early(q); };
     // raw row indices of the current and the next run: cp.async rows, then TMA rows
     int32_t raw[8], nraw[8];
     auto load_raw = [&](const SRun& r, int32_t (&dst)[8]) {
@@ -323,14 +371,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t g1 = row_base + p.tma_rows + rsub + 32 * j;
-        dst[j] = (j < n_cp && g1 < T) ? ld_idx_early(p.idx + g1 * p.S + r.s) : 0;
+        dst[j] = (j < n_cp && g1 < T) ? ld_idx(p.idx + g1 * p.S + r.s) : 0;
         const int64_t g2 = row_base + issuer * 4 + j;
-        dst[4 + j] = (tma_issuer && g2 < T) ? ld_idx_early(p.idx + g2 * p.S + r.s) : 0;
+        dst[4 + j] = (tma_issuer && g2 < T) ? ld_idx(p.idx + g2 * p.S + r.s) : 0;
       }
     };
     int stage = 0;
     uint32_t phase = 0;
-    bool ok = true;
+    bool ok = go;
     const Seg g0 = seg_first(wp, blockIdx.x);
     SRun cur = srun_at(g0, g0.i0, p.num_n_blocks, KB, kb_per_sub);
     if (cur.g.tile < num_tiles) load_raw(cur, raw);
@@ -424,6 +472,22 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       // Everything issued must complete before TMEM is released.
       umma_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0, 100ull * 1000 * 1000);
+    }
+  } else if (warp < kWarpEpi0) {
+    // ------------------------------------------------------------ warps 10-11: a fused
+    // decode step's commit and hashing, sequences blockIdx.x * 2 + (warp - 10), + 2 * grid
+    if (p.sh.on) {
+      int done = 0;
+      for (int32_t b = static_cast<int32_t>(blockIdx.x) * 2 + (warp - 10); b < p.sh.h.num_seqs;
+           b += 2 * static_cast<int32_t>(gridDim.x)) {
+        if (!commit_hash_warp_fast(p.sh.c, p.sh.h, b, lane)) commit_hash_warp(p.sh.c, p.sh.h, b, lane);
+        ++done;
+      }
+      __syncwarp();
+      if (lane == 0 && done) {
+        __threadfence();
+        atomicAdd(p.sh.ready, done);
+      }
     }
   } else if (warp >= kWarpEpi0) {
     // ------------------------------------------------------------ epilogue

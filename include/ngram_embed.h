@@ -387,6 +387,21 @@ int ngram_embed_plan_set_pair_wide(ngram_embed_plan* plan, int on);
  * as dense TMA boxes of G; negative on bad arguments. */
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens);
 
+/* ngram_embed_fwd_step in one launch (on request): where the step's projection runs the
+ * one-CTA tensor-core form and S <= 8, two otherwise idle warps of every CTA of that
+ * projection commit the previous step's ids and hash this step's (Eq. 2 of "Scaling
+ * Embeddings Outperforms Scaling Experts in Language Models", section 2, over the N-gram
+ * cache of section 4.2) for a share of the sequences, with the same code as the separate
+ * commit + hash launch, and the gather warps start once every sequence is done. The launch is
+ * cooperative (all CTAs resident, one per SM); the wait is bounded (TIMEOUT status). Outputs,
+ * indices (in the workspace), ring and status bits are those of the two-launch step. It
+ * counts sequences and CTAs in the workspace's status header (zero between calls;
+ * ngram_embed_clear_status re-arms them after a TIMEOUT). 1 = on; 0 = the separate commit +
+ * hash launch (default: measured on B200 at the 1280-token decode step, D = 4096, in graphs
+ * of 200 steps: 64.4 us in one launch against 62.6 us in two; the hash's latency then sits
+ * at the head of every CTA's main loop). NGRAM_ERR_INVALID_ARG for other values. */
+int ngram_embed_plan_set_fused_step(ngram_embed_plan* plan, int on);
+
 /* CTA-pair form over column ranges (Eq. 3 of "Scaling Embeddings Outperforms Scaling Experts
  * in Language Models", section 2, partitioned by output columns): the pairs are spread evenly
  * over the 256-token row blocks and each pair computes the full sum over K for a contiguous

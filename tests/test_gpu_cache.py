@@ -192,11 +192,13 @@ def test_evicted_context_is_flagged(ne):
     assert ne.status_names(ne.ngram_embed_get_status(ws)) == ["EVICTED"]
 
 
-@pytest.mark.parametrize("dense_a", [0, 1])
-def test_fused_commit_and_step_equals_separate_calls(ne, dense_a):
+@pytest.mark.parametrize("form", ["cta_pair", "cta_pair_dense", "one_cta", "one_cta_stream_k", "one_cta_2_launches"])
+def test_fused_commit_and_step_equals_separate_calls(ne, form):
     """ngram_embed_fwd_step (commit of the previous step fused with this step's hashing; with
-    the dense-A form also with the sub-row gather into G, one launch) gives the same outputs,
-    bit for bit, the same indices and the same ring as ngram_cache_commit + ngram_embed_fwd."""
+    the dense-A form also with the sub-row gather into G; with the one-CTA forms hashed inside
+    the projection and committed by its last CTA, one launch) gives the same outputs, bit for
+    bit, the same indices and the same ring as ngram_cache_commit + ngram_embed_fwd."""
+    dense_a = int(form == "cta_pair_dense")
     from tests.helpers import host_tables, to_device
     N, K, D, B, P, C = 3, 2, 512, 24, 5, 8
     V0, V = 3000, [4099, 5003, 6007, 7001]
@@ -205,7 +207,13 @@ def test_fused_commit_and_step_equals_separate_calls(ne, dense_a):
     E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
     plan = ne.ngram_embed_plan_create(V0, D, N, K, V, ne.NGRAM_BF16)
     ne.ngram_embed_plan_set_dense_a(plan, dense_a)
-    assert ne.ngram_embed_plan_kernel_form(plan, B * P) == ("cta_pair_dense" if dense_a else "cta_pair")
+    if form.startswith("one_cta"):
+        ne.ngram_embed_plan_set_cta_pair(plan, 0)
+        ne.ngram_embed_plan_set_stream_k(plan, 1 if form == "one_cta_stream_k" else 2)
+        if form == "one_cta_stream_k":
+            ne.ngram_embed_plan_set_sm_count(plan, 6)  # 16 units over 6 CTAs: tiles split
+    ne.ngram_embed_plan_set_fused_step(plan, form in ("one_cta", "one_cta_stream_k"))
+    assert ne.ngram_embed_plan_kernel_form(plan, B * P) == form.replace("_2_launches", "")
     ws1, ws2 = ne.new_workspace(plan, B * P), ne.new_workspace(plan, B * P)
     c1, c2 = ne.Cache.empty(B, C), ne.Cache.empty(B, C)
     for c, w in ((c1, ws1), (c2, ws2)):
@@ -232,9 +240,11 @@ def test_fused_commit_and_step_equals_separate_calls(ne, dense_a):
     assert ne.ngram_embed_get_status(ws1) == 0 and ne.ngram_embed_get_status(ws2) == 0
 
 
-def test_fused_step_edge_cases_match_separate_calls(ne):
-    """The fused step's per-sequence path (loads in three rounds, committed ids taken from the
-    commit buffer) against ngram_cache_commit + ngram_embed_fwd where it matters: a sequence
+@pytest.mark.parametrize("one_cta", [False, True], ids=["commit_hash_kernel", "in_projection"])
+def test_fused_step_edge_cases_match_separate_calls(ne, one_cta):
+    """The fused step's per-sequence paths (commit_hash_kernel: loads in three rounds; one-CTA
+    projection: windows hashed by its gather warps, commit by its last CTA; committed ids taken
+    from the commit buffer) against ngram_cache_commit + ngram_embed_fwd where it matters: a sequence
     of 40 ids (more than a warp's lanes: the one-load-at-a-time path), empty sequences,
     nothing to commit, a count above the stride (BAD_APPEND), an id outside the vocabulary
     in the commit buffer (BAD_TOKEN: that entry is not committed), and a history cut by
@@ -246,6 +256,12 @@ def test_fused_step_edge_cases_match_separate_calls(ne):
     E0h, Eh, Wh = host_tables(cfg)
     E0, E, W = to_device(E0h, torch.bfloat16), [to_device(e, torch.bfloat16) for e in Eh], to_device(Wh, torch.bfloat16)
     plan = ne.ngram_embed_plan_create(V0, D, N, K, V, ne.NGRAM_BF16)
+    if one_cta:
+        ne.ngram_embed_plan_set_cta_pair(plan, 0)
+        ne.ngram_embed_plan_set_stream_k(plan, 1)
+        ne.ngram_embed_plan_set_sm_count(plan, 4)  # 18 units over 4 CTAs
+        ne.ngram_embed_plan_set_fused_step(plan, True)
+        assert ne.ngram_embed_plan_kernel_form(plan, 52) == "one_cta_stream_k"
     lengths = [1, 40, 0, 6, 3, 2]
     off_h = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
     T = int(off_h[-1])

@@ -64,6 +64,9 @@ def test_decode_1000_steps_through_the_ring(ne, cfg):
     E0, E, W = device_tables(cfg)
     Wh = host_W(cfg)
     plan = ne.ngram_embed_plan_create(cfg.V0, cfg.D, cfg.N, cfg.K, cfg.V_nk, ne.NGRAM_BF16)
+    # the spec-decode run takes the step in one launch (commit and hashing inside the one-CTA
+    # projection), the full-scale run the default two
+    ne.ngram_embed_plan_set_fused_step(plan, cfg is configs.SPEC_DECODE)
     ws = ne.new_workspace(plan, T)
     cache = ne.Cache.empty(B, C)
     ne.ngram_cache_reset(plan, cache, ws)
