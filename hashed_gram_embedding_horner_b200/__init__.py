@@ -48,7 +48,7 @@ EXPORTED = [
     "ngram_hash_stats_workspace_bytes", "ngram_hash_stats",
     "ngram_draft_cache_reset", "ngram_embed_draft_workspace_bytes", "ngram_embed_fwd_draft",
     "ngram_embed_fwd_step", "ngram_embed_plan_set_dense_a", "ngram_embed_plan_set_pair_columns",
-    "ngram_embed_plan_set_fused_step",
+    "ngram_embed_plan_set_fused_step", "ngram_embed_plan_set_backward_pair",
 ]
 
 
@@ -92,6 +92,7 @@ _sig("ngram_embed_plan_set_cta_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pair_wide", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_dense_a", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pair_columns", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_backward_pair", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_fused_step", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_sm_count", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
@@ -270,6 +271,11 @@ def ngram_embed_plan_set_pair_columns(plan: Plan, on):
     """True/1: the pair form over column ranges whenever possible; False/0: never; None/-1: automatic."""
     v = -1 if on is None or on == -1 else int(bool(on))
     _check(_lib.ngram_embed_plan_set_pair_columns(plan.handle, v), "ngram_embed_plan_set_pair_columns")
+
+
+def ngram_embed_plan_set_backward_pair(plan: Plan, on: bool):
+    """The backward's GEMMs on CTA pairs (True, default) or one CTA per 128-row tile (False)."""
+    _check(_lib.ngram_embed_plan_set_backward_pair(plan.handle, int(bool(on))), "ngram_embed_plan_set_backward_pair")
 
 
 def ngram_embed_plan_set_sm_count(plan: Plan, sms: int):

@@ -443,4 +443,251 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+
+// CTA-pair form of the dense GEMM (tcgen05.mma.cta_group::2, M = 256): the pair computes a
+// 256 x BN tile; each CTA loads its 128 rows of A and BN/2 rows of B per stage (2-D TMA in
+// the .cta_group::2 form, byte counts completing on CTA 0's stage barrier), one thread of CTA 0
+// issues the MMAs and commits stage releases and "accumulator ready" to both CTAs, and each
+// CTA's epilogue drains its 128 accumulator rows as the one-CTA kernel does (CTA 1's warps
+// free the accumulator by remote arrivals on CTA 0's barrier). Per SM and k-block it loads
+// 16 KB of A + BN/2 x 128 B of B for the same FLOPs the one-CTA kernel needs 16 KB + BN x
+// 128 B for.
+template <int BN, int STAGES>
+struct DensePairSmem {
+  static constexpr int kABytes = kBM * kBK * 2;           // this CTA's 128 rows of A
+  static constexpr int kBBytes = (BN / 2) * kBK * 2;      // this CTA's BN/2 rows of B
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kEpiOffset = (kBarOffset + kNumBars * 8 + 16 + 127) / 128 * 128;
+  static constexpr int kBytes = kEpiOffset + 4 * 32 * 32 * 4;
+  static constexpr int kLaunchBytes = kBytes + 1024;
+  static constexpr int kTmemCols = 2 * BN;
+  static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of 128-byte swizzling");
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    dense_gemm_pair_kernel(const __grid_constant__ DenseMaps maps, const __grid_constant__ DenseParams p) {
+  using L = DensePairSmem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBarOffset;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + L::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto a_tile = [&](int s) { return sbase + s * L::kStageBytes; };
+  auto b_tile = [&](int s) { return sbase + s * L::kStageBytes + L::kABytes; };
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs and owns the stage barriers
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int num_pairs = static_cast<int>(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1u);   // CTA 0: its producer's byte count for both CTAs (CTA 1's: unused)
+      mbar_init(empty_bar(s), 1u);  // one tcgen05.commit from CTA 0's MMA thread
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1u);
+      mbar_init(tempty_bar(a), 128u + 4u);  // CTA 0's epilogue threads + one remote arrive per CTA 1 warp
+    }
+    mbar_init(drain_bar, 1u);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.A);
+    tma_prefetch_desc(&maps.B);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
+
+  const int num_units = p.num_m_blocks * p.num_n_blocks * p.splits;  // m blocks of 256 rows
+  auto unit_k = [&](int u, int& kb0, int& kb1) {
+    const int ks = u % p.splits;
+    kb0 = ks * p.kb_per_split;
+    kb1 = kb0 + p.kb_per_split < p.num_k_blocks ? kb0 + p.kb_per_split : p.num_k_blocks;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (own rows)
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = pair; u < num_units && ok; u += num_pairs) {
+        const int tile = u / p.splits;
+        const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
+        const int row_a = m_blk * (2 * kBM) + static_cast<int>(rank) * kBM;
+        const int row_b = n_blk * BN + static_cast<int>(rank) * (BN / 2);
+        int kb0, kb1;
+        unit_k(u, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          const uint32_t full0 = map_to_cta(full_bar(stage), 0);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2u * L::kStageBytes);
+          if (p.a_mn) {
+#pragma unroll
+            for (int j = 0; j < kBM / 64; ++j)
+              tma_load_2d_pair(a_tile(stage) + j * 8192, &maps.A, row_a + j * 64, kb * kBK, full0, pol);
+          } else {
+            tma_load_2d_pair(a_tile(stage), &maps.A, kb * kBK, row_a, full0, pol);
+          }
+          if (p.b_mn) {
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              tma_load_2d_pair(b_tile(stage) + j * 8192, &maps.B, row_b + j * 64, kb * kBK, full0, pol);
+          } else {
+            tma_load_2d_pair(b_tile(stage), &maps.B, kb * kBK, row_b, full0, pol);
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {  // aborting: the loads in flight land (bounded) before exit
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 1000ull * 1000ull) __nanosleep(1000);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (CTA 0)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = umma_idesc_bf16(2 * kBM, BN) | (p.a_mn ? 1u << 15 : 0u) | (p.b_mn ? 1u << 16 : 0u);
+      const uint32_t a_step = p.a_mn ? 2048u >> 4 : 32u >> 4;  // K += 16 in the descriptor's address field
+      const uint32_t b_step = p.b_mn ? 2048u >> 4 : 32u >> 4;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int u = pair; u < num_units && ok; u += num_pairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!mbar_wait_cluster(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        int kb0, kb1;
+        unit_k(u, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = p.a_mn ? sw128_mnmajor_desc(a_tile(stage)) : sw128_kmajor_desc(a_tile(stage));
+          const uint64_t bdesc = p.b_mn ? sw128_mnmajor_desc(b_tile(stage)) : sw128_kmajor_desc(b_tile(stage));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, (kb > kb0 || k != 0) ? 1u : 0u);
+          umma_commit_pair(map_to_cta(empty_bar(stage), 0));
+          umma_commit_pair(map_to_cta(empty_bar(stage), 1));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) {
+          umma_commit_pair(map_to_cta(tfull_bar(acc), 0));
+          umma_commit_pair(map_to_cta(tfull_bar(acc), 1));
+        }
+      }
+      umma_commit_pair(map_to_cta(drain_bar, 0));
+      mbar_wait_drain(drain_bar, 0, 100ull * 1000 * 1000);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue: atomic adds
+    // As in the one-CTA kernel (staged 32 x 32 chunks, eight lanes per row for the fp32
+    // reductions), for this CTA's 128 rows of the pair's tile.
+    const int q = warp & 3;
+    const uint32_t stg = sbase + L::kEpiOffset + static_cast<uint32_t>(q) * 4096u;
+    const uint32_t row_w = stg + static_cast<uint32_t>(lane) * 128u;
+    const int wv = lane & 7;
+    const int rq = lane >> 3;
+    const uint32_t tempty_remote0 = map_to_cta(tempty_bar(0), 0);
+    const uint32_t tempty_remote1 = map_to_cta(tempty_bar(1), 0);
+    int local = 0;
+    for (int u = pair; u < num_units; u += num_pairs, ++local) {
+      const int tile = u / p.splits;
+      const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
+      const int acc = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const int64_t row0 = static_cast<int64_t>(m_blk) * (2 * kBM) + rank * kBM + q * 32;  // this warp's first row
+      bool got = false;
+      if (lane == 0) got = mbar_wait_cluster(tfull_bar(acc), use & 1u, abort_flag, p.status);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      int s_cur = -1;
+      int32_t my_target = 0;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, v);
+        tmem_wait_ld();
+        if (c + 1 == BN / 32) {
+          tc_fence_before();
+          if (rank == 0) {
+            mbar_arrive(tempty_bar(acc));
+          } else {
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acc ? tempty_remote1 : tempty_remote0);
+          }
+        }
+        const int col0 = n_blk * BN + c * 32;
+        const int s = p.epi == kEpiScatterSub ? col0 / p.d : 0;  // 32 columns never straddle two sub-tables
+        if (p.epi == kEpiScatterSub && s != s_cur) {
+          s_cur = s;
+          my_target = 0;
+          if (row0 + lane < p.M) {
+            my_target = p.idx[(row0 + lane) * p.S + s];
+            if (static_cast<uint32_t>(my_target) >= p.Vs[s]) {
+              set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+              my_target = 0;
+            }
+          }
+        }
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+          st_shared_v4(row_w + (static_cast<uint32_t>(w ^ (lane & 7)) << 4),
+                       make_uint4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]));
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = i * 4 + rq;
+          const uint4 x = ld_shared_v4(stg + static_cast<uint32_t>(r) * 128u + (static_cast<uint32_t>(wv ^ (r & 7)) << 4));
+          const int32_t target = __shfl_sync(0xffffffffu, my_target, r);
+          const int64_t grow = row0 + r;
+          if (grow < p.M) {
+            float* dst = p.epi == kEpiScatterSub
+                             ? p.dE[s] + static_cast<int64_t>(target) * p.d + (col0 - s * p.d) + wv * 4
+                             : p.out + grow * p.N + col0 + wv * 4;
+            atomicAdd(reinterpret_cast<float4*>(dst),
+                      make_float4(__uint_as_float(x.x) * p.scale, __uint_as_float(x.y) * p.scale,
+                                  __uint_as_float(x.z) * p.scale, __uint_as_float(x.w) * p.scale));
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no remote arrive or pair MMA is outstanding past this point
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, L::kTmemCols);
+  }
+}
+
 }  // namespace ngram

@@ -74,9 +74,10 @@ struct ngram_embed_plan {
   int dense_a = 0;             // sub-rows gathered into G first, A by dense TMA: 1 on, 0 off
   const void* map_A = nullptr;  // the dense-A map's pointer and row count
   int64_t map_A_T = -1;
-  int max_clusters[5] = {0, 0, 0, 0, 0};  // co-resident CTA pairs, per kernel instance (0 = not queried)
+  int max_clusters[7] = {};    // co-resident CTA pairs, per kernel instance (0 = not queried)
   int pair_cols = 0;           // pair form over column ranges: 1 whenever possible, 0 off
   int fused_step = 0;          // decode step committed and hashed inside the one-CTA projection
+  int bwd_pair = 1;            // backward GEMMs: 1 CTA pairs (M = 256 tiles), 0 one CTA per 128-row tile
 };
 
 namespace {
@@ -526,6 +527,77 @@ int launch_dense_gemm(ngram_embed_plan* p, DenseParams prm, GemmOperand A, GemmO
   return launch(kern, dim3(grid), dim3(kGemmThreads), L::kLaunchBytes, st, p->pdl, 1, maps, prm);
 }
 
+// CTA-pair form of the same GEMM: 256-row tiles, each CTA of a pair loading its 128 rows of A
+// and half of B's BN rows per stage; units (tile, k range) strided over the co-resident pairs.
+constexpr int kBwdPairStages256 = 6;  // x (16 KB A + 16 KB B)
+constexpr int kBwdPairStages128 = 8;  // x (16 KB A + 8 KB B)
+
+template <int BN>
+int launch_dense_gemm_pair(ngram_embed_plan* p, DenseParams prm, GemmOperand A, GemmOperand B, int64_t K, bool split,
+                           cudaStream_t st) {
+  constexpr int STAGES = BN == 256 ? kBwdPairStages256 : kBwdPairStages128;
+  using L = DensePairSmem<BN, STAGES>;
+  auto kern = dense_gemm_pair_kernel<BN, STAGES>;
+  const int key = BN == 256 ? 14 : 15;
+  if (!p->smem_attr_set[key]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess)
+      return NGRAM_ERR_CUDA;
+    p->smem_attr_set[key] = true;
+  }
+  auto encode = [&](CUtensorMap* m, const GemmOperand& o, uint32_t box_rows) {
+    return o.mn ? encode_2d(m, o.base, static_cast<uint64_t>(o.rows), static_cast<uint64_t>(K),
+                            static_cast<uint64_t>(o.rows) * 2, 64, 64, CU_TENSOR_MAP_L2_PROMOTION_L2_256B)
+                : encode_2d(m, o.base, static_cast<uint64_t>(K), static_cast<uint64_t>(o.rows),
+                            static_cast<uint64_t>(K) * 2, kBK, box_rows, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  };
+  DenseMaps maps;
+  int rc = encode(&maps.A, A, kBM);
+  if (rc) return rc;
+  if ((rc = encode(&maps.B, B, BN / 2))) return rc;
+  prm.a_mn = A.mn ? 1 : 0;
+  prm.b_mn = B.mn ? 1 : 0;
+  prm.M = static_cast<int>(A.rows);
+  prm.N = static_cast<int>(B.rows);
+  prm.num_m_blocks = static_cast<int>((A.rows + 2 * kBM - 1) / (2 * kBM));
+  prm.num_n_blocks = static_cast<int>(B.rows / BN);
+  prm.num_k_blocks = static_cast<int>((K + kBK - 1) / kBK);
+  int& max_pairs = p->max_clusters[BN == 256 ? 5 : 6];
+  if (max_pairs == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (p->sms / 2));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = L::kLaunchBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return NGRAM_ERR_CUDA;
+    max_pairs = n;
+  }
+  const int pairs_avail = max_pairs < p->sms / 2 ? max_pairs : p->sms / 2;
+  if (pairs_avail < 1) return NGRAM_ERR_CUDA;
+  const int tiles = prm.num_m_blocks * prm.num_n_blocks;
+  const int s = split ? choose_splits(tiles, prm.num_k_blocks, pairs_avail) : 1;
+  prm.kb_per_split = (prm.num_k_blocks + s - 1) / s;
+  prm.splits = (prm.num_k_blocks + prm.kb_per_split - 1) / prm.kb_per_split;  // every split non-empty
+  const int units = tiles * prm.splits;
+  const int pairs = units < pairs_avail ? units : pairs_avail;
+  return launch(kern, dim3(2 * pairs), dim3(kGemmThreads), L::kLaunchBytes, st, p->pdl, 2, maps, prm);
+}
+
+// The backward's GEMMs in the plan's form (pairs need an even SM budget of at least 2).
+template <int BN>
+int launch_bwd_gemm(ngram_embed_plan* p, const DenseParams& prm, GemmOperand A, GemmOperand B, int64_t K, bool split,
+                    cudaStream_t st) {
+  if (p->bwd_pair == 1 && p->sms >= 2) return launch_dense_gemm_pair<BN>(p, prm, A, B, K, split, st);
+  return launch_dense_gemm<BN>(p, prm, A, B, K, split, st);
+}
+
 int validate_common(const ngram_embed_plan* p, void* ws, size_t ws_size, int64_t T) {
   if (!p || !ws || T < 0 || T > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
   if (!aligned16(ws)) return NGRAM_ERR_MISALIGNED;
@@ -924,6 +996,12 @@ int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_token
   return choose_form(plan, num_tokens, ws_bytes(plan, num_tokens), num_tokens, false);
 }
 
+int ngram_embed_plan_set_backward_pair(ngram_embed_plan* plan, int on) {
+  if (!plan || on < 0 || on > 1) return NGRAM_ERR_INVALID_ARG;
+  plan->bwd_pair = on;
+  return NGRAM_OK;
+}
+
 int ngram_embed_plan_set_fused_step(ngram_embed_plan* plan, int on) {
   if (!plan || on < 0 || on > 1) return NGRAM_ERR_INVALID_ARG;
   plan->fused_step = on;
@@ -1263,8 +1341,8 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     dp.d = p->d;
     dp.status = status_ptr(workspace);
     const GemmOperand A{g, T, false}, B{W_stacked, D, true};
-    if ((rc = p->D % 256 == 0 ? launch_dense_gemm<256>(p, dp, A, B, D, false, st)
-                              : launch_dense_gemm<128>(p, dp, A, B, D, false, st)))
+    if ((rc = p->D % 256 == 0 ? launch_bwd_gemm<256>(p, dp, A, B, D, false, st)
+                              : launch_bwd_gemm<128>(p, dp, A, B, D, false, st)))
       return rc;
   }
   if (dW) {
@@ -1278,8 +1356,8 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     dp.out = dW;
     dp.status = status_ptr(workspace);
     const GemmOperand A{g, D, true}, B{G, D, true};
-    if ((rc = p->D % 256 == 0 ? launch_dense_gemm<256>(p, dp, A, B, T, true, st)
-                              : launch_dense_gemm<128>(p, dp, A, B, T, true, st)))
+    if ((rc = p->D % 256 == 0 ? launch_bwd_gemm<256>(p, dp, A, B, T, true, st)
+                              : launch_bwd_gemm<128>(p, dp, A, B, T, true, st)))
       return rc;
   }
   return NGRAM_OK;

@@ -402,6 +402,15 @@ int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_token
  * at the head of every CTA's main loop). NGRAM_ERR_INVALID_ARG for other values. */
 int ngram_embed_plan_set_fused_step(ngram_embed_plan* plan, int on);
 
+/* Form of the backward pass's two dense GEMMs (dG = c g W_stacked and dW = c g^T G, the
+ * gradients of Eq. 3 of "Scaling Embeddings Outperforms Scaling Experts in Language Models",
+ * section 2): 1 = CTA pairs (tcgen05.mma.cta_group::2, 256-row tiles; each CTA of a pair
+ * loads its 128 rows of A and half of B per k-block; default), 0 = one CTA per 128-row tile.
+ * Pairs need a plan SM budget of at least 2 (otherwise the one-CTA form runs). A tuning knob:
+ * results agree within the stated tolerance (the fp32 atomic-add order differs).
+ * NGRAM_ERR_INVALID_ARG for other values or a null plan. */
+int ngram_embed_plan_set_backward_pair(ngram_embed_plan* plan, int on);
+
 /* CTA-pair form over column ranges (Eq. 3 of "Scaling Embeddings Outperforms Scaling Experts
  * in Language Models", section 2, partitioned by output columns): the pairs are spread evenly
  * over the 256-token row blocks and each pair computes the full sum over K for a contiguous

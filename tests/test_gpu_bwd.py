@@ -55,8 +55,11 @@ def small_problem(D=1024, N=3, K=2, V=(211, 223, 227, 229), V0=300, lengths=(1, 
     return dict(V0=V0, D=D, N=N, K=K, V=list(V), S=S, d=d, tok=tok, off=off, E=E, W=W, g=g, T=T)
 
 
-def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1):
+def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=True, sms=0):
     plan = ne.ngram_embed_plan_create(P["V0"], P["D"], P["N"], P["K"], P["V"], ne.NGRAM_BF16)
+    ne.ngram_embed_plan_set_backward_pair(plan, pair)
+    if sms:
+        ne.ngram_embed_plan_set_sm_count(plan, sms)
     if scale != 1.0:
         ne.ngram_embed_plan_set_output_scale(plan, scale)
     ws = ne.new_workspace(plan, P["T"])
@@ -82,9 +85,13 @@ def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1):
                                    dict(D=384, N=2, K=3, V=(61, 67, 71)),
                                    dict(lengths=(4096,), V=(4099, 5003, 6007, 7001), V0=131072)],
                          ids=["D1024_ragged", "D2048_dense_collisions", "D1536_N4", "D384_tile128", "T4096_wide_V"])
-def test_backward_matches_oracle(ne, shape):
+@pytest.mark.parametrize("form", [dict(pair=True), dict(pair=False), dict(pair=True, sms=4), dict(pair=True, sms=5)],
+                         ids=["pairs", "one_cta", "pairs_2", "pairs_odd_sms"])
+def test_backward_matches_oracle(ne, shape, form):
+    """Both GEMM forms; with 2 pairs (4 or 5 SMs) each pair runs many (tile, k range) units
+    through both accumulators."""
     P = small_problem(**shape)
-    dE0, dE, dW = run_bwd(ne, P, scale=3.0)
+    dE0, dE, dW = run_bwd(ne, P, scale=3.0, **form)
     w0, wE, wW = oracle.backward(P["V0"], P["D"], P["N"], P["K"], P["V"], P["tok"], P["off"], P["E"], P["W"],
                                  P["g"], scale=3.0)
     close(dE0, w0, "dE0")
@@ -97,16 +104,26 @@ def test_backward_matches_oracle(ne, shape):
     assert not dE0[~touched].any()
 
 
-def test_backward_accumulates_and_skips(ne):
-    """+= semantics (two calls give twice the gradient) and NULL gradients are skipped."""
+@pytest.mark.parametrize("pair", [True, False], ids=["pairs", "one_cta"])
+def test_backward_accumulates_and_skips(ne, pair):
+    """+= semantics (two calls give twice the gradient) and NULL gradients are skipped; a
+    single token (CTA 1 of the pair reads rows past the end only)."""
     P = small_problem(lengths=(64, 65))
-    once = run_bwd(ne, P)
-    twice = run_bwd(ne, P, repeat=2)
+    once = run_bwd(ne, P, pair=pair)
+    twice = run_bwd(ne, P, repeat=2, pair=pair)
     close(twice[0], 2 * once[0].astype(np.float64), "2 dE0")
     close(twice[2], 2 * once[2].astype(np.float64), "2 dW")
-    only_w = run_bwd(ne, P, which=("W",))
+    only_w = run_bwd(ne, P, which=("W",), pair=pair)
     assert only_w[0] is None and only_w[1] is None
     close(only_w[2], once[2].astype(np.float64), "dW alone")
+    P1 = small_problem(lengths=(1,))
+    dE0, dE, dW = run_bwd(ne, P1, pair=pair)
+    w0, wE, wW = oracle.backward(P1["V0"], P1["D"], P1["N"], P1["K"], P1["V"], P1["tok"], P1["off"], P1["E"],
+                                 P1["W"], P1["g"])
+    close(dE0, w0, "dE0 T=1")
+    for s in range(P1["S"]):
+        close(dE[s], wE[s], f"dE[{s}] T=1")
+    close(dW, wW, "dW T=1")
 
 
 def test_backward_full_tables_sampled(ne):
