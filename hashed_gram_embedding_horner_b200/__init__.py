@@ -273,9 +273,10 @@ def ngram_embed_plan_set_pair_columns(plan: Plan, on):
     _check(_lib.ngram_embed_plan_set_pair_columns(plan.handle, v), "ngram_embed_plan_set_pair_columns")
 
 
-def ngram_embed_plan_set_backward_pair(plan: Plan, on: bool):
-    """The backward's GEMMs on CTA pairs (True, default) or one CTA per 128-row tile (False)."""
-    _check(_lib.ngram_embed_plan_set_backward_pair(plan.handle, int(bool(on))), "ngram_embed_plan_set_backward_pair")
+def ngram_embed_plan_set_backward_pair(plan: Plan, mode):
+    """The backward's GEMMs: True/1 CTA pairs with 256-column tiles (default); 2 pairs with
+    512-column tiles where D allows; False/0 one CTA per 128-row tile."""
+    _check(_lib.ngram_embed_plan_set_backward_pair(plan.handle, int(mode)), "ngram_embed_plan_set_backward_pair")
 
 
 def ngram_embed_plan_set_sm_count(plan: Plan, sms: int):

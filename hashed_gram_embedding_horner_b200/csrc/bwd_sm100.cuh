@@ -28,8 +28,11 @@ namespace ngram {
 // dE0[v] += c * sum_{i : t_i = v} g_i. Token streams repeat ids heavily (Zipf: the commonest
 // id is ~10 % of a batch), so adding each row atomically into dE0 would serialise on the
 // hot rows. Instead: a counting sort of the positions by token id (histogram, exclusive scan
-// over V0, scatter), then each warp sums a run of kSegRows consecutive sorted positions and
-// adds one partial row per distinct id in its run — a hot id costs one add per run.
+// over V0, placement), then each warp sums a run of kSegRows consecutive sorted positions and
+// adds one partial row per distinct id in its run — a hot id costs one add per run. The
+// histogram and the placement aggregate equal ids within a warp first (one atomic per
+// distinct id per warp), which keeps the hot ids' counters from serialising tens of
+// thousands of atomics on one address.
 
 constexpr int kSegRows = 16;
 
@@ -41,11 +44,12 @@ struct ScatterE0Params {
   int D;
   uint32_t V0;
   float scale;
-  int32_t* counts;     // [V0 + 1]: histogram, then exclusive prefix (bin starts)
-  int32_t* cursor;     // [V0]: fill positions
+  int32_t* counts;     // [V0 + 1], zero on entry: histogram, then each bin's start within its
+                       // 1024-bin block, then (advanced by the placement) its end; counts[V0]
+                       // is the scan's block ticket
   int32_t* order;      // [T]: positions sorted by token id
   int32_t* sorted_tok; // [T]: their ids
-  int32_t* block_sums; // [num_blocks]: scan totals of 1024-bin blocks, then their prefixes
+  int32_t* block_sums; // [num_blocks]: totals of 1024-bin blocks, then their exclusive prefixes
   int num_blocks;
   int* status;
 };
@@ -59,14 +63,21 @@ __device__ __forceinline__ uint32_t e0_token(const ScatterE0Params& p, int64_t i
   return static_cast<uint32_t>(t);
 }
 
-__global__ void __launch_bounds__(256) e0_hist_kernel(const __grid_constant__ ScatterE0Params p) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < p.T) atomicAdd(p.counts + e0_token(p, i), 1);
+// Position i's id, or 0xFFFFFFFF past the end (never equal to an id: V0 < 2^31).
+__device__ __forceinline__ uint32_t e0_token_or_none(const ScatterE0Params& p, int64_t i) {
+  return i < p.T ? e0_token(p, i) : 0xFFFFFFFFu;
 }
 
-// Exclusive scan of counts[0..V0) in place, in three launches: each block of 1024 bins
-// scans itself and records its total; one block scans the totals (in chunks of 1024 when
-// there are more); each block adds its prefix.
+__global__ void __launch_bounds__(256) e0_hist_kernel(const __grid_constant__ ScatterE0Params p) {
+  pdl_wait();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const uint32_t t = e0_token_or_none(p, i);
+  const uint32_t peers = __match_any_sync(0xffffffffu, t);  // lanes holding the same id
+  if (i < p.T && lane == __ffs(peers) - 1) atomicAdd(p.counts + t, __popc(peers));
+}
+
+// Exclusive scan of a block's values (one per thread, up to 1024 threads).
 __device__ __forceinline__ int32_t block_exclusive_scan(int32_t c, int32_t* warp_sums, int32_t& total) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   int32_t x = c;
@@ -93,51 +104,62 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t c, int32_t* warp
   return r;
 }
 
-__global__ void __launch_bounds__(1024) e0_scan_blocks_kernel(const __grid_constant__ ScatterE0Params p) {
+// Each block of 1024 bins scans itself in place and records its total; the block that
+// finishes last (a ticket counter) then scans the totals into exclusive block prefixes, in
+// chunks of 1024. No block waits for another.
+__global__ void __launch_bounds__(1024) e0_scan_kernel(const __grid_constant__ ScatterE0Params p) {
+  pdl_wait();
   __shared__ int32_t warp_sums[32];
+  __shared__ int is_last;
   const int64_t b = static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x;
   const int32_t c = b < p.V0 ? p.counts[b] : 0;
   int32_t total;
   const int32_t ex = block_exclusive_scan(c, warp_sums, total);
   if (b < p.V0) p.counts[b] = ex;
-  if (threadIdx.x == 0) p.block_sums[blockIdx.x] = total;
-}
-
-__global__ void __launch_bounds__(1024) e0_scan_top_kernel(const __grid_constant__ ScatterE0Params p) {
-  __shared__ int32_t warp_sums[32];
-  __shared__ int32_t carry;
-  if (threadIdx.x == 0) carry = 0;
+  if (threadIdx.x == 0) {
+    p.block_sums[blockIdx.x] = total;
+    __threadfence();  // the total is visible before the ticket is taken
+    is_last = atomicAdd(p.counts + p.V0, 1) == static_cast<int>(gridDim.x) - 1;
+  }
   __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  int32_t carry = 0;
   for (int base = 0; base < p.num_blocks; base += 1024) {
     const int k = base + threadIdx.x;
-    const int32_t c = k < p.num_blocks ? p.block_sums[k] : 0;
-    int32_t total;
-    const int32_t ex = block_exclusive_scan(c, warp_sums, total);
-    if (k < p.num_blocks) p.block_sums[k] = carry + ex;
-    __syncthreads();
-    if (threadIdx.x == 0) carry += total;
-    __syncthreads();
+    const int32_t v = k < p.num_blocks ? __ldcg(p.block_sums + k) : 0;
+    int32_t chunk_total;
+    const int32_t e = block_exclusive_scan(v, warp_sums, chunk_total);
+    if (k < p.num_blocks) p.block_sums[k] = carry + e;
+    carry += chunk_total;
   }
 }
 
-__global__ void __launch_bounds__(1024) e0_scan_add_kernel(const __grid_constant__ ScatterE0Params p) {
-  const int64_t b = static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x;
-  if (b < p.V0) p.counts[b] += p.block_sums[blockIdx.x];
-}
-
+// Sorted slot of position i: its bin's start (block-local start + block prefix) plus the
+// count of equal ids placed before it; one atomic per distinct id in the warp advances the
+// bin's cursor (the block-local start in counts).
 __global__ void __launch_bounds__(256) e0_place_kernel(const __grid_constant__ ScatterE0Params p) {
+  pdl_wait();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= p.T) return;
-  const uint32_t t = e0_token(p, i);
-  const int32_t at = p.counts[t] + atomicAdd(p.cursor + t, 1);
-  p.order[at] = static_cast<int32_t>(i);
-  p.sorted_tok[at] = static_cast<int32_t>(t);
+  const int lane = threadIdx.x & 31;
+  const uint32_t t = e0_token_or_none(p, i);
+  const uint32_t peers = __match_any_sync(0xffffffffu, t);
+  const int leader = __ffs(peers) - 1;
+  int32_t base = 0;
+  if (i < p.T && lane == leader) base = atomicAdd(p.counts + t, __popc(peers)) + p.block_sums[t >> 10];
+  base = __shfl_sync(0xffffffffu, base, leader);
+  if (i < p.T) {
+    const int32_t at = base + __popc(peers & ((1u << lane) - 1u));
+    p.order[at] = static_cast<int32_t>(i);
+    p.sorted_tok[at] = static_cast<int32_t>(t);
+  }
 }
 
 // One warp per (run of kSegRows sorted positions, 256 columns): each lane loads its 8
 // columns (16 bytes) of all kSegRows rows first, then sums them in order, adding one
 // partial row into dE0 per distinct id in the run.
 __global__ void __launch_bounds__(256) e0_reduce_kernel(const __grid_constant__ ScatterE0Params p) {
+  pdl_wait();
   const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int chunks = (p.D + 255) / 256;
@@ -192,7 +214,9 @@ struct DenseMaps {
 struct DenseParams {
   int M, N;            // rows of A (tokens, or D) and of B (D)
   int num_m_blocks, num_n_blocks, num_k_blocks;
-  int splits;          // k ranges per tile (split-K): unit u = tile * splits + k range
+  int splits;          // k ranges per tile (split-K): unit u = k range * tiles + tile, so the
+                       // units running at once share their k range (A and B strips reused
+                       // from L2 across the tiles)
   int kb_per_split;
   float scale;
   int epi;             // GemmEpi
@@ -286,9 +310,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_launch_dependents();
   pdl_wait();
 
-  const int num_units = p.num_m_blocks * p.num_n_blocks * p.splits;
+  const int num_tiles = p.num_m_blocks * p.num_n_blocks;
+  const int num_units = num_tiles * p.splits;
   auto unit_k = [&](int u, int& kb0, int& kb1) {
-    const int ks = u % p.splits;
+    const int ks = u / num_tiles;
     kb0 = ks * p.kb_per_split;
     kb1 = kb0 + p.kb_per_split < p.num_k_blocks ? kb0 + p.kb_per_split : p.num_k_blocks;
   };
@@ -301,7 +326,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-        const int tile = u / p.splits;
+        const int tile = u % num_tiles;
         const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
         int kb0, kb1;
         unit_k(u, kb0, kb1);
@@ -376,7 +401,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int rq = lane >> 3;  // read-back: rows i * 4 + rq
     int local = 0;
     for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++local) {
-      const int tile = u / p.splits;
+      const int tile = u % num_tiles;
       const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
@@ -519,9 +544,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_launch_dependents();
   pdl_wait();
 
-  const int num_units = p.num_m_blocks * p.num_n_blocks * p.splits;  // m blocks of 256 rows
+  const int num_tiles = p.num_m_blocks * p.num_n_blocks;  // m blocks of 256 rows
+  const int num_units = num_tiles * p.splits;
   auto unit_k = [&](int u, int& kb0, int& kb1) {
-    const int ks = u % p.splits;
+    const int ks = u / num_tiles;
     kb0 = ks * p.kb_per_split;
     kb1 = kb0 + p.kb_per_split < p.num_k_blocks ? kb0 + p.kb_per_split : p.num_k_blocks;
   };
@@ -534,7 +560,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int u = pair; u < num_units && ok; u += num_pairs) {
-        const int tile = u / p.splits;
+        const int tile = u % num_tiles;
         const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
         const int row_a = m_blk * (2 * kBM) + static_cast<int>(rank) * kBM;
         const int row_b = n_blk * BN + static_cast<int>(rank) * (BN / 2);
@@ -592,13 +618,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
             umma_bf16_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, (kb > kb0 || k != 0) ? 1u : 0u);
-          umma_commit_pair(map_to_cta(empty_bar(stage), 0));
-          umma_commit_pair(map_to_cta(empty_bar(stage), 1));
+          umma_commit_pair_both(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (ok) {
-          umma_commit_pair(map_to_cta(tfull_bar(acc), 0));
-          umma_commit_pair(map_to_cta(tfull_bar(acc), 1));
+          umma_commit_pair_both(tfull_bar(acc));
         }
       }
       umma_commit_pair(map_to_cta(drain_bar, 0));
@@ -617,7 +641,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tempty_remote1 = map_to_cta(tempty_bar(1), 0);
     int local = 0;
     for (int u = pair; u < num_units; u += num_pairs, ++local) {
-      const int tile = u / p.splits;
+      const int tile = u % num_tiles;
       const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
@@ -684,6 +708,279 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // no remote arrive or pair MMA is outstanding past this point
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, L::kTmemCols);
+  }
+}
+
+
+// Wide CTA-pair form: 256 x 512 tiles, the pair's accumulator split in two halves of
+// 256 x 256 (TMEM columns 0-255 and 256-511 of both CTAs), one N = 256 pair MMA per half and
+// k-step. Per SM and k-block it loads 16 KB of A and 32 KB of B (its 128 rows of each half)
+// for twice the FLOPs of the 256 x 256 pair tile, so each stage covers twice the load latency.
+// With one accumulator the next tile's MMAs need the drain out of the way: eight epilogue
+// warps drain half 0 first and free it, then half 1; the MMA thread starts a tile with the
+// half-0 products of its first STAGES k-blocks while half 1 drains, then catches up on half 1.
+template <int STAGES>
+struct DenseWideSmem {
+  static constexpr int kABytes = kBM * kBK * 2;       // this CTA's 128 rows of A
+  static constexpr int kBSubBytes = kBM * kBK * 2;    // this CTA's 128 rows of one half's B
+  static constexpr int kStageBytes = kABytes + 2 * kBSubBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kEpiOffset = (kBarOffset + kNumBars * 8 + 16 + 127) / 128 * 128;
+  static constexpr int kBytes = kEpiOffset + 8 * 32 * 32 * 4;  // eight epilogue warps' staging
+  static constexpr int kLaunchBytes = kBytes + 1024;
+  static constexpr int kTmemCols = 512;
+};
+constexpr int kWideGemmThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4-11 epilogue
+
+template <int STAGES>
+__global__ void __launch_bounds__(kWideGemmThreads, 1)
+    dense_gemm_pair_wide_kernel(const __grid_constant__ DenseMaps maps, const __grid_constant__ DenseParams p) {
+  using L = DenseWideSmem<STAGES>;
+  constexpr int BN = 512;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBarOffset;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int h) { return bar0 + 8u * (2 * STAGES + h); };
+  auto tempty_bar = [&](int h) { return bar0 + 8u * (2 * STAGES + 2 + h); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + L::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto a_tile = [&](int s) { return sbase + s * L::kStageBytes; };
+  auto b_tile = [&](int s, int h) { return sbase + s * L::kStageBytes + L::kABytes + h * L::kBSubBytes; };
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int num_pairs = static_cast<int>(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1u);
+      mbar_init(empty_bar(s), 1u);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(tfull_bar(h), 1u);
+      mbar_init(tempty_bar(h), 256u + 8u);  // CTA 0's 8 epilogue warps + one remote arrive per CTA 1 warp
+    }
+    mbar_init(drain_bar, 1u);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.A);
+    tma_prefetch_desc(&maps.B);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
+
+  const int num_tiles = p.num_m_blocks * p.num_n_blocks;  // 256-row x 512-column tiles
+  const int num_units = num_tiles * p.splits;
+  auto unit_k = [&](int u, int& kb0, int& kb1) {
+    const int ks = u / num_tiles;
+    kb0 = ks * p.kb_per_split;
+    kb1 = kb0 + p.kb_per_split < p.num_k_blocks ? kb0 + p.kb_per_split : p.num_k_blocks;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (own rows)
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = pair; u < num_units && ok; u += num_pairs) {
+        const int tile = u % num_tiles;
+        const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
+        const int row_a = m_blk * (2 * kBM) + static_cast<int>(rank) * kBM;
+        int kb0, kb1;
+        unit_k(u, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          const uint32_t full0 = map_to_cta(full_bar(stage), 0);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2u * L::kStageBytes);
+          if (p.a_mn) {
+#pragma unroll
+            for (int j = 0; j < kBM / 64; ++j)
+              tma_load_2d_pair(a_tile(stage) + j * 8192, &maps.A, row_a + j * 64, kb * kBK, full0, pol);
+          } else {
+            tma_load_2d_pair(a_tile(stage), &maps.A, kb * kBK, row_a, full0, pol);
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row_b = n_blk * BN + h * 256 + static_cast<int>(rank) * kBM;
+            if (p.b_mn) {
+#pragma unroll
+              for (int j = 0; j < kBM / 64; ++j)
+                tma_load_2d_pair(b_tile(stage, h) + j * 8192, &maps.B, row_b + j * 64, kb * kBK, full0, pol);
+            } else {
+              tma_load_2d_pair(b_tile(stage, h), &maps.B, kb * kBK, row_b, full0, pol);
+            }
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {  // aborting: the loads in flight land (bounded) before exit
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 1000ull * 1000ull) __nanosleep(1000);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (CTA 0)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = umma_idesc_bf16(2 * kBM, 256) | (p.a_mn ? 1u << 15 : 0u) | (p.b_mn ? 1u << 16 : 0u);
+      const uint32_t a_step = p.a_mn ? 2048u >> 4 : 32u >> 4;
+      const uint32_t b_step = p.b_mn ? 2048u >> 4 : 32u >> 4;
+      auto mma_half = [&](int s, int h, bool first_kb) {
+        const uint64_t adesc = p.a_mn ? sw128_mnmajor_desc(a_tile(s)) : sw128_kmajor_desc(a_tile(s));
+        const uint64_t bdesc = p.b_mn ? sw128_mnmajor_desc(b_tile(s, h)) : sw128_kmajor_desc(b_tile(s, h));
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(h * 256);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k)
+          umma_bf16_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, (!first_kb || k != 0) ? 1u : 0u);
+      };
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int u = pair; u < num_units && ok; u += num_pairs, ++local) {
+        const uint32_t use = static_cast<uint32_t>(local);
+        int kb0, kb1;
+        unit_k(u, kb0, kb1);
+        const int n = kb1 - kb0;
+        const int head = n < STAGES ? n : STAGES;
+        // head: half 0 of the first `head` k-blocks (their stages stay held for half 1)
+        if (!mbar_wait_cluster(tempty_bar(0), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        int s = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < head; ++i) {
+          if (!mbar_wait_cluster(full_bar(s), ph, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          mma_half(s, 0, i == 0);
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        if (head == n) umma_commit_pair_both(tfull_bar(0));
+        if (!mbar_wait_cluster(tempty_bar(1), (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        for (int i = 0; i < head; ++i) {
+          mma_half(stage, 1, i == 0);
+          umma_commit_pair_both(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        // the rest: both halves per k-block
+        for (int i = head; i < n; ++i) {
+          if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          mma_half(stage, 0, false);
+          if (i + 1 == n) umma_commit_pair_both(tfull_bar(0));
+          mma_half(stage, 1, false);
+          umma_commit_pair_both(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) umma_commit_pair_both(tfull_bar(1));
+      }
+      umma_commit_pair(map_to_cta(drain_bar, 0));
+      mbar_wait_drain(drain_bar, 0, 100ull * 1000 * 1000);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue: atomic adds
+    // Warps 4-7 take columns 0-127 of each half, warps 8-11 columns 128-255; otherwise as in
+    // the one-CTA kernel (staged 32 x 32 chunks, eight lanes per row for the reductions).
+    const int q = warp & 3;
+    const int grp = (warp - 4) >> 2;
+    const uint32_t stg = sbase + L::kEpiOffset + static_cast<uint32_t>(warp - 4) * 4096u;
+    const uint32_t row_w = stg + static_cast<uint32_t>(lane) * 128u;
+    const int wv = lane & 7;
+    const int rq = lane >> 3;
+    int local = 0;
+    bool ok = true;
+    for (int u = pair; u < num_units && ok; u += num_pairs, ++local) {
+      const int tile = u % num_tiles;
+      const int m_blk = tile / p.num_n_blocks, n_blk = tile % p.num_n_blocks;
+      const uint32_t use = static_cast<uint32_t>(local);
+      const int64_t row0 = static_cast<int64_t>(m_blk) * (2 * kBM) + rank * kBM + q * 32;
+      for (int h = 0; h < 2 && ok; ++h) {
+        bool got = false;
+        if (lane == 0) got = mbar_wait_cluster(tfull_bar(h), use & 1u, abort_flag, p.status);
+        if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * 256 + grp * 128);
+        int s_cur = -1;
+        int32_t my_target = 0;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v);
+          tmem_wait_ld();
+          if (c == 3) {
+            tc_fence_before();
+            if (rank == 0) {
+              mbar_arrive(tempty_bar(h));
+            } else {
+              __syncwarp();
+              if (lane == 0) mbar_arrive_remote(map_to_cta(tempty_bar(h), 0));
+            }
+          }
+          const int col0 = n_blk * BN + h * 256 + grp * 128 + c * 32;
+          const int s = p.epi == kEpiScatterSub ? col0 / p.d : 0;
+          if (p.epi == kEpiScatterSub && s != s_cur) {
+            s_cur = s;
+            my_target = 0;
+            if (row0 + lane < p.M) {
+              my_target = p.idx[(row0 + lane) * p.S + s];
+              if (static_cast<uint32_t>(my_target) >= p.Vs[s]) {
+                set_status(p.status, NGRAM_STATUS_BAD_TOKEN);
+                my_target = 0;
+              }
+            }
+          }
+#pragma unroll
+          for (int w = 0; w < 8; ++w)
+            st_shared_v4(row_w + (static_cast<uint32_t>(w ^ (lane & 7)) << 4),
+                         make_uint4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]));
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = i * 4 + rq;
+            const uint4 x = ld_shared_v4(stg + static_cast<uint32_t>(r) * 128u + (static_cast<uint32_t>(wv ^ (r & 7)) << 4));
+            const int32_t target = __shfl_sync(0xffffffffu, my_target, r);
+            const int64_t grow = row0 + r;
+            if (grow < p.M) {
+              float* dst = p.epi == kEpiScatterSub
+                               ? p.dE[s] + static_cast<int64_t>(target) * p.d + (col0 - s * p.d) + wv * 4
+                               : p.out + grow * p.N + col0 + wv * 4;
+              atomicAdd(reinterpret_cast<float4*>(dst),
+                        make_float4(__uint_as_float(x.x) * p.scale, __uint_as_float(x.y) * p.scale,
+                                    __uint_as_float(x.z) * p.scale, __uint_as_float(x.w) * p.scale));
+            }
+          }
+          __syncwarp();
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, L::kTmemCols);

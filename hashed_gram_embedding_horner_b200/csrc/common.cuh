@@ -309,6 +309,17 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t cluster_addr) {
                : "memory");
 }
 
+// Pair form of umma_commit for both CTAs at once: one arrive on the mbarrier at shared-memory
+// address `bar` in each CTA of the pair (same offset in both; ctaMask 0b11) when every pair
+// MMA issued so far by this thread has completed. One instruction instead of a commit per CTA:
+// each commit holds the tensor pipe up for a while, so a pair MMA loop with one commit per
+// k-block runs measurably faster than with two.
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               ::"r"(bar), "h"(static_cast<uint16_t>(3))
+               : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)

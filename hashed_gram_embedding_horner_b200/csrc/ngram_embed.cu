@@ -64,7 +64,7 @@ struct ngram_embed_plan {
   bool maps_valid = false;
   const void* map_out = nullptr;  // the out map's pointer and row count
   int64_t map_out_T = -1;
-  bool smem_attr_set[16] = {};  // per kernel instance (form, tile width, rings), on `device`
+  bool smem_attr_set[17] = {};  // per kernel instance (form, tile width, rings), on `device`
   int a_stages = 0;            // one-CTA kernel: A ring depth (0 = default for the tile width)
   int cta_pair = -1;           // kernel form: 1 CTA pairs (cta_group::2), 0 one CTA per tile, -1 automatic
   int stream_k = 0;            // one-CTA kernel schedule: 0 automatic, 1 stream-K when possible, 2 never
@@ -74,10 +74,11 @@ struct ngram_embed_plan {
   int dense_a = 0;             // sub-rows gathered into G first, A by dense TMA: 1 on, 0 off
   const void* map_A = nullptr;  // the dense-A map's pointer and row count
   int64_t map_A_T = -1;
-  int max_clusters[7] = {};    // co-resident CTA pairs, per kernel instance (0 = not queried)
+  int max_clusters[8] = {};    // co-resident CTA pairs, per kernel instance (0 = not queried)
   int pair_cols = 0;           // pair form over column ranges: 1 whenever possible, 0 off
   int fused_step = 0;          // decode step committed and hashed inside the one-CTA projection
-  int bwd_pair = 1;            // backward GEMMs: 1 CTA pairs (M = 256 tiles), 0 one CTA per 128-row tile
+  int bwd_pair = 1;            // backward GEMMs: 1 CTA pairs (256-column tiles), 2 pairs with 512-column
+                               // tiles where possible, 0 one CTA per 128-row tile
 };
 
 namespace {
@@ -450,10 +451,10 @@ int launch_cols(ngram_embed_plan* p, const ProjParams& prm, int64_t T, cudaStrea
 constexpr int kBwdStages = 4;  // x (16 KB A + BN x 128 B B)
 
 size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
-// dE0's counting sort: counts [V0 + 1], cursor [V0], order [T], sorted ids [T] (int32).
+// dE0's counting sort: counts [V0 + 1], order [T], sorted ids [T], block sums (int32).
 size_t bwd_sort_bytes(const ngram_embed_plan* p, int64_t T) {
-  return round256((static_cast<size_t>(p->V0) + 1) * 4) + round256(static_cast<size_t>(p->V0) * 4) +
-         2 * round256(static_cast<size_t>(T) * 4) + round256((static_cast<size_t>(p->V0) + 1023) / 1024 * 4);
+  return round256((static_cast<size_t>(p->V0) + 1) * 4) + 2 * round256(static_cast<size_t>(T) * 4) +
+         round256((static_cast<size_t>(p->V0) + 1023) / 1024 * 4);
 }
 size_t bwd_g_bytes(const ngram_embed_plan* p, int64_t T) {
   return round256(static_cast<size_t>(T) * static_cast<size_t>(p->D) * 2);
@@ -590,11 +591,73 @@ int launch_dense_gemm_pair(ngram_embed_plan* p, DenseParams prm, GemmOperand A, 
   return launch(kern, dim3(2 * pairs), dim3(kGemmThreads), L::kLaunchBytes, st, p->pdl, 2, maps, prm);
 }
 
-// The backward's GEMMs in the plan's form (pairs need an even SM budget of at least 2).
+// Wide pair form: 256 x 512 tiles (B.rows % 512 == 0).
+constexpr int kBwdWideStages = 4;  // x (16 KB A + 32 KB B)
+
+int launch_dense_gemm_pair_wide(ngram_embed_plan* p, DenseParams prm, GemmOperand A, GemmOperand B, int64_t K,
+                                bool split, cudaStream_t st) {
+  using L = DenseWideSmem<kBwdWideStages>;
+  static_assert(L::kLaunchBytes <= 232448, "wide backward GEMM stages exceed 227 KB of shared memory");
+  auto kern = dense_gemm_pair_wide_kernel<kBwdWideStages>;
+  if (!p->smem_attr_set[16]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess)
+      return NGRAM_ERR_CUDA;
+    p->smem_attr_set[16] = true;
+  }
+  auto encode = [&](CUtensorMap* m, const GemmOperand& o) {
+    return o.mn ? encode_2d(m, o.base, static_cast<uint64_t>(o.rows), static_cast<uint64_t>(K),
+                            static_cast<uint64_t>(o.rows) * 2, 64, 64, CU_TENSOR_MAP_L2_PROMOTION_L2_256B)
+                : encode_2d(m, o.base, static_cast<uint64_t>(K), static_cast<uint64_t>(o.rows),
+                            static_cast<uint64_t>(K) * 2, kBK, kBM, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  };
+  DenseMaps maps;
+  int rc = encode(&maps.A, A);
+  if (rc) return rc;
+  if ((rc = encode(&maps.B, B))) return rc;
+  prm.a_mn = A.mn ? 1 : 0;
+  prm.b_mn = B.mn ? 1 : 0;
+  prm.M = static_cast<int>(A.rows);
+  prm.N = static_cast<int>(B.rows);
+  prm.num_m_blocks = static_cast<int>((A.rows + 2 * kBM - 1) / (2 * kBM));
+  prm.num_n_blocks = static_cast<int>(B.rows / 512);
+  prm.num_k_blocks = static_cast<int>((K + kBK - 1) / kBK);
+  int& max_pairs = p->max_clusters[7];
+  if (max_pairs == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (p->sms / 2));
+    cfg.blockDim = dim3(kWideGemmThreads);
+    cfg.dynamicSmemBytes = L::kLaunchBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return NGRAM_ERR_CUDA;
+    max_pairs = n;
+  }
+  const int pairs_avail = max_pairs < p->sms / 2 ? max_pairs : p->sms / 2;
+  if (pairs_avail < 1) return NGRAM_ERR_CUDA;
+  const int tiles = prm.num_m_blocks * prm.num_n_blocks;
+  const int s = split ? choose_splits(tiles, prm.num_k_blocks, pairs_avail) : 1;
+  prm.kb_per_split = (prm.num_k_blocks + s - 1) / s;
+  prm.splits = (prm.num_k_blocks + prm.kb_per_split - 1) / prm.kb_per_split;
+  const int units = tiles * prm.splits;
+  const int pairs = units < pairs_avail ? units : pairs_avail;
+  return launch(kern, dim3(2 * pairs), dim3(kWideGemmThreads), L::kLaunchBytes, st, p->pdl, 2, maps, prm);
+}
+
+// The backward's GEMMs in the plan's form (pairs need an SM budget of at least 2): 1 = pairs
+// with BN-column tiles, 2 = pairs with 512-column tiles where B's rows allow, 0 = one CTA.
 template <int BN>
 int launch_bwd_gemm(ngram_embed_plan* p, const DenseParams& prm, GemmOperand A, GemmOperand B, int64_t K, bool split,
                     cudaStream_t st) {
-  if (p->bwd_pair == 1 && p->sms >= 2) return launch_dense_gemm_pair<BN>(p, prm, A, B, K, split, st);
+  if (p->bwd_pair == 2 && p->sms >= 2 && B.rows % 512 == 0)
+    return launch_dense_gemm_pair_wide(p, prm, A, B, K, split, st);
+  if (p->bwd_pair >= 1 && p->sms >= 2) return launch_dense_gemm_pair<BN>(p, prm, A, B, K, split, st);
   return launch_dense_gemm<BN>(p, prm, A, B, K, split, st);
 }
 
@@ -997,7 +1060,7 @@ int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_token
 }
 
 int ngram_embed_plan_set_backward_pair(ngram_embed_plan* plan, int on) {
-  if (!plan || on < 0 || on > 1) return NGRAM_ERR_INVALID_ARG;
+  if (!plan || on < 0 || on > 2) return NGRAM_ERR_INVALID_ARG;
   plan->bwd_pair = on;
   return NGRAM_OK;
 }
@@ -1307,20 +1370,15 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     e.V0 = static_cast<uint32_t>(p->V0);
     e.scale = scale;
     e.counts = reinterpret_cast<int32_t*>(sort);
-    e.cursor = reinterpret_cast<int32_t*>(sort + round256((size_t(p->V0) + 1) * 4));
-    e.order = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(e.cursor) + round256(size_t(p->V0) * 4));
+    e.order = reinterpret_cast<int32_t*>(sort + round256((size_t(p->V0) + 1) * 4));
     e.sorted_tok = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(e.order) + round256(size_t(T) * 4));
     e.block_sums = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(e.sorted_tok) + round256(size_t(T) * 4));
     e.num_blocks = static_cast<int>((p->V0 + 1023) / 1024);
     e.status = status_ptr(workspace);
     const unsigned tb = static_cast<unsigned>((T + 255) / 256);
-    if (cudaMemsetAsync(e.counts, 0, (size_t(p->V0) + 1) * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(e.cursor, 0, size_t(p->V0) * 4, st) != cudaSuccess)
-      return NGRAM_ERR_CUDA;
+    if (cudaMemsetAsync(e.counts, 0, (size_t(p->V0) + 1) * 4, st) != cudaSuccess) return NGRAM_ERR_CUDA;
     if ((rc = launch(e0_hist_kernel, dim3(tb), dim3(256), 0, st, p->pdl, 1, e))) return rc;
-    if ((rc = launch(e0_scan_blocks_kernel, dim3(e.num_blocks), dim3(1024), 0, st, p->pdl, 1, e))) return rc;
-    if ((rc = launch(e0_scan_top_kernel, dim3(1), dim3(1024), 0, st, p->pdl, 1, e))) return rc;
-    if ((rc = launch(e0_scan_add_kernel, dim3(e.num_blocks), dim3(1024), 0, st, p->pdl, 1, e))) return rc;
+    if ((rc = launch(e0_scan_kernel, dim3(e.num_blocks), dim3(1024), 0, st, p->pdl, 1, e))) return rc;
     if ((rc = launch(e0_place_kernel, dim3(tb), dim3(256), 0, st, p->pdl, 1, e))) return rc;
     const int64_t items = (T + kSegRows - 1) / kSegRows * ((D + 255) / 256);  // one warp each
     if ((rc = launch(e0_reduce_kernel, dim3(static_cast<unsigned>((items + 7) / 8)), dim3(256), 0, st, p->pdl, 1, e)))

@@ -279,12 +279,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       bool ok = true;
       auto advance = [&](int& st, uint32_t& ph) { if (++st == STAGES) { st = 0; ph ^= 1u; } };
       auto release = [&](int st) {
-        umma_commit_pair(map_to_cta(empty_bar(st), 0));
-        umma_commit_pair(map_to_cta(empty_bar(st), 1));
+        umma_commit_pair_both(empty_bar(st));
       };
       auto done = [&](int h) {  // half h of the segment summed: its epilogue may start
-        umma_commit_pair(map_to_cta(tfull_bar(h), 0));
-        umma_commit_pair(map_to_cta(tfull_bar(h), 1));
+        umma_commit_pair_both(tfull_bar(h));
       };
       for (int k = 0; k < nsegs && ok; ++k) {
         const ColSeg sg = col_seg(cw, k);

@@ -551,13 +551,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         for (int k = 0; k < kBK / 16; ++k)
           umma_bf16_pair(d_tmem + h * kMmaN, adesc + 2u * k, bdesc + 2u * k, idesc, (j | k) != 0 ? 1u : 0u);
         if (kWide && j + 1 == nj) {  // half h complete: its epilogue may start
-          umma_commit_pair(map_to_cta(tfull_bar(h), 0));
-          umma_commit_pair(map_to_cta(tfull_bar(h), 1));
+          umma_commit_pair_both(tfull_bar(h));
         }
       };
       auto release = [&](int st) {
-        umma_commit_pair(map_to_cta(empty_bar(st), 0));
-        umma_commit_pair(map_to_cta(empty_bar(st), 1));
+        umma_commit_pair_both(empty_bar(st));
       };
       for (Seg g = seg_first(wp, pair); g.tile < num_tiles && ok; g = seg_next(wp, g), ++local) {
         // one accumulator of both halves (wide), else two alternating ones
@@ -604,8 +602,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           advance(stage, phase);
         }
         if (ok && !kWide) {
-          umma_commit_pair(map_to_cta(tfull_bar(acc), 0));
-          umma_commit_pair(map_to_cta(tfull_bar(acc), 1));
+          umma_commit_pair_both(tfull_bar(acc));
         }
       }
       umma_commit_pair(map_to_cta(drain_bar, 0));

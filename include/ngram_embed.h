@@ -276,7 +276,7 @@ int ngram_embed_fwd_draft(const ngram_embed_plan* plan, const int32_t* tokens,
  * [0, V_nk) read/write row 0 and set NGRAM_STATUS_BAD_TOKEN.
  *   workspace  >= ngram_embed_bwd_workspace_bytes(plan, num_tokens): G, the gathered
  *              sub-rows [num_tokens x D] bf16, and the dE0 sort buffers (about
- *              2 D num_tokens + 8 V0 + 8 num_tokens bytes); its head is the status word.
+ *              2 D num_tokens + 4 V0 + 8 num_tokens bytes); its head is the status word.
  * The GEMMs read g and W_stacked where they lie (the tensor cores take the operands that are
  * not K-major in memory as MN-major tiles): nothing is transposed. */
 size_t ngram_embed_bwd_workspace_bytes(const ngram_embed_plan* plan, int64_t max_tokens);
@@ -404,11 +404,15 @@ int ngram_embed_plan_set_fused_step(ngram_embed_plan* plan, int on);
 
 /* Form of the backward pass's two dense GEMMs (dG = c g W_stacked and dW = c g^T G, the
  * gradients of Eq. 3 of "Scaling Embeddings Outperforms Scaling Experts in Language Models",
- * section 2): 1 = CTA pairs (tcgen05.mma.cta_group::2, 256-row tiles; each CTA of a pair
- * loads its 128 rows of A and half of B per k-block; default), 0 = one CTA per 128-row tile.
- * Pairs need a plan SM budget of at least 2 (otherwise the one-CTA form runs). A tuning knob:
- * results agree within the stated tolerance (the fp32 atomic-add order differs).
- * NGRAM_ERR_INVALID_ARG for other values or a null plan. */
+ * section 2): 1 = CTA pairs (tcgen05.mma.cta_group::2, 256-row x 256-column tiles, 128 when
+ * D % 256 != 0; each CTA of a pair loads its 128 rows of A and half of B per k-block;
+ * default); 2 = CTA pairs with 256 x 512 tiles where D % 512 == 0 (two N = 256 accumulator
+ * halves filling TMEM, drained half by half; measured on B200 at D = 2048, T = 32768: 0.58 ms
+ * for the whole backward against 0.55 ms with 256-column tiles, the drain of the single
+ * accumulator stalling the MMAs); 0 = one CTA per 128-row tile (0.62 ms). Pairs need a plan
+ * SM budget of at least 2 (otherwise the one-CTA form runs). A tuning knob: results agree
+ * within the stated tolerance (the fp32 atomic-add order differs). NGRAM_ERR_INVALID_ARG for
+ * other values or a null plan. */
 int ngram_embed_plan_set_backward_pair(ngram_embed_plan* plan, int on);
 
 /* CTA-pair form over column ranges (Eq. 3 of "Scaling Embeddings Outperforms Scaling Experts

@@ -55,7 +55,7 @@ def small_problem(D=1024, N=3, K=2, V=(211, 223, 227, 229), V0=300, lengths=(1, 
     return dict(V0=V0, D=D, N=N, K=K, V=list(V), S=S, d=d, tok=tok, off=off, E=E, W=W, g=g, T=T)
 
 
-def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=True, sms=0):
+def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=1, sms=0):
     plan = ne.ngram_embed_plan_create(P["V0"], P["D"], P["N"], P["K"], P["V"], ne.NGRAM_BF16)
     ne.ngram_embed_plan_set_backward_pair(plan, pair)
     if sms:
@@ -85,11 +85,13 @@ def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=True, sms=0
                                    dict(D=384, N=2, K=3, V=(61, 67, 71)),
                                    dict(lengths=(4096,), V=(4099, 5003, 6007, 7001), V0=131072)],
                          ids=["D1024_ragged", "D2048_dense_collisions", "D1536_N4", "D384_tile128", "T4096_wide_V"])
-@pytest.mark.parametrize("form", [dict(pair=True), dict(pair=False), dict(pair=True, sms=4), dict(pair=True, sms=5)],
-                         ids=["pairs", "one_cta", "pairs_2", "pairs_odd_sms"])
+@pytest.mark.parametrize("form", [dict(pair=1), dict(pair=2), dict(pair=0), dict(pair=2, sms=4),
+                                  dict(pair=1, sms=5)],
+                         ids=["pairs_256", "pairs_wide", "one_cta", "pairs_wide_2", "pairs_256_odd_sms"])
 def test_backward_matches_oracle(ne, shape, form):
-    """Both GEMM forms; with 2 pairs (4 or 5 SMs) each pair runs many (tile, k range) units
-    through both accumulators."""
+    """Every GEMM form (pairs with 512-column tiles where D % 512 == 0, pairs with 256- or
+    128-column tiles, one CTA); with 2 pairs (4 or 5 SMs) each pair runs many (tile, k range)
+    units through its accumulators."""
     P = small_problem(**shape)
     dE0, dE, dW = run_bwd(ne, P, scale=3.0, **form)
     w0, wE, wW = oracle.backward(P["V0"], P["D"], P["N"], P["K"], P["V"], P["tok"], P["off"], P["E"], P["W"],
@@ -104,7 +106,7 @@ def test_backward_matches_oracle(ne, shape, form):
     assert not dE0[~touched].any()
 
 
-@pytest.mark.parametrize("pair", [True, False], ids=["pairs", "one_cta"])
+@pytest.mark.parametrize("pair", [1, 2, 0], ids=["pairs_256", "pairs_wide", "one_cta"])
 def test_backward_accumulates_and_skips(ne, pair):
     """+= semantics (two calls give twice the gradient) and NULL gradients are skipped; a
     single token (CTA 1 of the pair reads rows past the end only)."""
