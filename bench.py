@@ -49,6 +49,11 @@ WORKLOADS = {
     "profile_full_scale": configs.FULL_SCALE.with_(
         name="profile_full_scale_bf16_D4096_N5_K2_small",
         V_nk=tuple(configs.primes_from(300000 + 131072 // 2, 8))),
+    # the backward's shapes (T = 32768, D = 2048) over ~100k-row sub-tables: with the fp32
+    # gradient tables about 3 GB held, for multi-pass captures (--profile-backward)
+    "profile_d2048_bwd": configs.PREFILL_D2048.with_(
+        name="profile_bwd_bf16_D2048_N3_K2_small",
+        V_nk=tuple(configs.primes_from(100000, 4))),
 }
 HEADLINE = "full_scale_prefill"
 # the other prefill workloads, measured in the same run (each with its own roofline)
@@ -625,6 +630,8 @@ def main():
                     help="with --decode-only: the one decode workload to run")
     ap.add_argument("--decode-only", action="store_true",
                     help="only the speculative-decode measurement (one JSON line with the decode object)")
+    ap.add_argument("--profile-backward", action="store_true",
+                    help="with --profile-only: also run the backward (all three gradients) as many times")
     ap.add_argument("--profile-only", action="store_true",
                     help="warm up, run --steps forward calls back to back and exit (for profiler captures)")
     args = ap.parse_args()
@@ -674,8 +681,24 @@ def main():
         for _ in range(max(args.warmup, 3) + args.steps):
             ne.ngram_embed_fwd(plan, tokens, offsets, E0, E, W, out, ws, stream=stream)
         torch.cuda.synchronize()
+        bwd_status = None
+        if args.profile_backward:
+            T = len(tokens_h)
+            idx = torch.empty((T, cfg.S), dtype=torch.int32, device=dev)
+            ne.ngram_hash_indices(plan, tokens, offsets, idx, ws, stream=stream)
+            del out, E0
+            g_out = (torch.randn((T, cfg.D), device=dev) * 0.01).to(torch.bfloat16)
+            dE = [torch.zeros((v, cfg.d), dtype=torch.float32, device=dev) for v in cfg.V_nk]
+            dW = torch.zeros((cfg.D, cfg.D), dtype=torch.float32, device=dev)
+            dE0 = torch.zeros((cfg.V0, cfg.D), dtype=torch.float32, device=dev)
+            bws = ne.new_bwd_workspace(plan, T, device=dev)
+            for _ in range(max(args.warmup, 3) + args.steps):
+                ne.ngram_embed_bwd(plan, tokens, idx, g_out, bws, E_nk=E, W_stacked=W, dE0=dE0, dE_nk=dE, dW=dW,
+                                   stream=stream)
+            torch.cuda.synchronize()
+            bwd_status = ne.ngram_embed_get_status(bws)
         print(json.dumps({"profile_only": cfg.name, "steps": args.steps,
-                          "status": ne.ngram_embed_get_status(ws)}), flush=True)
+                          "status": ne.ngram_embed_get_status(ws), "backward_status": bwd_status}), flush=True)
         return
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)

@@ -49,6 +49,7 @@ EXPORTED = [
     "ngram_draft_cache_reset", "ngram_embed_draft_workspace_bytes", "ngram_embed_fwd_draft",
     "ngram_embed_fwd_step", "ngram_embed_plan_set_dense_a", "ngram_embed_plan_set_pair_columns",
     "ngram_embed_plan_set_fused_step", "ngram_embed_plan_set_backward_pair",
+    "ngram_embed_plan_set_backward_streams",
 ]
 
 
@@ -93,6 +94,7 @@ _sig("ngram_embed_plan_set_pair_wide", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_dense_a", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_pair_columns", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_backward_pair", [_P, ctypes.c_int])
+_sig("ngram_embed_plan_set_backward_streams", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_fused_step", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_sm_count", [_P, ctypes.c_int])
 _sig("ngram_embed_plan_set_stream_k", [_P, ctypes.c_int])
@@ -277,6 +279,13 @@ def ngram_embed_plan_set_backward_pair(plan: Plan, mode):
     """The backward's GEMMs: True/1 CTA pairs with 256-column tiles (default); 2 pairs with
     512-column tiles where D allows; False/0 one CTA per 128-row tile."""
     _check(_lib.ngram_embed_plan_set_backward_pair(plan.handle, int(mode)), "ngram_embed_plan_set_backward_pair")
+
+
+def ngram_embed_plan_set_backward_streams(plan: Plan, on: bool):
+    """True (default): the backward's memory-bound kernels overlap its dG GEMM on the plan's
+    auxiliary stream; False: everything on the caller's stream."""
+    _check(_lib.ngram_embed_plan_set_backward_streams(plan.handle, int(bool(on))),
+           "ngram_embed_plan_set_backward_streams")
 
 
 def ngram_embed_plan_set_sm_count(plan: Plan, sms: int):

@@ -79,6 +79,9 @@ struct ngram_embed_plan {
   int fused_step = 0;          // decode step committed and hashed inside the one-CTA projection
   int bwd_pair = 1;            // backward GEMMs: 1 CTA pairs (256-column tiles), 2 pairs with 512-column
                                // tiles where possible, 0 one CTA per 128-row tile
+  int bwd_streams = 1;         // backward: 1 the memory-bound kernels on an auxiliary stream, 0 all on the caller's
+  cudaStream_t aux = nullptr;  // the auxiliary stream (created by the first backward call that uses it)
+  cudaEvent_t aux_ev[3] = {};  // fork, G gathered, join
 };
 
 namespace {
@@ -1021,6 +1024,12 @@ int ngram_embed_plan_create(const ngram_embed_config* cfg, ngram_embed_plan** ou
 }
 
 int ngram_embed_plan_destroy(ngram_embed_plan* plan) {
+  if (plan && plan->aux && set_device(plan) == NGRAM_OK) {
+    cudaStreamSynchronize(plan->aux);
+    for (cudaEvent_t e : plan->aux_ev)
+      if (e) cudaEventDestroy(e);
+    cudaStreamDestroy(plan->aux);
+  }
   delete plan;
   return NGRAM_OK;
 }
@@ -1057,6 +1066,12 @@ int ngram_embed_plan_set_cta_pair(ngram_embed_plan* plan, int on) {
 int ngram_embed_plan_kernel_form(const ngram_embed_plan* plan, int64_t num_tokens) {
   if (!plan || num_tokens < 0 || num_tokens > INT32_MAX) return NGRAM_ERR_INVALID_ARG;
   return choose_form(plan, num_tokens, ws_bytes(plan, num_tokens), num_tokens, false);
+}
+
+int ngram_embed_plan_set_backward_streams(ngram_embed_plan* plan, int on) {
+  if (!plan || on < 0 || on > 1) return NGRAM_ERR_INVALID_ARG;
+  plan->bwd_streams = on;
+  return NGRAM_OK;
 }
 
 int ngram_embed_plan_set_backward_pair(ngram_embed_plan* plan, int on) {
@@ -1331,6 +1346,26 @@ size_t ngram_embed_bwd_workspace_bytes(const ngram_embed_plan* plan, int64_t max
   return bwd_ws_bytes(plan, max_tokens);
 }
 
+// The plan's auxiliary stream and its three events, created on first use (non-blocking
+// stream: no implicit ordering with the legacy default stream; events without timing).
+int ensure_aux(ngram_embed_plan* p) {
+  if (p->aux) return NGRAM_OK;
+  cudaStream_t s = nullptr;
+  if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return NGRAM_ERR_CUDA;
+  cudaEvent_t ev[3] = {};
+  for (auto& e : ev) {
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      for (cudaEvent_t x : ev)
+        if (x) cudaEventDestroy(x);
+      cudaStreamDestroy(s);
+      return NGRAM_ERR_CUDA;
+    }
+  }
+  p->aux = s;
+  for (int i = 0; i < 3; ++i) p->aux_ev[i] = ev[i];
+  return NGRAM_OK;
+}
+
 int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const int32_t* idx, int64_t num_tokens,
                     const void* const* E_nk, const void* W_stacked, const void* grad_out, float* dE0,
                     float* const* dE_nk, float* dW, void* workspace, size_t workspace_bytes, void* stream) {
@@ -1359,6 +1394,30 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
   const float scale = p->out_scale / static_cast<float>(p->S + 1);
   const auto* g = static_cast<const uint16_t*>(grad_out);
 
+  // The memory-bound kernels (the gather of G for dW, the dE0 sort and sums) run on the plan's
+  // auxiliary stream, forked from and joined back to `st`, so that they overlap the dG GEMM
+  // (persistent CTAs that leave registers and threads free on every SM); dW waits for G only.
+  const bool fork = p->bwd_streams == 1 && dE_nk && (dE0 || dW);
+  if (fork && (rc = ensure_aux(p))) return rc;
+  const cudaStream_t side = fork ? p->aux : st;
+  bool joined = !fork;
+  auto join = [&](int code) {
+    if (!joined) {
+      joined = true;
+      if ((cudaEventRecord(p->aux_ev[2], side) != cudaSuccess || cudaStreamWaitEvent(st, p->aux_ev[2], 0) != cudaSuccess) &&
+          code == NGRAM_OK)
+        code = NGRAM_ERR_CUDA;
+    }
+    return code;
+  };
+  if (fork && (cudaEventRecord(p->aux_ev[0], st) != cudaSuccess || cudaStreamWaitEvent(side, p->aux_ev[0], 0) != cudaSuccess)) {
+    joined = true;  // nothing was forked
+    return NGRAM_ERR_CUDA;
+  }
+  if (dW) {
+    if ((rc = launch_gather(p, idx, T, E_nk, G, nullptr, nullptr, nullptr, workspace, side))) return join(rc);
+    if (fork && cudaEventRecord(p->aux_ev[1], side) != cudaSuccess) return join(NGRAM_ERR_CUDA);
+  }
   if (dE0) {
     uint8_t* sort = base + kHeadBytes + bwd_g_bytes(p, T);
     ScatterE0Params e{};
@@ -1376,13 +1435,13 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     e.num_blocks = static_cast<int>((p->V0 + 1023) / 1024);
     e.status = status_ptr(workspace);
     const unsigned tb = static_cast<unsigned>((T + 255) / 256);
-    if (cudaMemsetAsync(e.counts, 0, (size_t(p->V0) + 1) * 4, st) != cudaSuccess) return NGRAM_ERR_CUDA;
-    if ((rc = launch(e0_hist_kernel, dim3(tb), dim3(256), 0, st, p->pdl, 1, e))) return rc;
-    if ((rc = launch(e0_scan_kernel, dim3(e.num_blocks), dim3(1024), 0, st, p->pdl, 1, e))) return rc;
-    if ((rc = launch(e0_place_kernel, dim3(tb), dim3(256), 0, st, p->pdl, 1, e))) return rc;
+    if (cudaMemsetAsync(e.counts, 0, (size_t(p->V0) + 1) * 4, side) != cudaSuccess) return join(NGRAM_ERR_CUDA);
+    if ((rc = launch(e0_hist_kernel, dim3(tb), dim3(256), 0, side, p->pdl, 1, e))) return join(rc);
+    if ((rc = launch(e0_scan_kernel, dim3(e.num_blocks), dim3(1024), 0, side, p->pdl, 1, e))) return join(rc);
+    if ((rc = launch(e0_place_kernel, dim3(tb), dim3(256), 0, side, p->pdl, 1, e))) return join(rc);
     const int64_t items = (T + kSegRows - 1) / kSegRows * ((D + 255) / 256);  // one warp each
-    if ((rc = launch(e0_reduce_kernel, dim3(static_cast<unsigned>((items + 7) / 8)), dim3(256), 0, st, p->pdl, 1, e)))
-      return rc;
+    if ((rc = launch(e0_reduce_kernel, dim3(static_cast<unsigned>((items + 7) / 8)), dim3(256), 0, side, p->pdl, 1, e)))
+      return join(rc);
   }
   if (dE_nk) {
     // dG = c g W_stacked: A = g [T x D] (K-major over D), B[n][k] = W_stacked[k][n] (W as it
@@ -1401,13 +1460,13 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     const GemmOperand A{g, T, false}, B{W_stacked, D, true};
     if ((rc = p->D % 256 == 0 ? launch_bwd_gemm<256>(p, dp, A, B, D, false, st)
                               : launch_bwd_gemm<128>(p, dp, A, B, D, false, st)))
-      return rc;
+      return join(rc);
   }
   if (dW) {
+    if (fork && cudaStreamWaitEvent(st, p->aux_ev[1], 0) != cudaSuccess) return join(NGRAM_ERR_CUDA);
     // dW += c g^T G: A[m][t] = g[t][m] and B[n][t] = G[t][n], both MN-major as they lie
-    // (G gathered row by row into the workspace first), K = T with split-K units adding
+    // (G gathered row by row into the workspace, above), K = T with split-K units adding
     // into dW.
-    if ((rc = launch_gather(p, idx, T, E_nk, G, nullptr, nullptr, nullptr, workspace, st))) return rc;
     DenseParams dp{};
     dp.scale = scale;
     dp.epi = kEpiAccumDense;
@@ -1416,9 +1475,9 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     const GemmOperand A{g, D, true}, B{G, D, true};
     if ((rc = p->D % 256 == 0 ? launch_bwd_gemm<256>(p, dp, A, B, T, true, st)
                               : launch_bwd_gemm<128>(p, dp, A, B, T, true, st)))
-      return rc;
+      return join(rc);
   }
-  return NGRAM_OK;
+  return join(NGRAM_OK);
 }
 
 int ngram_embed_layernorm(const ngram_embed_plan* plan, const void* x, int64_t num_tokens, const float* gamma,

@@ -415,6 +415,18 @@ int ngram_embed_plan_set_fused_step(ngram_embed_plan* plan, int on);
  * other values or a null plan. */
 int ngram_embed_plan_set_backward_pair(ngram_embed_plan* plan, int on);
 
+/* Streams of ngram_embed_bwd. 1 (default): the memory-bound kernels (the gather of G for dW,
+ * the dE0 counting sort and sums) run on an auxiliary stream that the plan owns, forked from
+ * the caller's stream with an event after everything queued there and joined back before the
+ * call returns (the caller's stream waits for all of the call's work; dW's GEMM waits for G
+ * only), so they overlap the dG GEMM. The first backward call that forks creates the stream
+ * and three events on the plan's device (do it once outside CUDA-graph capture); calls on one
+ * plan share them, so a plan's backward calls must be issued from one host thread at a time;
+ * ngram_embed_plan_destroy releases them. 0: every kernel on the caller's stream, in order.
+ * Results agree within the stated tolerance either way (the fp32 atomic-add order differs).
+ * NGRAM_ERR_INVALID_ARG for other values or a null plan. */
+int ngram_embed_plan_set_backward_streams(ngram_embed_plan* plan, int on);
+
 /* CTA-pair form over column ranges (Eq. 3 of "Scaling Embeddings Outperforms Scaling Experts
  * in Language Models", section 2, partitioned by output columns): the pairs are spread evenly
  * over the 256-token row blocks and each pair computes the full sum over K for a contiguous

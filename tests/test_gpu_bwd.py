@@ -55,9 +55,10 @@ def small_problem(D=1024, N=3, K=2, V=(211, 223, 227, 229), V0=300, lengths=(1, 
     return dict(V0=V0, D=D, N=N, K=K, V=list(V), S=S, d=d, tok=tok, off=off, E=E, W=W, g=g, T=T)
 
 
-def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=1, sms=0):
+def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=1, sms=0, streams=True):
     plan = ne.ngram_embed_plan_create(P["V0"], P["D"], P["N"], P["K"], P["V"], ne.NGRAM_BF16)
     ne.ngram_embed_plan_set_backward_pair(plan, pair)
+    ne.ngram_embed_plan_set_backward_streams(plan, streams)
     if sms:
         ne.ngram_embed_plan_set_sm_count(plan, sms)
     if scale != 1.0:
@@ -86,8 +87,9 @@ def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=1, sms=0):
                                    dict(lengths=(4096,), V=(4099, 5003, 6007, 7001), V0=131072)],
                          ids=["D1024_ragged", "D2048_dense_collisions", "D1536_N4", "D384_tile128", "T4096_wide_V"])
 @pytest.mark.parametrize("form", [dict(pair=1), dict(pair=2), dict(pair=0), dict(pair=2, sms=4),
-                                  dict(pair=1, sms=5)],
-                         ids=["pairs_256", "pairs_wide", "one_cta", "pairs_wide_2", "pairs_256_odd_sms"])
+                                  dict(pair=1, sms=5), dict(pair=1, streams=False)],
+                         ids=["pairs_256", "pairs_wide", "one_cta", "pairs_wide_2", "pairs_256_odd_sms",
+                              "one_stream"])
 def test_backward_matches_oracle(ne, shape, form):
     """Every GEMM form (pairs with 512-column tiles where D % 512 == 0, pairs with 256- or
     128-column tiles, one CTA); with 2 pairs (4 or 5 SMs) each pair runs many (tile, k range)
@@ -126,6 +128,47 @@ def test_backward_accumulates_and_skips(ne, pair):
     for s in range(P1["S"]):
         close(dE[s], wE[s], f"dE[{s}] T=1")
     close(dW, wW, "dW T=1")
+
+
+def test_backward_on_a_side_stream_in_a_cuda_graph(ne):
+    """The auxiliary-stream fork and join inside a captured graph: every replay adds the same
+    gradients as an eager call (after the warm-up call that creates the stream), on a
+    non-default stream, all three gradients and each alone."""
+    P = small_problem(lengths=(300, 77, 1))
+    plan = ne.ngram_embed_plan_create(P["V0"], P["D"], P["N"], P["K"], P["V"], ne.NGRAM_BF16)
+    ws = ne.new_workspace(plan, P["T"])
+    idx = torch.empty((P["T"], P["S"]), dtype=torch.int32, device="cuda")
+    ne.ngram_hash_indices(plan, dev_i32(P["tok"]), dev_i32(P["off"]), idx, ws)
+    Ed = [to_device(e, torch.bfloat16) for e in P["E"]]
+    Wd = to_device(P["W"], torch.bfloat16)
+    gd = to_device(P["g"], torch.bfloat16)
+    tok = dev_i32(P["tok"])
+    bws = ne.new_bwd_workspace(plan, P["T"])
+    w0, wE, wW = oracle.backward(P["V0"], P["D"], P["N"], P["K"], P["V"], P["tok"], P["off"], P["E"], P["W"], P["g"])
+    for which in (("E0", "E", "W"), ("E0", "E"), ("E", "W")):
+        dE0 = torch.zeros((P["V0"], P["D"]), dtype=torch.float32, device="cuda") if "E0" in which else None
+        dE = [torch.zeros((v, P["d"]), dtype=torch.float32, device="cuda") for v in P["V"]]
+        dW = torch.zeros((P["D"], P["D"]), dtype=torch.float32, device="cuda") if "W" in which else None
+        s = torch.cuda.Stream()
+        call = lambda: ne.ngram_embed_bwd(plan, tok, idx, gd, bws, E_nk=Ed, W_stacked=Wd, dE0=dE0, dE_nk=dE, dW=dW,
+                                          stream=s)
+        with torch.cuda.stream(s):
+            call()  # eager: creates the auxiliary stream
+        s.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            call()
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+        assert ne.ngram_embed_get_status(bws) == 0
+        if dE0 is not None:
+            close(dE0.cpu().numpy(), 3 * w0, f"{which} dE0")
+        for k in range(P["S"]):
+            close(dE[k].cpu().numpy(), 3 * wE[k], f"{which} dE[{k}]")
+        if dW is not None:
+            close(dW.cpu().numpy(), 3 * wW, f"{which} dW")
+        del graph
 
 
 def test_backward_full_tables_sampled(ne):
