@@ -470,18 +470,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 
 // CTA-pair form of the dense GEMM (tcgen05.mma.cta_group::2, M = 256): the pair computes a
-// 256 x BN tile; each CTA loads its 128 rows of A and BN/2 rows of B per stage (2-D TMA in
+// 256 x BN tile; each CTA loads its 128 rows of A and BN/2 rows of B per k-block (2-D TMA in
 // the .cta_group::2 form, byte counts completing on CTA 0's stage barrier), one thread of CTA 0
 // issues the MMAs and commits stage releases and "accumulator ready" to both CTAs, and each
 // CTA's epilogue drains its 128 accumulator rows as the one-CTA kernel does (CTA 1's warps
 // free the accumulator by remote arrivals on CTA 0's barrier). Per SM and k-block it loads
 // 16 KB of A + BN/2 x 128 B of B for the same FLOPs the one-CTA kernel needs 16 KB + BN x
-// 128 B for.
-template <int BN, int STAGES>
+// 128 B for. A stage holds KSUB consecutive k-blocks: every stage costs the MMA thread a
+// barrier wait and a commit, which hold the tensor pipe up for a while, so fewer, larger
+// stages leave more of its time to the MMAs.
+template <int BN, int STAGES, int KSUB>
 struct DensePairSmem {
-  static constexpr int kABytes = kBM * kBK * 2;           // this CTA's 128 rows of A
-  static constexpr int kBBytes = (BN / 2) * kBK * 2;      // this CTA's BN/2 rows of B
-  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kABytes = kBM * kBK * 2;           // this CTA's 128 rows of A, one k-block
+  static constexpr int kBBytes = (BN / 2) * kBK * 2;      // this CTA's BN/2 rows of B, one k-block
+  static constexpr int kSubBytes = kABytes + kBBytes;     // one k-block of both
+  static constexpr int kStageBytes = KSUB * kSubBytes;    // a stage: KSUB consecutive k-blocks
   static constexpr int kBarOffset = STAGES * kStageBytes;
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kEpiOffset = (kBarOffset + kNumBars * 8 + 16 + 127) / 128 * 128;
@@ -491,10 +494,10 @@ struct DensePairSmem {
   static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of 128-byte swizzling");
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int KSUB>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     dense_gemm_pair_kernel(const __grid_constant__ DenseMaps maps, const __grid_constant__ DenseParams p) {
-  using L = DensePairSmem<BN, STAGES>;
+  using L = DensePairSmem<BN, STAGES, KSUB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -506,8 +509,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOffset + L::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto a_tile = [&](int s) { return sbase + s * L::kStageBytes; };
-  auto b_tile = [&](int s) { return sbase + s * L::kStageBytes + L::kABytes; };
+  auto a_tile = [&](int s, int j) { return sbase + s * L::kStageBytes + j * L::kSubBytes; };
+  auto b_tile = [&](int s, int j) { return sbase + s * L::kStageBytes + j * L::kSubBytes + L::kABytes; };
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs and owns the stage barriers
@@ -566,23 +569,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int row_b = n_blk * BN + static_cast<int>(rank) * (BN / 2);
         int kb0, kb1;
         unit_k(u, kb0, kb1);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += KSUB) {
+          const int nsub = kb1 - kb < KSUB ? kb1 - kb : KSUB;  // k-blocks in this stage
           if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           const uint32_t full0 = map_to_cta(full_bar(stage), 0);
-          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2u * L::kStageBytes);
-          if (p.a_mn) {
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2u * nsub * L::kSubBytes);
+          for (int i = 0; i < nsub; ++i) {
+            const int kx = (kb + i) * kBK;
+            if (p.a_mn) {
 #pragma unroll
-            for (int j = 0; j < kBM / 64; ++j)
-              tma_load_2d_pair(a_tile(stage) + j * 8192, &maps.A, row_a + j * 64, kb * kBK, full0, pol);
-          } else {
-            tma_load_2d_pair(a_tile(stage), &maps.A, kb * kBK, row_a, full0, pol);
-          }
-          if (p.b_mn) {
+              for (int j = 0; j < kBM / 64; ++j)
+                tma_load_2d_pair(a_tile(stage, i) + j * 8192, &maps.A, row_a + j * 64, kx, full0, pol);
+            } else {
+              tma_load_2d_pair(a_tile(stage, i), &maps.A, kx, row_a, full0, pol);
+            }
+            if (p.b_mn) {
 #pragma unroll
-            for (int j = 0; j < BN / 128; ++j)
-              tma_load_2d_pair(b_tile(stage) + j * 8192, &maps.B, row_b + j * 64, kb * kBK, full0, pol);
-          } else {
-            tma_load_2d_pair(b_tile(stage), &maps.B, kb * kBK, row_b, full0, pol);
+              for (int j = 0; j < BN / 128; ++j)
+                tma_load_2d_pair(b_tile(stage, i) + j * 8192, &maps.B, row_b + j * 64, kx, full0, pol);
+            } else {
+              tma_load_2d_pair(b_tile(stage, i), &maps.B, kx, row_b, full0, pol);
+            }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -610,14 +617,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         int kb0, kb1;
         unit_k(u, kb0, kb1);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += KSUB) {
+          const int nsub = kb1 - kb < KSUB ? kb1 - kb : KSUB;
           if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = p.a_mn ? sw128_mnmajor_desc(a_tile(stage)) : sw128_kmajor_desc(a_tile(stage));
-          const uint64_t bdesc = p.b_mn ? sw128_mnmajor_desc(b_tile(stage)) : sw128_kmajor_desc(b_tile(stage));
+          for (int i = 0; i < nsub; ++i) {
+            const uint64_t adesc = p.a_mn ? sw128_mnmajor_desc(a_tile(stage, i)) : sw128_kmajor_desc(a_tile(stage, i));
+            const uint64_t bdesc = p.b_mn ? sw128_mnmajor_desc(b_tile(stage, i)) : sw128_kmajor_desc(b_tile(stage, i));
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, (kb > kb0 || k != 0) ? 1u : 0u);
+            for (int k = 0; k < kBK / 16; ++k)
+              umma_bf16_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, (kb + i > kb0 || k != 0) ? 1u : 0u);
+          }
           umma_commit_pair_both(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }

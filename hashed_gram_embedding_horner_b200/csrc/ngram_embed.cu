@@ -533,15 +533,17 @@ int launch_dense_gemm(ngram_embed_plan* p, DenseParams prm, GemmOperand A, GemmO
 
 // CTA-pair form of the same GEMM: 256-row tiles, each CTA of a pair loading its 128 rows of A
 // and half of B's BN rows per stage; units (tile, k range) strided over the co-resident pairs.
-constexpr int kBwdPairStages256 = 6;  // x (16 KB A + 16 KB B)
-constexpr int kBwdPairStages128 = 8;  // x (16 KB A + 8 KB B)
+constexpr int kBwdPairKsub = 2;        // k-blocks per stage
+constexpr int kBwdPairStages256 = 3;  // x 2 x (16 KB A + 16 KB B)
+constexpr int kBwdPairStages128 = 4;  // x 2 x (16 KB A + 8 KB B)
 
 template <int BN>
 int launch_dense_gemm_pair(ngram_embed_plan* p, DenseParams prm, GemmOperand A, GemmOperand B, int64_t K, bool split,
                            cudaStream_t st) {
   constexpr int STAGES = BN == 256 ? kBwdPairStages256 : kBwdPairStages128;
-  using L = DensePairSmem<BN, STAGES>;
-  auto kern = dense_gemm_pair_kernel<BN, STAGES>;
+  using L = DensePairSmem<BN, STAGES, kBwdPairKsub>;
+  static_assert(L::kLaunchBytes <= 232448, "pair backward GEMM stages exceed 227 KB of shared memory");
+  auto kern = dense_gemm_pair_kernel<BN, STAGES, kBwdPairKsub>;
   const int key = BN == 256 ? 14 : 15;
   if (!p->smem_attr_set[key]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kLaunchBytes) != cudaSuccess)
@@ -1397,6 +1399,8 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
   // The memory-bound kernels (the gather of G for dW, the dE0 sort and sums) run on the plan's
   // auxiliary stream, forked from and joined back to `st`, so that they overlap the dG GEMM
   // (persistent CTAs that leave registers and threads free on every SM); dW waits for G only.
+  // dG is launched first so that its CTAs take their places on the SMs before the side
+  // stream's blocks fill what is left.
   const bool fork = p->bwd_streams == 1 && dE_nk && (dE0 || dW);
   if (fork && (rc = ensure_aux(p))) return rc;
   const cudaStream_t side = fork ? p->aux : st;
@@ -1413,6 +1417,25 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
   if (fork && (cudaEventRecord(p->aux_ev[0], st) != cudaSuccess || cudaStreamWaitEvent(side, p->aux_ev[0], 0) != cudaSuccess)) {
     joined = true;  // nothing was forked
     return NGRAM_ERR_CUDA;
+  }
+  if (dE_nk) {
+    // dG = c g W_stacked: A = g [T x D] (K-major over D), B[n][k] = W_stacked[k][n] (W as it
+    // lies: MN-major); the epilogue adds each 32-column piece into its sub-table's gradient row.
+    DenseParams dp{};
+    dp.scale = scale;
+    dp.epi = kEpiScatterSub;
+    dp.idx = idx;
+    for (int s = 0; s < p->S; ++s) {
+      dp.dE[s] = dE_nk[s];
+      dp.Vs[s] = static_cast<uint32_t>(p->V[s]);
+    }
+    dp.S = p->S;
+    dp.d = p->d;
+    dp.status = status_ptr(workspace);
+    const GemmOperand A{g, T, false}, B{W_stacked, D, true};
+    if ((rc = p->D % 256 == 0 ? launch_bwd_gemm<256>(p, dp, A, B, D, false, st)
+                              : launch_bwd_gemm<128>(p, dp, A, B, D, false, st)))
+      return join(rc);
   }
   if (dW) {
     if ((rc = launch_gather(p, idx, T, E_nk, G, nullptr, nullptr, nullptr, workspace, side))) return join(rc);
@@ -1441,25 +1464,6 @@ int ngram_embed_bwd(const ngram_embed_plan* plan_c, const int32_t* tokens, const
     if ((rc = launch(e0_place_kernel, dim3(tb), dim3(256), 0, side, p->pdl, 1, e))) return join(rc);
     const int64_t items = (T + kSegRows - 1) / kSegRows * ((D + 255) / 256);  // one warp each
     if ((rc = launch(e0_reduce_kernel, dim3(static_cast<unsigned>((items + 7) / 8)), dim3(256), 0, side, p->pdl, 1, e)))
-      return join(rc);
-  }
-  if (dE_nk) {
-    // dG = c g W_stacked: A = g [T x D] (K-major over D), B[n][k] = W_stacked[k][n] (W as it
-    // lies: MN-major); the epilogue adds each 32-column piece into its sub-table's gradient row.
-    DenseParams dp{};
-    dp.scale = scale;
-    dp.epi = kEpiScatterSub;
-    dp.idx = idx;
-    for (int s = 0; s < p->S; ++s) {
-      dp.dE[s] = dE_nk[s];
-      dp.Vs[s] = static_cast<uint32_t>(p->V[s]);
-    }
-    dp.S = p->S;
-    dp.d = p->d;
-    dp.status = status_ptr(workspace);
-    const GemmOperand A{g, T, false}, B{W_stacked, D, true};
-    if ((rc = p->D % 256 == 0 ? launch_bwd_gemm<256>(p, dp, A, B, D, false, st)
-                              : launch_bwd_gemm<128>(p, dp, A, B, D, false, st)))
       return join(rc);
   }
   if (dW) {
