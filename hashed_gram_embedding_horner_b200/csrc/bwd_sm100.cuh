@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_wait_ld();
         if (c + 1 == BN / 32) {
           tc_fence_before();
-          mbar_arrive(tempty_bar(acc));
+          mbar_arrive_relaxed(tempty_bar(acc));
         }
         const int col0 = n_blk * BN + c * 32;
         const int s = p.epi == kEpiScatterSub ? col0 / p.d : 0;  // 32 columns never straddle two sub-tables
@@ -671,10 +671,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (c + 1 == BN / 32) {
           tc_fence_before();
           if (rank == 0) {
-            mbar_arrive(tempty_bar(acc));
+            mbar_arrive_relaxed(tempty_bar(acc));
           } else {
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(acc ? tempty_remote1 : tempty_remote0);
+            if (lane == 0) mbar_arrive_remote_relaxed(acc ? tempty_remote1 : tempty_remote0);
           }
         }
         const int col0 = n_blk * BN + c * 32;
@@ -943,10 +943,10 @@ __global__ void __launch_bounds__(kWideGemmThreads, 1)
           if (c == 3) {
             tc_fence_before();
             if (rank == 0) {
-              mbar_arrive(tempty_bar(h));
+              mbar_arrive_relaxed(tempty_bar(h));
             } else {
               __syncwarp();
-              if (lane == 0) mbar_arrive_remote(map_to_cta(tempty_bar(h), 0));
+              if (lane == 0) mbar_arrive_remote_relaxed(map_to_cta(tempty_bar(h), 0));
             }
           }
           const int col0 = n_blk * BN + h * 256 + grp * 128 + c * 32;

@@ -545,7 +545,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           tmem_wait_ld();
           if (c + 1 == BN / 32) {
             tc_fence_before();
-            mbar_arrive(tempty_bar(acc));  // accumulator fully read: MMA may reuse it
+            mbar_arrive_relaxed(tempty_bar(acc));  // accumulator fully read: MMA may reuse it
           }
 #pragma unroll
           for (int w = 0; w < 4; ++w) {  // columns 32c + 8w .. +7: chunk (4c + w) % 8 of box c / 2
@@ -706,7 +706,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           if (lane == 0) *cnt = 0;  // the tile is done: zero again for the next launch
         }
         tc_fence_before();
-        mbar_arrive(tempty_bar(acc));  // accumulator read for the last time: MMA may reuse it
+        mbar_arrive_relaxed(tempty_bar(acc));  // accumulator read for the last time: MMA may reuse it
       }
     }
     cp_async_wait_all();                   // E_0 rows still landing (after an abort)

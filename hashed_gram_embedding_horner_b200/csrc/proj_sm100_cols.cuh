@@ -448,10 +448,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         }
         tc_fence_before();  // this warp's last read of half h
         if (rank == 0) {
-          mbar_arrive(tempty_bar(h));
+          mbar_arrive_relaxed(tempty_bar(h));
         } else {
           __syncwarp();
-          if (lane == 0) mbar_arrive_remote(h ? tempty_remote1 : tempty_remote0);
+          if (lane == 0) mbar_arrive_remote_relaxed(h ? tempty_remote1 : tempty_remote0);
         }
       }
       if (!alive) break;

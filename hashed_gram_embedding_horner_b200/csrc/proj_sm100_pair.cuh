@@ -193,10 +193,10 @@ __device__ __noinline__ bool pair_sk_piece(const ProjParams& p, const PairPiece 
   }
   tc_fence_before();  // accumulator read for the last time: the MMA may reuse it
   if (a.rank == 0) {
-    mbar_arrive(a.tempty);
+    mbar_arrive_relaxed(a.tempty);
   } else {
     __syncwarp();
-    if (a.lane == 0) mbar_arrive_remote(a.tempty);
+    if (a.lane == 0) mbar_arrive_remote_relaxed(a.tempty);
   }
   return true;
 }
@@ -344,13 +344,13 @@ __device__ __noinline__ bool pair_sk_piece_wide(const ProjParams& p, const WideP
   }
   tc_fence_before();  // both halves read for the last time: the MMA may reuse them
   if (a.rank == 0) {
-    mbar_arrive(a.tempty0);
-    mbar_arrive(a.tempty1);
+    mbar_arrive_relaxed(a.tempty0);
+    mbar_arrive_relaxed(a.tempty1);
   } else {
     __syncwarp();
     if (a.lane == 0) {
-      mbar_arrive_remote(a.tempty0);
-      mbar_arrive_remote(a.tempty1);
+      mbar_arrive_remote_relaxed(a.tempty0);
+      mbar_arrive_remote_relaxed(a.tempty1);
     }
   }
   return true;
@@ -758,10 +758,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         if (cc % kSegChunks == kSegChunks - 1) {  // this warp's last read of the segment
           tc_fence_before();
           if (rank == 0) {
-            mbar_arrive(tempty_bar(bar));
+            mbar_arrive_relaxed(tempty_bar(bar));
           } else {
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(bar ? tempty_remote1 : tempty_remote0);
+            if (lane == 0) mbar_arrive_remote_relaxed(bar ? tempty_remote1 : tempty_remote0);
           }
         }
 #pragma unroll
