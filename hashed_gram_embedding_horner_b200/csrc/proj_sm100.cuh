@@ -31,8 +31,12 @@
 // Shared memory holds two rings with their own barriers: AST stages of gathered A rows and
 // WST stages of W tiles. A rows come from random table rows (often HBM misses, the longest
 // latency on the path) and W tiles from L2, so the A ring is the deeper one: decoupling the
-// rings lets more A bytes be in flight than a shared (A, W) stage would. TMEM holds two
-// BN-column fp32 accumulators so the epilogue of one tile overlaps the main loop of the next.
+// rings lets more A bytes be in flight than a shared (A, W) stage would. Where the A ring is
+// at least as deep as the W ring, the two still share one handshake per k-block (the W tile
+// completes on the A stage's full barrier; the A stage's empty barrier frees the W stage
+// WST k-blocks later): each barrier wait and tcgen05.commit of the MMA thread costs tensor-
+// pipe time. TMEM holds two BN-column fp32 accumulators so the epilogue of one tile overlaps
+// the main loop of the next.
 // Every wait is bounded (see mbar_wait); on a timeout all roles stop, drain what they
 // have in flight, free TMEM and return with NGRAM_STATUS_TIMEOUT set.
 #pragma once
@@ -257,6 +261,10 @@ template <int BN, int AST, int WST>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_sm100_kernel(const __grid_constant__ ProjMaps maps, const __grid_constant__ ProjParams p) {
   using L = ProjSmem<BN, AST, WST>;
+  // One stage handshake per k-block for both rings: the W tile of k-block c lands on the A
+  // stage's full barrier, and the W producer reuses a W stage once the A stage barrier says
+  // that k-block c - WST was consumed (unambiguous while AST >= WST).
+  constexpr bool kJoint = AST >= WST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -281,7 +289,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < AST; ++s) {
       // every A thread (cp.async completion) and thread 0's TMA byte count
-      mbar_init(full_bar(s), static_cast<uint32_t>(kAThreads) + 1u);
+      mbar_init(full_bar(s), static_cast<uint32_t>(kAThreads) + 1u + (kJoint ? 1u : 0u));
       mbar_init(empty_bar(s), 1u);  // one tcgen05.commit
     }
     for (int s = 0; s < WST; ++s) {
@@ -424,6 +432,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       const uint64_t pol = l2_policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
+      int c = 0;  // k-blocks produced so far
       bool ok = true;
       for (Seg g = seg_first(wp, blockIdx.x); g.tile < num_tiles && ok; g = seg_next(wp, g)) {
         const int n_blk = g.tile % p.num_n_blocks;
@@ -431,9 +440,19 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         for (int i = g.i0; i < g.i1; ++i) {
           int kb = i + rot;
           if (kb >= KB) kb -= KB;
-          if (!mbar_wait(wempty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(wfull_bar(stage), L::kBBytes);
-          tma_load_2d(b_tile(stage), &maps.W, kb * kBK, n_blk * BN, wfull_bar(stage), pol);
+          if constexpr (kJoint) {
+            if (c >= WST) {
+              const int j = c - WST;
+              if (!mbar_wait(empty_bar(j % AST), static_cast<uint32_t>((j / AST) & 1), abort_flag, p.status)) { ok = false; break; }
+            }
+            mbar_arrive_expect_tx(full_bar(c % AST), L::kBBytes);
+            tma_load_2d(b_tile(stage), &maps.W, kb * kBK, n_blk * BN, full_bar(c % AST), pol);
+            ++c;
+          } else {
+            if (!mbar_wait(wempty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+            mbar_arrive_expect_tx(wfull_bar(stage), L::kBBytes);
+            tma_load_2d(b_tile(stage), &maps.W, kb * kBK, n_blk * BN, wfull_bar(stage), pol);
+          }
           if (++stage == WST) { stage = 0; phase ^= 1u; }
         }
       }
@@ -453,7 +472,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int i = g.i0; i < g.i1; ++i) {
-          if (!mbar_wait(wfull_bar(wstage), wphase, abort_flag, p.status)) { ok = false; break; }
+          if (!kJoint && !mbar_wait(wfull_bar(wstage), wphase, abort_flag, p.status)) { ok = false; break; }
           if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           fence_proxy_async_smem();  // the stage's cp.async rows were written by the generic proxy
@@ -463,7 +482,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           for (int k = 0; k < kBK / 16; ++k)  // K = 16 per instruction: +32 B = +2 in the address field
             umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (i > g.i0 || k != 0) ? 1u : 0u);
           umma_commit(empty_bar(stage));
-          umma_commit(wempty_bar(wstage));
+          if (!kJoint) umma_commit(wempty_bar(wstage));
           if (++stage == AST) { stage = 0; phase ^= 1u; }
           if (++wstage == WST) { wstage = 0; wphase ^= 1u; }
         }
