@@ -10,14 +10,17 @@
 // Colliding rows (several tokens, one table row) add up: every scatter is an fp32 atomic
 // add, so the summation order (not the set of terms) varies between runs.
 //
-// Both GEMMs run on one kernel, `dense_gemm_sm100_kernel`: bf16 A (M x K) and B (N x K)
-// tiles brought in by 2-D TMA straight from the tensors as they lie in memory — K-major
-// (K contiguous: g for dG) or MN-major (M or N contiguous: W for dG, g and G for dW), the
-// tensor cores reading either layout from its shared-memory descriptor — fp32 accumulators
-// in TMEM, work units of (128 x BN tile, k range) handed out round-robin to persistent
-// CTAs (split-K where tiles are few), and an epilogue that atomically adds the scaled
-// partial tile into its destination: sub-table gradient rows (dG) or dW. The only copy is
-// G itself, gathered row by row from the sub-tables into the workspace for dW.
+// Both GEMMs run on one kernel: bf16 A (M x K) and B (N x K) tiles brought in by 2-D TMA
+// straight from the tensors as they lie in memory — K-major (K contiguous: g for dG) or
+// MN-major (M or N contiguous: W for dG, g and G for dW), the tensor cores reading either
+// layout from its shared-memory descriptor — fp32 accumulators in TMEM, work units of
+// (tile, k range) handed out round-robin to persistent CTAs or CTA pairs (split-K where
+// tiles are few, the units in flight sharing a k range), and an epilogue that atomically
+// adds the scaled partial tile into its destination: sub-table gradient rows (dG) or dW.
+// Three forms of it: `dense_gemm_pair_kernel` (CTA pairs, 256 x BN tiles, the default),
+// `dense_gemm_sm100_kernel` (one CTA per 128 x BN tile) and `dense_gemm_pair_wide_kernel`
+// (CTA pairs, 256 x 512 tiles). The only copy is G itself, gathered row by row from the
+// sub-tables into the workspace for dW.
 #pragma once
 
 #include "proj_sm100.cuh"
