@@ -109,6 +109,12 @@ def test_plan_without_device_validates_then_fails_launch(ne):
     assert with_g - lib.ngram_embed_workspace_bytes(h, 32768) == 32768 * 2048 * 2
     # 512-column pair tiles (D = 2048 here): on when forced, automatic needs the SM count
     assert lib.ngram_embed_plan_set_pair_wide(h, 2) == -1 and lib.ngram_embed_plan_set_pair_wide(h, -2) == -1
+    # the backward's GEMM forms (0, 1, 2) and streams (0, 1)
+    assert lib.ngram_embed_plan_set_backward_pair(h, 3) == -1 and lib.ngram_embed_plan_set_backward_pair(h, -1) == -1
+    assert all(lib.ngram_embed_plan_set_backward_pair(h, m) == 0 for m in (0, 2, 1))
+    assert lib.ngram_embed_plan_set_backward_streams(h, 2) == -1 and lib.ngram_embed_plan_set_backward_streams(h, -1) == -1
+    assert lib.ngram_embed_plan_set_backward_streams(h, 0) == 0 and lib.ngram_embed_plan_set_backward_streams(h, 1) == 0
+    assert lib.ngram_embed_plan_set_backward_pair(None, 1) == -1 and lib.ngram_embed_plan_set_backward_streams(None, 1) == -1
     assert lib.ngram_embed_plan_set_pair_wide(h, 1) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 4
     assert lib.ngram_embed_plan_set_dense_a(h, 1) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 8
     assert lib.ngram_embed_plan_set_tile_n(h, 128) == 0 and lib.ngram_embed_plan_kernel_form(h, 1280) == 3

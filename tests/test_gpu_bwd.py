@@ -171,6 +171,35 @@ def test_backward_on_a_side_stream_in_a_cuda_graph(ne):
         del graph
 
 
+def test_backward_plan_released_right_after_a_forked_call(ne):
+    """Destroying the plan straight after a call whose kernels are still running on its
+    auxiliary stream waits for them: the gradients are complete, and a new plan's call
+    (with its own auxiliary stream) adds the same again."""
+    P = small_problem(lengths=(200, 9))
+    w0, wE, wW = oracle.backward(P["V0"], P["D"], P["N"], P["K"], P["V"], P["tok"], P["off"], P["E"], P["W"], P["g"])
+    Ed = [to_device(e, torch.bfloat16) for e in P["E"]]
+    Wd = to_device(P["W"], torch.bfloat16)
+    gd = to_device(P["g"], torch.bfloat16)
+    tok = dev_i32(P["tok"])
+    dE0 = torch.zeros((P["V0"], P["D"]), dtype=torch.float32, device="cuda")
+    dE = [torch.zeros((v, P["d"]), dtype=torch.float32, device="cuda") for v in P["V"]]
+    dW = torch.zeros((P["D"], P["D"]), dtype=torch.float32, device="cuda")
+    for rep in (1, 2):
+        plan = ne.ngram_embed_plan_create(P["V0"], P["D"], P["N"], P["K"], P["V"], ne.NGRAM_BF16)
+        ws = ne.new_workspace(plan, P["T"])
+        idx = torch.empty((P["T"], P["S"]), dtype=torch.int32, device="cuda")
+        ne.ngram_hash_indices(plan, tok, dev_i32(P["off"]), idx, ws)
+        bws = ne.new_bwd_workspace(plan, P["T"])
+        ne.ngram_embed_bwd(plan, tok, idx, gd, bws, E_nk=Ed, W_stacked=Wd, dE0=dE0, dE_nk=dE, dW=dW)
+        del plan  # ngram_embed_plan_destroy: waits for the plan's auxiliary stream
+        torch.cuda.synchronize()
+        assert ne.ngram_embed_get_status(bws) == 0
+        close(dE0.cpu().numpy(), rep * w0, f"dE0 x{rep}")
+        for k in range(P["S"]):
+            close(dE[k].cpu().numpy(), rep * wE[k], f"dE[{k}] x{rep}")
+        close(dW.cpu().numpy(), rep * wW, f"dW x{rep}")
+
+
 def test_backward_full_tables_sampled(ne):
     """prefill D = 2048 tables (2.16M-row sub-tables, 8.9 GB), 4096 Zipf tokens: sampled rows
     of every gradient against the oracle computed for those rows only."""
