@@ -84,8 +84,11 @@ def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=1, sms=0, s
 @pytest.mark.parametrize("shape", [dict(), dict(D=2048, N=3, K=2, V=(97, 101, 103, 107)),
                                    dict(D=1536, N=4, K=1, V=(331, 337, 347)),
                                    dict(D=384, N=2, K=3, V=(61, 67, 71)),
-                                   dict(lengths=(4096,), V=(4099, 5003, 6007, 7001), V0=131072)],
-                         ids=["D1024_ragged", "D2048_dense_collisions", "D1536_N4", "D384_tile128", "T4096_wide_V"])
+                                   dict(lengths=(4096,), V=(4099, 5003, 6007, 7001), V0=131072),
+                                   dict(D=4096, N=5, K=2, V=(1009, 1013, 1019, 1021, 1031, 1033, 1039, 1049),
+                                        lengths=(130, 77))],
+                         ids=["D1024_ragged", "D2048_dense_collisions", "D1536_N4", "D384_tile128", "T4096_wide_V",
+                              "D4096_N5_K2"])
 @pytest.mark.parametrize("form", [dict(pair=1), dict(pair=2), dict(pair=0), dict(pair=2, sms=4),
                                   dict(pair=1, sms=5), dict(pair=1, streams=False)],
                          ids=["pairs_256", "pairs_wide", "one_cta", "pairs_wide_2", "pairs_256_odd_sms",
