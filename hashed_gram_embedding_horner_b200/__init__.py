@@ -370,7 +370,7 @@ def ngram_embed_plan_kernel_form(plan: Plan, num_tokens: int) -> str:
 
 
 def ngram_embed_plan_set_pdl(plan: Plan, on: bool):
-    """Launch the plan's kernels as programmatic dependent launches (default on)."""
+    """Launch the plan's kernels as programmatic dependent launches (default off)."""
     _check(_lib.ngram_embed_plan_set_pdl(plan.handle, int(bool(on))), "ngram_embed_plan_set_pdl")
 
 

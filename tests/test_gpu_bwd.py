@@ -55,10 +55,12 @@ def small_problem(D=1024, N=3, K=2, V=(211, 223, 227, 229), V0=300, lengths=(1, 
     return dict(V0=V0, D=D, N=N, K=K, V=list(V), S=S, d=d, tok=tok, off=off, E=E, W=W, g=g, T=T)
 
 
-def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=1, sms=0, streams=True):
+def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=1, sms=0, streams=True, pdl=False):
     plan = ne.ngram_embed_plan_create(P["V0"], P["D"], P["N"], P["K"], P["V"], ne.NGRAM_BF16)
     ne.ngram_embed_plan_set_backward_pair(plan, pair)
     ne.ngram_embed_plan_set_backward_streams(plan, streams)
+    if pdl:
+        ne.ngram_embed_plan_set_pdl(plan, 1)
     if sms:
         ne.ngram_embed_plan_set_sm_count(plan, sms)
     if scale != 1.0:
@@ -90,9 +92,9 @@ def run_bwd(ne, P, scale=1.0, which=("E0", "E", "W"), repeat=1, pair=1, sms=0, s
                          ids=["D1024_ragged", "D2048_dense_collisions", "D1536_N4", "D384_tile128", "T4096_wide_V",
                               "D4096_N5_K2"])
 @pytest.mark.parametrize("form", [dict(pair=1), dict(pair=2), dict(pair=0), dict(pair=2, sms=4),
-                                  dict(pair=1, sms=5), dict(pair=1, streams=False)],
+                                  dict(pair=1, sms=5), dict(pair=1, streams=False), dict(pair=1, pdl=True)],
                          ids=["pairs_256", "pairs_wide", "one_cta", "pairs_wide_2", "pairs_256_odd_sms",
-                              "one_stream"])
+                              "one_stream", "pdl"])
 def test_backward_matches_oracle(ne, shape, form):
     """Every GEMM form (pairs with 512-column tiles where D % 512 == 0, pairs with 256- or
     128-column tiles, one CTA); with 2 pairs (4 or 5 SMs) each pair runs many (tile, k range)
