@@ -127,7 +127,8 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """nvidia-smi clock / throttle-reason samples, each stamped with the host time it
+    arrived, so that a summary covers only a window in which the GPU was busy."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -136,46 +137,74 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.samples = []  # (host time, line)
+        self.marks = {}
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.samples.append((time.time(), ln))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
         except OSError:
             self.proc = None
         time.sleep(0.3)
         return self
 
+    def mark(self, name):
+        self.marks[name] = time.time()
+
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
-            time.sleep(0.25)
+            time.sleep(0.15)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+                self.proc.wait()
+            self.reader.join(timeout=5)
 
-    def summary(self):
+    def summary(self, start="load_start", end="load_end"):
+        """Median SM clock over the samples taken between the two marks (the whole run if
+        either is missing), the throttle reasons seen then or in the timed region."""
+        t0, t1 = self.marks.get(start), self.marks.get(end)
+        r0, r1 = self.marks.get("timed_start"), self.marks.get("timed_end")
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        for ts, ln in self.samples:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
+            in_load = t0 is None or t1 is None or t0 <= ts <= t1
+            in_timed = r0 is not None and r1 is not None and r0 <= ts <= r1
+            if not (in_load or in_timed):
+                continue
             try:
-                sm.append(float(f[1]))
+                clk = float(f[1])
                 mx = float(f[2])
             except ValueError:
                 continue
+            if in_load:
+                sm.append(clk)
             for name, val in zip(names, f[5:9]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        out = {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+               "samples": len(sm)}
+        if t0 is not None and t1 is not None:
+            out["window_s"] = round(t1 - t0, 3)
+            out["what"] = ("median of the samples taken while the timed step ran again back to back for a "
+                           "second after the timed measurements (those alone are shorter than the sampling "
+                           "interval); reasons from both")
+        return out
 
 
 def rank_config(cfg, rank: int):
@@ -337,6 +366,8 @@ def run_prefill(ne, cfg, tables, args, dev, flush, world, rank, clock_gpu=None, 
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
+    if clk:
+        clk.mark("timed_start")
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         ev[i][0].record(stream)
@@ -363,6 +394,16 @@ def run_prefill(ne, cfg, tables, args, dev, flush, world, rank, clock_gpu=None, 
         pe[i][1].record(stream)
     torch.cuda.synchronize()
     if clk:
+        clk.mark("timed_end")
+        # the clock under this load, after every timed number: the same step back to back
+        # for about a second (the timed steps alone are shorter than the sampling interval)
+        clk.mark("load_start")
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            for _ in range(8):
+                step()
+            torch.cuda.synchronize()
+        clk.mark("load_end")
         clk.__exit__(None, None, None)
     proj_ms = float(np.mean([a.elapsed_time(b) for a, b in pe]))
     hash_ms = float(np.mean([a.elapsed_time(b) for a, b in hs]))
